@@ -1,0 +1,9 @@
+"""CPU oracle for the 1SPSA / 1.5-SPSA zero-order training step.
+
+TEST INFRASTRUCTURE.  Plain, slow, obviously-correct reference code: a C library
+(zo_oracle.c: Philox probes, perturbation, quadratic loss, preconditioner, update) and
+numpy code (MLP and decoder losses, the step driver).  Only the tests, the smoke
+check and the benchmark's CPU-baseline leg may import it.  It shares no code with the
+CUDA library and neither imports the other; both take their inputs from `synth`.
+"""
+from . import core, mlp, step  # noqa: F401

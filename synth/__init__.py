@@ -1,0 +1,92 @@
+"""Seeded synthetic inputs shared by the CUDA path's tests/benchmark and the oracle.
+
+This module only draws inputs (weights, curvature vectors, data batches, loss values
+used as test inputs); it holds none of the zero-order method's arithmetic (no probes,
+perturbations, losses of the trained model, preconditioner or update).  Every array is
+a pure function of its arguments: numpy's PCG64 seeded with (seed, stream tag, ...).
+
+Workload shapes follow the pages' setups as restated in the design notes:
+  - diagonal quadratic: theta_0 ~ N(0, 1), D_j = 10^U(-3, 3) (log-uniform on [1e-3, 1e3]);
+  - MLP classifier 64 -> 256 (ReLU) -> 10, parameters N(0, 0.05), inputs N(0, 1),
+    labels = argmax of a fixed random teacher MLP of the same shape;
+  - OPT-shaped decoders: matrices and embeddings N(0, 0.02) in bf16, biases 0,
+    LayerNorm gains 1 and shifts 0, tokens uniform over the vocabulary, binary labels.
+"""
+import numpy as np
+
+_TAGS = {"quad": 1, "mlp": 2, "teacher": 3, "batch": 4, "loss": 5, "coef": 6, "opt": 7,
+         "tokens": 8, "labels": 9, "theta": 10}
+
+
+def rng(seed, tag, *more):
+    return np.random.default_rng([int(seed) & 0xFFFFFFFF, _TAGS[tag]] + [int(m) for m in more])
+
+
+def to_bf16_bits(x):
+    """float32 -> bf16 bit pattern (uint16), round to nearest even (inputs only)."""
+    u = np.ascontiguousarray(x, np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return u.astype(np.uint16)
+
+
+# ---------------------------------------------------------------- diagonal quadratic
+
+def quad_problem(M, seed=0):
+    """(theta_0 float32 [M], D float32 [M])."""
+    r = rng(seed, "quad", M)
+    theta = r.standard_normal(M, dtype=np.float32)
+    D = (10.0 ** r.uniform(-3.0, 3.0, M)).astype(np.float32)
+    return theta, D
+
+
+# ---------------------------------------------------------------- MLP classifier
+
+MLP_IN, MLP_HIDDEN, MLP_OUT, MLP_BATCH = 64, 256, 10, 64
+
+
+def mlp_param_count(n_in=MLP_IN, n_hidden=MLP_HIDDEN, n_out=MLP_OUT):
+    return n_hidden * n_in + n_hidden + n_out * n_hidden + n_out
+
+
+def mlp_params(seed=0, tag="mlp", n_in=MLP_IN, n_hidden=MLP_HIDDEN, n_out=MLP_OUT, std=0.05):
+    """Flat float32 parameters in the order W1[h][in], b1[h], W2[out][h], b2[out]."""
+    M = mlp_param_count(n_in, n_hidden, n_out)
+    return (rng(seed, tag, M).standard_normal(M) * std).astype(np.float32)
+
+
+def mlp_batch(seed, step, teacher, n_in=MLP_IN, n_hidden=MLP_HIDDEN, n_out=MLP_OUT,
+              batch=MLP_BATCH):
+    """(X float32 [batch][n_in], labels int32 [batch]) for one step.
+
+    Labels are the argmax (lowest index on ties) of the teacher network's outputs,
+    evaluated in fp64 here purely to label the synthetic data.
+    """
+    X = rng(seed, "batch", step).standard_normal((batch, n_in), dtype=np.float32)
+    t = teacher.astype(np.float64)
+    o = 0
+    W1 = t[o:o + n_hidden * n_in].reshape(n_hidden, n_in); o += n_hidden * n_in
+    b1 = t[o:o + n_hidden]; o += n_hidden
+    W2 = t[o:o + n_out * n_hidden].reshape(n_out, n_hidden); o += n_out * n_hidden
+    b2 = t[o:o + n_out]
+    h = np.maximum(X.astype(np.float64) @ W1.T + b1, 0.0)
+    y = np.argmax(h @ W2.T + b2, axis=1).astype(np.int32)
+    return X, y
+
+
+# ---------------------------------------------------------------- loss values as inputs
+
+def losses(n, seed=0, L0=2.3, eps=1e-3, g_scale=1.0, c_scale=50.0):
+    """Synthetic (loss_plus[n], loss_minus[n], loss0) in fp64, shaped like a real step:
+    L+- = L0 +- eps*g + eps^2*c/2 with random g, c (used as inputs to the update path)."""
+    r = rng(seed, "loss", n)
+    g = r.standard_normal(n) * g_scale
+    c = np.abs(r.standard_normal(n)) * c_scale * np.where(r.uniform(size=n) < 0.1, -1, 1)
+    lp = L0 + eps * g + 0.5 * eps * eps * c
+    lm = L0 - eps * g + 0.5 * eps * eps * c
+    return lp, lm, float(L0)
+
+
+def coefficients(n, seed=0, scale=1e-3):
+    """Synthetic fp32 update coefficients a[n] (mixed signs and magnitudes)."""
+    r = rng(seed, "coef", n)
+    return (r.standard_normal(n) * scale * 10.0 ** r.uniform(-2, 0, n)).astype(np.float32)
