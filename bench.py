@@ -1,0 +1,317 @@
+#!/usr/bin/env python
+"""Benchmark of one 1.5-SPSA step of the diagonal-quadratic workload on B200.
+
+Workload (the default, one GPU): L = 1/2 sum_j D_j theta_j^2 with M = 2^24 fp32
+parameters, D_j log-uniform in [1e-3, 1e3], theta_0 ~ N(0, 1); n_pert = 64,
+eps = 1e-3, lr = 4e-7, damping = 1e-3, 1.5-SPSA.  One step = clean loss + 2*n_pert
+perturbed losses + preconditioner + update, all through the C ABI of libzo.so.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  With N > 1 (torchrun, one rank per GPU) every rank runs
+its own replica of the workload (independent problems, no collective on the data path);
+`value` is the sum over ranks of steps/s, timed as the max over ranks.  `--impl
+reference` times the CPU oracle on a bounded slice of the same workload.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "1.5-SPSA steps/s & probe fwd tokens/s; perturb/update HBM GB/s as % of peak"
+M_FULL = 1 << 24
+N_PERT, EPS, LR, DAMPING = 64, 1e-3, 4e-7, 1e-3
+WORKLOAD = ("diagonal quadratic L=1/2*sum D_j theta_j^2, M=2^24 fp32, D log-uniform [1e-3,1e3], "
+            "theta0~N(0,1); 1.5-SPSA n_pert=64 eps=1e-3 lr=4e-7 damping=1e-3")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+def time_oracle(M_sample, n_steps, seed=0):
+    """Times the oracle's full step on the first M_sample elements of the workload.
+    Returns seconds per sample step (single-threaded C + numpy)."""
+    import oracle
+    import synth
+    th, D = synth.quad_problem(M_sample, seed=seed)
+    loss = lambda P: oracle.core.quad_loss(P, D)  # noqa: E731
+    times = []
+    for s in range(n_steps):
+        t0 = time.perf_counter()
+        th, _ = oracle.step.spsa_step(th, loss, N_PERT, EPS, LR, DAMPING, seed, s, update="mirror")
+        times.append(time.perf_counter() - t0)
+    return times
+
+
+def reference_arm(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    M_sample = 1 << 18
+    times = time_oracle(M_sample, args.warmup + args.steps)[args.warmup:]
+    per_step = sum(times) / len(times)
+    scale = M_sample / M_FULL
+    value = scale / per_step  # full-workload steps/s extrapolated linearly in M
+    sample = (f"oracle step on the first 2^18 of 2^24 parameters (1/64 of the workload), "
+              f"{args.steps} timed steps after {args.warmup} warm-up; steps/s scaled by 1/64")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "M": M_FULL, "n_pert": N_PERT},
+            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def gpu_arm(args):
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    import zero_order_forward_b200 as zo
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    dev = torch.device("cuda", local_rank)
+    hbm_peak, peak_kind = peaks()
+
+    th_np, D_np = synth.quad_problem(M_FULL, seed=rank)
+    theta = torch.from_numpy(th_np).to(dev)
+    D = torch.from_numpy(D_np).to(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    n = N_PERT
+    losses = torch.zeros(2 * n + 1, dtype=torch.float64, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ctx = zo.zo_create(theta, seed=rank, stream=stream.cuda_stream)
+
+    def one_step(ev=None):
+        """Step through the C ABI primitives; ev = 4 events at the phase boundaries."""
+        if ev:
+            ev[0].record(stream)
+        zo.zo_quad_loss(ctx, D, losses[0:1])
+        if ev:
+            ev[1].record(stream)
+        for i in range(n):
+            zo.zo_perturb(ctx, +1, EPS, i)
+            zo.zo_quad_loss(ctx, D, losses[1 + i:2 + i])
+            zo.zo_restore(ctx)
+            zo.zo_perturb(ctx, -1, EPS, i)
+            zo.zo_quad_loss(ctx, D, losses[1 + n + i:2 + n + i])
+            zo.zo_restore(ctx)
+        if ev:
+            ev[2].record(stream)
+        zo.zo_step(ctx, losses[1:1 + n], losses[1 + n:], n, losses[0:1], LR, EPS, DAMPING)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    for k in range(args.steps):
+        flush.zero_()  # evict theta and D from the 126 MB L2 between steps (not timed)
+        one_step(evs[k])
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    zo.zo_sync(ctx)
+
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    clean_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    probe_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    upd_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    total_s = sum(step_ms) / 1e3
+    if world > 1:
+        t = torch.tensor([total_s], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_s = float(t.item())
+    value = world * args.steps / total_s
+
+    # dominant kernel: the loss pass (perturbation on load); 2n launches per probe phase
+    loss_us = 1e3 * statistics.mean(probe_ms) / (2 * n)
+    loss_bytes = 8 * M_FULL  # theta and D read once, fp32
+    achieved = loss_bytes / (loss_us * 1e-6) / 1e9
+    upd_bytes = 8 * M_FULL  # theta read + written, fp32
+
+    # single-kernel timing of the update (same stream), for its own roofline
+    coef = torch.from_numpy(synth.coefficients(n, seed=1) * 0).to(dev)  # zero: theta unchanged
+    ue = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    flush.zero_()
+    ue[0].record(stream)
+    reps = 10
+    for _ in range(reps):
+        zo.zo_update(ctx, coef, n)
+    ue[1].record(stream)
+    torch.cuda.synchronize()
+    upd_us = 1e3 * ue[0].elapsed_time(ue[1]) / reps
+
+    # end to end through the host-buffer entry point: D copied in, losses copied out
+    D_host = torch.from_numpy(D_np).pin_memory()
+    L_host = torch.zeros(2 * n + 1, dtype=torch.float64).pin_memory()
+    zo.zo_quad_step_host(ctx, D_host, n, EPS, LR, DAMPING, True, L_host)  # staging alloc
+    e2e_steps = max(3, min(args.steps, 10))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        zo.zo_quad_step_host(ctx, D_host, n, EPS, LR, DAMPING, True, L_host)
+    e2e_s = time.perf_counter() - t0
+    if world > 1:
+        t = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_s = float(t.item())
+    e2e_value = world * e2e_steps / e2e_s
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            M_sample = 1 << 20
+            times = time_oracle(M_sample, 2)
+            per = sum(times) / len(times)
+            cpu = {"value": (M_sample / M_FULL) / per, "unit": "steps/s", "cores": 1,
+                   "kind": "oracle",
+                   "sample": "2 oracle steps on the first 2^20 of 2^24 parameters; steps/s scaled by 1/16"}
+        launches_per_step = 1 + 2 * n + 2
+        line = {
+            "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "M": M_FULL, "n_pert": n, "eps": EPS, "lr": LR,
+                       "damping": DAMPING, "parallelism": f"replicas{world}",
+                       "l2": "flushed between steps (256 MiB write, untimed); theta+D = 128 MiB"},
+            "roofline": {"kernel": "quad_loss_kernel (perturbation on load, fp64 accumulation)",
+                         "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "peak_kind": peak_kind,
+                         "bytes_per_launch": loss_bytes, "avg_launch_us": loss_us,
+                         "traffic": None},
+            "kernels": {
+                "update_kernel": {"avg_launch_us": upd_us, "bytes_per_launch": upd_bytes,
+                                  "achieved_GBps": upd_bytes / (upd_us * 1e-6) / 1e9,
+                                  "frac_hbm": upd_bytes / (upd_us * 1e-6) / 1e9 / hbm_peak},
+            },
+            "phases_ms": {"clean_loss": statistics.mean(clean_ms),
+                          "probe_losses": statistics.mean(probe_ms),
+                          "precond_update": statistics.mean(upd_ms)},
+            "tokens_per_s": None,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": 4 * M_FULL,
+                    "d2h_bytes_per_step": 8 * (2 * n + 1),
+                    "path": "zo_quad_step_host: D pinned host -> device each step, losses back"},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+        if args.traffic is not None:
+            line["roofline"]["traffic"] = args.traffic
+    ctx.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu dram bytes per launch of the loss kernel, if measured")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return reference_arm(args)
+    return gpu_arm(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,245 @@
+/*
+ * zo.h -- C ABI of libzo.so: the data-parallel hot path of 1SPSA / 1.5-SPSA
+ * zero-order training on one B200 (sm_100a).
+ *
+ * The method (cited by page title and section):
+ *   [HOW] "Stanford's 1.5-SPSA Trains OPT-30B Without Backpropagation", section
+ *         "How 1.5-SPSA Works": each step draws n_pert Rademacher probes z_i in
+ *         {-1,+1}^M, evaluates the loss at theta + eps*z_i and theta - eps*z_i, and
+ *         averages (L+ - L-)/(2 eps) * z_i over the probes.
+ *   [PSP] same page, section "Probe-Space Preconditioning": one extra clean loss
+ *         L0 per step gives a per-probe curvature; probes are weighted by
+ *         |c_i|^alpha (alpha = 0.1) so that high-curvature directions are
+ *         down-weighted.  The preconditioner lives in probe space (O(n_pert)).
+ *   [ABS] "Probe-Space Preconditioning for Fast and Stable Zero-Order Training",
+ *         abstract: training runs in inference mode with no stored activations,
+ *         gradients or optimizer state; probes come from a packed (8 signs per byte)
+ *         random generator and are applied by fused unpack/apply kernels.
+ *   [LOOP] "Pretraining Transformers Without Backprop: What Two Zero-Order Papers
+ *         Actually Measure", section "Backprop's memory tax", loop flowchart:
+ *         directions -> forward passes (loss only) -> preconditioned estimate ->
+ *         update -> repeat.
+ *
+ * Readings fixed by this library where the pages are silent:
+ *   - Probe bits: Philox4x32-10 (Salmon et al., SC'11), key = (seed lo, seed hi),
+ *     counter = (g lo, g hi, probe, step) with g = j >> 7; element j takes bit j & 31
+ *     of word (j >> 5) & 3; bit 1 means z_j = -1.  Packed byte q holds elements
+ *     8q..8q+7, bit t <-> element 8q+t.  Probes are regenerated, never stored.
+ *   - Perturbed value P_j = rd(theta_j + s*eps*z_j): one fp32 add (RNE); bf16 weights
+ *     are widened, added in fp32 and rounded to bf16 (RNE).
+ *   - g_i = (L+_i - L-_i)/(2 eps); c_i = (L+_i + L-_i - 2 L0)/eps^2;
+ *     w_i = (|c_i| + damping)^(-alpha) (1SPSA: w_i = 1); a_i = lr*w_i*g_i/n, all in
+ *     fp64, a_i rounded once to fp32.
+ *   - theta' = rd(theta - sum_i a_i z_i) with a fixed fp32 order: probes in groups of
+ *     8 (each group summed left to right from its first signed term), group sums
+ *     added left to right, one fp32 subtraction, one rounding to the storage type.
+ *   - "In place" and "exact restore": theta is written only by zo_step/zo_update.
+ *     A perturbation is a state of the context; kernels that need perturbed values
+ *     compute them on load or materialise them into a scratch window (the whole
+ *     vector when a live buffer is enabled, one decoder layer at a time otherwise).
+ *     zo_restore therefore returns theta bit-exactly, with no pass over memory.
+ *
+ * Conventions for every call:
+ *   - Pointers documented as "device" must be device memory of the current device
+ *     (e.g. torch CUDA tensors); "host" pointers are ordinary host memory.
+ *   - Calls enqueue work on the context's stream and return without synchronising,
+ *     unless documented otherwise.  The step counter lives in device memory, so a
+ *     sequence of calls can be captured into a CUDA graph and replayed.
+ *   - Every call returns a zo_status; on failure zo_last_error(ctx) describes it.
+ *     No call throws, aborts or prints.  A context is not thread-safe.
+ */
+#ifndef ZO_H
+#define ZO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct zo_ctx zo_ctx;
+
+typedef enum { ZO_F32 = 0, ZO_BF16 = 1 } zo_dtype;
+
+typedef enum {
+  ZO_OK = 0,
+  ZO_ERR_INVALID = 1,     /* bad argument (size, sign, eps, pointer alignment, dtype) */
+  ZO_ERR_STATE = 2,       /* call not allowed in the context's perturbation state */
+  ZO_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+  ZO_ERR_OOM = 4,         /* device allocation failed */
+  ZO_ERR_NONFINITE = 5,   /* a loss was NaN/Inf: the step was skipped (theta unchanged) */
+  ZO_ERR_UNSUPPORTED = 6  /* valid request this build does not support */
+} zo_status;
+
+/* Device-side status flags reported by zo_sync / zo_device_flags. */
+#define ZO_FLAG_NONFINITE 0x1u
+
+/* Largest n_pert accepted by zo_step / zo_update (the update keeps a 1 KB table per
+ * group of 8 probes in shared memory: 128 KB at this limit). */
+#define ZO_MAX_PROBES 1024
+
+/* ------------------------------------------------------------------ context */
+
+/* Create a context over the flat parameter vector theta [ABS: the weights are the only
+ * training state].
+ *   params  device, caller-owned, M elements of `dtype`, 16-byte aligned; must outlive
+ *           the context.  The library writes it only in zo_step / zo_update.
+ *   M       number of parameters, 1 <= M < 2^39.
+ *   dtype   ZO_F32 or ZO_BF16.
+ *   seed    64-bit probe seed (Philox key).
+ *   stream  cudaStream_t to enqueue on (NULL = legacy default stream).
+ * Allocates small device buffers (step counter, coefficients, reduction scratch).
+ * Errors: ZO_ERR_INVALID (null out/params, M out of range, misaligned params, dtype),
+ *         ZO_ERR_OOM, ZO_ERR_CUDA.  The step counter starts at 0. */
+zo_status zo_create(zo_ctx **out, void *params, int64_t M, int dtype, uint64_t seed,
+                    void *stream);
+
+/* Free the context and everything it allocated (synchronises its stream first).
+ * NULL is accepted.  theta is not touched. */
+zo_status zo_destroy(zo_ctx *ctx);
+
+/* Text of the last error on this context ("" if none); valid until the next call. */
+const char *zo_last_error(const zo_ctx *ctx);
+
+/* Constant name of a status code, e.g. "ZO_ERR_STATE". */
+const char *zo_status_name(int status);
+
+/* Exponent alpha of the probe-space weights (default 0.1 [PSP]); must be finite, >= 0. */
+zo_status zo_set_alpha(zo_ctx *ctx, float alpha);
+
+/* Enable (1) or disable (0) the full-size live buffer: while perturbed, a device copy
+ * P = rd(theta + s*eps*z_i) of all M parameters is materialised by zo_perturb and
+ * returned by zo_live_params.  Costs M elements of device memory.  Only allowed in the
+ * clean state.  Errors: ZO_ERR_STATE, ZO_ERR_OOM. */
+zo_status zo_set_live_buffer(zo_ctx *ctx, int enable);
+
+/* The parameters a loss evaluation should read now: theta when clean (or when no live
+ * buffer is enabled), else the live buffer.  NULL on a NULL context. */
+const void *zo_live_params(const zo_ctx *ctx);
+
+/* Synchronise the context's stream and return the sticky device flags (ZO_FLAG_*)
+ * raised since the last call, clearing them; *flags may be NULL.  Returns
+ * ZO_ERR_NONFINITE if ZO_FLAG_NONFINITE was raised, else ZO_OK. */
+zo_status zo_sync(zo_ctx *ctx, uint32_t *flags);
+
+/* Read (synchronising) or set (enqueued) the device-resident step counter, which keys
+ * the probes of the current step.  Setting it is how a run resumes from a checkpoint
+ * of (theta, seed, step): the method keeps no other state [ABS]. */
+zo_status zo_get_step(zo_ctx *ctx, uint32_t *step);
+zo_status zo_set_step(zo_ctx *ctx, uint32_t step);
+
+/* ------------------------------------------------------------------ zo_rng */
+
+/* Write packed probe bytes [first_byte, first_byte + nbytes) of probe `probe` at the
+ * current step into dev_out (device, nbytes bytes) [ABS: 8 signs per byte].  Bits of
+ * elements >= M are 0.  For tests and inspection: the training path regenerates probe
+ * bits in registers and never stores them.
+ * Errors: ZO_ERR_INVALID (probe < 0, range outside ceil(M/8) bytes, null dev_out). */
+zo_status zo_pack_probe(zo_ctx *ctx, int32_t probe, int64_t first_byte, int64_t nbytes,
+                        uint8_t *dev_out);
+
+/* ------------------------------------------------------------------ zo_perturb */
+
+/* Enter the perturbed state theta + sign*eps*z_probe [HOW].  If the live buffer is
+ * enabled this launches the fused unpack/apply kernel that writes all M perturbed
+ * values into it; otherwise it only records (sign, eps, probe) for the loss kernels.
+ *   sign  +1 or -1;  eps > 0 and finite;  probe >= 0.
+ * Errors: ZO_ERR_INVALID, ZO_ERR_STATE (already perturbed), ZO_ERR_CUDA. */
+zo_status zo_perturb(zo_ctx *ctx, int sign, float eps, int32_t probe);
+
+/* Return to the clean state.  theta was never written, so this is exact and moves no
+ * memory.  Errors: ZO_ERR_STATE (not perturbed). */
+zo_status zo_restore(zo_ctx *ctx);
+
+/* Materialise P = rd(theta + s*eps*z) (perturbed state) or theta (clean state) for
+ * elements [first, first + count) into dev_out (device, count elements of the
+ * context's dtype; 16-byte alignment and first % 8 == 0 give the vectorised path).
+ * This is the per-window form of the unpack/apply kernel.
+ * Errors: ZO_ERR_INVALID (range outside [0, M), null dev_out), ZO_ERR_CUDA. */
+zo_status zo_perturb_range(zo_ctx *ctx, int64_t first, int64_t count, void *dev_out);
+
+/* ------------------------------------------------------------------ losses (zo_forward) */
+
+/* Diagonal quadratic L = 1/2 sum_j D_j P_j^2 at the current state, perturbation applied
+ * on load (theta is read, never written), every term and sum in fp64, fixed reduction
+ * order (deterministic).  Requires an ZO_F32 context.
+ *   D         device, M floats.
+ *   loss_out  device, one double: *loss_out = L, or += L when accumulate != 0.
+ * Uses the context's reduction scratch; calls on one context must not overlap.
+ * Errors: ZO_ERR_INVALID, ZO_ERR_UNSUPPORTED (bf16 context), ZO_ERR_CUDA. */
+zo_status zo_quad_loss(zo_ctx *ctx, const float *D, double *loss_out, int accumulate);
+
+/* Cross-entropy of an MLP classifier in -> hidden (ReLU) -> out evaluated at
+ * zo_live_params(ctx) (fp32 CUDA-core arithmetic, no TF32), flat parameter order
+ * W1[hidden][in], b1[hidden], W2[out][hidden], b2[out] (M must match).
+ *   X        device, batch x n_in floats (row-major);  labels: device, batch int32 in
+ *            [0, n_out).
+ *   scale    multiplies the summed per-sample losses (1/batch gives the mean; 1/B_eff
+ *            accumulates micro-batches into an effective-batch mean).
+ *   loss_out device double: = scale*sum (accumulate == 0) or += scale*sum.
+ * Requires a ZO_F32 context with the live buffer enabled when perturbed.
+ * Limits: 1 <= n_in <= 1024, 1 <= n_hidden <= 1024, 1 <= n_out <= 1024, batch >= 1.
+ * Errors: ZO_ERR_INVALID, ZO_ERR_STATE (perturbed without a live buffer),
+ *         ZO_ERR_UNSUPPORTED, ZO_ERR_CUDA. */
+zo_status zo_mlp_loss(zo_ctx *ctx, const float *X, const int32_t *labels, int batch,
+                      int n_in, int n_hidden, int n_out, double scale, double *loss_out,
+                      int accumulate);
+
+/* ------------------------------------------------------------------ zo_precond + zo_update */
+
+/* One optimizer step from the losses of the current step [HOW][PSP]:
+ *   loss_plus, loss_minus  device, n_pert doubles each (L(theta +- eps z_i));
+ *   loss0                  device double (clean loss) for 1.5-SPSA, NULL for 1SPSA;
+ *   lr, eps, damping       eps must be the one the losses were taken with.
+ * Launches the probe-space preconditioner (one CTA, warp-shuffle reductions) and the
+ * single-pass update that regenerates every probe in registers: theta is read once and
+ * written once.  If any loss is not finite, theta and the step counter are left
+ * unchanged and ZO_FLAG_NONFINITE is raised (seen by zo_sync); otherwise the step
+ * counter advances by one.  No host synchronisation.
+ * Errors: ZO_ERR_INVALID (n_pert outside [1, ZO_MAX_PROBES], eps <= 0, non-finite lr or
+ *         damping < 0), ZO_ERR_STATE (perturbed), ZO_ERR_CUDA. */
+zo_status zo_step(zo_ctx *ctx, const double *loss_plus, const double *loss_minus,
+                  int32_t n_pert, const double *loss0, float lr, float eps, float damping);
+
+/* The update alone: theta <- rd(theta - sum_i coef_i z_i) with coef (device, n_pert
+ * floats) at the current step, in the fixed fp32 order above.  Does not advance the
+ * step counter.  Errors as zo_step. */
+zo_status zo_update(zo_ctx *ctx, const float *coef, int32_t n_pert);
+
+/* Copy the last zo_step's fp64 g_i, c_i, w_i (host arrays of n doubles each, any may be
+ * NULL) and fp32 coefficients a_i (host, n floats, may be NULL).  Synchronises.
+ * Errors: ZO_ERR_INVALID (n outside [1, last n_pert]). */
+zo_status zo_get_precond(zo_ctx *ctx, int32_t n, double *g, double *c, double *w,
+                         float *a);
+
+/* ------------------------------------------------------------------ step driver */
+
+/* One full step on the diagonal quadratic [LOOP]: clean loss (1.5-SPSA), then for each
+ * probe the losses at +eps and -eps (perturbation on load), then zo_step.
+ *   D           device, M floats;  losses_out device, 2*n_pert+1 doubles receiving
+ *               [L0, L+_0..L+_{n-1}, L-_0..L-_{n-1}] (L0 = 0 for 1SPSA).
+ *   preconditioned  1 = 1.5-SPSA, 0 = 1SPSA.
+ * Errors: as zo_quad_loss and zo_step. */
+zo_status zo_quad_step(zo_ctx *ctx, const float *D, int32_t n_pert, float eps, float lr,
+                       float damping, int preconditioned, double *losses_out);
+
+/* The same step with host buffers: copies D (host, M floats) to the device, runs the
+ * step, and copies the 2*n_pert+1 losses back to losses_host (host).  Synchronises.
+ * Device staging memory for D is owned by the context (allocated on first use). */
+zo_status zo_quad_step_host(zo_ctx *ctx, const float *D_host, int32_t n_pert, float eps,
+                            float lr, float damping, int preconditioned,
+                            double *losses_host);
+
+/* One full MLP step [LOOP] (live buffer enabled by the call if needed): clean loss,
+ * 2*n_pert perturbed losses through the live buffer, zo_step.  Arguments as
+ * zo_mlp_loss; losses_out as zo_quad_step. */
+zo_status zo_mlp_step(zo_ctx *ctx, const float *X, const int32_t *labels, int batch,
+                      int n_in, int n_hidden, int n_out, int32_t n_pert, float eps,
+                      float lr, float damping, int preconditioned, double *losses_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZO_H */

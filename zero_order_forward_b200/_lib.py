@@ -1,0 +1,229 @@
+"""ctypes binding of libzo.so: the C ABI of include/zo.h with the same names.
+
+Argument marshalling only: torch tensors are passed as raw device pointers and the
+current torch CUDA stream as the context's stream.  Every step of the hot path runs in
+the library's CUDA kernels; there is no Python or CPU fallback.  If libzo.so is
+missing, importing this module raises ImportError.
+"""
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libzo.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        "libzo.so is not built; run `python -m zero_order_forward_b200.build` "
+        "(nvcc, sm_100a) before using zero_order_forward_b200")
+
+_L = ctypes.CDLL(LIB_PATH)
+
+ZO_F32, ZO_BF16 = 0, 1
+ZO_OK, ZO_ERR_INVALID, ZO_ERR_STATE, ZO_ERR_CUDA, ZO_ERR_OOM, ZO_ERR_NONFINITE, ZO_ERR_UNSUPPORTED = range(7)
+ZO_FLAG_NONFINITE = 0x1
+ZO_MAX_PROBES = 1024
+
+_vp, _i32, _i64, _u32, _u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_uint64
+_f32, _f64, _int = ctypes.c_float, ctypes.c_double, ctypes.c_int
+
+_SIGS = {
+    "zo_create": [ctypes.POINTER(_vp), _vp, _i64, _int, _u64, _vp],
+    "zo_destroy": [_vp],
+    "zo_set_alpha": [_vp, _f32],
+    "zo_set_live_buffer": [_vp, _int],
+    "zo_sync": [_vp, ctypes.POINTER(_u32)],
+    "zo_get_step": [_vp, ctypes.POINTER(_u32)],
+    "zo_set_step": [_vp, _u32],
+    "zo_pack_probe": [_vp, _i32, _i64, _i64, _vp],
+    "zo_perturb": [_vp, _int, _f32, _i32],
+    "zo_restore": [_vp],
+    "zo_perturb_range": [_vp, _i64, _i64, _vp],
+    "zo_quad_loss": [_vp, _vp, _vp, _int],
+    "zo_mlp_loss": [_vp, _vp, _vp, _int, _int, _int, _int, _f64, _vp, _int],
+    "zo_step": [_vp, _vp, _vp, _i32, _vp, _f32, _f32, _f32],
+    "zo_update": [_vp, _vp, _i32],
+    "zo_get_precond": [_vp, _i32, _vp, _vp, _vp, _vp],
+    "zo_quad_step": [_vp, _vp, _i32, _f32, _f32, _f32, _int, _vp],
+    "zo_quad_step_host": [_vp, _vp, _i32, _f32, _f32, _f32, _int, _vp],
+    "zo_mlp_step": [_vp, _vp, _vp, _int, _int, _int, _int, _i32, _f32, _f32, _f32, _int, _vp],
+}
+for _name, _args in _SIGS.items():
+    _fn = getattr(_L, _name)
+    _fn.argtypes = _args
+    _fn.restype = _int
+_L.zo_last_error.argtypes = [_vp]
+_L.zo_last_error.restype = ctypes.c_char_p
+_L.zo_status_name.argtypes = [_int]
+_L.zo_status_name.restype = ctypes.c_char_p
+_L.zo_live_params.argtypes = [_vp]
+_L.zo_live_params.restype = _vp
+
+lib = _L
+
+
+class ZoError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"{_L.zo_status_name(status).decode()}: {msg}")
+        self.status = status
+
+
+def _ptr(t):
+    """Device (or host) address of a tensor / numpy array / int / None."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if hasattr(t, "data_ptr"):
+        return t.data_ptr()
+    if hasattr(t, "ctypes"):
+        return t.ctypes.data
+    raise TypeError(type(t))
+
+
+def _stream(stream):
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+class Ctx:
+    """Owns a zo_ctx*; keeps the parameter tensor alive."""
+
+    def __init__(self, handle, params, M, dtype):
+        self.handle, self.params, self.M, self.dtype = handle, params, M, dtype
+
+    def check(self, status):
+        if status != ZO_OK:
+            msg = _L.zo_last_error(self.handle) if self.handle else b""
+            raise ZoError(status, msg.decode() if msg else "")
+        return status
+
+    def close(self):
+        if self.handle:
+            _L.zo_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def zo_create(params, seed=0, stream=None, M=None, dtype=None):
+    """params: a CUDA tensor (float32 or bfloat16) holding the flat theta."""
+    import torch
+    if dtype is None:
+        dtype = {torch.float32: ZO_F32, torch.bfloat16: ZO_BF16}[params.dtype]
+    if M is None:
+        M = params.numel()
+    h = _vp()
+    st = _L.zo_create(ctypes.byref(h), _ptr(params), int(M), int(dtype), int(seed) & (2**64 - 1),
+                      _stream(stream))
+    if st != ZO_OK:
+        raise ZoError(st, "zo_create failed")
+    return Ctx(h, params, M, dtype)
+
+
+def zo_destroy(ctx):
+    ctx.close()
+
+
+def zo_last_error(ctx):
+    return _L.zo_last_error(ctx.handle).decode()
+
+
+def zo_status_name(status):
+    return _L.zo_status_name(status).decode()
+
+
+def zo_set_alpha(ctx, alpha):
+    return ctx.check(_L.zo_set_alpha(ctx.handle, alpha))
+
+
+def zo_set_live_buffer(ctx, enable):
+    return ctx.check(_L.zo_set_live_buffer(ctx.handle, int(bool(enable))))
+
+
+def zo_live_params(ctx):
+    return _L.zo_live_params(ctx.handle)
+
+
+def zo_sync(ctx, raise_nonfinite=True):
+    flags = _u32()
+    st = _L.zo_sync(ctx.handle, ctypes.byref(flags))
+    if st == ZO_ERR_NONFINITE and not raise_nonfinite:
+        return flags.value
+    ctx.check(st)
+    return flags.value
+
+
+def zo_get_step(ctx):
+    s = _u32()
+    ctx.check(_L.zo_get_step(ctx.handle, ctypes.byref(s)))
+    return s.value
+
+
+def zo_set_step(ctx, step):
+    return ctx.check(_L.zo_set_step(ctx.handle, step))
+
+
+def zo_pack_probe(ctx, probe, first_byte, nbytes, out):
+    return ctx.check(_L.zo_pack_probe(ctx.handle, probe, first_byte, nbytes, _ptr(out)))
+
+
+def zo_perturb(ctx, sign, eps, probe):
+    return ctx.check(_L.zo_perturb(ctx.handle, sign, eps, probe))
+
+
+def zo_restore(ctx):
+    return ctx.check(_L.zo_restore(ctx.handle))
+
+
+def zo_perturb_range(ctx, first, count, out):
+    return ctx.check(_L.zo_perturb_range(ctx.handle, first, count, _ptr(out)))
+
+
+def zo_quad_loss(ctx, D, loss_out, accumulate=False):
+    return ctx.check(_L.zo_quad_loss(ctx.handle, _ptr(D), _ptr(loss_out), int(accumulate)))
+
+
+def zo_mlp_loss(ctx, X, labels, batch, n_in, n_hidden, n_out, scale, loss_out, accumulate=False):
+    return ctx.check(_L.zo_mlp_loss(ctx.handle, _ptr(X), _ptr(labels), batch, n_in, n_hidden,
+                                    n_out, scale, _ptr(loss_out), int(accumulate)))
+
+
+def zo_step(ctx, loss_plus, loss_minus, n_pert, loss0, lr, eps, damping):
+    return ctx.check(_L.zo_step(ctx.handle, _ptr(loss_plus), _ptr(loss_minus), n_pert,
+                                _ptr(loss0), lr, eps, damping))
+
+
+def zo_update(ctx, coef, n_pert):
+    return ctx.check(_L.zo_update(ctx.handle, _ptr(coef), n_pert))
+
+
+def zo_get_precond(ctx, n):
+    """Returns (g, c, w, a) as numpy arrays from the last zo_step (synchronises)."""
+    import numpy as np
+    g, c, w = (np.zeros(n, np.float64) for _ in range(3))
+    a = np.zeros(n, np.float32)
+    ctx.check(_L.zo_get_precond(ctx.handle, n, g.ctypes.data, c.ctypes.data, w.ctypes.data, a.ctypes.data))
+    return g, c, w, a
+
+
+def zo_quad_step(ctx, D, n_pert, eps, lr, damping, preconditioned, losses_out):
+    return ctx.check(_L.zo_quad_step(ctx.handle, _ptr(D), n_pert, eps, lr, damping,
+                                     int(preconditioned), _ptr(losses_out)))
+
+
+def zo_quad_step_host(ctx, D_host, n_pert, eps, lr, damping, preconditioned, losses_host):
+    return ctx.check(_L.zo_quad_step_host(ctx.handle, _ptr(D_host), n_pert, eps, lr, damping,
+                                          int(preconditioned), _ptr(losses_host)))
+
+
+def zo_mlp_step(ctx, X, labels, batch, n_in, n_hidden, n_out, n_pert, eps, lr, damping,
+                preconditioned, losses_out):
+    return ctx.check(_L.zo_mlp_step(ctx.handle, _ptr(X), _ptr(labels), batch, n_in, n_hidden,
+                                    n_out, n_pert, eps, lr, damping, int(preconditioned),
+                                    _ptr(losses_out)))

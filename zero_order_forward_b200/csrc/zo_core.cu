@@ -1,0 +1,390 @@
+// zo_core.cu -- the C ABI of libzo.so: context, perturbation state machine, argument
+// checking, and the step drivers that order the kernels of one step.
+//
+// Step order ("Pretraining Transformers Without Backprop: What Two Zero-Order Papers
+// Actually Measure", section "Backprop's memory tax", loop flowchart; the clean pass of
+// 1.5-SPSA from "Stanford's 1.5-SPSA Trains OPT-30B Without Backpropagation", section
+// "Probe-Space Preconditioning"):
+//   clean loss L0 -> for each probe i: loss at theta+eps z_i, loss at theta-eps z_i ->
+//   preconditioner -> update (step counter + 1).
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "zo_internal.cuh"
+
+namespace zo {
+
+zo_status fail(zo_ctx *ctx, zo_status st, const char *fmt, ...) {
+  if (ctx) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    ctx->err = buf;
+  }
+  return st;
+}
+
+zo_status check_launch(zo_ctx *ctx, const char *what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess)
+    return fail(ctx, ZO_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return ZO_OK;
+}
+
+ProbeKey probe_key(const zo_ctx *ctx) {
+  ProbeKey pk;
+  pk.k0 = (uint32_t)ctx->seed;
+  pk.k1 = (uint32_t)(ctx->seed >> 32);
+  pk.step = &ctx->dstate->step;
+  pk.probe = (uint32_t)ctx->probe;
+  pk.sign = ctx->state == PState::Perturbed ? ctx->sign : 0;
+  pk.eps = ctx->eps;
+  return pk;
+}
+
+}  // namespace zo
+
+using namespace zo;
+
+namespace {
+
+size_t elem_size(int dtype) { return dtype == ZO_F32 ? 4 : 2; }
+
+zo_status cuda_fail(zo_ctx *ctx, cudaError_t e, const char *what) {
+  if (e == cudaErrorMemoryAllocation) {
+    cudaGetLastError();
+    return fail(ctx, ZO_ERR_OOM, "%s: out of device memory", what);
+  }
+  return fail(ctx, ZO_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define ZO_CUDA(ctx, call, what)                      \
+  do {                                                \
+    const cudaError_t e_ = (call);                    \
+    if (e_ != cudaSuccess) return cuda_fail(ctx, e_, what); \
+  } while (0)
+
+#define ZO_CHECK(expr)                 \
+  do {                                 \
+    const zo_status s_ = (expr);       \
+    if (s_ != ZO_OK) return s_;        \
+  } while (0)
+
+zo_status check_ctx(zo_ctx *ctx) {
+  if (!ctx) return ZO_ERR_INVALID;
+  ctx->err.clear();
+  ZO_CUDA(ctx, cudaSetDevice(ctx->device), "cudaSetDevice");
+  return ZO_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+zo_status check_step_args(zo_ctx *ctx, int32_t n, float lr, float eps, float damping) {
+  if (n < 1 || n > ZO_MAX_PROBES)
+    return fail(ctx, ZO_ERR_INVALID, "n_pert=%d outside [1, %d]", n, ZO_MAX_PROBES);
+  if (!(eps > 0.f) || !std::isfinite(eps)) return fail(ctx, ZO_ERR_INVALID, "eps must be finite and > 0");
+  if (!std::isfinite(lr)) return fail(ctx, ZO_ERR_INVALID, "lr must be finite");
+  if (!(damping >= 0.f) || !std::isfinite(damping))
+    return fail(ctx, ZO_ERR_INVALID, "damping must be finite and >= 0");
+  return ZO_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *zo_status_name(int s) {
+  switch (s) {
+    case ZO_OK: return "ZO_OK";
+    case ZO_ERR_INVALID: return "ZO_ERR_INVALID";
+    case ZO_ERR_STATE: return "ZO_ERR_STATE";
+    case ZO_ERR_CUDA: return "ZO_ERR_CUDA";
+    case ZO_ERR_OOM: return "ZO_ERR_OOM";
+    case ZO_ERR_NONFINITE: return "ZO_ERR_NONFINITE";
+    case ZO_ERR_UNSUPPORTED: return "ZO_ERR_UNSUPPORTED";
+    default: return "ZO_ERR_UNKNOWN";
+  }
+}
+
+const char *zo_last_error(const zo_ctx *ctx) { return ctx ? ctx->err.c_str() : "null context"; }
+
+zo_status zo_create(zo_ctx **out, void *params, int64_t M, int dtype, uint64_t seed,
+                    void *stream) {
+  if (!out) return ZO_ERR_INVALID;
+  *out = nullptr;
+  if (!params || M < 1 || M >= ((int64_t)1 << 39) || (dtype != ZO_F32 && dtype != ZO_BF16) ||
+      !aligned16(params))
+    return ZO_ERR_INVALID;
+  zo_ctx *ctx = new (std::nothrow) zo_ctx();
+  if (!ctx) return ZO_ERR_OOM;
+  ctx->params = params;
+  ctx->M = M;
+  ctx->dtype = dtype;
+  ctx->seed = seed;
+  ctx->stream = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaGetDevice(&ctx->device);
+  if (e == cudaSuccess) e = cudaMalloc(&ctx->dstate, sizeof(DevState));
+  if (e == cudaSuccess) e = cudaMalloc(&ctx->coef, ZO_MAX_PROBES * sizeof(float));
+  if (e == cudaSuccess) e = cudaMalloc(&ctx->diag, (3 * ZO_MAX_PROBES + 8) * sizeof(double));
+  if (e == cudaSuccess) e = cudaMalloc(&ctx->partials, kMaxPartials * sizeof(double));
+  if (e == cudaSuccess) e = cudaMalloc(&ctx->counter, sizeof(unsigned int));
+  if (e == cudaSuccess) e = cudaMemsetAsync(ctx->dstate, 0, sizeof(DevState), ctx->stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ctx->counter, 0, sizeof(unsigned int), ctx->stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ctx->diag, 0, (3 * ZO_MAX_PROBES + 8) * sizeof(double), ctx->stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->stream);
+  if (e != cudaSuccess) {
+    const zo_status st = e == cudaErrorMemoryAllocation ? ZO_ERR_OOM : ZO_ERR_CUDA;
+    cudaGetLastError();
+    zo_destroy(ctx);
+    return st;
+  }
+  *out = ctx;
+  return ZO_OK;
+}
+
+zo_status zo_destroy(zo_ctx *ctx) {
+  if (!ctx) return ZO_OK;
+  cudaSetDevice(ctx->device);
+  cudaStreamSynchronize(ctx->stream);
+  cudaFree(ctx->dstate);
+  cudaFree(ctx->coef);
+  cudaFree(ctx->diag);
+  cudaFree(ctx->partials);
+  cudaFree(ctx->counter);
+  cudaFree(ctx->live);
+  cudaFree(ctx->staging);
+  cudaFree(ctx->loss_scratch);
+  delete ctx;
+  return ZO_OK;
+}
+
+zo_status zo_set_alpha(zo_ctx *ctx, float alpha) {
+  ZO_CHECK(check_ctx(ctx));
+  if (!std::isfinite(alpha) || alpha < 0.f) return fail(ctx, ZO_ERR_INVALID, "alpha must be finite and >= 0");
+  ctx->alpha = alpha;
+  return ZO_OK;
+}
+
+zo_status zo_set_live_buffer(zo_ctx *ctx, int enable) {
+  ZO_CHECK(check_ctx(ctx));
+  if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "live buffer can only change when clean");
+  if (enable && !ctx->live) {
+    ZO_CUDA(ctx, cudaMalloc(&ctx->live, (size_t)ctx->M * elem_size(ctx->dtype)), "live buffer");
+  } else if (!enable && ctx->live) {
+    ZO_CUDA(ctx, cudaStreamSynchronize(ctx->stream), "sync");
+    cudaFree(ctx->live);
+    ctx->live = nullptr;
+  }
+  ctx->live_enabled = enable != 0;
+  return ZO_OK;
+}
+
+const void *zo_live_params(const zo_ctx *ctx) {
+  if (!ctx) return nullptr;
+  if (ctx->state == PState::Perturbed && ctx->live_enabled) return ctx->live;
+  return ctx->params;
+}
+
+zo_status zo_sync(zo_ctx *ctx, uint32_t *flags) {
+  ZO_CHECK(check_ctx(ctx));
+  ZO_CUDA(ctx, cudaStreamSynchronize(ctx->stream), "cudaStreamSynchronize");
+  DevState s;
+  ZO_CUDA(ctx, cudaMemcpy(&s, ctx->dstate, sizeof s, cudaMemcpyDeviceToHost), "read state");
+  if (s.flags) {
+    ZO_CUDA(ctx, cudaMemset(&ctx->dstate->flags, 0, sizeof(uint32_t)), "clear flags");
+  }
+  if (flags) *flags = s.flags;
+  if (s.flags & ZO_FLAG_NONFINITE) return fail(ctx, ZO_ERR_NONFINITE, "a loss was not finite; step skipped");
+  return ZO_OK;
+}
+
+zo_status zo_get_step(zo_ctx *ctx, uint32_t *step) {
+  ZO_CHECK(check_ctx(ctx));
+  if (!step) return fail(ctx, ZO_ERR_INVALID, "null step");
+  ZO_CUDA(ctx, cudaMemcpyAsync(step, &ctx->dstate->step, sizeof(uint32_t), cudaMemcpyDeviceToHost,
+                               ctx->stream), "read step");
+  ZO_CUDA(ctx, cudaStreamSynchronize(ctx->stream), "sync");
+  return ZO_OK;
+}
+
+zo_status zo_set_step(zo_ctx *ctx, uint32_t step) {
+  ZO_CHECK(check_ctx(ctx));
+  if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "set_step while perturbed");
+  static_assert(sizeof(uint32_t) == 4, "");
+  // cuMemsetD32-style enqueue through a tiny host->device copy of a pinned-free value.
+  ZO_CUDA(ctx, cudaMemcpyAsync(&ctx->dstate->step, &step, sizeof step, cudaMemcpyHostToDevice,
+                               ctx->stream), "write step");
+  ZO_CUDA(ctx, cudaStreamSynchronize(ctx->stream), "sync");
+  return ZO_OK;
+}
+
+zo_status zo_pack_probe(zo_ctx *ctx, int32_t probe, int64_t first_byte, int64_t nbytes,
+                        uint8_t *dev_out) {
+  ZO_CHECK(check_ctx(ctx));
+  const int64_t total = (ctx->M + 7) / 8;
+  if (probe < 0 || !dev_out || first_byte < 0 || nbytes < 0 || first_byte + nbytes > total)
+    return fail(ctx, ZO_ERR_INVALID, "pack range outside [0, %lld) bytes", (long long)total);
+  return launch_pack(ctx, (uint32_t)probe, first_byte, nbytes, dev_out);
+}
+
+zo_status zo_perturb(zo_ctx *ctx, int sign, float eps, int32_t probe) {
+  ZO_CHECK(check_ctx(ctx));
+  if (sign != 1 && sign != -1) return fail(ctx, ZO_ERR_INVALID, "sign must be +1 or -1");
+  if (!(eps > 0.f) || !std::isfinite(eps)) return fail(ctx, ZO_ERR_INVALID, "eps must be finite and > 0");
+  if (probe < 0) return fail(ctx, ZO_ERR_INVALID, "probe must be >= 0");
+  if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "already perturbed; call zo_restore first");
+  ctx->state = PState::Perturbed;
+  ctx->sign = sign;
+  ctx->eps = eps;
+  ctx->probe = probe;
+  if (ctx->live_enabled) {
+    const zo_status st = launch_perturb(ctx, probe_key(ctx), 0, ctx->M, ctx->live);
+    if (st != ZO_OK) {
+      ctx->state = PState::Clean;
+      return st;
+    }
+  }
+  return ZO_OK;
+}
+
+zo_status zo_restore(zo_ctx *ctx) {
+  ZO_CHECK(check_ctx(ctx));
+  if (ctx->state != PState::Perturbed) return fail(ctx, ZO_ERR_STATE, "not perturbed");
+  ctx->state = PState::Clean;
+  ctx->sign = 0;
+  return ZO_OK;
+}
+
+zo_status zo_perturb_range(zo_ctx *ctx, int64_t first, int64_t count, void *dev_out) {
+  ZO_CHECK(check_ctx(ctx));
+  if (!dev_out || first < 0 || count < 0 || first + count > ctx->M)
+    return fail(ctx, ZO_ERR_INVALID, "range outside [0, M)");
+  return launch_perturb(ctx, probe_key(ctx), first, count, dev_out);
+}
+
+zo_status zo_quad_loss(zo_ctx *ctx, const float *D, double *loss_out, int accumulate) {
+  ZO_CHECK(check_ctx(ctx));
+  if (ctx->dtype != ZO_F32) return fail(ctx, ZO_ERR_UNSUPPORTED, "quadratic loss needs an fp32 context");
+  if (!D || !loss_out || !aligned16(D)) return fail(ctx, ZO_ERR_INVALID, "D must be a 16-byte aligned device pointer");
+  return launch_quad_loss(ctx, probe_key(ctx), D, loss_out, accumulate, ctx->partials, ctx->counter);
+}
+
+zo_status zo_mlp_loss(zo_ctx *ctx, const float *X, const int32_t *labels, int batch, int n_in,
+                      int n_hidden, int n_out, double scale, double *loss_out, int accumulate) {
+  ZO_CHECK(check_ctx(ctx));
+  if (ctx->dtype != ZO_F32) return fail(ctx, ZO_ERR_UNSUPPORTED, "MLP loss needs an fp32 context");
+  if (!X || !labels || !loss_out || batch < 1 || n_in < 1 || n_hidden < 1 || n_out < 1)
+    return fail(ctx, ZO_ERR_INVALID, "bad MLP arguments");
+  const int64_t need = (int64_t)n_hidden * n_in + n_hidden + (int64_t)n_out * n_hidden + n_out;
+  if (need != ctx->M) return fail(ctx, ZO_ERR_INVALID, "MLP shape needs M=%lld", (long long)need);
+  if (ctx->state == PState::Perturbed && !ctx->live_enabled)
+    return fail(ctx, ZO_ERR_STATE, "perturbed MLP loss needs the live buffer");
+  return launch_mlp_loss(ctx, static_cast<const float *>(zo_live_params(ctx)), X, labels, batch,
+                         n_in, n_hidden, n_out, scale, loss_out, accumulate);
+}
+
+zo_status zo_step(zo_ctx *ctx, const double *loss_plus, const double *loss_minus, int32_t n_pert,
+                  const double *loss0, float lr, float eps, float damping) {
+  ZO_CHECK(check_ctx(ctx));
+  ZO_CHECK(check_step_args(ctx, n_pert, lr, eps, damping));
+  if (!loss_plus || !loss_minus) return fail(ctx, ZO_ERR_INVALID, "null loss arrays");
+  if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "zo_step while perturbed");
+  ZO_CHECK(launch_precond(ctx, loss_plus, loss_minus, loss0, n_pert, lr, eps, damping));
+  return launch_update(ctx, ctx->coef, n_pert, &ctx->dstate->upd_step, &ctx->dstate->upd_ok);
+}
+
+zo_status zo_update(zo_ctx *ctx, const float *coef, int32_t n_pert) {
+  ZO_CHECK(check_ctx(ctx));
+  if (n_pert < 1 || n_pert > ZO_MAX_PROBES) return fail(ctx, ZO_ERR_INVALID, "n_pert out of range");
+  if (!coef) return fail(ctx, ZO_ERR_INVALID, "null coefficients");
+  if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "zo_update while perturbed");
+  return launch_update(ctx, coef, n_pert, &ctx->dstate->step, nullptr);
+}
+
+zo_status zo_get_precond(zo_ctx *ctx, int32_t n, double *g, double *c, double *w, float *a) {
+  ZO_CHECK(check_ctx(ctx));
+  if (n < 1 || n > ctx->last_n) return fail(ctx, ZO_ERR_INVALID, "n outside [1, last n_pert]");
+  ZO_CUDA(ctx, cudaStreamSynchronize(ctx->stream), "sync");
+  if (g) ZO_CUDA(ctx, cudaMemcpy(g, ctx->diag, n * sizeof(double), cudaMemcpyDeviceToHost), "g");
+  if (c) ZO_CUDA(ctx, cudaMemcpy(c, ctx->diag + ZO_MAX_PROBES, n * sizeof(double), cudaMemcpyDeviceToHost), "c");
+  if (w) ZO_CUDA(ctx, cudaMemcpy(w, ctx->diag + 2 * ZO_MAX_PROBES, n * sizeof(double), cudaMemcpyDeviceToHost), "w");
+  if (a) ZO_CUDA(ctx, cudaMemcpy(a, ctx->coef, n * sizeof(float), cudaMemcpyDeviceToHost), "a");
+  return ZO_OK;
+}
+
+zo_status zo_quad_step(zo_ctx *ctx, const float *D, int32_t n_pert, float eps, float lr,
+                       float damping, int preconditioned, double *losses_out) {
+  ZO_CHECK(check_ctx(ctx));
+  ZO_CHECK(check_step_args(ctx, n_pert, lr, eps, damping));
+  if (!losses_out) return fail(ctx, ZO_ERR_INVALID, "null losses_out");
+  if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "step while perturbed");
+  double *L0 = losses_out, *Lp = losses_out + 1, *Lm = losses_out + 1 + n_pert;
+  if (preconditioned) {
+    ZO_CHECK(zo_quad_loss(ctx, D, L0, 0));
+  } else {
+    ZO_CUDA(ctx, cudaMemsetAsync(L0, 0, sizeof(double), ctx->stream), "clear L0");
+  }
+  for (int32_t i = 0; i < n_pert; ++i) {
+    ZO_CHECK(zo_perturb(ctx, +1, eps, i));
+    zo_status st = zo_quad_loss(ctx, D, Lp + i, 0);
+    zo_restore(ctx);
+    ZO_CHECK(st);
+    ZO_CHECK(zo_perturb(ctx, -1, eps, i));
+    st = zo_quad_loss(ctx, D, Lm + i, 0);
+    zo_restore(ctx);
+    ZO_CHECK(st);
+  }
+  return zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
+}
+
+zo_status zo_quad_step_host(zo_ctx *ctx, const float *D_host, int32_t n_pert, float eps,
+                            float lr, float damping, int preconditioned, double *losses_host) {
+  ZO_CHECK(check_ctx(ctx));
+  ZO_CHECK(check_step_args(ctx, n_pert, lr, eps, damping));
+  if (!D_host || !losses_host) return fail(ctx, ZO_ERR_INVALID, "null host buffer");
+  if (!ctx->staging)
+    ZO_CUDA(ctx, cudaMalloc(&ctx->staging, (size_t)ctx->M * sizeof(float)), "staging buffer");
+  if (!ctx->loss_scratch)
+    ZO_CUDA(ctx, cudaMalloc(&ctx->loss_scratch, (2 * ZO_MAX_PROBES + 1) * sizeof(double)), "loss scratch");
+  ZO_CUDA(ctx, cudaMemcpyAsync(ctx->staging, D_host, (size_t)ctx->M * sizeof(float),
+                               cudaMemcpyHostToDevice, ctx->stream), "copy D");
+  ZO_CHECK(zo_quad_step(ctx, ctx->staging, n_pert, eps, lr, damping, preconditioned, ctx->loss_scratch));
+  ZO_CUDA(ctx, cudaMemcpyAsync(losses_host, ctx->loss_scratch, (2 * n_pert + 1) * sizeof(double),
+                               cudaMemcpyDeviceToHost, ctx->stream), "copy losses");
+  ZO_CUDA(ctx, cudaStreamSynchronize(ctx->stream), "sync");
+  return ZO_OK;
+}
+
+zo_status zo_mlp_step(zo_ctx *ctx, const float *X, const int32_t *labels, int batch, int n_in,
+                      int n_hidden, int n_out, int32_t n_pert, float eps, float lr,
+                      float damping, int preconditioned, double *losses_out) {
+  ZO_CHECK(check_ctx(ctx));
+  ZO_CHECK(check_step_args(ctx, n_pert, lr, eps, damping));
+  if (!losses_out) return fail(ctx, ZO_ERR_INVALID, "null losses_out");
+  if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "step while perturbed");
+  if (!ctx->live_enabled) ZO_CHECK(zo_set_live_buffer(ctx, 1));
+  const double scale = 1.0 / (double)batch;
+  double *L0 = losses_out, *Lp = losses_out + 1, *Lm = losses_out + 1 + n_pert;
+  if (preconditioned) {
+    ZO_CHECK(zo_mlp_loss(ctx, X, labels, batch, n_in, n_hidden, n_out, scale, L0, 0));
+  } else {
+    ZO_CUDA(ctx, cudaMemsetAsync(L0, 0, sizeof(double), ctx->stream), "clear L0");
+  }
+  for (int32_t i = 0; i < n_pert; ++i) {
+    for (int s = +1; s >= -1; s -= 2) {
+      ZO_CHECK(zo_perturb(ctx, s, eps, i));
+      const zo_status st = zo_mlp_loss(ctx, X, labels, batch, n_in, n_hidden, n_out, scale,
+                                       (s > 0 ? Lp : Lm) + i, 0);
+      zo_restore(ctx);
+      ZO_CHECK(st);
+    }
+  }
+  return zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
+}
+
+}  // extern "C"

@@ -1,0 +1,138 @@
+// zo_internal.cuh -- shared definitions of libzo.so (context, device state, probe bits).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "zo.h"
+
+namespace zo {
+
+constexpr int kSmCount = 148;           // B200 SMs (two dies x 74)
+constexpr int kGroup = 128;             // elements per Philox block (128 sign bits)
+constexpr int kTileGroups = 32;         // groups per warp tile in the streaming kernels
+constexpr int kTileElems = kGroup * kTileGroups;
+
+// Device-resident step state.  `step` keys the probes of the current step; the
+// preconditioner copies it to `upd_step` and sets `upd_ok` before advancing it, so the
+// update kernel of the same step reads a stable value.
+struct DevState {
+  uint32_t step;
+  uint32_t flags;     // sticky ZO_FLAG_* bits
+  uint32_t upd_step;  // step the pending update belongs to
+  uint32_t upd_ok;    // 1 if the pending update may be applied
+};
+
+// Everything a streaming kernel needs to regenerate probe bits.
+struct ProbeKey {
+  uint32_t k0, k1;          // Philox key (seed low / high word)
+  const uint32_t *step;     // device step counter
+  uint32_t probe;
+  int sign;                 // +1 / -1 ; 0 = clean (no perturbation)
+  float eps;
+};
+
+// ------------------------------------------------------------------ Philox4x32-10
+// Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as 1, 2, 3" (SC'11):
+// ten rounds of two 32x32->64 multiplies whose high halves are xor-ed with the other
+// counter words and the round key; the key advances by the Weyl constants per round.
+__device__ __forceinline__ uint4 philox10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t a = c.x, b = c.z;
+    const uint32_t hi_a = __umulhi(0xD2511F53u, a), lo_a = 0xD2511F53u * a;
+    const uint32_t hi_b = __umulhi(0xCD9E8D57u, b), lo_b = 0xCD9E8D57u * b;
+    c = make_uint4(hi_b ^ c.y ^ k0, lo_b, hi_a ^ c.w ^ k1, lo_a);
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return c;
+}
+
+// The 128 sign bits of group g (elements 128g .. 128g+127) of probe `probe` at `step`.
+__device__ __forceinline__ uint4 probe_block(uint64_t g, uint32_t probe, uint32_t step,
+                                             uint32_t k0, uint32_t k1) {
+  return philox10(make_uint4((uint32_t)g, (uint32_t)(g >> 32), probe, step), k0, k1);
+}
+
+__device__ __forceinline__ uint32_t word_of(const uint4 &v, int w) {
+  return w == 0 ? v.x : w == 1 ? v.y : w == 2 ? v.z : v.w;
+}
+
+// bf16 <-> fp32 on raw bits (round to nearest even, as __float2bfloat16_rn).
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) {
+  return __uint_as_float((uint32_t)h << 16);
+}
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+// P = rd(theta + s*eps*z) for one element given its sign bit (bit 1 -> z = -1).
+// `delta` is s*eps; the xor of the bit into the sign flips it exactly.
+__device__ __forceinline__ float perturb_f32(float theta, float delta, uint32_t bit) {
+  return __fadd_rn(theta, __uint_as_float(__float_as_uint(delta) ^ (bit << 31)));
+}
+
+}  // namespace zo
+
+// ------------------------------------------------------------------ context
+
+enum class PState { Clean, Perturbed };
+
+struct zo_ctx {
+  void *params = nullptr;
+  int64_t M = 0;
+  int dtype = ZO_F32;
+  uint64_t seed = 0;
+  cudaStream_t stream = nullptr;
+  int device = 0;
+  float alpha = 0.1f;
+
+  PState state = PState::Clean;
+  int sign = 0;
+  float eps = 0.f;
+  int32_t probe = 0;
+
+  bool live_enabled = false;
+  void *live = nullptr;        // M elements when enabled
+
+  zo::DevState *dstate = nullptr;
+  float *coef = nullptr;       // ZO_MAX_PROBES fp32 update coefficients
+  double *diag = nullptr;      // 3 * ZO_MAX_PROBES fp64 (g, c, w) of the last step
+  int32_t last_n = 0;
+  double *partials = nullptr;  // reduction scratch (kMaxPartials doubles)
+  unsigned int *counter = nullptr;  // last-block ticket for the reductions
+  float *staging = nullptr;    // device staging for host-buffer entry points
+  double *loss_scratch = nullptr;  // 2*ZO_MAX_PROBES+1 doubles for host-buffer steps
+
+  std::string err;
+};
+
+namespace zo {
+
+constexpr int kMaxPartials = 4096;
+
+zo_status fail(zo_ctx *ctx, zo_status st, const char *fmt, ...);
+zo_status check_launch(zo_ctx *ctx, const char *what);
+
+ProbeKey probe_key(const zo_ctx *ctx);  // current perturbation (sign 0 when clean)
+
+// Launchers (each enqueues on ctx->stream and returns the launch status).
+zo_status launch_perturb(zo_ctx *ctx, const ProbeKey &pk, int64_t first, int64_t count,
+                         void *out);
+zo_status launch_pack(zo_ctx *ctx, uint32_t probe, int64_t first_byte, int64_t nbytes,
+                      uint8_t *out);
+zo_status launch_quad_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *out,
+                           int accumulate, double *partials, unsigned int *counter);
+zo_status launch_mlp_loss(zo_ctx *ctx, const float *P, const float *X, const int32_t *y,
+                          int batch, int n_in, int n_hidden, int n_out, double scale,
+                          double *out, int accumulate);
+zo_status launch_precond(zo_ctx *ctx, const double *lp, const double *lm, const double *l0,
+                         int n, float lr, float eps, float damping);
+zo_status launch_update(zo_ctx *ctx, const float *coef, int n, const uint32_t *step_ptr,
+                        const uint32_t *ok_ptr);
+
+}  // namespace zo

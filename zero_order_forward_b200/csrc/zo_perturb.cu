@@ -1,0 +1,159 @@
+// zo_perturb.cu -- the fused unpack/apply kernel (perturbed copy of a parameter window)
+// and the packed-probe writer.
+//
+// "Probe-Space Preconditioning for Fast and Stable Zero-Order Training", abstract:
+// probes come from a packed random generator (8 signs per byte) and are applied to the
+// weights by fused unpack/apply kernels.  Here the sign bits are regenerated in
+// registers (never stored): each lane of a warp computes the Philox block of one
+// 128-element group, the warp shares the 32 blocks through shared memory, and every
+// lane then streams 16-byte vectors of theta -> rd(theta + s*eps*z).
+#include <cstdio>
+
+#include "zo_internal.cuh"
+
+namespace zo {
+namespace {
+
+constexpr int kWarps = 8;  // warps per block
+
+template <typename T> struct Vec;
+template <> struct Vec<float> { static constexpr int N = 4; };
+template <> struct Vec<uint16_t> { static constexpr int N = 8; };
+
+// Apply the perturbation to one 16-byte vector of N elements whose sign bits are the
+// low N bits of `bits`.
+__device__ __forceinline__ uint4 apply_vec(uint4 v, uint32_t bits, float delta, float *) {
+  float f[4] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
+                __uint_as_float(v.w)};
+#pragma unroll
+  for (int t = 0; t < 4; ++t) f[t] = perturb_f32(f[t], delta, (bits >> t) & 1u);
+  return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                    __float_as_uint(f[3]));
+}
+__device__ __forceinline__ uint4 apply_vec(uint4 v, uint32_t bits, float delta, uint16_t *) {
+  uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const float lo = perturb_f32(bf16_bits_to_f32((uint16_t)(w[t] & 0xFFFFu)), delta,
+                                 (bits >> (2 * t)) & 1u);
+    const float hi = perturb_f32(bf16_bits_to_f32((uint16_t)(w[t] >> 16)), delta,
+                                 (bits >> (2 * t + 1)) & 1u);
+    w[t] = (uint32_t)f32_to_bf16_bits(lo) | ((uint32_t)f32_to_bf16_bits(hi) << 16);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__device__ __forceinline__ float apply_one(float v, uint32_t bit, float delta) {
+  return perturb_f32(v, delta, bit);
+}
+__device__ __forceinline__ uint16_t apply_one(uint16_t v, uint32_t bit, float delta) {
+  return f32_to_bf16_bits(perturb_f32(bf16_bits_to_f32(v), delta, bit));
+}
+
+// out[e - first] = P_e for e in [first, first + count).  Tiles of 32 groups (4096
+// elements) are aligned to groups in the global element index, so every group's
+// block is computed once per tile by one lane.
+template <typename T>
+__global__ void __launch_bounds__(kWarps * 32)
+perturb_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t first, int64_t count,
+               ProbeKey pk, int64_t n_tiles) {
+  constexpr int N = Vec<T>::N;
+  constexpr int kIters = kTileElems / (32 * N);
+  __shared__ uint4 blocks[kWarps][kTileGroups];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t end = first + count;
+  const int64_t g0 = first / kGroup;
+  const uint32_t step = pk.sign ? *pk.step : 0u;
+  const float delta = pk.sign > 0 ? pk.eps : -pk.eps;
+  const uint32_t *bw = reinterpret_cast<const uint32_t *>(blocks[warp]);
+
+  for (int64_t tile = (int64_t)blockIdx.x * kWarps + warp; tile < n_tiles;
+       tile += (int64_t)gridDim.x * kWarps) {
+    const int64_t base = (g0 + tile * kTileGroups) * kGroup;  // first element of the tile
+    if (pk.sign) {
+      const int64_t g = g0 + tile * kTileGroups + lane;
+      if (g * kGroup < end) blocks[warp][lane] = probe_block(g, pk.probe, step, pk.k0, pk.k1);
+      __syncwarp();
+    }
+#pragma unroll 4
+    for (int k = 0; k < kIters; ++k) {
+      const int e_rel = (k * 32 + lane) * N;
+      const int64_t e = base + e_rel;
+      uint32_t bits = 0;
+      if (pk.sign) bits = bw[(e_rel >> 7) * 4 + ((e_rel >> 5) & 3)] >> (e_rel & 31);
+      T *o = out + (e - first);
+      if (e >= first && e + N <= end && ((reinterpret_cast<uintptr_t>(o) & 15) == 0)) {
+        uint4 v = __ldg(reinterpret_cast<const uint4 *>(theta + e));
+        if (pk.sign) v = apply_vec(v, bits, delta, (T *)nullptr);
+        *reinterpret_cast<uint4 *>(o) = v;
+      } else {
+#pragma unroll
+        for (int t = 0; t < N; ++t) {
+          const int64_t et = e + t;
+          if (et >= first && et < end) {
+            T v = theta[et];
+            if (pk.sign) v = apply_one(v, (bits >> t) & 1u, delta);
+            out[et - first] = v;
+          }
+        }
+      }
+    }
+    if (pk.sign) __syncwarp();
+  }
+}
+
+// Packed probe bytes [first_byte, first_byte + nbytes): one thread per 16-byte group
+// block.  Bits of elements >= M are cleared.
+__global__ void pack_kernel(uint8_t *__restrict__ out, int64_t first_byte, int64_t nbytes,
+                            int64_t M, uint32_t probe, const uint32_t *step_ptr, uint32_t k0,
+                            uint32_t k1) {
+  const int64_t gfirst = first_byte / 16;
+  const int64_t glast = (first_byte + nbytes - 1) / 16;
+  const int64_t g = gfirst + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (g > glast) return;
+  const uint4 b = probe_block((uint64_t)g, probe, *step_ptr, k0, k1);
+  const uint32_t words[4] = {b.x, b.y, b.z, b.w};
+  for (int q = 0; q < 16; ++q) {
+    const int64_t byte = g * 16 + q;
+    if (byte < first_byte || byte >= first_byte + nbytes) continue;
+    uint32_t v = (words[q >> 2] >> (8 * (q & 3))) & 0xFFu;
+    const int64_t e0 = byte * 8;
+    if (e0 + 8 > M) v &= (M > e0) ? ((1u << (M - e0)) - 1u) : 0u;
+    out[byte - first_byte] = (uint8_t)v;
+  }
+}
+
+}  // namespace
+
+zo_status launch_perturb(zo_ctx *ctx, const ProbeKey &pk, int64_t first, int64_t count,
+                         void *out) {
+  if (count <= 0) return ZO_OK;
+  const int64_t g0 = first / kGroup;
+  const int64_t g1 = (first + count + kGroup - 1) / kGroup;
+  const int64_t n_tiles = (g1 - g0 + kTileGroups - 1) / kTileGroups;
+  int64_t blocks = (n_tiles + kWarps - 1) / kWarps;
+  if (blocks > (int64_t)kSmCount * 8) blocks = (int64_t)kSmCount * 8;
+  if (ctx->dtype == ZO_F32)
+    perturb_kernel<float><<<(unsigned)blocks, kWarps * 32, 0, ctx->stream>>>(
+        static_cast<const float *>(ctx->params), static_cast<float *>(out), first, count, pk,
+        n_tiles);
+  else
+    perturb_kernel<uint16_t><<<(unsigned)blocks, kWarps * 32, 0, ctx->stream>>>(
+        static_cast<const uint16_t *>(ctx->params), static_cast<uint16_t *>(out), first,
+        count, pk, n_tiles);
+  return check_launch(ctx, "perturb_kernel");
+}
+
+zo_status launch_pack(zo_ctx *ctx, uint32_t probe, int64_t first_byte, int64_t nbytes,
+                      uint8_t *out) {
+  if (nbytes <= 0) return ZO_OK;
+  const int64_t groups = (first_byte + nbytes - 1) / 16 - first_byte / 16 + 1;
+  const int threads = 256;
+  const int64_t blocks = (groups + threads - 1) / threads;
+  ProbeKey pk = probe_key(ctx);
+  pack_kernel<<<(unsigned)blocks, threads, 0, ctx->stream>>>(
+      out, first_byte, nbytes, ctx->M, probe, &ctx->dstate->step, pk.k0, pk.k1);
+  return check_launch(ctx, "pack_kernel");
+}
+
+}  // namespace zo
