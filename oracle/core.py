@@ -25,16 +25,15 @@ def lib():
         L.zo_oracle_probe_sign.argtypes = [u64, u32, u32, i64]
         L.zo_oracle_probe_sign.restype = i32
         L.zo_oracle_pack_probe.argtypes = [u64, u32, u32, i64, vp]
-        L.zo_oracle_perturb_f32.argtypes = [vp, i64, u64, u32, u32, i32, f32, vp]
-        L.zo_oracle_perturb_bf16.argtypes = [vp, i64, u64, u32, u32, i32, f32, vp]
+        L.zo_oracle_perturb_f32.argtypes = [vp, i64, i64, u64, u32, u32, i32, f32, vp]
+        L.zo_oracle_perturb_bf16.argtypes = [vp, i64, i64, u64, u32, u32, i32, f32, vp]
         L.zo_oracle_quad_loss.argtypes = [vp, vp, i64]
         L.zo_oracle_quad_loss.restype = f64
         L.zo_oracle_precond.argtypes = [vp, vp, vp, i32, f64, f64, f64, f64, vp, vp, vp, vp]
         L.zo_oracle_precond.restype = i32
-        L.zo_oracle_update_f64_f32.argtypes = [vp, i64, vp, i32, u64, u32]
-        L.zo_oracle_update_f64_bf16.argtypes = [vp, i64, vp, i32, u64, u32]
-        L.zo_oracle_update_mirror_f32.argtypes = [vp, i64, vp, i32, u64, u32]
-        L.zo_oracle_update_mirror_bf16.argtypes = [vp, i64, vp, i32, u64, u32]
+        for nm in ("zo_oracle_update_f64_f32", "zo_oracle_update_f64_bf16",
+                   "zo_oracle_update_mirror_f32", "zo_oracle_update_mirror_bf16"):
+            getattr(L, nm).argtypes = [vp, i64, i64, vp, i32, u64, u32]
         L.zo_oracle_f32_to_bf16.argtypes = [f32]
         L.zo_oracle_f32_to_bf16.restype = ctypes.c_uint16
         _LIB = L
@@ -75,17 +74,18 @@ def probe_signs(seed, step, probe, M):
     return (1 - 2 * bits.astype(np.int8)).astype(np.int8)
 
 
-def perturb(theta, seed, step, probe, sign, eps):
-    """P = rd(theta + sign*eps*z_probe); theta is float32 or bf16 bits (uint16)."""
+def perturb(theta, seed, step, probe, sign, eps, j0=0):
+    """P = rd(theta + sign*eps*z_probe); theta is float32 or bf16 bits (uint16) and its
+    element k is global parameter j0 + k."""
     M = theta.size
     if theta.dtype == np.float32:
         t = _c(theta, np.float32)
         out = np.empty_like(t)
-        lib().zo_oracle_perturb_f32(_ptr(t), M, seed, step, probe, sign, eps, _ptr(out))
+        lib().zo_oracle_perturb_f32(_ptr(t), j0, M, seed, step, probe, sign, eps, _ptr(out))
     elif theta.dtype == np.uint16:
         t = _c(theta, np.uint16)
         out = np.empty_like(t)
-        lib().zo_oracle_perturb_bf16(_ptr(t), M, seed, step, probe, sign, eps, _ptr(out))
+        lib().zo_oracle_perturb_bf16(_ptr(t), j0, M, seed, step, probe, sign, eps, _ptr(out))
     else:
         raise TypeError("theta must be float32 or bf16 bits (uint16)")
     return out
@@ -112,27 +112,29 @@ def precond(loss_plus, loss_minus, loss0, eps, lr, damping, alpha=0.1):
     return {"g": g, "c": c, "w": w, "a": a}
 
 
-def update_f64(theta, a, seed, step):
-    """theta' = rd(theta - sum_i a_i z_i) with the probe sum in fp64 (new array)."""
+def update_f64(theta, a, seed, step, j0=0):
+    """theta' = rd(theta - sum_i a_i z_i) with the probe sum in fp64 (new array); element
+    k of theta is global parameter j0 + k."""
     a = _c(a, np.float64)
     t = np.array(theta, copy=True)
     if t.dtype == np.float32:
-        lib().zo_oracle_update_f64_f32(_ptr(t), t.size, _ptr(a), a.size, seed, step)
+        lib().zo_oracle_update_f64_f32(_ptr(t), j0, t.size, _ptr(a), a.size, seed, step)
     elif t.dtype == np.uint16:
-        lib().zo_oracle_update_f64_bf16(_ptr(t), t.size, _ptr(a), a.size, seed, step)
+        lib().zo_oracle_update_f64_bf16(_ptr(t), j0, t.size, _ptr(a), a.size, seed, step)
     else:
         raise TypeError("theta must be float32 or bf16 bits (uint16)")
     return t
 
 
-def update_mirror(theta, a32, seed, step):
-    """theta' in the fixed fp32 order (groups of 8 probes) from fp32 coefficients."""
+def update_mirror(theta, a32, seed, step, j0=0):
+    """theta' in the fixed fp32 order (groups of 8 probes) from fp32 coefficients;
+    element k of theta is global parameter j0 + k."""
     a32 = _c(a32, np.float32)
     t = np.array(theta, copy=True)
     if t.dtype == np.float32:
-        lib().zo_oracle_update_mirror_f32(_ptr(t), t.size, _ptr(a32), a32.size, seed, step)
+        lib().zo_oracle_update_mirror_f32(_ptr(t), j0, t.size, _ptr(a32), a32.size, seed, step)
     elif t.dtype == np.uint16:
-        lib().zo_oracle_update_mirror_bf16(_ptr(t), t.size, _ptr(a32), a32.size, seed, step)
+        lib().zo_oracle_update_mirror_bf16(_ptr(t), j0, t.size, _ptr(a32), a32.size, seed, step)
     else:
         raise TypeError("theta must be float32 or bf16 bits (uint16)")
     return t

@@ -123,21 +123,22 @@ float zo_oracle_bf16_to_f32(uint16_t h) { return bf16_to_f32(h); }
 
 /* ------------------------------------------------------------------ perturbation */
 
-/* P_j = rd32(theta_j + s*eps*z_j), out of place; theta is not written [HOW]. */
-void zo_oracle_perturb_f32(const float *theta, int64_t M, uint64_t seed, uint32_t step,
-                           uint32_t probe, int sign, float eps, float *out) {
-  for (int64_t j = 0; j < M; ++j) {
-    float delta = (float)(sign * zo_oracle_probe_sign(seed, step, probe, j)) * eps;
-    out[j] = theta[j] + delta;
+/* P_j = rd32(theta_j + s*eps*z_j), out of place; theta is not written [HOW].
+ * Array element k holds global parameter j = j0 + k (the probe bits depend on j). */
+void zo_oracle_perturb_f32(const float *theta, int64_t j0, int64_t count, uint64_t seed,
+                           uint32_t step, uint32_t probe, int sign, float eps, float *out) {
+  for (int64_t k = 0; k < count; ++k) {
+    float delta = (float)(sign * zo_oracle_probe_sign(seed, step, probe, j0 + k)) * eps;
+    out[k] = theta[k] + delta;
   }
 }
 
-void zo_oracle_perturb_bf16(const uint16_t *theta, int64_t M, uint64_t seed, uint32_t step,
-                            uint32_t probe, int sign, float eps, uint16_t *out) {
-  for (int64_t j = 0; j < M; ++j) {
-    float delta = (float)(sign * zo_oracle_probe_sign(seed, step, probe, j)) * eps;
-    float sum = bf16_to_f32(theta[j]) + delta;
-    out[j] = f32_to_bf16_rne(sum);
+void zo_oracle_perturb_bf16(const uint16_t *theta, int64_t j0, int64_t count, uint64_t seed,
+                            uint32_t step, uint32_t probe, int sign, float eps, uint16_t *out) {
+  for (int64_t k = 0; k < count; ++k) {
+    float delta = (float)(sign * zo_oracle_probe_sign(seed, step, probe, j0 + k)) * eps;
+    float sum = bf16_to_f32(theta[k]) + delta;
+    out[k] = f32_to_bf16_rne(sum);
   }
 }
 
@@ -187,25 +188,28 @@ int zo_oracle_precond(const double *loss_plus, const double *loss_minus,
 
 /* ------------------------------------------------------------------ update */
 
-/* theta' = rd32(theta - sum_i a_i z_i), the sum over probes taken in fp64. */
-void zo_oracle_update_f64_f32(float *theta, int64_t M, const double *a, int n,
+/* theta' = rd32(theta - sum_i a_i z_i), the sum over probes taken in fp64.
+ * Array element k holds global parameter j0 + k. */
+void zo_oracle_update_f64_f32(float *theta, int64_t j0, int64_t count, const double *a, int n,
                               uint64_t seed, uint32_t step) {
-  for (int64_t j = 0; j < M; ++j) {
+  for (int64_t k = 0; k < count; ++k) {
     double acc = 0.0;
-    for (int i = 0; i < n; ++i) acc += a[i] * (double)zo_oracle_probe_sign(seed, step, (uint32_t)i, j);
-    theta[j] = (float)((double)theta[j] - acc);
+    for (int i = 0; i < n; ++i)
+      acc += a[i] * (double)zo_oracle_probe_sign(seed, step, (uint32_t)i, j0 + k);
+    theta[k] = (float)((double)theta[k] - acc);
   }
 }
 
-void zo_oracle_update_f64_bf16(uint16_t *theta, int64_t M, const double *a, int n,
-                               uint64_t seed, uint32_t step) {
-  for (int64_t j = 0; j < M; ++j) {
+/* bf16: the fp64 value is rounded to fp32 and then to bf16 (two roundings; the tests
+ * allow one bf16 ulp against a single rounding). */
+void zo_oracle_update_f64_bf16(uint16_t *theta, int64_t j0, int64_t count, const double *a,
+                               int n, uint64_t seed, uint32_t step) {
+  for (int64_t k = 0; k < count; ++k) {
     double acc = 0.0;
-    for (int i = 0; i < n; ++i) acc += a[i] * (double)zo_oracle_probe_sign(seed, step, (uint32_t)i, j);
-    double v = (double)bf16_to_f32(theta[j]) - acc;
-    /* one rounding from the fp64 value: via fp32 is exact enough except at ties of
-       the two roundings; the tests allow one bf16 ulp for that reason. */
-    theta[j] = f32_to_bf16_rne((float)v);
+    for (int i = 0; i < n; ++i)
+      acc += a[i] * (double)zo_oracle_probe_sign(seed, step, (uint32_t)i, j0 + k);
+    double v = (double)bf16_to_f32(theta[k]) - acc;
+    theta[k] = f32_to_bf16_rne((float)v);
   }
 }
 
@@ -222,13 +226,14 @@ static float mirror_sum(const float *a32, int n, uint64_t seed, uint32_t step, i
   return acc;
 }
 
-void zo_oracle_update_mirror_f32(float *theta, int64_t M, const float *a32, int n,
-                                 uint64_t seed, uint32_t step) {
-  for (int64_t j = 0; j < M; ++j) theta[j] = theta[j] - mirror_sum(a32, n, seed, step, j);
+void zo_oracle_update_mirror_f32(float *theta, int64_t j0, int64_t count, const float *a32,
+                                 int n, uint64_t seed, uint32_t step) {
+  for (int64_t k = 0; k < count; ++k)
+    theta[k] = theta[k] - mirror_sum(a32, n, seed, step, j0 + k);
 }
 
-void zo_oracle_update_mirror_bf16(uint16_t *theta, int64_t M, const float *a32, int n,
-                                  uint64_t seed, uint32_t step) {
-  for (int64_t j = 0; j < M; ++j)
-    theta[j] = f32_to_bf16_rne(bf16_to_f32(theta[j]) - mirror_sum(a32, n, seed, step, j));
+void zo_oracle_update_mirror_bf16(uint16_t *theta, int64_t j0, int64_t count, const float *a32,
+                                  int n, uint64_t seed, uint32_t step) {
+  for (int64_t k = 0; k < count; ++k)
+    theta[k] = f32_to_bf16_rne(bf16_to_f32(theta[k]) - mirror_sum(a32, n, seed, step, j0 + k));
 }
