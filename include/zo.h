@@ -186,6 +186,35 @@ zo_status zo_mlp_loss(zo_ctx *ctx, const float *X, const int32_t *labels, int ba
                       int n_in, int n_hidden, int n_out, double scale, double *loss_out,
                       int accumulate);
 
+/* Largest batch accepted by zo_mlp_loss_noalloc: its static scratch holds one fp64
+ * partial per sample (32 KB) plus the reduction's ticket counter. */
+#define ZO_NOALLOC_MAX_BATCH 4096
+
+/* zo_mlp_loss without a context and without any device allocation.  The pages have no
+ * counterpart: this entry point exists for callers that must not call cudaMalloc, e.g.
+ * code running inside a host framework that owns every device allocation through its own
+ * pool, or code that enqueues work while a stream is being captured, where a new
+ * allocation would break the capture or its memory budget.  Such callers pass inputs and
+ * outputs only; the reduction scratch is a static device array of libzo.so, which every GPU
+ * that loads the library holds (about 32 KB) until the process exits.
+ *   P          device, M = n_hidden*n_in + n_hidden + n_out*n_hidden + n_out floats,
+ *              flat order W1[hidden][in], b1[hidden], W2[out][hidden], b2[out] (the
+ *              parameters to evaluate: theta, or a perturbed copy the caller made).
+ *   X, labels, batch, n_in, n_hidden, n_out, scale, loss_out, accumulate: as zo_mlp_loss.
+ *   stream     cudaStream_t to enqueue on (NULL = legacy default stream).
+ * The first call on a device looks up the scratch array's device address (once per
+ * device, with that device current); make that first call before any stream capture.
+ * Every call clears the scratch's counter before its kernel.  All calls in the process
+ * share the one scratch array, which keeps the last call's contents: calls that overlap
+ * on the GPU (other streams, other threads) race and must be serialised by the caller.
+ * Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ * Errors (returned; there is no context to hold a message): ZO_ERR_INVALID for null
+ * pointers, sizes outside the zo_mlp_loss limits, or batch > ZO_NOALLOC_MAX_BATCH;
+ * ZO_ERR_CUDA if the scratch lookup, the counter reset or the launch fails. */
+zo_status zo_mlp_loss_noalloc(const float *P, const float *X, const int32_t *labels,
+                              int batch, int n_in, int n_hidden, int n_out, double scale,
+                              double *loss_out, int accumulate, void *stream);
+
 /* ------------------------------------------------------------------ zo_precond + zo_update */
 
 /* One optimizer step from the losses of the current step [HOW][PSP]:

@@ -22,6 +22,7 @@ ZO_F32, ZO_BF16 = 0, 1
 ZO_OK, ZO_ERR_INVALID, ZO_ERR_STATE, ZO_ERR_CUDA, ZO_ERR_OOM, ZO_ERR_NONFINITE, ZO_ERR_UNSUPPORTED = range(7)
 ZO_FLAG_NONFINITE = 0x1
 ZO_MAX_PROBES = 1024
+ZO_NOALLOC_MAX_BATCH = 4096
 
 _vp, _i32, _i64, _u32, _u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_uint64
 _f32, _f64, _int = ctypes.c_float, ctypes.c_double, ctypes.c_int
@@ -46,6 +47,7 @@ _SIGS = {
     "zo_quad_step": [_vp, _vp, _i32, _f32, _f32, _f32, _int, _vp],
     "zo_quad_step_host": [_vp, _vp, _i32, _f32, _f32, _f32, _int, _vp],
     "zo_mlp_step": [_vp, _vp, _vp, _int, _int, _int, _int, _i32, _f32, _f32, _f32, _int, _vp],
+    "zo_mlp_loss_noalloc": [_vp, _vp, _vp, _int, _int, _int, _int, _f64, _vp, _int, _vp],
 }
 for _name, _args in _SIGS.items():
     _fn = getattr(_L, _name)
@@ -227,3 +229,14 @@ def zo_mlp_step(ctx, X, labels, batch, n_in, n_hidden, n_out, n_pert, eps, lr, d
     return ctx.check(_L.zo_mlp_step(ctx.handle, _ptr(X), _ptr(labels), batch, n_in, n_hidden,
                                     n_out, n_pert, eps, lr, damping, int(preconditioned),
                                     _ptr(losses_out)))
+
+
+def zo_mlp_loss_noalloc(P, X, labels, batch, n_in, n_hidden, n_out, scale, loss_out,
+                        accumulate=False, stream=None):
+    """MLP loss for callers that cannot allocate device memory (see include/zo.h): no
+    context, scratch in the library's static device memory.  Raises ZoError on failure."""
+    st = _L.zo_mlp_loss_noalloc(_ptr(P), _ptr(X), _ptr(labels), batch, n_in, n_hidden, n_out,
+                                scale, _ptr(loss_out), int(accumulate), _stream(stream))
+    if st != ZO_OK:
+        raise ZoError(st, "zo_mlp_loss_noalloc failed")
+    return st

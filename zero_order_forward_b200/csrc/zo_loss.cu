@@ -6,6 +6,8 @@
 //
 // Reductions are deterministic: each block writes one fp64 partial, and the last block
 // to finish (ticket on a counter) adds the partials in index order with a fixed tree.
+#include <mutex>
+
 #include "zo_internal.cuh"
 
 namespace zo {
@@ -182,3 +184,68 @@ zo_status launch_mlp_loss(zo_ctx *ctx, const float *P, const float *X, const int
 }
 
 }  // namespace zo
+
+// ------------------------------------------------------------------ allocation-free MLP loss
+// For callers that cannot allocate device memory: the same mlp_loss_kernel, with its
+// per-sample partials and ticket counter in a static device array of this module instead
+// of a context's cudaMalloc'd scratch.
+
+namespace zo {
+namespace {
+
+constexpr size_t kNoallocPartialsBytes = (size_t)ZO_NOALLOC_MAX_BATCH * sizeof(double);
+constexpr int kNoallocMaxDevices = 64;
+
+// [0, kNoallocPartialsBytes): fp64 partials; then the unsigned ticket counter.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocPartialsBytes + 256];
+
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[kNoallocMaxDevices] = {};
+
+// Device address of the scratch on the current device.  In host code the array's name is
+// only a host-side stand-in, so the address is looked up once per device.
+cudaError_t noalloc_scratch(void **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kNoallocMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace zo
+
+extern "C" zo_status zo_mlp_loss_noalloc(const float *P, const float *X, const int32_t *labels,
+                                         int batch, int n_in, int n_hidden, int n_out,
+                                         double scale, double *loss_out, int accumulate,
+                                         void *stream) {
+  using namespace zo;
+  if (!P || !X || !labels || !loss_out || batch < 1 || n_in < 1 || n_hidden < 1 || n_out < 1 ||
+      n_in > kMlpMax || n_hidden > kMlpMax || n_out > kMlpMax || batch > ZO_NOALLOC_MAX_BATCH)
+    return ZO_ERR_INVALID;
+  void *base = nullptr;
+  if (noalloc_scratch(&base) != cudaSuccess) {
+    cudaGetLastError();
+    return ZO_ERR_CUDA;
+  }
+  double *partials = static_cast<double *>(base);
+  unsigned int *counter =
+      reinterpret_cast<unsigned int *>(static_cast<unsigned char *>(base) + kNoallocPartialsBytes);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(counter, 0, sizeof(unsigned int), s) != cudaSuccess) {
+    cudaGetLastError();
+    return ZO_ERR_CUDA;
+  }
+  mlp_loss_kernel<<<batch, 256, 0, s>>>(P, X, labels, n_in, n_hidden, n_out, partials, counter,
+                                        loss_out, accumulate, scale);
+  if (cudaGetLastError() != cudaSuccess) return ZO_ERR_CUDA;
+  return ZO_OK;
+}
