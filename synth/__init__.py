@@ -90,3 +90,61 @@ def coefficients(n, seed=0, scale=1e-3):
     """Synthetic fp32 update coefficients a[n] (mixed signs and magnitudes)."""
     r = rng(seed, "coef", n)
     return (r.standard_normal(n) * scale * 10.0 ** r.uniform(-2, 0, n)).astype(np.float32)
+
+
+# ---------------------------------------------------------------- OPT-shaped decoders
+
+OPT_CONFIGS = {
+    # the pages' model family at three sizes; vocabulary and position table of OPT
+    "opt-125m": dict(n_layers=12, d_model=768, n_heads=12, d_ffn=3072, vocab=50272,
+                     max_pos=2048, class_ids=(1000, 2000)),
+    "opt-1.3b": dict(n_layers=24, d_model=2048, n_heads=32, d_ffn=8192, vocab=50272,
+                     max_pos=2048, class_ids=(1000, 2000)),
+    "opt-30b": dict(n_layers=48, d_model=7168, n_heads=56, d_ffn=28672, vocab=50272,
+                    max_pos=2048, class_ids=(1000, 2000)),
+}
+
+
+def opt_segments(cfg):
+    """(kind, count) runs of the flat parameter vector in order; kind is one of
+    'matrix' (embeddings and projection weights), 'bias', 'gain', 'shift'."""
+    d, f, V, P = cfg["d_model"], cfg["d_ffn"], cfg["vocab"], cfg["max_pos"] + 2
+    segs = [("matrix", V * d), ("matrix", P * d)]
+    for _ in range(cfg["n_layers"]):
+        segs += [("gain", d), ("shift", d), ("matrix", 3 * d * d), ("bias", 3 * d),
+                 ("matrix", d * d), ("bias", d), ("gain", d), ("shift", d),
+                 ("matrix", f * d), ("bias", f), ("matrix", d * f), ("bias", d)]
+    segs += [("gain", d), ("shift", d)]
+    return segs
+
+
+def opt_params(cfg, seed=0, varied=False):
+    """bf16 bits (uint16) of the flat parameters.  OPT-style init (varied=False): matrices
+    N(0, 0.02), biases 0, LayerNorm gains 1 and shifts 0.  varied=True (parity tests)
+    also draws biases N(0, 0.02), gains 1 + N(0, 0.1) and shifts N(0, 0.02) so that every
+    parameter kind influences the loss."""
+    segs = opt_segments(cfg)
+    total = sum(n for _, n in segs)
+    r = rng(seed, "opt", total)
+    out = np.empty(total, np.uint16)
+    o = 0
+    for kind, n in segs:
+        if kind == "matrix":
+            x = r.standard_normal(n, dtype=np.float32) * np.float32(0.02)
+        elif kind == "bias" or kind == "shift":
+            x = (r.standard_normal(n, dtype=np.float32) * np.float32(0.02) if varied
+                 else np.zeros(n, np.float32))
+        else:  # gain
+            x = (1.0 + r.standard_normal(n, dtype=np.float32) * np.float32(0.1) if varied
+                 else np.ones(n, np.float32))
+        out[o:o + n] = to_bf16_bits(x)
+        o += n
+    return out
+
+
+def opt_batch(cfg, batch, seq, seed=0, step=0):
+    """(tokens int32 [batch][seq] uniform over the vocabulary, labels int32 [batch] in {0,1})."""
+    tokens = rng(seed, "tokens", step, batch, seq).integers(0, cfg["vocab"], (batch, seq),
+                                                            dtype=np.int32)
+    labels = rng(seed, "labels", step, batch).integers(0, 2, batch, dtype=np.int32)
+    return tokens, labels
