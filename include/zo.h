@@ -69,11 +69,14 @@ typedef enum {
   ZO_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
   ZO_ERR_OOM = 4,         /* device allocation failed */
   ZO_ERR_NONFINITE = 5,   /* a loss was NaN/Inf: the step was skipped (theta unchanged) */
-  ZO_ERR_UNSUPPORTED = 6  /* valid request this build does not support */
+  ZO_ERR_UNSUPPORTED = 6, /* valid request this build does not support */
+  ZO_ERR_TIMEOUT = 7      /* a kernel gave up a bounded wait (see ZO_FLAG_TIMEOUT) */
 } zo_status;
 
-/* Device-side status flags reported by zo_sync / zo_device_flags. */
-#define ZO_FLAG_NONFINITE 0x1u
+/* Device-side status flags reported by zo_sync. */
+#define ZO_FLAG_NONFINITE 0x1u /* a loss was not finite; that step was skipped */
+#define ZO_FLAG_TIMEOUT 0x2u   /* a tensor-core kernel's pipeline wait expired (about 2 s);
+                                  its output is invalid */
 
 /* Largest n_pert accepted by zo_step / zo_update (the update keeps a 1 KB table per
  * group of 8 probes in shared memory: 128 KB at this limit). */
@@ -120,7 +123,8 @@ const void *zo_live_params(const zo_ctx *ctx);
 
 /* Synchronise the context's stream and return the sticky device flags (ZO_FLAG_*)
  * raised since the last call, clearing them; *flags may be NULL.  Returns
- * ZO_ERR_NONFINITE if ZO_FLAG_NONFINITE was raised, else ZO_OK. */
+ * ZO_ERR_TIMEOUT if ZO_FLAG_TIMEOUT was raised, else ZO_ERR_NONFINITE if
+ * ZO_FLAG_NONFINITE was raised, else ZO_OK. */
 zo_status zo_sync(zo_ctx *ctx, uint32_t *flags);
 
 /* Read (synchronising) or set (enqueued) the device-resident step counter, which keys
@@ -266,6 +270,98 @@ zo_status zo_quad_step_host(zo_ctx *ctx, const float *D_host, int32_t n_pert, fl
 zo_status zo_mlp_step(zo_ctx *ctx, const float *X, const int32_t *labels, int batch,
                       int n_in, int n_hidden, int n_out, int32_t n_pert, float eps,
                       float lr, float damping, int preconditioned, double *losses_out);
+
+/* ------------------------------------------------------------------ decoder (zo_forward) */
+
+/* Loss-only forward of an OPT-shaped decoder: pre-LN, learned positions (table of max_pos+2
+ * rows, position s uses row s+2), ReLU FFN, biases on every projection, LayerNorm eps
+ * 1e-5, final LayerNorm, head tied to the token embedding.  The loss is the 2-class
+ * cross-entropy of the last position's logits restricted to class_ids[0..1] (label 0 or
+ * 1 per sequence): the prompt-classification shape of the pages' fine-tuning benchmarks
+ * ("Probe-Space Preconditioning for Fast and Stable Zero-Order Training", abstract:
+ * OPT and Qwen3 post-training in inference mode).
+ * Flat parameter order, all bf16 (d = d_model, f = d_ffn, V = vocab, P = max_pos + 2):
+ *   E[V][d], Pos[P][d], then per layer: ln1.g[d], ln1.b[d], Wqkv[3d][d] (rows q, k, v),
+ *   bqkv[3d], Wo[d][d], bo[d], ln2.g[d], ln2.b[d], W1[f][d], b1[f], W2[d][f], b2[d];
+ *   then lnf.g[d], lnf.b[d].  Linear weights are [out][in] (row-major, in contiguous). */
+typedef struct {
+  int32_t n_layers;
+  int32_t d_model;      /* multiple of 64 */
+  int32_t n_heads;      /* d_model / n_heads must be 64 or 128 */
+  int32_t d_ffn;        /* multiple of 8 */
+  int32_t vocab;
+  int32_t max_pos;      /* longest sequence */
+  int32_t class_ids[2]; /* token ids whose last-position logits are the two classes */
+} zo_model_cfg;
+
+typedef struct zo_model zo_model;
+
+/* Number of parameters M of the layout above.  Errors: ZO_ERR_INVALID (bad config). */
+zo_status zo_model_param_count(const zo_model_cfg *cfg, int64_t *M_out);
+
+/* Bind a decoder to a bf16 context whose params hold the flat layout (ctx M must equal
+ * zo_model_param_count).  Allocates, owned by the model: the layer window (one layer's
+ * perturbed parameters) and activations for up to max_tokens = batch*seq tokens (fp32
+ * residual stream [T][d], bf16 [T][d] x2, [T][3d], [T][f]).  The context must outlive
+ * the model.  Errors: ZO_ERR_INVALID, ZO_ERR_OOM. */
+zo_status zo_model_create(zo_model **out, zo_ctx *ctx, const zo_model_cfg *cfg,
+                          int64_t max_tokens);
+zo_status zo_model_destroy(zo_model *m);
+
+/* Loss of one micro-batch at the context's current state (clean or perturbed):
+ *   tokens  device int32 [batch][seq], ids in [0, vocab) (an id outside that range makes
+ *           the loss NaN, so the step is skipped);  labels device int32 [batch] in {0, 1}.
+ *   loss_out device double: = scale * sum of per-sequence losses (accumulate == 0) or +=.
+ * With a perturbed context each layer's parameters are first materialised into the
+ * layer window by the unpack/apply kernel (theta is not written); embeddings, the final
+ * LayerNorm and the head rows are perturbed on load.
+ * Errors: ZO_ERR_INVALID (seq > max_pos, batch*seq > max_tokens, batch > 4096, nulls),
+ *         ZO_ERR_CUDA. */
+zo_status zo_model_loss(zo_model *m, const int32_t *tokens, const int32_t *labels,
+                        int32_t batch, int32_t seq, double scale, double *loss_out,
+                        int accumulate);
+
+/* Embedding plus the first n_layers_run layers of one micro-batch at the current state;
+ * copies the fp32 residual stream [batch*seq][d_model] into h_out (device).  For
+ * layer-by-layer parity checks. */
+zo_status zo_model_hidden(zo_model *m, const int32_t *tokens, int32_t batch, int32_t seq,
+                          int32_t n_layers_run, float *h_out);
+
+/* One full step [LOOP][BUD]: the effective batch is n_micro micro-batches of
+ * batch x seq (tokens device [n_micro][batch][seq], labels device [n_micro][batch]);
+ * each loss is the mean over the effective batch, accumulated micro-batch by micro-batch.
+ * Order: clean loss (1.5-SPSA), then for each probe the +eps and -eps losses, then
+ * zo_step.  losses_out: device, 2*n_pert+1 doubles [L0, L+..., L-...]. */
+zo_status zo_model_step(zo_model *m, const int32_t *tokens, const int32_t *labels,
+                        int32_t batch, int32_t seq, int32_t n_micro, int32_t n_pert,
+                        float eps, float lr, float damping, int preconditioned,
+                        double *losses_out);
+
+/* ------------------------------------------------------------------ decoder components */
+
+/* Epilogues of zo_gemm_bf16. */
+#define ZO_EPI_BIAS_BF16 0  /* out bf16 = A.B^T + bias */
+#define ZO_EPI_RELU_BF16 1  /* out bf16 = max(A.B^T + bias, 0) */
+#define ZO_EPI_RESID_F32 2  /* out fp32 += A.B^T + bias (residual add) */
+
+/* out[M][ldo] = epilogue(A[M][K] . B[N][K]^T + bias[N]) on the tcgen05 tensor cores:
+ * bf16 operands (device, row-major, K contiguous), fp32 accumulation in TMEM, bias bf16
+ * (device, may be NULL).  K % 8 == 0, ldo % 8 == 0, ldo >= N, all pointers 16-byte
+ * aligned; ragged M, N, K are handled (zero fill).  Enqueued on ctx's stream; a
+ * pipeline stall beyond the bounded wait raises ZO_FLAG_TIMEOUT (seen by zo_sync). */
+zo_status zo_gemm_bf16(zo_ctx *ctx, const void *A, const void *B, const void *bias, void *out,
+                       int32_t M, int32_t N, int32_t K, int32_t ldo, int32_t epilogue);
+
+/* Causal multi-head attention: qkv device bf16 [batch*seq][3*d_model] (q, k, v at column
+ * offsets 0, d, 2d; head h at +h*hd), out device bf16 [batch*seq][d_model];
+ * softmax(q.k^T / sqrt(hd)) over keys <= query, hd = d_model/n_heads in {64, 128}. */
+zo_status zo_attention(zo_ctx *ctx, const void *qkv, void *out, int32_t batch, int32_t seq,
+                       int32_t n_heads, int32_t d_model);
+
+/* out bf16 [rows][d] = LayerNorm(x fp32 [rows][d]) * gamma + beta (bf16 [d]), eps 1e-5,
+ * d <= 8192. */
+zo_status zo_layernorm(zo_ctx *ctx, const float *x, const void *gamma, const void *beta,
+                       void *out, int32_t rows, int32_t d);
 
 #ifdef __cplusplus
 }

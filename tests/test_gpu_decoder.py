@@ -1,0 +1,239 @@
+"""Parity of the decoder forward (tcgen05 GEMM, attention, LayerNorm, embedding, head) with
+the CPU oracle and with plain numpy references of each component.
+
+Tolerances:
+  - GEMM, bf16 output: |gpu - ref| <= 2^-8 |ref| + 2^-8 * rms(ref) (one bf16 rounding of
+    an fp32-accumulated dot product); fp32 residual output: 1e-5 of sum |a_k b_k|;
+  - attention (bf16 probabilities and output): 2e-2 absolute on unit-scale inputs;
+  - LayerNorm (bf16 output): 2^-8 relative + 1e-3 absolute;
+  - decoder hidden states: relative Frobenius error <= 1e-2 per layer;
+  - decoder loss (bf16 forward): 2e-2 relative.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from oracle import core
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+
+def bf16(x):
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).cuda()
+
+
+def f64(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+@pytest.fixture(scope="module")
+def ctx(zo):
+    th = torch.zeros(1024, dtype=torch.bfloat16, device="cuda")
+    c = zo.zo_create(th, seed=0)
+    yield c
+    c.close()
+
+
+GEMM_SHAPES = [(128, 128, 64), (256, 384, 256), (300, 200, 72), (129, 136, 8),
+               (2048, 2560, 512), (4096, 768, 768)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+@pytest.mark.parametrize("epi", [0, 1, 2])
+def test_gemm_matches_numpy(zo, ctx, M, N, K, epi):
+    r = np.random.default_rng(M * 7 + N * 3 + K + epi)
+    A = bf16(r.standard_normal((M, K)))
+    B = bf16(r.standard_normal((N, K)) * 0.05)
+    bias = bf16(r.standard_normal(N))
+    ref = f64(A) @ f64(B).T + f64(bias)
+    if epi == 2:
+        h0 = torch.from_numpy(r.standard_normal((M, N)).astype(np.float32)).cuda()
+        out = h0.clone()
+    else:
+        out = torch.zeros((M, N), dtype=torch.bfloat16, device="cuda")
+    zo.zo_gemm_bf16(ctx, A, B, bias, out, M, N, K, N, epi)
+    torch.cuda.synchronize()
+    assert zo.zo_sync(ctx) == 0
+    if epi == 2:
+        scale = np.abs(f64(A)) @ np.abs(f64(B)).T + np.abs(f64(bias))
+        got = out.cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(got - (h0.cpu().numpy() + ref)) <= 1e-5 * (scale + 1) + 1e-6)
+    else:
+        if epi == 1:
+            ref = np.maximum(ref, 0.0)
+        got = f64(out)
+        rms = np.sqrt(np.mean(ref ** 2)) + 1e-30
+        assert np.all(np.abs(got - ref) <= 2.0 ** -8 * (np.abs(ref) + rms))
+
+
+def _np_attention(qkv, B, S, H, d):
+    hd = d // H
+    x = qkv.reshape(B, S, 3, H, hd)
+    q, k, v = (x[:, :, i].transpose(0, 2, 1, 3) for i in range(3))
+    s = q @ k.transpose(0, 1, 3, 2) / np.sqrt(hd)
+    s = np.where(np.triu(np.ones((S, S), bool), 1), -np.inf, s)
+    w = np.exp(s - s.max(-1, keepdims=True))
+    w /= w.sum(-1, keepdims=True)
+    return (w @ v).transpose(0, 2, 1, 3).reshape(B * S, d)
+
+
+@pytest.mark.parametrize("B,S,H,d", [(2, 64, 2, 128), (2, 200, 2, 256), (1, 256, 4, 256),
+                                     (3, 130, 3, 192), (1, 512, 1, 128)])
+def test_attention_matches_numpy(zo, ctx, B, S, H, d):
+    r = np.random.default_rng(S + d)
+    qkv = bf16(r.standard_normal((B * S, 3 * d)))
+    out = torch.zeros((B * S, d), dtype=torch.bfloat16, device="cuda")
+    zo.zo_attention(ctx, qkv, out, B, S, H, d)
+    torch.cuda.synchronize()
+    ref = _np_attention(f64(qkv), B, S, H, d)
+    assert np.max(np.abs(f64(out) - ref)) <= 2e-2
+
+
+def test_layernorm_matches_numpy(zo, ctx):
+    r = np.random.default_rng(0)
+    rows, d = 37, 7168
+    x = torch.from_numpy((r.standard_normal((rows, d)) * 3 + 1).astype(np.float32)).cuda()
+    g = bf16(1 + 0.1 * r.standard_normal(d))
+    b = bf16(0.1 * r.standard_normal(d))
+    out = torch.zeros((rows, d), dtype=torch.bfloat16, device="cuda")
+    zo.zo_layernorm(ctx, x, g, b, out, rows, d)
+    torch.cuda.synchronize()
+    xx = x.cpu().numpy().astype(np.float64)
+    ref = (xx - xx.mean(1, keepdims=True)) / np.sqrt(xx.var(1, keepdims=True) + 1e-5) * f64(g) + f64(b)
+    assert np.all(np.abs(f64(out) - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-3)
+
+
+TINY = [
+    dict(n_layers=2, d_model=128, n_heads=2, d_ffn=512, vocab=1000, max_pos=128, class_ids=(3, 7)),
+    dict(n_layers=2, d_model=256, n_heads=2, d_ffn=320, vocab=777, max_pos=160, class_ids=(0, 776)),
+]
+
+
+def _setup(zo, cfg, B, S, seed=0, max_tokens=None):
+    bits = synth.opt_params(cfg, seed=seed, varied=True)
+    theta = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    ctx = zo.zo_create(theta, seed=seed)
+    model = zo.zo_model_create(ctx, cfg, max_tokens or B * S)
+    tokens, labels = synth.opt_batch(cfg, B, S, seed=seed)
+    return bits, theta, ctx, model, tokens, labels
+
+
+def _rel_fro(a, b):
+    return np.linalg.norm(a - b) / np.linalg.norm(b)
+
+
+@pytest.mark.parametrize("cfg", TINY)
+@pytest.mark.parametrize("B,S", [(3, 100), (2, 128)])
+def test_decoder_hidden_states_and_loss(zo, cfg, B, S):
+    bits, theta, ctx, model, tokens, labels = _setup(zo, cfg, B, S)
+    dtok = torch.from_numpy(tokens).cuda()
+    dlab = torch.from_numpy(labels).cuda()
+    d = cfg["d_model"]
+    for sign, probe in ((0, 0), (+1, 3), (-1, 3)):
+        if sign:
+            zo.zo_perturb(ctx, sign, 1e-3, probe)
+            P = core.bf16_to_f32(core.perturb(bits, 0, 0, probe, sign, 1e-3)).astype(np.float64)
+        else:
+            P = core.bf16_to_f32(bits).astype(np.float64)
+        for n_run in range(cfg["n_layers"] + 1):
+            h = torch.zeros((B * S, d), dtype=torch.float32, device="cuda")
+            zo.zo_model_hidden(model, dtok, B, S, n_run, h)
+            torch.cuda.synchronize()
+            ref = oracle.opt.hidden_states(P, cfg, tokens, n_layers=n_run).reshape(B * S, d)
+            assert _rel_fro(h.cpu().numpy().astype(np.float64), ref) <= 1e-2, (sign, n_run)
+        out = torch.zeros(1, dtype=torch.float64, device="cuda")
+        zo.zo_model_loss(model, dtok, dlab, B, S, 1.0 / B, out)
+        torch.cuda.synchronize()
+        ref = oracle.opt.loss(P, cfg, tokens, labels)
+        assert abs(out.item() - ref) <= 2e-2 * abs(ref), (sign, out.item(), ref)
+        if sign:
+            zo.zo_restore(ctx)
+    assert zo.zo_sync(ctx) == 0
+    model.close()
+    ctx.close()
+
+
+def test_decoder_rejects_bad_tokens_without_reading_out_of_range(zo):
+    cfg = TINY[0]
+    bits, theta, ctx, model, tokens, labels = _setup(zo, cfg, 2, 64)
+    tokens[1, 5] = cfg["vocab"] + 10
+    out = torch.zeros(1, dtype=torch.float64, device="cuda")
+    zo.zo_model_loss(model, torch.from_numpy(tokens).cuda(), torch.from_numpy(labels).cuda(),
+                     2, 64, 0.5, out)
+    torch.cuda.synchronize()
+    assert np.isnan(out.item())
+    with pytest.raises(zo.ZoError):  # longer than the position table
+        zo.zo_model_loss(model, torch.from_numpy(tokens).cuda(), torch.from_numpy(labels).cuda(),
+                         1, cfg["max_pos"] + 1, 1.0, out)
+    model.close()
+    ctx.close()
+
+
+def test_decoder_step_matches_oracle(zo):
+    """One 1.5-SPSA step with 2 micro-batches: losses against the oracle's, and theta'
+    within the bound propagated from the measured loss discrepancy."""
+    cfg = TINY[0]
+    B, S, n_micro, n, eps, lr, lam = 2, 64, 2, 4, 1e-3, 2e-2, 1e-3
+    bits = synth.opt_params(cfg, seed=1, varied=True)
+    theta = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    ctx = zo.zo_create(theta, seed=1)
+    model = zo.zo_model_create(ctx, cfg, B * S)
+    toks, labs = zip(*(synth.opt_batch(cfg, B, S, seed=1, step=k) for k in range(n_micro)))
+    tokens, labels = np.stack(toks), np.stack(labs)
+    losses = torch.zeros(2 * n + 1, dtype=torch.float64, device="cuda")
+    zo.zo_model_step(model, torch.from_numpy(tokens).cuda(), torch.from_numpy(labels).cuda(),
+                     B, S, n_micro, n, eps, lr, lam, True, losses)
+    assert zo.zo_sync(ctx) == 0
+    assert zo.zo_get_step(ctx) == 1
+    flat_t, flat_l = tokens.reshape(-1, S), labels.reshape(-1)
+    loss = lambda Pb: oracle.opt.loss(core.bf16_to_f32(Pb), cfg, flat_t, flat_l)  # noqa: E731
+    nxt, rec = oracle.step.spsa_step(bits, loss, n, eps, lr, lam, 1, 0)
+    L = losses.cpu().numpy()
+    ref = np.concatenate([[rec["L0"]], rec["Lp"], rec["Lm"]])
+    assert np.allclose(L, ref, rtol=2e-2, atol=0)
+    dL = np.abs(L - ref).max()
+    dg = dL / eps
+    dc = 4 * dL / eps ** 2
+    dw = 0.1 * rec["w"] * dc / (np.abs(rec["c"]) + lam)
+    da = float(np.float32(lr)) / n * (rec["w"] * dg + dw * np.abs(rec["g"]))
+    got = core.bf16_to_f32(theta.view(torch.int16).cpu().numpy().view(np.uint16)).astype(np.float64)
+    exp = core.bf16_to_f32(nxt).astype(np.float64)
+    ulp = np.spacing(np.abs(exp).astype(np.float32)).astype(np.float64) * 65536
+    assert np.all(np.abs(got - exp) <= da.sum() + 2 * ulp)
+    model.close()
+    ctx.close()
+
+
+def test_opt125m_full_size_sampled(zo):
+    """The OPT-125M-shaped workload at full size (16 x 256 tokens): the clean loss and one
+    perturbed loss against the oracle (fp32 numpy forward), and the hidden state after the
+    first layer."""
+    cfg = synth.OPT_CONFIGS["opt-125m"]
+    B, S = 16, 256
+    bits = synth.opt_params(cfg, seed=0)
+    theta = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    ctx = zo.zo_create(theta, seed=0)
+    model = zo.zo_model_create(ctx, cfg, B * S)
+    tokens, labels = synth.opt_batch(cfg, B, S, seed=0)
+    dtok, dlab = torch.from_numpy(tokens).cuda(), torch.from_numpy(labels).cuda()
+    out = torch.zeros(2, dtype=torch.float64, device="cuda")
+    zo.zo_model_loss(model, dtok, dlab, B, S, 1.0 / B, out[0:1])
+    h = torch.zeros((B * S, cfg["d_model"]), dtype=torch.float32, device="cuda")
+    zo.zo_model_hidden(model, dtok, B, S, 1, h)
+    zo.zo_perturb(ctx, +1, 1e-3, 0)
+    zo.zo_model_loss(model, dtok, dlab, B, S, 1.0 / B, out[1:2])
+    zo.zo_restore(ctx)
+    assert zo.zo_sync(ctx) == 0
+    P0 = core.bf16_to_f32(bits)
+    ref0 = oracle.opt.loss(P0, cfg, tokens, labels, dtype=np.float32)
+    href = oracle.opt.hidden_states(P0, cfg, tokens, n_layers=1, dtype=np.float32)
+    assert _rel_fro(h.cpu().numpy().astype(np.float64), href.reshape(B * S, -1).astype(np.float64)) <= 1e-2
+    P1 = core.bf16_to_f32(core.perturb(bits, 0, 0, 0, +1, 1e-3))
+    ref1 = oracle.opt.loss(P1, cfg, tokens, labels, dtype=np.float32)
+    got = out.cpu().numpy()
+    assert abs(got[0] - ref0) <= 2e-2 * abs(ref0)
+    assert abs(got[1] - ref1) <= 2e-2 * abs(ref1)
+    model.close()
+    ctx.close()

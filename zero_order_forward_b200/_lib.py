@@ -19,8 +19,11 @@ if not os.path.exists(LIB_PATH):
 _L = ctypes.CDLL(LIB_PATH)
 
 ZO_F32, ZO_BF16 = 0, 1
-ZO_OK, ZO_ERR_INVALID, ZO_ERR_STATE, ZO_ERR_CUDA, ZO_ERR_OOM, ZO_ERR_NONFINITE, ZO_ERR_UNSUPPORTED = range(7)
+(ZO_OK, ZO_ERR_INVALID, ZO_ERR_STATE, ZO_ERR_CUDA, ZO_ERR_OOM, ZO_ERR_NONFINITE,
+ ZO_ERR_UNSUPPORTED, ZO_ERR_TIMEOUT) = range(8)
 ZO_FLAG_NONFINITE = 0x1
+ZO_FLAG_TIMEOUT = 0x2
+ZO_EPI_BIAS_BF16, ZO_EPI_RELU_BF16, ZO_EPI_RESID_F32 = 0, 1, 2
 ZO_MAX_PROBES = 1024
 ZO_NOALLOC_MAX_BATCH = 4096
 
@@ -48,6 +51,15 @@ _SIGS = {
     "zo_quad_step_host": [_vp, _vp, _i32, _f32, _f32, _f32, _int, _vp],
     "zo_mlp_step": [_vp, _vp, _vp, _int, _int, _int, _int, _i32, _f32, _f32, _f32, _int, _vp],
     "zo_mlp_loss_noalloc": [_vp, _vp, _vp, _int, _int, _int, _int, _f64, _vp, _int, _vp],
+    "zo_model_param_count": [_vp, ctypes.POINTER(_i64)],
+    "zo_model_create": [ctypes.POINTER(_vp), _vp, _vp, _i64],
+    "zo_model_destroy": [_vp],
+    "zo_model_loss": [_vp, _vp, _vp, _i32, _i32, _f64, _vp, _int],
+    "zo_model_hidden": [_vp, _vp, _i32, _i32, _i32, _vp],
+    "zo_model_step": [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _f32, _f32, _f32, _int, _vp],
+    "zo_gemm_bf16": [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32],
+    "zo_attention": [_vp, _vp, _vp, _i32, _i32, _i32, _i32],
+    "zo_layernorm": [_vp, _vp, _vp, _vp, _vp, _i32, _i32],
 }
 for _name, _args in _SIGS.items():
     _fn = getattr(_L, _name)
@@ -240,3 +252,86 @@ def zo_mlp_loss_noalloc(P, X, labels, batch, n_in, n_hidden, n_out, scale, loss_
     if st != ZO_OK:
         raise ZoError(st, "zo_mlp_loss_noalloc failed")
     return st
+
+
+# ------------------------------------------------------------------ decoder
+
+
+class zo_model_cfg(ctypes.Structure):
+    _fields_ = [("n_layers", _i32), ("d_model", _i32), ("n_heads", _i32), ("d_ffn", _i32),
+                ("vocab", _i32), ("max_pos", _i32), ("class_ids", _i32 * 2)]
+
+    @classmethod
+    def from_dict(cls, c):
+        return cls(c["n_layers"], c["d_model"], c["n_heads"], c["d_ffn"], c["vocab"],
+                   c["max_pos"], (_i32 * 2)(*c["class_ids"]))
+
+
+class Model:
+    """Owns a zo_model*; keeps its context alive."""
+
+    def __init__(self, handle, ctx, cfg):
+        self.handle, self.ctx, self.cfg = handle, ctx, cfg
+
+    def close(self):
+        if self.handle:
+            _L.zo_model_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def zo_model_param_count(cfg):
+    m = _i64()
+    c = zo_model_cfg.from_dict(cfg)
+    st = _L.zo_model_param_count(ctypes.byref(c), ctypes.byref(m))
+    if st != ZO_OK:
+        raise ZoError(st, "invalid model configuration")
+    return m.value
+
+
+def zo_model_create(ctx, cfg, max_tokens):
+    h = _vp()
+    c = zo_model_cfg.from_dict(cfg)
+    ctx.check(_L.zo_model_create(ctypes.byref(h), ctx.handle, ctypes.byref(c), int(max_tokens)))
+    return Model(h, ctx, cfg)
+
+
+def zo_model_destroy(model):
+    model.close()
+
+
+def zo_model_loss(model, tokens, labels, batch, seq, scale, loss_out, accumulate=False):
+    return model.ctx.check(_L.zo_model_loss(model.handle, _ptr(tokens), _ptr(labels), batch, seq,
+                                            scale, _ptr(loss_out), int(accumulate)))
+
+
+def zo_model_hidden(model, tokens, batch, seq, n_layers_run, h_out):
+    return model.ctx.check(_L.zo_model_hidden(model.handle, _ptr(tokens), batch, seq,
+                                              n_layers_run, _ptr(h_out)))
+
+
+def zo_model_step(model, tokens, labels, batch, seq, n_micro, n_pert, eps, lr, damping,
+                  preconditioned, losses_out):
+    return model.ctx.check(_L.zo_model_step(model.handle, _ptr(tokens), _ptr(labels), batch, seq,
+                                            n_micro, n_pert, eps, lr, damping,
+                                            int(preconditioned), _ptr(losses_out)))
+
+
+def zo_gemm_bf16(ctx, A, B, bias, out, M, N, K, ldo, epilogue):
+    return ctx.check(_L.zo_gemm_bf16(ctx.handle, _ptr(A), _ptr(B), _ptr(bias), _ptr(out), M, N,
+                                     K, ldo, epilogue))
+
+
+def zo_attention(ctx, qkv, out, batch, seq, n_heads, d_model):
+    return ctx.check(_L.zo_attention(ctx.handle, _ptr(qkv), _ptr(out), batch, seq, n_heads,
+                                     d_model))
+
+
+def zo_layernorm(ctx, x, gamma, beta, out, rows, d):
+    return ctx.check(_L.zo_layernorm(ctx.handle, _ptr(x), _ptr(gamma), _ptr(beta), _ptr(out),
+                                     rows, d))

@@ -1,0 +1,243 @@
+// zo_attn.cu -- causal multi-head attention of the decoder forward (inference only).
+//
+//   out[b, s, h, :] = sum_{s' <= s} softmax_s'( q[b,s,h,:] . k[b,s',h,:] / sqrt(hd) ) v[b,s',h,:]
+//
+// Layout: qkv is the bf16 output of the fused QKV projection, [B*S][3*d] with q, k, v at
+// column offsets 0, d, 2d and head h at +h*hd; out is bf16 [B*S][d].
+//
+// One CTA (4 warps) per (64-query tile, head, sequence); each warp owns 16 query rows.
+// Key/value tiles of 64 rows stream through shared memory (cp.async, double-buffered);
+// scores and the probability-weighted sum use bf16 mma.sync (m16n8k16, fp32 accumulate)
+// with an online softmax in fp32 (running max and sum per row).  Attention is a few per
+// cent of the forward's FLOPs; the projections around it run on tcgen05.
+#include "zo_internal.cuh"
+
+namespace zo {
+namespace {
+
+constexpr int kQT = 64, kKT = 64, kThreads = 128;
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool valid) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  const int n = valid ? 16 : 0;  // 0 source bytes -> zero fill
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t r[4], const void *p) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(s));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t r[4], const void *p) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(s));
+}
+
+// D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col)
+__device__ __forceinline__ void mma16816(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  return (uint32_t)f32_to_bf16_bits(lo) | ((uint32_t)f32_to_bf16_bits(hi) << 16);
+}
+
+template <int HD>
+struct AttnSmem {
+  static constexpr int kStride = HD + 8;  // bf16 elements per smem row (16-byte pad)
+  static constexpr int kTile = kQT * kStride;
+  static constexpr int kBytes = (kTile + 4 * kTile) * 2;  // Q + 2 x (K, V)
+};
+
+template <int HD>
+__global__ void __launch_bounds__(kThreads)
+attn_causal_kernel(const uint16_t *__restrict__ qkv, uint16_t *__restrict__ out, int S, int H,
+                   int d, float scale_log2) {
+  using SM = AttnSmem<HD>;
+  constexpr int ST = SM::kStride;
+  extern __shared__ __align__(16) uint16_t sm[];
+  uint16_t *sQ = sm;
+  // K and V tiles of buffer `buf` at sm + (1 + buf) * kTile and sm + (3 + buf) * kTile
+  auto sK = [&](int buf) { return sm + (1 + buf) * SM::kTile; };
+  auto sV = [&](int buf) { return sm + (3 + buf) * SM::kTile; };
+
+  const int qt = gridDim.x - 1 - blockIdx.x;  // heavy (late) query tiles first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t row0 = (int64_t)b * S;
+  const int64_t ld = 3 * (int64_t)d;
+  const uint16_t *Qg = qkv + h * HD;
+  const uint16_t *Kg = qkv + d + h * HD;
+  const uint16_t *Vg = qkv + 2 * d + h * HD;
+  constexpr int kChunks = HD / 8;  // 16-byte chunks per row
+
+  auto load_tile = [&](uint16_t *dst, const uint16_t *src, int r0) {
+    for (int i = tid; i < kQT * kChunks; i += kThreads) {
+      const int r = i / kChunks, c = i % kChunks;
+      const bool valid = r0 + r < S;
+      const uint16_t *g = src + (row0 + (valid ? r0 + r : 0)) * ld + c * 8;
+      cp_async16(dst + r * ST + c * 8, g, valid);
+    }
+  };
+
+  load_tile(sQ, Qg, qt * kQT);
+  load_tile(sK(0), Kg, 0);
+  load_tile(sV(0), Vg, 0);
+  cp_async_commit();
+
+  float o[HD / 8][4];
+#pragma unroll
+  for (int j = 0; j < HD / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+  uint32_t qf[HD / 16][4];
+  const int g = lane >> 2, t = lane & 3;
+  const int qrow0 = qt * kQT + warp * 16;  // first query row of this warp
+
+  const int n_kt = qt + 1;  // causal: key tiles 0..qt
+  for (int kt = 0; kt < n_kt; ++kt) {
+    const int buf = kt & 1;
+    if (kt + 1 < n_kt) {
+      load_tile(sK(buf ^ 1), Kg, (kt + 1) * kKT);
+      load_tile(sV(buf ^ 1), Vg, (kt + 1) * kKT);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    if (kt == 0) {
+#pragma unroll
+      for (int kk = 0; kk < HD / 16; ++kk)
+        ldsm_x4(qf[kk], sQ + (warp * 16 + (lane & 15)) * ST + kk * 16 + (lane >> 4) * 8);
+    }
+    // scores S = Q K^T for 16 rows x 64 keys
+    float s[kKT / 8][4];
+#pragma unroll
+    for (int j = 0; j < kKT / 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < HD / 16; ++kk) {
+#pragma unroll
+      for (int jj = 0; jj < kKT / 16; ++jj) {
+        uint32_t kb[4];
+        const int key = jj * 16 + (lane & 7) + ((lane >> 4) << 3);
+        const int dim = kk * 16 + ((lane >> 3) & 1) * 8;
+        ldsm_x4(kb, sK(buf) + key * ST + dim);
+        mma16816(s[2 * jj], qf[kk], kb[0], kb[1]);
+        mma16816(s[2 * jj + 1], qf[kk], kb[2], kb[3]);
+      }
+    }
+    // mask (causal on the diagonal tile, and keys beyond S) and online softmax
+    const int key0 = kt * kKT;
+    float mnew[2] = {mrow[0], mrow[1]};
+#pragma unroll
+    for (int j = 0; j < kKT / 8; ++j) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int qr = qrow0 + g + (e >> 1) * 8;
+        const int kc = key0 + 8 * j + 2 * t + (e & 1);
+        if (kc > qr || kc >= S) s[j][e] = -INFINITY;
+        mnew[e >> 1] = fmaxf(mnew[e >> 1], s[j][e]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      mnew[r] = fmaxf(mnew[r], __shfl_xor_sync(0xFFFFFFFFu, mnew[r], 1));
+      mnew[r] = fmaxf(mnew[r], __shfl_xor_sync(0xFFFFFFFFu, mnew[r], 2));
+    }
+    float corr[2], msc[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      // rows that have seen no key yet keep m = -inf; use 0 as the shift then
+      msc[r] = (mnew[r] == -INFINITY) ? 0.f : mnew[r] * scale_log2;
+      corr[r] = (mrow[r] == -INFINITY) ? 0.f : exp2f(mrow[r] * scale_log2 - msc[r]);
+      mrow[r] = mnew[r];
+      lrow[r] *= corr[r];
+    }
+#pragma unroll
+    for (int j = 0; j < HD / 8; ++j) {
+      o[j][0] *= corr[0]; o[j][1] *= corr[0];
+      o[j][2] *= corr[1]; o[j][3] *= corr[1];
+    }
+    uint32_t pf[kKT / 16][4];
+#pragma unroll
+    for (int j = 0; j < kKT / 8; ++j) {
+      float p[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        p[e] = exp2f(s[j][e] * scale_log2 - msc[e >> 1]);
+        lrow[e >> 1] += p[e];
+      }
+      pf[j >> 1][(j & 1) * 2 + 0] = pack_bf16(p[0], p[1]);
+      pf[j >> 1][(j & 1) * 2 + 1] = pack_bf16(p[2], p[3]);
+    }
+    // O += P V
+#pragma unroll
+    for (int kb = 0; kb < kKT / 16; ++kb) {
+      const uint32_t a[4] = {pf[kb][0], pf[kb][1], pf[kb][2], pf[kb][3]};
+#pragma unroll
+      for (int jj = 0; jj < HD / 16; ++jj) {
+        uint32_t vb[4];
+        const int key = kb * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int dim = jj * 16 + (lane >> 4) * 8;
+        ldsm_x4_t(vb, sV(buf) + key * ST + dim);
+        mma16816(o[2 * jj], a, vb[0], vb[1]);
+        mma16816(o[2 * jj + 1], a, vb[2], vb[3]);
+      }
+    }
+    __syncthreads();  // the buffer is refilled two iterations later
+  }
+  // normalise and store
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    lrow[r] += __shfl_xor_sync(0xFFFFFFFFu, lrow[r], 1);
+    lrow[r] += __shfl_xor_sync(0xFFFFFFFFu, lrow[r], 2);
+  }
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int qr = qrow0 + g + r * 8;
+    if (qr >= S) continue;
+    const float inv = lrow[r] > 0.f ? 1.f / lrow[r] : 0.f;
+    uint16_t *orow = out + (row0 + qr) * (int64_t)d + h * HD;
+#pragma unroll
+    for (int j = 0; j < HD / 8; ++j) {
+      const uint32_t v = pack_bf16(o[j][2 * r] * inv, o[j][2 * r + 1] * inv);
+      *reinterpret_cast<uint32_t *>(orow + 8 * j + 2 * t) = v;
+    }
+  }
+}
+
+}  // namespace
+
+zo_status launch_attention(zo_ctx *ctx, const uint16_t *qkv, uint16_t *out, int B, int S, int H,
+                           int d) {
+  if (B < 1 || S < 1 || H < 1 || d % H != 0)
+    return fail(ctx, ZO_ERR_INVALID, "attention: bad shape");
+  const int hd = d / H;
+  if (hd != 64 && hd != 128) return fail(ctx, ZO_ERR_UNSUPPORTED, "attention: head dim must be 64 or 128");
+  if ((reinterpret_cast<uintptr_t>(qkv) | reinterpret_cast<uintptr_t>(out)) & 15u)
+    return fail(ctx, ZO_ERR_INVALID, "attention: buffers must be 16-byte aligned");
+  const float scale_log2 = 1.4426950408889634f / sqrtf((float)hd);
+  dim3 grid((S + kQT - 1) / kQT, H, B);
+  if (hd == 64) {
+    constexpr int bytes = AttnSmem<64>::kBytes;
+    cudaFuncSetAttribute(attn_causal_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    attn_causal_kernel<64><<<grid, kThreads, bytes, ctx->stream>>>(qkv, out, S, H, d, scale_log2);
+  } else {
+    constexpr int bytes = AttnSmem<128>::kBytes;
+    cudaFuncSetAttribute(attn_causal_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    attn_causal_kernel<128><<<grid, kThreads, bytes, ctx->stream>>>(qkv, out, S, H, d, scale_log2);
+  }
+  return check_launch(ctx, "attn_causal_kernel");
+}
+
+}  // namespace zo

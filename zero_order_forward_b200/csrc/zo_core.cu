@@ -107,6 +107,7 @@ const char *zo_status_name(int s) {
     case ZO_ERR_OOM: return "ZO_ERR_OOM";
     case ZO_ERR_NONFINITE: return "ZO_ERR_NONFINITE";
     case ZO_ERR_UNSUPPORTED: return "ZO_ERR_UNSUPPORTED";
+    case ZO_ERR_TIMEOUT: return "ZO_ERR_TIMEOUT";
     default: return "ZO_ERR_UNKNOWN";
   }
 }
@@ -199,6 +200,7 @@ zo_status zo_sync(zo_ctx *ctx, uint32_t *flags) {
     ZO_CUDA(ctx, cudaMemset(&ctx->dstate->flags, 0, sizeof(uint32_t)), "clear flags");
   }
   if (flags) *flags = s.flags;
+  if (s.flags & ZO_FLAG_TIMEOUT) return fail(ctx, ZO_ERR_TIMEOUT, "a kernel gave up a bounded wait");
   if (s.flags & ZO_FLAG_NONFINITE) return fail(ctx, ZO_ERR_NONFINITE, "a loss was not finite; step skipped");
   return ZO_OK;
 }

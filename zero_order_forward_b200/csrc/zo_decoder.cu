@@ -1,0 +1,441 @@
+// zo_decoder.cu -- loss-only forward of an OPT-shaped decoder (pre-LN, learned positions
+// with offset 2, ReLU FFN, biases everywhere, head tied to the token embedding) and the
+// model-level C ABI.
+//
+// Inference mode only ("Probe-Space Preconditioning for Fast and Stable Zero-Order
+// Training", abstract): each layer's activations overwrite the previous layer's, nothing is
+// kept for a backward pass, and memory does not grow with the number of probes.
+//
+// Perturbed evaluation ("Stanford's 1.5-SPSA Trains OPT-30B Without Backpropagation",
+// section "How 1.5-SPSA Works"): the loss at theta + s*eps*z_i.  theta is never written:
+// before a layer runs, the fused unpack/apply kernel materialises that layer's perturbed
+// parameters into one reusable layer window; the token/position embeddings, the final
+// LayerNorm and the tied head rows are perturbed on load.
+//
+// Flat parameter order (bf16), d = d_model, f = d_ffn, V = vocab, P = max_pos + 2:
+//   E[V][d], Pos[P][d],
+//   per layer: ln1.g[d], ln1.b[d], Wqkv[3d][d], bqkv[3d], Wo[d][d], bo[d],
+//              ln2.g[d], ln2.b[d], W1[f][d], b1[f], W2[d][f], b2[d],
+//   final: lnf.g[d], lnf.b[d].
+#include <cstring>
+#include <new>
+
+#include "zo_internal.cuh"
+
+namespace zo {
+
+zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bias, void *out,
+                      int M, int N, int K, int ldo, int epi);
+zo_status launch_attention(zo_ctx *ctx, const uint16_t *qkv, uint16_t *out, int B, int S, int H,
+                           int d);
+
+struct Layout {
+  int64_t E, Pos, layers, layer_size, fin, total;
+  // offsets inside a layer block
+  int64_t ln1g, ln1b, wqkv, bqkv, wo, bo, ln2g, ln2b, w1, b1, w2, b2;
+};
+
+bool make_layout(const zo_model_cfg &c, Layout *L) {
+  if (c.n_layers < 1 || c.d_model < 64 || c.d_model % 64 || c.n_heads < 1 ||
+      c.d_model % c.n_heads || c.d_ffn < 8 || c.d_ffn % 8 || c.vocab < 2 || c.max_pos < 1 ||
+      c.class_ids[0] < 0 || c.class_ids[0] >= c.vocab || c.class_ids[1] < 0 ||
+      c.class_ids[1] >= c.vocab)
+    return false;
+  const int64_t d = c.d_model, f = c.d_ffn;
+  L->E = 0;
+  L->Pos = (int64_t)c.vocab * d;
+  L->layers = L->Pos + (int64_t)(c.max_pos + 2) * d;
+  int64_t o = 0;
+  L->ln1g = o; o += d;
+  L->ln1b = o; o += d;
+  L->wqkv = o; o += 3 * d * d;
+  L->bqkv = o; o += 3 * d;
+  L->wo = o; o += d * d;
+  L->bo = o; o += d;
+  L->ln2g = o; o += d;
+  L->ln2b = o; o += d;
+  L->w1 = o; o += f * d;
+  L->b1 = o; o += f;
+  L->w2 = o; o += d * f;
+  L->b2 = o; o += d;
+  L->layer_size = o;
+  L->fin = L->layers + (int64_t)c.n_layers * o;
+  L->total = L->fin + 2 * d;
+  return true;
+}
+
+namespace {
+
+constexpr int kRowThreads = 256;
+
+// 8 perturbed bf16 parameters starting at global element j (j % 8 == 0), widened to fp32.
+__device__ __forceinline__ void load8_perturbed(const uint16_t *theta, int64_t j,
+                                                const ProbeKey &pk, uint32_t step, float out[8]) {
+  const uint4 v = *reinterpret_cast<const uint4 *>(theta + j);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    out[2 * t] = __uint_as_float(w[t] << 16);
+    out[2 * t + 1] = __uint_as_float(w[t] & 0xFFFF0000u);
+  }
+  if (pk.sign) {
+    const uint4 b = probe_block((uint64_t)j >> 7, pk.probe, step, pk.k0, pk.k1);
+    const uint32_t bits = word_of(b, (int)((j >> 5) & 3)) >> (j & 31);
+    const float delta = pk.sign > 0 ? pk.eps : -pk.eps;
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+      out[t] = bf16_bits_to_f32(f32_to_bf16_bits(perturb_f32(out[t], delta, (bits >> t) & 1u)));
+  }
+}
+
+// h[t][:] = P_E[token] + P_Pos[s + 2] (fp32), one block per token.  An out-of-range
+// token id writes NaN (the loss becomes non-finite and the step is skipped).
+__global__ void __launch_bounds__(kRowThreads)
+embed_kernel(const uint16_t *__restrict__ theta, const int32_t *__restrict__ tokens, int S, int d,
+             int vocab, int64_t pos_off, ProbeKey pk, float *__restrict__ h) {
+  const int64_t t = blockIdx.x;
+  const int s = (int)(t % S);
+  const int tok = tokens[t];
+  const uint32_t step = pk.sign ? *pk.step : 0u;
+  float *hrow = h + t * d;
+  const bool ok = tok >= 0 && tok < vocab;
+  for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
+    if (!ok) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) hrow[c + i] = __int_as_float(0x7FC00000);
+      continue;
+    }
+    float e[8], p[8];
+    load8_perturbed(theta, (int64_t)tok * d + c, pk, step, e);
+    load8_perturbed(theta, pos_off + (int64_t)(s + 2) * d + c, pk, step, p);
+    float4 *o = reinterpret_cast<float4 *>(hrow + c);
+    o[0] = make_float4(e[0] + p[0], e[1] + p[1], e[2] + p[2], e[3] + p[3]);
+    o[1] = make_float4(e[4] + p[4], e[5] + p[5], e[6] + p[6], e[7] + p[7]);
+  }
+}
+
+__device__ __forceinline__ float block_allreduce_sum(float v, float *red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float s = 0.f;
+  for (int i = 0; i < nw; ++i) s += red[i];
+  return s;
+}
+
+// xn = bf16(LayerNorm(x) * g + b), eps 1e-5, one block per row, two passes in fp32.
+constexpr int kMaxPerThread = 32;  // d <= 8192
+
+__global__ void __launch_bounds__(kRowThreads)
+layernorm_kernel(const float *__restrict__ x, const uint16_t *__restrict__ g,
+                 const uint16_t *__restrict__ b, uint16_t *__restrict__ y, int d) {
+  __shared__ float red[kRowThreads / 32];
+  const float *row = x + (int64_t)blockIdx.x * d;
+  float v[kMaxPerThread];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxPerThread; ++i) {
+    const int c = threadIdx.x + i * kRowThreads;
+    v[i] = c < d ? row[c] : 0.f;
+    s += v[i];
+  }
+  const float mean = block_allreduce_sum(s, red) / (float)d;
+  float q = 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxPerThread; ++i) {
+    const int c = threadIdx.x + i * kRowThreads;
+    const float u = c < d ? v[i] - mean : 0.f;
+    q += u * u;
+  }
+  const float var = block_allreduce_sum(q, red) / (float)d;
+  const float rstd = rsqrtf(var + 1e-5f);
+  uint16_t *out = y + (int64_t)blockIdx.x * d;
+#pragma unroll
+  for (int i = 0; i < kMaxPerThread; ++i) {
+    const int c = threadIdx.x + i * kRowThreads;
+    if (c < d)
+      out[c] = f32_to_bf16_bits((v[i] - mean) * rstd * bf16_bits_to_f32(g[c]) + bf16_bits_to_f32(b[c]));
+  }
+}
+
+// Per sample: final LayerNorm of the last position, logits of the two class tokens through
+// the tied head, 2-class cross-entropy.  Parameters perturbed on load.
+__global__ void __launch_bounds__(kRowThreads)
+head_ce_kernel(const float *__restrict__ h, const uint16_t *__restrict__ theta, int S, int d,
+               int64_t fin_off, int id0, int id1, const int32_t *__restrict__ labels,
+               ProbeKey pk, double *partials, unsigned int *counter, double *out, int accumulate,
+               double scale) {
+  __shared__ float red[kRowThreads / 32];
+  __shared__ bool last;
+  const int b = blockIdx.x;
+  const float *row = h + ((int64_t)b * S + S - 1) * d;
+  const uint32_t step = pk.sign ? *pk.step : 0u;
+  float s = 0.f;
+  for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8)
+    for (int i = 0; i < 8; ++i) s += row[c + i];
+  const float mean = block_allreduce_sum(s, red) / (float)d;
+  float q = 0.f;
+  for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8)
+    for (int i = 0; i < 8; ++i) {
+      const float u = row[c + i] - mean;
+      q += u * u;
+    }
+  const float rstd = rsqrtf(block_allreduce_sum(q, red) / (float)d + 1e-5f);
+  float l0 = 0.f, l1 = 0.f;
+  for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
+    float g[8], bb[8], e0[8], e1[8];
+    load8_perturbed(theta, fin_off + c, pk, step, g);
+    load8_perturbed(theta, fin_off + d + c, pk, step, bb);
+    load8_perturbed(theta, (int64_t)id0 * d + c, pk, step, e0);
+    load8_perturbed(theta, (int64_t)id1 * d + c, pk, step, e1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float xn = (row[c + i] - mean) * rstd * g[i] + bb[i];
+      l0 = fmaf(xn, e0[i], l0);
+      l1 = fmaf(xn, e1[i], l1);
+    }
+  }
+  l0 = block_allreduce_sum(l0, red);
+  l1 = block_allreduce_sum(l1, red);
+  if (threadIdx.x == 0) {
+    const int y = labels[b];
+    const float m = fmaxf(l0, l1);
+    const double lse = (double)m + (double)logf(expf(l0 - m) + expf(l1 - m));
+    const double ce = (y == 0 || y == 1) ? lse - (double)(y == 0 ? l0 : l1) : (double)NAN;
+    partials[b] = ce;
+    __threadfence();
+    last = atomicAdd(counter, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!last || threadIdx.x != 0) return;
+  __threadfence();
+  double tot = 0.0;
+  for (unsigned int i = 0; i < gridDim.x; ++i) tot += __ldcg(partials + i);  // fixed order
+  *out = (accumulate ? *out : 0.0) + scale * tot;
+  *counter = 0u;
+}
+
+}  // namespace
+}  // namespace zo
+
+using namespace zo;
+
+struct zo_model {
+  zo_ctx *ctx = nullptr;
+  zo_model_cfg cfg{};
+  Layout L{};
+  int64_t max_tokens = 0;
+  uint16_t *window = nullptr;
+  float *h = nullptr;
+  uint16_t *xn = nullptr, *qkv = nullptr, *attn = nullptr, *mid = nullptr;
+};
+
+namespace {
+
+zo_status model_cuda(zo_ctx *ctx, cudaError_t e, const char *what) {
+  if (e == cudaSuccess) return ZO_OK;
+  cudaGetLastError();
+  return fail(ctx, e == cudaErrorMemoryAllocation ? ZO_ERR_OOM : ZO_ERR_CUDA, "%s: %s", what,
+              cudaGetErrorString(e));
+}
+
+// Embedding plus the first n_run layers for one micro-batch; leaves the residual in m->h.
+zo_status run_layers(zo_model *m, const int32_t *tokens, int B, int S, int n_run) {
+  zo_ctx *ctx = m->ctx;
+  const zo_model_cfg &c = m->cfg;
+  const Layout &L = m->L;
+  const int d = c.d_model, f = c.d_ffn;
+  const int T = B * S;
+  const uint16_t *theta = static_cast<const uint16_t *>(ctx->params);
+  const ProbeKey pk = probe_key(ctx);
+  embed_kernel<<<T, kRowThreads, 0, ctx->stream>>>(theta, tokens, S, d, c.vocab, L.Pos, pk, m->h);
+  zo_status st = check_launch(ctx, "embed_kernel");
+  if (st != ZO_OK) return st;
+  for (int l = 0; l < n_run; ++l) {
+    const int64_t off = L.layers + (int64_t)l * L.layer_size;
+    const uint16_t *lp = theta + off;
+    if (pk.sign) {  // materialise this layer's perturbed parameters into the window
+      st = launch_perturb(ctx, pk, off, L.layer_size, m->window);
+      if (st != ZO_OK) return st;
+      lp = m->window;
+    }
+    layernorm_kernel<<<T, kRowThreads, 0, ctx->stream>>>(m->h, lp + L.ln1g, lp + L.ln1b, m->xn, d);
+    if ((st = check_launch(ctx, "layernorm_kernel")) != ZO_OK) return st;
+    if ((st = launch_gemm(ctx, m->xn, lp + L.wqkv, lp + L.bqkv, m->qkv, T, 3 * d, d, 3 * d,
+                          ZO_EPI_BIAS_BF16)) != ZO_OK) return st;
+    if ((st = launch_attention(ctx, m->qkv, m->attn, B, S, c.n_heads, d)) != ZO_OK) return st;
+    if ((st = launch_gemm(ctx, m->attn, lp + L.wo, lp + L.bo, m->h, T, d, d, d,
+                          ZO_EPI_RESID_F32)) != ZO_OK) return st;
+    layernorm_kernel<<<T, kRowThreads, 0, ctx->stream>>>(m->h, lp + L.ln2g, lp + L.ln2b, m->xn, d);
+    if ((st = check_launch(ctx, "layernorm_kernel")) != ZO_OK) return st;
+    if ((st = launch_gemm(ctx, m->xn, lp + L.w1, lp + L.b1, m->mid, T, f, d, f,
+                          ZO_EPI_RELU_BF16)) != ZO_OK) return st;
+    if ((st = launch_gemm(ctx, m->mid, lp + L.w2, lp + L.b2, m->h, T, d, f, d,
+                          ZO_EPI_RESID_F32)) != ZO_OK) return st;
+  }
+  return ZO_OK;
+}
+
+zo_status check_batch(zo_model *m, const int32_t *tokens, int B, int S) {
+  if (!tokens || B < 1 || S < 1 || S > m->cfg.max_pos || (int64_t)B * S > m->max_tokens)
+    return fail(m->ctx, ZO_ERR_INVALID, "batch %d x seq %d: need seq <= max_pos and B*S <= %lld",
+                B, S, (long long)m->max_tokens);
+  return ZO_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+zo_status zo_model_param_count(const zo_model_cfg *cfg, int64_t *M_out) {
+  Layout L;
+  if (!cfg || !M_out || !make_layout(*cfg, &L)) return ZO_ERR_INVALID;
+  *M_out = L.total;
+  return ZO_OK;
+}
+
+zo_status zo_model_create(zo_model **out, zo_ctx *ctx, const zo_model_cfg *cfg, int64_t max_tokens) {
+  if (!out) return ZO_ERR_INVALID;
+  *out = nullptr;
+  if (!ctx || !cfg) return ZO_ERR_INVALID;
+  Layout L;
+  if (!make_layout(*cfg, &L)) return fail(ctx, ZO_ERR_INVALID, "invalid model configuration");
+  if (ctx->dtype != ZO_BF16 || ctx->M != L.total)
+    return fail(ctx, ZO_ERR_INVALID, "model needs a bf16 context with M = %lld", (long long)L.total);
+  if (max_tokens < 1) return fail(ctx, ZO_ERR_INVALID, "max_tokens must be >= 1");
+  zo_model *m = new (std::nothrow) zo_model();
+  if (!m) return ZO_ERR_OOM;
+  m->ctx = ctx;
+  m->cfg = *cfg;
+  m->L = L;
+  m->max_tokens = max_tokens;
+  const int64_t T = max_tokens, d = cfg->d_model, f = cfg->d_ffn;
+  cudaError_t e = cudaMalloc(&m->window, (size_t)L.layer_size * 2);
+  if (e == cudaSuccess) e = cudaMalloc(&m->h, (size_t)T * d * 4);
+  if (e == cudaSuccess) e = cudaMalloc(&m->xn, (size_t)T * d * 2);
+  if (e == cudaSuccess) e = cudaMalloc(&m->qkv, (size_t)T * 3 * d * 2);
+  if (e == cudaSuccess) e = cudaMalloc(&m->attn, (size_t)T * d * 2);
+  if (e == cudaSuccess) e = cudaMalloc(&m->mid, (size_t)T * f * 2);
+  if (e != cudaSuccess) {
+    const zo_status st = model_cuda(ctx, e, "model buffers");
+    zo_model_destroy(m);
+    return st;
+  }
+  *out = m;
+  return ZO_OK;
+}
+
+zo_status zo_model_destroy(zo_model *m) {
+  if (!m) return ZO_OK;
+  cudaStreamSynchronize(m->ctx->stream);
+  cudaFree(m->window);
+  cudaFree(m->h);
+  cudaFree(m->xn);
+  cudaFree(m->qkv);
+  cudaFree(m->attn);
+  cudaFree(m->mid);
+  delete m;
+  return ZO_OK;
+}
+
+zo_status zo_model_loss(zo_model *m, const int32_t *tokens, const int32_t *labels, int32_t batch,
+                        int32_t seq, double scale, double *loss_out, int accumulate) {
+  if (!m) return ZO_ERR_INVALID;
+  zo_ctx *ctx = m->ctx;
+  ctx->err.clear();
+  zo_status st = check_batch(m, tokens, batch, seq);
+  if (st != ZO_OK) return st;
+  if (!labels || !loss_out) return fail(ctx, ZO_ERR_INVALID, "null labels or loss_out");
+  if (batch > kMaxPartials) return fail(ctx, ZO_ERR_INVALID, "batch above %d", kMaxPartials);
+  if ((st = run_layers(m, tokens, batch, seq, m->cfg.n_layers)) != ZO_OK) return st;
+  const ProbeKey pk = probe_key(ctx);
+  head_ce_kernel<<<batch, kRowThreads, 0, ctx->stream>>>(
+      m->h, static_cast<const uint16_t *>(ctx->params), seq, m->cfg.d_model, m->L.fin,
+      m->cfg.class_ids[0], m->cfg.class_ids[1], labels, pk, ctx->partials, ctx->counter, loss_out,
+      accumulate, scale);
+  return check_launch(ctx, "head_ce_kernel");
+}
+
+zo_status zo_model_hidden(zo_model *m, const int32_t *tokens, int32_t batch, int32_t seq,
+                          int32_t n_layers_run, float *h_out) {
+  if (!m) return ZO_ERR_INVALID;
+  zo_ctx *ctx = m->ctx;
+  ctx->err.clear();
+  zo_status st = check_batch(m, tokens, batch, seq);
+  if (st != ZO_OK) return st;
+  if (!h_out || n_layers_run < 0 || n_layers_run > m->cfg.n_layers)
+    return fail(ctx, ZO_ERR_INVALID, "bad hidden-state request");
+  if ((st = run_layers(m, tokens, batch, seq, n_layers_run)) != ZO_OK) return st;
+  return model_cuda(ctx,
+                    cudaMemcpyAsync(h_out, m->h, (size_t)batch * seq * m->cfg.d_model * 4,
+                                    cudaMemcpyDeviceToDevice, ctx->stream),
+                    "copy hidden state");
+}
+
+zo_status zo_model_step(zo_model *m, const int32_t *tokens, const int32_t *labels, int32_t batch,
+                        int32_t seq, int32_t n_micro, int32_t n_pert, float eps, float lr,
+                        float damping, int preconditioned, double *losses_out) {
+  if (!m) return ZO_ERR_INVALID;
+  zo_ctx *ctx = m->ctx;
+  if (n_micro < 1 || !losses_out) return fail(ctx, ZO_ERR_INVALID, "bad step arguments");
+  if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "step while perturbed");
+  const double scale = 1.0 / ((double)n_micro * batch);
+  const int64_t tok_stride = (int64_t)batch * seq;
+  double *L0 = losses_out, *Lp = losses_out + 1, *Lm = losses_out + 1 + n_pert;
+  zo_status st;
+  if (n_pert < 1 || n_pert > ZO_MAX_PROBES) return fail(ctx, ZO_ERR_INVALID, "n_pert out of range");
+  if (preconditioned) {
+    for (int k = 0; k < n_micro; ++k)
+      if ((st = zo_model_loss(m, tokens + k * tok_stride, labels + (int64_t)k * batch, batch, seq,
+                              scale, L0, k > 0)) != ZO_OK)
+        return st;
+  } else if ((st = model_cuda(ctx, cudaMemsetAsync(L0, 0, sizeof(double), ctx->stream),
+                              "clear L0")) != ZO_OK) {
+    return st;
+  }
+  for (int32_t i = 0; i < n_pert; ++i) {
+    for (int s = +1; s >= -1; s -= 2) {
+      if ((st = zo_perturb(ctx, s, eps, i)) != ZO_OK) return st;
+      for (int k = 0; k < n_micro && st == ZO_OK; ++k)
+        st = zo_model_loss(m, tokens + k * tok_stride, labels + (int64_t)k * batch, batch, seq,
+                           scale, (s > 0 ? Lp : Lm) + i, k > 0);
+      zo_restore(ctx);
+      if (st != ZO_OK) return st;
+    }
+  }
+  return zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
+}
+
+zo_status zo_gemm_bf16(zo_ctx *ctx, const void *A, const void *B, const void *bias, void *out,
+                       int32_t M, int32_t N, int32_t K, int32_t ldo, int32_t epilogue) {
+  if (!ctx) return ZO_ERR_INVALID;
+  ctx->err.clear();
+  if (!A || !B || !out) return fail(ctx, ZO_ERR_INVALID, "null gemm operand");
+  return launch_gemm(ctx, A, B, bias, out, M, N, K, ldo, epilogue);
+}
+
+zo_status zo_attention(zo_ctx *ctx, const void *qkv, void *out, int32_t batch, int32_t seq,
+                       int32_t n_heads, int32_t d_model) {
+  if (!ctx) return ZO_ERR_INVALID;
+  ctx->err.clear();
+  if (!qkv || !out) return fail(ctx, ZO_ERR_INVALID, "null attention buffer");
+  return launch_attention(ctx, static_cast<const uint16_t *>(qkv), static_cast<uint16_t *>(out),
+                          batch, seq, n_heads, d_model);
+}
+
+zo_status zo_layernorm(zo_ctx *ctx, const float *x, const void *gamma, const void *beta, void *out,
+                       int32_t rows, int32_t d) {
+  if (!ctx) return ZO_ERR_INVALID;
+  ctx->err.clear();
+  if (!x || !gamma || !beta || !out || rows < 1 || d < 1 || d > kMaxPerThread * kRowThreads)
+    return fail(ctx, ZO_ERR_INVALID, "bad layernorm arguments");
+  layernorm_kernel<<<rows, kRowThreads, 0, ctx->stream>>>(
+      x, static_cast<const uint16_t *>(gamma), static_cast<const uint16_t *>(beta),
+      static_cast<uint16_t *>(out), d);
+  return check_launch(ctx, "layernorm_kernel");
+}
+
+}  // extern "C"

@@ -1,0 +1,310 @@
+// zo_gemm.cu -- bf16 GEMM on the 5th-generation tensor cores for the decoder forward:
+//   out[M][N] = epilogue(A[M][K] . B[N][K]^T + bias[N])
+// A (activations) and B (weights, nn.Linear layout) are both K-major.  This is the only
+// dense contraction on the path (the decoder's QKV, output, FC1 and FC2 projections).
+//
+// Design (one 128 x BN output tile per CTA, 192 threads):
+//   warp 0     one lane issues TMA tile loads (128-byte swizzle) into a STAGES-deep ring
+//              of shared-memory stages, paced by "empty" mbarriers;
+//   warp 1     allocates BN TMEM columns; one lane issues tcgen05.mma (M=128, N=BN,
+//              K=16, bf16 x bf16 -> fp32 in TMEM) and commits each stage back to its
+//              "empty" barrier, then commits the finished accumulator;
+//   warps 2-5  the epilogue: tcgen05.ld 32 columns at a time (warp w reads TMEM lanes
+//              32*(w%4)..+31 = its 32 output rows), adds the bias, applies ReLU or the
+//              fp32 residual add, and stores.
+// Tiles are visited in groups of kGroupM row tiles so that the weight tiles of a group are
+// reused from L2.  All waits are bounded (see zo_tc.cuh); a timeout sets an error bit.
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <mutex>
+
+#include "zo_internal.cuh"
+#include "zo_tc.cuh"
+
+namespace zo {
+
+namespace {
+
+constexpr int kBM = 128, kBK = 64, kGroupM = 8;
+
+struct GemmArgs {
+  int M, N, K;
+  const uint16_t *bias;  // [N] bf16 or null
+  void *out;             // bf16 [M][ldo] or fp32 [M][ldo]
+  int ldo;
+  uint32_t *err;         // device error word (ZO_FLAG_TIMEOUT raised on a bounded-wait expiry)
+};
+
+__device__ __forceinline__ void load_bias32(const uint16_t *bias, int col0, int N, float b[32]) {
+  if (bias == nullptr) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) b[i] = 0.f;
+    return;
+  }
+  if (col0 + 32 <= N) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4 *>(bias + col0) + k);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        b[8 * k + 2 * t] = __uint_as_float(w[t] << 16);
+        b[8 * k + 2 * t + 1] = __uint_as_float(w[t] & 0xFFFF0000u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) b[i] = (col0 + i < N) ? bf16_bits_to_f32(bias[col0 + i]) : 0.f;
+  }
+}
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_store(const float acc[32], int row, int col0,
+                                               const GemmArgs &a) {
+  float b[32];
+  load_bias32(a.bias, col0, a.N, b);
+  if (EPI == ZO_EPI_RESID_F32) {
+    float *o = static_cast<float *>(a.out) + (int64_t)row * a.ldo + col0;
+    if (col0 + 32 <= a.N) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        float4 h = reinterpret_cast<float4 *>(o)[k];
+        h.x = __fadd_rn(h.x, __fadd_rn(acc[4 * k], b[4 * k]));
+        h.y = __fadd_rn(h.y, __fadd_rn(acc[4 * k + 1], b[4 * k + 1]));
+        h.z = __fadd_rn(h.z, __fadd_rn(acc[4 * k + 2], b[4 * k + 2]));
+        h.w = __fadd_rn(h.w, __fadd_rn(acc[4 * k + 3], b[4 * k + 3]));
+        reinterpret_cast<float4 *>(o)[k] = h;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (col0 + i < a.N) o[i] = __fadd_rn(o[i], __fadd_rn(acc[i], b[i]));
+    }
+  } else {
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      v[i] = __fadd_rn(acc[i], b[i]);
+      if (EPI == ZO_EPI_RELU_BF16) v[i] = fmaxf(v[i], 0.f);
+    }
+    uint16_t *o = static_cast<uint16_t *>(a.out) + (int64_t)row * a.ldo + col0;
+    if (col0 + 32 <= a.N) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint32_t w[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          w[t] = (uint32_t)f32_to_bf16_bits(v[8 * k + 2 * t]) |
+                 ((uint32_t)f32_to_bf16_bits(v[8 * k + 2 * t + 1]) << 16);
+        reinterpret_cast<uint4 *>(o)[k] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (col0 + i < a.N) o[i] = f32_to_bf16_bits(v[i]);
+    }
+  }
+}
+
+template <int BN, int STAGES>
+struct GemmSmem {
+  static constexpr uint32_t kABytes = kBM * kBK * 2;
+  static constexpr uint32_t kBBytes = BN * kBK * 2;
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  static constexpr uint32_t kBarOffset = STAGES * kStageBytes;
+  static constexpr uint32_t kBytes = kBarOffset + 256 + 1024;  // + barriers + alignment slack
+};
+
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(192, 1)
+gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 GemmArgs args) {
+  using S = GemmSmem<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + STAGES * S::kABytes;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + S::kBarOffset);
+  uint64_t *empty = full + STAGES;
+  uint64_t *done = empty + STAGES;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(done + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // grouped tile order: kGroupM row tiles share each sweep over the column tiles
+  const int num_m = (args.M + kBM - 1) / kBM, num_n = (args.N + BN - 1) / BN;
+  const int pid = blockIdx.x;
+  const int group = pid / (kGroupM * num_n);
+  const int first_m = group * kGroupM;
+  const int gsize = min(num_m - first_m, kGroupM);
+  const int m_tile = first_m + (pid % gsize);
+  const int n_tile = (pid % (kGroupM * num_n)) / gsize;
+  const int m0 = m_tile * kBM, n0 = n_tile * BN;
+  const int nk = (args.K + kBK - 1) / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(done, 1);
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) tc::tmem_alloc(tmem_holder, BN);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  int issued = 0;
+  if (warp == 0 && lane == 0) {
+    tc::tma_prefetch_desc(&tmA);
+    tc::tma_prefetch_desc(&tmB);
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % STAGES;
+      const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+      if (*abort_flag || !tc::mbar_wait(&empty[s], ph ^ 1u)) {
+        atomicOr(args.err, ZO_FLAG_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      tc::mbar_arrive_expect_tx(&full[s], S::kStageBytes);
+      tc::tma_load_2d(sA + s * S::kABytes, &tmA, &full[s], kb * kBK, m0);
+      tc::tma_load_2d(sB + s * S::kBBytes, &tmB, &full[s], kb * kBK, n0);
+      issued = kb + 1;
+    }
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc = tc::idesc_bf16_f32(kBM, BN);
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % STAGES;
+      const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+      if (*abort_flag || !tc::mbar_wait(&full[s], ph)) {
+        atomicOr(args.err, ZO_FLAG_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      tc::tc_fence_after();
+      const uint32_t a0 = tc::smem_addr(sA + s * S::kABytes);
+      const uint32_t b0 = tc::smem_addr(sB + s * S::kBBytes);
+#pragma unroll
+      for (int k = 0; k < kBK / 16; ++k)
+        tc::mma_bf16(tmem, tc::smem_desc_k128(a0 + 32 * k), tc::smem_desc_k128(b0 + 32 * k), idesc,
+                     (kb | k) != 0 ? 1u : 0u);
+      tc::mma_commit(&empty[s]);
+    }
+    tc::mma_commit(done);  // also covers an aborted loop: waits for the MMAs issued so far
+  } else if (warp >= 2) {
+    const int q = warp & 3;
+    const bool ok = tc::mbar_wait(done, 0);
+    if (!ok) atomicOr(args.err, ZO_FLAG_TIMEOUT);
+    tc::tc_fence_after();
+    if (ok && !*abort_flag) {
+      const int row = m0 + q * 32 + lane;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        if (n0 + c0 >= args.N) break;
+        float v[32];
+        tc::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+        if (row < args.M) epilogue_store<EPI>(v, row, n0 + c0, args);
+      }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0 && lane == 0 && *abort_flag) {
+    // wait (bounded) for this CTA's TMA loads still in flight before the CTA exits
+    for (int s = 0; s < STAGES; ++s) {
+      int last = -1;
+      for (int kb = s; kb < issued; kb += STAGES) last = kb;
+      if (last >= 0 && !tc::mbar_wait(&full[s], (uint32_t)(last / STAGES) & 1u))
+        atomicOr(args.err, ZO_FLAG_TIMEOUT);
+    }
+  }
+  if (warp == 1) {
+    if (lane == 0 && *abort_flag && !tc::mbar_wait(done, 0)) atomicOr(args.err, ZO_FLAG_TIMEOUT);
+    __syncwarp();
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, BN);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [rows][cols] (row-major, cols contiguous), box = box_rows x 64 columns,
+// 128-byte swizzle, zero fill outside the tensor.
+bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES, int EPI>
+cudaError_t launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &g,
+                       cudaStream_t st) {
+  using S = GemmSmem<BN, STAGES>;
+  auto kern = gemm_bf16_kernel<BN, STAGES, EPI>;
+  static bool attr_set = false;  // per instantiation; benign race (idempotent call)
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::kBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int num_m = (g.M + kBM - 1) / kBM, num_n = (g.N + BN - 1) / BN;
+  kern<<<num_m * num_n, 192, S::kBytes, st>>>(ta, tb, g);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bias, void *out,
+                      int M, int N, int K, int ldo, int epi) {
+  if (M < 1 || N < 1 || K < 1 || (K % 8) != 0 || (ldo % 8) != 0 || ldo < N)
+    return fail(ctx, ZO_ERR_INVALID, "gemm: need M,N,K >= 1, K %% 8 == 0, ldo %% 8 == 0, ldo >= N");
+  if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B) |
+       reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(bias)) & 15u)
+    return fail(ctx, ZO_ERR_INVALID, "gemm: operands must be 16-byte aligned");
+  if (epi < ZO_EPI_BIAS_BF16 || epi > ZO_EPI_RESID_F32) return fail(ctx, ZO_ERR_INVALID, "gemm: bad epilogue");
+  // N <= 128 tiles use BN = 128 to fill the machine on narrow outputs.
+  const bool wide = N > 128 && ((int64_t)((M + 127) / 128) * ((N + 255) / 256) >= kSmCount);
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, A, M, K, kBM) || !make_map(&tb, B, N, K, wide ? 256 : 128))
+    return fail(ctx, ZO_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
+  GemmArgs g{M, N, K, static_cast<const uint16_t *>(bias), out, ldo, &ctx->dstate->flags};
+  cudaError_t e;
+  if (wide) {
+    if (epi == ZO_EPI_BIAS_BF16) e = launch_one<256, 4, ZO_EPI_BIAS_BF16>(ta, tb, g, ctx->stream);
+    else if (epi == ZO_EPI_RELU_BF16) e = launch_one<256, 4, ZO_EPI_RELU_BF16>(ta, tb, g, ctx->stream);
+    else e = launch_one<256, 4, ZO_EPI_RESID_F32>(ta, tb, g, ctx->stream);
+  } else {
+    if (epi == ZO_EPI_BIAS_BF16) e = launch_one<128, 6, ZO_EPI_BIAS_BF16>(ta, tb, g, ctx->stream);
+    else if (epi == ZO_EPI_RELU_BF16) e = launch_one<128, 6, ZO_EPI_RELU_BF16>(ta, tb, g, ctx->stream);
+    else e = launch_one<128, 6, ZO_EPI_RESID_F32>(ta, tb, g, ctx->stream);
+  }
+  if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "gemm launch: %s", cudaGetErrorString(e));
+  return ZO_OK;
+}
+
+}  // namespace zo
