@@ -7,6 +7,11 @@ eps = 1e-3, lr = 4e-7, damping = 1e-3, 1.5-SPSA.  One step = clean loss + 2*n_pe
 perturbed losses + preconditioner + update, all through the C ABI of libzo.so.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload quadratic|opt-125m|opt-1.3b|opt-30b]
+
+The decoder workloads (OPT-shaped, bf16 weights N(0, 0.02), uniform tokens, 2-class
+last-token loss) time whole 1.5-SPSA steps through zo_model_step and add a per-GEMM-shape
+breakdown of the tcgen05 projections against the measured bf16 peak.
 
 Prints ONE JSON line (rank 0).  With N > 1 (torchrun, one rank per GPU) every rank runs
 its own replica of the workload (independent problems, no collective on the data path);
@@ -34,6 +39,16 @@ WORKLOAD = ("diagonal quadratic L=1/2*sum D_j theta_j^2, M=2^24 fp32, D log-unif
 FALLBACK_HBM_GBS = 6650.0
 
 
+FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS_SUSTAINED = 1590.0, 1400.0
+
+DECODER_WORKLOADS = {
+    # model shape, micro-batch, micro-batches per effective batch, probes per step
+    "opt-125m": dict(batch=16, seq=256, n_micro=1, n_pert=32),
+    "opt-1.3b": dict(batch=16, seq=512, n_micro=8, n_pert=160),
+    "opt-30b": dict(batch=8, seq=2048, n_micro=1, n_pert=16),
+}
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -41,6 +56,15 @@ def peaks():
         return float(p["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def bf16_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback"
 
 
 def dist_env():
@@ -296,6 +320,141 @@ def gpu_arm(args):
     return 0
 
 
+# ------------------------------------------------------------------ decoder workloads
+
+def init_decoder_params(theta, cfg, seed):
+    """OPT-style synthetic initialisation on the device (too large for host numpy at 30B):
+    matrices N(0, 0.02) in bf16, biases 0, LayerNorm gains 1 and shifts 0."""
+    import torch
+
+    import synth
+    g = torch.Generator(device=theta.device)
+    g.manual_seed(seed)
+    o = 0
+    for kind, n in synth.opt_segments(cfg):
+        seg = theta[o:o + n]
+        if kind == "matrix":
+            step = 1 << 28
+            for a in range(0, n, step):
+                seg[a:a + step].normal_(0.0, 0.02, generator=g)
+        elif kind == "gain":
+            seg.fill_(1.0)
+        else:
+            seg.zero_()
+        o += n
+
+
+def decoder_arm(args):
+    import torch
+
+    import synth
+    import zero_order_forward_b200 as zo
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    name = args.workload
+    cfg = synth.OPT_CONFIGS[name]
+    w = dict(DECODER_WORKLOADS[name])
+    if args.n_pert:
+        w["n_pert"] = args.n_pert
+    B, S, k, n = w["batch"], w["seq"], w["n_micro"], w["n_pert"]
+    M = zo.zo_model_param_count(cfg)
+    theta = torch.empty(M, dtype=torch.bfloat16, device=dev)
+    init_decoder_params(theta, cfg, seed=rank)
+    stream = torch.cuda.current_stream(dev)
+    ctx = zo.zo_create(theta, seed=rank, stream=stream.cuda_stream)
+    model = zo.zo_model_create(ctx, cfg, B * S)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1000 + rank)
+    tokens = torch.randint(0, cfg["vocab"], (k, B, S), dtype=torch.int32, device=dev, generator=gen)
+    labels = torch.randint(0, 2, (k, B), dtype=torch.int32, device=dev, generator=gen)
+    losses = torch.zeros(2 * n + 1, dtype=torch.float64, device=dev)
+    eps, lr, lam = 1e-3, 1e-6, 1e-3
+
+    def step():
+        zo.zo_model_step(model, tokens, labels, B, S, k, n, eps, lr, lam, True, losses)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    ev[0].record(stream)
+    for i in range(args.steps):
+        step()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    zo.zo_sync(ctx)
+    total_s = ev[0].elapsed_time(ev[-1]) / 1e3
+    peak_mem = torch.cuda.max_memory_allocated(dev)
+    free_b, tot_b = torch.cuda.mem_get_info(dev)
+
+    # one clean forward, and each projection GEMM at this micro-batch's shape
+    T, d, f = B * S, cfg["d_model"], cfg["d_ffn"]
+    fe = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    fe[0].record(stream)
+    zo.zo_model_loss(model, tokens[0], labels[0], B, S, 1.0 / B, losses[0:1])
+    fe[1].record(stream)
+    torch.cuda.synchronize()
+    fwd_ms = fe[0].elapsed_time(fe[1])
+    peak_b, peak_s, peak_kind = bf16_peaks()
+    shapes = {"qkv": (T, 3 * d, d, 0), "out": (T, d, d, 2), "fc1": (T, f, d, 1), "fc2": (T, d, f, 2)}
+    gemm = {}
+    A = torch.randn(T * max(d, f), dtype=torch.bfloat16, device=dev)
+    Wt = torch.randn(max(3 * d * d, f * d), dtype=torch.bfloat16, device=dev) * 0.02
+    bias = torch.zeros(max(3 * d, f), dtype=torch.bfloat16, device=dev)
+    out_b = torch.empty(T * max(3 * d, f), dtype=torch.bfloat16, device=dev)
+    out_f = torch.zeros(T * d, dtype=torch.float32, device=dev)
+    flops_layer = 0
+    for key, (Mm, N, K, epi) in shapes.items():
+        out = out_f if epi == 2 else out_b
+        for _ in range(2):
+            zo.zo_gemm_bf16(ctx, A, Wt, bias, out, Mm, N, K, N, epi)
+        reps = 5
+        ge = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ge[0].record(stream)
+        for _ in range(reps):
+            zo.zo_gemm_bf16(ctx, A, Wt, bias, out, Mm, N, K, N, epi)
+        ge[1].record(stream)
+        torch.cuda.synchronize()
+        us = 1e3 * ge[0].elapsed_time(ge[1]) / reps
+        fl = 2.0 * Mm * N * K
+        flops_layer += fl
+        gemm[key] = {"shape": [Mm, N, K], "avg_launch_us": us, "tflops": fl / us / 1e6,
+                     "frac_burst": fl / us / 1e6 / peak_b}
+    zo.zo_sync(ctx)
+    gemm_us = sum(g["avg_launch_us"] for g in gemm.values())
+    gemm_tflops = flops_layer / gemm_us / 1e6
+    fwds = (2 * n + 1) * k
+    tokens_per_step = fwds * T
+    value = args.steps / total_s
+    line = {
+        "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{name}-shaped decoder, micro-batch {B}x{S}, {k} micro-batches, "
+                               f"n_pert={n}, 1.5-SPSA", "layers": cfg["n_layers"], "d_model": d,
+                   "params": M},
+        "tokens_per_s": tokens_per_step * args.steps / total_s,
+        "forward_ms": fwd_ms,
+        "forwards_per_step": fwds,
+        "roofline": {"kernel": "gemm_bf16_kernel (tcgen05, 4 projections of one layer)",
+                     "bound": "tensor", "achieved": gemm_tflops, "peak": peak_b,
+                     "unit": "TFLOP/s", "frac": gemm_tflops / peak_b, "peak_kind": peak_kind,
+                     "flops_per_layer": flops_layer, "traffic": None},
+        "gemm": gemm,
+        "memory": {"peak_allocated_GB": peak_mem / 1e9, "device_used_GB": (tot_b - free_b) / 1e9},
+        "clocks": clocks,
+    }
+    model.close()
+    ctx.close()
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -305,11 +464,16 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per launch of the loss kernel, if measured")
+    ap.add_argument("--workload", default="quadratic",
+                    choices=["quadratic"] + sorted(DECODER_WORKLOADS))
+    ap.add_argument("--n-pert", type=int, default=None, help="override n_pert (decoder workloads)")
     args = ap.parse_args()
-    if args.warmup < 3:
+    if args.warmup < 3 and args.workload == "quadratic":
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return reference_arm(args)
+    if args.workload != "quadratic":
+        return decoder_arm(args)
     return gpu_arm(args)
 
 

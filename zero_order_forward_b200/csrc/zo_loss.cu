@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "zo_internal.cuh"
+#include "zo_tc.cuh"
 
 namespace zo {
 namespace {
@@ -60,54 +61,125 @@ __device__ void finish_reduction(double v, double *partials, unsigned int *count
 }
 
 // L = 1/2 sum_j D_j P_j^2 with P_j = rd(theta_j + s*eps*z_j) computed on load.
-__global__ void __launch_bounds__(kWarps * 32)
+//
+// A persistent producer/consumer pipeline: warp 0 streams 2048-element chunks of theta and
+// D into a ring of shared-memory stages with bulk asynchronous copies (one mbarrier per
+// stage), and its first 16 lanes compute the chunk's 16 Philox blocks into the stage; the
+// 8 consumer warps apply the perturbation and accumulate in fp64, then release the stage.
+// Chunks are assigned round-robin (chunk = blockIdx.x + k * gridDim.x), so the grid size
+// and every summation order depend on M only: the result is deterministic.
+constexpr int kQChunk = 2048;
+constexpr int kQStages = 6;
+constexpr int kQConsumers = 8;
+constexpr int kQThreads = 32 * (1 + kQConsumers);
+constexpr int kQStageBytes = 2 * kQChunk * 4 + 16 * 16;  // theta, D, 16 Philox blocks
+constexpr int kQSmemBytes = kQStages * kQStageBytes + 2 * kQStages * 8;
+
+__global__ void __launch_bounds__(kQThreads)
 quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, int64_t M,
-                 ProbeKey pk, int64_t n_tiles, double *partials, unsigned int *counter,
-                 double *out, int accumulate) {
-  constexpr int N = 4;
-  constexpr int kIters = kTileElems / (32 * N);
-  __shared__ uint4 blocks[kWarps][kTileGroups];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+                 ProbeKey pk, int64_t n_chunks, double *partials, unsigned int *counter,
+                 double *out, int accumulate, uint32_t *err) {
+  extern __shared__ __align__(128) uint8_t qsm[];
+  uint64_t *full = reinterpret_cast<uint64_t *>(qsm + kQStages * kQStageBytes);
+  uint64_t *empty = full + kQStages;
+  __shared__ volatile int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kQStages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], kQConsumers);
+    }
+    abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  __syncthreads();
   const uint32_t step = pk.sign ? *pk.step : 0u;
   const float delta = pk.sign > 0 ? pk.eps : -pk.eps;
-  const uint32_t *bw = reinterpret_cast<const uint32_t *>(blocks[warp]);
   double acc = 0.0;
 
-  for (int64_t tile = (int64_t)blockIdx.x * kWarps + warp; tile < n_tiles;
-       tile += (int64_t)gridDim.x * kWarps) {
-    const int64_t base = tile * kTileElems;
-    if (pk.sign) {
-      const int64_t g = tile * kTileGroups + lane;
-      if (g * kGroup < M) blocks[warp][lane] = probe_block(g, pk.probe, step, pk.k0, pk.k1);
+  if (warp == 0) {  // producer
+    int it = 0, issued = 0;
+    for (int64_t chunk = blockIdx.x; chunk < n_chunks; chunk += gridDim.x, ++it) {
+      const int s = it % kQStages;
+      const uint32_t ph = (uint32_t)(it / kQStages) & 1u;
+      int ok = 1;
+      if (lane == 0) ok = tc::mbar_wait(&empty[s], ph ^ 1u) ? 1 : 0;
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok || abort_flag) {
+        if (lane == 0) { atomicOr(err, ZO_FLAG_TIMEOUT); abort_flag = 1; }
+        break;
+      }
+      uint8_t *st = qsm + s * kQStageBytes;
+      const int64_t base = chunk * kQChunk;
+      const int cnt = (int)(M - base < (int64_t)kQChunk ? M - base : (int64_t)kQChunk);
+      const int copy = cnt & ~3;
+      if (pk.sign && lane < 16 && (int64_t)lane * kGroup < cnt)
+        reinterpret_cast<uint4 *>(st + 2 * kQChunk * 4)[lane] =
+            probe_block((uint64_t)(base / kGroup) + lane, pk.probe, step, pk.k0, pk.k1);
       __syncwarp();
+      if (lane == 0) {
+        tc::mbar_arrive_expect_tx(&full[s], 2u * (uint32_t)copy * 4u);
+        if (copy) {
+          tc::bulk_load(st, theta + base, (uint32_t)copy * 4u, &full[s]);
+          tc::bulk_load(st + kQChunk * 4, D + base, (uint32_t)copy * 4u, &full[s]);
+        }
+      }
+      issued = it + 1;
     }
-#pragma unroll 4
-    for (int k = 0; k < kIters; ++k) {
-      const int e_rel = (k * 32 + lane) * N;
-      const int64_t e = base + e_rel;
-      uint32_t bits = 0;
-      if (pk.sign) bits = bw[(e_rel >> 7) * 4 + ((e_rel >> 5) & 3)] >> (e_rel & 31);
-      if (e + N <= M) {
-        const float4 t = __ldcs(reinterpret_cast<const float4 *>(theta + e));
-        const float4 d = __ldcs(reinterpret_cast<const float4 *>(D + e));
-        const float tv[4] = {t.x, t.y, t.z, t.w}, dv[4] = {d.x, d.y, d.z, d.w};
+    if (abort_flag && lane == 0) {  // let this CTA's copies land before it exits
+      for (int s = 0; s < kQStages; ++s) {
+        int last = -1;
+        for (int i = s; i < issued; i += kQStages) last = i;
+        if (last >= 0) tc::mbar_wait(&full[s], (uint32_t)(last / kQStages) & 1u);
+      }
+    }
+  } else {  // consumers
+    const int ct = threadIdx.x - 32;  // 0 .. 255
+    int it = 0;
+    for (int64_t chunk = blockIdx.x; chunk < n_chunks; chunk += gridDim.x, ++it) {
+      const int s = it % kQStages;
+      const uint32_t ph = (uint32_t)(it / kQStages) & 1u;
+      if (abort_flag || !tc::mbar_wait(&full[s], ph)) {
+        atomicOr(err, ZO_FLAG_TIMEOUT);
+        abort_flag = 1;
+        break;
+      }
+      const uint8_t *st = qsm + s * kQStageBytes;
+      const float *sT = reinterpret_cast<const float *>(st);
+      const float *sD = reinterpret_cast<const float *>(st + kQChunk * 4);
+      const uint32_t *sB = reinterpret_cast<const uint32_t *>(st + 2 * kQChunk * 4);
+      const int64_t base = chunk * kQChunk;
+      const int cnt = (int)(M - base < (int64_t)kQChunk ? M - base : (int64_t)kQChunk);
+      const int copy = cnt & ~3;
+#pragma unroll
+      for (int k = 0; k < kQChunk / (4 * 32 * kQConsumers); ++k) {
+        const int e = 4 * (ct + k * 32 * kQConsumers);
+        if (e >= cnt) continue;
+        const uint32_t bits = pk.sign ? sB[(e >> 7) * 4 + ((e >> 5) & 3)] >> (e & 31) : 0u;
+        float tv[4], dv[4];
+        if (e + 4 <= copy) {
+          const float4 t = reinterpret_cast<const float4 *>(sT)[e >> 2];
+          const float4 dd = reinterpret_cast<const float4 *>(sD)[e >> 2];
+          tv[0] = t.x; tv[1] = t.y; tv[2] = t.z; tv[3] = t.w;
+          dv[0] = dd.x; dv[1] = dd.y; dv[2] = dd.z; dv[3] = dd.w;
+        } else {  // the last < 4 elements of theta (not covered by the 16-byte copies)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const bool in = e + q < cnt;
+            tv[q] = in ? theta[base + e + q] : 0.f;
+            dv[q] = in ? D[base + e + q] : 0.f;
+          }
+        }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float p = pk.sign ? perturb_f32(tv[q], delta, (bits >> q) & 1u) : tv[q];
           const double pd = (double)p;
           acc = __dadd_rn(acc, __dmul_rn(__dmul_rn(0.5, (double)dv[q]), __dmul_rn(pd, pd)));
         }
-      } else {
-        for (int q = 0; q < N; ++q) {
-          if (e + q >= M) break;
-          const float tq = theta[e + q];
-          const float p = pk.sign ? perturb_f32(tq, delta, (bits >> q) & 1u) : tq;
-          const double pd = (double)p;
-          acc = __dadd_rn(acc, __dmul_rn(__dmul_rn(0.5, (double)D[e + q]), __dmul_rn(pd, pd)));
-        }
       }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&empty[s]);
     }
-    if (pk.sign) __syncwarp();
   }
   acc = block_sum(acc);
   finish_reduction(acc, partials, counter, out, accumulate, 1.0);
@@ -164,12 +236,18 @@ mlp_loss_kernel(const float *__restrict__ P, const float *__restrict__ X,
 
 zo_status launch_quad_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *out,
                            int accumulate, double *partials, unsigned int *counter) {
-  const int64_t n_tiles = (ctx->M + kTileElems - 1) / kTileElems;
-  int64_t blocks = (n_tiles + kWarps - 1) / kWarps;
-  if (blocks > (int64_t)kSmCount * 4) blocks = (int64_t)kSmCount * 4;
-  quad_loss_kernel<<<(unsigned)blocks, kWarps * 32, 0, ctx->stream>>>(
-      static_cast<const float *>(ctx->params), D, ctx->M, pk, n_tiles, partials, counter, out,
-      accumulate);
+  const int64_t n_chunks = (ctx->M + kQChunk - 1) / kQChunk;
+  int64_t blocks = n_chunks < (int64_t)kSmCount * 2 ? n_chunks : (int64_t)kSmCount * 2;
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e = cudaFuncSetAttribute(quad_loss_kernel,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes);
+    if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "quad_loss_kernel attribute: %s", cudaGetErrorString(e));
+    attr = true;
+  }
+  quad_loss_kernel<<<(unsigned)blocks, kQThreads, kQSmemBytes, ctx->stream>>>(
+      static_cast<const float *>(ctx->params), D, ctx->M, pk, n_chunks, partials, counter, out,
+      accumulate, &ctx->dstate->flags);
   return check_launch(ctx, "quad_loss_kernel");
 }
 
