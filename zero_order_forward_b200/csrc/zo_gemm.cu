@@ -3,15 +3,16 @@
 // A (activations) and B (weights, nn.Linear layout) are both K-major.  This is the only
 // dense contraction on the path (the decoder's QKV, output, FC1 and FC2 projections).
 //
-// Design (one 128 x BN output tile per CTA, 192 threads):
+// Design (persistent, one CTA of 192 threads per SM, 128 x BN output tiles):
 //   warp 0     one lane issues TMA tile loads (128-byte swizzle) into a STAGES-deep ring
 //              of shared-memory stages, paced by "empty" mbarriers;
-//   warp 1     allocates BN TMEM columns; one lane issues tcgen05.mma (M=128, N=BN,
-//              K=16, bf16 x bf16 -> fp32 in TMEM) and commits each stage back to its
-//              "empty" barrier, then commits the finished accumulator;
+//   warp 1     allocates 2*BN TMEM columns (two accumulators); one lane issues
+//              tcgen05.mma (M=128, N=BN, K=16, bf16 x bf16 -> fp32 in TMEM), commits each
+//              stage back to its "empty" barrier and each finished accumulator to the
+//              epilogue;
 //   warps 2-5  the epilogue: tcgen05.ld 32 columns at a time (warp w reads TMEM lanes
 //              32*(w%4)..+31 = its 32 output rows), adds the bias, applies ReLU or the
-//              fp32 residual add, and stores.
+//              fp32 residual add, stores, and hands the accumulator back.
 // Tiles are visited in groups of kGroupM row tiles so that the weight tiles of a group are
 // reused from L2.  All waits are bounded (see zo_tc.cuh); a timeout sets an error bit.
 #include <cudaTypedefs.h>
@@ -116,6 +117,25 @@ struct GemmSmem {
   static constexpr uint32_t kBytes = kBarOffset + 256 + 1024;  // + barriers + alignment slack
 };
 
+struct TileCoord {
+  int m0, n0;
+};
+
+// Grouped order: kGroupM row tiles share each sweep over the column tiles, so a group's
+// weight tiles are reused from L2.
+__device__ __forceinline__ TileCoord tile_coord(int t, int num_m, int num_n, int BN) {
+  const int group = t / (kGroupM * num_n);
+  const int first_m = group * kGroupM;
+  const int gsize = min(num_m - first_m, kGroupM);
+  const int m_tile = first_m + (t % gsize);
+  const int n_tile = (t % (kGroupM * num_n)) / gsize;
+  return {m_tile * kBM, n_tile * BN};
+}
+
+// Persistent: one CTA per SM walks tiles t = blockIdx.x, blockIdx.x + gridDim.x, ...
+// The shared-memory ring runs across tile boundaries, and the accumulator is
+// double-buffered in TMEM (2 x BN columns) so the epilogue of tile i overlaps the
+// main loop of tile i+1.
 template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(192, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -128,20 +148,15 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   uint8_t *sB = smem + STAGES * S::kABytes;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + S::kBarOffset);
   uint64_t *empty = full + STAGES;
-  uint64_t *done = empty + STAGES;
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(done + 1);
+  uint64_t *acc_full = empty + STAGES;   // [2] MMA -> epilogue
+  uint64_t *acc_empty = acc_full + 2;    // [2] epilogue -> MMA
+  uint64_t *mma_done = acc_empty + 2;    // all MMAs of this CTA retired
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // grouped tile order: kGroupM row tiles share each sweep over the column tiles
   const int num_m = (args.M + kBM - 1) / kBM, num_n = (args.N + BN - 1) / BN;
-  const int pid = blockIdx.x;
-  const int group = pid / (kGroupM * num_n);
-  const int first_m = group * kGroupM;
-  const int gsize = min(num_m - first_m, kGroupM);
-  const int m_tile = first_m + (pid % gsize);
-  const int n_tile = (pid % (kGroupM * num_n)) / gsize;
-  const int m0 = m_tile * kBM, n0 = n_tile * BN;
+  const int num_tiles = num_m * num_n;
   const int nk = (args.K + kBK - 1) / kBK;
 
   if (threadIdx.x == 0) {
@@ -149,85 +164,116 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       tc::mbar_init(&full[s], 1);
       tc::mbar_init(&empty[s], 1);
     }
-    tc::mbar_init(done, 1);
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&acc_full[b], 1);
+      tc::mbar_init(&acc_empty[b], 4);  // one arrival per epilogue warp
+    }
+    tc::mbar_init(mma_done, 1);
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
-  if (warp == 1) tc::tmem_alloc(tmem_holder, BN);
+  if (warp == 1) tc::tmem_alloc(tmem_holder, 2 * BN);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  int issued = 0;
+  uint32_t issued = 0;  // producer: k-blocks issued (global ring position)
   if (warp == 0 && lane == 0) {
     tc::tma_prefetch_desc(&tmA);
     tc::tma_prefetch_desc(&tmB);
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-      if (*abort_flag || !tc::mbar_wait(&empty[s], ph ^ 1u)) {
-        atomicOr(args.err, ZO_FLAG_TIMEOUT);
-        *abort_flag = 1;
-        break;
+    for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+      const TileCoord tc0 = tile_coord(t, num_m, num_n, BN);
+      for (int kb = 0; kb < nk; ++kb) {
+        const uint32_t s = issued % STAGES, ph = (issued / STAGES) & 1u;
+        if (*abort_flag || !tc::mbar_wait(&empty[s], ph ^ 1u)) {
+          atomicOr(args.err, ZO_FLAG_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
+        tc::mbar_arrive_expect_tx(&full[s], S::kStageBytes);
+        tc::tma_load_2d(sA + s * S::kABytes, &tmA, &full[s], kb * kBK, tc0.m0);
+        tc::tma_load_2d(sB + s * S::kBBytes, &tmB, &full[s], kb * kBK, tc0.n0);
+        ++issued;
       }
-      tc::mbar_arrive_expect_tx(&full[s], S::kStageBytes);
-      tc::tma_load_2d(sA + s * S::kABytes, &tmA, &full[s], kb * kBK, m0);
-      tc::tma_load_2d(sB + s * S::kBBytes, &tmB, &full[s], kb * kBK, n0);
-      issued = kb + 1;
     }
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc = tc::idesc_bf16_f32(kBM, BN);
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-      if (*abort_flag || !tc::mbar_wait(&full[s], ph)) {
+    uint32_t consumed = 0;
+    int i = 0;
+    for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x, ++i) {
+      const int b = i & 1;
+      const uint32_t aph = (uint32_t)(i >> 1) & 1u;
+      if (!tc::mbar_wait(&acc_empty[b], aph ^ 1u)) {
         atomicOr(args.err, ZO_FLAG_TIMEOUT);
         *abort_flag = 1;
         break;
       }
       tc::tc_fence_after();
-      const uint32_t a0 = tc::smem_addr(sA + s * S::kABytes);
-      const uint32_t b0 = tc::smem_addr(sB + s * S::kBBytes);
+      const uint32_t d = tmem + (uint32_t)(b * BN);
+      for (int kb = 0; kb < nk; ++kb) {
+        const uint32_t s = consumed % STAGES, ph = (consumed / STAGES) & 1u;
+        if (*abort_flag || !tc::mbar_wait(&full[s], ph)) {
+          atomicOr(args.err, ZO_FLAG_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
+        tc::tc_fence_after();
+        const uint32_t a0 = tc::smem_addr(sA + s * S::kABytes);
+        const uint32_t b0 = tc::smem_addr(sB + s * S::kBBytes);
 #pragma unroll
-      for (int k = 0; k < kBK / 16; ++k)
-        tc::mma_bf16(tmem, tc::smem_desc_k128(a0 + 32 * k), tc::smem_desc_k128(b0 + 32 * k), idesc,
-                     (kb | k) != 0 ? 1u : 0u);
-      tc::mma_commit(&empty[s]);
+        for (int k = 0; k < kBK / 16; ++k)
+          tc::mma_bf16(d, tc::smem_desc_k128(a0 + 32 * k), tc::smem_desc_k128(b0 + 32 * k), idesc,
+                       (kb | k) != 0 ? 1u : 0u);
+        tc::mma_commit(&empty[s]);
+        ++consumed;
+      }
+      if (*abort_flag) break;
+      tc::mma_commit(&acc_full[b]);
     }
-    tc::mma_commit(done);  // also covers an aborted loop: waits for the MMAs issued so far
+    tc::mma_commit(mma_done);  // arrives once every MMA issued above has retired
   } else if (warp >= 2) {
     const int q = warp & 3;
-    const bool ok = tc::mbar_wait(done, 0);
-    if (!ok) atomicOr(args.err, ZO_FLAG_TIMEOUT);
-    tc::tc_fence_after();
-    if (ok && !*abort_flag) {
-      const int row = m0 + q * 32 + lane;
+    int i = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++i) {
+      const int b = i & 1;
+      const uint32_t aph = (uint32_t)(i >> 1) & 1u;
+      if (*abort_flag || !tc::mbar_wait(&acc_full[b], aph)) {
+        if (lane == 0) atomicOr(args.err, ZO_FLAG_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      tc::tc_fence_after();
+      const TileCoord tc0 = tile_coord(t, num_m, num_n, BN);
+      const int row = tc0.m0 + q * 32 + lane;
+      const uint32_t base = tmem + (uint32_t)(b * BN) + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
-        if (n0 + c0 >= args.N) break;
+        if (tc0.n0 + c0 >= args.N) break;
         float v[32];
-        tc::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
-        if (row < args.M) epilogue_store<EPI>(v, row, n0 + c0, args);
+        tc::tmem_ld32(base + (uint32_t)c0, v);
+        if (row < args.M) epilogue_store<EPI>(v, row, tc0.n0 + c0, args);
       }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&acc_empty[b]);
     }
   }
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 0 && lane == 0 && *abort_flag) {
-    // wait (bounded) for this CTA's TMA loads still in flight before the CTA exits
-    for (int s = 0; s < STAGES; ++s) {
-      int last = -1;
-      for (int kb = s; kb < issued; kb += STAGES) last = kb;
-      if (last >= 0 && !tc::mbar_wait(&full[s], (uint32_t)(last / STAGES) & 1u))
-        atomicOr(args.err, ZO_FLAG_TIMEOUT);
+    // let this CTA's TMA loads still in flight land before it exits (bounded)
+    for (uint32_t s = 0; s < STAGES; ++s) {
+      if (issued <= s) continue;
+      const uint32_t last = s + ((issued - 1 - s) / STAGES) * STAGES;
+      if (!tc::mbar_wait(&full[s], (last / STAGES) & 1u)) atomicOr(args.err, ZO_FLAG_TIMEOUT);
     }
   }
   if (warp == 1) {
-    if (lane == 0 && *abort_flag && !tc::mbar_wait(done, 0)) atomicOr(args.err, ZO_FLAG_TIMEOUT);
+    if (lane == 0 && !tc::mbar_wait(mma_done, 0)) atomicOr(args.err, ZO_FLAG_TIMEOUT);
     __syncwarp();
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem, BN);
+    tc::tmem_dealloc(tmem, 2 * BN);
   }
 }
 
@@ -273,7 +319,8 @@ cudaError_t launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const GemmA
     attr_set = true;
   }
   const int num_m = (g.M + kBM - 1) / kBM, num_n = (g.N + BN - 1) / BN;
-  kern<<<num_m * num_n, 192, S::kBytes, st>>>(ta, tb, g);
+  const int tiles = num_m * num_n;
+  kern<<<tiles < kSmCount ? tiles : kSmCount, 192, S::kBytes, st>>>(ta, tb, g);
   return cudaGetLastError();
 }
 
