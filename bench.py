@@ -13,10 +13,11 @@ The decoder workloads (OPT-shaped, bf16 weights N(0, 0.02), uniform tokens, 2-cl
 last-token loss) time whole 1.5-SPSA steps through zo_model_step and add a per-GEMM-shape
 breakdown of the tcgen05 projections against the measured bf16 peak.
 
-Prints ONE JSON line (rank 0).  With N > 1 (torchrun, one rank per GPU) every rank runs
-its own replica of the workload (independent problems, no collective on the data path);
-`value` is the sum over ranks of steps/s, timed as the max over ranks.  `--impl
-reference` times the CPU oracle on a bounded slice of the same workload.
+Prints ONE JSON line (rank 0).  With N > 1 (torchrun, one rank per GPU) the ranks share
+one model: every rank holds theta, evaluates its share of the probes (i = rank mod N), the
+2*n_pert fp64 losses are all-gathered over NCCL, and every rank applies the identical
+update ("scaling": "strong"); the step time is the max over ranks.  `--impl reference`
+times the CPU oracle on a bounded slice of the same workload.
 """
 import argparse
 import json
@@ -102,7 +103,7 @@ def reference_arm(args):
               f"{args.steps} timed steps after {args.warmup} warm-up; steps/s scaled by 1/64")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1e3 / value, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": 1e3 / value, "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "M": M_FULL, "n_pert": N_PERT},
             "cpu_baseline": {"value": value, "unit": "steps/s", "cores": 1, "kind": "oracle",
@@ -177,17 +178,35 @@ def gpu_arm(args):
     dev = torch.device("cuda", local_rank)
     hbm_peak, peak_kind = peaks()
 
-    th_np, D_np = synth.quad_problem(M_FULL, seed=rank)
+    th_np, D_np = synth.quad_problem(M_FULL, seed=0)  # one shared model across ranks
     theta = torch.from_numpy(th_np).to(dev)
     D = torch.from_numpy(D_np).to(dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     n = N_PERT
     losses = torch.zeros(2 * n + 1, dtype=torch.float64, device=dev)
     stream = torch.cuda.current_stream(dev)
-    ctx = zo.zo_create(theta, seed=rank, stream=stream.cuda_stream)
+    ctx = zo.zo_create(theta, seed=0, stream=stream.cuda_stream)
+
+    def loss_at(sign, probe, out):
+        zo.zo_perturb(ctx, sign, EPS, probe)
+        zo.zo_quad_loss(ctx, D, out)
+        zo.zo_restore(ctx)
+
+    def apply_step(Lp, Lm, L0):
+        zo.zo_step(ctx, Lp, Lm, n, L0, LR, EPS, DAMPING)
 
     def one_step(ev=None):
         """Step through the C ABI primitives; ev = 4 events at the phase boundaries."""
+        if world > 1:  # probe-parallel: this rank's probes, loss all-gather, same update
+            from zero_order_forward_b200 import dist as zdist
+            if ev:
+                ev[0].record(stream)
+            zdist.probe_parallel_step(n, loss_at, lambda o: zo.zo_quad_loss(ctx, D, o),
+                                      apply_step, dev)
+            if ev:
+                for e in ev[1:]:
+                    e.record(stream)
+            return
         if ev:
             ev[0].record(stream)
         zo.zo_quad_loss(ctx, D, losses[0:1])
@@ -231,9 +250,19 @@ def gpu_arm(args):
         t = torch.tensor([total_s], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_s = float(t.item())
-    value = world * args.steps / total_s
+    value = args.steps / total_s  # steps of the one shared model
 
     # dominant kernel: the loss pass (perturbation on load); 2n launches per probe phase
+    # (with N ranks the probe phase is not bracketed separately: time the kernel alone)
+    if world > 1:
+        le = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        flush.zero_()
+        le[0].record(stream)
+        for i in range(2 * n):
+            zo.zo_quad_loss(ctx, D, losses[0:1])
+        le[1].record(stream)
+        torch.cuda.synchronize()
+        probe_ms = [le[0].elapsed_time(le[1])]
     loss_us = 1e3 * statistics.mean(probe_ms) / (2 * n)
     loss_bytes = 8 * M_FULL  # theta and D read once, fp32
     achieved = loss_bytes / (loss_us * 1e-6) / 1e9
@@ -251,23 +280,34 @@ def gpu_arm(args):
     torch.cuda.synchronize()
     upd_us = 1e3 * ue[0].elapsed_time(ue[1]) / reps
 
-    # end to end through the host-buffer entry point: D copied in, losses copied out
+    # end to end through the public API with host buffers: D copied in, losses copied out
     D_host = torch.from_numpy(D_np).pin_memory()
     L_host = torch.zeros(2 * n + 1, dtype=torch.float64).pin_memory()
-    zo.zo_quad_step_host(ctx, D_host, n, EPS, LR, DAMPING, True, L_host)  # staging alloc
     e2e_steps = max(3, min(args.steps, 10))
+
+    def e2e_step():
+        if world == 1:
+            zo.zo_quad_step_host(ctx, D_host, n, EPS, LR, DAMPING, True, L_host)
+            return
+        D.copy_(D_host, non_blocking=True)
+        from zero_order_forward_b200 import dist as zdist
+        L0, Lp, Lm = zdist.probe_parallel_step(n, loss_at, lambda o: zo.zo_quad_loss(ctx, D, o),
+                                               apply_step, dev)
+        L_host.copy_(torch.cat([L0, Lp, Lm]))  # synchronous device -> host read
+    e2e_step()  # staging allocation
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     for _ in range(e2e_steps):
-        zo.zo_quad_step_host(ctx, D_host, n, EPS, LR, DAMPING, True, L_host)
+        e2e_step()
+    torch.cuda.synchronize()
     e2e_s = time.perf_counter() - t0
     if world > 1:
         t = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_s = float(t.item())
-    e2e_value = world * e2e_steps / e2e_s
+    e2e_value = e2e_steps / e2e_s
 
     line = None
     if rank == 0:
@@ -279,14 +319,14 @@ def gpu_arm(args):
             cpu = {"value": (M_sample / M_FULL) / per, "unit": "steps/s", "cores": 1,
                    "kind": "oracle",
                    "sample": "2 oracle steps on the first 2^20 of 2^24 parameters; steps/s scaled by 1/16"}
-        launches_per_step = 1 + 2 * n + 2
+        launches_per_step = 1 + 2 * len(range(rank, n, world)) + 2
         line = {
             "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "M": M_FULL, "n_pert": n, "eps": EPS, "lr": LR,
-                       "damping": DAMPING, "parallelism": f"replicas{world}",
+                       "damping": DAMPING, "parallelism": f"probe-parallel x{world}",
                        "l2": "flushed between steps (256 MiB write, untimed); theta+D = 128 MiB"},
             "roofline": {"kernel": "quad_loss_kernel (perturbation on load, fp64 accumulation)",
                          "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
@@ -303,9 +343,10 @@ def gpu_arm(args):
                           "precond_update": statistics.mean(upd_ms)},
             "tokens_per_s": None,
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": 4 * M_FULL,
-                    "d2h_bytes_per_step": 8 * (2 * n + 1),
-                    "path": "zo_quad_step_host: D pinned host -> device each step, losses back"},
+            "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": 4 * M_FULL * world,
+                    "d2h_bytes_per_step": 8 * (2 * n + 1) * world,
+                    "path": "D pinned host -> device every step on every rank, losses back "
+                            "(zo_quad_step_host at one GPU)"},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
         }

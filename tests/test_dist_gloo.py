@@ -1,0 +1,83 @@
+"""Host-side logic of the probe-parallel step on 2 and 3 CPU ranks (gloo): the probe
+partition, the loss exchange and bit-identical replicas.  The per-probe loss and the update
+are the oracle's here (CPU); on GPUs the same driver calls the CUDA library over NCCL."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+from zero_order_forward_b200 import dist as zdist
+
+
+def test_partition_covers_every_probe_once():
+    for n in (1, 2, 5, 16, 64, 161):
+        for world in (1, 2, 3, 8):
+            seen = sorted(i for r in range(world) for i in zdist.rank_probes(n, r, world))
+            assert seen == list(range(n))
+            idx = zdist.global_order(n, world)
+            assert idx.shape == (world, zdist.slots(n, world))
+            assert sorted(idx[idx >= 0].tolist()) == list(range(n))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+M, N_PERT, EPS, LR, LAM, SEED = 3000, 7, 1e-3, 1e-5, 1e-3, 5
+
+
+def _worker(rank, world, port, out_dir):
+    import torch.distributed as dist
+
+    import oracle
+    import synth
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        theta, D = synth.quad_problem(M, seed=1)
+        state = {"theta": theta}
+        e32 = float(np.float32(EPS))
+
+        def loss_at(sign, probe, out):
+            P = oracle.core.perturb(state["theta"], SEED, 0, probe, sign, e32)
+            out[0] = oracle.core.quad_loss(P, D)
+
+        def clean(out):
+            out[0] = oracle.core.quad_loss(state["theta"], D)
+
+        def apply_step(Lp, Lm, L0):
+            pc = oracle.core.precond(Lp.numpy(), Lm.numpy(), float(L0[0]), e32,
+                                     float(np.float32(LR)), float(np.float32(LAM)),
+                                     float(np.float32(0.1)))
+            state["theta"] = oracle.core.update_mirror(state["theta"], pc["a"].astype(np.float32),
+                                                       SEED, 0)
+
+        L0, Lp, Lm = zdist.probe_parallel_step(N_PERT, loss_at, clean, apply_step, "cpu")
+        np.savez(os.path.join(out_dir, f"r{rank}.npz"), theta=state["theta"], L0=L0.numpy(),
+                 Lp=Lp.numpy(), Lm=Lm.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_probe_parallel_step_matches_single_rank(tmp_path, world):
+    import oracle
+    import synth
+    mp.start_processes(_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    theta, D = synth.quad_problem(M, seed=1)
+    nxt, rec = oracle.step.spsa_step(theta, lambda P: oracle.core.quad_loss(P, D), N_PERT, EPS,
+                                     LR, LAM, SEED, 0, update="mirror")
+    outs = [np.load(tmp_path / f"r{r}.npz") for r in range(world)]
+    for o in outs:
+        assert np.array_equal(o["Lp"], rec["Lp"]) and np.array_equal(o["Lm"], rec["Lm"])
+        assert o["L0"][0] == rec["L0"]
+        assert o["theta"].tobytes() == nxt.tobytes()  # bit-identical replicas

@@ -3,16 +3,17 @@
 // A (activations) and B (weights, nn.Linear layout) are both K-major.  This is the only
 // dense contraction on the path (the decoder's QKV, output, FC1 and FC2 projections).
 //
-// Design (persistent, one CTA of 192 threads per SM, 128 x BN output tiles):
+// Design (persistent, one CTA of 320 threads per SM, 128 x BN output tiles):
 //   warp 0     one lane issues TMA tile loads (128-byte swizzle) into a STAGES-deep ring
 //              of shared-memory stages, paced by "empty" mbarriers;
 //   warp 1     allocates 2*BN TMEM columns (two accumulators); one lane issues
 //              tcgen05.mma (M=128, N=BN, K=16, bf16 x bf16 -> fp32 in TMEM), commits each
 //              stage back to its "empty" barrier and each finished accumulator to the
 //              epilogue;
-//   warps 2-5  the epilogue: tcgen05.ld 32 columns at a time (warp w reads TMEM lanes
-//              32*(w%4)..+31 = its 32 output rows), adds the bias, applies ReLU or the
-//              fp32 residual add, stores, and hands the accumulator back.
+//   warps 2-9  the epilogue, two warps per TMEM lane quadrant (warp w reads TMEM lanes
+//              32*(w%4)..+31 = its 32 output rows, half of the columns each): tcgen05.ld
+//              32 columns at a time, bias, ReLU or the fp32 residual add (residual loaded
+//              before the TMEM read), store, and hand the accumulator back.
 // Tiles are visited in groups of kGroupM row tiles so that the weight tiles of a group are
 // reused from L2.  All waits are bounded (see zo_tc.cuh); a timeout sets an error bit.
 #include <cudaTypedefs.h>
@@ -60,9 +61,20 @@ __device__ __forceinline__ void load_bias32(const uint16_t *bias, int col0, int 
   }
 }
 
+// Residual values of a full 32-column chunk, loaded before the accumulator is read so
+// that the global-load latency overlaps the TMEM load.
+__device__ __forceinline__ void load_resid32(const GemmArgs &a, int row, int col0, float4 h[8]) {
+  if (row < a.M && col0 + 32 <= a.N) {
+    const float4 *o = reinterpret_cast<const float4 *>(static_cast<const float *>(a.out) +
+                                                       (int64_t)row * a.ldo + col0);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) h[k] = o[k];
+  }
+}
+
 template <int EPI>
 __device__ __forceinline__ void epilogue_store(const float acc[32], int row, int col0,
-                                               const GemmArgs &a) {
+                                               const GemmArgs &a, const float4 hpre[8]) {
   float b[32];
   load_bias32(a.bias, col0, a.N, b);
   if (EPI == ZO_EPI_RESID_F32) {
@@ -70,7 +82,7 @@ __device__ __forceinline__ void epilogue_store(const float acc[32], int row, int
     if (col0 + 32 <= a.N) {
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        float4 h = reinterpret_cast<float4 *>(o)[k];
+        float4 h = hpre[k];
         h.x = __fadd_rn(h.x, __fadd_rn(acc[4 * k], b[4 * k]));
         h.y = __fadd_rn(h.y, __fadd_rn(acc[4 * k + 1], b[4 * k + 1]));
         h.z = __fadd_rn(h.z, __fadd_rn(acc[4 * k + 2], b[4 * k + 2]));
@@ -136,8 +148,11 @@ __device__ __forceinline__ TileCoord tile_coord(int t, int num_m, int num_n, int
 // The shared-memory ring runs across tile boundaries, and the accumulator is
 // double-buffered in TMEM (2 x BN columns) so the epilogue of tile i overlaps the
 // main loop of tile i+1.
+constexpr int kEpiWarps = 8;                      // two warps per TMEM lane quadrant
+constexpr int kGemmThreads = 32 * (2 + kEpiWarps);  // producer, MMA, epilogue
+
 template <int BN, int STAGES, int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  GemmArgs args) {
   using S = GemmSmem<BN, STAGES>;
@@ -166,7 +181,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&acc_full[b], 1);
-      tc::mbar_init(&acc_empty[b], 4);  // one arrival per epilogue warp
+      tc::mbar_init(&acc_empty[b], kEpiWarps);  // one arrival per epilogue warp
     }
     tc::mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -233,7 +248,9 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
     tc::mma_commit(mma_done);  // arrives once every MMA issued above has retired
   } else if (warp >= 2) {
-    const int q = warp & 3;
+    const int q = warp & 3;                    // TMEM lanes 32q..32q+31 (this warp's rows)
+    const int half = (warp - 2) / 4;           // which half of the BN columns
+    const int cbeg = half * (BN / 2), cend = cbeg + BN / 2;
     int i = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++i) {
       const int b = i & 1;
@@ -248,11 +265,13 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const int row = tc0.m0 + q * 32 + lane;
       const uint32_t base = tmem + (uint32_t)(b * BN) + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int c0 = cbeg; c0 < cend; c0 += 32) {
         if (tc0.n0 + c0 >= args.N) break;
+        float4 hpre[8];
+        if (EPI == ZO_EPI_RESID_F32) load_resid32(args, row, tc0.n0 + c0, hpre);
         float v[32];
         tc::tmem_ld32(base + (uint32_t)c0, v);
-        if (row < args.M) epilogue_store<EPI>(v, row, tc0.n0 + c0, args);
+        if (row < args.M) epilogue_store<EPI>(v, row, tc0.n0 + c0, args, hpre);
       }
       tc::tc_fence_before();
       __syncwarp();
@@ -320,7 +339,7 @@ cudaError_t launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const GemmA
   }
   const int num_m = (g.M + kBM - 1) / kBM, num_n = (g.N + BN - 1) / BN;
   const int tiles = num_m * num_n;
-  kern<<<tiles < kSmCount ? tiles : kSmCount, 192, S::kBytes, st>>>(ta, tb, g);
+  kern<<<tiles < kSmCount ? tiles : kSmCount, kGemmThreads, S::kBytes, st>>>(ta, tb, g);
   return cudaGetLastError();
 }
 
