@@ -359,7 +359,7 @@ zo_status zo_attention(zo_ctx *ctx, const void *qkv, void *out, int32_t batch, i
                        int32_t n_heads, int32_t d_model);
 
 /* out bf16 [rows][d] = LayerNorm(x fp32 [rows][d]) * gamma + beta (bf16 [d]), eps 1e-5,
- * d <= 8192. */
+ * d <= 8192, d % 8 == 0, pointers 16-byte aligned. */
 zo_status zo_layernorm(zo_ctx *ctx, const float *x, const void *gamma, const void *beta,
                        void *out, int32_t rows, int32_t d);
 

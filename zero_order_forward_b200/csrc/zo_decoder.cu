@@ -126,40 +126,68 @@ __device__ __forceinline__ float block_allreduce_sum(float v, float *red) {
   return s;
 }
 
-// xn = bf16(LayerNorm(x) * g + b), eps 1e-5, one block per row, two passes in fp32.
-constexpr int kMaxPerThread = 32;  // d <= 8192
+// xn = bf16(LayerNorm(x) * g + b), eps 1e-5, two passes in fp32 over registers.
+// One block per row; each thread owns 8 consecutive columns (two 16-byte loads), so a
+// block has ceil(d/8) threads rounded up to a warp (d <= 8192).
+constexpr int kLnVec = 8;
+constexpr int kLnMaxThreads = 1024;
 
-__global__ void __launch_bounds__(kRowThreads)
+__device__ __forceinline__ float ln_block_sum(float v, float *red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float s = 0.f;
+  for (int i = 0; i < nw; ++i) s += red[i];  // same order in every thread
+  __syncthreads();                           // red is reused by the next reduction
+  return s;
+}
+
+__global__ void __launch_bounds__(kLnMaxThreads)
 layernorm_kernel(const float *__restrict__ x, const uint16_t *__restrict__ g,
                  const uint16_t *__restrict__ b, uint16_t *__restrict__ y, int d) {
-  __shared__ float red[kRowThreads / 32];
+  __shared__ float red[kLnMaxThreads / 32];
+  const int c = threadIdx.x * kLnVec;
+  const bool on = c < d;
   const float *row = x + (int64_t)blockIdx.x * d;
-  float v[kMaxPerThread];
+  float v[kLnVec];
+  if (on) {
+    const float4 a = reinterpret_cast<const float4 *>(row + c)[0];
+    const float4 bb = reinterpret_cast<const float4 *>(row + c)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = bb.x; v[5] = bb.y; v[6] = bb.z; v[7] = bb.w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < kLnVec; ++i) v[i] = 0.f;
+  }
   float s = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxPerThread; ++i) {
-    const int c = threadIdx.x + i * kRowThreads;
-    v[i] = c < d ? row[c] : 0.f;
-    s += v[i];
-  }
-  const float mean = block_allreduce_sum(s, red) / (float)d;
+  for (int i = 0; i < kLnVec; ++i) s += v[i];
+  const float mean = ln_block_sum(s, red) / (float)d;
   float q = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxPerThread; ++i) {
-    const int c = threadIdx.x + i * kRowThreads;
-    const float u = c < d ? v[i] - mean : 0.f;
+  for (int i = 0; i < kLnVec; ++i) {
+    const float u = on ? v[i] - mean : 0.f;
     q += u * u;
   }
-  const float var = block_allreduce_sum(q, red) / (float)d;
-  const float rstd = rsqrtf(var + 1e-5f);
-  uint16_t *out = y + (int64_t)blockIdx.x * d;
+  const float rstd = rsqrtf(ln_block_sum(q, red) / (float)d + 1e-5f);
+  if (!on) return;
+  const uint4 gg = *reinterpret_cast<const uint4 *>(g + c);
+  const uint4 bv = *reinterpret_cast<const uint4 *>(b + c);
+  const uint32_t gw[4] = {gg.x, gg.y, gg.z, gg.w}, bw[4] = {bv.x, bv.y, bv.z, bv.w};
+  uint32_t o[4];
 #pragma unroll
-  for (int i = 0; i < kMaxPerThread; ++i) {
-    const int c = threadIdx.x + i * kRowThreads;
-    if (c < d)
-      out[c] = f32_to_bf16_bits((v[i] - mean) * rstd * bf16_bits_to_f32(g[c]) + bf16_bits_to_f32(b[c]));
+  for (int t = 0; t < 4; ++t) {
+    const float y0 = (v[2 * t] - mean) * rstd * __uint_as_float(gw[t] << 16) + __uint_as_float(bw[t] << 16);
+    const float y1 = (v[2 * t + 1] - mean) * rstd * __uint_as_float(gw[t] & 0xFFFF0000u) +
+                     __uint_as_float(bw[t] & 0xFFFF0000u);
+    o[t] = (uint32_t)f32_to_bf16_bits(y0) | ((uint32_t)f32_to_bf16_bits(y1) << 16);
   }
+  *reinterpret_cast<uint4 *>(y + (int64_t)blockIdx.x * d + c) = make_uint4(o[0], o[1], o[2], o[3]);
 }
+
+int ln_threads(int d) { return ((d / kLnVec + 31) / 32) * 32; }
 
 // Per sample: final LayerNorm of the last position, logits of the two class tokens through
 // the tied head, 2-class cross-entropy.  Parameters perturbed on load.
@@ -262,14 +290,14 @@ zo_status run_layers(zo_model *m, const int32_t *tokens, int B, int S, int n_run
       if (st != ZO_OK) return st;
       lp = m->window;
     }
-    layernorm_kernel<<<T, kRowThreads, 0, ctx->stream>>>(m->h, lp + L.ln1g, lp + L.ln1b, m->xn, d);
+    layernorm_kernel<<<T, ln_threads(d), 0, ctx->stream>>>(m->h, lp + L.ln1g, lp + L.ln1b, m->xn, d);
     if ((st = check_launch(ctx, "layernorm_kernel")) != ZO_OK) return st;
     if ((st = launch_gemm(ctx, m->xn, lp + L.wqkv, lp + L.bqkv, m->qkv, T, 3 * d, d, 3 * d,
                           ZO_EPI_BIAS_BF16)) != ZO_OK) return st;
     if ((st = launch_attention(ctx, m->qkv, m->attn, B, S, c.n_heads, d)) != ZO_OK) return st;
     if ((st = launch_gemm(ctx, m->attn, lp + L.wo, lp + L.bo, m->h, T, d, d, d,
                           ZO_EPI_RESID_F32)) != ZO_OK) return st;
-    layernorm_kernel<<<T, kRowThreads, 0, ctx->stream>>>(m->h, lp + L.ln2g, lp + L.ln2b, m->xn, d);
+    layernorm_kernel<<<T, ln_threads(d), 0, ctx->stream>>>(m->h, lp + L.ln2g, lp + L.ln2b, m->xn, d);
     if ((st = check_launch(ctx, "layernorm_kernel")) != ZO_OK) return st;
     if ((st = launch_gemm(ctx, m->xn, lp + L.w1, lp + L.b1, m->mid, T, f, d, f,
                           ZO_EPI_RELU_BF16)) != ZO_OK) return st;
@@ -430,9 +458,12 @@ zo_status zo_layernorm(zo_ctx *ctx, const float *x, const void *gamma, const voi
                        int32_t rows, int32_t d) {
   if (!ctx) return ZO_ERR_INVALID;
   ctx->err.clear();
-  if (!x || !gamma || !beta || !out || rows < 1 || d < 1 || d > kMaxPerThread * kRowThreads)
-    return fail(ctx, ZO_ERR_INVALID, "bad layernorm arguments");
-  layernorm_kernel<<<rows, kRowThreads, 0, ctx->stream>>>(
+  if (!x || !gamma || !beta || !out || rows < 1 || d < kLnVec || d % kLnVec ||
+      d > kLnVec * kLnMaxThreads ||
+      ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(gamma) |
+        reinterpret_cast<uintptr_t>(beta) | reinterpret_cast<uintptr_t>(out)) & 15u))
+    return fail(ctx, ZO_ERR_INVALID, "bad layernorm arguments (d %% 8 == 0, d <= 8192, 16-byte aligned)");
+  layernorm_kernel<<<rows, ln_threads(d), 0, ctx->stream>>>(
       x, static_cast<const uint16_t *>(gamma), static_cast<const uint16_t *>(beta),
       static_cast<uint16_t *>(out), d);
   return check_launch(ctx, "layernorm_kernel");

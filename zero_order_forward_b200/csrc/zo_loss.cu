@@ -63,9 +63,11 @@ __device__ void finish_reduction(double v, double *partials, unsigned int *count
 // L = 1/2 sum_j D_j P_j^2 with P_j = rd(theta_j + s*eps*z_j) computed on load.
 //
 // A persistent producer/consumer pipeline: warp 0 streams 2048-element chunks of theta and
-// D into a ring of shared-memory stages with bulk asynchronous copies (one mbarrier per
-// stage), and its first 16 lanes compute the chunk's 16 Philox blocks into the stage; the
-// 8 consumer warps apply the perturbation and accumulate in fp64, then release the stage.
+// D into a ring of shared-memory stages with bulk asynchronous copies, then its first 16
+// lanes compute the chunk's 16 Philox blocks into the stage while the copies are in flight
+// (each stage's full barrier takes two arrivals: the copies' and the blocks'); the 8
+// consumer warps apply the perturbation and accumulate in fp64 (four independent partial
+// sums per thread), then release the stage.
 // Chunks are assigned round-robin (chunk = blockIdx.x + k * gridDim.x), so the grid size
 // and every summation order depend on M only: the result is deterministic.
 constexpr int kQChunk = 2048;
@@ -86,7 +88,7 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kQStages; ++s) {
-      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&full[s], 2);
       tc::mbar_init(&empty[s], kQConsumers);
     }
     abort_flag = 0;
@@ -95,7 +97,7 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
   __syncthreads();
   const uint32_t step = pk.sign ? *pk.step : 0u;
   const float delta = pk.sign > 0 ? pk.eps : -pk.eps;
-  double acc = 0.0;
+  double acc4[4] = {0.0, 0.0, 0.0, 0.0};
 
   if (warp == 0) {  // producer
     int it = 0, issued = 0;
@@ -113,10 +115,6 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
       const int64_t base = chunk * kQChunk;
       const int cnt = (int)(M - base < (int64_t)kQChunk ? M - base : (int64_t)kQChunk);
       const int copy = cnt & ~3;
-      if (pk.sign && lane < 16 && (int64_t)lane * kGroup < cnt)
-        reinterpret_cast<uint4 *>(st + 2 * kQChunk * 4)[lane] =
-            probe_block((uint64_t)(base / kGroup) + lane, pk.probe, step, pk.k0, pk.k1);
-      __syncwarp();
       if (lane == 0) {
         tc::mbar_arrive_expect_tx(&full[s], 2u * (uint32_t)copy * 4u);
         if (copy) {
@@ -124,6 +122,11 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
           tc::bulk_load(st + kQChunk * 4, D + base, (uint32_t)copy * 4u, &full[s]);
         }
       }
+      if (pk.sign && lane < 16 && (int64_t)lane * kGroup < cnt)
+        reinterpret_cast<uint4 *>(st + 2 * kQChunk * 4)[lane] =
+            probe_block((uint64_t)(base / kGroup) + lane, pk.probe, step, pk.k0, pk.k1);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&full[s]);
       issued = it + 1;
     }
     if (abort_flag && lane == 0) {  // let this CTA's copies land before it exits
@@ -174,13 +177,14 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
         for (int q = 0; q < 4; ++q) {
           const float p = pk.sign ? perturb_f32(tv[q], delta, (bits >> q) & 1u) : tv[q];
           const double pd = (double)p;
-          acc = __dadd_rn(acc, __dmul_rn(__dmul_rn(0.5, (double)dv[q]), __dmul_rn(pd, pd)));
+          acc4[q] = __dadd_rn(acc4[q], __dmul_rn(__dmul_rn(0.5, (double)dv[q]), __dmul_rn(pd, pd)));
         }
       }
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&empty[s]);
     }
   }
+  double acc = __dadd_rn(__dadd_rn(acc4[0], acc4[1]), __dadd_rn(acc4[2], acc4[3]));
   acc = block_sum(acc);
   finish_reduction(acc, partials, counter, out, accumulate, 1.0);
 }

@@ -10,6 +10,7 @@
 #include <cstdio>
 
 #include "zo_internal.cuh"
+#include "zo_tc.cuh"
 
 namespace zo {
 namespace {
@@ -102,6 +103,131 @@ perturb_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t first, 
   }
 }
 
+// Pipelined form for 16-byte-aligned windows (first % (16 / sizeof(T)) == 0, out 16-byte
+// aligned): chunks of 32 groups (4096 elements, aligned to groups in the global index)
+// stream through a ring of shared-memory stages.  Warp 0 issues the bulk copy of a chunk
+// first and then computes its 32 Philox blocks into the stage (the stage's full barrier
+// takes two arrivals: the copy's and the blocks'); 8 consumer warps apply the perturbation
+// and write the window with 16-byte stores.
+constexpr int kPChunk = kTileElems;  // 4096
+constexpr int kPStages = 6;
+constexpr int kPConsumers = 8;
+constexpr int kPThreads = 32 * (1 + kPConsumers);
+
+template <typename T>
+struct PipeSmem {
+  static constexpr int kData = kPChunk * (int)sizeof(T);
+  static constexpr int kStage = kData + kTileGroups * 16;
+  static constexpr int kBytes = kPStages * kStage + 2 * kPStages * 8;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kPThreads)
+perturb_pipe_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t first,
+                    int64_t count, ProbeKey pk, int64_t n_chunks, uint32_t *err) {
+  using SM = PipeSmem<T>;
+  constexpr int N = Vec<T>::N;
+  extern __shared__ __align__(128) uint8_t psm[];
+  uint64_t *full = reinterpret_cast<uint64_t *>(psm + kPStages * SM::kStage);
+  uint64_t *empty = full + kPStages;
+  __shared__ volatile int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPStages; ++s) {
+      tc::mbar_init(&full[s], 2);
+      tc::mbar_init(&empty[s], kPConsumers);
+    }
+    abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  __syncthreads();
+  const int64_t end = first + count;
+  const int64_t g0 = first / kGroup;
+  const uint32_t step = pk.sign ? *pk.step : 0u;
+  const float delta = pk.sign > 0 ? pk.eps : -pk.eps;
+
+  if (warp == 0) {
+    int it = 0, issued = 0;
+    for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
+      const int s = it % kPStages;
+      const uint32_t ph = (uint32_t)(it / kPStages) & 1u;
+      int ok = 1;
+      if (lane == 0) ok = tc::mbar_wait(&empty[s], ph ^ 1u) ? 1 : 0;
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok || abort_flag) {
+        if (lane == 0) { atomicOr(err, ZO_FLAG_TIMEOUT); abort_flag = 1; }
+        break;
+      }
+      uint8_t *st = psm + s * SM::kStage;
+      const int64_t cs = (g0 + c * kTileGroups) * kGroup;
+      const int64_t vs = cs > first ? cs : first;
+      const int64_t ve = cs + kPChunk < end ? cs + kPChunk : end;
+      const int64_t copy = (ve - vs) & ~(int64_t)(N - 1);
+      if (lane == 0) {
+        tc::mbar_arrive_expect_tx(&full[s], (uint32_t)(copy * (int64_t)sizeof(T)));
+        if (copy > 0)
+          tc::bulk_load(st + (vs - cs) * (int64_t)sizeof(T), theta + vs,
+                        (uint32_t)(copy * (int64_t)sizeof(T)), &full[s]);
+      }
+      const int64_t g = g0 + c * kTileGroups + lane;
+      if (pk.sign && g * kGroup < end && (g + 1) * kGroup > first)
+        reinterpret_cast<uint4 *>(st + SM::kData)[lane] = probe_block(g, pk.probe, step, pk.k0, pk.k1);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&full[s]);
+      issued = it + 1;
+    }
+    if (abort_flag && lane == 0) {
+      for (int s = 0; s < kPStages; ++s) {
+        int last = -1;
+        for (int i = s; i < issued; i += kPStages) last = i;
+        if (last >= 0) tc::mbar_wait(&full[s], (uint32_t)(last / kPStages) & 1u);
+      }
+    }
+  } else {
+    const int ct = threadIdx.x - 32;
+    int it = 0;
+    for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
+      const int s = it % kPStages;
+      const uint32_t ph = (uint32_t)(it / kPStages) & 1u;
+      if (abort_flag || !tc::mbar_wait(&full[s], ph)) {
+        atomicOr(err, ZO_FLAG_TIMEOUT);
+        abort_flag = 1;
+        break;
+      }
+      const uint8_t *st = psm + s * SM::kStage;
+      const uint32_t *bw = reinterpret_cast<const uint32_t *>(st + SM::kData);
+      const int64_t cs = (g0 + c * kTileGroups) * kGroup;
+      const int64_t vs = cs > first ? cs : first;
+      const int64_t ve = cs + kPChunk < end ? cs + kPChunk : end;
+      const int64_t copy_end = vs + ((ve - vs) & ~(int64_t)(N - 1));
+#pragma unroll
+      for (int k = 0; k < kPChunk / (N * 32 * kPConsumers); ++k) {
+        const int e_rel = (ct + k * 32 * kPConsumers) * N;
+        const int64_t e = cs + e_rel;
+        if (e + N <= vs || e >= ve) continue;
+        const uint32_t bits = pk.sign ? bw[(e_rel >> 7) * 4 + ((e_rel >> 5) & 3)] >> (e_rel & 31) : 0u;
+        if (e >= vs && e + N <= copy_end) {
+          uint4 v = *reinterpret_cast<const uint4 *>(st + (int64_t)e_rel * (int64_t)sizeof(T));
+          if (pk.sign) v = apply_vec(v, bits, delta, (T *)nullptr);
+          *reinterpret_cast<uint4 *>(out + (e - first)) = v;
+        } else {
+#pragma unroll
+          for (int t = 0; t < N; ++t) {
+            const int64_t et = e + t;
+            if (et >= first && et < end) {
+              T v = theta[et];
+              if (pk.sign) v = apply_one(v, (bits >> t) & 1u, delta);
+              out[et - first] = v;
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&empty[s]);
+    }
+  }
+}
+
 // Packed probe bytes [first_byte, first_byte + nbytes): one thread per 16-byte group
 // block.  Bits of elements >= M are cleared.
 __global__ void pack_kernel(uint8_t *__restrict__ out, int64_t first_byte, int64_t nbytes,
@@ -125,9 +251,33 @@ __global__ void pack_kernel(uint8_t *__restrict__ out, int64_t first_byte, int64
 
 }  // namespace
 
+template <typename T>
+zo_status launch_pipe(zo_ctx *ctx, const ProbeKey &pk, int64_t first, int64_t count, void *out) {
+  using SM = PipeSmem<T>;
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e = cudaFuncSetAttribute(perturb_pipe_kernel<T>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
+    if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "perturb_pipe_kernel attribute: %s", cudaGetErrorString(e));
+    attr = true;
+  }
+  const int64_t g0 = first / kGroup;
+  const int64_t g1 = (first + count + kGroup - 1) / kGroup;
+  const int64_t n_chunks = (g1 - g0 + kTileGroups - 1) / kTileGroups;
+  const int64_t blocks = n_chunks < (int64_t)kSmCount * 2 ? n_chunks : (int64_t)kSmCount * 2;
+  perturb_pipe_kernel<T><<<(unsigned)blocks, kPThreads, SM::kBytes, ctx->stream>>>(
+      static_cast<const T *>(ctx->params), static_cast<T *>(out), first, count, pk, n_chunks,
+      &ctx->dstate->flags);
+  return check_launch(ctx, "perturb_pipe_kernel");
+}
+
 zo_status launch_perturb(zo_ctx *ctx, const ProbeKey &pk, int64_t first, int64_t count,
                          void *out) {
   if (count <= 0) return ZO_OK;
+  const int vec = ctx->dtype == ZO_F32 ? 4 : 8;
+  if (count >= kPChunk && first % vec == 0 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0)
+    return ctx->dtype == ZO_F32 ? launch_pipe<float>(ctx, pk, first, count, out)
+                                : launch_pipe<uint16_t>(ctx, pk, first, count, out);
   const int64_t g0 = first / kGroup;
   const int64_t g1 = (first + count + kGroup - 1) / kGroup;
   const int64_t n_tiles = (g1 - g0 + kTileGroups - 1) / kTileGroups;
