@@ -195,35 +195,13 @@ def gpu_arm(args):
     def apply_step(Lp, Lm, L0):
         zo.zo_step(ctx, Lp, Lm, n, L0, LR, EPS, DAMPING)
 
-    def one_step(ev=None):
-        """Step through the C ABI primitives; ev = 4 events at the phase boundaries."""
+    def one_step():
         if world > 1:  # probe-parallel: this rank's probes, loss all-gather, same update
             from zero_order_forward_b200 import dist as zdist
-            if ev:
-                ev[0].record(stream)
             zdist.probe_parallel_step(n, loss_at, lambda o: zo.zo_quad_loss(ctx, D, o),
                                       apply_step, dev)
-            if ev:
-                for e in ev[1:]:
-                    e.record(stream)
-            return
-        if ev:
-            ev[0].record(stream)
-        zo.zo_quad_loss(ctx, D, losses[0:1])
-        if ev:
-            ev[1].record(stream)
-        for i in range(n):
-            zo.zo_perturb(ctx, +1, EPS, i)
-            zo.zo_quad_loss(ctx, D, losses[1 + i:2 + i])
-            zo.zo_restore(ctx)
-            zo.zo_perturb(ctx, -1, EPS, i)
-            zo.zo_quad_loss(ctx, D, losses[1 + n + i:2 + n + i])
-            zo.zo_restore(ctx)
-        if ev:
-            ev[2].record(stream)
-        zo.zo_step(ctx, losses[1:1 + n], losses[1 + n:], n, losses[0:1], LR, EPS, DAMPING)
-        if ev:
-            ev[3].record(stream)
+        else:  # the native step driver: every launch of the step enqueued from C++
+            zo.zo_quad_step(ctx, D, n, EPS, LR, DAMPING, True, losses)
 
     for _ in range(args.warmup):
         one_step()
@@ -232,19 +210,26 @@ def gpu_arm(args):
         dist.barrier()
     torch.cuda.synchronize()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    if world == 1:
+        zo.zo_enable_phase_timing(ctx, args.steps)  # events at the step's phase boundaries
     sampler = ClockSampler(local_rank) if rank == 0 else None
     for k in range(args.steps):
         flush.zero_()  # evict theta and D from the 126 MB L2 between steps (not timed)
-        one_step(evs[k])
+        evs[k][0].record(stream)
+        one_step()
+        evs[k][1].record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
     zo.zo_sync(ctx)
 
-    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    clean_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    probe_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    upd_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    if world == 1:
+        ph = zo.zo_phase_times(ctx, args.steps)
+        zo.zo_enable_phase_timing(ctx, 0)
+        clean_ms, probe_ms, upd_ms = (list(map(float, ph[:, i])) for i in range(3))
+    else:
+        clean_ms = probe_ms = upd_ms = [float("nan")]
     total_s = sum(step_ms) / 1e3
     if world > 1:
         t = torch.tensor([total_s], dtype=torch.float64, device=dev)

@@ -133,6 +133,19 @@ zo_status zo_sync(zo_ctx *ctx, uint32_t *flags);
 zo_status zo_get_step(zo_ctx *ctx, uint32_t *step);
 zo_status zo_set_step(zo_ctx *ctx, uint32_t step);
 
+/* ------------------------------------------------------------------ tracing */
+
+/* Phase timing of the step drivers (zo_quad_step, zo_mlp_step, zo_model_step): the next
+ * n_steps driver calls record CUDA events on the context's stream at four points (step
+ * start, after the clean loss, after the last perturbed loss, step end); n_steps = 0
+ * disables recording.  At most 4096 steps.  Errors: ZO_ERR_INVALID, ZO_ERR_CUDA. */
+zo_status zo_enable_phase_timing(zo_ctx *ctx, int32_t n_steps);
+
+/* After the recorded steps, synchronise and write ms (host, n_steps x 3 floats):
+ * per step the clean-loss, perturbed-losses and preconditioner+update times in
+ * milliseconds.  Errors: ZO_ERR_INVALID (n_steps outside what was recorded). */
+zo_status zo_phase_times(zo_ctx *ctx, int32_t n_steps, float *ms);
+
 /* ------------------------------------------------------------------ zo_rng */
 
 /* Write packed probe bytes [first_byte, first_byte + nbytes) of probe `probe` at the

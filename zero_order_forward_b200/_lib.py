@@ -51,6 +51,8 @@ _SIGS = {
     "zo_quad_step_host": [_vp, _vp, _i32, _f32, _f32, _f32, _int, _vp],
     "zo_mlp_step": [_vp, _vp, _vp, _int, _int, _int, _int, _i32, _f32, _f32, _f32, _int, _vp],
     "zo_mlp_loss_noalloc": [_vp, _vp, _vp, _int, _int, _int, _int, _f64, _vp, _int, _vp],
+    "zo_enable_phase_timing": [_vp, _i32],
+    "zo_phase_times": [_vp, _i32, _vp],
     "zo_model_param_count": [_vp, ctypes.POINTER(_i64)],
     "zo_model_create": [ctypes.POINTER(_vp), _vp, _vp, _i64],
     "zo_model_destroy": [_vp],
@@ -335,3 +337,15 @@ def zo_attention(ctx, qkv, out, batch, seq, n_heads, d_model):
 def zo_layernorm(ctx, x, gamma, beta, out, rows, d):
     return ctx.check(_L.zo_layernorm(ctx.handle, _ptr(x), _ptr(gamma), _ptr(beta), _ptr(out),
                                      rows, d))
+
+
+def zo_enable_phase_timing(ctx, n_steps):
+    return ctx.check(_L.zo_enable_phase_timing(ctx.handle, n_steps))
+
+
+def zo_phase_times(ctx, n_steps):
+    """[n_steps][3] ms (clean loss, perturbed losses, precond + update) of recorded steps."""
+    import numpy as np
+    ms = np.zeros((n_steps, 3), np.float32)
+    ctx.check(_L.zo_phase_times(ctx.handle, n_steps, ms.ctypes.data))
+    return ms

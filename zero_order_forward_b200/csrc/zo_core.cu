@@ -47,6 +47,12 @@ ProbeKey probe_key(const zo_ctx *ctx) {
   return pk;
 }
 
+void phase_mark(zo_ctx *ctx, int which) {
+  if (!ctx->phase_ev || ctx->phase_used >= ctx->phase_cap) return;
+  cudaEventRecord(ctx->phase_ev[4 * ctx->phase_used + which], ctx->stream);
+  if (which == 3) ctx->phase_used += 1;
+}
+
 }  // namespace zo
 
 using namespace zo;
@@ -160,7 +166,49 @@ zo_status zo_destroy(zo_ctx *ctx) {
   cudaFree(ctx->live);
   cudaFree(ctx->staging);
   cudaFree(ctx->loss_scratch);
+  if (ctx->phase_ev) {
+    for (int i = 0; i < 4 * ctx->phase_cap; ++i) cudaEventDestroy(ctx->phase_ev[i]);
+    delete[] ctx->phase_ev;
+  }
   delete ctx;
+  return ZO_OK;
+}
+
+zo_status zo_enable_phase_timing(zo_ctx *ctx, int32_t n_steps) {
+  ZO_CHECK(check_ctx(ctx));
+  if (n_steps < 0 || n_steps > 4096) return fail(ctx, ZO_ERR_INVALID, "n_steps outside [0, 4096]");
+  ZO_CUDA(ctx, cudaStreamSynchronize(ctx->stream), "sync");
+  if (ctx->phase_ev) {
+    for (int i = 0; i < 4 * ctx->phase_cap; ++i) cudaEventDestroy(ctx->phase_ev[i]);
+    delete[] ctx->phase_ev;
+    ctx->phase_ev = nullptr;
+  }
+  ctx->phase_cap = ctx->phase_used = 0;
+  if (n_steps == 0) return ZO_OK;
+  ctx->phase_ev = new (std::nothrow) cudaEvent_t[4 * n_steps];
+  if (!ctx->phase_ev) return fail(ctx, ZO_ERR_OOM, "phase events");
+  for (int i = 0; i < 4 * n_steps; ++i) {
+    const cudaError_t e = cudaEventCreate(&ctx->phase_ev[i]);
+    if (e != cudaSuccess) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(ctx->phase_ev[j]);
+      delete[] ctx->phase_ev;
+      ctx->phase_ev = nullptr;
+      return cuda_fail(ctx, e, "cudaEventCreate");
+    }
+  }
+  ctx->phase_cap = n_steps;
+  return ZO_OK;
+}
+
+zo_status zo_phase_times(zo_ctx *ctx, int32_t n_steps, float *ms) {
+  ZO_CHECK(check_ctx(ctx));
+  if (!ms || n_steps < 1 || n_steps > ctx->phase_used)
+    return fail(ctx, ZO_ERR_INVALID, "only %d steps were recorded", ctx->phase_used);
+  ZO_CUDA(ctx, cudaStreamSynchronize(ctx->stream), "sync");
+  for (int k = 0; k < n_steps; ++k)
+    for (int p = 0; p < 3; ++p)
+      ZO_CUDA(ctx, cudaEventElapsedTime(&ms[3 * k + p], ctx->phase_ev[4 * k + p],
+                                        ctx->phase_ev[4 * k + p + 1]), "cudaEventElapsedTime");
   return ZO_OK;
 }
 
@@ -326,11 +374,13 @@ zo_status zo_quad_step(zo_ctx *ctx, const float *D, int32_t n_pert, float eps, f
   if (!losses_out) return fail(ctx, ZO_ERR_INVALID, "null losses_out");
   if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "step while perturbed");
   double *L0 = losses_out, *Lp = losses_out + 1, *Lm = losses_out + 1 + n_pert;
+  phase_mark(ctx, 0);
   if (preconditioned) {
     ZO_CHECK(zo_quad_loss(ctx, D, L0, 0));
   } else {
     ZO_CUDA(ctx, cudaMemsetAsync(L0, 0, sizeof(double), ctx->stream), "clear L0");
   }
+  phase_mark(ctx, 1);
   for (int32_t i = 0; i < n_pert; ++i) {
     ZO_CHECK(zo_perturb(ctx, +1, eps, i));
     zo_status st = zo_quad_loss(ctx, D, Lp + i, 0);
@@ -341,7 +391,10 @@ zo_status zo_quad_step(zo_ctx *ctx, const float *D, int32_t n_pert, float eps, f
     zo_restore(ctx);
     ZO_CHECK(st);
   }
-  return zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
+  phase_mark(ctx, 2);
+  const zo_status st = zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
+  phase_mark(ctx, 3);
+  return st;
 }
 
 zo_status zo_quad_step_host(zo_ctx *ctx, const float *D_host, int32_t n_pert, float eps,
@@ -372,11 +425,13 @@ zo_status zo_mlp_step(zo_ctx *ctx, const float *X, const int32_t *labels, int ba
   if (!ctx->live_enabled) ZO_CHECK(zo_set_live_buffer(ctx, 1));
   const double scale = 1.0 / (double)batch;
   double *L0 = losses_out, *Lp = losses_out + 1, *Lm = losses_out + 1 + n_pert;
+  phase_mark(ctx, 0);
   if (preconditioned) {
     ZO_CHECK(zo_mlp_loss(ctx, X, labels, batch, n_in, n_hidden, n_out, scale, L0, 0));
   } else {
     ZO_CUDA(ctx, cudaMemsetAsync(L0, 0, sizeof(double), ctx->stream), "clear L0");
   }
+  phase_mark(ctx, 1);
   for (int32_t i = 0; i < n_pert; ++i) {
     for (int s = +1; s >= -1; s -= 2) {
       ZO_CHECK(zo_perturb(ctx, s, eps, i));
@@ -386,7 +441,10 @@ zo_status zo_mlp_step(zo_ctx *ctx, const float *X, const int32_t *labels, int ba
       ZO_CHECK(st);
     }
   }
-  return zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
+  phase_mark(ctx, 2);
+  const zo_status st = zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
+  phase_mark(ctx, 3);
+  return st;
 }
 
 }  // extern "C"

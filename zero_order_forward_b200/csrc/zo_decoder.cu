@@ -415,6 +415,7 @@ zo_status zo_model_step(zo_model *m, const int32_t *tokens, const int32_t *label
   double *L0 = losses_out, *Lp = losses_out + 1, *Lm = losses_out + 1 + n_pert;
   zo_status st;
   if (n_pert < 1 || n_pert > ZO_MAX_PROBES) return fail(ctx, ZO_ERR_INVALID, "n_pert out of range");
+  phase_mark(ctx, 0);
   if (preconditioned) {
     for (int k = 0; k < n_micro; ++k)
       if ((st = zo_model_loss(m, tokens + k * tok_stride, labels + (int64_t)k * batch, batch, seq,
@@ -424,6 +425,7 @@ zo_status zo_model_step(zo_model *m, const int32_t *tokens, const int32_t *label
                               "clear L0")) != ZO_OK) {
     return st;
   }
+  phase_mark(ctx, 1);
   for (int32_t i = 0; i < n_pert; ++i) {
     for (int s = +1; s >= -1; s -= 2) {
       if ((st = zo_perturb(ctx, s, eps, i)) != ZO_OK) return st;
@@ -434,7 +436,10 @@ zo_status zo_model_step(zo_model *m, const int32_t *tokens, const int32_t *label
       if (st != ZO_OK) return st;
     }
   }
-  return zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
+  phase_mark(ctx, 2);
+  st = zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
+  phase_mark(ctx, 3);
+  return st;
 }
 
 zo_status zo_gemm_bf16(zo_ctx *ctx, const void *A, const void *B, const void *bias, void *out,

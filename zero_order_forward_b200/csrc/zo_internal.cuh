@@ -108,6 +108,10 @@ struct zo_ctx {
   float *staging = nullptr;    // device staging for host-buffer entry points
   double *loss_scratch = nullptr;  // 2*ZO_MAX_PROBES+1 doubles for host-buffer steps
 
+  // phase timing of the step drivers: 4 events per recorded step
+  cudaEvent_t *phase_ev = nullptr;
+  int32_t phase_cap = 0, phase_used = 0;
+
   std::string err;
 };
 
@@ -119,6 +123,10 @@ zo_status fail(zo_ctx *ctx, zo_status st, const char *fmt, ...);
 zo_status check_launch(zo_ctx *ctx, const char *what);
 
 ProbeKey probe_key(const zo_ctx *ctx);  // current perturbation (sign 0 when clean)
+
+// Record phase event `which` (0..3) of the current step if phase timing is enabled;
+// which == 3 closes the step.
+void phase_mark(zo_ctx *ctx, int which);
 
 // Launchers (each enqueues on ctx->stream and returns the launch status).
 zo_status launch_perturb(zo_ctx *ctx, const ProbeKey &pk, int64_t first, int64_t count,

@@ -62,19 +62,20 @@ __device__ void finish_reduction(double v, double *partials, unsigned int *count
 
 // L = 1/2 sum_j D_j P_j^2 with P_j = rd(theta_j + s*eps*z_j) computed on load.
 //
-// A persistent producer/consumer pipeline: warp 0 streams 2048-element chunks of theta and
-// D into a ring of shared-memory stages with bulk asynchronous copies, then its first 16
-// lanes compute the chunk's 16 Philox blocks into the stage while the copies are in flight
+// A persistent producer/consumer pipeline: warp 0 streams 4096-element chunks of theta and
+// D into a ring of shared-memory stages with bulk asynchronous copies, then its 32 lanes
+// compute the chunk's 32 Philox blocks into the stage while the copies are in flight
 // (each stage's full barrier takes two arrivals: the copies' and the blocks'); the 8
 // consumer warps apply the perturbation and accumulate in fp64 (four independent partial
 // sums per thread), then release the stage.
 // Chunks are assigned round-robin (chunk = blockIdx.x + k * gridDim.x), so the grid size
 // and every summation order depend on M only: the result is deterministic.
-constexpr int kQChunk = 2048;
-constexpr int kQStages = 6;
+constexpr int kQChunk = 4096;
+constexpr int kQStages = 3;
 constexpr int kQConsumers = 8;
 constexpr int kQThreads = 32 * (1 + kQConsumers);
-constexpr int kQStageBytes = 2 * kQChunk * 4 + 16 * 16;  // theta, D, 16 Philox blocks
+constexpr int kQGroups = kQChunk / kGroup;                    // Philox blocks per chunk (32)
+constexpr int kQStageBytes = 2 * kQChunk * 4 + kQGroups * 16;  // theta, D, Philox blocks
 constexpr int kQSmemBytes = kQStages * kQStageBytes + 2 * kQStages * 8;
 
 __global__ void __launch_bounds__(kQThreads)
@@ -122,7 +123,7 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
           tc::bulk_load(st + kQChunk * 4, D + base, (uint32_t)copy * 4u, &full[s]);
         }
       }
-      if (pk.sign && lane < 16 && (int64_t)lane * kGroup < cnt)
+      if (pk.sign && lane < kQGroups && (int64_t)lane * kGroup < cnt)
         reinterpret_cast<uint4 *>(st + 2 * kQChunk * 4)[lane] =
             probe_block((uint64_t)(base / kGroup) + lane, pk.probe, step, pk.k0, pk.k1);
       __syncwarp();
@@ -185,6 +186,10 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
     }
   }
   double acc = __dadd_rn(__dadd_rn(acc4[0], acc4[1]), __dadd_rn(acc4[2], acc4[3]));
+  // The next loss pass may start streaming now; the reduction scratch (partials, counter,
+  // out) is touched only after the previous kernel in the stream has fully completed.
+  tc::pdl_launch_dependents();
+  tc::pdl_wait();
   acc = block_sum(acc);
   finish_reduction(acc, partials, counter, out, accumulate, 1.0);
 }
@@ -249,9 +254,24 @@ zo_status launch_quad_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, doub
     if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "quad_loss_kernel attribute: %s", cudaGetErrorString(e));
     attr = true;
   }
-  quad_loss_kernel<<<(unsigned)blocks, kQThreads, kQSmemBytes, ctx->stream>>>(
-      static_cast<const float *>(ctx->params), D, ctx->M, pk, n_chunks, partials, counter, out,
-      accumulate, &ctx->dstate->flags);
+  // Programmatic dependent launch: this pass may begin while the previous loss pass of
+  // the stream finishes its reduction (see pdl_wait in the kernel).  Kernels that write
+  // theta or the step counter never signal early, so they still complete first.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(kQThreads);
+  cfg.dynamicSmemBytes = kQSmemBytes;
+  cfg.stream = ctx->stream;
+  cudaLaunchAttribute attr_pdl[1];
+  attr_pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr_pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr_pdl;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, quad_loss_kernel,
+                                           static_cast<const float *>(ctx->params), D, ctx->M, pk,
+                                           n_chunks, partials, counter, out, accumulate,
+                                           &ctx->dstate->flags);
+  if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "quad_loss_kernel: %s", cudaGetErrorString(e));
   return check_launch(ctx, "quad_loss_kernel");
 }
 
