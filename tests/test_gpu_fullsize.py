@@ -1,0 +1,144 @@
+"""Full-size checks of the decoder workloads in the launch configuration the benchmark
+times (OPT-1.3B-shaped: micro-batch 16 x 512; OPT-30B-shaped: 8 x 2048), and of
+checkpoint/resume and allocation failure.
+
+Sampled outputs the oracle can compute one by one: causal attention makes the residual
+stream at positions < P depend on the first P tokens only, so the GPU's hidden state of
+sequence 0 at positions 0..P-1 (computed on the full batch) must match the oracle's
+forward over that P-token prefix.  Tolerance: relative Frobenius error <= 1e-2.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from oracle import core
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+PREFIX = 64
+
+
+def _device_params(cfg, seed):
+    """OPT-style synthetic weights generated on the device by torch (inputs, not outputs
+    of this library): matrices N(0, 0.02), biases 0, LayerNorm gains 1 / shifts 0."""
+    M = oracle.opt.param_count(cfg)
+    theta = torch.empty(M, dtype=torch.bfloat16, device="cuda")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    o = 0
+    for kind, n in synth.opt_segments(cfg):
+        seg = theta[o:o + n]
+        if kind == "matrix":
+            for a in range(0, n, 1 << 28):
+                seg[a:a + (1 << 28)].normal_(0.0, 0.02, generator=g)
+        elif kind == "gain":
+            seg.fill_(1.0)
+        else:
+            seg.zero_()
+        o += n
+    return theta
+
+
+def _host_window(theta, off, n):
+    return theta[off:off + n].view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _prefix_oracle(theta, cfg, tokens0, n_layers, perturb=None, dtype=np.float64):
+    """Oracle hidden state after n_layers for the prefix tokens0 [P], from the slices of
+    theta it needs (embedding rows, position rows, the first n_layers layer blocks)."""
+    lay = oracle.opt.layout(cfg)
+    d, P = cfg["d_model"], len(tokens0)
+    small = dict(cfg, vocab=len(tokens0), max_pos=P, n_layers=n_layers)
+    # a compact parameter vector in the same layout: E rows = the prefix's tokens
+    parts = []
+    off_E = lay["E"][0]
+    rows = [_host_window(theta, off_E + int(t) * d, d) for t in tokens0]
+    pos_off = lay["Pos"][0]
+    pos = _host_window(theta, pos_off, (P + 2) * d)
+    first_layer = lay["L0.ln1g"][0]
+    layer_size = lay["L1.ln1g"][0] - first_layer if cfg["n_layers"] > 1 else None
+    blocks = _host_window(theta, first_layer, n_layers * layer_size)
+    fin = np.zeros(2 * d, np.uint16)
+    if perturb is not None:  # (seed, step, probe, sign, eps): perturb each slice at its global index
+        seed, step, probe, sign, eps = perturb
+        rows = [core.perturb(r, seed, step, probe, sign, eps, j0=off_E + int(t) * d)
+                for r, t in zip(rows, tokens0)]
+        pos = core.perturb(pos, seed, step, probe, sign, eps, j0=pos_off)
+        blocks = core.perturb(blocks, seed, step, probe, sign, eps, j0=first_layer)
+    parts = [np.concatenate(rows), pos, blocks, fin]
+    flat = core.bf16_to_f32(np.concatenate(parts)).astype(dtype)
+    assert flat.size == oracle.opt.param_count(small)
+    return oracle.opt.hidden_states(flat, small, np.arange(P)[None, :], dtype=dtype)[0]
+
+
+@pytest.mark.parametrize("name,B,S,n_layers,perturbed,dtype", [
+    ("opt-1.3b", 16, 512, 24, False, np.float32),
+    ("opt-1.3b", 16, 512, 2, True, np.float64),
+    ("opt-30b", 8, 2048, 1, False, np.float32)])
+def test_fullsize_prefix_hidden_state(zo, name, B, S, n_layers, perturbed, dtype):
+    cfg = synth.OPT_CONFIGS[name]
+    free, _ = torch.cuda.mem_get_info()
+    if free < oracle.opt.param_count(cfg) * 2 + (4 << 30):
+        pytest.skip("not enough device memory for this workload")
+    theta = _device_params(cfg, seed=7)
+    ctx = zo.zo_create(theta, seed=7)
+    model = zo.zo_model_create(ctx, cfg, B * S)
+    tokens, _ = synth.opt_batch(cfg, B, S, seed=7)
+    dtok = torch.from_numpy(tokens).cuda()
+    h = torch.empty((B * S, cfg["d_model"]), dtype=torch.float32, device="cuda")
+    if perturbed:
+        zo.zo_perturb(ctx, -1, 1e-3, 5)
+    zo.zo_model_hidden(model, dtok, B, S, n_layers, h)
+    if perturbed:
+        zo.zo_restore(ctx)
+    assert zo.zo_sync(ctx) == 0
+    got = h[:PREFIX].cpu().numpy().astype(np.float64)
+    ref = _prefix_oracle(theta, cfg, tokens[0, :PREFIX], n_layers,
+                         perturb=(7, 0, 5, -1, 1e-3) if perturbed else None, dtype=dtype)
+    err = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert err <= 1e-2, err
+    model.close()
+    ctx.close()
+    del theta
+    torch.cuda.empty_cache()
+
+
+def test_checkpoint_resume_is_bit_identical(zo):
+    """The training state is theta plus (seed, step): 10 steps equal 5 steps, a
+    checkpoint (copy of theta and the step counter), a fresh context, and 5 more."""
+    M, n = 1 << 16, 8
+    th_np, D_np = synth.quad_problem(M, seed=9)
+    D = torch.from_numpy(D_np).cuda()
+    losses = torch.zeros(2 * n + 1, dtype=torch.float64, device="cuda")
+    a = torch.from_numpy(th_np).cuda()
+    ca = zo.zo_create(a, seed=11)
+    for _ in range(10):
+        zo.zo_quad_step(ca, D, n, 1e-3, 1e-6, 1e-3, True, losses)
+    b = torch.from_numpy(th_np).cuda()
+    cb = zo.zo_create(b, seed=11)
+    for _ in range(5):
+        zo.zo_quad_step(cb, D, n, 1e-3, 1e-6, 1e-3, True, losses)
+    ckpt_theta, ckpt_step = b.cpu().clone(), zo.zo_get_step(cb)
+    cb.close()
+    c = ckpt_theta.cuda()
+    cc = zo.zo_create(c, seed=11)
+    zo.zo_set_step(cc, ckpt_step)
+    for _ in range(5):
+        zo.zo_quad_step(cc, D, n, 1e-3, 1e-6, 1e-3, True, losses)
+    assert zo.zo_get_step(ca) == zo.zo_get_step(cc) == 10
+    assert torch.equal(a.view(torch.int32), c.view(torch.int32))
+    ca.close()
+    cc.close()
+
+
+def test_allocation_failure_reports_oom(zo):
+    """A live buffer larger than the device returns ZO_ERR_OOM (the context stays usable)."""
+    th = torch.zeros(1024, device="cuda")
+    ctx = zo.zo_create(th, M=1 << 38)  # the live buffer would need 1 TiB
+    with pytest.raises(zo.ZoError) as ei:
+        zo.zo_set_live_buffer(ctx, True)
+    assert ei.value.status == zo.ZO_ERR_OOM
+    assert zo.zo_sync(ctx) == 0
+    ctx.close()
