@@ -12,8 +12,10 @@
 //              epilogue;
 //   warps 2-9  the epilogue, two warps per TMEM lane quadrant (warp w reads TMEM lanes
 //              32*(w%4)..+31 = its 32 output rows, half of the columns each): tcgen05.ld
-//              32 columns at a time, bias, ReLU or the fp32 residual add (residual loaded
-//              before the TMEM read), store, and hand the accumulator back.
+//              32 columns at a time, bias and ReLU, a swizzled 32 x 32 staging tile in
+//              shared memory, then one TMA tile store (bf16 outputs) or TMA add-reduce into
+//              the fp32 residual stream (global += tile in L2, no load by the SM); the
+//              accumulator is handed back after its last TMEM read.
 // Tiles are visited in groups of kGroupM row tiles so that the weight tiles of a group are
 // reused from L2.  All waits are bounded (see zo_tc.cuh); a timeout sets an error bit.
 #include <cudaTypedefs.h>
@@ -61,71 +63,42 @@ __device__ __forceinline__ void load_bias32(const uint16_t *bias, int col0, int 
   }
 }
 
-// Residual values of a full 32-column chunk, loaded before the accumulator is read so
-// that the global-load latency overlaps the TMEM load.
-__device__ __forceinline__ void load_resid32(const GemmArgs &a, int row, int col0, float4 h[8]) {
-  if (row < a.M && col0 + 32 <= a.N) {
-    const float4 *o = reinterpret_cast<const float4 *>(static_cast<const float *>(a.out) +
-                                                       (int64_t)row * a.ldo + col0);
+// Write one accumulator row chunk (32 columns of row `r` of a 32 x 32 tile) into the
+// warp's staging tile in the layout the output tensor map's swizzle expects:
+//   fp32: 128-byte rows, 16-byte chunk c stored at chunk c ^ (r & 7)   (128B swizzle);
+//   bf16:  64-byte rows, 16-byte chunk c stored at chunk c ^ ((r >> 1) & 3) (64B swizzle).
+template <int EPI>
+__device__ __forceinline__ void stage_row(uint8_t *stage, int r, const float v[32]) {
+  if (EPI == ZO_EPI_RESID_F32) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) h[k] = o[k];
+    for (int c = 0; c < 8; ++c)
+      *reinterpret_cast<float4 *>(stage + r * 128 + ((c ^ (r & 7)) << 4)) =
+          make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+  } else {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t w[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        w[t] = (uint32_t)f32_to_bf16_bits(v[8 * c + 2 * t]) |
+               ((uint32_t)f32_to_bf16_bits(v[8 * c + 2 * t + 1]) << 16);
+      *reinterpret_cast<uint4 *>(stage + r * 64 + ((c ^ ((r >> 1) & 3)) << 4)) =
+          make_uint4(w[0], w[1], w[2], w[3]);
+    }
   }
 }
 
-template <int EPI>
-__device__ __forceinline__ void epilogue_store(const float acc[32], int row, int col0,
-                                               const GemmArgs &a, const float4 hpre[8]) {
-  float b[32];
-  load_bias32(a.bias, col0, a.N, b);
-  if (EPI == ZO_EPI_RESID_F32) {
-    float *o = static_cast<float *>(a.out) + (int64_t)row * a.ldo + col0;
-    if (col0 + 32 <= a.N) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        float4 h = hpre[k];
-        h.x = __fadd_rn(h.x, __fadd_rn(acc[4 * k], b[4 * k]));
-        h.y = __fadd_rn(h.y, __fadd_rn(acc[4 * k + 1], b[4 * k + 1]));
-        h.z = __fadd_rn(h.z, __fadd_rn(acc[4 * k + 2], b[4 * k + 2]));
-        h.w = __fadd_rn(h.w, __fadd_rn(acc[4 * k + 3], b[4 * k + 3]));
-        reinterpret_cast<float4 *>(o)[k] = h;
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (col0 + i < a.N) o[i] = __fadd_rn(o[i], __fadd_rn(acc[i], b[i]));
-    }
-  } else {
-    float v[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      v[i] = __fadd_rn(acc[i], b[i]);
-      if (EPI == ZO_EPI_RELU_BF16) v[i] = fmaxf(v[i], 0.f);
-    }
-    uint16_t *o = static_cast<uint16_t *>(a.out) + (int64_t)row * a.ldo + col0;
-    if (col0 + 32 <= a.N) {
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        uint32_t w[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-          w[t] = (uint32_t)f32_to_bf16_bits(v[8 * k + 2 * t]) |
-                 ((uint32_t)f32_to_bf16_bits(v[8 * k + 2 * t + 1]) << 16);
-        reinterpret_cast<uint4 *>(o)[k] = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (col0 + i < a.N) o[i] = f32_to_bf16_bits(v[i]);
-    }
-  }
-}
+constexpr int kEpiWarps = 8;                      // two warps per TMEM lane quadrant
+constexpr int kGemmThreads = 32 * (2 + kEpiWarps);  // producer, MMA, epilogue
+constexpr uint32_t kStageTile = 32 * 128;           // one 32 x 32 fp32 (or bf16) output tile
 
 template <int BN, int STAGES>
 struct GemmSmem {
   static constexpr uint32_t kABytes = kBM * kBK * 2;
   static constexpr uint32_t kBBytes = BN * kBK * 2;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr uint32_t kBarOffset = STAGES * kStageBytes;
+  static constexpr uint32_t kOutOffset = STAGES * kStageBytes;         // 1024-aligned
+  static constexpr uint32_t kBarOffset = kOutOffset + kEpiWarps * kStageTile;
   static constexpr uint32_t kBytes = kBarOffset + 256 + 1024;  // + barriers + alignment slack
 };
 
@@ -148,19 +121,17 @@ __device__ __forceinline__ TileCoord tile_coord(int t, int num_m, int num_n, int
 // The shared-memory ring runs across tile boundaries, and the accumulator is
 // double-buffered in TMEM (2 x BN columns) so the epilogue of tile i overlaps the
 // main loop of tile i+1.
-constexpr int kEpiWarps = 8;                      // two warps per TMEM lane quadrant
-constexpr int kGemmThreads = 32 * (2 + kEpiWarps);  // producer, MMA, epilogue
-
 template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 GemmArgs args) {
+                 const __grid_constant__ CUtensorMap tmC, GemmArgs args) {
   using S = GemmSmem<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *sA = smem;
   uint8_t *sB = smem + STAGES * S::kABytes;
+  uint8_t *sOut = smem + S::kOutOffset;  // one 32 x 32 staging tile per epilogue warp
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + S::kBarOffset);
   uint64_t *empty = full + STAGES;
   uint64_t *acc_full = empty + STAGES;   // [2] MMA -> epilogue
@@ -251,6 +222,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const int q = warp & 3;                    // TMEM lanes 32q..32q+31 (this warp's rows)
     const int half = (warp - 2) / 4;           // which half of the BN columns
     const int cbeg = half * (BN / 2), cend = cbeg + BN / 2;
+    uint8_t *stage = sOut + (warp - 2) * kStageTile;
+    if (lane == 0) tc::tma_prefetch_desc(&tmC);
     int i = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++i) {
       const int b = i & 1;
@@ -262,21 +235,36 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       }
       tc::tc_fence_after();
       const TileCoord tc0 = tile_coord(t, num_m, num_n, BN);
-      const int row = tc0.m0 + q * 32 + lane;
+      const int row0 = tc0.m0 + q * 32;
       const uint32_t base = tmem + (uint32_t)(b * BN) + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
       for (int c0 = cbeg; c0 < cend; c0 += 32) {
         if (tc0.n0 + c0 >= args.N) break;
-        float4 hpre[8];
-        if (EPI == ZO_EPI_RESID_F32) load_resid32(args, row, tc0.n0 + c0, hpre);
-        float v[32];
+        float v[32], bias[32];
         tc::tmem_ld32(base + (uint32_t)c0, v);
-        if (row < args.M) epilogue_store<EPI>(v, row, tc0.n0 + c0, args, hpre);
+        load_bias32(args.bias, tc0.n0 + c0, args.N, bias);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          v[k] = __fadd_rn(v[k], bias[k]);
+          if (EPI == ZO_EPI_RELU_BF16) v[k] = fmaxf(v[k], 0.f);
+        }
+        // the previous chunk's bulk store must have finished reading the staging tile
+        if (lane == 0) tc::bulk_wait_read0();
+        __syncwarp();
+        stage_row<EPI>(stage, lane, v);
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < args.M) {
+          if (EPI == ZO_EPI_RESID_F32) tc::tma_reduce_add_2d(&tmC, stage, tc0.n0 + c0, row0);
+          else tc::tma_store_2d(&tmC, stage, tc0.n0 + c0, row0);
+          tc::bulk_commit();
+        }
       }
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&acc_empty[b]);
     }
+    if (lane == 0) tc::bulk_wait0();  // this warp's stores and reductions have landed
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -311,6 +299,24 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// Output tile map: [rows][cols] with row stride ld elements, box 32 x 32; fp32 uses the
+// 128-byte swizzle (128-byte box rows), bf16 the 64-byte swizzle (64-byte box rows).
+// Stores outside [rows][cols] are clipped by the hardware.
+bool make_out_map(CUtensorMap *m, void *base, int64_t rows, int64_t cols, int64_t ld, bool f32) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const int es = f32 ? 4 : 2;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(ld * es)};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                        base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // 2-D bf16 tensor [rows][cols] (row-major, cols contiguous), box = box_rows x 64 columns,
 // 128-byte swizzle, zero fill outside the tensor.
 bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int box_rows) {
@@ -327,8 +333,8 @@ bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int 
 }
 
 template <int BN, int STAGES, int EPI>
-cudaError_t launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &g,
-                       cudaStream_t st) {
+cudaError_t launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tcm,
+                       const GemmArgs &g, cudaStream_t st) {
   using S = GemmSmem<BN, STAGES>;
   auto kern = gemm_bf16_kernel<BN, STAGES, EPI>;
   static bool attr_set = false;  // per instantiation; benign race (idempotent call)
@@ -339,7 +345,7 @@ cudaError_t launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const GemmA
   }
   const int num_m = (g.M + kBM - 1) / kBM, num_n = (g.N + BN - 1) / BN;
   const int tiles = num_m * num_n;
-  kern<<<tiles < kSmCount ? tiles : kSmCount, kGemmThreads, S::kBytes, st>>>(ta, tb, g);
+  kern<<<tiles < kSmCount ? tiles : kSmCount, kGemmThreads, S::kBytes, st>>>(ta, tb, tcm, g);
   return cudaGetLastError();
 }
 
@@ -355,19 +361,20 @@ zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bia
   if (epi < ZO_EPI_BIAS_BF16 || epi > ZO_EPI_RESID_F32) return fail(ctx, ZO_ERR_INVALID, "gemm: bad epilogue");
   // N <= 128 tiles use BN = 128 to fill the machine on narrow outputs.
   const bool wide = N > 128 && ((int64_t)((M + 127) / 128) * ((N + 255) / 256) >= kSmCount);
-  CUtensorMap ta, tb;
-  if (!make_map(&ta, A, M, K, kBM) || !make_map(&tb, B, N, K, wide ? 256 : 128))
+  CUtensorMap ta, tb, tcm;
+  if (!make_map(&ta, A, M, K, kBM) || !make_map(&tb, B, N, K, wide ? 256 : 128) ||
+      !make_out_map(&tcm, out, M, N, ldo, epi == ZO_EPI_RESID_F32))
     return fail(ctx, ZO_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
   GemmArgs g{M, N, K, static_cast<const uint16_t *>(bias), out, ldo, &ctx->dstate->flags};
   cudaError_t e;
   if (wide) {
-    if (epi == ZO_EPI_BIAS_BF16) e = launch_one<256, 4, ZO_EPI_BIAS_BF16>(ta, tb, g, ctx->stream);
-    else if (epi == ZO_EPI_RELU_BF16) e = launch_one<256, 4, ZO_EPI_RELU_BF16>(ta, tb, g, ctx->stream);
-    else e = launch_one<256, 4, ZO_EPI_RESID_F32>(ta, tb, g, ctx->stream);
+    if (epi == ZO_EPI_BIAS_BF16) e = launch_one<256, 4, ZO_EPI_BIAS_BF16>(ta, tb, tcm, g, ctx->stream);
+    else if (epi == ZO_EPI_RELU_BF16) e = launch_one<256, 4, ZO_EPI_RELU_BF16>(ta, tb, tcm, g, ctx->stream);
+    else e = launch_one<256, 4, ZO_EPI_RESID_F32>(ta, tb, tcm, g, ctx->stream);
   } else {
-    if (epi == ZO_EPI_BIAS_BF16) e = launch_one<128, 6, ZO_EPI_BIAS_BF16>(ta, tb, g, ctx->stream);
-    else if (epi == ZO_EPI_RELU_BF16) e = launch_one<128, 6, ZO_EPI_RELU_BF16>(ta, tb, g, ctx->stream);
-    else e = launch_one<128, 6, ZO_EPI_RESID_F32>(ta, tb, g, ctx->stream);
+    if (epi == ZO_EPI_BIAS_BF16) e = launch_one<128, 6, ZO_EPI_BIAS_BF16>(ta, tb, tcm, g, ctx->stream);
+    else if (epi == ZO_EPI_RELU_BF16) e = launch_one<128, 6, ZO_EPI_RELU_BF16>(ta, tb, tcm, g, ctx->stream);
+    else e = launch_one<128, 6, ZO_EPI_RESID_F32>(ta, tb, tcm, g, ctx->stream);
   }
   if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "gemm launch: %s", cudaGetErrorString(e));
   return ZO_OK;
