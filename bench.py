@@ -39,6 +39,23 @@ WORKLOAD = ("diagonal quadratic L=1/2*sum D_j theta_j^2, M=2^24 fp32, D log-unif
             "theta0~N(0,1); 1.5-SPSA n_pert=64 eps=1e-3 lr=4e-7 damping=1e-3")
 FALLBACK_HBM_GBS = 6650.0
 
+# DRAM bytes (read + write) per launch of the loss kernel from the ncu capture summarised
+# in profiles/quad_loss_kernel.quadratic_M2p24.md, valid for the kernel source whose SHA-256
+# (of zero_order_forward_b200/csrc/zo_loss.cu) is recorded with it; reported as null when
+# the source has changed since the capture.
+LOSS_TRAFFIC = {"zo_loss_sha256": "522a5168ba23829afcb9f7887abebc28a98e7a44f0509c447d75d14b0bded121",
+                "bytes": 138.17e6}
+
+
+def loss_traffic():
+    import hashlib
+    src = os.path.join(ROOT, "zero_order_forward_b200", "csrc", "zo_loss.cu")
+    try:
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    return LOSS_TRAFFIC["bytes"] if h == LOSS_TRAFFIC["zo_loss_sha256"] else None
+
 
 FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS_SUSTAINED = 1590.0, 1400.0
 
@@ -335,8 +352,7 @@ def gpu_arm(args):
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
         }
-        if args.traffic is not None:
-            line["roofline"]["traffic"] = args.traffic
+        line["roofline"]["traffic"] = args.traffic if args.traffic is not None else loss_traffic()
     ctx.close()
     if world > 1:
         dist.barrier()
@@ -481,6 +497,49 @@ def decoder_arm(args):
     return 0
 
 
+# ------------------------------------------------------------------ MLP workload
+
+def mlp_arm(args):
+    import torch
+
+    import synth
+    import zero_order_forward_b200 as zo
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    n, eps, lr, lam, B = 16, 1e-3, 1e-2, 1e-3, synth.MLP_BATCH
+    theta = torch.from_numpy(synth.mlp_params(0)).to(dev)
+    teacher = synth.mlp_params(0, tag="teacher")
+    batches = [synth.mlp_batch(0, k, teacher) for k in range(args.warmup + args.steps)]
+    Xs = [torch.from_numpy(x).to(dev) for x, _ in batches]
+    ys = [torch.from_numpy(y).to(dev) for _, y in batches]
+    stream = torch.cuda.current_stream(dev)
+    ctx = zo.zo_create(theta, seed=0, stream=stream.cuda_stream)
+    losses = torch.zeros(2 * n + 1, dtype=torch.float64, device=dev)
+    for k in range(args.warmup):
+        zo.zo_mlp_step(ctx, Xs[k], ys[k], B, 64, 256, 10, n, eps, lr, lam, True, losses)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record(stream)
+    for k in range(args.warmup, args.warmup + args.steps):
+        zo.zo_mlp_step(ctx, Xs[k], ys[k], B, 64, 256, 10, n, eps, lr, lam, True, losses)
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    zo.zo_sync(ctx)
+    total_s = ev[0].elapsed_time(ev[1]) / 1e3
+    line = {"metric": METRIC, "value": args.steps / total_s, "unit": "steps/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": "MLP 64-256-10 fp32 (M=19,210), batch 64, teacher labels, "
+                                   "n_pert=16, eps=1e-3, lr=1e-2, damping=1e-3, 1.5-SPSA"},
+            "final_loss": float(losses[0].item()),
+            "gpu_launches": (1 + 2 * n * 2 + 2) * args.steps}
+    ctx.close()
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -491,13 +550,15 @@ def main():
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per launch of the loss kernel, if measured")
     ap.add_argument("--workload", default="quadratic",
-                    choices=["quadratic"] + sorted(DECODER_WORKLOADS))
+                    choices=["quadratic", "mlp"] + sorted(DECODER_WORKLOADS))
     ap.add_argument("--n-pert", type=int, default=None, help="override n_pert (decoder workloads)")
     args = ap.parse_args()
     if args.warmup < 3 and args.workload == "quadratic":
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return reference_arm(args)
+    if args.workload == "mlp":
+        return mlp_arm(args)
     if args.workload != "quadratic":
         return decoder_arm(args)
     return gpu_arm(args)
