@@ -39,10 +39,10 @@ WORKLOAD = ("diagonal quadratic L=1/2*sum D_j theta_j^2, M=2^24 fp32, D log-unif
             "theta0~N(0,1); 1.5-SPSA n_pert=64 eps=1e-3 lr=4e-7 damping=1e-3")
 FALLBACK_HBM_GBS = 6650.0
 
-# DRAM bytes (read + write) per launch of the loss kernel from the ncu capture summarised
-# in profiles/quad_loss_kernel.quadratic_M2p24.md, valid for the kernel source whose SHA-256
-# (of zero_order_forward_b200/csrc/zo_loss.cu) is recorded with it; reported as null when
-# the source has changed since the capture.
+# DRAM bytes (read + write) per launch of the loss-pair kernel from the ncu capture
+# summarised in profiles/quad_loss_kernel.quadratic_M2p24.md, valid for the kernel source
+# whose SHA-256 (of zero_order_forward_b200/csrc/zo_loss.cu) is recorded with it; reported
+# as null when the source has changed since the capture.
 LOSS_TRAFFIC = {"zo_loss_sha256": "522a5168ba23829afcb9f7887abebc28a98e7a44f0509c447d75d14b0bded121",
                 "bytes": 138.17e6}
 
@@ -254,19 +254,20 @@ def gpu_arm(args):
         total_s = float(t.item())
     value = args.steps / total_s  # steps of the one shared model
 
-    # dominant kernel: the loss pass (perturbation on load); 2n launches per probe phase
-    # (with N ranks the probe phase is not bracketed separately: time the kernel alone)
+    # dominant kernel: the loss pass (perturbation on load).  At one GPU the probe phase
+    # holds n launches of the pair kernel (L(theta +- eps z_i) from one pass over theta and
+    # D); with N ranks the phase is not bracketed separately: time the pair kernel alone.
     if world > 1:
         le = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         flush.zero_()
         le[0].record(stream)
-        for i in range(2 * n):
-            zo.zo_quad_loss(ctx, D, losses[0:1])
+        for i in range(n):
+            zo.zo_quad_loss_pair(ctx, D, i, EPS, losses[1:2], losses[2:3])
         le[1].record(stream)
         torch.cuda.synchronize()
         probe_ms = [le[0].elapsed_time(le[1])]
-    loss_us = 1e3 * statistics.mean(probe_ms) / (2 * n)
-    loss_bytes = 8 * M_FULL  # theta and D read once, fp32
+    loss_us = 1e3 * statistics.mean(probe_ms) / n
+    loss_bytes = 8 * M_FULL  # theta and D read once per pass, fp32
     achieved = loss_bytes / (loss_us * 1e-6) / 1e9
     upd_bytes = 8 * M_FULL  # theta read + written, fp32
 
@@ -321,7 +322,7 @@ def gpu_arm(args):
             cpu = {"value": (M_sample / M_FULL) / per, "unit": "steps/s", "cores": 1,
                    "kind": "oracle",
                    "sample": "2 oracle steps on the first 2^20 of 2^24 parameters; steps/s scaled by 1/16"}
-        launches_per_step = 1 + 2 * len(range(rank, n, world)) + 2
+        launches_per_step = (1 + n + 2) if world == 1 else (1 + 2 * len(range(rank, n, world)) + 2)
         line = {
             "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
@@ -330,7 +331,8 @@ def gpu_arm(args):
             "config": {"workload": WORKLOAD, "M": M_FULL, "n_pert": n, "eps": EPS, "lr": LR,
                        "damping": DAMPING, "parallelism": f"probe-parallel x{world}",
                        "l2": "flushed between steps (256 MiB write, untimed); theta+D = 128 MiB"},
-            "roofline": {"kernel": "quad_loss_kernel (perturbation on load, fp64 accumulation)",
+            "roofline": {"kernel": "quad_loss_kernel<pair> (L(theta +- eps z_i) in one pass, "
+                                   "perturbation on load, fp64 accumulation)",
                          "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "peak_kind": peak_kind,
                          "bytes_per_launch": loss_bytes, "avg_launch_us": loss_us,

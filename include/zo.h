@@ -187,6 +187,16 @@ zo_status zo_perturb_range(zo_ctx *ctx, int64_t first, int64_t count, void *dev_
  * Errors: ZO_ERR_INVALID, ZO_ERR_UNSUPPORTED (bf16 context), ZO_ERR_CUDA. */
 zo_status zo_quad_loss(zo_ctx *ctx, const float *D, double *loss_out, int accumulate);
 
+/* Both losses of probe `probe`, L(theta + eps z) -> *loss_plus and L(theta - eps z) ->
+ * *loss_minus (device doubles), from one pass over theta and D: the two perturbed vectors
+ * share every load.  Each loss is the sum over all M elements of its own perturbed terms in
+ * the same order as zo_quad_loss, so the results are bit-identical to perturb(+1) /
+ * zo_quad_loss / restore / perturb(-1) / zo_quad_loss / restore.  Requires the clean state
+ * (it does not change it); uses the current step counter.  zo_quad_step evaluates every
+ * probe this way.  Errors: as zo_quad_loss, ZO_ERR_STATE if perturbed. */
+zo_status zo_quad_loss_pair(zo_ctx *ctx, const float *D, int32_t probe, float eps,
+                            double *loss_plus, double *loss_minus);
+
 /* Cross-entropy of an MLP classifier in -> hidden (ReLU) -> out evaluated at
  * zo_live_params(ctx) (fp32 CUDA-core arithmetic, no TF32), flat parameter order
  * W1[hidden][in], b1[hidden], W2[out][hidden], b2[out] (M must match).
@@ -262,7 +272,8 @@ zo_status zo_get_precond(zo_ctx *ctx, int32_t n, double *g, double *c, double *w
 /* ------------------------------------------------------------------ step driver */
 
 /* One full step on the diagonal quadratic [LOOP]: clean loss (1.5-SPSA), then for each
- * probe the losses at +eps and -eps (perturbation on load), then zo_step.
+ * probe the losses at +eps and -eps (perturbation on load, both from one pass:
+ * zo_quad_loss_pair), then zo_step.
  *   D           device, M floats;  losses_out device, 2*n_pert+1 doubles receiving
  *               [L0, L+_0..L+_{n-1}, L-_0..L-_{n-1}] (L0 = 0 for 1SPSA).
  *   preconditioned  1 = 1.5-SPSA, 0 = 1SPSA.

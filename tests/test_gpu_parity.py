@@ -398,3 +398,33 @@ def test_quad_full_size_sampled(zo):
         assert (np.abs(got[win].astype(np.float64) - ref) <=
                 2 * np.spacing(np.abs(ref)) + 4 * 2.0 ** -24 * np.abs(pc["a"]).sum()).all()
     ctx.close()
+
+
+@pytest.mark.parametrize("M", [1, 5, 4096 + 3, 1 << 20, (1 << 22) + 17])
+def test_quad_loss_pair_is_bit_identical_to_two_passes(zo, M):
+    """zo_quad_loss_pair computes L(theta +- eps z) in one pass; each result must equal the
+    corresponding single-sign pass bit for bit (same terms, same order), and the oracle."""
+    th_np, D_np = synth.quad_problem(M, seed=12)
+    th, D = dev(th_np), dev(D_np)
+    ctx = zo.zo_create(th, seed=4)
+    zo.zo_set_step(ctx, 3)
+    out = torch.zeros(4, dtype=torch.float64, device="cuda")
+    zo.zo_quad_loss_pair(ctx, D, 9, 1e-3, out[0:1], out[1:2])
+    zo.zo_perturb(ctx, +1, 1e-3, 9)
+    zo.zo_quad_loss(ctx, D, out[2:3])
+    zo.zo_restore(ctx)
+    zo.zo_perturb(ctx, -1, 1e-3, 9)
+    zo.zo_quad_loss(ctx, D, out[3:4])
+    zo.zo_restore(ctx)
+    v = out.cpu().numpy()
+    assert v[0] == v[2] and v[1] == v[3]
+    refp = core.quad_loss(core.perturb(th_np, 4, 3, 9, +1, 1e-3), D_np)
+    refm = core.quad_loss(core.perturb(th_np, 4, 3, 9, -1, 1e-3), D_np)
+    assert abs(v[0] - refp) <= 1e-12 * refp and abs(v[1] - refm) <= 1e-12 * refm
+    with pytest.raises(zo.ZoError):  # needs the clean state
+        zo.zo_perturb(ctx, +1, 1e-3, 0)
+        try:
+            zo.zo_quad_loss_pair(ctx, D, 0, 1e-3, out[0:1], out[1:2])
+        finally:
+            zo.zo_restore(ctx)
+    ctx.close()

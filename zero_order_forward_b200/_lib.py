@@ -43,6 +43,7 @@ _SIGS = {
     "zo_restore": [_vp],
     "zo_perturb_range": [_vp, _i64, _i64, _vp],
     "zo_quad_loss": [_vp, _vp, _vp, _int],
+    "zo_quad_loss_pair": [_vp, _vp, _i32, _f32, _vp, _vp],
     "zo_mlp_loss": [_vp, _vp, _vp, _int, _int, _int, _int, _f64, _vp, _int],
     "zo_step": [_vp, _vp, _vp, _i32, _vp, _f32, _f32, _f32],
     "zo_update": [_vp, _vp, _i32],
@@ -203,6 +204,11 @@ def zo_perturb_range(ctx, first, count, out):
 
 def zo_quad_loss(ctx, D, loss_out, accumulate=False):
     return ctx.check(_L.zo_quad_loss(ctx.handle, _ptr(D), _ptr(loss_out), int(accumulate)))
+
+
+def zo_quad_loss_pair(ctx, D, probe, eps, loss_plus, loss_minus):
+    return ctx.check(_L.zo_quad_loss_pair(ctx.handle, _ptr(D), probe, eps, _ptr(loss_plus),
+                                          _ptr(loss_minus)))
 
 
 def zo_mlp_loss(ctx, X, labels, batch, n_in, n_hidden, n_out, scale, loss_out, accumulate=False):

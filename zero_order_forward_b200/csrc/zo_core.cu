@@ -324,6 +324,21 @@ zo_status zo_quad_loss(zo_ctx *ctx, const float *D, double *loss_out, int accumu
   return launch_quad_loss(ctx, probe_key(ctx), D, loss_out, accumulate, ctx->partials, ctx->counter);
 }
 
+zo_status zo_quad_loss_pair(zo_ctx *ctx, const float *D, int32_t probe, float eps,
+                            double *loss_plus, double *loss_minus) {
+  ZO_CHECK(check_ctx(ctx));
+  if (ctx->dtype != ZO_F32) return fail(ctx, ZO_ERR_UNSUPPORTED, "quadratic loss needs an fp32 context");
+  if (!D || !loss_plus || !loss_minus || !aligned16(D))
+    return fail(ctx, ZO_ERR_INVALID, "D must be a 16-byte aligned device pointer; outputs non-null");
+  if (probe < 0 || !(eps > 0.f) || !std::isfinite(eps)) return fail(ctx, ZO_ERR_INVALID, "bad probe or eps");
+  if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "pair evaluation needs the clean state");
+  ProbeKey pk = probe_key(ctx);
+  pk.sign = +1;
+  pk.probe = (uint32_t)probe;
+  pk.eps = eps;
+  return launch_quad_loss_pair(ctx, pk, D, loss_plus, loss_minus);
+}
+
 zo_status zo_mlp_loss(zo_ctx *ctx, const float *X, const int32_t *labels, int batch, int n_in,
                       int n_hidden, int n_out, double scale, double *loss_out, int accumulate) {
   ZO_CHECK(check_ctx(ctx));
@@ -381,16 +396,8 @@ zo_status zo_quad_step(zo_ctx *ctx, const float *D, int32_t n_pert, float eps, f
     ZO_CUDA(ctx, cudaMemsetAsync(L0, 0, sizeof(double), ctx->stream), "clear L0");
   }
   phase_mark(ctx, 1);
-  for (int32_t i = 0; i < n_pert; ++i) {
-    ZO_CHECK(zo_perturb(ctx, +1, eps, i));
-    zo_status st = zo_quad_loss(ctx, D, Lp + i, 0);
-    zo_restore(ctx);
-    ZO_CHECK(st);
-    ZO_CHECK(zo_perturb(ctx, -1, eps, i));
-    st = zo_quad_loss(ctx, D, Lm + i, 0);
-    zo_restore(ctx);
-    ZO_CHECK(st);
-  }
+  for (int32_t i = 0; i < n_pert; ++i)  // L(theta +- eps z_i) from one pass each
+    ZO_CHECK(zo_quad_loss_pair(ctx, D, i, eps, Lp + i, Lm + i));
   phase_mark(ctx, 2);
   const zo_status st = zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
   phase_mark(ctx, 3);

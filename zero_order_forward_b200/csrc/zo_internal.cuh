@@ -135,6 +135,8 @@ zo_status launch_pack(zo_ctx *ctx, uint32_t probe, int64_t first_byte, int64_t n
                       uint8_t *out);
 zo_status launch_quad_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *out,
                            int accumulate, double *partials, unsigned int *counter);
+zo_status launch_quad_loss_pair(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *out_plus,
+                                double *out_minus);
 zo_status launch_mlp_loss(zo_ctx *ctx, const float *P, const float *X, const int32_t *y,
                           int batch, int n_in, int n_hidden, int n_out, double scale,
                           double *out, int accumulate);

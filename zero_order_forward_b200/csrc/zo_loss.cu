@@ -36,13 +36,16 @@ __device__ double block_sum(double v) {
   return v;
 }
 
-// Block `blockIdx.x` contributes `v` (valid in thread 0); the last block writes
-// out = (accumulate ? out : 0) + scale * sum(partials[0..gridDim.x)) and re-arms counter.
-__device__ void finish_reduction(double v, double *partials, unsigned int *counter,
-                                 double *out, int accumulate, double scale) {
+// Block `blockIdx.x` contributes v[0..NV) (valid in thread 0); the last block writes
+// out[k] = (accumulate ? out[k] : 0) + scale * sum_b partials[k][b] for each k, summing
+// the blocks in index order, and re-arms the counter.
+template <int NV>
+__device__ void finish_reduction_n(const double v[NV], double *partials, unsigned int *counter,
+                                   double *const out[NV], int accumulate, double scale) {
   __shared__ bool last;
   if (threadIdx.x == 0) {
-    partials[blockIdx.x] = v;
+#pragma unroll
+    for (int k = 0; k < NV; ++k) partials[k * gridDim.x + blockIdx.x] = v[k];
     __threadfence();
     const unsigned int ticket = atomicAdd(counter, 1u);
     last = (ticket == gridDim.x - 1);
@@ -50,14 +53,24 @@ __device__ void finish_reduction(double v, double *partials, unsigned int *count
   __syncthreads();
   if (!last) return;
   __threadfence();
-  double s = 0.0;
-  for (unsigned int i = threadIdx.x; i < gridDim.x; i += blockDim.x) s += __ldcg(partials + i);
-  s = block_sum(s);
-  if (threadIdx.x == 0) {
-    const double prev = accumulate ? *out : 0.0;
-    *out = prev + scale * s;
-    *counter = 0u;
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    double s = 0.0;
+    for (unsigned int i = threadIdx.x; i < gridDim.x; i += blockDim.x)
+      s += __ldcg(partials + k * gridDim.x + i);
+    s = block_sum(s);
+    if (threadIdx.x == 0) {
+      const double prev = accumulate ? *out[k] : 0.0;
+      *out[k] = prev + scale * s;
+    }
   }
+  if (threadIdx.x == 0) *counter = 0u;
+}
+
+__device__ void finish_reduction(double v, double *partials, unsigned int *counter,
+                                 double *out, int accumulate, double scale) {
+  double *const o[1] = {out};
+  finish_reduction_n<1>(&v, partials, counter, o, accumulate, scale);
 }
 
 // L = 1/2 sum_j D_j P_j^2 with P_j = rd(theta_j + s*eps*z_j) computed on load.
@@ -78,10 +91,14 @@ constexpr int kQGroups = kQChunk / kGroup;                    // Philox blocks p
 constexpr int kQStageBytes = 2 * kQChunk * 4 + kQGroups * 16;  // theta, D, Philox blocks
 constexpr int kQSmemBytes = kQStages * kQStageBytes + 2 * kQStages * 8;
 
+// PAIR: both losses of one probe, L(theta + eps z) into out and L(theta - eps z) into
+// out_minus, from one pass over theta and D (pk.sign must be +1); each sum follows exactly
+// the order of a single-sign pass, so the results are bit-identical to two passes.
+template <bool PAIR>
 __global__ void __launch_bounds__(kQThreads)
 quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, int64_t M,
                  ProbeKey pk, int64_t n_chunks, double *partials, unsigned int *counter,
-                 double *out, int accumulate, uint32_t *err) {
+                 double *out, double *out_minus, int accumulate, uint32_t *err) {
   extern __shared__ __align__(128) uint8_t qsm[];
   uint64_t *full = reinterpret_cast<uint64_t *>(qsm + kQStages * kQStageBytes);
   uint64_t *empty = full + kQStages;
@@ -99,6 +116,7 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
   const uint32_t step = pk.sign ? *pk.step : 0u;
   const float delta = pk.sign > 0 ? pk.eps : -pk.eps;
   double acc4[4] = {0.0, 0.0, 0.0, 0.0};
+  double accm4[4] = {0.0, 0.0, 0.0, 0.0};  // PAIR: the -eps loss
 
   if (warp == 0) {  // producer
     int it = 0, issued = 0;
@@ -178,7 +196,12 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
         for (int q = 0; q < 4; ++q) {
           const float p = pk.sign ? perturb_f32(tv[q], delta, (bits >> q) & 1u) : tv[q];
           const double pd = (double)p;
-          acc4[q] = __dadd_rn(acc4[q], __dmul_rn(__dmul_rn(0.5, (double)dv[q]), __dmul_rn(pd, pd)));
+          const double hd = __dmul_rn(0.5, (double)dv[q]);
+          acc4[q] = __dadd_rn(acc4[q], __dmul_rn(hd, __dmul_rn(pd, pd)));
+          if (PAIR) {
+            const double pm = (double)perturb_f32(tv[q], -delta, (bits >> q) & 1u);
+            accm4[q] = __dadd_rn(accm4[q], __dmul_rn(hd, __dmul_rn(pm, pm)));
+          }
         }
       }
       __syncwarp();
@@ -186,12 +209,20 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
     }
   }
   double acc = __dadd_rn(__dadd_rn(acc4[0], acc4[1]), __dadd_rn(acc4[2], acc4[3]));
+  double accm = __dadd_rn(__dadd_rn(accm4[0], accm4[1]), __dadd_rn(accm4[2], accm4[3]));
   // The next loss pass may start streaming now; the reduction scratch (partials, counter,
   // out) is touched only after the previous kernel in the stream has fully completed.
   tc::pdl_launch_dependents();
   tc::pdl_wait();
   acc = block_sum(acc);
-  finish_reduction(acc, partials, counter, out, accumulate, 1.0);
+  if (PAIR) {
+    accm = block_sum(accm);
+    const double v[2] = {acc, accm};
+    double *const o[2] = {out, out_minus};
+    finish_reduction_n<2>(v, partials, counter, o, accumulate, 1.0);
+  } else {
+    finish_reduction(acc, partials, counter, out, accumulate, 1.0);
+  }
 }
 
 constexpr int kMlpMax = 1024;
@@ -243,13 +274,16 @@ mlp_loss_kernel(const float *__restrict__ P, const float *__restrict__ X,
 
 }  // namespace
 
-zo_status launch_quad_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *out,
-                           int accumulate, double *partials, unsigned int *counter) {
+namespace {
+
+template <bool PAIR>
+zo_status launch_quad(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *out,
+                      double *out_minus, int accumulate, double *partials, unsigned int *counter) {
   const int64_t n_chunks = (ctx->M + kQChunk - 1) / kQChunk;
   int64_t blocks = n_chunks < (int64_t)kSmCount * 2 ? n_chunks : (int64_t)kSmCount * 2;
   static bool attr = false;
   if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(quad_loss_kernel,
+    const cudaError_t e = cudaFuncSetAttribute(quad_loss_kernel<PAIR>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes);
     if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "quad_loss_kernel attribute: %s", cudaGetErrorString(e));
     attr = true;
@@ -267,12 +301,24 @@ zo_status launch_quad_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, doub
   attr_pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr_pdl;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, quad_loss_kernel,
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, quad_loss_kernel<PAIR>,
                                            static_cast<const float *>(ctx->params), D, ctx->M, pk,
-                                           n_chunks, partials, counter, out, accumulate,
+                                           n_chunks, partials, counter, out, out_minus, accumulate,
                                            &ctx->dstate->flags);
   if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "quad_loss_kernel: %s", cudaGetErrorString(e));
   return check_launch(ctx, "quad_loss_kernel");
+}
+
+}  // namespace
+
+zo_status launch_quad_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *out,
+                           int accumulate, double *partials, unsigned int *counter) {
+  return launch_quad<false>(ctx, pk, D, out, nullptr, accumulate, partials, counter);
+}
+
+zo_status launch_quad_loss_pair(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *out_plus,
+                                double *out_minus) {
+  return launch_quad<true>(ctx, pk, D, out_plus, out_minus, 0, ctx->partials, ctx->counter);
 }
 
 zo_status launch_mlp_loss(zo_ctx *ctx, const float *P, const float *X, const int32_t *y,
