@@ -212,11 +212,14 @@ def gpu_arm(args):
     def apply_step(Lp, Lm, L0):
         zo.zo_step(ctx, Lp, Lm, n, L0, LR, EPS, DAMPING)
 
+    def pair_at(probe, out_plus, out_minus):
+        zo.zo_quad_loss_pair(ctx, D, probe, EPS, out_plus, out_minus)
+
     def one_step():
         if world > 1:  # probe-parallel: this rank's probes, loss all-gather, same update
             from zero_order_forward_b200 import dist as zdist
             zdist.probe_parallel_step(n, loss_at, lambda o: zo.zo_quad_loss(ctx, D, o),
-                                      apply_step, dev)
+                                      apply_step, dev, pair_at=pair_at)
         else:  # the native step driver: every launch of the step enqueued from C++
             zo.zo_quad_step(ctx, D, n, EPS, LR, DAMPING, True, losses)
 
@@ -295,7 +298,7 @@ def gpu_arm(args):
         D.copy_(D_host, non_blocking=True)
         from zero_order_forward_b200 import dist as zdist
         L0, Lp, Lm = zdist.probe_parallel_step(n, loss_at, lambda o: zo.zo_quad_loss(ctx, D, o),
-                                               apply_step, dev)
+                                               apply_step, dev, pair_at=pair_at)
         L_host.copy_(torch.cat([L0, Lp, Lm]))  # synchronous device -> host read
     e2e_step()  # staging allocation
     if world > 1:

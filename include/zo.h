@@ -376,6 +376,15 @@ zo_status zo_model_step(zo_model *m, const int32_t *tokens, const int32_t *label
 zo_status zo_gemm_bf16(zo_ctx *ctx, const void *A, const void *B, const void *bias, void *out,
                        int32_t M, int32_t N, int32_t K, int32_t ldo, int32_t epilogue);
 
+/* Test hook for the bounded waits of the tensor-core pipeline: runs zo_gemm_bf16 (no
+ * bias, bf16 output) with the first stage's expected transaction count 16 bytes larger than
+ * what its loads deliver, so that stage's barrier is never satisfied.  Every waiter gives
+ * up after about 2 s, the kernel raises ZO_FLAG_TIMEOUT, lets its own loads land, waits for
+ * issued MMAs, frees its TMEM and returns; out is left unspecified.  zo_sync then reports
+ * ZO_ERR_TIMEOUT and the context remains usable.  No fault, trap or unbounded wait. */
+zo_status zo_debug_gemm_timeout(zo_ctx *ctx, const void *A, const void *B, void *out, int32_t M,
+                                int32_t N, int32_t K);
+
 /* Causal multi-head attention: qkv device bf16 [batch*seq][3*d_model] (q, k, v at column
  * offsets 0, d, 2d; head h at +h*hd), out device bf16 [batch*seq][d_model];
  * softmax(q.k^T / sqrt(hd)) over keys <= query, hd = d_model/n_heads in {64, 128}. */

@@ -237,3 +237,24 @@ def test_opt125m_full_size_sampled(zo):
     assert abs(got[1] - ref1) <= 2e-2 * abs(ref1)
     model.close()
     ctx.close()
+
+
+def test_bounded_wait_expiry_is_reported_and_context_survives(zo):
+    """A pipeline barrier that is never satisfied (test hook: 16 bytes more expected than
+    the loads deliver) makes every waiter give up after ~2 s: ZO_ERR_TIMEOUT is reported by
+    zo_sync, and the same context then runs a correct GEMM."""
+    th = torch.zeros(1024, dtype=torch.bfloat16, device="cuda")
+    ctx = zo.zo_create(th, seed=0)
+    r = np.random.default_rng(5)
+    A = bf16(r.standard_normal((128, 64)))
+    B = bf16(r.standard_normal((128, 64)))
+    out = torch.zeros((128, 128), dtype=torch.bfloat16, device="cuda")
+    zo.zo_debug_gemm_timeout(ctx, A, B, out, 128, 128, 64)
+    with pytest.raises(zo.ZoError) as ei:
+        zo.zo_sync(ctx)
+    assert ei.value.status == zo.ZO_ERR_TIMEOUT
+    zo.zo_gemm_bf16(ctx, A, B, None, out, 128, 128, 64, 128, 0)
+    assert zo.zo_sync(ctx) == 0
+    ref = f64(A) @ f64(B).T
+    assert np.all(np.abs(f64(out) - ref) <= 2.0 ** -8 * (np.abs(ref) + np.sqrt(np.mean(ref ** 2))))
+    ctx.close()

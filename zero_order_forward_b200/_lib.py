@@ -62,6 +62,7 @@ _SIGS = {
     "zo_model_step": [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _f32, _f32, _f32, _int, _vp],
     "zo_gemm_bf16": [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32],
     "zo_attention": [_vp, _vp, _vp, _i32, _i32, _i32, _i32],
+    "zo_debug_gemm_timeout": [_vp, _vp, _vp, _vp, _i32, _i32, _i32],
     "zo_layernorm": [_vp, _vp, _vp, _vp, _vp, _i32, _i32],
 }
 for _name, _args in _SIGS.items():
@@ -355,3 +356,7 @@ def zo_phase_times(ctx, n_steps):
     ms = np.zeros((n_steps, 3), np.float32)
     ctx.check(_L.zo_phase_times(ctx.handle, n_steps, ms.ctypes.data))
     return ms
+
+
+def zo_debug_gemm_timeout(ctx, A, B, out, M, N, K):
+    return ctx.check(_L.zo_debug_gemm_timeout(ctx.handle, _ptr(A), _ptr(B), _ptr(out), M, N, K))

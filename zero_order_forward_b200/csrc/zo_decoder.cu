@@ -25,7 +25,7 @@
 namespace zo {
 
 zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bias, void *out,
-                      int M, int N, int K, int ldo, int epi);
+                      int M, int N, int K, int ldo, int epi, uint32_t extra_tx = 0);
 zo_status launch_attention(zo_ctx *ctx, const uint16_t *qkv, uint16_t *out, int B, int S, int H,
                            int d);
 
@@ -448,6 +448,14 @@ zo_status zo_gemm_bf16(zo_ctx *ctx, const void *A, const void *B, const void *bi
   ctx->err.clear();
   if (!A || !B || !out) return fail(ctx, ZO_ERR_INVALID, "null gemm operand");
   return launch_gemm(ctx, A, B, bias, out, M, N, K, ldo, epilogue);
+}
+
+zo_status zo_debug_gemm_timeout(zo_ctx *ctx, const void *A, const void *B, void *out, int32_t M,
+                                int32_t N, int32_t K) {
+  if (!ctx) return ZO_ERR_INVALID;
+  ctx->err.clear();
+  if (!A || !B || !out) return fail(ctx, ZO_ERR_INVALID, "null gemm operand");
+  return launch_gemm(ctx, A, B, nullptr, out, M, N, K, N, ZO_EPI_BIAS_BF16, 16u);
 }
 
 zo_status zo_attention(zo_ctx *ctx, const void *qkv, void *out, int32_t batch, int32_t seq,

@@ -38,6 +38,7 @@ struct GemmArgs {
   void *out;             // bf16 [M][ldo] or fp32 [M][ldo]
   int ldo;
   uint32_t *err;         // device error word (ZO_FLAG_TIMEOUT raised on a bounded-wait expiry)
+  uint32_t extra_tx;     // 0; a test hook sets it so that the first stage never completes
 };
 
 __device__ __forceinline__ void load_bias32(const uint16_t *bias, int col0, int N, float b[32]) {
@@ -177,7 +178,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           *abort_flag = 1;
           break;
         }
-        tc::mbar_arrive_expect_tx(&full[s], S::kStageBytes);
+        tc::mbar_arrive_expect_tx(&full[s], S::kStageBytes + (issued == 0 ? args.extra_tx : 0u));
         tc::tma_load_2d(sA + s * S::kABytes, &tmA, &full[s], kb * kBK, tc0.m0);
         tc::tma_load_2d(sB + s * S::kBBytes, &tmB, &full[s], kb * kBK, tc0.n0);
         ++issued;
@@ -352,7 +353,7 @@ cudaError_t launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const CUten
 }  // namespace
 
 zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bias, void *out,
-                      int M, int N, int K, int ldo, int epi) {
+                      int M, int N, int K, int ldo, int epi, uint32_t extra_tx) {
   if (M < 1 || N < 1 || K < 1 || (K % 8) != 0 || (ldo % 8) != 0 || ldo < N)
     return fail(ctx, ZO_ERR_INVALID, "gemm: need M,N,K >= 1, K %% 8 == 0, ldo %% 8 == 0, ldo >= N");
   if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B) |
@@ -365,7 +366,7 @@ zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bia
   if (!make_map(&ta, A, M, K, kBM) || !make_map(&tb, B, N, K, wide ? 256 : 128) ||
       !make_out_map(&tcm, out, M, N, ldo, epi == ZO_EPI_RESID_F32))
     return fail(ctx, ZO_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
-  GemmArgs g{M, N, K, static_cast<const uint16_t *>(bias), out, ldo, &ctx->dstate->flags};
+  GemmArgs g{M, N, K, static_cast<const uint16_t *>(bias), out, ldo, &ctx->dstate->flags, extra_tx};
   cudaError_t e;
   if (wide) {
     if (epi == ZO_EPI_BIAS_BF16) e = launch_one<256, 4, ZO_EPI_BIAS_BF16>(ta, tb, tcm, g, ctx->stream);

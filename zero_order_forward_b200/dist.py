@@ -62,12 +62,13 @@ def gather_losses(local, n_pert, group=None):
 
 
 def probe_parallel_step(n_pert, loss_at, clean_loss, apply_step, device, dtype=torch.float64,
-                        group=None):
+                        group=None, pair_at=None):
     """One step with this rank's share of the probes.
 
     loss_at(sign, probe, out) writes L(theta + sign*eps*z_probe) into the 1-element tensor
-    `out`; clean_loss(out) writes L0 (every rank computes it: same theta, same data, same
-    value, no exchange); apply_step(Lp, Lm, L0) runs the preconditioner and the update.
+    `out`; pair_at(probe, out_plus, out_minus), if given, writes both signs at once instead;
+    clean_loss(out) writes L0 (every rank computes it: same theta, same data, same value, no
+    exchange); apply_step(Lp, Lm, L0) runs the preconditioner and the update.
     Returns (L0, Lp, Lm)."""
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
@@ -76,8 +77,11 @@ def probe_parallel_step(n_pert, loss_at, clean_loss, apply_step, device, dtype=t
     L0 = torch.zeros(1, dtype=dtype, device=device)
     clean_loss(L0)
     for j, i in enumerate(rank_probes(n_pert, rank, world)):
-        loss_at(+1, i, local[0, j:j + 1])
-        loss_at(-1, i, local[1, j:j + 1])
+        if pair_at is not None:
+            pair_at(i, local[0, j:j + 1], local[1, j:j + 1])
+        else:
+            loss_at(+1, i, local[0, j:j + 1])
+            loss_at(-1, i, local[1, j:j + 1])
     Lp, Lm = gather_losses(local, n_pert, group)
     apply_step(Lp, Lm, L0)
     return L0, Lp, Lm
