@@ -426,6 +426,7 @@ def decoder_arm(args):
         step()
     torch.cuda.synchronize()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    zo.zo_enable_phase_timing(ctx, args.steps)
     sampler = ClockSampler(local_rank) if rank == 0 else None
     ev[0].record(stream)
     for i in range(args.steps):
@@ -434,7 +435,11 @@ def decoder_arm(args):
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
     zo.zo_sync(ctx)
+    phases = zo.zo_phase_times(ctx, args.steps)
+    zo.zo_enable_phase_timing(ctx, 0)
     total_s = ev[0].elapsed_time(ev[-1]) / 1e3
+    upd_ms = float(phases[:, 2].mean())  # preconditioner (one CTA, ~5 us) + update
+    upd_bytes = 2 * 2 * M  # bf16 theta read + written once
     peak_mem = torch.cuda.max_memory_allocated(dev)
     free_b, tot_b = torch.cuda.mem_get_info(dev)
 
@@ -471,6 +476,19 @@ def decoder_arm(args):
         flops_layer += fl
         gemm[key] = {"shape": [Mm, N, K], "avg_launch_us": us, "tflops": fl / us / 1e6,
                      "frac_burst": fl / us / 1e6 / peak_b}
+    # causal attention at this micro-batch's shape (mma.sync path)
+    qkv = torch.randn(T * 3 * d, dtype=torch.bfloat16, device=dev)
+    att = torch.empty(T * d, dtype=torch.bfloat16, device=dev)
+    for _ in range(2):
+        zo.zo_attention(ctx, qkv, att, B, S, cfg["n_heads"], d)
+    ae = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ae[0].record(stream)
+    for _ in range(5):
+        zo.zo_attention(ctx, qkv, att, B, S, cfg["n_heads"], d)
+    ae[1].record(stream)
+    torch.cuda.synchronize()
+    attn_us = 1e3 * ae[0].elapsed_time(ae[1]) / 5
+    attn_flops = 2.0 * B * cfg["n_heads"] * S * S * (d // cfg["n_heads"])  # causal half of 4BHS^2hd
     zo.zo_sync(ctx)
     gemm_us = sum(g["avg_launch_us"] for g in gemm.values())
     gemm_tflops = flops_layer / gemm_us / 1e6
@@ -493,6 +511,12 @@ def decoder_arm(args):
                      "unit": "TFLOP/s", "frac": gemm_tflops / peak_b, "peak_kind": peak_kind,
                      "flops_per_layer": flops_layer, "traffic": None},
         "gemm": gemm,
+        "attention": {"avg_launch_us": attn_us, "tflops": attn_flops / attn_us / 1e6},
+        "phases_ms": {"clean_loss": float(phases[:, 0].mean()),
+                      "probe_losses": float(phases[:, 1].mean()), "precond_update": upd_ms},
+        "kernels": {"update_kernel": {"n_pert": n, "bytes": upd_bytes,
+                                      "achieved_GBps": upd_bytes / (upd_ms * 1e-3) / 1e9,
+                                      "frac_hbm": upd_bytes / (upd_ms * 1e-3) / 1e9 / peaks()[0]}},
         "memory": {"peak_allocated_GB": peak_mem / 1e9, "device_used_GB": (tot_b - free_b) / 1e9},
         "clocks": clocks,
     }

@@ -5,7 +5,7 @@
 // Layout: qkv is the bf16 output of the fused QKV projection, [B*S][3*d] with q, k, v at
 // column offsets 0, d, 2d and head h at +h*hd; out is bf16 [B*S][d].
 //
-// One CTA (4 warps) per (64-query tile, head, sequence); each warp owns 16 query rows.
+// One CTA (8 warps) per (128-query tile, head, sequence); each warp owns 16 query rows.
 // Key/value tiles of 64 rows stream through shared memory (cp.async, double-buffered);
 // scores and the probability-weighted sum use bf16 mma.sync (m16n8k16, fp32 accumulate)
 // with an online softmax in fp32 (running max and sum per row).  Attention is a few per
@@ -15,7 +15,7 @@
 namespace zo {
 namespace {
 
-constexpr int kQT = 64, kKT = 64, kThreads = 128;
+constexpr int kQT = 128, kKT = 64, kThreads = 256;  // 8 warps x 16 query rows
 
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool valid) {
   const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
@@ -48,6 +48,13 @@ __device__ __forceinline__ void mma16816(float d[4], const uint32_t a[4], uint32
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// 2^x via the multi-function unit (max error ~2 ulp; the probabilities are rounded to bf16).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return (uint32_t)f32_to_bf16_bits(lo) | ((uint32_t)f32_to_bf16_bits(hi) << 16);
 }
@@ -55,8 +62,9 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 template <int HD>
 struct AttnSmem {
   static constexpr int kStride = HD + 8;  // bf16 elements per smem row (16-byte pad)
-  static constexpr int kTile = kQT * kStride;
-  static constexpr int kBytes = (kTile + 4 * kTile) * 2;  // Q + 2 x (K, V)
+  static constexpr int kQTile = kQT * kStride;
+  static constexpr int kKVTile = kKT * kStride;
+  static constexpr int kBytes = (kQTile + 4 * kKVTile) * 2;  // Q + 2 x (K, V)
 };
 
 template <int HD>
@@ -67,9 +75,9 @@ attn_causal_kernel(const uint16_t *__restrict__ qkv, uint16_t *__restrict__ out,
   constexpr int ST = SM::kStride;
   extern __shared__ __align__(16) uint16_t sm[];
   uint16_t *sQ = sm;
-  // K and V tiles of buffer `buf` at sm + (1 + buf) * kTile and sm + (3 + buf) * kTile
-  auto sK = [&](int buf) { return sm + (1 + buf) * SM::kTile; };
-  auto sV = [&](int buf) { return sm + (3 + buf) * SM::kTile; };
+  // K and V tiles of buffer `buf` after the Q tile
+  auto sK = [&](int buf) { return sm + SM::kQTile + buf * SM::kKVTile; };
+  auto sV = [&](int buf) { return sm + SM::kQTile + (2 + buf) * SM::kKVTile; };
 
   const int qt = gridDim.x - 1 - blockIdx.x;  // heavy (late) query tiles first
   const int h = blockIdx.y, b = blockIdx.z;
@@ -81,8 +89,8 @@ attn_causal_kernel(const uint16_t *__restrict__ qkv, uint16_t *__restrict__ out,
   const uint16_t *Vg = qkv + 2 * d + h * HD;
   constexpr int kChunks = HD / 8;  // 16-byte chunks per row
 
-  auto load_tile = [&](uint16_t *dst, const uint16_t *src, int r0) {
-    for (int i = tid; i < kQT * kChunks; i += kThreads) {
+  auto load_tile = [&](uint16_t *dst, const uint16_t *src, int r0, int rows) {
+    for (int i = tid; i < rows * kChunks; i += kThreads) {
       const int r = i / kChunks, c = i % kChunks;
       const bool valid = r0 + r < S;
       const uint16_t *g = src + (row0 + (valid ? r0 + r : 0)) * ld + c * 8;
@@ -90,9 +98,9 @@ attn_causal_kernel(const uint16_t *__restrict__ qkv, uint16_t *__restrict__ out,
     }
   };
 
-  load_tile(sQ, Qg, qt * kQT);
-  load_tile(sK(0), Kg, 0);
-  load_tile(sV(0), Vg, 0);
+  load_tile(sQ, Qg, qt * kQT, kQT);
+  load_tile(sK(0), Kg, 0, kKT);
+  load_tile(sV(0), Vg, 0, kKT);
   cp_async_commit();
 
   float o[HD / 8][4];
@@ -103,12 +111,14 @@ attn_causal_kernel(const uint16_t *__restrict__ qkv, uint16_t *__restrict__ out,
   const int g = lane >> 2, t = lane & 3;
   const int qrow0 = qt * kQT + warp * 16;  // first query row of this warp
 
-  const int n_kt = qt + 1;  // causal: key tiles 0..qt
+  // causal: the key tiles that hold keys <= the last query row of this CTA
+  const int last_q = min(qt * kQT + kQT, S) - 1;
+  const int n_kt = last_q / kKT + 1;
   for (int kt = 0; kt < n_kt; ++kt) {
     const int buf = kt & 1;
     if (kt + 1 < n_kt) {
-      load_tile(sK(buf ^ 1), Kg, (kt + 1) * kKT);
-      load_tile(sV(buf ^ 1), Vg, (kt + 1) * kKT);
+      load_tile(sK(buf ^ 1), Kg, (kt + 1) * kKT, kKT);
+      load_tile(sV(buf ^ 1), Vg, (kt + 1) * kKT, kKT);
       cp_async_commit();
       cp_async_wait<1>();
     } else {
@@ -136,18 +146,25 @@ attn_causal_kernel(const uint16_t *__restrict__ qkv, uint16_t *__restrict__ out,
         mma16816(s[2 * jj + 1], qf[kk], kb[2], kb[3]);
       }
     }
-    // mask (causal on the diagonal tile, and keys beyond S) and online softmax
+    // mask (keys after the query, or beyond S: only on tiles that reach past the warp's
+    // first query row or the end of the sequence) and online softmax
     const int key0 = kt * kKT;
     float mnew[2] = {mrow[0], mrow[1]};
+    if (key0 + kKT - 1 > qrow0 || key0 + kKT > S) {
+#pragma unroll
+      for (int j = 0; j < kKT / 8; ++j) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int qr = qrow0 + g + (e >> 1) * 8;
+          const int kc = key0 + 8 * j + 2 * t + (e & 1);
+          if (kc > qr || kc >= S) s[j][e] = -INFINITY;
+        }
+      }
+    }
 #pragma unroll
     for (int j = 0; j < kKT / 8; ++j) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int qr = qrow0 + g + (e >> 1) * 8;
-        const int kc = key0 + 8 * j + 2 * t + (e & 1);
-        if (kc > qr || kc >= S) s[j][e] = -INFINITY;
-        mnew[e >> 1] = fmaxf(mnew[e >> 1], s[j][e]);
-      }
+      for (int e = 0; e < 4; ++e) mnew[e >> 1] = fmaxf(mnew[e >> 1], s[j][e]);
     }
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
@@ -159,7 +176,7 @@ attn_causal_kernel(const uint16_t *__restrict__ qkv, uint16_t *__restrict__ out,
     for (int r = 0; r < 2; ++r) {
       // rows that have seen no key yet keep m = -inf; use 0 as the shift then
       msc[r] = (mnew[r] == -INFINITY) ? 0.f : mnew[r] * scale_log2;
-      corr[r] = (mrow[r] == -INFINITY) ? 0.f : exp2f(mrow[r] * scale_log2 - msc[r]);
+      corr[r] = (mrow[r] == -INFINITY) ? 0.f : fast_exp2(mrow[r] * scale_log2 - msc[r]);
       mrow[r] = mnew[r];
       lrow[r] *= corr[r];
     }
@@ -174,7 +191,7 @@ attn_causal_kernel(const uint16_t *__restrict__ qkv, uint16_t *__restrict__ out,
       float p[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        p[e] = exp2f(s[j][e] * scale_log2 - msc[e >> 1]);
+        p[e] = fast_exp2(s[j][e] * scale_log2 - msc[e >> 1]);
         lrow[e >> 1] += p[e];
       }
       pf[j >> 1][(j & 1) * 2 + 0] = pack_bf16(p[0], p[1]);
