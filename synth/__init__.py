@@ -148,3 +148,47 @@ def opt_batch(cfg, batch, seq, seed=0, step=0):
                                                             dtype=np.int32)
     labels = rng(seed, "labels", step, batch).integers(0, 2, batch, dtype=np.int32)
     return tokens, labels
+
+
+# ---------------------------------------------------------------- Qwen3-shaped decoders
+
+QWEN_CONFIGS = {
+    # the pages' second model family (synthetic weights; the head is tied to the embedding)
+    "qwen3-1.7b": dict(family="qwen3", n_layers=28, d_model=2048, n_heads=16, n_kv_heads=8,
+                       head_dim=128, d_ffn=6144, vocab=151936, max_pos=4096, rope_theta=1.0e6,
+                       norm_eps=1e-6, class_ids=(1000, 2000)),
+    "qwen3-8b": dict(family="qwen3", n_layers=36, d_model=4096, n_heads=32, n_kv_heads=8,
+                     head_dim=128, d_ffn=12288, vocab=151936, max_pos=4096, rope_theta=1.0e6,
+                     norm_eps=1e-6, class_ids=(1000, 2000)),
+}
+
+
+def qwen_segments(cfg):
+    """(kind, count) runs of the flat Qwen3-shaped parameter vector: 'matrix' or 'gain'."""
+    d, H, Hk, e, f = (cfg["d_model"], cfg["n_heads"], cfg["n_kv_heads"], cfg["head_dim"],
+                      cfg["d_ffn"])
+    segs = [("matrix", cfg["vocab"] * d)]
+    for _ in range(cfg["n_layers"]):
+        segs += [("gain", d), ("matrix", (H + 2 * Hk) * e * d), ("gain", e), ("gain", e),
+                 ("matrix", d * H * e), ("gain", d), ("matrix", 2 * f * d), ("matrix", d * f)]
+    segs += [("gain", d)]
+    return segs
+
+
+def qwen_params(cfg, seed=0, varied=False):
+    """bf16 bits of the flat parameters: matrices N(0, 0.02), RMSNorm gains 1 (varied=True:
+    1 + N(0, 0.1), for parity tests)."""
+    segs = qwen_segments(cfg)
+    total = sum(n for _, n in segs)
+    r = rng(seed, "opt", total, 3)
+    out = np.empty(total, np.uint16)
+    o = 0
+    for kind, n in segs:
+        if kind == "matrix":
+            x = r.standard_normal(n, dtype=np.float32) * np.float32(0.02)
+        else:
+            x = (1.0 + r.standard_normal(n, dtype=np.float32) * np.float32(0.1) if varied
+                 else np.ones(n, np.float32))
+        out[o:o + n] = to_bf16_bits(x)
+        o += n
+    return out
