@@ -19,11 +19,15 @@
  *          (SC'11), the Philox-4x32 bijection with R = 10 rounds.
  *
  * Readings where the pages are silent (each restated in the design notes):
- *   - Probe bits: Philox4x32-10 with key = (seed low word, seed high word) and
- *     counter = (g low word, g high word, probe, step) where g = j >> 7 is the index
- *     of the 128-element group of element j.  Element j takes bit (j & 31) of output
- *     word ((j >> 5) & 3); bit 0 means z = +1, bit 1 means z = -1.  Packed probe byte
- *     q holds elements 8q..8q+7 (bit t <-> element 8q+t).
+ *   - Probe bits, 8 signs per byte [ABS] with the byte holding the signs of one element
+ *     under 8 consecutive probes: Philox4x32-10 with key = (seed low word, seed high
+ *     word) and counter = (g low word, g high word, p, step), where g = j >> 4 is the
+ *     index of the 16-element group of element j and p = probe >> 3 the index of the
+ *     8-probe octet.  The 16 output bytes (little-endian words w0..w3) belong to the 16
+ *     elements of the group: element j takes byte (j & 15), i.e. bits 8*(j & 3)..+7 of
+ *     word ((j >> 2) & 3); probe i takes bit (i & 7) of that byte; bit 0 means z = +1,
+ *     bit 1 means z = -1.  The packed form of ONE probe (an export format) holds its
+ *     elements 8q..8q+7 in byte q (bit t <-> element 8q+t).
  *   - Perturbation: P_j = rd(theta_j + s*eps*z_j) as one fp32 add with
  *     round-to-nearest-even; bf16 weights are widened exactly, added in fp32, and
  *     rounded to bf16 (RNE).  theta itself is never written by a perturbation.
@@ -70,11 +74,12 @@ void zo_oracle_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2],
   out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
 }
 
-/* The 128 sign bits of the group holding element j, for (seed, step, probe). */
+/* The 128 sign bits of the 16-element group holding element j under the probe octet
+ * holding `probe`, for (seed, step). */
 static void probe_group_words(uint64_t seed, uint32_t step, uint32_t probe, int64_t j,
                               uint32_t out[4]) {
-  uint64_t g = (uint64_t)j >> 7;
-  uint32_t ctr[4] = {(uint32_t)g, (uint32_t)(g >> 32), probe, step};
+  uint64_t g = (uint64_t)j >> 4;
+  uint32_t ctr[4] = {(uint32_t)g, (uint32_t)(g >> 32), probe >> 3, step};
   uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
   zo_oracle_philox4x32_10(ctr, key, out);
 }
@@ -83,7 +88,8 @@ static void probe_group_words(uint64_t seed, uint32_t step, uint32_t probe, int6
 int zo_oracle_probe_sign(uint64_t seed, uint32_t step, uint32_t probe, int64_t j) {
   uint32_t w[4];
   probe_group_words(seed, step, probe, j, w);
-  uint32_t bit = (w[(j >> 5) & 3] >> (j & 31)) & 1u;
+  uint32_t byte = (w[(j >> 2) & 3] >> (8 * (j & 3))) & 0xFFu;
+  uint32_t bit = (byte >> (probe & 7)) & 1u;
   return bit ? -1 : +1;
 }
 

@@ -85,23 +85,28 @@ def test_philox_counter_words_1_and_3_matter():
 
 # ------------------------------------------------------------------ probe layout and statistics
 
-def test_pack_layout_is_little_endian_group_bytes():
-    """Packed byte q = byte (q & 15) of the little-endian 16-byte Philox block of group q>>4,
-    with counter (group, 0, probe, step): rebuilt here from raw blocks by numpy's byte view."""
-    seed, step, probe, M = 0xABCDEF0123, 7, 5, 128 * 9 + 77
-    packed = core.pack_probe(seed, step, probe, M)
+def test_sign_layout_from_raw_philox_blocks():
+    """Element j, probe i: bit (i & 7) of byte (j & 15) of the little-endian 16-byte Philox
+    block with counter (j >> 4, 0, i >> 3, step); rebuilt here from raw blocks by numpy's
+    byte view, and the packed form of one probe holds element 8q + t in bit t of byte q."""
+    seed, step, M = 0xABCDEF0123, 7, 16 * 9 + 13
     key = [seed & 0xFFFFFFFF, seed >> 32]
-    groups = (M + 127) // 128
-    raw = np.concatenate([core.philox4x32_10([g, 0, probe, step], key) for g in range(groups)])
-    expect = raw.astype("<u4").view(np.uint8)[: (M + 7) // 8].copy()
-    tail_bits = M % 8
-    if tail_bits:
-        expect[-1] &= (1 << tail_bits) - 1
-    assert (packed == expect).all()
-    # and the per-element sign accessor agrees with the packed bits
-    for j in [0, 1, 31, 32, 127, 128, 129, M - 1]:
-        bit = (packed[j >> 3] >> (j & 7)) & 1
-        assert core.probe_sign(seed, step, probe, j) == (-1 if bit else 1)
+    groups = (M + 15) // 16
+    for probe in (0, 5, 8, 13, 70):
+        raw = np.concatenate([core.philox4x32_10([g, 0, probe >> 3, step], key)
+                              for g in range(groups)])
+        byte = raw.astype("<u4").view(np.uint8)[:M]
+        bits = (byte >> (probe & 7)) & 1
+        packed = core.pack_probe(seed, step, probe, M)
+        assert (np.unpackbits(packed, bitorder="little")[:M] == bits).all()
+        assert not np.unpackbits(packed, bitorder="little")[M:].any()  # padding bits are 0
+        for j in [0, 1, 3, 4, 15, 16, 17, M - 1]:
+            assert core.probe_sign(seed, step, probe, j) == (-1 if bits[j] else 1)
+    # the 8 probes of an octet share one block: byte j of that block is element j's signs
+    raw = core.philox4x32_10([2, 0, 1, step], key).astype("<u4").view(np.uint8)
+    for t in range(8):
+        z = [core.probe_sign(seed, step, 8 + t, 32 + b) for b in range(16)]
+        assert z == [-1 if (raw[b] >> t) & 1 else 1 for b in range(16)]
 
 
 def test_probe_statistics():
@@ -113,9 +118,9 @@ def test_probe_statistics():
         assert abs(Z[i].sum()) < 5 * sigma  # sum of M +/-1 has std sqrt(M)
         for k in range(i + 1, n):
             assert abs((Z[i] * Z[k]).sum()) < 5 * sigma  # agreement rate 1/2
-    # per bit position within the 128-element group
-    pos = Z[:, : M - M % 128].reshape(n, -1, 128).sum(axis=(0, 1))
-    assert np.abs(pos).max() < 5 * math.sqrt(n * M / 128) * 1.2
+    # per byte position within the 16-element group, for every bit position of the octet
+    pos = Z[:, : M - M % 16].reshape(n, -1, 16).sum(axis=1)  # [probe][byte position]
+    assert np.abs(pos).max() < 5 * math.sqrt(M / 16) * 1.2
     # different steps give independent probes
     Z2 = core.probe_signs(3, 12, 0, M).astype(np.int64)
     assert abs((Z[0] * Z2).sum()) < 5 * sigma
