@@ -6,4 +6,4 @@ numpy code (MLP and decoder losses, the step driver).  Only the tests, the smoke
 check and the benchmark's CPU-baseline leg may import it.  It shares no code with the
 CUDA library and neither imports the other; both take their inputs from `synth`.
 """
-from . import core, mlp, opt, qwen, step  # noqa: F401
+from . import core, lowrank, mlp, opt, qwen, step  # noqa: F401

@@ -10,12 +10,15 @@ Workload shapes follow the pages' setups as restated in the design notes:
   - MLP classifier 64 -> 256 (ReLU) -> 10, parameters N(0, 0.05), inputs N(0, 1),
     labels = argmax of a fixed random teacher MLP of the same shape;
   - OPT-shaped decoders: matrices and embeddings N(0, 0.02) in bf16, biases 0,
-    LayerNorm gains 1 and shifts 0, tokens uniform over the vocabulary, binary labels.
+    LayerNorm gains 1 and shifts 0, tokens uniform over the vocabulary, binary labels;
+  - Qwen3-shaped decoders: the same, with RMSNorm gains 1 and no biases;
+  - the conditioning-study quadratic: theta_0 ~ N(0, 1), D log-uniform on [1e-3, 1e-1],
+    eigenvalues of the rank-one terms tr(D) * (30, 10, 3, 1), a seed for their directions.
 """
 import numpy as np
 
 _TAGS = {"quad": 1, "mlp": 2, "teacher": 3, "batch": 4, "loss": 5, "coef": 6, "opt": 7,
-         "tokens": 8, "labels": 9, "theta": 10}
+         "tokens": 8, "labels": 9, "theta": 10, "lowrank": 11}
 
 
 def rng(seed, tag, *more):
@@ -37,6 +40,21 @@ def quad_problem(M, seed=0):
     theta = r.standard_normal(M, dtype=np.float32)
     D = (10.0 ** r.uniform(-3.0, 3.0, M)).astype(np.float32)
     return theta, D
+
+
+LOWRANK_SCALES = (30.0, 10.0, 3.0, 1.0)  # eigenvalues of the directions, in units of tr(D)
+
+
+def lowrank_problem(M, seed=0, rank=4):
+    """Conditioning-study quadratic: (theta_0 float32 [M], D float32 [M] log-uniform in
+    [1e-3, 1e-1], lam [rank] = tr(D) * LOWRANK_SCALES[:rank], vseed)."""
+    r = rng(seed, "lowrank", M)
+    theta = r.standard_normal(M, dtype=np.float32)
+    D = (10.0 ** r.uniform(-3.0, -1.0, M)).astype(np.float32)
+    tr = float(D.astype(np.float64).sum())
+    lam = [float(np.float32(tr * c)) for c in LOWRANK_SCALES[:rank]]
+    vseed = int(r.integers(1, 2 ** 63))
+    return theta, D, lam, vseed
 
 
 # ---------------------------------------------------------------- MLP classifier
