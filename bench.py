@@ -7,11 +7,11 @@ eps = 1e-3, lr = 4e-7, damping = 1e-3, 1.5-SPSA.  One step = clean loss + 2*n_pe
 perturbed losses + preconditioner + update, all through the C ABI of libzo.so.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload quadratic|opt-125m|opt-1.3b|opt-30b]
+                  [--workload quadratic|mlp|opt-125m|opt-1.3b|opt-30b|qwen3-1.7b|qwen3-8b]
 
-The decoder workloads (OPT-shaped, bf16 weights N(0, 0.02), uniform tokens, 2-class
-last-token loss) time whole 1.5-SPSA steps through zo_model_step and add a per-GEMM-shape
-breakdown of the tcgen05 projections against the measured bf16 peak.
+The decoder workloads (OPT- or Qwen3-shaped, bf16 weights N(0, 0.02), uniform tokens,
+2-class last-token loss) time whole 1.5-SPSA steps through zo_model_step and add a
+per-GEMM-shape breakdown of the tcgen05 projections against the measured bf16 peak.
 
 Prints ONE JSON line (rank 0).  With N > 1 (torchrun, one rank per GPU) the ranks share
 one model: every rank holds theta, evaluates its share of the probes (i = rank mod N), the
@@ -40,21 +40,28 @@ WORKLOAD = ("diagonal quadratic L=1/2*sum D_j theta_j^2, M=2^24 fp32, D log-unif
 FALLBACK_HBM_GBS = 6650.0
 
 # DRAM bytes (read + write) per launch of the loss-pair kernel from the ncu capture
-# summarised in profiles/quad_loss_kernel.quadratic_M2p24.md, valid for the kernel source
-# whose SHA-256 (of zero_order_forward_b200/csrc/zo_loss.cu) is recorded with it; reported
-# as null when the source has changed since the capture.
-LOSS_TRAFFIC = {"zo_loss_sha256": "522a5168ba23829afcb9f7887abebc28a98e7a44f0509c447d75d14b0bded121",
-                "bytes": 138.17e6}
+# summarised in profiles/quad_loss_kernel.quadratic_M2p24.md, valid for the kernel sources
+# whose SHA-256 (of zo_loss.cu, zo_internal.cuh and zo_tc.cuh, concatenated) is recorded
+# with it; reported as null when a source has changed since the capture.
+LOSS_TRAFFIC = {"sources_sha256": None, "bytes": None}
+LOSS_SOURCES = ("zo_loss.cu", "zo_internal.cuh", "zo_tc.cuh")
+
+
+def loss_sources_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    for name in LOSS_SOURCES:
+        with open(os.path.join(ROOT, "zero_order_forward_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def loss_traffic():
-    import hashlib
-    src = os.path.join(ROOT, "zero_order_forward_b200", "csrc", "zo_loss.cu")
     try:
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        h = loss_sources_sha256()
     except OSError:
         return None
-    return LOSS_TRAFFIC["bytes"] if h == LOSS_TRAFFIC["zo_loss_sha256"] else None
+    return LOSS_TRAFFIC["bytes"] if h == LOSS_TRAFFIC["sources_sha256"] else None
 
 
 FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS_SUSTAINED = 1590.0, 1400.0
@@ -64,6 +71,8 @@ DECODER_WORKLOADS = {
     "opt-125m": dict(batch=16, seq=256, n_micro=1, n_pert=32),
     "opt-1.3b": dict(batch=16, seq=512, n_micro=8, n_pert=160),
     "opt-30b": dict(batch=8, seq=2048, n_micro=1, n_pert=16),
+    "qwen3-1.7b": dict(batch=16, seq=512, n_micro=1, n_pert=32),
+    "qwen3-8b": dict(batch=8, seq=1024, n_micro=1, n_pert=16),
 }
 
 
@@ -369,16 +378,22 @@ def gpu_arm(args):
 
 # ------------------------------------------------------------------ decoder workloads
 
+def decoder_cfg(name):
+    import synth
+    return synth.QWEN_CONFIGS[name] if name.startswith("qwen") else synth.OPT_CONFIGS[name]
+
+
 def init_decoder_params(theta, cfg, seed):
-    """OPT-style synthetic initialisation on the device (too large for host numpy at 30B):
-    matrices N(0, 0.02) in bf16, biases 0, LayerNorm gains 1 and shifts 0."""
+    """Synthetic initialisation on the device (too large for host numpy at 30B): matrices
+    N(0, 0.02) in bf16, biases 0, norm gains 1 and shifts 0."""
     import torch
 
     import synth
     g = torch.Generator(device=theta.device)
     g.manual_seed(seed)
     o = 0
-    for kind, n in synth.opt_segments(cfg):
+    segs = synth.qwen_segments if cfg.get("family") == "qwen3" else synth.opt_segments
+    for kind, n in segs(cfg):
         seg = theta[o:o + n]
         if kind == "matrix":
             step = 1 << 28
@@ -401,7 +416,8 @@ def decoder_arm(args):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     name = args.workload
-    cfg = synth.OPT_CONFIGS[name]
+    cfg = decoder_cfg(name)
+    qwen = cfg.get("family") == "qwen3"
     w = dict(DECODER_WORKLOADS[name])
     if args.n_pert:
         w["n_pert"] = args.n_pert
@@ -452,12 +468,22 @@ def decoder_arm(args):
     torch.cuda.synchronize()
     fwd_ms = fe[0].elapsed_time(fe[1])
     peak_b, peak_s, peak_kind = bf16_peaks()
-    shapes = {"qkv": (T, 3 * d, d, 0), "out": (T, d, d, 2), "fc1": (T, f, d, 1), "fc2": (T, d, f, 2)}
+    H = cfg["n_heads"]
+    Hk, e = (cfg["n_kv_heads"], cfg["head_dim"]) if qwen else (H, d // H)
+    nq, na = (H + 2 * Hk) * e, H * e
+    if qwen:  # no biases; SwiGLU's gate and up projections are one GEMM of width 2f
+        shapes = {"qkv": (T, nq, d, 0), "out": (T, d, na, 2), "gate_up": (T, 2 * f, d, 0),
+                  "down": (T, d, f, 2)}
+    else:
+        shapes = {"qkv": (T, nq, d, 0), "out": (T, d, na, 2), "fc1": (T, f, d, 1),
+                  "fc2": (T, d, f, 2)}
     gemm = {}
-    A = torch.randn(T * max(d, f), dtype=torch.bfloat16, device=dev)
-    Wt = torch.randn(max(3 * d * d, f * d), dtype=torch.bfloat16, device=dev) * 0.02
-    bias = torch.zeros(max(3 * d, f), dtype=torch.bfloat16, device=dev)
-    out_b = torch.empty(T * max(3 * d, f), dtype=torch.bfloat16, device=dev)
+    A = torch.randn(T * max(K for _, _, K, _ in shapes.values()), dtype=torch.bfloat16, device=dev)
+    Wt = torch.randn(max(N * K for _, N, K, _ in shapes.values()), dtype=torch.bfloat16,
+                     device=dev) * 0.02
+    max_n = max(N for _, N, _, _ in shapes.values())
+    bias = None if qwen else torch.zeros(max_n, dtype=torch.bfloat16, device=dev)
+    out_b = torch.empty(T * max_n, dtype=torch.bfloat16, device=dev)
     out_f = torch.zeros(T * d, dtype=torch.float32, device=dev)
     flops_layer = 0
     for key, (Mm, N, K, epi) in shapes.items():
@@ -477,18 +503,18 @@ def decoder_arm(args):
         gemm[key] = {"shape": [Mm, N, K], "avg_launch_us": us, "tflops": fl / us / 1e6,
                      "frac_burst": fl / us / 1e6 / peak_b}
     # causal attention at this micro-batch's shape (mma.sync path)
-    qkv = torch.randn(T * 3 * d, dtype=torch.bfloat16, device=dev)
-    att = torch.empty(T * d, dtype=torch.bfloat16, device=dev)
+    qkv = torch.randn(T * nq, dtype=torch.bfloat16, device=dev)
+    att = torch.empty(T * na, dtype=torch.bfloat16, device=dev)
     for _ in range(2):
-        zo.zo_attention(ctx, qkv, att, B, S, cfg["n_heads"], d)
+        zo.zo_attention_gqa(ctx, qkv, att, B, S, H, Hk, e)
     ae = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     ae[0].record(stream)
     for _ in range(5):
-        zo.zo_attention(ctx, qkv, att, B, S, cfg["n_heads"], d)
+        zo.zo_attention_gqa(ctx, qkv, att, B, S, H, Hk, e)
     ae[1].record(stream)
     torch.cuda.synchronize()
     attn_us = 1e3 * ae[0].elapsed_time(ae[1]) / 5
-    attn_flops = 2.0 * B * cfg["n_heads"] * S * S * (d // cfg["n_heads"])  # causal half of 4BHS^2hd
+    attn_flops = 2.0 * B * H * S * S * e  # causal half of 4 B H S^2 e
     zo.zo_sync(ctx)
     gemm_us = sum(g["avg_launch_us"] for g in gemm.values())
     gemm_tflops = flops_layer / gemm_us / 1e6
@@ -522,6 +548,120 @@ def decoder_arm(args):
     }
     model.close()
     ctx.close()
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ conditioning study
+
+STUDY_M, STUDY_N, STUDY_STEPS = 1 << 20, 16, 400
+# learning rates in units of 2 n / tr(H) (the SPSA step's stability scale: the estimator's
+# noise grows with tr(H) / n), so the sweep means the same at any M
+STUDY_LR_UNITS = (0.035, 0.05, 0.07, 0.1, 0.14, 0.2, 0.28, 0.4)
+
+
+def lowrank_arm(args):
+    """The low-rank-plus-diagonal quadratic (per-probe curvature differs, so 1.5-SPSA's
+    weights do): steps/s of full 1.5-SPSA steps at M = 2^24, n = 64, and a learning-rate
+    sweep of 1SPSA against 1.5-SPSA at M = 2^20, n = 16, 400 steps each."""
+    import torch
+
+    import synth
+    import zero_order_forward_b200 as zo
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    hbm_peak, peak_kind = peaks()
+    stream = torch.cuda.current_stream(dev)
+    n = N_PERT
+    th_np, D_np, lam, vseed = synth.lowrank_problem(M_FULL, seed=0)
+    theta = torch.from_numpy(th_np).to(dev)
+    D = torch.from_numpy(D_np).to(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    losses = torch.zeros(2 * n + 1, dtype=torch.float64, device=dev)
+    ctx = zo.zo_create(theta, seed=0, stream=stream.cuda_stream)
+    lr_time = 1e-9  # timing run: any stable lr
+
+    def step():
+        zo.zo_lowrank_step(ctx, D, lam, vseed, n, EPS, lr_time, DAMPING, True, losses)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    zo.zo_enable_phase_timing(ctx, args.steps)
+    sampler = ClockSampler(0)
+    for k in range(args.steps):
+        flush.zero_()
+        evs[k][0].record(stream)
+        step()
+        evs[k][1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    zo.zo_sync(ctx)
+    ph = zo.zo_phase_times(ctx, args.steps)
+    zo.zo_enable_phase_timing(ctx, 0)
+    total_s = sum(e[0].elapsed_time(e[1]) for e in evs) / 1e3
+    loss_us = 1e3 * float(ph[:, 1].mean()) / n
+    achieved = 8 * M_FULL / (loss_us * 1e-6) / 1e9
+    ctx.close()
+
+    # the study: the same problem at M = 2^20, both methods, a learning-rate sweep
+    sth, sD, slam, svseed = synth.lowrank_problem(STUDY_M, seed=1)
+    trH = float(sD.astype(np.float64).sum()) + sum(slam)
+    unit = 2 * STUDY_N / trH
+    Dd = torch.from_numpy(sD).to(dev)
+    sl = torch.zeros(2 * STUDY_N + 1, dtype=torch.float64, device=dev)
+    out = torch.zeros(1, dtype=torch.float64, device=dev)
+    rows = []
+    for u in STUDY_LR_UNITS:
+        lr = u * unit
+        row = {"lr": lr, "lr_units": u}
+        for name, pre in (("1spsa", False), ("1.5spsa", True)):
+            th = torch.from_numpy(sth).to(dev)
+            c = zo.zo_create(th, seed=2, stream=stream.cuda_stream)
+            zo.zo_lowrank_loss(c, Dd, slam, svseed, out)
+            L_init = float(out.item())
+            skipped = 0
+            for k in range(STUDY_STEPS):
+                zo.zo_lowrank_step(c, Dd, slam, svseed, STUDY_N, EPS, lr, DAMPING, pre, sl)
+                if k % 50 == 49:  # diverged runs stop early (their losses overflow)
+                    zo.zo_lowrank_loss(c, Dd, slam, svseed, out)
+                    if not np.isfinite(out.item()) or out.item() > 1e6 * L_init:
+                        break
+            skipped = zo.zo_sync(c, raise_nonfinite=False)
+            zo.zo_lowrank_loss(c, Dd, slam, svseed, out)
+            ratio = float(out.item()) / L_init
+            ok = bool(np.isfinite(ratio)) and ratio < 1.0 and not skipped
+            row[name] = ratio if ok else None  # None: diverged
+            if pre and ok:  # the weights of the last step: their spread is the preconditioning
+                w = zo.zo_get_precond(c, STUDY_N)[2]
+                row["w_min_max"] = [float(w.min()), float(w.max())]
+            c.close()
+        rows.append(row)
+    stable = {m: max([r["lr"] for r in rows if r[m] is not None], default=None)
+              for m in ("1spsa", "1.5spsa")}
+    line = {
+        "metric": METRIC, "value": args.steps / total_s, "unit": "steps/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": "low-rank-plus-diagonal quadratic, M=2^24 fp32, rank 4, "
+                               f"n_pert={n}, 1.5-SPSA", "M": M_FULL, "n_pert": n,
+                   "l2": "flushed between steps (256 MiB write, untimed)"},
+        "roofline": {"kernel": "quad_loss_kernel<pair, rank 4>", "bound": "hbm",
+                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "peak_kind": peak_kind,
+                     "bytes_per_launch": 8 * M_FULL, "avg_launch_us": loss_us, "traffic": None},
+        "phases_ms": {"clean_loss": float(ph[:, 0].mean()), "probe_losses": float(ph[:, 1].mean()),
+                      "precond_update": float(ph[:, 2].mean())},
+        "study": {"M": STUDY_M, "n_pert": STUDY_N, "steps": STUDY_STEPS, "eps": EPS,
+                  "lr_unit": unit, "trace_H": trH,
+                  "damping": DAMPING, "alpha": 0.1, "eigenvalues_over_trD": list(synth.LOWRANK_SCALES),
+                  "final_over_initial_loss": rows, "largest_stable_lr": stable},
+        "gpu_launches": (1 + n + 2) * args.steps,
+        "clocks": clocks,
+    }
     print(json.dumps(line), flush=True)
     return 0
 
@@ -579,7 +719,7 @@ def main():
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per launch of the loss kernel, if measured")
     ap.add_argument("--workload", default="quadratic",
-                    choices=["quadratic", "mlp"] + sorted(DECODER_WORKLOADS))
+                    choices=["quadratic", "mlp", "lowrank"] + sorted(DECODER_WORKLOADS))
     ap.add_argument("--n-pert", type=int, default=None, help="override n_pert (decoder workloads)")
     args = ap.parse_args()
     if args.warmup < 3 and args.workload == "quadratic":
@@ -588,6 +728,8 @@ def main():
         return reference_arm(args)
     if args.workload == "mlp":
         return mlp_arm(args)
+    if args.workload == "lowrank":
+        return lowrank_arm(args)
     if args.workload != "quadratic":
         return decoder_arm(args)
     return gpu_arm(args)

@@ -21,17 +21,20 @@
  *         update -> repeat.
  *
  * Readings fixed by this library where the pages are silent:
- *   - Probe bits: Philox4x32-10 (Salmon et al., SC'11), key = (seed lo, seed hi),
- *     counter = (g lo, g hi, probe, step) with g = j >> 7; element j takes bit j & 31
- *     of word (j >> 5) & 3; bit 1 means z_j = -1.  Packed byte q holds elements
- *     8q..8q+7, bit t <-> element 8q+t.  Probes are regenerated, never stored.
+ *   - Probe bits, 8 signs per byte with a byte holding one element's signs under 8
+ *     consecutive probes: Philox4x32-10 (Salmon et al., SC'11), key = (seed lo,
+ *     seed hi), counter = (g lo, g hi, i >> 3, step) with g = j >> 4; element j of
+ *     probe i takes bit (i & 7) of byte (j & 15) of the little-endian 16-byte block
+ *     (word (j >> 2) & 3, bits 8 (j & 3)..); bit 1 means z_ij = -1.  Probes are
+ *     regenerated, never stored.  zo_pack_probe exports one probe with 8 elements per
+ *     byte: byte q holds elements 8q..8q+7, bit t <-> element 8q+t.
  *   - Perturbed value P_j = rd(theta_j + s*eps*z_j): one fp32 add (RNE); bf16 weights
  *     are widened, added in fp32 and rounded to bf16 (RNE).
  *   - g_i = (L+_i - L-_i)/(2 eps); c_i = (L+_i + L-_i - 2 L0)/eps^2;
  *     w_i = (|c_i| + damping)^(-alpha) (1SPSA: w_i = 1); a_i = lr*w_i*g_i/n, all in
  *     fp64, a_i rounded once to fp32.
- *   - theta' = rd(theta - sum_i a_i z_i) with a fixed fp32 order: probes in groups of
- *     8 (each group summed left to right from its first signed term), group sums
+ *   - theta' = rd(theta - sum_i a_i z_i) with a fixed fp32 order: probes in octets of
+ *     8 (each octet summed left to right from its first signed term), octet sums
  *     added left to right, one fp32 subtraction, one rounding to the storage type.
  *   - "In place" and "exact restore": theta is written only by zo_step/zo_update.
  *     A perturbation is a state of the context; kernels that need perturbed values
@@ -149,7 +152,8 @@ zo_status zo_phase_times(zo_ctx *ctx, int32_t n_steps, float *ms);
 /* ------------------------------------------------------------------ zo_rng */
 
 /* Write packed probe bytes [first_byte, first_byte + nbytes) of probe `probe` at the
- * current step into dev_out (device, nbytes bytes) [ABS: 8 signs per byte].  Bits of
+ * current step into dev_out (device, nbytes bytes), 8 elements of the one probe per byte
+ * (byte q: elements 8q..8q+7, bit t <-> element 8q+t).  Bits of
  * elements >= M are 0.  For tests and inspection: the training path regenerates probe
  * bits in registers and never stores them.
  * Errors: ZO_ERR_INVALID (probe < 0, range outside ceil(M/8) bytes, null dev_out). */
@@ -295,7 +299,48 @@ zo_status zo_mlp_step(zo_ctx *ctx, const float *X, const int32_t *labels, int ba
                       int n_in, int n_hidden, int n_out, int32_t n_pert, float eps,
                       float lr, float damping, int preconditioned, double *losses_out);
 
+/* ------------------------------------------------------------------ conditioning study */
+
+/* The low-rank-plus-diagonal quadratic, a synthetic loss whose curvature differs from probe
+ * to probe (on the diagonal quadratic every probe sees z^T D z = tr D, so 1.5-SPSA's
+ * weights are all equal; "Stanford's 1.5-SPSA Trains OPT-30B Without Backpropagation",
+ * section "Probe-Space Preconditioning", is about losses where they are not):
+ *   L = 1/2 sum_j D_j P_j^2 + 1/2 sum_{k < rank} (lam[k] / M) (v_k . P)^2,
+ * with v_k in {-1,+1}^M the generator's probe k at step 0 under seed vseed (so each adds
+ * the eigenvalue lam[k] along v_k / sqrt(M)).  fp32 context, D device fp32 [M] 16-byte
+ * aligned; every sum in fp64; the perturbation as in zo_quad_loss. */
+typedef struct {
+  int32_t rank;    /* 1..4 */
+  float lam[4];    /* eigenvalue of each direction (entries past rank ignored) */
+  uint64_t vseed;  /* seed of the directions */
+} zo_lowrank;
+
+/* L at the context's current state (clean or perturbed) into *loss_out (device fp64);
+ * accumulate adds to it. */
+zo_status zo_lowrank_loss(zo_ctx *ctx, const float *D, const zo_lowrank *q, double *loss_out,
+                          int accumulate);
+
+/* L(theta + eps z_probe) and L(theta - eps z_probe) from one pass (clean state only). */
+zo_status zo_lowrank_loss_pair(zo_ctx *ctx, const float *D, const zo_lowrank *q, int32_t probe,
+                               float eps, double *loss_plus, double *loss_minus);
+
+/* One full step on this loss, as zo_quad_step. */
+zo_status zo_lowrank_step(zo_ctx *ctx, const float *D, const zo_lowrank *q, int32_t n_pert,
+                          float eps, float lr, float damping, int preconditioned,
+                          double *losses_out);
+
 /* ------------------------------------------------------------------ decoder (zo_forward) */
+
+/* Two decoder families share this interface (cfg.family):
+ * OPT (ZO_FAMILY_OPT), described next, and Qwen3 (ZO_FAMILY_QWEN3): pre-RMSNorm layers
+ * (eps norm_eps), grouped-query attention (n_heads query heads of head_dim, n_kv_heads
+ * key/value heads) with per-head RMSNorm on queries and keys followed by rotary embeddings
+ * (rotate-half convention, base rope_theta), no projection biases, SwiGLU feed-forward
+ * silu(x Wg^T) * (x Wu^T) Wd^T, final RMSNorm, head tied to the token embedding; the same
+ * 2-class last-position loss.  Qwen3 flat parameter order (bf16; H, Hk, e = head_dim):
+ *   E[V][d], then per layer: in_norm[d], Wqkv[(H+2Hk)e][d] (rows q, k, v), q_norm[e],
+ *   k_norm[e], Wo[d][H e], post_norm[d], Wgu[2f][d] (rows gate, up), Wd[d][f];
+ *   then final_norm[d]. */
 
 /* Loss-only forward of an OPT-shaped decoder: pre-LN, learned positions (table of max_pos+2
  * rows, position s uses row s+2), ReLU FFN, biases on every projection, LayerNorm eps
@@ -308,14 +353,23 @@ zo_status zo_mlp_step(zo_ctx *ctx, const float *X, const int32_t *labels, int ba
  *   E[V][d], Pos[P][d], then per layer: ln1.g[d], ln1.b[d], Wqkv[3d][d] (rows q, k, v),
  *   bqkv[3d], Wo[d][d], bo[d], ln2.g[d], ln2.b[d], W1[f][d], b1[f], W2[d][f], b2[d];
  *   then lnf.g[d], lnf.b[d].  Linear weights are [out][in] (row-major, in contiguous). */
+/* Model families of zo_model_cfg.family. */
+#define ZO_FAMILY_OPT 0
+#define ZO_FAMILY_QWEN3 1
+
 typedef struct {
   int32_t n_layers;
   int32_t d_model;      /* multiple of 64 */
-  int32_t n_heads;      /* d_model / n_heads must be 64 or 128 */
+  int32_t n_heads;      /* OPT: d_model / n_heads must be 64 or 128 */
   int32_t d_ffn;        /* multiple of 8 */
   int32_t vocab;
   int32_t max_pos;      /* longest sequence */
   int32_t class_ids[2]; /* token ids whose last-position logits are the two classes */
+  int32_t family;       /* ZO_FAMILY_OPT or ZO_FAMILY_QWEN3 */
+  int32_t n_kv_heads;   /* Qwen3: key/value heads, dividing n_heads (OPT: ignored) */
+  int32_t head_dim;     /* Qwen3: 64 or 128 (OPT: ignored, d_model / n_heads) */
+  float rope_theta;     /* Qwen3: rotary base (OPT: ignored) */
+  float norm_eps;       /* Qwen3: RMSNorm epsilon (OPT: ignored, LayerNorm uses 1e-5) */
 } zo_model_cfg;
 
 typedef struct zo_model zo_model;
@@ -345,6 +399,13 @@ zo_status zo_model_loss(zo_model *m, const int32_t *tokens, const int32_t *label
                         int32_t batch, int32_t seq, double scale, double *loss_out,
                         int accumulate);
 
+/* Loss-only forwards (zo_model_loss, zo_model_step) run the last layer pruned to what the
+ * loss reads: keys and values for every position, everything else (queries, attention,
+ * output projection, feed-forward) for the last position of each sequence only.  On by
+ * default; enabled = 0 runs the full last layer (for comparisons).  Batches above
+ * min(max_tokens, 512) sequences and single-token sequences always run the full layer. */
+zo_status zo_model_set_pruning(zo_model *m, int enabled);
+
 /* Embedding plus the first n_layers_run layers of one micro-batch at the current state;
  * copies the fp32 residual stream [batch*seq][d_model] into h_out (device).  For
  * layer-by-layer parity checks. */
@@ -367,11 +428,16 @@ zo_status zo_model_step(zo_model *m, const int32_t *tokens, const int32_t *label
 #define ZO_EPI_BIAS_BF16 0  /* out bf16 = A.B^T + bias */
 #define ZO_EPI_RELU_BF16 1  /* out bf16 = max(A.B^T + bias, 0) */
 #define ZO_EPI_RESID_F32 2  /* out fp32 += A.B^T + bias (residual add) */
+#define ZO_EPI_SWIGLU_BF16 3 /* out bf16 [M][N] = silu(A.Bg^T) * (A.Bu^T), B = [Bg; Bu] [2N][K],
+                              * no bias (the Qwen3 gate and up projections in one GEMM) */
 
 /* out[M][ldo] = epilogue(A[M][K] . B[N][K]^T + bias[N]) on the tcgen05 tensor cores:
  * bf16 operands (device, row-major, K contiguous), fp32 accumulation in TMEM, bias bf16
  * (device, may be NULL).  K % 8 == 0, ldo % 8 == 0, ldo >= N, all pointers 16-byte
- * aligned; ragged M, N, K are handled (zero fill).  Enqueued on ctx's stream; a
+ * aligned; ragged M, N, K are handled (zero fill).  With ZO_EPI_SWIGLU_BF16, B holds 2N
+ * rows (gate rows, then up rows), N is the output width and bias must be NULL; the gate
+ * and up products of a tile share one TMEM accumulator and are combined in fp32 before the
+ * single bf16 rounding.  Enqueued on ctx's stream; a
  * pipeline stall beyond the bounded wait raises ZO_FLAG_TIMEOUT (seen by zo_sync). */
 zo_status zo_gemm_bf16(zo_ctx *ctx, const void *A, const void *B, const void *bias, void *out,
                        int32_t M, int32_t N, int32_t K, int32_t ldo, int32_t epilogue);
@@ -390,6 +456,19 @@ zo_status zo_debug_gemm_timeout(zo_ctx *ctx, const void *A, const void *B, void 
  * softmax(q.k^T / sqrt(hd)) over keys <= query, hd = d_model/n_heads in {64, 128}. */
 zo_status zo_attention(zo_ctx *ctx, const void *qkv, void *out, int32_t batch, int32_t seq,
                        int32_t n_heads, int32_t d_model);
+
+/* Grouped-query causal attention (the Qwen3 layer): qkv device bf16
+ * [batch*seq][(n_heads + 2 n_kv_heads) head_dim] with the n_heads query heads first, then
+ * the key heads, then the value heads; query head h reads key/value head
+ * h / (n_heads / n_kv_heads).  out device bf16 [batch*seq][n_heads head_dim].
+ * n_heads % n_kv_heads == 0, head_dim in {64, 128}, buffers 16-byte aligned. */
+zo_status zo_attention_gqa(zo_ctx *ctx, const void *qkv, void *out, int32_t batch, int32_t seq,
+                           int32_t n_heads, int32_t n_kv_heads, int32_t head_dim);
+
+/* out bf16 [rows][d] = x / sqrt(mean(x^2) + eps) * w (x fp32 [rows][d], w bf16 [d]), the
+ * Qwen3 RMSNorm; d <= 8192, d % 8 == 0, pointers 16-byte aligned. */
+zo_status zo_rmsnorm(zo_ctx *ctx, const float *x, const void *w, void *out, int32_t rows,
+                     int32_t d, float eps);
 
 /* out bf16 [rows][d] = LayerNorm(x fp32 [rows][d]) * gamma + beta (bf16 [d]), eps 1e-5,
  * d <= 8192, d % 8 == 0, pointers 16-byte aligned. */

@@ -258,3 +258,34 @@ def test_bounded_wait_expiry_is_reported_and_context_survives(zo):
     ref = f64(A) @ f64(B).T
     assert np.all(np.abs(f64(out) - ref) <= 2.0 ** -8 * (np.abs(ref) + np.sqrt(np.mean(ref ** 2))))
     ctx.close()
+
+
+@pytest.mark.parametrize("B,S", [(3, 100), (2, 1), (1, 127)])
+def test_pruned_last_layer_matches_full_layer(zo, B, S):
+    """The loss forward prunes the last layer to the last position of each sequence (keys
+    and values still for every position).  Same loss as the full layer, clean and perturbed:
+    the only difference is the last query's softmax probabilities, kept in fp32 by the
+    pruned kernel and rounded to bf16 by the full one (5e-3 relative); and both against the
+    oracle (2e-2)."""
+    cfg = TINY[0]
+    bits, theta, ctx, model, tokens, labels = _setup(zo, cfg, B, S)
+    dtok, dlab = torch.from_numpy(tokens).cuda(), torch.from_numpy(labels).cuda()
+    out = torch.zeros(4, dtype=torch.float64, device="cuda")
+    for i, (sign, probe) in enumerate(((0, 0), (+1, 2))):
+        if sign:
+            zo.zo_perturb(ctx, sign, 1e-3, probe)
+        zo.zo_model_set_pruning(model, True)
+        zo.zo_model_loss(model, dtok, dlab, B, S, 1.0 / B, out[2 * i:2 * i + 1])
+        zo.zo_model_set_pruning(model, False)
+        zo.zo_model_loss(model, dtok, dlab, B, S, 1.0 / B, out[2 * i + 1:2 * i + 2])
+        if sign:
+            zo.zo_restore(ctx)
+    assert zo.zo_sync(ctx) == 0
+    got = out.cpu().numpy()
+    for i, (sign, probe) in enumerate(((0, 0), (+1, 2))):
+        P = core.bf16_to_f32(core.perturb(bits, 0, 0, probe, sign, 1e-3) if sign else bits)
+        ref = oracle.opt.loss(P.astype(np.float64), cfg, tokens, labels)
+        assert abs(got[2 * i] - got[2 * i + 1]) <= 5e-3 * abs(got[2 * i + 1])
+        assert abs(got[2 * i] - ref) <= 2e-2 * abs(ref)
+    model.close()
+    ctx.close()

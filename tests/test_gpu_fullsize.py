@@ -21,14 +21,15 @@ PREFIX = 64
 
 
 def _device_params(cfg, seed):
-    """OPT-style synthetic weights generated on the device by torch (inputs, not outputs
-    of this library): matrices N(0, 0.02), biases 0, LayerNorm gains 1 / shifts 0."""
-    M = oracle.opt.param_count(cfg)
+    """Synthetic weights generated on the device by torch (inputs, not outputs of this
+    library): matrices N(0, 0.02), biases 0, norm gains 1 / shifts 0."""
+    qwen = cfg.get("family") == "qwen3"
+    M = (oracle.qwen if qwen else oracle.opt).param_count(cfg)
     theta = torch.empty(M, dtype=torch.bfloat16, device="cuda")
     g = torch.Generator(device="cuda")
     g.manual_seed(seed)
     o = 0
-    for kind, n in synth.opt_segments(cfg):
+    for kind, n in (synth.qwen_segments if qwen else synth.opt_segments)(cfg):
         seg = theta[o:o + n]
         if kind == "matrix":
             for a in range(0, n, 1 << 28):
@@ -71,6 +72,64 @@ def _prefix_oracle(theta, cfg, tokens0, n_layers, perturb=None, dtype=np.float64
     flat = core.bf16_to_f32(np.concatenate(parts)).astype(dtype)
     assert flat.size == oracle.opt.param_count(small)
     return oracle.opt.hidden_states(flat, small, np.arange(P)[None, :], dtype=dtype)[0]
+
+
+def _prefix_oracle_qwen(theta, cfg, tokens0, n_layers, perturb=None, dtype=np.float64):
+    """As _prefix_oracle, for the Qwen3-shaped layout (no position table)."""
+    lay = oracle.qwen.layout(cfg)
+    d, P = cfg["d_model"], len(tokens0)
+    small = dict(cfg, vocab=P, max_pos=P, n_layers=n_layers)
+    off_E = lay["E"][0]
+    rows = [_host_window(theta, off_E + int(t) * d, d) for t in tokens0]
+    first_layer = lay["L0.in_norm"][0]
+    layer_size = lay["L1.in_norm"][0] - first_layer
+    blocks = _host_window(theta, first_layer, n_layers * layer_size)
+    if perturb is not None:
+        seed, step, probe, sign, eps = perturb
+        rows = [core.perturb(r, seed, step, probe, sign, eps, j0=off_E + int(t) * d)
+                for r, t in zip(rows, tokens0)]
+        blocks = core.perturb(blocks, seed, step, probe, sign, eps, j0=first_layer)
+    flat = core.bf16_to_f32(np.concatenate(rows + [blocks, np.zeros(d, np.uint16)])).astype(dtype)
+    assert flat.size == oracle.qwen.param_count(small)
+    return oracle.qwen.hidden_states(flat, small, np.arange(P)[None, :], dtype=dtype)[0]
+
+
+# The Qwen3 shapes' bf16 activation error grows with depth (QK-norm makes attention
+# sharper): an fp64 forward that rounds to bf16 where the kernels do (norm outputs, QKV,
+# rotated q/k, probabilities, attention output, SwiGLU output) deviates from the exact one
+# by 0.69% after 1 layer, 0.84% after 2, 1.02% after 4, 1.21% after 8 and 1.34% after 12
+# at the Qwen3-1.7B layer shape; the GPU measures 0.70% .. 1.83% after 28.  Bound: 1e-2
+# up to 2 layers, 2.5e-2 for the full 28.
+@pytest.mark.parametrize("name,B,S,n_layers,perturbed,dtype,tol", [
+    ("qwen3-1.7b", 16, 512, 28, False, np.float32, 2.5e-2),
+    ("qwen3-1.7b", 16, 512, 2, True, np.float64, 1e-2),
+    ("qwen3-8b", 8, 1024, 1, False, np.float32, 1e-2)])
+def test_fullsize_qwen_prefix_hidden_state(zo, name, B, S, n_layers, perturbed, dtype, tol):
+    cfg = synth.QWEN_CONFIGS[name]
+    free, _ = torch.cuda.mem_get_info()
+    if free < oracle.qwen.param_count(cfg) * 2 + (4 << 30):
+        pytest.skip("not enough device memory for this workload")
+    theta = _device_params(cfg, seed=8)
+    ctx = zo.zo_create(theta, seed=8)
+    model = zo.zo_model_create(ctx, cfg, B * S)
+    tokens, _ = synth.opt_batch(cfg, B, S, seed=8)
+    dtok = torch.from_numpy(tokens).cuda()
+    h = torch.empty((B * S, cfg["d_model"]), dtype=torch.float32, device="cuda")
+    if perturbed:
+        zo.zo_perturb(ctx, +1, 1e-3, 9)
+    zo.zo_model_hidden(model, dtok, B, S, n_layers, h)
+    if perturbed:
+        zo.zo_restore(ctx)
+    assert zo.zo_sync(ctx) == 0
+    got = h[:PREFIX].cpu().numpy().astype(np.float64)
+    ref = _prefix_oracle_qwen(theta, cfg, tokens[0, :PREFIX], n_layers,
+                              perturb=(8, 0, 9, +1, 1e-3) if perturbed else None, dtype=dtype)
+    err = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert err <= tol, err
+    model.close()
+    ctx.close()
+    del theta
+    torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("name,B,S,n_layers,perturbed,dtype", [

@@ -61,3 +61,19 @@ def test_product_path_has_no_oracle_dependency():
             if fn.endswith((".py", ".cu", ".cuh", ".h")):
                 txt = open(os.path.join(dirpath, fn)).read()
                 assert "oracle" not in txt.lower(), os.path.join(dirpath, fn)
+
+
+def test_model_param_count_matches_both_layouts(zo):
+    """zo_model_param_count is host-only: the flat layouts of both decoder families agree in
+    size with the oracle's, and invalid configurations are rejected."""
+    import oracle
+    import synth
+    for cfg in synth.OPT_CONFIGS.values():
+        assert zo.zo_model_param_count(cfg) == oracle.opt.param_count(cfg)
+    for cfg in synth.QWEN_CONFIGS.values():
+        assert zo.zo_model_param_count(cfg) == oracle.qwen.param_count(cfg)
+    q = dict(synth.QWEN_CONFIGS["qwen3-1.7b"])
+    for bad in (dict(n_kv_heads=3), dict(head_dim=96), dict(rope_theta=0.0), dict(d_model=2000),
+                dict(d_ffn=6145), dict(class_ids=(0, q["vocab"]))):
+        with pytest.raises(zo.ZoError):
+            zo.zo_model_param_count({**q, **bad})

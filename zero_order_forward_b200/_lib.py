@@ -62,6 +62,12 @@ _SIGS = {
     "zo_model_step": [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _f32, _f32, _f32, _int, _vp],
     "zo_gemm_bf16": [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32],
     "zo_attention": [_vp, _vp, _vp, _i32, _i32, _i32, _i32],
+    "zo_attention_gqa": [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32],
+    "zo_model_set_pruning": [_vp, _int],
+    "zo_lowrank_loss": [_vp, _vp, _vp, _vp, _int],
+    "zo_lowrank_loss_pair": [_vp, _vp, _vp, _i32, _f32, _vp, _vp],
+    "zo_lowrank_step": [_vp, _vp, _vp, _i32, _f32, _f32, _f32, _int, _vp],
+    "zo_rmsnorm": [_vp, _vp, _vp, _vp, _i32, _i32, _f32],
     "zo_debug_gemm_timeout": [_vp, _vp, _vp, _vp, _i32, _i32, _i32],
     "zo_layernorm": [_vp, _vp, _vp, _vp, _vp, _i32, _i32],
 }
@@ -266,14 +272,35 @@ def zo_mlp_loss_noalloc(P, X, labels, batch, n_in, n_hidden, n_out, scale, loss_
 # ------------------------------------------------------------------ decoder
 
 
+ZO_FAMILY_OPT, ZO_FAMILY_QWEN3 = 0, 1
+
+
+class zo_lowrank(ctypes.Structure):
+    _fields_ = [("rank", _i32), ("lam", _f32 * 4), ("vseed", ctypes.c_uint64)]
+
+    @classmethod
+    def make(cls, lam, vseed):
+        lam = list(lam)
+        if not 1 <= len(lam) <= 4:
+            raise ValueError("rank must be 1..4")
+        return cls(len(lam), (_f32 * 4)(*(lam + [0.0] * (4 - len(lam)))), vseed)
+
+
 class zo_model_cfg(ctypes.Structure):
     _fields_ = [("n_layers", _i32), ("d_model", _i32), ("n_heads", _i32), ("d_ffn", _i32),
-                ("vocab", _i32), ("max_pos", _i32), ("class_ids", _i32 * 2)]
+                ("vocab", _i32), ("max_pos", _i32), ("class_ids", _i32 * 2), ("family", _i32),
+                ("n_kv_heads", _i32), ("head_dim", _i32), ("rope_theta", _f32),
+                ("norm_eps", _f32)]
 
     @classmethod
     def from_dict(cls, c):
+        qwen = c.get("family") == "qwen3"
         return cls(c["n_layers"], c["d_model"], c["n_heads"], c["d_ffn"], c["vocab"],
-                   c["max_pos"], (_i32 * 2)(*c["class_ids"]))
+                   c["max_pos"], (_i32 * 2)(*c["class_ids"]),
+                   ZO_FAMILY_QWEN3 if qwen else ZO_FAMILY_OPT,
+                   c.get("n_kv_heads", c["n_heads"]),
+                   c.get("head_dim", c["d_model"] // c["n_heads"]),
+                   float(c.get("rope_theta", 0.0)), float(c.get("norm_eps", 0.0)))
 
 
 class Model:
@@ -310,6 +337,28 @@ def zo_model_create(ctx, cfg, max_tokens):
     return Model(h, ctx, cfg)
 
 
+def zo_lowrank_loss(ctx, D, lam, vseed, loss_out, accumulate=False):
+    q = zo_lowrank.make(lam, vseed)
+    return ctx.check(_L.zo_lowrank_loss(ctx.handle, _ptr(D), ctypes.byref(q), _ptr(loss_out),
+                                        1 if accumulate else 0))
+
+
+def zo_lowrank_loss_pair(ctx, D, lam, vseed, probe, eps, loss_plus, loss_minus):
+    q = zo_lowrank.make(lam, vseed)
+    return ctx.check(_L.zo_lowrank_loss_pair(ctx.handle, _ptr(D), ctypes.byref(q), probe, eps,
+                                             _ptr(loss_plus), _ptr(loss_minus)))
+
+
+def zo_lowrank_step(ctx, D, lam, vseed, n_pert, eps, lr, damping, preconditioned, losses_out):
+    q = zo_lowrank.make(lam, vseed)
+    return ctx.check(_L.zo_lowrank_step(ctx.handle, _ptr(D), ctypes.byref(q), n_pert, eps, lr,
+                                        damping, 1 if preconditioned else 0, _ptr(losses_out)))
+
+
+def zo_model_set_pruning(model, enabled):
+    return model.ctx.check(_L.zo_model_set_pruning(model.handle, 1 if enabled else 0))
+
+
 def zo_model_destroy(model):
     model.close()
 
@@ -339,6 +388,15 @@ def zo_gemm_bf16(ctx, A, B, bias, out, M, N, K, ldo, epilogue):
 def zo_attention(ctx, qkv, out, batch, seq, n_heads, d_model):
     return ctx.check(_L.zo_attention(ctx.handle, _ptr(qkv), _ptr(out), batch, seq, n_heads,
                                      d_model))
+
+
+def zo_attention_gqa(ctx, qkv, out, batch, seq, n_heads, n_kv_heads, head_dim):
+    return ctx.check(_L.zo_attention_gqa(ctx.handle, _ptr(qkv), _ptr(out), batch, seq, n_heads,
+                                         n_kv_heads, head_dim))
+
+
+def zo_rmsnorm(ctx, x, w, out, rows, d, eps):
+    return ctx.check(_L.zo_rmsnorm(ctx.handle, _ptr(x), _ptr(w), _ptr(out), rows, d, eps))
 
 
 def zo_layernorm(ctx, x, gamma, beta, out, rows, d):

@@ -382,6 +382,66 @@ zo_status zo_get_precond(zo_ctx *ctx, int32_t n, double *g, double *c, double *w
   return ZO_OK;
 }
 
+namespace {
+zo_status check_lowrank(zo_ctx *ctx, const float *D, const zo_lowrank *q, float lam[4]) {
+  if (ctx->dtype != ZO_F32) return fail(ctx, ZO_ERR_UNSUPPORTED, "quadratic loss needs an fp32 context");
+  if (!D || !aligned16(D)) return fail(ctx, ZO_ERR_INVALID, "D must be a 16-byte aligned device pointer");
+  if (!q || q->rank < 1 || q->rank > 4) return fail(ctx, ZO_ERR_INVALID, "rank must be 1..4");
+  for (int k = 0; k < 4; ++k) {
+    lam[k] = k < q->rank ? q->lam[k] : 0.f;
+    if (!std::isfinite(lam[k])) return fail(ctx, ZO_ERR_INVALID, "non-finite eigenvalue");
+  }
+  return ZO_OK;
+}
+}  // namespace
+
+zo_status zo_lowrank_loss(zo_ctx *ctx, const float *D, const zo_lowrank *q, double *loss_out,
+                          int accumulate) {
+  ZO_CHECK(check_ctx(ctx));
+  float lam[4];
+  ZO_CHECK(check_lowrank(ctx, D, q, lam));
+  if (!loss_out) return fail(ctx, ZO_ERR_INVALID, "null loss_out");
+  return launch_lowrank_loss(ctx, probe_key(ctx), D, lam, q->vseed, loss_out, nullptr, accumulate);
+}
+
+zo_status zo_lowrank_loss_pair(zo_ctx *ctx, const float *D, const zo_lowrank *q, int32_t probe,
+                               float eps, double *loss_plus, double *loss_minus) {
+  ZO_CHECK(check_ctx(ctx));
+  float lam[4];
+  ZO_CHECK(check_lowrank(ctx, D, q, lam));
+  if (!loss_plus || !loss_minus) return fail(ctx, ZO_ERR_INVALID, "null output");
+  if (probe < 0 || !(eps > 0.f) || !std::isfinite(eps)) return fail(ctx, ZO_ERR_INVALID, "bad probe or eps");
+  if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "pair evaluation needs the clean state");
+  ProbeKey pk = probe_key(ctx);
+  pk.sign = +1;
+  pk.probe = (uint32_t)probe;
+  pk.eps = eps;
+  return launch_lowrank_loss(ctx, pk, D, lam, q->vseed, loss_plus, loss_minus, 0);
+}
+
+zo_status zo_lowrank_step(zo_ctx *ctx, const float *D, const zo_lowrank *q, int32_t n_pert,
+                          float eps, float lr, float damping, int preconditioned,
+                          double *losses_out) {
+  ZO_CHECK(check_ctx(ctx));
+  ZO_CHECK(check_step_args(ctx, n_pert, lr, eps, damping));
+  if (!losses_out) return fail(ctx, ZO_ERR_INVALID, "null losses_out");
+  if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "step while perturbed");
+  double *L0 = losses_out, *Lp = losses_out + 1, *Lm = losses_out + 1 + n_pert;
+  phase_mark(ctx, 0);
+  if (preconditioned) {
+    ZO_CHECK(zo_lowrank_loss(ctx, D, q, L0, 0));
+  } else {
+    ZO_CUDA(ctx, cudaMemsetAsync(L0, 0, sizeof(double), ctx->stream), "clear L0");
+  }
+  phase_mark(ctx, 1);
+  for (int32_t i = 0; i < n_pert; ++i)
+    ZO_CHECK(zo_lowrank_loss_pair(ctx, D, q, i, eps, Lp + i, Lm + i));
+  phase_mark(ctx, 2);
+  const zo_status st = zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
+  phase_mark(ctx, 3);
+  return st;
+}
+
 zo_status zo_quad_step(zo_ctx *ctx, const float *D, int32_t n_pert, float eps, float lr,
                        float damping, int preconditioned, double *losses_out) {
   ZO_CHECK(check_ctx(ctx));

@@ -1,6 +1,7 @@
-// zo_decoder.cu -- loss-only forward of an OPT-shaped decoder (pre-LN, learned positions
-// with offset 2, ReLU FFN, biases everywhere, head tied to the token embedding) and the
-// model-level C ABI.
+// zo_decoder.cu -- loss-only forward of the two decoder families and the model-level C ABI:
+// OPT-shaped (pre-LN, learned positions with offset 2, ReLU FFN, biases everywhere) and
+// Qwen3-shaped (pre-RMSNorm, grouped-query attention with QK-norm and rotary embeddings,
+// SwiGLU FFN, no biases); both tie the head to the token embedding.
 //
 // Inference mode only ("Probe-Space Preconditioning for Fast and Stable Zero-Order
 // Training", abstract): each layer's activations overwrite the previous layer's, nothing is
@@ -12,13 +13,20 @@
 // parameters into one reusable layer window; the token/position embeddings, the final
 // LayerNorm and the tied head rows are perturbed on load.
 //
-// Flat parameter order (bf16), d = d_model, f = d_ffn, V = vocab, P = max_pos + 2:
+// OPT flat parameter order (bf16), d = d_model, f = d_ffn, V = vocab, P = max_pos + 2:
 //   E[V][d], Pos[P][d],
 //   per layer: ln1.g[d], ln1.b[d], Wqkv[3d][d], bqkv[3d], Wo[d][d], bo[d],
 //              ln2.g[d], ln2.b[d], W1[f][d], b1[f], W2[d][f], b2[d],
 //   final: lnf.g[d], lnf.b[d].
+// Qwen3 flat parameter order (bf16), H / Hk query / key-value heads of e features:
+//   E[V][d],
+//   per layer: in_norm[d], Wqkv[(H+2Hk)e][d], q_norm[e], k_norm[e], Wo[d][He], post_norm[d],
+//              Wgu[2f][d] (gate rows, then up rows), Wd[d][f],
+//   final: final_norm[d].
+#include <cmath>
 #include <cstring>
 #include <new>
+#include <vector>
 
 #include "zo_internal.cuh"
 
@@ -28,20 +36,63 @@ zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bia
                       int M, int N, int K, int ldo, int epi, uint32_t extra_tx = 0);
 zo_status launch_attention(zo_ctx *ctx, const uint16_t *qkv, uint16_t *out, int B, int S, int H,
                            int d);
+zo_status launch_attention_gqa(zo_ctx *ctx, const uint16_t *qkv, uint16_t *out, int B, int S,
+                               int H, int Hk, int hd);
+zo_status launch_rmsnorm(zo_ctx *ctx, const float *x, const uint16_t *w, uint16_t *y, int rows,
+                         int d, float eps);
+zo_status launch_qk_norm_rope(zo_ctx *ctx, uint16_t *x, int64_t ld, int hbeg, int hcount, int H,
+                              const uint16_t *qn, const uint16_t *kn, const float2 *rope, int64_t T,
+                              int S, int pos_fixed, int hd, float eps);
+zo_status launch_attention_last(zo_ctx *ctx, const uint16_t *q, int ldq, const uint16_t *qkv,
+                                uint16_t *out, int B, int S, int H, int Hk, int hd);
 
 struct Layout {
-  int64_t E, Pos, layers, layer_size, fin, total;
-  // offsets inside a layer block
+  int64_t E, Pos, layers, layer_size, fin, total;  // Pos = -1: no position table (Qwen3)
+  // offsets inside an OPT layer block
   int64_t ln1g, ln1b, wqkv, bqkv, wo, bo, ln2g, ln2b, w1, b1, w2, b2;
+  // offsets inside a Qwen3 layer block (wqkv and wo above are shared)
+  int64_t in_norm, q_norm, k_norm, post_norm, wgu, wd;
+  int64_t qkv_cols, attn_cols;  // width of the QKV projection output and of attention's
 };
 
-bool make_layout(const zo_model_cfg &c, Layout *L) {
-  if (c.n_layers < 1 || c.d_model < 64 || c.d_model % 64 || c.n_heads < 1 ||
-      c.d_model % c.n_heads || c.d_ffn < 8 || c.d_ffn % 8 || c.vocab < 2 || c.max_pos < 1 ||
-      c.class_ids[0] < 0 || c.class_ids[0] >= c.vocab || c.class_ids[1] < 0 ||
-      c.class_ids[1] >= c.vocab)
+bool common_cfg_ok(const zo_model_cfg &c) {
+  return c.n_layers >= 1 && c.d_model >= 64 && c.d_model % 64 == 0 && c.d_model <= 8192 &&
+         c.n_heads >= 1 && c.d_ffn >= 8 && c.d_ffn % 8 == 0 && c.vocab >= 2 && c.max_pos >= 1 &&
+         c.class_ids[0] >= 0 && c.class_ids[0] < c.vocab && c.class_ids[1] >= 0 &&
+         c.class_ids[1] < c.vocab;
+}
+
+bool make_qwen_layout(const zo_model_cfg &c, Layout *L) {
+  if (!common_cfg_ok(c) || c.n_kv_heads < 1 || c.n_heads % c.n_kv_heads ||
+      (c.head_dim != 64 && c.head_dim != 128) || !(c.rope_theta > 0.f) || !(c.norm_eps >= 0.f))
     return false;
+  const int64_t d = c.d_model, f = c.d_ffn, e = c.head_dim, H = c.n_heads, Hk = c.n_kv_heads;
+  L->E = 0;
+  L->Pos = -1;
+  L->layers = (int64_t)c.vocab * d;
+  int64_t o = 0;
+  L->in_norm = o; o += d;
+  L->wqkv = o; o += (H + 2 * Hk) * e * d;
+  L->q_norm = o; o += e;
+  L->k_norm = o; o += e;
+  L->wo = o; o += d * H * e;
+  L->post_norm = o; o += d;
+  L->wgu = o; o += 2 * f * d;
+  L->wd = o; o += d * f;
+  L->layer_size = o;
+  L->fin = L->layers + (int64_t)c.n_layers * o;
+  L->total = L->fin + d;
+  L->qkv_cols = (H + 2 * Hk) * e;
+  L->attn_cols = H * e;
+  return true;
+}
+
+bool make_layout(const zo_model_cfg &c, Layout *L) {
+  if (c.family == ZO_FAMILY_QWEN3) return make_qwen_layout(c, L);
+  if (c.family != ZO_FAMILY_OPT || !common_cfg_ok(c) || c.d_model % c.n_heads) return false;
   const int64_t d = c.d_model, f = c.d_ffn;
+  L->qkv_cols = 3 * d;
+  L->attn_cols = d;
   L->E = 0;
   L->Pos = (int64_t)c.vocab * d;
   L->layers = L->Pos + (int64_t)(c.max_pos + 2) * d;
@@ -79,8 +130,8 @@ __device__ __forceinline__ void load8_perturbed(const uint16_t *theta, int64_t j
     out[2 * t + 1] = __uint_as_float(w[t] & 0xFFFF0000u);
   }
   if (pk.sign) {
-    const uint4 b = probe_block((uint64_t)j >> 7, pk.probe, step, pk.k0, pk.k1);
-    const uint32_t bits = word_of(b, (int)((j >> 5) & 3)) >> (j & 31);
+    // j % 8 == 0: the 8 elements are one half of a 16-element group
+    const uint32_t bits = probe_group_bits((uint64_t)j >> 4, pk.probe, step, pk.k0, pk.k1) >> (j & 8);
     const float delta = pk.sign > 0 ? pk.eps : -pk.eps;
 #pragma unroll
     for (int t = 0; t < 8; ++t)
@@ -88,8 +139,9 @@ __device__ __forceinline__ void load8_perturbed(const uint16_t *theta, int64_t j
   }
 }
 
-// h[t][:] = P_E[token] + P_Pos[s + 2] (fp32), one block per token.  An out-of-range
-// token id writes NaN (the loss becomes non-finite and the step is skipped).
+// h[t][:] = P_E[token] + P_Pos[s + 2] (fp32), one block per token; without a position
+// table (pos_off < 0) h[t][:] = P_E[token].  An out-of-range token id writes NaN (the loss
+// becomes non-finite and the step is skipped).
 __global__ void __launch_bounds__(kRowThreads)
 embed_kernel(const uint16_t *__restrict__ theta, const int32_t *__restrict__ tokens, int S, int d,
              int vocab, int64_t pos_off, ProbeKey pk, float *__restrict__ h) {
@@ -105,9 +157,9 @@ embed_kernel(const uint16_t *__restrict__ theta, const int32_t *__restrict__ tok
       for (int i = 0; i < 8; ++i) hrow[c + i] = __int_as_float(0x7FC00000);
       continue;
     }
-    float e[8], p[8];
+    float e[8], p[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     load8_perturbed(theta, (int64_t)tok * d + c, pk, step, e);
-    load8_perturbed(theta, pos_off + (int64_t)(s + 2) * d + c, pk, step, p);
+    if (pos_off >= 0) load8_perturbed(theta, pos_off + (int64_t)(s + 2) * d + c, pk, step, p);
     float4 *o = reinterpret_cast<float4 *>(hrow + c);
     o[0] = make_float4(e[0] + p[0], e[1] + p[1], e[2] + p[2], e[3] + p[3]);
     o[1] = make_float4(e[4] + p[4], e[5] + p[5], e[6] + p[6], e[7] + p[7]);
@@ -189,34 +241,50 @@ layernorm_kernel(const float *__restrict__ x, const uint16_t *__restrict__ g,
 
 int ln_threads(int d) { return ((d / kLnVec + 31) / 32) * 32; }
 
-// Per sample: final LayerNorm of the last position, logits of the two class tokens through
-// the tied head, 2-class cross-entropy.  Parameters perturbed on load.
+// dst[b][:] = src[b * S + S - 1][:] (rows of row_bytes, a multiple of 16): the last
+// position of every sequence, for the pruned last layer.
+__global__ void __launch_bounds__(kRowThreads)
+gather_last_kernel(const uint8_t *__restrict__ src, uint8_t *__restrict__ dst, int64_t row_bytes,
+                   int S) {
+  const int64_t b = blockIdx.x;
+  const uint4 *from = reinterpret_cast<const uint4 *>(src + (b * S + S - 1) * row_bytes);
+  uint4 *to = reinterpret_cast<uint4 *>(dst + b * row_bytes);
+  for (int64_t i = threadIdx.x; i < row_bytes / 16; i += blockDim.x) to[i] = from[i];
+}
+
+// Per sample: final norm of the last position (LayerNorm with gain and bias at fin_off, or
+// with RMS = true RMSNorm with gain only), logits of the two class tokens through the tied
+// head, 2-class cross-entropy.  Parameters perturbed on load.
+template <bool RMS>
 __global__ void __launch_bounds__(kRowThreads)
 head_ce_kernel(const float *__restrict__ h, const uint16_t *__restrict__ theta, int S, int d,
                int64_t fin_off, int id0, int id1, const int32_t *__restrict__ labels,
                ProbeKey pk, double *partials, unsigned int *counter, double *out, int accumulate,
-               double scale) {
+               double scale, float eps) {
   __shared__ float red[kRowThreads / 32];
   __shared__ bool last;
   const int b = blockIdx.x;
   const float *row = h + ((int64_t)b * S + S - 1) * d;
   const uint32_t step = pk.sign ? *pk.step : 0u;
-  float s = 0.f;
-  for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8)
-    for (int i = 0; i < 8; ++i) s += row[c + i];
-  const float mean = block_allreduce_sum(s, red) / (float)d;
+  float mean = 0.f;
+  if (!RMS) {
+    float s = 0.f;
+    for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8)
+      for (int i = 0; i < 8; ++i) s += row[c + i];
+    mean = block_allreduce_sum(s, red) / (float)d;
+  }
   float q = 0.f;
   for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8)
     for (int i = 0; i < 8; ++i) {
       const float u = row[c + i] - mean;
       q += u * u;
     }
-  const float rstd = rsqrtf(block_allreduce_sum(q, red) / (float)d + 1e-5f);
+  const float rstd = rsqrtf(block_allreduce_sum(q, red) / (float)d + eps);
   float l0 = 0.f, l1 = 0.f;
   for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
-    float g[8], bb[8], e0[8], e1[8];
+    float g[8], bb[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, e0[8], e1[8];
     load8_perturbed(theta, fin_off + c, pk, step, g);
-    load8_perturbed(theta, fin_off + d + c, pk, step, bb);
+    if (!RMS) load8_perturbed(theta, fin_off + d + c, pk, step, bb);
     load8_perturbed(theta, (int64_t)id0 * d + c, pk, step, e0);
     load8_perturbed(theta, (int64_t)id1 * d + c, pk, step, e1);
 #pragma unroll
@@ -259,6 +327,13 @@ struct zo_model {
   uint16_t *window = nullptr;
   float *h = nullptr;
   uint16_t *xn = nullptr, *qkv = nullptr, *attn = nullptr, *mid = nullptr;
+  float2 *rope = nullptr;   // Qwen3: (cos, sin) of position s and pair i at [s][e/2]
+  bool qwen = false;
+  // pruned last layer of the loss forward: the last position of each sequence only
+  int prune_rows = 0;       // capacity in sequences
+  bool prune_enabled = true;
+  float *hl = nullptr;      // residual rows [prune_rows][d]
+  uint16_t *xl = nullptr, *ql = nullptr, *al = nullptr, *midl = nullptr;
 };
 
 namespace {
@@ -270,8 +345,93 @@ zo_status model_cuda(zo_ctx *ctx, cudaError_t e, const char *what) {
               cudaGetErrorString(e));
 }
 
-// Embedding plus the first n_run layers for one micro-batch; leaves the residual in m->h.
-zo_status run_layers(zo_model *m, const int32_t *tokens, int B, int S, int n_run) {
+// Qwen3 layer: RMSNorm -> QKV projection -> per-head QK-norm + rotary -> grouped-query
+// attention -> output projection added into the residual -> RMSNorm -> gate|up projection
+// with the SwiGLU combination in its epilogue -> down projection added into the residual.
+zo_status run_qwen_layer(zo_model *m, const uint16_t *lp, int B, int S) {
+  zo_ctx *ctx = m->ctx;
+  const zo_model_cfg &c = m->cfg;
+  const Layout &L = m->L;
+  const int d = c.d_model, f = c.d_ffn, e = c.head_dim, H = c.n_heads, Hk = c.n_kv_heads;
+  const int T = B * S, nq = (int)L.qkv_cols, na = (int)L.attn_cols;
+  const float eps = c.norm_eps;
+  zo_status st;
+  if ((st = launch_rmsnorm(ctx, m->h, lp + L.in_norm, m->xn, T, d, eps)) != ZO_OK) return st;
+  if ((st = launch_gemm(ctx, m->xn, lp + L.wqkv, nullptr, m->qkv, T, nq, d, nq,
+                        ZO_EPI_BIAS_BF16)) != ZO_OK) return st;
+  if ((st = launch_qk_norm_rope(ctx, m->qkv, nq, 0, H + Hk, H, lp + L.q_norm, lp + L.k_norm, m->rope,
+                                T, S, -1, e, eps)) != ZO_OK) return st;
+  if ((st = launch_attention_gqa(ctx, m->qkv, m->attn, B, S, H, Hk, e)) != ZO_OK) return st;
+  if ((st = launch_gemm(ctx, m->attn, lp + L.wo, nullptr, m->h, T, d, na, d,
+                        ZO_EPI_RESID_F32)) != ZO_OK) return st;
+  if ((st = launch_rmsnorm(ctx, m->h, lp + L.post_norm, m->xn, T, d, eps)) != ZO_OK) return st;
+  if ((st = launch_gemm(ctx, m->xn, lp + L.wgu, nullptr, m->mid, T, f, d, f,
+                        ZO_EPI_SWIGLU_BF16)) != ZO_OK) return st;
+  return launch_gemm(ctx, m->mid, lp + L.wd, nullptr, m->h, T, d, f, d, ZO_EPI_RESID_F32);
+}
+
+zo_status gather_last(zo_model *m, const void *src, void *dst, int64_t row_bytes, int B, int S) {
+  gather_last_kernel<<<B, kRowThreads, 0, m->ctx->stream>>>(static_cast<const uint8_t *>(src),
+                                                            static_cast<uint8_t *>(dst), row_bytes, S);
+  return check_launch(m->ctx, "gather_last_kernel");
+}
+
+// The last layer of a loss-only forward, pruned to what the loss reads: keys and values
+// for every position (the last query attends to all of them), everything else for the
+// last position of each sequence only.  Leaves those residual rows in m->hl [B][d].
+zo_status run_last_layer_pruned(zo_model *m, const uint16_t *lp, int B, int S) {
+  zo_ctx *ctx = m->ctx;
+  const zo_model_cfg &c = m->cfg;
+  const Layout &L = m->L;
+  const int d = c.d_model, f = c.d_ffn, T = B * S;
+  const int nq = (int)L.qkv_cols, na = (int)L.attn_cols;
+  zo_status st;
+  if (m->qwen) {
+    const int H = c.n_heads, Hk = c.n_kv_heads, e = c.head_dim;
+    const float eps = c.norm_eps;
+    if ((st = launch_rmsnorm(ctx, m->h, lp + L.in_norm, m->xn, T, d, eps)) != ZO_OK) return st;
+    if ((st = launch_gemm(ctx, m->xn, lp + L.wqkv + (int64_t)H * e * d, nullptr, m->qkv + H * e, T,
+                          2 * Hk * e, d, nq, ZO_EPI_BIAS_BF16)) != ZO_OK) return st;
+    if ((st = launch_qk_norm_rope(ctx, m->qkv, nq, H, Hk, H, lp + L.q_norm, lp + L.k_norm, m->rope, T,
+                                  S, -1, e, eps)) != ZO_OK) return st;
+    if ((st = gather_last(m, m->xn, m->xl, (int64_t)d * 2, B, S)) != ZO_OK) return st;
+    if ((st = gather_last(m, m->h, m->hl, (int64_t)d * 4, B, S)) != ZO_OK) return st;
+    if ((st = launch_gemm(ctx, m->xl, lp + L.wqkv, nullptr, m->ql, B, na, d, na,
+                          ZO_EPI_BIAS_BF16)) != ZO_OK) return st;
+    if ((st = launch_qk_norm_rope(ctx, m->ql, na, 0, H, H, lp + L.q_norm, lp + L.k_norm, m->rope, B, S,
+                                  S - 1, e, eps)) != ZO_OK) return st;
+    if ((st = launch_attention_last(ctx, m->ql, na, m->qkv, m->al, B, S, H, Hk, e)) != ZO_OK) return st;
+    if ((st = launch_gemm(ctx, m->al, lp + L.wo, nullptr, m->hl, B, d, na, d, ZO_EPI_RESID_F32)) != ZO_OK)
+      return st;
+    if ((st = launch_rmsnorm(ctx, m->hl, lp + L.post_norm, m->xl, B, d, eps)) != ZO_OK) return st;
+    if ((st = launch_gemm(ctx, m->xl, lp + L.wgu, nullptr, m->midl, B, f, d, f,
+                          ZO_EPI_SWIGLU_BF16)) != ZO_OK) return st;
+    return launch_gemm(ctx, m->midl, lp + L.wd, nullptr, m->hl, B, d, f, d, ZO_EPI_RESID_F32);
+  }
+  layernorm_kernel<<<T, ln_threads(d), 0, ctx->stream>>>(m->h, lp + L.ln1g, lp + L.ln1b, m->xn, d);
+  if ((st = check_launch(ctx, "layernorm_kernel")) != ZO_OK) return st;
+  if ((st = launch_gemm(ctx, m->xn, lp + L.wqkv + (int64_t)d * d, lp + L.bqkv + d, m->qkv + d, T,
+                        2 * d, d, nq, ZO_EPI_BIAS_BF16)) != ZO_OK) return st;
+  if ((st = gather_last(m, m->xn, m->xl, (int64_t)d * 2, B, S)) != ZO_OK) return st;
+  if ((st = gather_last(m, m->h, m->hl, (int64_t)d * 4, B, S)) != ZO_OK) return st;
+  if ((st = launch_gemm(ctx, m->xl, lp + L.wqkv, lp + L.bqkv, m->ql, B, d, d, d,
+                        ZO_EPI_BIAS_BF16)) != ZO_OK) return st;
+  if ((st = launch_attention_last(ctx, m->ql, d, m->qkv, m->al, B, S, c.n_heads, c.n_heads,
+                                  d / c.n_heads)) != ZO_OK) return st;
+  if ((st = launch_gemm(ctx, m->al, lp + L.wo, lp + L.bo, m->hl, B, d, d, d, ZO_EPI_RESID_F32)) != ZO_OK)
+    return st;
+  layernorm_kernel<<<B, ln_threads(d), 0, ctx->stream>>>(m->hl, lp + L.ln2g, lp + L.ln2b, m->xl, d);
+  if ((st = check_launch(ctx, "layernorm_kernel")) != ZO_OK) return st;
+  if ((st = launch_gemm(ctx, m->xl, lp + L.w1, lp + L.b1, m->midl, B, f, d, f, ZO_EPI_RELU_BF16)) != ZO_OK)
+    return st;
+  return launch_gemm(ctx, m->midl, lp + L.w2, lp + L.b2, m->hl, B, d, f, d, ZO_EPI_RESID_F32);
+}
+
+// Embedding plus the first n_run layers for one micro-batch; leaves the residual in m->h,
+// or, when *pruned comes back true (prune requested and possible), the last layer ran
+// pruned and the last positions' residual rows are in m->hl.
+zo_status run_layers(zo_model *m, const int32_t *tokens, int B, int S, int n_run,
+                     bool prune = false, bool *pruned = nullptr) {
   zo_ctx *ctx = m->ctx;
   const zo_model_cfg &c = m->cfg;
   const Layout &L = m->L;
@@ -282,6 +442,8 @@ zo_status run_layers(zo_model *m, const int32_t *tokens, int B, int S, int n_run
   embed_kernel<<<T, kRowThreads, 0, ctx->stream>>>(theta, tokens, S, d, c.vocab, L.Pos, pk, m->h);
   zo_status st = check_launch(ctx, "embed_kernel");
   if (st != ZO_OK) return st;
+  const bool do_prune = prune && n_run >= 1 && S >= 2 && B <= m->prune_rows && S <= 32768;
+  if (pruned) *pruned = do_prune;
   for (int l = 0; l < n_run; ++l) {
     const int64_t off = L.layers + (int64_t)l * L.layer_size;
     const uint16_t *lp = theta + off;
@@ -289,6 +451,14 @@ zo_status run_layers(zo_model *m, const int32_t *tokens, int B, int S, int n_run
       st = launch_perturb(ctx, pk, off, L.layer_size, m->window);
       if (st != ZO_OK) return st;
       lp = m->window;
+    }
+    if (do_prune && l == n_run - 1) {
+      if ((st = run_last_layer_pruned(m, lp, B, S)) != ZO_OK) return st;
+      continue;
+    }
+    if (m->qwen) {
+      if ((st = run_qwen_layer(m, lp, B, S)) != ZO_OK) return st;
+      continue;
     }
     layernorm_kernel<<<T, ln_threads(d), 0, ctx->stream>>>(m->h, lp + L.ln1g, lp + L.ln1b, m->xn, d);
     if ((st = check_launch(ctx, "layernorm_kernel")) != ZO_OK) return st;
@@ -340,13 +510,34 @@ zo_status zo_model_create(zo_model **out, zo_ctx *ctx, const zo_model_cfg *cfg, 
   m->cfg = *cfg;
   m->L = L;
   m->max_tokens = max_tokens;
+  m->qwen = cfg->family == ZO_FAMILY_QWEN3;
   const int64_t T = max_tokens, d = cfg->d_model, f = cfg->d_ffn;
   cudaError_t e = cudaMalloc(&m->window, (size_t)L.layer_size * 2);
   if (e == cudaSuccess) e = cudaMalloc(&m->h, (size_t)T * d * 4);
   if (e == cudaSuccess) e = cudaMalloc(&m->xn, (size_t)T * d * 2);
-  if (e == cudaSuccess) e = cudaMalloc(&m->qkv, (size_t)T * 3 * d * 2);
-  if (e == cudaSuccess) e = cudaMalloc(&m->attn, (size_t)T * d * 2);
-  if (e == cudaSuccess) e = cudaMalloc(&m->mid, (size_t)T * f * 2);
+  if (e == cudaSuccess) e = cudaMalloc(&m->qkv, (size_t)T * L.qkv_cols * 2);
+  if (e == cudaSuccess) e = cudaMalloc(&m->attn, (size_t)T * L.attn_cols * 2);
+  if (e == cudaSuccess) e = cudaMalloc(&m->mid, (size_t)T * f * 2);  // FC1 / SwiGLU output
+  m->prune_rows = (int)(max_tokens < 512 ? max_tokens : 512);
+  const int64_t R = m->prune_rows;
+  if (e == cudaSuccess) e = cudaMalloc(&m->hl, (size_t)R * d * 4);
+  if (e == cudaSuccess) e = cudaMalloc(&m->xl, (size_t)R * d * 2);
+  if (e == cudaSuccess) e = cudaMalloc(&m->ql, (size_t)R * L.attn_cols * 2);
+  if (e == cudaSuccess) e = cudaMalloc(&m->al, (size_t)R * L.attn_cols * 2);
+  if (e == cudaSuccess) e = cudaMalloc(&m->midl, (size_t)R * f * 2);
+  if (e == cudaSuccess && m->qwen) {
+    // Rotary table: angle(s, i) = s * rope_theta^(-2i/e), evaluated in fp64 and rounded once.
+    const int half = cfg->head_dim / 2;
+    std::vector<float2> tab((size_t)cfg->max_pos * half);
+    for (int s = 0; s < cfg->max_pos; ++s)
+      for (int i = 0; i < half; ++i) {
+        const double ang = (double)s * std::pow((double)cfg->rope_theta, -2.0 * i / cfg->head_dim);
+        tab[(size_t)s * half + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+      }
+    e = cudaMalloc(&m->rope, tab.size() * sizeof(float2));
+    if (e == cudaSuccess)
+      e = cudaMemcpy(m->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice);
+  }
   if (e != cudaSuccess) {
     const zo_status st = model_cuda(ctx, e, "model buffers");
     zo_model_destroy(m);
@@ -365,6 +556,12 @@ zo_status zo_model_destroy(zo_model *m) {
   cudaFree(m->qkv);
   cudaFree(m->attn);
   cudaFree(m->mid);
+  cudaFree(m->rope);
+  cudaFree(m->hl);
+  cudaFree(m->xl);
+  cudaFree(m->ql);
+  cudaFree(m->al);
+  cudaFree(m->midl);
   delete m;
   return ZO_OK;
 }
@@ -378,13 +575,29 @@ zo_status zo_model_loss(zo_model *m, const int32_t *tokens, const int32_t *label
   if (st != ZO_OK) return st;
   if (!labels || !loss_out) return fail(ctx, ZO_ERR_INVALID, "null labels or loss_out");
   if (batch > kMaxPartials) return fail(ctx, ZO_ERR_INVALID, "batch above %d", kMaxPartials);
-  if ((st = run_layers(m, tokens, batch, seq, m->cfg.n_layers)) != ZO_OK) return st;
+  bool pruned = false;
+  if ((st = run_layers(m, tokens, batch, seq, m->cfg.n_layers, m->prune_enabled, &pruned)) != ZO_OK)
+    return st;
   const ProbeKey pk = probe_key(ctx);
-  head_ce_kernel<<<batch, kRowThreads, 0, ctx->stream>>>(
-      m->h, static_cast<const uint16_t *>(ctx->params), seq, m->cfg.d_model, m->L.fin,
-      m->cfg.class_ids[0], m->cfg.class_ids[1], labels, pk, ctx->partials, ctx->counter, loss_out,
-      accumulate, scale);
+  const uint16_t *theta = static_cast<const uint16_t *>(ctx->params);
+  const zo_model_cfg &c = m->cfg;
+  const float *hsrc = pruned ? m->hl : m->h;  // pruned: one row per sequence
+  const int hS = pruned ? 1 : seq;
+  if (m->qwen)
+    head_ce_kernel<true><<<batch, kRowThreads, 0, ctx->stream>>>(
+        hsrc, theta, hS, c.d_model, m->L.fin, c.class_ids[0], c.class_ids[1], labels, pk,
+        ctx->partials, ctx->counter, loss_out, accumulate, scale, c.norm_eps);
+  else
+    head_ce_kernel<false><<<batch, kRowThreads, 0, ctx->stream>>>(
+        hsrc, theta, hS, c.d_model, m->L.fin, c.class_ids[0], c.class_ids[1], labels, pk,
+        ctx->partials, ctx->counter, loss_out, accumulate, scale, 1e-5f);
   return check_launch(ctx, "head_ce_kernel");
+}
+
+zo_status zo_model_set_pruning(zo_model *m, int enabled) {
+  if (!m) return ZO_ERR_INVALID;
+  m->prune_enabled = enabled != 0;
+  return ZO_OK;
 }
 
 zo_status zo_model_hidden(zo_model *m, const int32_t *tokens, int32_t batch, int32_t seq,
@@ -465,6 +678,24 @@ zo_status zo_attention(zo_ctx *ctx, const void *qkv, void *out, int32_t batch, i
   if (!qkv || !out) return fail(ctx, ZO_ERR_INVALID, "null attention buffer");
   return launch_attention(ctx, static_cast<const uint16_t *>(qkv), static_cast<uint16_t *>(out),
                           batch, seq, n_heads, d_model);
+}
+
+zo_status zo_attention_gqa(zo_ctx *ctx, const void *qkv, void *out, int32_t batch, int32_t seq,
+                           int32_t n_heads, int32_t n_kv_heads, int32_t head_dim) {
+  if (!ctx) return ZO_ERR_INVALID;
+  ctx->err.clear();
+  if (!qkv || !out) return fail(ctx, ZO_ERR_INVALID, "null attention buffer");
+  return launch_attention_gqa(ctx, static_cast<const uint16_t *>(qkv), static_cast<uint16_t *>(out),
+                              batch, seq, n_heads, n_kv_heads, head_dim);
+}
+
+zo_status zo_rmsnorm(zo_ctx *ctx, const float *x, const void *w, void *out, int32_t rows, int32_t d,
+                     float eps) {
+  if (!ctx) return ZO_ERR_INVALID;
+  ctx->err.clear();
+  if (!x || !w || !out) return fail(ctx, ZO_ERR_INVALID, "null rmsnorm buffer");
+  return launch_rmsnorm(ctx, x, static_cast<const uint16_t *>(w), static_cast<uint16_t *>(out), rows,
+                        d, eps);
 }
 
 zo_status zo_layernorm(zo_ctx *ctx, const float *x, const void *gamma, const void *beta, void *out,

@@ -16,6 +16,10 @@
 //              shared memory, then one TMA tile store (bf16 outputs) or TMA add-reduce into
 //              the fp32 residual stream (global += tile in L2, no load by the SM); the
 //              accumulator is handed back after its last TMEM read.
+// SwiGLU epilogue (ZO_EPI_SWIGLU_BF16): the weight is [Wg; Wu] (2N rows); a tile of BN/2
+// output columns loads BN/2 gate rows and the matching BN/2 up rows into one BN-row
+// operand stage, so TMEM columns c and BN/2 + c of the accumulator hold the gate and up
+// products of output column c, combined as silu(g) * u in fp32 before one bf16 rounding.
 // Tiles are visited in groups of kGroupM row tiles so that the weight tiles of a group are
 // reused from L2.  All waits are bounded (see zo_tc.cuh); a timeout sets an error bit.
 #include <cudaTypedefs.h>
@@ -68,6 +72,8 @@ __device__ __forceinline__ void load_bias32(const uint16_t *bias, int col0, int 
 // warp's staging tile in the layout the output tensor map's swizzle expects:
 //   fp32: 128-byte rows, 16-byte chunk c stored at chunk c ^ (r & 7)   (128B swizzle);
 //   bf16:  64-byte rows, 16-byte chunk c stored at chunk c ^ ((r >> 1) & 3) (64B swizzle).
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.f + expf(-g)) * u; }
+
 template <int EPI>
 __device__ __forceinline__ void stage_row(uint8_t *stage, int r, const float v[32]) {
   if (EPI == ZO_EPI_RESID_F32) {
@@ -141,8 +147,10 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
+  constexpr bool kSwiGLU = EPI == ZO_EPI_SWIGLU_BF16;
+  constexpr int OUT_BN = kSwiGLU ? BN / 2 : BN;  // output columns per tile
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int num_m = (args.M + kBM - 1) / kBM, num_n = (args.N + BN - 1) / BN;
+  const int num_m = (args.M + kBM - 1) / kBM, num_n = (args.N + OUT_BN - 1) / OUT_BN;
   const int num_tiles = num_m * num_n;
   const int nk = (args.K + kBK - 1) / kBK;
 
@@ -170,7 +178,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     tc::tma_prefetch_desc(&tmA);
     tc::tma_prefetch_desc(&tmB);
     for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
-      const TileCoord tc0 = tile_coord(t, num_m, num_n, BN);
+      const TileCoord tc0 = tile_coord(t, num_m, num_n, OUT_BN);
       for (int kb = 0; kb < nk; ++kb) {
         const uint32_t s = issued % STAGES, ph = (issued / STAGES) & 1u;
         if (*abort_flag || !tc::mbar_wait(&empty[s], ph ^ 1u)) {
@@ -180,7 +188,13 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
         tc::mbar_arrive_expect_tx(&full[s], S::kStageBytes + (issued == 0 ? args.extra_tx : 0u));
         tc::tma_load_2d(sA + s * S::kABytes, &tmA, &full[s], kb * kBK, tc0.m0);
-        tc::tma_load_2d(sB + s * S::kBBytes, &tmB, &full[s], kb * kBK, tc0.n0);
+        if (kSwiGLU) {  // gate rows n0.., then up rows N + n0.. (the map's box is BN/2 rows)
+          tc::tma_load_2d(sB + s * S::kBBytes, &tmB, &full[s], kb * kBK, tc0.n0);
+          tc::tma_load_2d(sB + s * S::kBBytes + S::kBBytes / 2, &tmB, &full[s], kb * kBK,
+                          args.N + tc0.n0);
+        } else {
+          tc::tma_load_2d(sB + s * S::kBBytes, &tmB, &full[s], kb * kBK, tc0.n0);
+        }
         ++issued;
       }
     }
@@ -221,8 +235,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     tc::mma_commit(mma_done);  // arrives once every MMA issued above has retired
   } else if (warp >= 2) {
     const int q = warp & 3;                    // TMEM lanes 32q..32q+31 (this warp's rows)
-    const int half = (warp - 2) / 4;           // which half of the BN columns
-    const int cbeg = half * (BN / 2), cend = cbeg + BN / 2;
+    const int half = (warp - 2) / 4;           // which half of the output columns
+    const int cbeg = half * (OUT_BN / 2), cend = cbeg + OUT_BN / 2;
     uint8_t *stage = sOut + (warp - 2) * kStageTile;
     if (lane == 0) tc::tma_prefetch_desc(&tmC);
     int i = 0;
@@ -235,19 +249,27 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         break;
       }
       tc::tc_fence_after();
-      const TileCoord tc0 = tile_coord(t, num_m, num_n, BN);
+      const TileCoord tc0 = tile_coord(t, num_m, num_n, OUT_BN);
       const int row0 = tc0.m0 + q * 32;
       const uint32_t base = tmem + (uint32_t)(b * BN) + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
       for (int c0 = cbeg; c0 < cend; c0 += 32) {
         if (tc0.n0 + c0 >= args.N) break;
-        float v[32], bias[32];
+        float v[32];
         tc::tmem_ld32(base + (uint32_t)c0, v);
-        load_bias32(args.bias, tc0.n0 + c0, args.N, bias);
+        if (kSwiGLU) {
+          float u[32];
+          tc::tmem_ld32(base + (uint32_t)(BN / 2 + c0), u);
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          v[k] = __fadd_rn(v[k], bias[k]);
-          if (EPI == ZO_EPI_RELU_BF16) v[k] = fmaxf(v[k], 0.f);
+          for (int k = 0; k < 32; ++k) v[k] = silu_mul(v[k], u[k]);
+        } else {
+          float bias[32];
+          load_bias32(args.bias, tc0.n0 + c0, args.N, bias);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            v[k] = __fadd_rn(v[k], bias[k]);
+            if (EPI == ZO_EPI_RELU_BF16) v[k] = fmaxf(v[k], 0.f);
+          }
         }
         // the previous chunk's bulk store must have finished reading the staging tile
         if (lane == 0) tc::bulk_wait_read0();
@@ -344,7 +366,8 @@ cudaError_t launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const CUten
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int num_m = (g.M + kBM - 1) / kBM, num_n = (g.N + BN - 1) / BN;
+  constexpr int OUT_BN = EPI == ZO_EPI_SWIGLU_BF16 ? BN / 2 : BN;
+  const int num_m = (g.M + kBM - 1) / kBM, num_n = (g.N + OUT_BN - 1) / OUT_BN;
   const int tiles = num_m * num_n;
   kern<<<tiles < kSmCount ? tiles : kSmCount, kGemmThreads, S::kBytes, st>>>(ta, tb, tcm, g);
   return cudaGetLastError();
@@ -359,11 +382,15 @@ zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bia
   if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B) |
        reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(bias)) & 15u)
     return fail(ctx, ZO_ERR_INVALID, "gemm: operands must be 16-byte aligned");
-  if (epi < ZO_EPI_BIAS_BF16 || epi > ZO_EPI_RESID_F32) return fail(ctx, ZO_ERR_INVALID, "gemm: bad epilogue");
+  if (epi < ZO_EPI_BIAS_BF16 || epi > ZO_EPI_SWIGLU_BF16) return fail(ctx, ZO_ERR_INVALID, "gemm: bad epilogue");
+  const bool swiglu = epi == ZO_EPI_SWIGLU_BF16;
+  if (swiglu && bias) return fail(ctx, ZO_ERR_INVALID, "gemm: the SwiGLU epilogue takes no bias");
+  const int NB = swiglu ? 2 * N : N;  // rows of B, = accumulator columns over all tiles
   // N <= 128 tiles use BN = 128 to fill the machine on narrow outputs.
-  const bool wide = N > 128 && ((int64_t)((M + 127) / 128) * ((N + 255) / 256) >= kSmCount);
+  const bool wide = NB > 128 && ((int64_t)((M + 127) / 128) * ((NB + 255) / 256) >= kSmCount);
+  const int box_b = (wide ? 256 : 128) / (swiglu ? 2 : 1);
   CUtensorMap ta, tb, tcm;
-  if (!make_map(&ta, A, M, K, kBM) || !make_map(&tb, B, N, K, wide ? 256 : 128) ||
+  if (!make_map(&ta, A, M, K, kBM) || !make_map(&tb, B, NB, K, box_b) ||
       !make_out_map(&tcm, out, M, N, ldo, epi == ZO_EPI_RESID_F32))
     return fail(ctx, ZO_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
   GemmArgs g{M, N, K, static_cast<const uint16_t *>(bias), out, ldo, &ctx->dstate->flags, extra_tx};
@@ -371,11 +398,13 @@ zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bia
   if (wide) {
     if (epi == ZO_EPI_BIAS_BF16) e = launch_one<256, 4, ZO_EPI_BIAS_BF16>(ta, tb, tcm, g, ctx->stream);
     else if (epi == ZO_EPI_RELU_BF16) e = launch_one<256, 4, ZO_EPI_RELU_BF16>(ta, tb, tcm, g, ctx->stream);
-    else e = launch_one<256, 4, ZO_EPI_RESID_F32>(ta, tb, tcm, g, ctx->stream);
+    else if (epi == ZO_EPI_RESID_F32) e = launch_one<256, 4, ZO_EPI_RESID_F32>(ta, tb, tcm, g, ctx->stream);
+    else e = launch_one<256, 4, ZO_EPI_SWIGLU_BF16>(ta, tb, tcm, g, ctx->stream);
   } else {
     if (epi == ZO_EPI_BIAS_BF16) e = launch_one<128, 6, ZO_EPI_BIAS_BF16>(ta, tb, tcm, g, ctx->stream);
     else if (epi == ZO_EPI_RELU_BF16) e = launch_one<128, 6, ZO_EPI_RELU_BF16>(ta, tb, tcm, g, ctx->stream);
-    else e = launch_one<128, 6, ZO_EPI_RESID_F32>(ta, tb, tcm, g, ctx->stream);
+    else if (epi == ZO_EPI_RESID_F32) e = launch_one<128, 6, ZO_EPI_RESID_F32>(ta, tb, tcm, g, ctx->stream);
+    else e = launch_one<128, 6, ZO_EPI_SWIGLU_BF16>(ta, tb, tcm, g, ctx->stream);
   }
   if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "gemm launch: %s", cudaGetErrorString(e));
   return ZO_OK;

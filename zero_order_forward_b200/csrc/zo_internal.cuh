@@ -12,9 +12,10 @@
 namespace zo {
 
 constexpr int kSmCount = 148;           // B200 SMs (two dies x 74)
-constexpr int kGroup = 128;             // elements per Philox block (128 sign bits)
-constexpr int kTileGroups = 32;         // groups per warp tile in the streaming kernels
-constexpr int kTileElems = kGroup * kTileGroups;
+constexpr int kGroup = 16;              // elements per Philox block (16 elements x 8 probes)
+constexpr int kOctet = 8;               // probes per Philox block
+constexpr int kTileElems = 4096;        // elements per tile / chunk of the streaming kernels
+constexpr int kTileGroups = kTileElems / kGroup;  // 256
 
 // Device-resident step state.  `step` keys the probes of the current step; the
 // preconditioner copies it to `upd_step` and sets `upd_ok` before advancing it, so the
@@ -52,10 +53,28 @@ __device__ __forceinline__ uint4 philox10(uint4 c, uint32_t k0, uint32_t k1) {
   return c;
 }
 
-// The 128 sign bits of group g (elements 128g .. 128g+127) of probe `probe` at `step`.
-__device__ __forceinline__ uint4 probe_block(uint64_t g, uint32_t probe, uint32_t step,
-                                             uint32_t k0, uint32_t k1) {
-  return philox10(make_uint4((uint32_t)g, (uint32_t)(g >> 32), probe, step), k0, k1);
+// Sign layout ("8 signs per byte"): one Philox block holds the signs of the 16 elements of
+// group g (elements 16g .. 16g+15) under the 8 probes of one octet (probes 8p .. 8p+7).
+// Byte b of the little-endian block (bits 8(b&3).. of word b>>2) belongs to element 16g+b,
+// and bit k of that byte to probe 8p+k; bit 1 means z = -1.  The update, which needs every
+// probe of an element, reads whole bytes; a single-probe pass extracts one bit per byte.
+__device__ __forceinline__ uint4 sign_block(uint64_t g, uint32_t octet, uint32_t step,
+                                            uint32_t k0, uint32_t k1) {
+  return philox10(make_uint4((uint32_t)g, (uint32_t)(g >> 32), octet, step), k0, k1);
+}
+
+// The 16 sign bits of probe `probe` in the block of its octet: element 16g+b at bit b.
+__device__ __forceinline__ uint32_t probe_bits16(const uint4 &v, uint32_t probe) {
+  const uint32_t k = probe & 7u;
+  // bits k, k+8, k+16, k+24 of a word -> bits 0..3 (the multiply gathers them at 24..27)
+  auto nib = [k](uint32_t w) { return ((((w >> k) & 0x01010101u) * 0x01020408u) >> 24) & 0xFu; };
+  return nib(v.x) | (nib(v.y) << 4) | (nib(v.z) << 8) | (nib(v.w) << 12);
+}
+
+// The 16 sign bits of probe `probe` for element group g.
+__device__ __forceinline__ uint32_t probe_group_bits(uint64_t g, uint32_t probe, uint32_t step,
+                                                     uint32_t k0, uint32_t k1) {
+  return probe_bits16(sign_block(g, probe >> 3, step, k0, k1), probe);
 }
 
 __device__ __forceinline__ uint32_t word_of(const uint4 &v, int w) {
@@ -137,6 +156,10 @@ zo_status launch_quad_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, doub
                            int accumulate, double *partials, unsigned int *counter);
 zo_status launch_quad_loss_pair(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *out_plus,
                                 double *out_minus);
+// The conditioning-study quadratic (lam[4]: eigenvalue of each direction, 0 if unused;
+// directions from vseed); out_minus != null evaluates both signs of pk's probe in one pass.
+zo_status launch_lowrank_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, const float lam[4],
+                              uint64_t vseed, double *out, double *out_minus, int accumulate);
 zo_status launch_mlp_loss(zo_ctx *ctx, const float *P, const float *X, const int32_t *y,
                           int batch, int n_in, int n_hidden, int n_out, double scale,
                           double *out, int accumulate);

@@ -73,32 +73,68 @@ __device__ void finish_reduction(double v, double *partials, unsigned int *count
   finish_reduction_n<1>(&v, partials, counter, o, accumulate, scale);
 }
 
+// As finish_reduction_n, but returns the NV grid totals (in thread 0 of the last block,
+// which alone gets true) for a caller that combines them non-linearly.
+template <int NV>
+__device__ bool last_block_totals(const double v[NV], double *partials, unsigned int *counter,
+                                  double tot[NV]) {
+  __shared__ bool last;
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int k = 0; k < NV; ++k) partials[k * gridDim.x + blockIdx.x] = v[k];
+    __threadfence();
+    last = (atomicAdd(counter, 1u) == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (!last) return false;
+  __threadfence();
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    double s = 0.0;
+    for (unsigned int i = threadIdx.x; i < gridDim.x; i += blockDim.x)
+      s += __ldcg(partials + k * gridDim.x + i);
+    s = block_sum(s);
+    if (threadIdx.x == 0) tot[k] = s;
+  }
+  if (threadIdx.x == 0) *counter = 0u;
+  return threadIdx.x == 0;
+}
+
 // L = 1/2 sum_j D_j P_j^2 with P_j = rd(theta_j + s*eps*z_j) computed on load.
 //
 // A persistent producer/consumer pipeline: warp 0 streams 4096-element chunks of theta and
-// D into a ring of shared-memory stages with bulk asynchronous copies, then its 32 lanes
-// compute the chunk's 32 Philox blocks into the stage while the copies are in flight
-// (each stage's full barrier takes two arrivals: the copies' and the blocks'); the 8
-// consumer warps apply the perturbation and accumulate in fp64 (four independent partial
-// sums per thread), then release the stage.
+// D into a ring of shared-memory stages with bulk asynchronous copies; the 8 consumer warps
+// regenerate the chunk's sign bits (each lane one Philox block: the 16 elements of one
+// group that its warp reads, shared through warp shuffles), apply the perturbation and
+// accumulate in fp64 (four independent partial sums per thread), then release the stage.
 // Chunks are assigned round-robin (chunk = blockIdx.x + k * gridDim.x), so the grid size
 // and every summation order depend on M only: the result is deterministic.
 constexpr int kQChunk = 4096;
 constexpr int kQStages = 3;
 constexpr int kQConsumers = 8;
 constexpr int kQThreads = 32 * (1 + kQConsumers);
-constexpr int kQGroups = kQChunk / kGroup;                    // Philox blocks per chunk (32)
-constexpr int kQStageBytes = 2 * kQChunk * 4 + kQGroups * 16;  // theta, D, Philox blocks
+constexpr int kQStageBytes = 2 * kQChunk * 4;  // theta, D
 constexpr int kQSmemBytes = kQStages * kQStageBytes + 2 * kQStages * 8;
 
 // PAIR: both losses of one probe, L(theta + eps z) into out and L(theta - eps z) into
 // out_minus, from one pass over theta and D (pk.sign must be +1); each sum follows exactly
 // the order of a single-sign pass, so the results are bit-identical to two passes.
-template <bool PAIR>
+//
+// R > 0 adds the low-rank term of the conditioning-study quadratic,
+//   L = 1/2 sum_j D_j P_j^2 + 1/2 sum_k (lam_k / M) (v_k . P)^2   (k < R),
+// with the directions v_k in {-1,+1}^M regenerated like the probes (probes 0..R-1 of step 0
+// under their own key): the same pass accumulates the R dot products in fp64 and the last
+// block combines the grid totals.
+struct LowRankArgs {
+  float lam[4];       // eigenvalue each direction adds (0 for unused directions)
+  uint32_t vk0, vk1;  // Philox key of the directions
+};
+
+template <bool PAIR, int R>
 __global__ void __launch_bounds__(kQThreads)
 quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, int64_t M,
                  ProbeKey pk, int64_t n_chunks, double *partials, unsigned int *counter,
-                 double *out, double *out_minus, int accumulate, uint32_t *err) {
+                 double *out, double *out_minus, int accumulate, uint32_t *err, LowRankArgs lr) {
   extern __shared__ __align__(128) uint8_t qsm[];
   uint64_t *full = reinterpret_cast<uint64_t *>(qsm + kQStages * kQStageBytes);
   uint64_t *empty = full + kQStages;
@@ -106,7 +142,7 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kQStages; ++s) {
-      tc::mbar_init(&full[s], 2);
+      tc::mbar_init(&full[s], 1);
       tc::mbar_init(&empty[s], kQConsumers);
     }
     abort_flag = 0;
@@ -117,6 +153,9 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
   const float delta = pk.sign > 0 ? pk.eps : -pk.eps;
   double acc4[4] = {0.0, 0.0, 0.0, 0.0};
   double accm4[4] = {0.0, 0.0, 0.0, 0.0};  // PAIR: the -eps loss
+  double dot[R > 0 ? R : 1], dotm[R > 0 ? R : 1];  // R > 0: v_k . P (and for the -eps side)
+#pragma unroll
+  for (int k = 0; k < (R > 0 ? R : 1); ++k) dot[k] = dotm[k] = 0.0;
 
   if (warp == 0) {  // producer
     int it = 0, issued = 0;
@@ -141,11 +180,7 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
           tc::bulk_load(st + kQChunk * 4, D + base, (uint32_t)copy * 4u, &full[s]);
         }
       }
-      if (pk.sign && lane < kQGroups && (int64_t)lane * kGroup < cnt)
-        reinterpret_cast<uint4 *>(st + 2 * kQChunk * 4)[lane] =
-            probe_block((uint64_t)(base / kGroup) + lane, pk.probe, step, pk.k0, pk.k1);
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&full[s]);
       issued = it + 1;
     }
     if (abort_flag && lane == 0) {  // let this CTA's copies land before it exits
@@ -157,27 +192,49 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
     }
   } else {  // consumers
     const int ct = threadIdx.x - 32;  // 0 .. 255
+    const int cw = ct >> 5;           // consumer warp: elements 4 (32 cw + lane + 256 k) + 0..3
     int it = 0;
     for (int64_t chunk = blockIdx.x; chunk < n_chunks; chunk += gridDim.x, ++it) {
       const int s = it % kQStages;
       const uint32_t ph = (uint32_t)(it / kQStages) & 1u;
-      if (abort_flag || !tc::mbar_wait(&full[s], ph)) {
-        atomicOr(err, ZO_FLAG_TIMEOUT);
-        abort_flag = 1;
+      // lane 0 decides for the warp (all lanes leave together or none), then every lane
+      // observes the completed phase itself (immediate once lane 0 has seen it)
+      int ok = 1;
+      if (lane == 0) ok = (!abort_flag && tc::mbar_wait(&full[s], ph)) ? 1 : 0;
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (ok && lane != 0) ok = tc::mbar_wait(&full[s], ph) ? 1 : 0;
+      if (!__all_sync(0xFFFFFFFFu, ok)) {
+        if (lane == 0) { atomicOr(err, ZO_FLAG_TIMEOUT); abort_flag = 1; }
         break;
       }
       const uint8_t *st = qsm + s * kQStageBytes;
       const float *sT = reinterpret_cast<const float *>(st);
       const float *sD = reinterpret_cast<const float *>(st + kQChunk * 4);
-      const uint32_t *sB = reinterpret_cast<const uint32_t *>(st + 2 * kQChunk * 4);
       const int64_t base = chunk * kQChunk;
       const int cnt = (int)(M - base < (int64_t)kQChunk ? M - base : (int64_t)kQChunk);
       const int copy = cnt & ~3;
+      // The warp's 32 groups: slot q = 8 k + j is group 8 cw + 64 k + j of the chunk; lane q
+      // computes its 16 bits (groups past M are computed and never used).
+      const uint64_t my_group = (uint64_t)(base / kGroup) + 8 * cw + 64 * (lane >> 3) + (lane & 7);
+      uint32_t mine = 0u;
+      if (pk.sign) mine = probe_group_bits(my_group, pk.probe, step, pk.k0, pk.k1);
+      uint4 vmine = make_uint4(0u, 0u, 0u, 0u);
+      if (R > 0) vmine = sign_block(my_group, 0u, 0u, lr.vk0, lr.vk1);
 #pragma unroll
       for (int k = 0; k < kQChunk / (4 * 32 * kQConsumers); ++k) {
         const int e = 4 * (ct + k * 32 * kQConsumers);
+        const int src = 8 * k + (lane >> 2);
+        const uint32_t bits = pk.sign ? __shfl_sync(0xFFFFFFFFu, mine, src) >> (4 * (lane & 3)) : 0u;
+        uint32_t vw = 0u;  // R > 0: the direction bytes of this thread's 4 elements
+        if (R > 0) {
+          const uint32_t w0 = __shfl_sync(0xFFFFFFFFu, vmine.x, src);
+          const uint32_t w1 = __shfl_sync(0xFFFFFFFFu, vmine.y, src);
+          const uint32_t w2 = __shfl_sync(0xFFFFFFFFu, vmine.z, src);
+          const uint32_t w3 = __shfl_sync(0xFFFFFFFFu, vmine.w, src);
+          const int q = lane & 3;
+          vw = q == 0 ? w0 : q == 1 ? w1 : q == 2 ? w2 : w3;
+        }
         if (e >= cnt) continue;
-        const uint32_t bits = pk.sign ? sB[(e >> 7) * 4 + ((e >> 5) & 3)] >> (e & 31) : 0u;
         float tv[4], dv[4];
         if (e + 4 <= copy) {
           const float4 t = reinterpret_cast<const float4 *>(sT)[e >> 2];
@@ -198,9 +255,19 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
           const double pd = (double)p;
           const double hd = __dmul_rn(0.5, (double)dv[q]);
           acc4[q] = __dadd_rn(acc4[q], __dmul_rn(hd, __dmul_rn(pd, pd)));
+          double pm = 0.0;
           if (PAIR) {
-            const double pm = (double)perturb_f32(tv[q], -delta, (bits >> q) & 1u);
+            pm = (double)perturb_f32(tv[q], -delta, (bits >> q) & 1u);
             accm4[q] = __dadd_rn(accm4[q], __dmul_rn(hd, __dmul_rn(pm, pm)));
+          }
+          if (R > 0 && e + q < cnt) {
+            const uint32_t vb = vw >> (8 * q);
+#pragma unroll
+            for (int r = 0; r < (R > 0 ? R : 1); ++r) {
+              const bool neg = (vb >> r) & 1u;
+              dot[r] = __dadd_rn(dot[r], neg ? -pd : pd);
+              if (PAIR) dotm[r] = __dadd_rn(dotm[r], neg ? -pm : pm);
+            }
           }
         }
       }
@@ -214,6 +281,32 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
   // out) is touched only after the previous kernel in the stream has fully completed.
   tc::pdl_launch_dependents();
   tc::pdl_wait();
+  if (R > 0) {
+    constexpr int NS = PAIR ? 2 : 1, NV = NS * (1 + (R > 0 ? R : 1));
+    double v[NV], tot[NV];
+    v[0] = block_sum(acc);
+#pragma unroll
+    for (int r = 0; r < (R > 0 ? R : 1); ++r) v[1 + r] = block_sum(dot[r]);
+    if (PAIR) {
+      v[1 + R] = block_sum(accm);
+#pragma unroll
+      for (int r = 0; r < (R > 0 ? R : 1); ++r) v[2 + R + r] = block_sum(dotm[r]);
+    }
+    if (last_block_totals<NV>(v, partials, counter, tot)) {
+      const double inv_m = 1.0 / (double)M;
+#pragma unroll
+      for (int sgn = 0; sgn < NS; ++sgn) {
+        const double *t = tot + sgn * (1 + R);
+        double L = t[0];
+#pragma unroll
+        for (int r = 0; r < (R > 0 ? R : 1); ++r)
+          L = __dadd_rn(L, __dmul_rn(__dmul_rn(0.5 * (double)lr.lam[r], inv_m), __dmul_rn(t[1 + r], t[1 + r])));
+        double *o = sgn == 0 ? out : out_minus;
+        *o = (accumulate ? *o : 0.0) + L;
+      }
+    }
+    return;
+  }
   acc = block_sum(acc);
   if (PAIR) {
     accm = block_sum(accm);
@@ -276,14 +369,15 @@ mlp_loss_kernel(const float *__restrict__ P, const float *__restrict__ X,
 
 namespace {
 
-template <bool PAIR>
+template <bool PAIR, int R>
 zo_status launch_quad(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *out,
-                      double *out_minus, int accumulate, double *partials, unsigned int *counter) {
+                      double *out_minus, int accumulate, double *partials, unsigned int *counter,
+                      const LowRankArgs &lr = LowRankArgs{}) {
   const int64_t n_chunks = (ctx->M + kQChunk - 1) / kQChunk;
   int64_t blocks = n_chunks < (int64_t)kSmCount * 2 ? n_chunks : (int64_t)kSmCount * 2;
   static bool attr = false;
   if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(quad_loss_kernel<PAIR>,
+    const cudaError_t e = cudaFuncSetAttribute(quad_loss_kernel<PAIR, R>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes);
     if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "quad_loss_kernel attribute: %s", cudaGetErrorString(e));
     attr = true;
@@ -301,10 +395,10 @@ zo_status launch_quad(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *o
   attr_pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr_pdl;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, quad_loss_kernel<PAIR>,
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, quad_loss_kernel<PAIR, R>,
                                            static_cast<const float *>(ctx->params), D, ctx->M, pk,
                                            n_chunks, partials, counter, out, out_minus, accumulate,
-                                           &ctx->dstate->flags);
+                                           &ctx->dstate->flags, lr);
   if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "quad_loss_kernel: %s", cudaGetErrorString(e));
   return check_launch(ctx, "quad_loss_kernel");
 }
@@ -313,12 +407,23 @@ zo_status launch_quad(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *o
 
 zo_status launch_quad_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *out,
                            int accumulate, double *partials, unsigned int *counter) {
-  return launch_quad<false>(ctx, pk, D, out, nullptr, accumulate, partials, counter);
+  return launch_quad<false, 0>(ctx, pk, D, out, nullptr, accumulate, partials, counter);
 }
 
 zo_status launch_quad_loss_pair(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *out_plus,
                                 double *out_minus) {
-  return launch_quad<true>(ctx, pk, D, out_plus, out_minus, 0, ctx->partials, ctx->counter);
+  return launch_quad<true, 0>(ctx, pk, D, out_plus, out_minus, 0, ctx->partials, ctx->counter);
+}
+
+zo_status launch_lowrank_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, const float lam[4],
+                              uint64_t vseed, double *out, double *out_minus, int accumulate) {
+  LowRankArgs lr;
+  for (int k = 0; k < 4; ++k) lr.lam[k] = lam[k];
+  lr.vk0 = (uint32_t)vseed;
+  lr.vk1 = (uint32_t)(vseed >> 32);
+  if (out_minus)
+    return launch_quad<true, 4>(ctx, pk, D, out, out_minus, 0, ctx->partials, ctx->counter, lr);
+  return launch_quad<false, 4>(ctx, pk, D, out, nullptr, accumulate, ctx->partials, ctx->counter, lr);
 }
 
 zo_status launch_mlp_loss(zo_ctx *ctx, const float *P, const float *X, const int32_t *y,

@@ -4,9 +4,10 @@
 // "Probe-Space Preconditioning for Fast and Stable Zero-Order Training", abstract:
 // probes come from a packed random generator (8 signs per byte) and are applied to the
 // weights by fused unpack/apply kernels.  Here the sign bits are regenerated in
-// registers (never stored): each lane of a warp computes the Philox block of one
-// 128-element group, the warp shares the 32 blocks through shared memory, and every
-// lane then streams 16-byte vectors of theta -> rd(theta + s*eps*z).
+// registers (never stored): the lanes of a warp compute the Philox blocks of the
+// 16-element groups the warp streams, extract the probe's bit from each element byte, and
+// share the 16-bit masks (through shared memory or warp shuffles) while every lane streams
+// 16-byte vectors of theta -> rd(theta + s*eps*z).
 #include <cstdio>
 
 #include "zo_internal.cuh"
@@ -51,29 +52,34 @@ __device__ __forceinline__ uint16_t apply_one(uint16_t v, uint32_t bit, float de
   return f32_to_bf16_bits(perturb_f32(bf16_bits_to_f32(v), delta, bit));
 }
 
-// out[e - first] = P_e for e in [first, first + count).  Tiles of 32 groups (4096
-// elements) are aligned to groups in the global element index, so every group's
-// block is computed once per tile by one lane.
+// out[e - first] = P_e for e in [first, first + count).  Tiles of 256 groups (4096
+// elements) are aligned to groups in the global element index; a warp owns a tile, its
+// lane l computes the bits of groups l, l + 32, ..., l + 224 into the warp's 512-byte
+// mask (element e of the tile at bit e), and then streams the tile.
 template <typename T>
 __global__ void __launch_bounds__(kWarps * 32)
 perturb_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t first, int64_t count,
                ProbeKey pk, int64_t n_tiles) {
   constexpr int N = Vec<T>::N;
   constexpr int kIters = kTileElems / (32 * N);
-  __shared__ uint4 blocks[kWarps][kTileGroups];
+  __shared__ uint16_t masks[kWarps][kTileGroups];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t end = first + count;
   const int64_t g0 = first / kGroup;
   const uint32_t step = pk.sign ? *pk.step : 0u;
   const float delta = pk.sign > 0 ? pk.eps : -pk.eps;
-  const uint32_t *bw = reinterpret_cast<const uint32_t *>(blocks[warp]);
+  const uint32_t *bw = reinterpret_cast<const uint32_t *>(masks[warp]);
 
   for (int64_t tile = (int64_t)blockIdx.x * kWarps + warp; tile < n_tiles;
        tile += (int64_t)gridDim.x * kWarps) {
     const int64_t base = (g0 + tile * kTileGroups) * kGroup;  // first element of the tile
     if (pk.sign) {
-      const int64_t g = g0 + tile * kTileGroups + lane;
-      if (g * kGroup < end) blocks[warp][lane] = probe_block(g, pk.probe, step, pk.k0, pk.k1);
+#pragma unroll
+      for (int i = 0; i < kTileGroups / 32; ++i) {
+        const int64_t g = g0 + tile * kTileGroups + lane + 32 * i;
+        masks[warp][lane + 32 * i] =
+            g * kGroup < end ? (uint16_t)probe_group_bits(g, pk.probe, step, pk.k0, pk.k1) : 0;
+      }
       __syncwarp();
     }
 #pragma unroll 4
@@ -81,7 +87,7 @@ perturb_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t first, 
       const int e_rel = (k * 32 + lane) * N;
       const int64_t e = base + e_rel;
       uint32_t bits = 0;
-      if (pk.sign) bits = bw[(e_rel >> 7) * 4 + ((e_rel >> 5) & 3)] >> (e_rel & 31);
+      if (pk.sign) bits = bw[e_rel >> 5] >> (e_rel & 31);
       T *o = out + (e - first);
       if (e >= first && e + N <= end && ((reinterpret_cast<uintptr_t>(o) & 15) == 0)) {
         uint4 v = __ldg(reinterpret_cast<const uint4 *>(theta + e));
@@ -104,11 +110,11 @@ perturb_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t first, 
 }
 
 // Pipelined form for 16-byte-aligned windows (first % (16 / sizeof(T)) == 0, out 16-byte
-// aligned): chunks of 32 groups (4096 elements, aligned to groups in the global index)
-// stream through a ring of shared-memory stages.  Warp 0 issues the bulk copy of a chunk
-// first and then computes its 32 Philox blocks into the stage (the stage's full barrier
-// takes two arrivals: the copy's and the blocks'); 8 consumer warps apply the perturbation
-// and write the window with 16-byte stores.
+// aligned): chunks of 256 groups (4096 elements, aligned to groups in the global index)
+// stream through a ring of shared-memory stages.  Warp 0 issues the bulk copy of a chunk;
+// 8 consumer warps each regenerate the bits of the 32 groups they write (one Philox block
+// per lane, shared by warp shuffles), apply the perturbation and write the window with
+// 16-byte stores.
 constexpr int kPChunk = kTileElems;  // 4096
 constexpr int kPStages = 6;
 constexpr int kPConsumers = 8;
@@ -117,7 +123,7 @@ constexpr int kPThreads = 32 * (1 + kPConsumers);
 template <typename T>
 struct PipeSmem {
   static constexpr int kData = kPChunk * (int)sizeof(T);
-  static constexpr int kStage = kData + kTileGroups * 16;
+  static constexpr int kStage = kData;
   static constexpr int kBytes = kPStages * kStage + 2 * kPStages * 8;
 };
 
@@ -134,7 +140,7 @@ perturb_pipe_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t fi
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPStages; ++s) {
-      tc::mbar_init(&full[s], 2);
+      tc::mbar_init(&full[s], 1);
       tc::mbar_init(&empty[s], kPConsumers);
     }
     abort_flag = 0;
@@ -169,11 +175,7 @@ perturb_pipe_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t fi
           tc::bulk_load(st + (vs - cs) * (int64_t)sizeof(T), theta + vs,
                         (uint32_t)(copy * (int64_t)sizeof(T)), &full[s]);
       }
-      const int64_t g = g0 + c * kTileGroups + lane;
-      if (pk.sign && g * kGroup < end && (g + 1) * kGroup > first)
-        reinterpret_cast<uint4 *>(st + SM::kData)[lane] = probe_block(g, pk.probe, step, pk.k0, pk.k1);
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&full[s]);
       issued = it + 1;
     }
     if (abort_flag && lane == 0) {
@@ -185,27 +187,38 @@ perturb_pipe_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t fi
     }
   } else {
     const int ct = threadIdx.x - 32;
+    const int cw = ct >> 5;  // consumer warp: vectors (32 cw + lane + 256 k) N of the chunk
     int it = 0;
     for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
       const int s = it % kPStages;
       const uint32_t ph = (uint32_t)(it / kPStages) & 1u;
-      if (abort_flag || !tc::mbar_wait(&full[s], ph)) {
-        atomicOr(err, ZO_FLAG_TIMEOUT);
-        abort_flag = 1;
+      int ok = 1;  // decided per warp, as in the loss pipeline
+      if (lane == 0) ok = (!abort_flag && tc::mbar_wait(&full[s], ph)) ? 1 : 0;
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (ok && lane != 0) ok = tc::mbar_wait(&full[s], ph) ? 1 : 0;
+      if (!__all_sync(0xFFFFFFFFu, ok)) {
+        if (lane == 0) { atomicOr(err, ZO_FLAG_TIMEOUT); abort_flag = 1; }
         break;
       }
       const uint8_t *st = psm + s * SM::kStage;
-      const uint32_t *bw = reinterpret_cast<const uint32_t *>(st + SM::kData);
       const int64_t cs = (g0 + c * kTileGroups) * kGroup;
       const int64_t vs = cs > first ? cs : first;
       const int64_t ve = cs + kPChunk < end ? cs + kPChunk : end;
       const int64_t copy_end = vs + ((ve - vs) & ~(int64_t)(N - 1));
+      // The warp's 32 groups: slot q = 2N k + j is group 2N cw + 16N k + j of the chunk.
+      uint32_t mine = 0u;
+      if (pk.sign)
+        mine = probe_group_bits((uint64_t)(g0 + c * kTileGroups) + 2 * N * cw +
+                                    16 * N * (lane / (2 * N)) + lane % (2 * N),
+                                pk.probe, step, pk.k0, pk.k1);
 #pragma unroll
       for (int k = 0; k < kPChunk / (N * 32 * kPConsumers); ++k) {
         const int e_rel = (ct + k * 32 * kPConsumers) * N;
         const int64_t e = cs + e_rel;
+        const uint32_t bits =
+            pk.sign ? __shfl_sync(0xFFFFFFFFu, mine, 2 * N * k + lane * N / 16) >> ((lane * N) & 15)
+                    : 0u;
         if (e + N <= vs || e >= ve) continue;
-        const uint32_t bits = pk.sign ? bw[(e_rel >> 7) * 4 + ((e_rel >> 5) & 3)] >> (e_rel & 31) : 0u;
         if (e >= vs && e + N <= copy_end) {
           uint4 v = *reinterpret_cast<const uint4 *>(st + (int64_t)e_rel * (int64_t)sizeof(T));
           if (pk.sign) v = apply_vec(v, bits, delta, (T *)nullptr);
@@ -228,21 +241,21 @@ perturb_pipe_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t fi
   }
 }
 
-// Packed probe bytes [first_byte, first_byte + nbytes): one thread per 16-byte group
-// block.  Bits of elements >= M are cleared.
+// Packed bytes of one probe [first_byte, first_byte + nbytes) (byte q: elements 8q..8q+7,
+// bit t <-> element 8q+t): one thread per 16-element group, i.e. per 2 output bytes.
+// Bits of elements >= M are cleared.
 __global__ void pack_kernel(uint8_t *__restrict__ out, int64_t first_byte, int64_t nbytes,
                             int64_t M, uint32_t probe, const uint32_t *step_ptr, uint32_t k0,
                             uint32_t k1) {
-  const int64_t gfirst = first_byte / 16;
-  const int64_t glast = (first_byte + nbytes - 1) / 16;
+  const int64_t gfirst = first_byte / 2;
+  const int64_t glast = (first_byte + nbytes - 1) / 2;
   const int64_t g = gfirst + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (g > glast) return;
-  const uint4 b = probe_block((uint64_t)g, probe, *step_ptr, k0, k1);
-  const uint32_t words[4] = {b.x, b.y, b.z, b.w};
-  for (int q = 0; q < 16; ++q) {
-    const int64_t byte = g * 16 + q;
+  const uint32_t m = probe_group_bits((uint64_t)g, probe, *step_ptr, k0, k1);
+  for (int q = 0; q < 2; ++q) {
+    const int64_t byte = g * 2 + q;
     if (byte < first_byte || byte >= first_byte + nbytes) continue;
-    uint32_t v = (words[q >> 2] >> (8 * (q & 3))) & 0xFFu;
+    uint32_t v = (m >> (8 * q)) & 0xFFu;
     const int64_t e0 = byte * 8;
     if (e0 + 8 > M) v &= (M > e0) ? ((1u << (M - e0)) - 1u) : 0u;
     out[byte - first_byte] = (uint8_t)v;
@@ -297,7 +310,7 @@ zo_status launch_perturb(zo_ctx *ctx, const ProbeKey &pk, int64_t first, int64_t
 zo_status launch_pack(zo_ctx *ctx, uint32_t probe, int64_t first_byte, int64_t nbytes,
                       uint8_t *out) {
   if (nbytes <= 0) return ZO_OK;
-  const int64_t groups = (first_byte + nbytes - 1) / 16 - first_byte / 16 + 1;
+  const int64_t groups = (first_byte + nbytes - 1) / 2 - first_byte / 2 + 1;
   const int threads = 256;
   const int64_t blocks = (groups + threads - 1) / threads;
   ProbeKey pk = probe_key(ctx);

@@ -10,8 +10,8 @@
 // update keeps no optimizer state; theta <- theta - sum_i a_i z_i with a_i = lr*w_i*g_i/n.
 //
 // The update regenerates all n probes in registers, so theta is read once and written
-// once per step.  Its fp32 summation order is fixed (groups of 8 probes through a
-// 256-entry table of signed partial sums per group, group sums added in order).
+// once per step.  Its fp32 summation order is fixed (octets of 8 probes through a
+// 256-entry table of signed partial sums per octet, octet sums added in order).
 #include "zo_internal.cuh"
 
 namespace zo {
@@ -95,71 +95,28 @@ precond_kernel(const double *__restrict__ lp, const double *__restrict__ lm,
   }
 }
 
-constexpr int kUpdWarps = 8;
-
-// 4x4 byte transpose: out[k] byte t = w[t] byte k.
-__device__ __forceinline__ void byte_transpose4(uint32_t w0, uint32_t w1, uint32_t w2,
-                                                uint32_t w3, uint32_t out[4]) {
-  const uint32_t t0 = __byte_perm(w0, w1, 0x5140), t1 = __byte_perm(w0, w1, 0x7362);
-  const uint32_t t2 = __byte_perm(w2, w3, 0x5140), t3 = __byte_perm(w2, w3, 0x7362);
-  out[0] = __byte_perm(t0, t2, 0x5410);
-  out[1] = __byte_perm(t0, t2, 0x7632);
-  out[2] = __byte_perm(t1, t3, 0x5410);
-  out[3] = __byte_perm(t1, t3, 0x7632);
-}
-
-// Transpose the 8x8 bit matrix held in (lo = bytes 0..3, hi = bytes 4..7), byte = row,
-// bit = column: afterwards bit i of byte j is the former bit j of byte i.
-__device__ __forceinline__ void bit_transpose8(uint32_t &lo, uint32_t &hi) {
-  uint32_t t;
-  t = (lo ^ (lo >> 7)) & 0x00AA00AAu; lo ^= t ^ (t << 7);
-  t = (hi ^ (hi >> 7)) & 0x00AA00AAu; hi ^= t ^ (t << 7);
-  t = (lo ^ (lo >> 14)) & 0x0000CCCCu; lo ^= t ^ (t << 14);
-  t = (hi ^ (hi >> 14)) & 0x0000CCCCu; hi ^= t ^ (t << 14);
-  t = (lo ^ __funnelshift_r(lo, hi, 28)) & 0xF0F0F0F0u;
-  lo ^= t;
-  hi ^= t >> 4;
-}
-
-// Quad exchange: lane q of a quad holds the block r of probe p0+q; afterwards W[p] is
-// word q of the block of probe p0+p.
-__device__ __forceinline__ void quad_exchange(const uint4 &r, int q, int lane, uint32_t W[4]) {
-  uint32_t R[4];
-#pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    const uint32_t send = word_of(r, (q - t) & 3);
-    R[t] = __shfl_sync(0xFFFFFFFFu, send, (lane & ~3) | ((q + t) & 3));  // probe (q+t)&3
-  }
-#pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    // W[p] = R[(p - q) & 3]
-    const int t = (p - q) & 3;
-    W[p] = t == 0 ? R[0] : t == 1 ? R[1] : t == 2 ? R[2] : R[3];
-  }
-}
-
 template <typename T> struct Elem;
 template <> struct Elem<float> {
-  __device__ static void load32(const float *p, float v[32]) {
+  __device__ static void load16(const float *p, float v[16]) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float4 x = reinterpret_cast<const float4 *>(p)[k];
+    for (int k = 0; k < 4; ++k) {
+      const float4 x = __ldg(reinterpret_cast<const float4 *>(p) + k);
       v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
     }
   }
-  __device__ static void store32(float *p, const float v[32]) {
+  __device__ static void store16(float *p, const float v[16]) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
+    for (int k = 0; k < 4; ++k)
       reinterpret_cast<float4 *>(p)[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
   }
   __device__ static float get(const float *p, int64_t i) { return p[i]; }
   __device__ static void put(float *p, int64_t i, float v) { p[i] = v; }
 };
 template <> struct Elem<uint16_t> {
-  __device__ static void load32(const uint16_t *p, float v[32]) {
+  __device__ static void load16(const uint16_t *p, float v[16]) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint4 x = reinterpret_cast<const uint4 *>(p)[k];
+    for (int k = 0; k < 2; ++k) {
+      const uint4 x = __ldg(reinterpret_cast<const uint4 *>(p) + k);
       const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
@@ -168,9 +125,9 @@ template <> struct Elem<uint16_t> {
       }
     }
   }
-  __device__ static void store32(uint16_t *p, const float v[32]) {
+  __device__ static void store16(uint16_t *p, const float v[16]) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < 2; ++k) {
       uint32_t w[4];
 #pragma unroll
       for (int t = 0; t < 4; ++t)
@@ -183,73 +140,117 @@ template <> struct Elem<uint16_t> {
   __device__ static void put(uint16_t *p, int64_t i, float v) { p[i] = f32_to_bf16_bits(v); }
 };
 
-// theta <- rd(theta - sum_i coef_i z_i).  A warp covers 8 groups (1024 elements) per
-// slab: lane l owns the 32 elements of word slot (l & 3) of group (l >> 2).
-template <typename T>
-__global__ void __launch_bounds__(kUpdWarps * 32)
+constexpr int kUpdThreads = 512;
+
+// theta <- rd(theta - sum_i coef_i z_i).  One thread per 16-element group: for each probe
+// octet it computes the group's Philox block, whose byte b holds the octet's 8 signs of
+// element b, and adds to element b the octet's table entry for that byte.  Entry e of an
+// octet's table is the fp32 sum, left to right from its first signed term, of
+// (bit t of e ? -a : +a) over the octet's probes t; the octet sums are added in order and
+// subtracted once.  The tables are replicated R = 2^LOG_R times and lane l reads replica
+// l mod R, so the 32 lookups of a warp meet at most 32/R to a bank (none at R = 32).
+template <typename T, int LOG_R>
+__global__ void __launch_bounds__(kUpdThreads)
 update_kernel(T *__restrict__ theta, int64_t M, const float *__restrict__ coef, int n,
-              const uint32_t *step_ptr, const uint32_t *ok_ptr, uint32_t k0, uint32_t k1,
-              int64_t n_slabs) {
-  extern __shared__ float lut[];  // [ngroups][256]
+              const uint32_t *step_ptr, const uint32_t *ok_ptr, uint32_t k0, uint32_t k1) {
+  constexpr int R = 1 << LOG_R;
+  extern __shared__ float lut[];  // [octet][256 entries][R replicas]
   if (ok_ptr != nullptr && *ok_ptr == 0u) return;
   const uint32_t step = *step_ptr;
-  const int ngroups = (n + 7) >> 3;
-  // Tables of signed partial sums: entry b of group g is the fp32 sum, left to right,
-  // of (bit t of b ? -a : +a) over the group's probes t.
-  for (int idx = threadIdx.x; idx < ngroups * 256; idx += blockDim.x) {
-    const int g = idx >> 8, b = idx & 255;
-    const int p0 = 8 * g, cnt = min(8, n - p0);
-    float a0 = __ldg(coef + p0);
+  const int octets = (n + 7) >> 3;
+  // A warp computes 32 consecutive entries (one per lane) and writes their R replicas as
+  // 32 R consecutive words, 32 per store: no bank conflicts.
+  const int lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int base = (threadIdx.x >> 5) * 32; base < octets * 256; base += nwarps * 32) {
+    const int idx = base + lane;  // octets * 256 is a multiple of 32
+    const int o = idx >> 8, b = idx & 255;
+    const int p0 = 8 * o, cnt = min(8, n - p0);
+    const float a0 = __ldg(coef + p0);
     float s = (b & 1) ? -a0 : a0;
     for (int t = 1; t < cnt; ++t) {
       const float a = __ldg(coef + p0 + t);
       s = __fadd_rn(s, ((b >> t) & 1) ? -a : a);
     }
-    lut[idx] = s;
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+      const int word = j * 32 + lane;  // replica (word & (R-1)) of entry base + (word >> LOG_R)
+      lut[(base << LOG_R) + word] = __shfl_sync(0xFFFFFFFFu, s, word >> LOG_R);
+    }
   }
   __syncthreads();
 
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, q = lane & 3;
-  for (int64_t slab = (int64_t)blockIdx.x * kUpdWarps + warp; slab < n_slabs;
-       slab += (int64_t)gridDim.x * kUpdWarps) {
-    const uint64_t g = (uint64_t)slab * 8 + (lane >> 2);
-    const int64_t e0 = (int64_t)g * kGroup + q * 32;
-    float acc[32];
-#pragma unroll
-    for (int e = 0; e < 32; ++e) acc[e] = 0.f;
-    for (int grp = 0; grp < ngroups; ++grp) {
-      const int pa = 8 * grp + q, pb = 8 * grp + 4 + q;
-      const uint4 ra = pa < n ? probe_block(g, (uint32_t)pa, step, k0, k1) : make_uint4(0, 0, 0, 0);
-      const uint4 rb = pb < n ? probe_block(g, (uint32_t)pb, step, k0, k1) : make_uint4(0, 0, 0, 0);
-      uint32_t W[8];
-      quad_exchange(ra, q, lane, W);
-      quad_exchange(rb, q, lane, W + 4);
-      uint32_t L[4], H[4];
-      byte_transpose4(W[0], W[1], W[2], W[3], L);
-      byte_transpose4(W[4], W[5], W[6], W[7], H);
-      const float *tab = lut + grp * 256;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        uint32_t lo = L[k], hi = H[k];
-        bit_transpose8(lo, hi);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          acc[8 * k + e] = __fadd_rn(acc[8 * k + e], tab[(lo >> (8 * e)) & 0xFFu]);
-          acc[8 * k + 4 + e] = __fadd_rn(acc[8 * k + 4 + e], tab[(hi >> (8 * e)) & 0xFFu]);
-        }
-      }
-    }
-    if (e0 + 32 <= M) {
-      float v[32];
-      Elem<T>::load32(theta + e0, v);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) v[e] = __fsub_rn(v[e], acc[e]);
-      Elem<T>::store32(theta + e0, v);
+  const float *mine = lut + (threadIdx.x & (R - 1));
+  const int64_t n_groups = (M + kGroup - 1) / kGroup;
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n_groups;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t e0 = g * kGroup;
+    const bool whole = e0 + kGroup <= M;
+    float v[16];
+    if (whole) {
+      Elem<T>::load16(theta + e0, v);
     } else {
 #pragma unroll
-      for (int e = 0; e < 32; ++e)
-        if (e0 + e < M) Elem<T>::put(theta, e0 + e, __fsub_rn(Elem<T>::get(theta, e0 + e), acc[e]));
+      for (int e = 0; e < 16; ++e) v[e] = e0 + e < M ? Elem<T>::get(theta, e0 + e) : 0.f;
     }
+    float acc[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+    for (int o = 0; o < octets; ++o) {
+      const uint4 blk = sign_block((uint64_t)g, (uint32_t)o, step, k0, k1);
+      const uint32_t w[4] = {blk.x, blk.y, blk.z, blk.w};
+      const float *tab = mine + ((o * 256) << LOG_R);
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        acc[e] = __fadd_rn(acc[e], tab[((w[e >> 2] >> (8 * (e & 3))) & 0xFFu) << LOG_R]);
+    }
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[e] = __fsub_rn(v[e], acc[e]);
+    if (whole) {
+      Elem<T>::store16(theta + e0, v);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        if (e0 + e < M) Elem<T>::put(theta, e0 + e, v[e]);
+    }
+  }
+}
+
+// Replicas of the tables that fit in about 160 KB of shared memory for n probes.
+int update_log_replicas(int n) {
+  const int64_t per_replica = (int64_t)((n + 7) / 8) * 256 * 4;
+  int lr = 5;
+  while (lr > 0 && (per_replica << lr) > 160 * 1024) --lr;
+  return lr;
+}
+
+template <typename T, int LOG_R>
+zo_status launch_update_t(zo_ctx *ctx, const float *coef, int n, const uint32_t *step_ptr,
+                          const uint32_t *ok_ptr, uint32_t k0, uint32_t k1) {
+  const size_t smem = (size_t)((n + 7) / 8) * 256 * sizeof(float) << LOG_R;
+  auto kern = update_kernel<T, LOG_R>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  int per_sm = 1;
+  if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kUpdThreads, smem);
+  if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "update_kernel setup: %s", cudaGetErrorString(e));
+  const int64_t n_groups = (ctx->M + kGroup - 1) / kGroup;
+  int64_t blocks = (n_groups + kUpdThreads - 1) / kUpdThreads;
+  const int64_t cap = (int64_t)kSmCount * (per_sm > 0 ? per_sm : 1);
+  if (blocks > cap) blocks = cap;
+  kern<<<(unsigned)blocks, kUpdThreads, smem, ctx->stream>>>(static_cast<T *>(ctx->params), ctx->M,
+                                                             coef, n, step_ptr, ok_ptr, k0, k1);
+  return check_launch(ctx, "update_kernel");
+}
+
+template <typename T>
+zo_status launch_update_r(zo_ctx *ctx, const float *coef, int n, const uint32_t *step_ptr,
+                          const uint32_t *ok_ptr, uint32_t k0, uint32_t k1) {
+  switch (update_log_replicas(n)) {
+    case 5: return launch_update_t<T, 5>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
+    case 4: return launch_update_t<T, 4>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
+    case 3: return launch_update_t<T, 3>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
+    case 2: return launch_update_t<T, 2>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
+    case 1: return launch_update_t<T, 1>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
+    default: return launch_update_t<T, 0>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
   }
 }
 
@@ -266,22 +267,9 @@ zo_status launch_precond(zo_ctx *ctx, const double *lp, const double *lm, const 
 
 zo_status launch_update(zo_ctx *ctx, const float *coef, int n, const uint32_t *step_ptr,
                         const uint32_t *ok_ptr) {
-  const int64_t n_groups = (ctx->M + kGroup - 1) / kGroup;
-  const int64_t n_slabs = (n_groups + 7) / 8;
-  const size_t smem = (size_t)((n + 7) / 8) * 256 * sizeof(float);
-  int64_t blocks = (n_slabs + kUpdWarps - 1) / kUpdWarps;
-  if (blocks > (int64_t)kSmCount * 4) blocks = (int64_t)kSmCount * 4;
-  ProbeKey pk = probe_key(ctx);
-  if (ctx->dtype == ZO_F32) {
-    cudaFuncSetAttribute(update_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    update_kernel<float><<<(unsigned)blocks, kUpdWarps * 32, smem, ctx->stream>>>(
-        static_cast<float *>(ctx->params), ctx->M, coef, n, step_ptr, ok_ptr, pk.k0, pk.k1, n_slabs);
-  } else {
-    cudaFuncSetAttribute(update_kernel<uint16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    update_kernel<uint16_t><<<(unsigned)blocks, kUpdWarps * 32, smem, ctx->stream>>>(
-        static_cast<uint16_t *>(ctx->params), ctx->M, coef, n, step_ptr, ok_ptr, pk.k0, pk.k1, n_slabs);
-  }
-  return check_launch(ctx, "update_kernel");
+  const ProbeKey pk = probe_key(ctx);
+  return ctx->dtype == ZO_F32 ? launch_update_r<float>(ctx, coef, n, step_ptr, ok_ptr, pk.k0, pk.k1)
+                              : launch_update_r<uint16_t>(ctx, coef, n, step_ptr, ok_ptr, pk.k0, pk.k1);
 }
 
 }  // namespace zo
