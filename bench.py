@@ -4,7 +4,8 @@
 Workload (the default, one GPU): L = 1/2 sum_j D_j theta_j^2 with M = 2^24 fp32
 parameters, D_j log-uniform in [1e-3, 1e3], theta_0 ~ N(0, 1); n_pert = 64,
 eps = 1e-3, lr = 4e-7, damping = 1e-3, 1.5-SPSA.  One step = clean loss + 2*n_pert
-perturbed losses + preconditioner + update, all through the C ABI of libzo.so.
+perturbed losses (the 16 losses of each probe octet from one pass over theta and D) +
+preconditioner + update, all through the C ABI of libzo.so.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload quadratic|mlp|opt-125m|opt-1.3b|opt-30b|qwen3-1.7b|qwen3-8b]
@@ -39,11 +40,12 @@ WORKLOAD = ("diagonal quadratic L=1/2*sum D_j theta_j^2, M=2^24 fp32, D log-unif
             "theta0~N(0,1); 1.5-SPSA n_pert=64 eps=1e-3 lr=4e-7 damping=1e-3")
 FALLBACK_HBM_GBS = 6650.0
 
-# DRAM bytes (read + write) per launch of the loss-pair kernel from the ncu capture
-# summarised in profiles/quad_loss_kernel.quadratic_M2p24.md, valid for the kernel sources
+# DRAM bytes (read + write) per launch of the octet loss kernel from the ncu capture
+# summarised in profiles/quad_octet_kernel.quadratic_M2p24.md, valid for the kernel sources
 # whose SHA-256 (of zo_loss.cu, zo_internal.cuh and zo_tc.cuh, concatenated) is recorded
 # with it; reported as null when a source has changed since the capture.
-LOSS_TRAFFIC = {"sources_sha256": None, "bytes": None}
+LOSS_TRAFFIC = {"sources_sha256": "4a84d525dcd5fe39c19878adf9f4e370982c6b27459898565928a4cedd483eed",
+                "bytes": 139.6e6}
 LOSS_SOURCES = ("zo_loss.cu", "zo_internal.cuh", "zo_tc.cuh")
 
 
@@ -120,13 +122,21 @@ def reference_arm(args):
     rank, _, world = dist_env()
     if rank != 0:
         return 0
+    # the sample per step shrinks with the step count so that the run stays near 30 s: a
+    # power of two <= 2^18 elements, from a calibration step on 2^12
+    t_cal = min(time_oracle(1 << 12, 2))
+    per_elem = t_cal / (1 << 12)
     M_sample = 1 << 18
+    while M_sample > (1 << 10) and per_elem * M_sample * (args.warmup + args.steps) > 30.0:
+        M_sample >>= 1
     times = time_oracle(M_sample, args.warmup + args.steps)[args.warmup:]
     per_step = sum(times) / len(times)
     scale = M_sample / M_FULL
     value = scale / per_step  # full-workload steps/s extrapolated linearly in M
-    sample = (f"oracle step on the first 2^18 of 2^24 parameters (1/64 of the workload), "
-              f"{args.steps} timed steps after {args.warmup} warm-up; steps/s scaled by 1/64")
+    lg = M_sample.bit_length() - 1
+    sample = (f"oracle step on the first 2^{lg} of 2^24 parameters (1/{M_FULL // M_sample} of the "
+              f"workload), {args.steps} timed steps after {args.warmup} warm-up; steps/s scaled "
+              f"by 1/{M_FULL // M_sample}")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 / value, "higher_is_better": True, "scaling": "strong",
@@ -148,27 +158,46 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index):
-        self.proc = None
+        """Starts sampling every 20 ms and returns once the first sample is in, so that the
+        samples cover the region that follows."""
+        import threading
+        self.proc, self.lines = None, []
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+            return
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+        self._wait_for(1, 10.0)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line)
+
+    def _wait_for(self, n, timeout):
+        t0 = time.perf_counter()
+        while len(self.lines) < n and time.perf_counter() - t0 < timeout:
+            time.sleep(0.005)
 
     def stop(self):
+        """Takes one more sample after the region (so that a short region is bracketed),
+        then stops."""
         if self.proc is None:
             return None
+        self._wait_for(len(self.lines) + 1, 2.0)
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-            out, _ = self.proc.communicate()
+        self.reader.join(timeout=5)
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
+        for line in self.lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 8:
                 continue
@@ -221,14 +250,14 @@ def gpu_arm(args):
     def apply_step(Lp, Lm, L0):
         zo.zo_step(ctx, Lp, Lm, n, L0, LR, EPS, DAMPING)
 
-    def pair_at(probe, out_plus, out_minus):
-        zo.zo_quad_loss_pair(ctx, D, probe, EPS, out_plus, out_minus)
+    def octet_at(first, count, out_plus, out_minus):
+        zo.zo_quad_loss_octet(ctx, D, first, count, EPS, out_plus, out_minus)
 
     def one_step():
-        if world > 1:  # probe-parallel: this rank's probes, loss all-gather, same update
+        if world > 1:  # probe-parallel: this rank's probe octets, loss all-gather, same update
             from zero_order_forward_b200 import dist as zdist
             zdist.probe_parallel_step(n, loss_at, lambda o: zo.zo_quad_loss(ctx, D, o),
-                                      apply_step, dev, pair_at=pair_at)
+                                      apply_step, dev, block=8, block_at=octet_at)
         else:  # the native step driver: every launch of the step enqueued from C++
             zo.zo_quad_step(ctx, D, n, EPS, LR, DAMPING, True, losses)
 
@@ -267,21 +296,34 @@ def gpu_arm(args):
     value = args.steps / total_s  # steps of the one shared model
 
     # dominant kernel: the loss pass (perturbation on load).  At one GPU the probe phase
-    # holds n launches of the pair kernel (L(theta +- eps z_i) from one pass over theta and
-    # D); with N ranks the phase is not bracketed separately: time the pair kernel alone.
+    # holds n/8 launches of the octet kernel (the 16 losses L(theta +- eps z_i) of 8 probes
+    # from one pass over theta and D); with N ranks the phase is not bracketed separately:
+    # time the octet kernel alone.
+    n_oct = (n + 7) // 8
     if world > 1:
         le = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         flush.zero_()
         le[0].record(stream)
-        for i in range(n):
-            zo.zo_quad_loss_pair(ctx, D, i, EPS, losses[1:2], losses[2:3])
+        for o in range(n_oct):
+            zo.zo_quad_loss_octet(ctx, D, 8 * o, min(8, n - 8 * o), EPS, losses[1:9], losses[9:17],
+                                  losses[0:1] if o == 0 else None)
         le[1].record(stream)
         torch.cuda.synchronize()
         probe_ms = [le[0].elapsed_time(le[1])]
-    loss_us = 1e3 * statistics.mean(probe_ms) / n
+    loss_us = 1e3 * statistics.mean(probe_ms) / n_oct
     loss_bytes = 8 * M_FULL  # theta and D read once per pass, fp32
     achieved = loss_bytes / (loss_us * 1e-6) / 1e9
     upd_bytes = 8 * M_FULL  # theta read + written, fp32
+
+    # the one-probe form (both signs of one probe per pass), timed alone for comparison
+    pe = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    flush.zero_()
+    pe[0].record(stream)
+    for i in range(n):
+        zo.zo_quad_loss_pair(ctx, D, i, EPS, losses[1:2], losses[2:3])
+    pe[1].record(stream)
+    torch.cuda.synchronize()
+    pair_us = 1e3 * pe[0].elapsed_time(pe[1]) / n
 
     # single-kernel timing of the update (same stream), for its own roofline
     coef = torch.from_numpy(synth.coefficients(n, seed=1) * 0).to(dev)  # zero: theta unchanged
@@ -334,7 +376,7 @@ def gpu_arm(args):
             cpu = {"value": (M_sample / M_FULL) / per, "unit": "steps/s", "cores": 1,
                    "kind": "oracle",
                    "sample": "2 oracle steps on the first 2^20 of 2^24 parameters; steps/s scaled by 1/16"}
-        launches_per_step = (1 + n + 2) if world == 1 else (1 + 2 * len(range(rank, n, world)) + 2)
+        launches_per_step = 1 + len(range(rank, n_oct, world)) + 2
         line = {
             "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
@@ -343,13 +385,18 @@ def gpu_arm(args):
             "config": {"workload": WORKLOAD, "M": M_FULL, "n_pert": n, "eps": EPS, "lr": LR,
                        "damping": DAMPING, "parallelism": f"probe-parallel x{world}",
                        "l2": "flushed between steps (256 MiB write, untimed); theta+D = 128 MiB"},
-            "roofline": {"kernel": "quad_loss_kernel<pair> (L(theta +- eps z_i) in one pass, "
-                                   "perturbation on load, fp64 accumulation)",
+            "roofline": {"kernel": "quad_octet_kernel (the 16 losses L(theta +- eps z_i) of a "
+                                   "probe octet in one pass, perturbation on load, fp64 "
+                                   "accumulation)",
                          "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "peak_kind": peak_kind,
                          "bytes_per_launch": loss_bytes, "avg_launch_us": loss_us,
                          "traffic": None},
             "kernels": {
+                "quad_loss_kernel<pair>": {"avg_launch_us": pair_us, "losses_per_launch": 2,
+                                           "bytes_per_launch": loss_bytes,
+                                           "achieved_GBps": loss_bytes / (pair_us * 1e-6) / 1e9,
+                                           "frac_hbm": loss_bytes / (pair_us * 1e-6) / 1e9 / hbm_peak},
                 "update_kernel": {"avg_launch_us": upd_us, "bytes_per_launch": upd_bytes,
                                   "achieved_GBps": upd_bytes / (upd_us * 1e-6) / 1e9,
                                   "frac_hbm": upd_bytes / (upd_us * 1e-6) / 1e9 / hbm_peak},
@@ -712,7 +759,9 @@ def mlp_arm(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 300 for the quadratic workloads and the MLP, 3 "
+                         "for the decoders)")
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -722,6 +771,8 @@ def main():
                     choices=["quadratic", "mlp", "lowrank"] + sorted(DECODER_WORKLOADS))
     ap.add_argument("--n-pert", type=int, default=None, help="override n_pert (decoder workloads)")
     args = ap.parse_args()
+    if args.steps is None:
+        args.steps = 3 if args.workload in DECODER_WORKLOADS else 300
     if args.warmup < 3 and args.workload == "quadratic":
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

@@ -196,10 +196,26 @@ zo_status zo_quad_loss(zo_ctx *ctx, const float *D, double *loss_out, int accumu
  * share every load.  Each loss is the sum over all M elements of its own perturbed terms in
  * the same order as zo_quad_loss, so the results are bit-identical to perturb(+1) /
  * zo_quad_loss / restore / perturb(-1) / zo_quad_loss / restore.  Requires the clean state
- * (it does not change it); uses the current step counter.  zo_quad_step evaluates every
- * probe this way.  Errors: as zo_quad_loss, ZO_ERR_STATE if perturbed. */
+ * (it does not change it); uses the current step counter.  The probe-parallel driver
+ * evaluates probes this way.  Errors: as zo_quad_loss, ZO_ERR_STATE if perturbed. */
 zo_status zo_quad_loss_pair(zo_ctx *ctx, const float *D, int32_t probe, float eps,
                             double *loss_plus, double *loss_minus);
+
+/* The 2*count losses of the probes first_probe .. first_probe+count-1 (first_probe a
+ * multiple of 8, count 1..8: the probes of one octet, whose signs share one generator
+ * block) from ONE pass over theta and D: L(theta + eps z_i) -> loss_plus[i - first_probe],
+ * L(theta - eps z_i) -> loss_minus[i - first_probe] (device doubles).  Each element has
+ * two perturbed values, rd(theta_j + eps) and rd(theta_j - eps), and each loss takes one of
+ * them per element: L+_i is the fp64 sum of its M terms, and L-_i, which takes the other
+ * term of every element, is formed as sum_j (t_a + t_b)_j - L+_i from one common sum.  The
+ * results equal zo_quad_loss_pair's to fp64 rounding (not bit for bit: the grid and the
+ * L- formula differ).  loss_clean (device double, or NULL) receives the clean loss L(theta)
+ * from the same pass.  zo_quad_step evaluates its probes this way (and its clean loss in
+ * the first pass).  Clean state required.  Errors: as zo_quad_loss_pair, ZO_ERR_INVALID for
+ * a bad first_probe / count. */
+zo_status zo_quad_loss_octet(zo_ctx *ctx, const float *D, int32_t first_probe, int32_t count,
+                             float eps, double *loss_plus, double *loss_minus,
+                             double *loss_clean);
 
 /* Cross-entropy of an MLP classifier in -> hidden (ReLU) -> out evaluated at
  * zo_live_params(ctx) (fp32 CUDA-core arithmetic, no TF32), flat parameter order

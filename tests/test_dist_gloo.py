@@ -15,11 +15,16 @@ from zero_order_forward_b200 import dist as zdist
 def test_partition_covers_every_probe_once():
     for n in (1, 2, 5, 16, 64, 161):
         for world in (1, 2, 3, 8):
-            seen = sorted(i for r in range(world) for i in zdist.rank_probes(n, r, world))
-            assert seen == list(range(n))
-            idx = zdist.global_order(n, world)
-            assert idx.shape == (world, zdist.slots(n, world))
-            assert sorted(idx[idx >= 0].tolist()) == list(range(n))
+            for block in (1, 8):
+                seen = sorted(i for r in range(world)
+                              for i in zdist.rank_probes(n, r, world, block))
+                assert seen == list(range(n))
+                idx = zdist.global_order(n, world, block=block)
+                assert idx.shape == (world, zdist.slots(n, world, block))
+                assert sorted(idx[idx >= 0].tolist()) == list(range(n))
+                for r in range(world):  # blocks are whole octets except the last
+                    for first, count in zdist.rank_units(n, r, world, block):
+                        assert first % block == 0 and 1 <= count <= block
 
 
 def _free_port():
@@ -33,7 +38,7 @@ def _free_port():
 M, N_PERT, EPS, LR, LAM, SEED = 3000, 7, 1e-3, 1e-5, 1e-3, 5
 
 
-def _worker(rank, world, port, out_dir):
+def _worker(rank, world, port, out_dir, block=1):
     import torch.distributed as dist
 
     import oracle
@@ -60,18 +65,25 @@ def _worker(rank, world, port, out_dir):
             state["theta"] = oracle.core.update_mirror(state["theta"], pc["a"].astype(np.float32),
                                                        SEED, 0)
 
-        L0, Lp, Lm = zdist.probe_parallel_step(N_PERT, loss_at, clean, apply_step, "cpu")
+        def block_at(first, count, out_p, out_m):  # a block's losses written at once
+            for t in range(count):
+                loss_at(+1, first + t, out_p[t:t + 1])
+                loss_at(-1, first + t, out_m[t:t + 1])
+
+        L0, Lp, Lm = zdist.probe_parallel_step(N_PERT, loss_at, clean, apply_step, "cpu",
+                                               block=block,
+                                               block_at=block_at if block > 1 else None)
         np.savez(os.path.join(out_dir, f"r{rank}.npz"), theta=state["theta"], L0=L0.numpy(),
                  Lp=Lp.numpy(), Lm=Lm.numpy())
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_probe_parallel_step_matches_single_rank(tmp_path, world):
+@pytest.mark.parametrize("world,block", [(2, 1), (3, 1), (2, 4)])
+def test_probe_parallel_step_matches_single_rank(tmp_path, world, block):
     import oracle
     import synth
-    mp.start_processes(_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+    mp.start_processes(_worker, args=(world, _free_port(), str(tmp_path), block), nprocs=world,
                        join=True, start_method="spawn")
     theta, D = synth.quad_problem(M, seed=1)
     nxt, rec = oracle.step.spsa_step(theta, lambda P: oracle.core.quad_loss(P, D), N_PERT, EPS,

@@ -428,3 +428,40 @@ def test_quad_loss_pair_is_bit_identical_to_two_passes(zo, M):
         finally:
             zo.zo_restore(ctx)
     ctx.close()
+
+
+@pytest.mark.parametrize("M", [1, 7, 4096 * 3 + 5, 1 << 20, (1 << 22) + 17])
+@pytest.mark.parametrize("first,count", [(0, 8), (16, 8), (8, 3)])
+def test_quad_loss_octet_matches_pairs_and_oracle(zo, M, first, count):
+    """zo_quad_loss_octet computes the 2*count losses of one probe octet in one pass (each
+    element's two perturbed values, each loss taking one per element; L- from the common
+    sum of both terms): equal to the per-probe pair passes and to the oracle within fp64
+    rounding of sums of M terms (1e-12 relative), the clean loss from the same pass too.
+    Outputs past count are left untouched."""
+    th_np, D_np = synth.quad_problem(M, seed=13)
+    th, D = dev(th_np), dev(D_np)
+    ctx = zo.zo_create(th, seed=6)
+    zo.zo_set_step(ctx, 2)
+    oct_p = torch.full((9,), -7.0, dtype=torch.float64, device="cuda")
+    oct_m = torch.full((9,), -7.0, dtype=torch.float64, device="cuda")
+    clean = torch.zeros(2, dtype=torch.float64, device="cuda")
+    zo.zo_quad_loss_octet(ctx, D, first, count, 1e-3, oct_p, oct_m, clean[0:1])
+    zo.zo_quad_loss(ctx, D, clean[1:2])
+    pair = torch.zeros((count, 2), dtype=torch.float64, device="cuda")
+    for t in range(count):
+        zo.zo_quad_loss_pair(ctx, D, first + t, 1e-3, pair[t, 0:1], pair[t, 1:2])
+    assert zo.zo_sync(ctx) == 0
+    P, Mn, pr = oct_p.cpu().numpy(), oct_m.cpu().numpy(), pair.cpu().numpy()
+    assert np.allclose(P[:count], pr[:, 0], rtol=1e-13, atol=0)
+    assert np.allclose(Mn[:count], pr[:, 1], rtol=1e-13, atol=0)
+    assert (P[count:] == -7.0).all() and (Mn[count:] == -7.0).all()
+    c = clean.cpu().numpy()
+    assert abs(c[0] - c[1]) <= 1e-13 * c[1] and abs(c[0] - core.quad_loss(th_np, D_np)) <= 1e-12 * c[1]
+    e32 = float(np.float32(1e-3))
+    for t in range(count):
+        refp = core.quad_loss(core.perturb(th_np, 6, 2, first + t, +1, e32), D_np)
+        refm = core.quad_loss(core.perturb(th_np, 6, 2, first + t, -1, e32), D_np)
+        assert abs(P[t] - refp) <= 1e-12 * refp and abs(Mn[t] - refm) <= 1e-12 * refm
+    with pytest.raises(zo.ZoError):
+        zo.zo_quad_loss_octet(ctx, D, 3, 8, 1e-3, oct_p, oct_m)  # not an octet boundary
+    ctx.close()

@@ -64,6 +64,7 @@ _SIGS = {
     "zo_attention": [_vp, _vp, _vp, _i32, _i32, _i32, _i32],
     "zo_attention_gqa": [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32],
     "zo_model_set_pruning": [_vp, _int],
+    "zo_quad_loss_octet": [_vp, _vp, _i32, _i32, _f32, _vp, _vp, _vp],
     "zo_lowrank_loss": [_vp, _vp, _vp, _vp, _int],
     "zo_lowrank_loss_pair": [_vp, _vp, _vp, _i32, _f32, _vp, _vp],
     "zo_lowrank_step": [_vp, _vp, _vp, _i32, _f32, _f32, _f32, _int, _vp],
@@ -335,6 +336,11 @@ def zo_model_create(ctx, cfg, max_tokens):
     c = zo_model_cfg.from_dict(cfg)
     ctx.check(_L.zo_model_create(ctypes.byref(h), ctx.handle, ctypes.byref(c), int(max_tokens)))
     return Model(h, ctx, cfg)
+
+
+def zo_quad_loss_octet(ctx, D, first_probe, count, eps, loss_plus, loss_minus, loss_clean=None):
+    return ctx.check(_L.zo_quad_loss_octet(ctx.handle, _ptr(D), first_probe, count, eps,
+                                           _ptr(loss_plus), _ptr(loss_minus), _ptr(loss_clean)))
 
 
 def zo_lowrank_loss(ctx, D, lam, vseed, loss_out, accumulate=False):

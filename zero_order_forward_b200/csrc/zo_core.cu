@@ -138,7 +138,7 @@ zo_status zo_create(zo_ctx **out, void *params, int64_t M, int dtype, uint64_t s
   if (e == cudaSuccess) e = cudaMalloc(&ctx->dstate, sizeof(DevState));
   if (e == cudaSuccess) e = cudaMalloc(&ctx->coef, ZO_MAX_PROBES * sizeof(float));
   if (e == cudaSuccess) e = cudaMalloc(&ctx->diag, (3 * ZO_MAX_PROBES + 8) * sizeof(double));
-  if (e == cudaSuccess) e = cudaMalloc(&ctx->partials, kMaxPartials * sizeof(double));
+  if (e == cudaSuccess) e = cudaMalloc(&ctx->partials, (kMaxPartials + 8) * sizeof(double));
   if (e == cudaSuccess) e = cudaMalloc(&ctx->counter, sizeof(unsigned int));
   if (e == cudaSuccess) e = cudaMemsetAsync(ctx->dstate, 0, sizeof(DevState), ctx->stream);
   if (e == cudaSuccess) e = cudaMemsetAsync(ctx->counter, 0, sizeof(unsigned int), ctx->stream);
@@ -442,6 +442,22 @@ zo_status zo_lowrank_step(zo_ctx *ctx, const float *D, const zo_lowrank *q, int3
   return st;
 }
 
+zo_status zo_quad_loss_octet(zo_ctx *ctx, const float *D, int32_t first_probe, int32_t count,
+                             float eps, double *loss_plus, double *loss_minus, double *loss_clean) {
+  ZO_CHECK(check_ctx(ctx));
+  if (ctx->dtype != ZO_F32) return fail(ctx, ZO_ERR_UNSUPPORTED, "quadratic loss needs an fp32 context");
+  if (!D || !loss_plus || !loss_minus || !aligned16(D))
+    return fail(ctx, ZO_ERR_INVALID, "D must be a 16-byte aligned device pointer; outputs non-null");
+  if (first_probe < 0 || first_probe % 8 || count < 1 || count > 8 || !(eps > 0.f) || !std::isfinite(eps))
+    return fail(ctx, ZO_ERR_INVALID, "first_probe must be a multiple of 8, count 1..8, eps > 0");
+  if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "octet evaluation needs the clean state");
+  ProbeKey pk = probe_key(ctx);
+  pk.sign = +1;
+  pk.eps = eps;
+  return launch_quad_octet(ctx, pk, (uint32_t)(first_probe / 8), count, D, loss_plus, loss_minus,
+                           loss_clean);
+}
+
 zo_status zo_quad_step(zo_ctx *ctx, const float *D, int32_t n_pert, float eps, float lr,
                        float damping, int preconditioned, double *losses_out) {
   ZO_CHECK(check_ctx(ctx));
@@ -450,14 +466,13 @@ zo_status zo_quad_step(zo_ctx *ctx, const float *D, int32_t n_pert, float eps, f
   if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "step while perturbed");
   double *L0 = losses_out, *Lp = losses_out + 1, *Lm = losses_out + 1 + n_pert;
   phase_mark(ctx, 0);
-  if (preconditioned) {
-    ZO_CHECK(zo_quad_loss(ctx, D, L0, 0));
-  } else {
+  if (!preconditioned)
     ZO_CUDA(ctx, cudaMemsetAsync(L0, 0, sizeof(double), ctx->stream), "clear L0");
-  }
   phase_mark(ctx, 1);
-  for (int32_t i = 0; i < n_pert; ++i)  // L(theta +- eps z_i) from one pass each
-    ZO_CHECK(zo_quad_loss_pair(ctx, D, i, eps, Lp + i, Lm + i));
+  // the 16 losses of a probe octet from one pass; the first pass also adds the clean loss
+  for (int32_t i = 0; i < n_pert; i += 8)
+    ZO_CHECK(zo_quad_loss_octet(ctx, D, i, n_pert - i < 8 ? n_pert - i : 8, eps, Lp + i, Lm + i,
+                                (preconditioned && i == 0) ? L0 : nullptr));
   phase_mark(ctx, 2);
   const zo_status st = zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
   phase_mark(ctx, 3);

@@ -122,7 +122,7 @@ struct zo_ctx {
   float *coef = nullptr;       // ZO_MAX_PROBES fp32 update coefficients
   double *diag = nullptr;      // 3 * ZO_MAX_PROBES fp64 (g, c, w) of the last step
   int32_t last_n = 0;
-  double *partials = nullptr;  // reduction scratch (kMaxPartials doubles)
+  double *partials = nullptr;  // reduction scratch (kMaxPartials doubles + 8 discard slots)
   unsigned int *counter = nullptr;  // last-block ticket for the reductions
   float *staging = nullptr;    // device staging for host-buffer entry points
   double *loss_scratch = nullptr;  // 2*ZO_MAX_PROBES+1 doubles for host-buffer steps
@@ -136,7 +136,7 @@ struct zo_ctx {
 
 namespace zo {
 
-constexpr int kMaxPartials = 4096;
+constexpr int kMaxPartials = 8192;
 
 zo_status fail(zo_ctx *ctx, zo_status st, const char *fmt, ...);
 zo_status check_launch(zo_ctx *ctx, const char *what);
@@ -156,6 +156,11 @@ zo_status launch_quad_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, doub
                            int accumulate, double *partials, unsigned int *counter);
 zo_status launch_quad_loss_pair(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *out_plus,
                                 double *out_minus);
+// The 2 count losses of probes 8 octet .. 8 octet + count - 1 (count <= 8) in one pass,
+// and the clean loss into *out_clean in the same pass when out_clean is not null.
+zo_status launch_quad_octet(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, int count,
+                            const float *D, double *out_plus, double *out_minus,
+                            double *out_clean = nullptr);
 // The conditioning-study quadratic (lam[4]: eigenvalue of each direction, 0 if unused;
 // directions from vseed); out_minus != null evaluates both signs of pk's probe in one pass.
 zo_status launch_lowrank_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, const float lam[4],

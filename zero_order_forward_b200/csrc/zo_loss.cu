@@ -104,21 +104,145 @@ __device__ bool last_block_totals(const double v[NV], double *partials, unsigned
 //
 // A persistent producer/consumer pipeline: warp 0 streams 4096-element chunks of theta and
 // D into a ring of shared-memory stages with bulk asynchronous copies; the 8 consumer warps
-// regenerate the chunk's sign bits (each lane one Philox block: the 16 elements of one
-// group that its warp reads, shared through warp shuffles), apply the perturbation and
-// accumulate in fp64 (four independent partial sums per thread), then release the stage.
-// Chunks are assigned round-robin (chunk = blockIdx.x + k * gridDim.x), so the grid size
-// and every summation order depend on M only: the result is deterministic.
+// regenerate the chunk's sign bits (one Philox block per lane: a 16-element group of the
+// elements its warp reads, shared through warp shuffles), apply the perturbation and
+// accumulate in fp64, then release the stage.  Consumer thread ct takes the 4-element
+// vectors 4 (ct + 256 k), k = 0..3, of every chunk and adds its terms to one accumulator
+// per loss in that order; the grid walks chunks round-robin (chunk = blockIdx.x + i gridDim.x)
+// and its size depends on M only, so every loss's summation order is fixed, and the same
+// in the single-loss, pair and octet forms (their results are bit-identical).
 constexpr int kQChunk = 4096;
 constexpr int kQStages = 3;
 constexpr int kQConsumers = 8;
 constexpr int kQThreads = 32 * (1 + kQConsumers);
 constexpr int kQStageBytes = 2 * kQChunk * 4;  // theta, D
 constexpr int kQSmemBytes = kQStages * kQStageBytes + 2 * kQStages * 8;
+constexpr int kQIters = kQChunk / (4 * 32 * kQConsumers);  // 4 vectors per thread per chunk
+// The octet pass is bound by its per-probe arithmetic, not by the stream: two stages and
+// 72 registers give three CTAs (27 warps) per SM.
+constexpr int kOStages = 2;
+constexpr int kOSmemBytes = kOStages * kQStageBytes + 2 * kOStages * 8;
+constexpr int kOBlocksPerSm = 3;
+
+struct QuadPipe {
+  uint8_t *sm;
+  uint64_t *full, *empty;
+  int stages;
+};
+
+__device__ __forceinline__ QuadPipe quad_pipe_init(uint8_t *qsm, volatile int *abort_flag,
+                                                   int stages = kQStages) {
+  QuadPipe p{qsm, reinterpret_cast<uint64_t *>(qsm + stages * kQStageBytes), nullptr, stages};
+  p.empty = p.full + stages;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      tc::mbar_init(&p.full[s], 1);
+      tc::mbar_init(&p.empty[s], kQConsumers);
+    }
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  __syncthreads();
+  return p;
+}
+
+// Warp 0: stream the CTA's chunks of theta and D into the stage ring (bounded waits).
+__device__ __forceinline__ void quad_produce(const QuadPipe &p, const float *theta, const float *D,
+                                             int64_t M, int64_t n_chunks, volatile int *abort_flag,
+                                             uint32_t *err) {
+  const int lane = threadIdx.x & 31;
+  const int S = p.stages;
+  int it = 0, issued = 0;
+  for (int64_t chunk = blockIdx.x; chunk < n_chunks; chunk += gridDim.x, ++it) {
+    const int s = it % S;
+    const uint32_t ph = (uint32_t)(it / S) & 1u;
+    int ok = 1;
+    if (lane == 0) ok = tc::mbar_wait(&p.empty[s], ph ^ 1u) ? 1 : 0;
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    if (!ok || *abort_flag) {
+      if (lane == 0) { atomicOr(err, ZO_FLAG_TIMEOUT); *abort_flag = 1; }
+      break;
+    }
+    uint8_t *st = p.sm + s * kQStageBytes;
+    const int64_t base = chunk * kQChunk;
+    const int cnt = (int)(M - base < (int64_t)kQChunk ? M - base : (int64_t)kQChunk);
+    const int copy = cnt & ~3;
+    if (lane == 0) {
+      tc::mbar_arrive_expect_tx(&p.full[s], 2u * (uint32_t)copy * 4u);
+      if (copy) {
+        tc::bulk_load(st, theta + base, (uint32_t)copy * 4u, &p.full[s]);
+        tc::bulk_load(st + kQChunk * 4, D + base, (uint32_t)copy * 4u, &p.full[s]);
+      }
+    }
+    __syncwarp();
+    issued = it + 1;
+  }
+  if (*abort_flag && lane == 0) {  // let this CTA's copies land before it exits
+    for (int s = 0; s < S; ++s) {
+      int last = -1;
+      for (int i = s; i < issued; i += S) last = i;
+      if (last >= 0) tc::mbar_wait(&p.full[s], (uint32_t)(last / S) & 1u);
+    }
+  }
+}
+
+// A consumer warp takes stage s (phase ph): lane 0 decides for the warp (all lanes leave
+// together or none), then every lane observes the completed phase itself.
+__device__ __forceinline__ bool quad_acquire(const QuadPipe &p, int s, uint32_t ph,
+                                             volatile int *abort_flag, uint32_t *err) {
+  const int lane = threadIdx.x & 31;
+  int ok = 1;
+  if (lane == 0) ok = (!*abort_flag && tc::mbar_wait(&p.full[s], ph)) ? 1 : 0;
+  ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+  if (ok && lane != 0) ok = tc::mbar_wait(&p.full[s], ph) ? 1 : 0;
+  if (__all_sync(0xFFFFFFFFu, ok)) return true;
+  if (lane == 0) { atomicOr(err, ZO_FLAG_TIMEOUT); *abort_flag = 1; }
+  return false;
+}
+
+// The 4 theta and D values of vector e (0 past the end of the chunk: their terms are 0).
+__device__ __forceinline__ void quad_load4(const uint8_t *st, const float *theta, const float *D,
+                                           int64_t base, int e, int cnt, float tv[4], float dv[4]) {
+  if (e + 4 <= (cnt & ~3)) {
+    const float4 t = reinterpret_cast<const float4 *>(st)[e >> 2];
+    const float4 dd = reinterpret_cast<const float4 *>(st + kQChunk * 4)[e >> 2];
+    tv[0] = t.x; tv[1] = t.y; tv[2] = t.z; tv[3] = t.w;
+    dv[0] = dd.x; dv[1] = dd.y; dv[2] = dd.z; dv[3] = dd.w;
+  } else {  // the last < 4 elements of theta (not covered by the 16-byte copies)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const bool in = e + q < cnt;
+      tv[q] = in ? theta[base + e + q] : 0.f;
+      dv[q] = in ? D[base + e + q] : 0.f;
+    }
+  }
+}
+
+// term = (D/2) P^2 in fp64 (P^2 of an fp32 value is exact in fp64).
+__device__ __forceinline__ double quad_term(float d, float p) {
+  const double pd = (double)p;
+  return __dmul_rn(__dmul_rn(0.5, (double)d), __dmul_rn(pd, pd));
+}
+
+// Quad exchange: lane q of a quad holds block r; afterwards W[k] is word q of the block held
+// by lane k of the quad.
+__device__ __forceinline__ void quad_exchange(const uint4 &r, int lane, uint32_t W[4]) {
+  const int q = lane & 3;
+  uint32_t R[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const uint32_t send = word_of(r, (q - t) & 3);
+    R[t] = __shfl_sync(0xFFFFFFFFu, send, (lane & ~3) | ((q + t) & 3));
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int t = (k - q) & 3;  // W[k] = R[(k - q) & 3]
+    W[k] = t == 0 ? R[0] : t == 1 ? R[1] : t == 2 ? R[2] : R[3];
+  }
+}
 
 // PAIR: both losses of one probe, L(theta + eps z) into out and L(theta - eps z) into
-// out_minus, from one pass over theta and D (pk.sign must be +1); each sum follows exactly
-// the order of a single-sign pass, so the results are bit-identical to two passes.
+// out_minus, from one pass over theta and D (pk.sign must be +1).
 //
 // R > 0 adds the low-rank term of the conditioning-study quadratic,
 //   L = 1/2 sum_j D_j P_j^2 + 1/2 sum_k (lam_k / M) (v_k . P)^2   (k < R),
@@ -136,83 +260,29 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
                  ProbeKey pk, int64_t n_chunks, double *partials, unsigned int *counter,
                  double *out, double *out_minus, int accumulate, uint32_t *err, LowRankArgs lr) {
   extern __shared__ __align__(128) uint8_t qsm[];
-  uint64_t *full = reinterpret_cast<uint64_t *>(qsm + kQStages * kQStageBytes);
-  uint64_t *empty = full + kQStages;
   __shared__ volatile int abort_flag;
+  const QuadPipe pipe = quad_pipe_init(qsm, &abort_flag);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kQStages; ++s) {
-      tc::mbar_init(&full[s], 1);
-      tc::mbar_init(&empty[s], kQConsumers);
-    }
-    abort_flag = 0;
-    tc::fence_barrier_init();
-  }
-  __syncthreads();
   const uint32_t step = pk.sign ? *pk.step : 0u;
   const float delta = pk.sign > 0 ? pk.eps : -pk.eps;
-  double acc4[4] = {0.0, 0.0, 0.0, 0.0};
-  double accm4[4] = {0.0, 0.0, 0.0, 0.0};  // PAIR: the -eps loss
-  double dot[R > 0 ? R : 1], dotm[R > 0 ? R : 1];  // R > 0: v_k . P (and for the -eps side)
+  constexpr int RR = R > 0 ? R : 1;
+  double acc = 0.0, accm = 0.0;   // accm: PAIR, the -eps loss
+  double dot[RR], dotm[RR];       // R > 0: v_k . P (and for the -eps side)
 #pragma unroll
-  for (int k = 0; k < (R > 0 ? R : 1); ++k) dot[k] = dotm[k] = 0.0;
+  for (int k = 0; k < RR; ++k) dot[k] = dotm[k] = 0.0;
 
-  if (warp == 0) {  // producer
-    int it = 0, issued = 0;
-    for (int64_t chunk = blockIdx.x; chunk < n_chunks; chunk += gridDim.x, ++it) {
-      const int s = it % kQStages;
-      const uint32_t ph = (uint32_t)(it / kQStages) & 1u;
-      int ok = 1;
-      if (lane == 0) ok = tc::mbar_wait(&empty[s], ph ^ 1u) ? 1 : 0;
-      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      if (!ok || abort_flag) {
-        if (lane == 0) { atomicOr(err, ZO_FLAG_TIMEOUT); abort_flag = 1; }
-        break;
-      }
-      uint8_t *st = qsm + s * kQStageBytes;
-      const int64_t base = chunk * kQChunk;
-      const int cnt = (int)(M - base < (int64_t)kQChunk ? M - base : (int64_t)kQChunk);
-      const int copy = cnt & ~3;
-      if (lane == 0) {
-        tc::mbar_arrive_expect_tx(&full[s], 2u * (uint32_t)copy * 4u);
-        if (copy) {
-          tc::bulk_load(st, theta + base, (uint32_t)copy * 4u, &full[s]);
-          tc::bulk_load(st + kQChunk * 4, D + base, (uint32_t)copy * 4u, &full[s]);
-        }
-      }
-      __syncwarp();
-      issued = it + 1;
-    }
-    if (abort_flag && lane == 0) {  // let this CTA's copies land before it exits
-      for (int s = 0; s < kQStages; ++s) {
-        int last = -1;
-        for (int i = s; i < issued; i += kQStages) last = i;
-        if (last >= 0) tc::mbar_wait(&full[s], (uint32_t)(last / kQStages) & 1u);
-      }
-    }
-  } else {  // consumers
+  if (warp == 0) {
+    quad_produce(pipe, theta, D, M, n_chunks, &abort_flag, err);
+  } else {
     const int ct = threadIdx.x - 32;  // 0 .. 255
     const int cw = ct >> 5;           // consumer warp: elements 4 (32 cw + lane + 256 k) + 0..3
     int it = 0;
     for (int64_t chunk = blockIdx.x; chunk < n_chunks; chunk += gridDim.x, ++it) {
       const int s = it % kQStages;
-      const uint32_t ph = (uint32_t)(it / kQStages) & 1u;
-      // lane 0 decides for the warp (all lanes leave together or none), then every lane
-      // observes the completed phase itself (immediate once lane 0 has seen it)
-      int ok = 1;
-      if (lane == 0) ok = (!abort_flag && tc::mbar_wait(&full[s], ph)) ? 1 : 0;
-      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      if (ok && lane != 0) ok = tc::mbar_wait(&full[s], ph) ? 1 : 0;
-      if (!__all_sync(0xFFFFFFFFu, ok)) {
-        if (lane == 0) { atomicOr(err, ZO_FLAG_TIMEOUT); abort_flag = 1; }
-        break;
-      }
-      const uint8_t *st = qsm + s * kQStageBytes;
-      const float *sT = reinterpret_cast<const float *>(st);
-      const float *sD = reinterpret_cast<const float *>(st + kQChunk * 4);
+      if (!quad_acquire(pipe, s, (uint32_t)(it / kQStages) & 1u, &abort_flag, err)) break;
+      const uint8_t *st = pipe.sm + s * kQStageBytes;
       const int64_t base = chunk * kQChunk;
       const int cnt = (int)(M - base < (int64_t)kQChunk ? M - base : (int64_t)kQChunk);
-      const int copy = cnt & ~3;
       // The warp's 32 groups: slot q = 8 k + j is group 8 cw + 64 k + j of the chunk; lane q
       // computes its 16 bits (groups past M are computed and never used).
       const uint64_t my_group = (uint64_t)(base / kGroup) + 8 * cw + 64 * (lane >> 3) + (lane & 7);
@@ -221,7 +291,7 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
       uint4 vmine = make_uint4(0u, 0u, 0u, 0u);
       if (R > 0) vmine = sign_block(my_group, 0u, 0u, lr.vk0, lr.vk1);
 #pragma unroll
-      for (int k = 0; k < kQChunk / (4 * 32 * kQConsumers); ++k) {
+      for (int k = 0; k < kQIters; ++k) {
         const int e = 4 * (ct + k * 32 * kQConsumers);
         const int src = 8 * k + (lane >> 2);
         const uint32_t bits = pk.sign ? __shfl_sync(0xFFFFFFFFu, mine, src) >> (4 * (lane & 3)) : 0u;
@@ -236,70 +306,58 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
         }
         if (e >= cnt) continue;
         float tv[4], dv[4];
-        if (e + 4 <= copy) {
-          const float4 t = reinterpret_cast<const float4 *>(sT)[e >> 2];
-          const float4 dd = reinterpret_cast<const float4 *>(sD)[e >> 2];
-          tv[0] = t.x; tv[1] = t.y; tv[2] = t.z; tv[3] = t.w;
-          dv[0] = dd.x; dv[1] = dd.y; dv[2] = dd.z; dv[3] = dd.w;
-        } else {  // the last < 4 elements of theta (not covered by the 16-byte copies)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const bool in = e + q < cnt;
-            tv[q] = in ? theta[base + e + q] : 0.f;
-            dv[q] = in ? D[base + e + q] : 0.f;
-          }
-        }
+        quad_load4(st, theta, D, base, e, cnt, tv, dv);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float p = pk.sign ? perturb_f32(tv[q], delta, (bits >> q) & 1u) : tv[q];
-          const double pd = (double)p;
-          const double hd = __dmul_rn(0.5, (double)dv[q]);
-          acc4[q] = __dadd_rn(acc4[q], __dmul_rn(hd, __dmul_rn(pd, pd)));
-          double pm = 0.0;
+          acc = __dadd_rn(acc, quad_term(dv[q], p));
+          float pm = 0.f;
           if (PAIR) {
-            pm = (double)perturb_f32(tv[q], -delta, (bits >> q) & 1u);
-            accm4[q] = __dadd_rn(accm4[q], __dmul_rn(hd, __dmul_rn(pm, pm)));
+            pm = perturb_f32(tv[q], -delta, (bits >> q) & 1u);
+            accm = __dadd_rn(accm, quad_term(dv[q], pm));
           }
           if (R > 0 && e + q < cnt) {
             const uint32_t vb = vw >> (8 * q);
 #pragma unroll
-            for (int r = 0; r < (R > 0 ? R : 1); ++r) {
+            for (int r = 0; r < RR; ++r) {
               const bool neg = (vb >> r) & 1u;
+              const double pd = (double)p;
               dot[r] = __dadd_rn(dot[r], neg ? -pd : pd);
-              if (PAIR) dotm[r] = __dadd_rn(dotm[r], neg ? -pm : pm);
+              if (PAIR) {
+                const double pmd = (double)pm;
+                dotm[r] = __dadd_rn(dotm[r], neg ? -pmd : pmd);
+              }
             }
           }
         }
       }
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&empty[s]);
+      if (lane == 0) tc::mbar_arrive(&pipe.empty[s]);
     }
   }
-  double acc = __dadd_rn(__dadd_rn(acc4[0], acc4[1]), __dadd_rn(acc4[2], acc4[3]));
-  double accm = __dadd_rn(__dadd_rn(accm4[0], accm4[1]), __dadd_rn(accm4[2], accm4[3]));
   // The next loss pass may start streaming now; the reduction scratch (partials, counter,
   // out) is touched only after the previous kernel in the stream has fully completed.
   tc::pdl_launch_dependents();
   tc::pdl_wait();
   if (R > 0) {
-    constexpr int NS = PAIR ? 2 : 1, NV = NS * (1 + (R > 0 ? R : 1));
+    constexpr int NS = PAIR ? 2 : 1, NV = NS * (1 + RR);
     double v[NV], tot[NV];
     v[0] = block_sum(acc);
 #pragma unroll
-    for (int r = 0; r < (R > 0 ? R : 1); ++r) v[1 + r] = block_sum(dot[r]);
+    for (int r = 0; r < RR; ++r) v[1 + r] = block_sum(dot[r]);
     if (PAIR) {
-      v[1 + R] = block_sum(accm);
+      v[1 + RR] = block_sum(accm);
 #pragma unroll
-      for (int r = 0; r < (R > 0 ? R : 1); ++r) v[2 + R + r] = block_sum(dotm[r]);
+      for (int r = 0; r < RR; ++r) v[2 + RR + r] = block_sum(dotm[r]);
     }
     if (last_block_totals<NV>(v, partials, counter, tot)) {
       const double inv_m = 1.0 / (double)M;
 #pragma unroll
       for (int sgn = 0; sgn < NS; ++sgn) {
-        const double *t = tot + sgn * (1 + R);
+        const double *t = tot + sgn * (1 + RR);
         double L = t[0];
 #pragma unroll
-        for (int r = 0; r < (R > 0 ? R : 1); ++r)
+        for (int r = 0; r < RR; ++r)
           L = __dadd_rn(L, __dmul_rn(__dmul_rn(0.5 * (double)lr.lam[r], inv_m), __dmul_rn(t[1 + r], t[1 + r])));
         double *o = sgn == 0 ? out : out_minus;
         *o = (accumulate ? *o : 0.0) + L;
@@ -315,6 +373,93 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
     finish_reduction_n<2>(v, partials, counter, o, accumulate, 1.0);
   } else {
     finish_reduction(acc, partials, counter, out, accumulate, 1.0);
+  }
+}
+
+// The 16 losses L(theta +- eps z_i) of the 8 probes i = 8 octet + t of one octet from one
+// pass over theta and D.  Each element has only two perturbed values, P_a = rd(theta + eps)
+// and P_b = rd(theta - eps), with terms t_a = (D/2) P_a^2 and t_b = (D/2) P_b^2; the
+// element's byte of the octet's Philox block says which one each loss takes (bit t set:
+// L+_t takes t_b and L-_t takes t_a; clear: the reverse).  L+_t is accumulated term by term
+// in quad_loss_kernel's order; L-_t takes, element by element, the other term, so
+// L-_t = sum_j (t_a + t_b)_j - L+_t exactly, and the pass accumulates the one common sum
+// T = sum_j (t_a + t_b)_j instead of eight more per-probe sums (fp64 throughout; the results
+// agree with the one-probe passes to rounding).  Probes t >= count are computed and not
+// stored.  CLEAN also adds the clean loss L(theta) to the same pass (into *out_clean,
+// bit-identical to the clean quad_loss_kernel pass).
+template <bool CLEAN>
+__global__ void __launch_bounds__(kQThreads, kOBlocksPerSm)
+quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, int64_t M,
+                  ProbeKey pk, uint32_t octet, int count, int64_t n_chunks, double *partials,
+                  unsigned int *counter, double *out_plus, double *out_minus, double *out_clean,
+                  uint32_t *err) {
+  extern __shared__ __align__(128) uint8_t qsm[];
+  __shared__ volatile int abort_flag;
+  const QuadPipe pipe = quad_pipe_init(qsm, &abort_flag, kOStages);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t step = *pk.step;
+  double lp[8], tsum = 0.0, l0 = 0.0;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) lp[t] = 0.0;
+
+  if (warp == 0) {
+    quad_produce(pipe, theta, D, M, n_chunks, &abort_flag, err);
+  } else {
+    const int ct = threadIdx.x - 32;
+    const int cw = ct >> 5;
+    const int q = lane & 3, quad = lane >> 2;
+    int it = 0;
+    for (int64_t chunk = blockIdx.x; chunk < n_chunks; chunk += gridDim.x, ++it) {
+      const int s = it % kOStages;
+      if (!quad_acquire(pipe, s, (uint32_t)(it / kOStages) & 1u, &abort_flag, err)) break;
+      const uint8_t *st = pipe.sm + s * kQStageBytes;
+      const int64_t base = chunk * kQChunk;
+      const int cnt = (int)(M - base < (int64_t)kQChunk ? M - base : (int64_t)kQChunk);
+      // Vector k of this thread lies in group 8 cw + 64 k + quad of the chunk, bytes 4q..4q+3
+      // (word q of the block).  Lane q of the quad computes the block of iteration k = q; the
+      // quad exchange hands every lane word q of all four.
+      const uint4 blk = sign_block((uint64_t)(base / kGroup) + 8 * cw + 64 * q + quad, octet, step,
+                                   pk.k0, pk.k1);
+      uint32_t W[4];
+      quad_exchange(blk, lane, W);
+#pragma unroll
+      for (int k = 0; k < kQIters; ++k) {
+        const int e = 4 * (ct + k * 32 * kQConsumers);
+        if (e >= cnt) continue;
+        float tv[4], dv[4];
+        quad_load4(st, theta, D, base, e, cnt, tv, dv);
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const double ta = quad_term(dv[qq], __fadd_rn(tv[qq], pk.eps));
+          const double tb = quad_term(dv[qq], __fadd_rn(tv[qq], -pk.eps));
+          tsum = __dadd_rn(tsum, __dadd_rn(ta, tb));
+          if (CLEAN) l0 = __dadd_rn(l0, quad_term(dv[qq], tv[qq]));
+          const uint32_t byte = W[k] >> (8 * qq);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) lp[t] = __dadd_rn(lp[t], ((byte >> t) & 1u) ? tb : ta);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&pipe.empty[s]);
+    }
+  }
+  tc::pdl_launch_dependents();
+  tc::pdl_wait();
+  constexpr int NV = CLEAN ? 10 : 9;
+  double v[NV], tot[NV];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) v[t] = block_sum(lp[t]);
+  v[8] = block_sum(tsum);
+  if (CLEAN) v[NV - 1] = block_sum(l0);
+  if (last_block_totals<NV>(v, partials, counter, tot)) {
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      if (t < count) {
+        out_plus[t] = tot[t];
+        out_minus[t] = tot[8] - tot[t];
+      }
+    }
+    if (CLEAN) *out_clean = tot[NV - 1];
   }
 }
 
@@ -413,6 +558,44 @@ zo_status launch_quad_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, doub
 zo_status launch_quad_loss_pair(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *out_plus,
                                 double *out_minus) {
   return launch_quad<true, 0>(ctx, pk, D, out_plus, out_minus, 0, ctx->partials, ctx->counter);
+}
+
+template <bool CLEAN>
+zo_status launch_quad_octet_t(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, int count,
+                              const float *D, double *out_plus, double *out_minus, double *out_clean) {
+  const int64_t n_chunks = (ctx->M + kQChunk - 1) / kQChunk;
+  const int64_t cap = (int64_t)kSmCount * kOBlocksPerSm;
+  const int64_t blocks = n_chunks < cap ? n_chunks : cap;
+  static_assert(10 * kSmCount * kOBlocksPerSm <= kMaxPartials, "partials too small for the octet pass");
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e = cudaFuncSetAttribute(quad_octet_kernel<CLEAN>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kOSmemBytes);
+    if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "quad_octet_kernel attribute: %s", cudaGetErrorString(e));
+    attr = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(kQThreads);
+  cfg.dynamicSmemBytes = kOSmemBytes;
+  cfg.stream = ctx->stream;
+  cudaLaunchAttribute attr_pdl[1];
+  attr_pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr_pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr_pdl;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, quad_octet_kernel<CLEAN>,
+                                           static_cast<const float *>(ctx->params), D, ctx->M, pk,
+                                           octet, count, n_chunks, ctx->partials, ctx->counter,
+                                           out_plus, out_minus, out_clean, &ctx->dstate->flags);
+  if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "quad_octet_kernel: %s", cudaGetErrorString(e));
+  return check_launch(ctx, "quad_octet_kernel");
+}
+
+zo_status launch_quad_octet(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, int count,
+                            const float *D, double *out_plus, double *out_minus, double *out_clean) {
+  return out_clean ? launch_quad_octet_t<true>(ctx, pk, octet, count, D, out_plus, out_minus, out_clean)
+                   : launch_quad_octet_t<false>(ctx, pk, octet, count, D, out_plus, out_minus, nullptr);
 }
 
 zo_status launch_lowrank_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, const float lam[4],

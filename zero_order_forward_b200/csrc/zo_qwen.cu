@@ -87,12 +87,23 @@ qk_norm_rope_kernel(uint16_t *__restrict__ qkv, int64_t ld, int hbeg, int hcount
   const uint16_t *w = hh < H ? qn : kn;
   const int f0 = lane * V;
   float a[V], b[V], wa[V], wb[V];
+  if (V == 2) {  // one 4-byte load per half (f0 even, rows 16-byte aligned)
+    const uint32_t xa = *reinterpret_cast<const uint32_t *>(x + f0);
+    const uint32_t xb = *reinterpret_cast<const uint32_t *>(x + HALF + f0);
+    const uint32_t ga = *reinterpret_cast<const uint32_t *>(w + f0);
+    const uint32_t gb = *reinterpret_cast<const uint32_t *>(w + HALF + f0);
+    a[0] = __uint_as_float(xa << 16); a[V - 1] = __uint_as_float(xa & 0xFFFF0000u);
+    b[0] = __uint_as_float(xb << 16); b[V - 1] = __uint_as_float(xb & 0xFFFF0000u);
+    wa[0] = __uint_as_float(ga << 16); wa[V - 1] = __uint_as_float(ga & 0xFFFF0000u);
+    wb[0] = __uint_as_float(gb << 16); wb[V - 1] = __uint_as_float(gb & 0xFFFF0000u);
+  } else {
 #pragma unroll
-  for (int i = 0; i < V; ++i) {
-    a[i] = bf16_bits_to_f32(x[f0 + i]);
-    b[i] = bf16_bits_to_f32(x[HALF + f0 + i]);
-    wa[i] = bf16_bits_to_f32(w[f0 + i]);
-    wb[i] = bf16_bits_to_f32(w[HALF + f0 + i]);
+    for (int i = 0; i < V; ++i) {
+      a[i] = bf16_bits_to_f32(x[f0 + i]);
+      b[i] = bf16_bits_to_f32(x[HALF + f0 + i]);
+      wa[i] = bf16_bits_to_f32(w[f0 + i]);
+      wb[i] = bf16_bits_to_f32(w[HALF + f0 + i]);
+    }
   }
   float ss = 0.f;
 #pragma unroll
@@ -101,12 +112,23 @@ qk_norm_rope_kernel(uint16_t *__restrict__ qkv, int64_t ld, int hbeg, int hcount
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
   const float rstd = rsqrtf(ss / (float)HD + eps);
   const float2 *cs = rope + (int64_t)s * HALF + f0;
+  uint16_t oa[V], ob[V];
 #pragma unroll
   for (int i = 0; i < V; ++i) {
     const float x1 = a[i] * rstd * wa[i], x2 = b[i] * rstd * wb[i];
     const float2 r = cs[i];
-    x[f0 + i] = f32_to_bf16_bits(x1 * r.x - x2 * r.y);
-    x[HALF + f0 + i] = f32_to_bf16_bits(x2 * r.x + x1 * r.y);
+    oa[i] = f32_to_bf16_bits(x1 * r.x - x2 * r.y);
+    ob[i] = f32_to_bf16_bits(x2 * r.x + x1 * r.y);
+  }
+  if (V == 2) {
+    *reinterpret_cast<uint32_t *>(x + f0) = (uint32_t)oa[0] | ((uint32_t)oa[V - 1] << 16);
+    *reinterpret_cast<uint32_t *>(x + HALF + f0) = (uint32_t)ob[0] | ((uint32_t)ob[V - 1] << 16);
+  } else {
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+      x[f0 + i] = oa[i];
+      x[HALF + f0 + i] = ob[i];
+    }
   }
 }
 

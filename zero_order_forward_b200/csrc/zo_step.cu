@@ -140,7 +140,7 @@ template <> struct Elem<uint16_t> {
   __device__ static void put(uint16_t *p, int64_t i, float v) { p[i] = f32_to_bf16_bits(v); }
 };
 
-constexpr int kUpdThreads = 512;
+constexpr int kUpdThreads = 1024;
 
 // theta <- rd(theta - sum_i coef_i z_i).  One thread per 16-element group: for each probe
 // octet it computes the group's Philox block, whose byte b holds the octet's 8 signs of

@@ -4,7 +4,8 @@ Splitting probe evaluation across devices needs no gradient communication
 ("Stanford's 1.5-SPSA Trains OPT-30B Without Backpropagation", section "How 1.5-SPSA
 Works", implementation paragraph: there are no gradients to communicate).  Every rank holds
 the same theta and seed, so the probes z_i are identical everywhere; rank r evaluates the
-probes i = r, r + N, r + 2N, ... .  The only exchange is an all-gather of the 2*n_pert fp64
+probes i = r, r + N, r + 2N, ... (or, with block = B, the blocks of B consecutive probes
+u = r, r + N, ...: the probe octets of the quadratic's one-pass evaluation).  The only exchange is an all-gather of the 2*n_pert fp64
 losses; afterwards every rank runs the same deterministic preconditioner and update, so the
 replicas of theta stay bit-identical with no parameter traffic.
 
@@ -18,41 +19,49 @@ import torch
 import torch.distributed as dist
 
 
-def rank_probes(n_pert, rank, world):
-    """Probes evaluated by `rank`, ascending: i = rank (mod world)."""
-    if not (0 <= rank < world) or n_pert < 1:
+def rank_units(n_pert, rank, world, block=1):
+    """(first, count) of the probe blocks evaluated by `rank`: blocks u = rank (mod world)
+    of `block` consecutive probes (the last block may be short)."""
+    if not (0 <= rank < world) or n_pert < 1 or block < 1:
         raise ValueError("bad partition arguments")
-    return list(range(rank, n_pert, world))
+    units = math.ceil(n_pert / block)
+    return [(u * block, min(block, n_pert - u * block)) for u in range(rank, units, world)]
 
 
-def slots(n_pert, world):
+def rank_probes(n_pert, rank, world, block=1):
+    """Probes evaluated by `rank`, ascending."""
+    return [f + t for f, c in rank_units(n_pert, rank, world, block) for t in range(c)]
+
+
+def slots(n_pert, world, block=1):
     """Loss slots per rank in the exchange buffer (the largest share)."""
-    return math.ceil(n_pert / world)
+    return max(len(rank_probes(n_pert, r, world, block)) for r in range(world))
 
 
-def global_order(n_pert, world, device=None):
+def global_order(n_pert, world, device=None, block=1):
     """Index of each gathered slot in the global probe order, -1 for padding.
 
-    The gathered buffer is [world][2][slots]; entry (r, s, k) holds probe r + k*world."""
-    k = slots(n_pert, world)
+    The gathered buffer is [world][2][slots]; entry (r, s, k) holds the k-th probe of
+    rank_probes(n_pert, r, world, block)."""
+    k = slots(n_pert, world, block)
     idx = torch.full((world, k), -1, dtype=torch.long)
     for r in range(world):
-        p = rank_probes(n_pert, r, world)
+        p = rank_probes(n_pert, r, world, block)
         idx[r, :len(p)] = torch.tensor(p, dtype=torch.long)
     return idx.to(device) if device is not None else idx
 
 
-def gather_losses(local, n_pert, group=None):
+def gather_losses(local, n_pert, group=None, block=1):
     """All-gather every rank's [2][slots] losses (row 0: L+, row 1: L-) and return the
     full (L+[n_pert], L-[n_pert]) in global probe order, on every rank."""
     world = dist.get_world_size(group)
-    k = slots(n_pert, world)
+    k = slots(n_pert, world, block)
     if tuple(local.shape) != (2, k):
         raise ValueError(f"local losses must be [2][{k}]")
     parts = [torch.empty_like(local) for _ in range(world)]
     dist.all_gather(parts, local.contiguous(), group=group)
     full = torch.stack(parts)  # [world][2][k]
-    idx = global_order(n_pert, world, full.device)
+    idx = global_order(n_pert, world, full.device, block)
     valid = idx >= 0
     Lp = torch.empty(n_pert, dtype=local.dtype, device=local.device)
     Lm = torch.empty(n_pert, dtype=local.dtype, device=local.device)
@@ -62,26 +71,37 @@ def gather_losses(local, n_pert, group=None):
 
 
 def probe_parallel_step(n_pert, loss_at, clean_loss, apply_step, device, dtype=torch.float64,
-                        group=None, pair_at=None):
+                        group=None, pair_at=None, block=1, block_at=None):
     """One step with this rank's share of the probes.
 
     loss_at(sign, probe, out) writes L(theta + sign*eps*z_probe) into the 1-element tensor
     `out`; pair_at(probe, out_plus, out_minus), if given, writes both signs at once instead;
+    block_at(first, count, out_plus, out_minus), if given, writes both signs of the `count`
+    probes from `first` (one block of the partition, `block` probes) at once;
     clean_loss(out) writes L0 (every rank computes it: same theta, same data, same value, no
     exchange); apply_step(Lp, Lm, L0) runs the preconditioner and the update.
     Returns (L0, Lp, Lm)."""
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
-    k = slots(n_pert, world)
+    if block_at is None:
+        block = 1
+    k = slots(n_pert, world, block)
     local = torch.zeros((2, k), dtype=dtype, device=device)
     L0 = torch.zeros(1, dtype=dtype, device=device)
     clean_loss(L0)
-    for j, i in enumerate(rank_probes(n_pert, rank, world)):
-        if pair_at is not None:
-            pair_at(i, local[0, j:j + 1], local[1, j:j + 1])
+    j = 0
+    for first, count in rank_units(n_pert, rank, world, block):
+        if block_at is not None:
+            block_at(first, count, local[0, j:j + count], local[1, j:j + count])
         else:
-            loss_at(+1, i, local[0, j:j + 1])
-            loss_at(-1, i, local[1, j:j + 1])
-    Lp, Lm = gather_losses(local, n_pert, group)
+            for i in range(first, first + count):
+                jj = j + i - first
+                if pair_at is not None:
+                    pair_at(i, local[0, jj:jj + 1], local[1, jj:jj + 1])
+                else:
+                    loss_at(+1, i, local[0, jj:jj + 1])
+                    loss_at(-1, i, local[1, jj:jj + 1])
+        j += count
+    Lp, Lm = gather_losses(local, n_pert, group, block)
     apply_step(Lp, Lm, L0)
     return L0, Lp, Lm
