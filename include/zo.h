@@ -469,7 +469,9 @@ zo_status zo_debug_gemm_timeout(zo_ctx *ctx, const void *A, const void *B, void 
 
 /* Causal multi-head attention: qkv device bf16 [batch*seq][3*d_model] (q, k, v at column
  * offsets 0, d, 2d; head h at +h*hd), out device bf16 [batch*seq][d_model];
- * softmax(q.k^T / sqrt(hd)) over keys <= query, hd = d_model/n_heads in {64, 128}. */
+ * softmax(q.k^T / sqrt(hd)) over keys <= query, hd = d_model/n_heads in {64, 128}.  Runs on
+ * the tcgen05 tensor cores: fp32 scores, probabilities rounded to bf16 for P V, fp32
+ * accumulation, one bf16 rounding of the output. */
 zo_status zo_attention(zo_ctx *ctx, const void *qkv, void *out, int32_t batch, int32_t seq,
                        int32_t n_heads, int32_t d_model);
 
