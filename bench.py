@@ -4,7 +4,7 @@
 Workload (the default, one GPU): L = 1/2 sum_j D_j theta_j^2 with M = 2^24 fp32
 parameters, D_j log-uniform in [1e-3, 1e3], theta_0 ~ N(0, 1); n_pert = 64,
 eps = 1e-3, lr = 4e-7, damping = 1e-3, 1.5-SPSA.  One step = clean loss + 2*n_pert
-perturbed losses (the 16 losses of each probe octet from one pass over theta and D) +
+perturbed losses (the 32 losses of each two probe octets from one pass over theta and D) +
 preconditioner + update, all through the C ABI of libzo.so.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -42,11 +42,16 @@ FALLBACK_HBM_GBS = 6650.0
 
 # DRAM bytes (read + write) per launch of the octet loss kernel from the ncu capture
 # summarised in profiles/quad_octet_kernel.quadratic_M2p24.md, valid for the kernel sources
-# whose SHA-256 (of zo_loss.cu, zo_internal.cuh and zo_tc.cuh, concatenated) is recorded
-# with it; reported as null when a source has changed since the capture.
-LOSS_TRAFFIC = {"sources_sha256": "4a84d525dcd5fe39c19878adf9f4e370982c6b27459898565928a4cedd483eed",
-                "bytes": 139.6e6}
-LOSS_SOURCES = ("zo_loss.cu", "zo_internal.cuh", "zo_tc.cuh")
+# whose SHA-256 (of zo_loss.cu and zo_internal.cuh, concatenated) is recorded with it;
+# reported as null when a source has changed since the capture.
+LOSS_TRAFFIC = {"sources_sha256": "2cc2d6dc244cd2ccb386fb3a99781ddac60b79ddda3ae0ed1ee57f7e7c5eebab",
+                "bytes": 138.7e6}
+LOSS_SOURCES = ("zo_loss.cu", "zo_internal.cuh")
+# Warp instructions one launch of the loss kernel executes (ncu smsp__inst_executed.sum, same
+# capture and validity rule as LOSS_TRAFFIC): the pass is bound by instruction issue, so its
+# roofline is the issue limit, 148 SMs x 4 warp-instructions per clock at the sampled clock.
+LOSS_WARP_INSTRUCTIONS = 55.36e6
+SM_COUNT, ISSUE_PER_SM_CLOCK = 148, 4
 
 
 def loss_sources_sha256():
@@ -257,7 +262,7 @@ def gpu_arm(args):
         if world > 1:  # probe-parallel: this rank's probe octets, loss all-gather, same update
             from zero_order_forward_b200 import dist as zdist
             zdist.probe_parallel_step(n, loss_at, lambda o: zo.zo_quad_loss(ctx, D, o),
-                                      apply_step, dev, block=8, block_at=octet_at)
+                                      apply_step, dev, block=16, block_at=octet_at)
         else:  # the native step driver: every launch of the step enqueued from C++
             zo.zo_quad_step(ctx, D, n, EPS, LR, DAMPING, True, losses)
 
@@ -296,17 +301,17 @@ def gpu_arm(args):
     value = args.steps / total_s  # steps of the one shared model
 
     # dominant kernel: the loss pass (perturbation on load).  At one GPU the probe phase
-    # holds n/8 launches of the octet kernel (the 16 losses L(theta +- eps z_i) of 8 probes
-    # from one pass over theta and D); with N ranks the phase is not bracketed separately:
-    # time the octet kernel alone.
-    n_oct = (n + 7) // 8
+    # holds n/16 launches of the octet kernel (the 32 losses L(theta +- eps z_i) of two probe
+    # octets from one pass over theta and D); with N ranks the phase is not bracketed
+    # separately: time the kernel alone.
+    n_oct = (n + 15) // 16
     if world > 1:
         le = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         flush.zero_()
         le[0].record(stream)
         for o in range(n_oct):
-            zo.zo_quad_loss_octet(ctx, D, 8 * o, min(8, n - 8 * o), EPS, losses[1:9], losses[9:17],
-                                  losses[0:1] if o == 0 else None)
+            zo.zo_quad_loss_octet(ctx, D, 16 * o, min(16, n - 16 * o), EPS, losses[1:17],
+                                  losses[17:33], losses[0:1] if o == 0 else None)
         le[1].record(stream)
         torch.cuda.synchronize()
         probe_ms = [le[0].elapsed_time(le[1])]
@@ -340,16 +345,16 @@ def gpu_arm(args):
     # end to end through the public API with host buffers: D copied in, losses copied out
     D_host = torch.from_numpy(D_np).pin_memory()
     L_host = torch.zeros(2 * n + 1, dtype=torch.float64).pin_memory()
-    e2e_steps = max(3, min(args.steps, 10))
+    e2e_steps = max(3, min(args.steps, 30))
 
     def e2e_step():
-        if world == 1:
-            zo.zo_quad_step_host(ctx, D_host, n, EPS, LR, DAMPING, True, L_host)
+        if world == 1:  # pipelined: step k+1's copy of D overlaps step k's kernels
+            zo.zo_quad_step_host_async(ctx, D_host, n, EPS, LR, DAMPING, True, L_host)
             return
         D.copy_(D_host, non_blocking=True)
         from zero_order_forward_b200 import dist as zdist
         L0, Lp, Lm = zdist.probe_parallel_step(n, loss_at, lambda o: zo.zo_quad_loss(ctx, D, o),
-                                               apply_step, dev, pair_at=pair_at)
+                                               apply_step, dev, block=16, block_at=octet_at)
         L_host.copy_(torch.cat([L0, Lp, Lm]))  # synchronous device -> host read
     e2e_step()  # staging allocation
     if world > 1:
@@ -385,8 +390,8 @@ def gpu_arm(args):
             "config": {"workload": WORKLOAD, "M": M_FULL, "n_pert": n, "eps": EPS, "lr": LR,
                        "damping": DAMPING, "parallelism": f"probe-parallel x{world}",
                        "l2": "flushed between steps (256 MiB write, untimed); theta+D = 128 MiB"},
-            "roofline": {"kernel": "quad_octet_kernel (the 16 losses L(theta +- eps z_i) of a "
-                                   "probe octet in one pass, perturbation on load, fp64 "
+            "roofline": {"kernel": "quad_octet_kernel (the 32 losses L(theta +- eps z_i) of two "
+                                   "probe octets in one pass, perturbation on load, fp64 "
                                    "accumulation)",
                          "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "peak_kind": peak_kind,
@@ -409,11 +414,23 @@ def gpu_arm(args):
             "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": 4 * M_FULL * world,
                     "d2h_bytes_per_step": 8 * (2 * n + 1) * world,
                     "path": "D pinned host -> device every step on every rank, losses back "
-                            "(zo_quad_step_host at one GPU)"},
+                            "(zo_quad_step_host_async at one GPU: copies on the context's copy "
+                            "stream overlap the previous step's kernels)"},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
         }
         line["roofline"]["traffic"] = args.traffic if args.traffic is not None else loss_traffic()
+        if loss_traffic() is not None:  # the recorded instruction count is valid: issue roofline
+            mhz = (clocks or {}).get("sm_mhz") or 1965.0
+            peak_inst = SM_COUNT * ISSUE_PER_SM_CLOCK * mhz * 1e6 / 1e9  # G warp-instr/s
+            ach_inst = LOSS_WARP_INSTRUCTIONS / (loss_us * 1e-6) / 1e9
+            hbm_view = {k: line["roofline"][k] for k in ("achieved", "peak", "unit", "frac")}
+            line["roofline"].update({
+                "bound": "alu", "achieved": ach_inst, "peak": peak_inst,
+                "unit": "G warp-instructions/s", "frac": ach_inst / peak_inst,
+                "peak_kind": f"issue limit: {SM_COUNT} SMs x {ISSUE_PER_SM_CLOCK} per clock at "
+                             f"{mhz:.0f} MHz",
+                "warp_instructions_per_launch": LOSS_WARP_INSTRUCTIONS, "hbm_view": hbm_view})
     ctx.close()
     if world > 1:
         dist.barrier()

@@ -202,8 +202,8 @@ zo_status zo_quad_loss_pair(zo_ctx *ctx, const float *D, int32_t probe, float ep
                             double *loss_plus, double *loss_minus);
 
 /* The 2*count losses of the probes first_probe .. first_probe+count-1 (first_probe a
- * multiple of 8, count 1..8: the probes of one octet, whose signs share one generator
- * block) from ONE pass over theta and D: L(theta + eps z_i) -> loss_plus[i - first_probe],
+ * multiple of 8, count 1..16: the probes of one or two octets; an octet's signs share one
+ * generator block) from ONE pass over theta and D: L(theta + eps z_i) -> loss_plus[i - first_probe],
  * L(theta - eps z_i) -> loss_minus[i - first_probe] (device doubles).  Each element has
  * two perturbed values, rd(theta_j + eps) and rd(theta_j - eps), and each loss takes one of
  * them per element: L+_i is the fp64 sum of its M terms, and L-_i, which takes the other
@@ -307,6 +307,16 @@ zo_status zo_quad_step(zo_ctx *ctx, const float *D, int32_t n_pert, float eps, f
 zo_status zo_quad_step_host(zo_ctx *ctx, const float *D_host, int32_t n_pert, float eps,
                             float lr, float damping, int preconditioned,
                             double *losses_host);
+
+/* The same step without the final synchronisation, for pipelining: the copy of D (host,
+ * M floats, pinned) runs on the context's own copy stream into one of two device staging
+ * slots, so the next call's copy overlaps this step's kernels; the losses are copied back
+ * to losses_host (pinned) on the context's stream.  D_host and losses_host must stay valid,
+ * and losses_host unread, until the context's stream has been synchronised (zo_sync or the
+ * caller's stream synchronisation).  Staging slots are owned by the context. */
+zo_status zo_quad_step_host_async(zo_ctx *ctx, const float *D_host, int32_t n_pert, float eps,
+                                  float lr, float damping, int preconditioned,
+                                  double *losses_host);
 
 /* One full MLP step [LOOP] (live buffer enabled by the call if needed): clean loss,
  * 2*n_pert perturbed losses through the live buffer, zo_step.  Arguments as

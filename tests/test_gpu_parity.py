@@ -431,7 +431,7 @@ def test_quad_loss_pair_is_bit_identical_to_two_passes(zo, M):
 
 
 @pytest.mark.parametrize("M", [1, 7, 4096 * 3 + 5, 1 << 20, (1 << 22) + 17])
-@pytest.mark.parametrize("first,count", [(0, 8), (16, 8), (8, 3)])
+@pytest.mark.parametrize("first,count", [(0, 8), (16, 8), (8, 3), (0, 16), (24, 11)])
 def test_quad_loss_octet_matches_pairs_and_oracle(zo, M, first, count):
     """zo_quad_loss_octet computes the 2*count losses of one probe octet in one pass (each
     element's two perturbed values, each loss taking one per element; L- from the common
@@ -442,8 +442,8 @@ def test_quad_loss_octet_matches_pairs_and_oracle(zo, M, first, count):
     th, D = dev(th_np), dev(D_np)
     ctx = zo.zo_create(th, seed=6)
     zo.zo_set_step(ctx, 2)
-    oct_p = torch.full((9,), -7.0, dtype=torch.float64, device="cuda")
-    oct_m = torch.full((9,), -7.0, dtype=torch.float64, device="cuda")
+    oct_p = torch.full((17,), -7.0, dtype=torch.float64, device="cuda")
+    oct_m = torch.full((17,), -7.0, dtype=torch.float64, device="cuda")
     clean = torch.zeros(2, dtype=torch.float64, device="cuda")
     zo.zo_quad_loss_octet(ctx, D, first, count, 1e-3, oct_p, oct_m, clean[0:1])
     zo.zo_quad_loss(ctx, D, clean[1:2])
@@ -464,4 +464,29 @@ def test_quad_loss_octet_matches_pairs_and_oracle(zo, M, first, count):
         assert abs(P[t] - refp) <= 1e-12 * refp and abs(Mn[t] - refm) <= 1e-12 * refm
     with pytest.raises(zo.ZoError):
         zo.zo_quad_loss_octet(ctx, D, 3, 8, 1e-3, oct_p, oct_m)  # not an octet boundary
+    with pytest.raises(zo.ZoError):
+        zo.zo_quad_loss_octet(ctx, D, 0, 17, 1e-3, oct_p, oct_m)  # more than two octets
     ctx.close()
+
+
+def test_pipelined_host_steps_equal_synchronous_steps(zo):
+    """zo_quad_step_host_async (D copied on the context's copy stream into alternating
+    staging slots, no synchronisation) gives the same theta, step counter and losses as
+    the synchronous host-buffer step, bit for bit."""
+    M, n = (1 << 16) + 5, 16
+    th_np, D_np = synth.quad_problem(M, seed=21)
+    D_pin = torch.from_numpy(D_np).pin_memory()
+    a, b = dev(th_np), dev(th_np)
+    ca, cb = zo.zo_create(a, seed=3), zo.zo_create(b, seed=3)
+    La = torch.zeros((4, 2 * n + 1), dtype=torch.float64).pin_memory()
+    Lb = torch.zeros((4, 2 * n + 1), dtype=torch.float64).pin_memory()
+    for k in range(4):
+        zo.zo_quad_step_host(ca, D_pin, n, 1e-3, 1e-5, 1e-3, True, La[k])
+        zo.zo_quad_step_host_async(cb, D_pin, n, 1e-3, 1e-5, 1e-3, True, Lb[k])
+    assert zo.zo_sync(cb) == 0 and zo.zo_sync(ca) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+    assert torch.equal(La, Lb)
+    assert zo.zo_get_step(ca) == zo.zo_get_step(cb) == 4
+    ca.close()
+    cb.close()

@@ -50,6 +50,7 @@ _SIGS = {
     "zo_get_precond": [_vp, _i32, _vp, _vp, _vp, _vp],
     "zo_quad_step": [_vp, _vp, _i32, _f32, _f32, _f32, _int, _vp],
     "zo_quad_step_host": [_vp, _vp, _i32, _f32, _f32, _f32, _int, _vp],
+    "zo_quad_step_host_async": [_vp, _vp, _i32, _f32, _f32, _f32, _int, _vp],
     "zo_mlp_step": [_vp, _vp, _vp, _int, _int, _int, _int, _i32, _f32, _f32, _f32, _int, _vp],
     "zo_mlp_loss_noalloc": [_vp, _vp, _vp, _int, _int, _int, _int, _f64, _vp, _int, _vp],
     "zo_enable_phase_timing": [_vp, _i32],
@@ -249,6 +250,11 @@ def zo_quad_step(ctx, D, n_pert, eps, lr, damping, preconditioned, losses_out):
 
 def zo_quad_step_host(ctx, D_host, n_pert, eps, lr, damping, preconditioned, losses_host):
     return ctx.check(_L.zo_quad_step_host(ctx.handle, _ptr(D_host), n_pert, eps, lr, damping,
+                                          int(preconditioned), _ptr(losses_host)))
+
+
+def zo_quad_step_host_async(ctx, D_host, n_pert, eps, lr, damping, preconditioned, losses_host):
+    return ctx.check(_L.zo_quad_step_host_async(ctx.handle, _ptr(D_host), n_pert, eps, lr, damping,
                                           int(preconditioned), _ptr(losses_host)))
 
 

@@ -239,14 +239,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
       if (lane == 0) tc::mbar_arrive(s_free);  // S may be overwritten by the next tile
       const int key0 = j * kTBN;
       const bool edge = key0 + kTBN - 1 > q_first || key0 + kTBN > a.S;
-      float mx = -INFINITY;
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // 4 independent chains
 #pragma unroll
       for (int c = 0; c < kTBN; ++c) {
         float v = s[c] * a.scale_log2;
         if (edge && (key0 + c > r || key0 + c >= a.S)) v = -INFINITY;
         s[c] = v;
-        mx = fmaxf(mx, v);
+        mx4[c & 3] = fmaxf(mx4[c & 3], v);
       }
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       const float m_new = fmaxf(m_used, mx);
       // Lazy rescaling: keep the running maximum unless it grows by more than 2^8 (then
       // O and l are rescaled below, once the previous tile's P V has completed).
@@ -255,13 +256,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
       if (j == 0 || need) m_used = m_new;
       const float msc = m_used == -INFINITY ? 0.f : m_used;
       uint32_t pk[kTBN / 2];
-      float lsum = 0.f;
+      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < kTBN; c += 2) {
         const float p0 = ex2(s[c] - msc), p1 = ex2(s[c + 1] - msc);
-        lsum += p0 + p1;
+        ls4[(c >> 1) & 3] += p0 + p1;
         pk[c / 2] = pack2_bf16(p0, p1);
       }
+      const float lsum = (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
       if (j > 0) {
         // P and O are free once the previous tile's P V has completed
         if (!warp_wait(pv_done, (uint32_t)(j - 1) & 1u, abort_flag)) { ok = false; break; }

@@ -166,6 +166,14 @@ zo_status zo_destroy(zo_ctx *ctx) {
   cudaFree(ctx->live);
   cudaFree(ctx->staging);
   cudaFree(ctx->loss_scratch);
+  if (ctx->copy_stream) cudaStreamSynchronize(ctx->copy_stream);
+  for (int b = 0; b < 2; ++b) {
+    cudaFree(ctx->pipe_d[b]);
+    cudaFree(ctx->pipe_l[b]);
+    if (ctx->pipe_copied[b]) cudaEventDestroy(ctx->pipe_copied[b]);
+    if (ctx->pipe_consumed[b]) cudaEventDestroy(ctx->pipe_consumed[b]);
+  }
+  if (ctx->copy_stream) cudaStreamDestroy(ctx->copy_stream);
   if (ctx->phase_ev) {
     for (int i = 0; i < 4 * ctx->phase_cap; ++i) cudaEventDestroy(ctx->phase_ev[i]);
     delete[] ctx->phase_ev;
@@ -448,8 +456,8 @@ zo_status zo_quad_loss_octet(zo_ctx *ctx, const float *D, int32_t first_probe, i
   if (ctx->dtype != ZO_F32) return fail(ctx, ZO_ERR_UNSUPPORTED, "quadratic loss needs an fp32 context");
   if (!D || !loss_plus || !loss_minus || !aligned16(D))
     return fail(ctx, ZO_ERR_INVALID, "D must be a 16-byte aligned device pointer; outputs non-null");
-  if (first_probe < 0 || first_probe % 8 || count < 1 || count > 8 || !(eps > 0.f) || !std::isfinite(eps))
-    return fail(ctx, ZO_ERR_INVALID, "first_probe must be a multiple of 8, count 1..8, eps > 0");
+  if (first_probe < 0 || first_probe % 8 || count < 1 || count > 16 || !(eps > 0.f) || !std::isfinite(eps))
+    return fail(ctx, ZO_ERR_INVALID, "first_probe must be a multiple of 8, count 1..16, eps > 0");
   if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "octet evaluation needs the clean state");
   ProbeKey pk = probe_key(ctx);
   pk.sign = +1;
@@ -469,14 +477,43 @@ zo_status zo_quad_step(zo_ctx *ctx, const float *D, int32_t n_pert, float eps, f
   if (!preconditioned)
     ZO_CUDA(ctx, cudaMemsetAsync(L0, 0, sizeof(double), ctx->stream), "clear L0");
   phase_mark(ctx, 1);
-  // the 16 losses of a probe octet from one pass; the first pass also adds the clean loss
-  for (int32_t i = 0; i < n_pert; i += 8)
-    ZO_CHECK(zo_quad_loss_octet(ctx, D, i, n_pert - i < 8 ? n_pert - i : 8, eps, Lp + i, Lm + i,
+  // the 32 losses of two probe octets from one pass; the first pass also adds the clean loss
+  for (int32_t i = 0; i < n_pert; i += 16)
+    ZO_CHECK(zo_quad_loss_octet(ctx, D, i, n_pert - i < 16 ? n_pert - i : 16, eps, Lp + i, Lm + i,
                                 (preconditioned && i == 0) ? L0 : nullptr));
   phase_mark(ctx, 2);
   const zo_status st = zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
   phase_mark(ctx, 3);
   return st;
+}
+
+zo_status zo_quad_step_host_async(zo_ctx *ctx, const float *D_host, int32_t n_pert, float eps,
+                                  float lr, float damping, int preconditioned, double *losses_host) {
+  ZO_CHECK(check_ctx(ctx));
+  ZO_CHECK(check_step_args(ctx, n_pert, lr, eps, damping));
+  if (!D_host || !losses_host) return fail(ctx, ZO_ERR_INVALID, "null host buffer");
+  if (!ctx->copy_stream) {
+    ZO_CUDA(ctx, cudaStreamCreateWithFlags(&ctx->copy_stream, cudaStreamNonBlocking), "copy stream");
+    for (int b = 0; b < 2; ++b) {
+      ZO_CUDA(ctx, cudaMalloc(&ctx->pipe_d[b], (size_t)ctx->M * sizeof(float)), "staging slot");
+      ZO_CUDA(ctx, cudaMalloc(&ctx->pipe_l[b], (2 * ZO_MAX_PROBES + 1) * sizeof(double)), "loss slot");
+      ZO_CUDA(ctx, cudaEventCreateWithFlags(&ctx->pipe_copied[b], cudaEventDisableTiming), "event");
+      ZO_CUDA(ctx, cudaEventCreateWithFlags(&ctx->pipe_consumed[b], cudaEventDisableTiming), "event");
+      ZO_CUDA(ctx, cudaEventRecord(ctx->pipe_consumed[b], ctx->stream), "event");
+    }
+  }
+  const int b = (int)(ctx->pipe_k++ & 1u);
+  // the slot's previous step must have finished reading it before it is refilled
+  ZO_CUDA(ctx, cudaStreamWaitEvent(ctx->copy_stream, ctx->pipe_consumed[b], 0), "wait slot");
+  ZO_CUDA(ctx, cudaMemcpyAsync(ctx->pipe_d[b], D_host, (size_t)ctx->M * sizeof(float),
+                               cudaMemcpyHostToDevice, ctx->copy_stream), "copy D");
+  ZO_CUDA(ctx, cudaEventRecord(ctx->pipe_copied[b], ctx->copy_stream), "event");
+  ZO_CUDA(ctx, cudaStreamWaitEvent(ctx->stream, ctx->pipe_copied[b], 0), "wait copy");
+  ZO_CHECK(zo_quad_step(ctx, ctx->pipe_d[b], n_pert, eps, lr, damping, preconditioned, ctx->pipe_l[b]));
+  ZO_CUDA(ctx, cudaEventRecord(ctx->pipe_consumed[b], ctx->stream), "event");
+  ZO_CUDA(ctx, cudaMemcpyAsync(losses_host, ctx->pipe_l[b], (2 * n_pert + 1) * sizeof(double),
+                               cudaMemcpyDeviceToHost, ctx->stream), "copy losses");
+  return ZO_OK;
 }
 
 zo_status zo_quad_step_host(zo_ctx *ctx, const float *D_host, int32_t n_pert, float eps,

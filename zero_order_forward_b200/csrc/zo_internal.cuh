@@ -127,6 +127,13 @@ struct zo_ctx {
   float *staging = nullptr;    // device staging for host-buffer entry points
   double *loss_scratch = nullptr;  // 2*ZO_MAX_PROBES+1 doubles for host-buffer steps
 
+  // pipelined host-buffer steps: two staging slots, a copy stream, per-slot events
+  float *pipe_d[2] = {nullptr, nullptr};
+  double *pipe_l[2] = {nullptr, nullptr};
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t pipe_copied[2] = {nullptr, nullptr}, pipe_consumed[2] = {nullptr, nullptr};
+  uint64_t pipe_k = 0;
+
   // phase timing of the step drivers: 4 events per recorded step
   cudaEvent_t *phase_ev = nullptr;
   int32_t phase_cap = 0, phase_used = 0;

@@ -376,8 +376,8 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
   }
 }
 
-// The 16 losses L(theta +- eps z_i) of the 8 probes i = 8 octet + t of one octet from one
-// pass over theta and D.  Each element has only two perturbed values, P_a = rd(theta + eps)
+// The losses L(theta +- eps z_i) of the 8 NO probes i = 8 octet + t of NO consecutive
+// octets (NO = 1 or 2: 16 or 32 losses) from one pass over theta and D.  Each element has only two perturbed values, P_a = rd(theta + eps)
 // and P_b = rd(theta - eps), with terms t_a = (D/2) P_a^2 and t_b = (D/2) P_b^2; the
 // element's byte of the octet's Philox block says which one each loss takes (bit t set:
 // L+_t takes t_b and L-_t takes t_a; clear: the reverse).  L+_t is accumulated term by term
@@ -387,7 +387,7 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
 // agree with the one-probe passes to rounding).  Probes t >= count are computed and not
 // stored.  CLEAN also adds the clean loss L(theta) to the same pass (into *out_clean,
 // bit-identical to the clean quad_loss_kernel pass).
-template <bool CLEAN>
+template <bool CLEAN, int NO>
 __global__ void __launch_bounds__(kQThreads, kOBlocksPerSm)
 quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, int64_t M,
                   ProbeKey pk, uint32_t octet, int count, int64_t n_chunks, double *partials,
@@ -398,9 +398,10 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
   const QuadPipe pipe = quad_pipe_init(qsm, &abort_flag, kOStages);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t step = *pk.step;
-  double lp[8], tsum = 0.0, l0 = 0.0;
+  constexpr int NP = 8 * NO;  // probes per pass
+  double lp[NP], tsum = 0.0, l0 = 0.0;
 #pragma unroll
-  for (int t = 0; t < 8; ++t) lp[t] = 0.0;
+  for (int t = 0; t < NP; ++t) lp[t] = 0.0;
 
   if (warp == 0) {
     quad_produce(pipe, theta, D, M, n_chunks, &abort_flag, err);
@@ -418,10 +419,12 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
       // Vector k of this thread lies in group 8 cw + 64 k + quad of the chunk, bytes 4q..4q+3
       // (word q of the block).  Lane q of the quad computes the block of iteration k = q; the
       // quad exchange hands every lane word q of all four.
-      const uint4 blk = sign_block((uint64_t)(base / kGroup) + 8 * cw + 64 * q + quad, octet, step,
-                                   pk.k0, pk.k1);
-      uint32_t W[4];
-      quad_exchange(blk, lane, W);
+      uint32_t W[NO][4];
+#pragma unroll
+      for (int o = 0; o < NO; ++o)
+        quad_exchange(sign_block((uint64_t)(base / kGroup) + 8 * cw + 64 * q + quad, octet + o, step,
+                                 pk.k0, pk.k1),
+                      lane, W[o]);
 #pragma unroll
       for (int k = 0; k < kQIters; ++k) {
         const int e = 4 * (ct + k * 32 * kQConsumers);
@@ -434,9 +437,13 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
           const double tb = quad_term(dv[qq], __fadd_rn(tv[qq], -pk.eps));
           tsum = __dadd_rn(tsum, __dadd_rn(ta, tb));
           if (CLEAN) l0 = __dadd_rn(l0, quad_term(dv[qq], tv[qq]));
-          const uint32_t byte = W[k] >> (8 * qq);
 #pragma unroll
-          for (int t = 0; t < 8; ++t) lp[t] = __dadd_rn(lp[t], ((byte >> t) & 1u) ? tb : ta);
+          for (int o = 0; o < NO; ++o) {
+            const uint32_t byte = W[o][k] >> (8 * qq);
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+              lp[8 * o + t] = __dadd_rn(lp[8 * o + t], ((byte >> t) & 1u) ? tb : ta);
+          }
         }
       }
       __syncwarp();
@@ -445,18 +452,18 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
   }
   tc::pdl_launch_dependents();
   tc::pdl_wait();
-  constexpr int NV = CLEAN ? 10 : 9;
+  constexpr int NV = NP + (CLEAN ? 2 : 1);
   double v[NV], tot[NV];
 #pragma unroll
-  for (int t = 0; t < 8; ++t) v[t] = block_sum(lp[t]);
-  v[8] = block_sum(tsum);
+  for (int t = 0; t < NP; ++t) v[t] = block_sum(lp[t]);
+  v[NP] = block_sum(tsum);
   if (CLEAN) v[NV - 1] = block_sum(l0);
   if (last_block_totals<NV>(v, partials, counter, tot)) {
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
+    for (int t = 0; t < NP; ++t) {
       if (t < count) {
         out_plus[t] = tot[t];
-        out_minus[t] = tot[8] - tot[t];
+        out_minus[t] = tot[NP] - tot[t];
       }
     }
     if (CLEAN) *out_clean = tot[NV - 1];
@@ -560,16 +567,17 @@ zo_status launch_quad_loss_pair(zo_ctx *ctx, const ProbeKey &pk, const float *D,
   return launch_quad<true, 0>(ctx, pk, D, out_plus, out_minus, 0, ctx->partials, ctx->counter);
 }
 
-template <bool CLEAN>
+template <bool CLEAN, int NO>
 zo_status launch_quad_octet_t(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, int count,
                               const float *D, double *out_plus, double *out_minus, double *out_clean) {
   const int64_t n_chunks = (ctx->M + kQChunk - 1) / kQChunk;
   const int64_t cap = (int64_t)kSmCount * kOBlocksPerSm;
   const int64_t blocks = n_chunks < cap ? n_chunks : cap;
-  static_assert(10 * kSmCount * kOBlocksPerSm <= kMaxPartials, "partials too small for the octet pass");
+  static_assert((8 * NO + 2) * kSmCount * kOBlocksPerSm <= kMaxPartials,
+                "partials too small for the octet pass");
   static bool attr = false;
   if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(quad_octet_kernel<CLEAN>,
+    const cudaError_t e = cudaFuncSetAttribute(quad_octet_kernel<CLEAN, NO>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kOSmemBytes);
     if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "quad_octet_kernel attribute: %s", cudaGetErrorString(e));
     attr = true;
@@ -584,7 +592,7 @@ zo_status launch_quad_octet_t(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, i
   attr_pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr_pdl;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, quad_octet_kernel<CLEAN>,
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, quad_octet_kernel<CLEAN, NO>,
                                            static_cast<const float *>(ctx->params), D, ctx->M, pk,
                                            octet, count, n_chunks, ctx->partials, ctx->counter,
                                            out_plus, out_minus, out_clean, &ctx->dstate->flags);
@@ -594,8 +602,11 @@ zo_status launch_quad_octet_t(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, i
 
 zo_status launch_quad_octet(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, int count,
                             const float *D, double *out_plus, double *out_minus, double *out_clean) {
-  return out_clean ? launch_quad_octet_t<true>(ctx, pk, octet, count, D, out_plus, out_minus, out_clean)
-                   : launch_quad_octet_t<false>(ctx, pk, octet, count, D, out_plus, out_minus, nullptr);
+  if (count > 8)
+    return out_clean ? launch_quad_octet_t<true, 2>(ctx, pk, octet, count, D, out_plus, out_minus, out_clean)
+                     : launch_quad_octet_t<false, 2>(ctx, pk, octet, count, D, out_plus, out_minus, nullptr);
+  return out_clean ? launch_quad_octet_t<true, 1>(ctx, pk, octet, count, D, out_plus, out_minus, out_clean)
+                   : launch_quad_octet_t<false, 1>(ctx, pk, octet, count, D, out_plus, out_minus, nullptr);
 }
 
 zo_status launch_lowrank_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, const float lam[4],
