@@ -4,7 +4,7 @@
 Workload (the default, one GPU): L = 1/2 sum_j D_j theta_j^2 with M = 2^24 fp32
 parameters, D_j log-uniform in [1e-3, 1e3], theta_0 ~ N(0, 1); n_pert = 64,
 eps = 1e-3, lr = 4e-7, damping = 1e-3, 1.5-SPSA.  One step = clean loss + 2*n_pert
-perturbed losses (the 32 losses of each two probe octets from one pass over theta and D) +
+perturbed losses (the 64 losses of each four probe octets from one pass over theta and D) +
 preconditioner + update, all through the C ABI of libzo.so.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -255,6 +255,9 @@ def gpu_arm(args):
     def apply_step(Lp, Lm, L0):
         zo.zo_step(ctx, Lp, Lm, n, L0, LR, EPS, DAMPING)
 
+    # probes per rank and pass: up to four octets, fewer when the ranks would otherwise idle
+    block = min(32, max(8, -(-(n // world) // 8) * 8))
+
     def octet_at(first, count, out_plus, out_minus):
         zo.zo_quad_loss_octet(ctx, D, first, count, EPS, out_plus, out_minus)
 
@@ -262,7 +265,7 @@ def gpu_arm(args):
         if world > 1:  # probe-parallel: this rank's probe octets, loss all-gather, same update
             from zero_order_forward_b200 import dist as zdist
             zdist.probe_parallel_step(n, loss_at, lambda o: zo.zo_quad_loss(ctx, D, o),
-                                      apply_step, dev, block=16, block_at=octet_at)
+                                      apply_step, dev, block=block, block_at=octet_at)
         else:  # the native step driver: every launch of the step enqueued from C++
             zo.zo_quad_step(ctx, D, n, EPS, LR, DAMPING, True, losses)
 
@@ -301,17 +304,17 @@ def gpu_arm(args):
     value = args.steps / total_s  # steps of the one shared model
 
     # dominant kernel: the loss pass (perturbation on load).  At one GPU the probe phase
-    # holds n/16 launches of the octet kernel (the 32 losses L(theta +- eps z_i) of two probe
+    # holds n/32 launches of the octet kernel (the 64 losses L(theta +- eps z_i) of four probe
     # octets from one pass over theta and D); with N ranks the phase is not bracketed
     # separately: time the kernel alone.
-    n_oct = (n + 15) // 16
+    n_oct = (n + 31) // 32
     if world > 1:
         le = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         flush.zero_()
         le[0].record(stream)
         for o in range(n_oct):
-            zo.zo_quad_loss_octet(ctx, D, 16 * o, min(16, n - 16 * o), EPS, losses[1:17],
-                                  losses[17:33], losses[0:1] if o == 0 else None)
+            zo.zo_quad_loss_octet(ctx, D, 32 * o, min(32, n - 32 * o), EPS, losses[1:33],
+                                  losses[33:65], losses[0:1] if o == 0 else None)
         le[1].record(stream)
         torch.cuda.synchronize()
         probe_ms = [le[0].elapsed_time(le[1])]
@@ -341,6 +344,46 @@ def gpu_arm(args):
     ue[1].record(stream)
     torch.cuda.synchronize()
     upd_us = 1e3 * ue[0].elapsed_time(ue[1]) / reps
+
+    # the streaming kernels across probe counts and dtypes (theta 128 MiB, larger than L2):
+    # the update's and the unpack/apply kernel's bandwidth against the measured HBM peak
+    streaming = {}
+    if world == 1:
+        for dt, elems, esz in (("f32", 1 << 25, 4), ("bf16", 1 << 26, 2)):
+            g = torch.Generator(device=dev)
+            g.manual_seed(5)
+            th_s = (torch.randn(elems, device=dev, generator=g)
+                    .to(torch.float32 if dt == "f32" else torch.bfloat16))
+            out_s = torch.empty_like(th_s)
+            cs = zo.zo_create(th_s, seed=7, stream=stream.cuda_stream)
+            ent = {"elements": elems, "update": {}}
+            for nn in (1, 2, 4, 8, 16, 32, 64, 160):
+                cz = torch.zeros(nn, dtype=torch.float32, device=dev)  # theta unchanged
+                zo.zo_update(cs, cz, nn)
+                ue2 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                ue2[0].record(stream)
+                for _ in range(5):
+                    zo.zo_update(cs, cz, nn)
+                ue2[1].record(stream)
+                torch.cuda.synchronize()
+                us = 1e3 * ue2[0].elapsed_time(ue2[1]) / 5
+                gbs = 2 * esz * elems / (us * 1e-6) / 1e9
+                ent["update"][str(nn)] = {"us": us, "GBps": gbs, "frac_hbm": gbs / hbm_peak}
+            zo.zo_perturb(cs, +1, EPS, 3)
+            zo.zo_perturb_range(cs, 0, elems, out_s)
+            pe2 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            pe2[0].record(stream)
+            for _ in range(5):
+                zo.zo_perturb_range(cs, 0, elems, out_s)
+            pe2[1].record(stream)
+            torch.cuda.synchronize()
+            zo.zo_restore(cs)
+            us = 1e3 * pe2[0].elapsed_time(pe2[1]) / 5
+            gbs = 2 * esz * elems / (us * 1e-6) / 1e9
+            ent["perturb"] = {"us": us, "GBps": gbs, "frac_hbm": gbs / hbm_peak}
+            cs.close()
+            streaming[dt] = ent
+            del th_s, out_s
 
     # end to end through the public API with host buffers: D copied in, losses copied out
     D_host = torch.from_numpy(D_np).pin_memory()
@@ -390,7 +433,7 @@ def gpu_arm(args):
             "config": {"workload": WORKLOAD, "M": M_FULL, "n_pert": n, "eps": EPS, "lr": LR,
                        "damping": DAMPING, "parallelism": f"probe-parallel x{world}",
                        "l2": "flushed between steps (256 MiB write, untimed); theta+D = 128 MiB"},
-            "roofline": {"kernel": "quad_octet_kernel (the 32 losses L(theta +- eps z_i) of two "
+            "roofline": {"kernel": "quad_octet_kernel (the 64 losses L(theta +- eps z_i) of four "
                                    "probe octets in one pass, perturbation on load, fp64 "
                                    "accumulation)",
                          "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
@@ -406,6 +449,7 @@ def gpu_arm(args):
                                   "achieved_GBps": upd_bytes / (upd_us * 1e-6) / 1e9,
                                   "frac_hbm": upd_bytes / (upd_us * 1e-6) / 1e9 / hbm_peak},
             },
+            "streaming": streaming,
             "phases_ms": {"clean_loss": statistics.mean(clean_ms),
                           "probe_losses": statistics.mean(probe_ms),
                           "precond_update": statistics.mean(upd_ms)},

@@ -110,7 +110,7 @@ __device__ bool last_block_totals(const double v[NV], double *partials, unsigned
 // vectors 4 (ct + 256 k), k = 0..3, of every chunk and adds its terms to one accumulator
 // per loss in that order; the grid walks chunks round-robin (chunk = blockIdx.x + i gridDim.x)
 // and its size depends on M only, so every loss's summation order is fixed, and the same
-// in the single-loss, pair and octet forms (their results are bit-identical).
+// in the single-loss and pair forms (their results are bit-identical).
 constexpr int kQChunk = 4096;
 constexpr int kQStages = 3;
 constexpr int kQConsumers = 8;
@@ -118,21 +118,29 @@ constexpr int kQThreads = 32 * (1 + kQConsumers);
 constexpr int kQStageBytes = 2 * kQChunk * 4;  // theta, D
 constexpr int kQSmemBytes = kQStages * kQStageBytes + 2 * kQStages * 8;
 constexpr int kQIters = kQChunk / (4 * 32 * kQConsumers);  // 4 vectors per thread per chunk
-// The octet pass is bound by its per-probe arithmetic, not by the stream: two stages and
-// 72 registers give three CTAs (27 warps) per SM.
+// The octet pass is bound by its per-probe arithmetic, not by the stream: two stages of
+// 2048-element chunks plus the 32 KB of nibble tables and at most 72 registers give three
+// CTAs (27 warps) per SM.
+constexpr int kOChunk = 2048;
 constexpr int kOStages = 2;
-constexpr int kOSmemBytes = kOStages * kQStageBytes + 2 * kOStages * 8;
+constexpr int kOStageBytes = 2 * kOChunk * 4;
+constexpr int kOIters = kOChunk / (4 * 32 * kQConsumers);  // 2 vectors per thread per chunk
+constexpr int kOTableBytes = 16 * 32 * kQConsumers * 8;    // 16 fp64 entries per consumer thread
+constexpr int kOTableOff = kOStages * kOStageBytes + 2 * kOStages * 8;
+constexpr int kOSmemBytes = kOTableOff + kOTableBytes;
 constexpr int kOBlocksPerSm = 3;
 
 struct QuadPipe {
   uint8_t *sm;
   uint64_t *full, *empty;
   int stages;
+  int chunk;  // elements per stage; a stage holds theta then D
 };
 
 __device__ __forceinline__ QuadPipe quad_pipe_init(uint8_t *qsm, volatile int *abort_flag,
-                                                   int stages = kQStages) {
-  QuadPipe p{qsm, reinterpret_cast<uint64_t *>(qsm + stages * kQStageBytes), nullptr, stages};
+                                                   int stages = kQStages, int chunk = kQChunk) {
+  QuadPipe p{qsm, reinterpret_cast<uint64_t *>(qsm + stages * 2 * chunk * 4), nullptr, stages,
+             chunk};
   p.empty = p.full + stages;
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
@@ -163,15 +171,15 @@ __device__ __forceinline__ void quad_produce(const QuadPipe &p, const float *the
       if (lane == 0) { atomicOr(err, ZO_FLAG_TIMEOUT); *abort_flag = 1; }
       break;
     }
-    uint8_t *st = p.sm + s * kQStageBytes;
-    const int64_t base = chunk * kQChunk;
-    const int cnt = (int)(M - base < (int64_t)kQChunk ? M - base : (int64_t)kQChunk);
+    uint8_t *st = p.sm + s * 2 * p.chunk * 4;
+    const int64_t base = chunk * p.chunk;
+    const int cnt = (int)(M - base < (int64_t)p.chunk ? M - base : (int64_t)p.chunk);
     const int copy = cnt & ~3;
     if (lane == 0) {
       tc::mbar_arrive_expect_tx(&p.full[s], 2u * (uint32_t)copy * 4u);
       if (copy) {
         tc::bulk_load(st, theta + base, (uint32_t)copy * 4u, &p.full[s]);
-        tc::bulk_load(st + kQChunk * 4, D + base, (uint32_t)copy * 4u, &p.full[s]);
+        tc::bulk_load(st + p.chunk * 4, D + base, (uint32_t)copy * 4u, &p.full[s]);
       }
     }
     __syncwarp();
@@ -201,11 +209,12 @@ __device__ __forceinline__ bool quad_acquire(const QuadPipe &p, int s, uint32_t 
 }
 
 // The 4 theta and D values of vector e (0 past the end of the chunk: their terms are 0).
+template <int CHUNK = kQChunk>
 __device__ __forceinline__ void quad_load4(const uint8_t *st, const float *theta, const float *D,
                                            int64_t base, int e, int cnt, float tv[4], float dv[4]) {
   if (e + 4 <= (cnt & ~3)) {
     const float4 t = reinterpret_cast<const float4 *>(st)[e >> 2];
-    const float4 dd = reinterpret_cast<const float4 *>(st + kQChunk * 4)[e >> 2];
+    const float4 dd = reinterpret_cast<const float4 *>(st + CHUNK * 4)[e >> 2];
     tv[0] = t.x; tv[1] = t.y; tv[2] = t.z; tv[3] = t.w;
     dv[0] = dd.x; dv[1] = dd.y; dv[2] = dd.z; dv[3] = dd.w;
   } else {  // the last < 4 elements of theta (not covered by the 16-byte copies)
@@ -376,73 +385,171 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
   }
 }
 
-// The losses L(theta +- eps z_i) of the 8 NO probes i = 8 octet + t of NO consecutive
-// octets (NO = 1 or 2: 16 or 32 losses) from one pass over theta and D.  Each element has only two perturbed values, P_a = rd(theta + eps)
-// and P_b = rd(theta - eps), with terms t_a = (D/2) P_a^2 and t_b = (D/2) P_b^2; the
-// element's byte of the octet's Philox block says which one each loss takes (bit t set:
-// L+_t takes t_b and L-_t takes t_a; clear: the reverse).  L+_t is accumulated term by term
-// in quad_loss_kernel's order; L-_t takes, element by element, the other term, so
-// L-_t = sum_j (t_a + t_b)_j - L+_t exactly, and the pass accumulates the one common sum
-// T = sum_j (t_a + t_b)_j instead of eight more per-probe sums (fp64 throughout; the results
-// agree with the one-probe passes to rounding).  Probes t >= count are computed and not
-// stored.  CLEAN also adds the clean loss L(theta) to the same pass (into *out_clean,
-// bit-identical to the clean quad_loss_kernel pass).
-template <bool CLEAN, int NO>
+// Sign word of 4 elements (byte q = element q, bit t = probe t of an octet) -> 8 nibbles:
+// nibble t (bits 4t..4t+3) holds bit t of bytes 0..3.  Bit 8q + t moves to 4t + q, a
+// rotation of the 5 bit-index bits, done as four swaps of index bits (4,2), (3,1), (2,0),
+// (1,0), each a masked exchange of the bit pairs that differ in them.
+__device__ __forceinline__ uint32_t delta_swap(uint32_t x, uint32_t m, int d) {
+  const uint32_t t = ((x >> d) ^ x) & m;
+  return x ^ t ^ (t << d);
+}
+__device__ __forceinline__ uint32_t probe_nibbles(uint32_t w) {
+  w = delta_swap(w, 0x0000F0F0u, 12);
+  w = delta_swap(w, 0x00CC00CCu, 6);
+  w = delta_swap(w, 0x0A0A0A0Au, 3);
+  return delta_swap(w, 0x22222222u, 1);
+}
+// 2048 * (nibble t of x): the byte offset of that table entry (t a compile-time constant).
+__device__ __forceinline__ uint32_t nibble_offset(uint32_t x, int t) {
+  const int s = 4 * t - 11;
+  return (s >= 0 ? x >> s : x << -s) & 0x7800u;
+}
+
+// The losses L(theta +- eps z_i) of the 8 NOCT probes i = 8 octet + p, p < 8 NOCT (NOCT = 2
+// or 4 consecutive octets: 32 or 64 losses), from one pass over theta and D.
+//
+// Each element has only two perturbed values, P_a = rd(theta + eps) and P_b = rd(theta - eps),
+// with terms t_a = (D/2) P_a^2 and t_b = (D/2) P_b^2 (fp64); the sign bit of probe i says
+// which one L+_i takes (set: t_b, z = -1; clear: t_a) and L-_i takes the other, so
+// L-_i = T - L+_i with T = sum_j (t_a + t_b)_j.
+//
+// A consumer thread holds 4 consecutive elements per vector; the 4 sign bits of one probe
+// for them form a nibble, and the 16 possible sums (x_0 + x_1) + (x_2 + x_3), x_q in
+// {t_a, t_b}, go into the thread's table in shared memory once per vector.  Two neighbouring
+// lanes (a pair: adjacent vectors of one 16-element group) read each other's table: the even
+// lane accumulates the first NOCT/2 octets and the odd lane the others, for both vectors,
+// so a thread keeps 4 NOCT accumulators while each vector's terms and table serve all
+// 8 NOCT probes.  A probe then costs, per vector, a shift and a mask of the transposed
+// sign word, one table load and one fp64 add.  Summation order per loss: the vectors of a
+// thread in chunk order, each pair step adding the thread's own vector and then its
+// partner's; block and grid totals in a fixed order (8 lanes per value over a fixed
+// stride, then a butterfly).  Probes p >= count are computed and not stored.  CLEAN also
+// adds the clean loss L(theta) to the same pass (into *out_clean).
+template <bool CLEAN, int NOCT>
 __global__ void __launch_bounds__(kQThreads, kOBlocksPerSm)
 quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, int64_t M,
                   ProbeKey pk, uint32_t octet, int count, int64_t n_chunks, double *partials,
                   unsigned int *counter, double *out_plus, double *out_minus, double *out_clean,
                   uint32_t *err) {
+  static_assert(NOCT == 2 || NOCT == 4, "two or four octets per pass");
+  constexpr int LO = NOCT / 2;       // octets per thread
+  constexpr int NL = 8 * LO;         // accumulators per thread
+  constexpr int NP = 8 * NOCT;       // probes per pass
+  constexpr int NV = NP + 2;         // block values: probes, T, clean loss
+  static_assert(8 * NV <= kQThreads, "eight lanes per value in the epilogue");
+  static_assert(kOStages * kOStageBytes == 16 * 2048 && kOTableBytes == 16 * 2048 && NL + 2 <= 32,
+                "epilogue rows: 16 in the stage buffers, the rest in the tables");
   extern __shared__ __align__(128) uint8_t qsm[];
   __shared__ volatile int abort_flag;
-  const QuadPipe pipe = quad_pipe_init(qsm, &abort_flag, kOStages);
+  __shared__ double totals[NV];
+  __shared__ bool last;
+  const QuadPipe pipe = quad_pipe_init(qsm, &abort_flag, kOStages, kOChunk);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t step = *pk.step;
-  constexpr int NP = 8 * NO;  // probes per pass
-  double lp[NP], tsum = 0.0, l0 = 0.0;
+  double lp[NL], tsum = 0.0, l0 = 0.0;
 #pragma unroll
-  for (int t = 0; t < NP; ++t) lp[t] = 0.0;
+  for (int t = 0; t < NL; ++t) lp[t] = 0.0;
+  const int ct = threadIdx.x - 32;  // consumer thread 0..255 (warp 0 produces)
 
   if (warp == 0) {
     quad_produce(pipe, theta, D, M, n_chunks, &abort_flag, err);
   } else {
-    const int ct = threadIdx.x - 32;
     const int cw = ct >> 5;
-    const int q = lane & 3, quad = lane >> 2;
+    const int q = lane & 3, quad = lane >> 2, h = lane & 1;
+    const uint32_t own8 = (uint32_t)ct * 8u, par8 = (uint32_t)(ct ^ 1) * 8u;
+    uint8_t *const tab = qsm + kOTableOff;  // entry n of thread c at byte 2048 n + 8 c
     int it = 0;
     for (int64_t chunk = blockIdx.x; chunk < n_chunks; chunk += gridDim.x, ++it) {
       const int s = it % kOStages;
       if (!quad_acquire(pipe, s, (uint32_t)(it / kOStages) & 1u, &abort_flag, err)) break;
-      const uint8_t *st = pipe.sm + s * kQStageBytes;
-      const int64_t base = chunk * kQChunk;
-      const int cnt = (int)(M - base < (int64_t)kQChunk ? M - base : (int64_t)kQChunk);
-      // Vector k of this thread lies in group 8 cw + 64 k + quad of the chunk, bytes 4q..4q+3
-      // (word q of the block).  Lane q of the quad computes the block of iteration k = q; the
-      // quad exchange hands every lane word q of all four.
-      uint32_t W[NO][4];
+      const uint8_t *st = pipe.sm + s * kOStageBytes;
+      const int64_t base = chunk * kOChunk;
+      const int cnt = (int)(M - base < (int64_t)kOChunk ? M - base : (int64_t)kOChunk);
+      // Vector k of this thread lies in group g_k = 8 cw + 64 k + quad of the chunk, bytes
+      // 4q..4q+3 (word q of each block of that group); the pair's vectors are words
+      // 2 (q >> 1) and 2 (q >> 1) + 1.  The quad's lanes generate the blocks it needs and
+      // four shuffles hand each lane the pair's two words of each of its octets.
+      const uint64_t g0 = (uint64_t)(base / kGroup) + 8 * cw + quad;
+      // NOCT 2: once per chunk, lane q generates (vector q >> 1, octet q & 1); lane l reads
+      // lane l in rounds 0, 1 and lane l ^ 2 (the other vector) in rounds 2, 3.
+      uint32_t wo2[kOIters], wp2[kOIters];
+      if constexpr (NOCT == 2) {
+        const uint4 blk = sign_block(g0 + 64 * (q >> 1), octet + (uint32_t)(q & 1), step, pk.k0, pk.k1);
+        uint32_t R[4];
 #pragma unroll
-      for (int o = 0; o < NO; ++o)
-        quad_exchange(sign_block((uint64_t)(base / kGroup) + 8 * cw + 64 * q + quad, octet + o, step,
-                                 pk.k0, pk.k1),
-                      lane, W[o]);
+        for (int r = 0; r < 4; ++r) {
+          const int c = r >> 1;
+          R[r] = __shfl_sync(0xFFFFFFFFu, word_of(blk, 2 * ((q >> 1) ^ c) + (r & 1)),
+                             lane ^ (2 * c));
+        }
+        const bool x = q >> 1;  // rounds 0, 1 carried vector 1
+        const uint32_t e0 = x ? R[2] : R[0], o0 = x ? R[3] : R[1];
+        const uint32_t e1 = x ? R[0] : R[2], o1 = x ? R[1] : R[3];
+        wo2[0] = h ? o0 : e0;
+        wp2[0] = h ? e0 : o0;
+        wo2[kOIters - 1] = h ? o1 : e1;
+        wp2[kOIters - 1] = h ? e1 : o1;
+      }
 #pragma unroll
-      for (int k = 0; k < kQIters; ++k) {
+      for (int k = 0; k < kOIters; ++k) {
+        // elements past the chunk's end load as 0 (terms 0): both lanes of a pair always
+        // build a table
         const int e = 4 * (ct + k * 32 * kQConsumers);
-        if (e >= cnt) continue;
         float tv[4], dv[4];
-        quad_load4(st, theta, D, base, e, cnt, tv, dv);
+        quad_load4<kOChunk>(st, theta, D, base, e, cnt, tv, dv);
+        // wo / wp: the own / partner vector's word of each local octet j
+        uint32_t wo[LO], wp[LO];
+        if constexpr (NOCT == 4) {
+          // lane q generates octet q; lane l reads octet sw(l) in rounds 0, 1 and octet
+          // sw(l) ^ 1 in rounds 2, 3 (sw swaps the two bits of q), even word then odd
+          const int sw = ((q & 1) << 1) | (q >> 1);
+          const uint4 blk = sign_block(g0 + 64 * k, octet + (uint32_t)q, step, pk.k0, pk.k1);
+          uint32_t R[4];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int c = r >> 1;
+            R[r] = __shfl_sync(0xFFFFFFFFu, word_of(blk, 2 * ((q & 1) ^ c) + (r & 1)),
+                               (lane & ~3) | (sw ^ c));
+          }
+          const bool x = sw & 1;  // rounds 0, 1 carried local octet 1
+          const uint32_t e0 = x ? R[2] : R[0], o0 = x ? R[3] : R[1];
+          const uint32_t e1 = x ? R[0] : R[2], o1 = x ? R[1] : R[3];
+          wo[0] = h ? o0 : e0;
+          wp[0] = h ? e0 : o0;
+          wo[LO - 1] = h ? o1 : e1;
+          wp[LO - 1] = h ? e1 : o1;
+        } else {
+          wo[0] = wo2[k];
+          wp[0] = wp2[k];
+        }
+        double ta[4], tb[4];
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) {
-          const double ta = quad_term(dv[qq], __fadd_rn(tv[qq], pk.eps));
-          const double tb = quad_term(dv[qq], __fadd_rn(tv[qq], -pk.eps));
-          tsum = __dadd_rn(tsum, __dadd_rn(ta, tb));
+          ta[qq] = quad_term(dv[qq], __fadd_rn(tv[qq], pk.eps));
+          tb[qq] = quad_term(dv[qq], __fadd_rn(tv[qq], -pk.eps));
+          tsum = __dadd_rn(tsum, __dadd_rn(ta[qq], tb[qq]));
           if (CLEAN) l0 = __dadd_rn(l0, quad_term(dv[qq], tv[qq]));
+        }
+        // table entry n: element q takes t_b if bit q of n is set
+        double lo[4], hi[4];
 #pragma unroll
-          for (int o = 0; o < NO; ++o) {
-            const uint32_t byte = W[o][k] >> (8 * qq);
+        for (int n = 0; n < 4; ++n) {
+          lo[n] = __dadd_rn(n & 1 ? tb[0] : ta[0], n & 2 ? tb[1] : ta[1]);
+          hi[n] = __dadd_rn(n & 1 ? tb[2] : ta[2], n & 2 ? tb[3] : ta[3]);
+        }
+        __syncwarp();  // the partner has read this table's previous contents
 #pragma unroll
-            for (int t = 0; t < 8; ++t)
-              lp[8 * o + t] = __dadd_rn(lp[8 * o + t], ((byte >> t) & 1u) ? tb : ta);
+        for (int n = 0; n < 16; ++n)
+          *reinterpret_cast<double *>(tab + 2048 * n + own8) = __dadd_rn(lo[n & 3], hi[n >> 2]);
+        __syncwarp();  // both tables of the pair are written
+#pragma unroll
+        for (int j = 0; j < LO; ++j) {
+          const uint32_t xo = probe_nibbles(wo[j]), xp = probe_nibbles(wp[j]);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const double vo = *reinterpret_cast<const double *>(tab + (nibble_offset(xo, t) | own8));
+            const double vq = *reinterpret_cast<const double *>(tab + (nibble_offset(xp, t) | par8));
+            lp[8 * j + t] = __dadd_rn(__dadd_rn(lp[8 * j + t], vo), vq);
           }
         }
       }
@@ -451,22 +558,65 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
     }
   }
   tc::pdl_launch_dependents();
+
+  // Block totals through shared memory: row i holds accumulator i of the 256 consumer
+  // threads (rows 0..15 in the stage buffers, the rest in the tables; the mbarriers between
+  // them are left alone).  Both areas are idle once every warp has passed this barrier: the
+  // producer returned only after its copies landed.
+  __syncthreads();
+  auto red_row = [](int i) {
+    return reinterpret_cast<double *>(i < 16 ? qsm + 2048 * i : qsm + kOTableOff + 2048 * (i - 16));
+  };
+  if (warp > 0) {
+#pragma unroll
+    for (int i = 0; i < NL; ++i) red_row(i)[ct] = lp[i];
+    red_row(NL)[ct] = tsum;
+    red_row(NL + 1)[ct] = l0;
+  }
+  __syncthreads();
+  // value v: probe v (accumulator v mod NL of the threads of parity v / NL), then T, then
+  // the clean loss; lane g of the value's 8 sums a fixed stride, then a butterfly
+  const int v = threadIdx.x >> 3, g = threadIdx.x & 7;
+  double bv = 0.0;
+  if (v < NP) {
+    const double *row = red_row(v % NL) + v / NL;
+    for (int m = g; m < 128; m += 8) bv = __dadd_rn(bv, row[2 * m]);
+  } else if (v < NV) {
+    const double *row = red_row(NL + v - NP);
+    for (int c = g; c < 256; c += 8) bv = __dadd_rn(bv, row[c]);
+  }
+  bv = __dadd_rn(bv, __shfl_xor_sync(0xFFFFFFFFu, bv, 4));
+  bv = __dadd_rn(bv, __shfl_xor_sync(0xFFFFFFFFu, bv, 2));
+  bv = __dadd_rn(bv, __shfl_xor_sync(0xFFFFFFFFu, bv, 1));
+
+  // The reduction scratch (partials, counter) is touched only after the previous kernel
+  // in the stream has fully completed.
   tc::pdl_wait();
-  constexpr int NV = NP + (CLEAN ? 2 : 1);
-  double v[NV], tot[NV];
-#pragma unroll
-  for (int t = 0; t < NP; ++t) v[t] = block_sum(lp[t]);
-  v[NP] = block_sum(tsum);
-  if (CLEAN) v[NV - 1] = block_sum(l0);
-  if (last_block_totals<NV>(v, partials, counter, tot)) {
-#pragma unroll
-    for (int t = 0; t < NP; ++t) {
-      if (t < count) {
-        out_plus[t] = tot[t];
-        out_minus[t] = tot[NP] - tot[t];
-      }
-    }
-    if (CLEAN) *out_clean = tot[NV - 1];
+  if (g == 0 && v < NV) {
+    partials[v * gridDim.x + blockIdx.x] = bv;
+    __threadfence();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) last = (atomicAdd(counter, 1u) == gridDim.x - 1);
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  double tot = 0.0;
+  if (v < NV)
+    for (unsigned int b = g; b < gridDim.x; b += 8) tot = __dadd_rn(tot, __ldcg(partials + v * gridDim.x + b));
+  tot = __dadd_rn(tot, __shfl_xor_sync(0xFFFFFFFFu, tot, 4));
+  tot = __dadd_rn(tot, __shfl_xor_sync(0xFFFFFFFFu, tot, 2));
+  tot = __dadd_rn(tot, __shfl_xor_sync(0xFFFFFFFFu, tot, 1));
+  if (g == 0 && v < NV) totals[v] = tot;
+  __syncthreads();
+  const int p = threadIdx.x;
+  if (p < NP && p < count) {
+    out_plus[p] = totals[p];
+    out_minus[p] = totals[NP] - totals[p];
+  }
+  if (p == 0) {
+    if (CLEAN) *out_clean = totals[NP + 1];
+    *counter = 0u;
   }
 }
 
@@ -567,17 +717,17 @@ zo_status launch_quad_loss_pair(zo_ctx *ctx, const ProbeKey &pk, const float *D,
   return launch_quad<true, 0>(ctx, pk, D, out_plus, out_minus, 0, ctx->partials, ctx->counter);
 }
 
-template <bool CLEAN, int NO>
+template <bool CLEAN, int NOCT>
 zo_status launch_quad_octet_t(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, int count,
                               const float *D, double *out_plus, double *out_minus, double *out_clean) {
-  const int64_t n_chunks = (ctx->M + kQChunk - 1) / kQChunk;
+  const int64_t n_chunks = (ctx->M + kOChunk - 1) / kOChunk;
   const int64_t cap = (int64_t)kSmCount * kOBlocksPerSm;
   const int64_t blocks = n_chunks < cap ? n_chunks : cap;
-  static_assert((8 * NO + 2) * kSmCount * kOBlocksPerSm <= kMaxPartials,
+  static_assert((8 * NOCT + 2) * kSmCount * kOBlocksPerSm <= kMaxPartials,
                 "partials too small for the octet pass");
   static bool attr = false;
   if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(quad_octet_kernel<CLEAN, NO>,
+    const cudaError_t e = cudaFuncSetAttribute(quad_octet_kernel<CLEAN, NOCT>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kOSmemBytes);
     if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "quad_octet_kernel attribute: %s", cudaGetErrorString(e));
     attr = true;
@@ -592,7 +742,7 @@ zo_status launch_quad_octet_t(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, i
   attr_pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr_pdl;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, quad_octet_kernel<CLEAN, NO>,
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, quad_octet_kernel<CLEAN, NOCT>,
                                            static_cast<const float *>(ctx->params), D, ctx->M, pk,
                                            octet, count, n_chunks, ctx->partials, ctx->counter,
                                            out_plus, out_minus, out_clean, &ctx->dstate->flags);
@@ -602,11 +752,11 @@ zo_status launch_quad_octet_t(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, i
 
 zo_status launch_quad_octet(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, int count,
                             const float *D, double *out_plus, double *out_minus, double *out_clean) {
-  if (count > 8)
-    return out_clean ? launch_quad_octet_t<true, 2>(ctx, pk, octet, count, D, out_plus, out_minus, out_clean)
-                     : launch_quad_octet_t<false, 2>(ctx, pk, octet, count, D, out_plus, out_minus, nullptr);
-  return out_clean ? launch_quad_octet_t<true, 1>(ctx, pk, octet, count, D, out_plus, out_minus, out_clean)
-                   : launch_quad_octet_t<false, 1>(ctx, pk, octet, count, D, out_plus, out_minus, nullptr);
+  if (count > 16)
+    return out_clean ? launch_quad_octet_t<true, 4>(ctx, pk, octet, count, D, out_plus, out_minus, out_clean)
+                     : launch_quad_octet_t<false, 4>(ctx, pk, octet, count, D, out_plus, out_minus, nullptr);
+  return out_clean ? launch_quad_octet_t<true, 2>(ctx, pk, octet, count, D, out_plus, out_minus, out_clean)
+                   : launch_quad_octet_t<false, 2>(ctx, pk, octet, count, D, out_plus, out_minus, nullptr);
 }
 
 zo_status launch_lowrank_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, const float lam[4],
