@@ -44,13 +44,13 @@ FALLBACK_HBM_GBS = 6650.0
 # summarised in profiles/quad_octet_kernel.quadratic_M2p24.md, valid for the kernel sources
 # whose SHA-256 (of zo_loss.cu and zo_internal.cuh, concatenated) is recorded with it;
 # reported as null when a source has changed since the capture.
-LOSS_TRAFFIC = {"sources_sha256": "2cc2d6dc244cd2ccb386fb3a99781ddac60b79ddda3ae0ed1ee57f7e7c5eebab",
-                "bytes": 138.7e6}
+LOSS_TRAFFIC = {"sources_sha256": "7bb7608b166db3be56fe2cf7593aff6d2a3b6efe28ae4edad4ee009c29282f7b",
+                "bytes": 140.3e6}
 LOSS_SOURCES = ("zo_loss.cu", "zo_internal.cuh")
 # Warp instructions one launch of the loss kernel executes (ncu smsp__inst_executed.sum, same
 # capture and validity rule as LOSS_TRAFFIC): the pass is bound by instruction issue, so its
 # roofline is the issue limit, 148 SMs x 4 warp-instructions per clock at the sampled clock.
-LOSS_WARP_INSTRUCTIONS = 55.36e6
+LOSS_WARP_INSTRUCTIONS = 66.51e6
 SM_COUNT, ISSUE_PER_SM_CLOCK = 148, 4
 
 
@@ -424,7 +424,11 @@ def gpu_arm(args):
             cpu = {"value": (M_sample / M_FULL) / per, "unit": "steps/s", "cores": 1,
                    "kind": "oracle",
                    "sample": "2 oracle steps on the first 2^20 of 2^24 parameters; steps/s scaled by 1/16"}
-        launches_per_step = 1 + len(range(rank, n_oct, world)) + 2
+        if world == 1:  # the loss passes (clean loss fused into the first), precond, update
+            launches_per_step = n_oct + 2
+        else:  # the clean loss, this rank's probe blocks, precond, update
+            from zero_order_forward_b200 import dist as zdist
+            launches_per_step = 1 + len(list(zdist.rank_units(n, rank, world, block))) + 2
         line = {
             "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
