@@ -123,6 +123,41 @@ def time_oracle(M_sample, n_steps, seed=0):
     return times
 
 
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_workers(jobs, threads=1, timeout=900):
+    """Runs `python -m oracle.timing <job...>` once per job, all concurrently, each limited to
+    `threads` BLAS/OpenMP threads; returns their JSON results in job order."""
+    env = dict(os.environ, OMP_NUM_THREADS=str(threads), OPENBLAS_NUM_THREADS=str(threads),
+               MKL_NUM_THREADS=str(threads))
+    procs = [subprocess.Popen([sys.executable, "-m", "oracle.timing"] + [str(a) for a in job],
+                              cwd=ROOT, env=env, stdout=subprocess.PIPE, stderr=subprocess.PIPE,
+                              text=True) for job in jobs]
+    out = []
+    for p in procs:
+        o, e = p.communicate(timeout=timeout)
+        if p.returncode:
+            raise RuntimeError("oracle worker failed: " + e[-400:])
+        out.append(json.loads(o.strip().splitlines()[-1]))
+    return out
+
+
+def oracle_all_cores(M_sample, warmup, steps, max_procs=32):
+    """Oracle steps on every host core: one single-threaded process per core (at most
+    max_procs), each on its own M_sample-element sample of the workload.  Returns
+    (steps/s of the full workload, processes): total work / the union of the timed phases."""
+    P = max(1, min(host_cores(), max_procs))
+    res = oracle_workers([("steps", M_sample, 100 + i, N_PERT, EPS, LR, DAMPING, warmup, steps)
+                          for i in range(P)])
+    wall = max(r["t_end"] for r in res) - min(r["t_start"] for r in res)
+    return P * steps * (M_sample / M_FULL) / wall, P
+
+
 def reference_arm(args):
     rank, _, world = dist_env()
     if rank != 0:
@@ -134,20 +169,19 @@ def reference_arm(args):
     M_sample = 1 << 18
     while M_sample > (1 << 10) and per_elem * M_sample * (args.warmup + args.steps) > 30.0:
         M_sample >>= 1
-    times = time_oracle(M_sample, args.warmup + args.steps)[args.warmup:]
-    per_step = sum(times) / len(times)
-    scale = M_sample / M_FULL
-    value = scale / per_step  # full-workload steps/s extrapolated linearly in M
+    # every host core runs the oracle as it stands (single-threaded) on its own sample
+    value, P = oracle_all_cores(M_sample, args.warmup, args.steps)
     lg = M_sample.bit_length() - 1
-    sample = (f"oracle step on the first 2^{lg} of 2^24 parameters (1/{M_FULL // M_sample} of the "
-              f"workload), {args.steps} timed steps after {args.warmup} warm-up; steps/s scaled "
-              f"by 1/{M_FULL // M_sample}")
+    sample = (f"{P} concurrent single-threaded oracle processes, each {args.steps} timed steps "
+              f"after {args.warmup} warm-up on its own 2^{lg}-element sample of the workload "
+              f"(1/{M_FULL // M_sample} of 2^24 parameters); full-workload steps/s = total "
+              f"sample steps / wall time, scaled by 1/{M_FULL // M_sample}")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 / value, "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "M": M_FULL, "n_pert": N_PERT},
-            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": P, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -424,6 +458,18 @@ def gpu_arm(args):
             cpu = {"value": (M_sample / M_FULL) / per, "unit": "steps/s", "cores": 1,
                    "kind": "oracle",
                    "sample": "2 oracle steps on the first 2^20 of 2^24 parameters; steps/s scaled by 1/16"}
+            import oracle.timing
+            ac, P = oracle_all_cores(M_sample, 0, 1)
+            cpu["all_cores"] = {
+                "value": ac, "unit": "steps/s", "cores": P,
+                "sample": f"{P} concurrent single-threaded oracle processes, one step each on its "
+                          "own 2^20-element sample; steps/s scaled by 1/16"}
+            rates = oracle.timing.element_rates(1 << 22, 1 << 20, (16, 32, 64, 160))
+            cpu["element_rates"] = {
+                "unit": "elements/s", "cores": 1, "perturb": rates["perturb"],
+                "update": rates["update"],
+                "sample": "oracle perturbation of 2^22 elements (one probe); oracle fp32-order "
+                          "update of 2^20 elements with n probes regenerated"}
         if world == 1:  # the loss passes (clean loss fused into the first), precond, update
             launches_per_step = n_oct + 2
         else:  # the clean loss, this rank's probe blocks, precond, update
@@ -633,6 +679,22 @@ def decoder_arm(args):
     fwds = (2 * n + 1) * k
     tokens_per_step = fwds * T
     value = args.steps / total_s
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        # the oracle's forward of one layer at the real width (vocabulary cut to 4096: it only
+        # feeds the gather and the 2-row head), one thread; the step extrapolated from it
+        red = dict(cfg, n_layers=1, vocab=4096)
+        seq = 64
+        tps = oracle_workers([("forward", "qwen3" if qwen else "opt", json.dumps(red), seq)])[0][
+            "tokens_per_s"]
+        cpu_step_s = fwds * B * S * cfg["n_layers"] / tps
+        cpu = {"value": 1.0 / cpu_step_s, "unit": "steps/s", "cores": 1, "kind": "oracle",
+               "extrapolated": True,
+               "sample": f"oracle fp64 forward of 1 layer at the real width, 1 x {seq} tokens "
+                         f"(vocabulary cut to 4096): {tps:.1f} tokens/s; the step extrapolated "
+                         f"linearly in layers and tokens ({fwds} forwards of {B * S} tokens x "
+                         f"{cfg['n_layers']} layers), attention's quadratic term at the full "
+                         f"length not included"}
     line = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps,
@@ -657,6 +719,7 @@ def decoder_arm(args):
                                       "frac_hbm": upd_bytes / (upd_ms * 1e-3) / 1e9 / peaks()[0]}},
         "memory": {"peak_allocated_GB": peak_mem / 1e9, "device_used_GB": (tot_b - free_b) / 1e9},
         "clocks": clocks,
+        "cpu_baseline": cpu,
     }
     model.close()
     ctx.close()

@@ -1,0 +1,93 @@
+"""Timing of the oracle as it stands, for the benchmark's CPU baseline.
+
+TEST INFRASTRUCTURE, like the rest of this package: only the benchmark's CPU-baseline and
+reference legs run it.  Nothing here changes what the oracle computes; it times the
+unmodified functions on samples of the benchmark's workloads, either in the calling process
+or as a command-line worker that the benchmark starts once per host core (independent
+processes on disjoint samples, each single-threaded).
+
+  python -m oracle.timing steps M_SAMPLE SEED N_PERT EPS LR DAMPING WARMUP STEPS
+  python -m oracle.timing forward FAMILY CFG_JSON SEQ
+
+print one JSON object on stdout.
+"""
+import json
+import sys
+import time
+
+import numpy as np
+
+
+def quad_steps(M_sample, seed, n_pert, eps, lr, damping, warmup, steps):
+    """warmup + steps full 1.5-SPSA steps of the oracle on a diagonal quadratic of M_sample
+    elements (the benchmark workload's distribution, sample `seed`).  Returns the seconds of
+    each timed step and the wall-clock bounds of the timed phase."""
+    import synth
+
+    from . import core, step
+    th, D = synth.quad_problem(M_sample, seed=seed)
+
+    def loss(P):
+        return core.quad_loss(P, D)
+
+    times, t_start = [], None
+    for s in range(warmup + steps):
+        if s == warmup:
+            t_start = time.time()
+        t0 = time.perf_counter()
+        th, _ = step.spsa_step(th, loss, n_pert, eps, lr, damping, seed, s, update="mirror")
+        if s >= warmup:
+            times.append(time.perf_counter() - t0)
+    return {"times": times, "t_start": t_start, "t_end": time.time()}
+
+
+def element_rates(M_perturb, M_update, ns):
+    """Elements per second of the oracle's perturbation (one probe, one sign) and of its
+    fp32-order update with n regenerated probes, for each n in ns (one thread)."""
+    import synth
+
+    from . import core
+    th, _ = synth.quad_problem(max(M_perturb, M_update), seed=1)
+    t0 = time.perf_counter()
+    core.perturb(th[:M_perturb], 0, 0, 3, +1, 1e-3)
+    out = {"perturb": M_perturb / (time.perf_counter() - t0), "update": {}}
+    for n in ns:
+        a = synth.coefficients(n)
+        t0 = time.perf_counter()
+        core.update_mirror(th[:M_update], a, 0, 0)
+        out["update"][str(n)] = M_update / (time.perf_counter() - t0)
+    return out
+
+
+def forward_tokens_per_s(family, cfg, seq, batch=1):
+    """Tokens per second of the oracle's decoder loss (fp64) at the given configuration."""
+    import synth
+
+    from . import opt, qwen
+    if family == "qwen3":
+        mod, bits = qwen, synth.qwen_params(cfg)
+    else:
+        mod, bits = opt, synth.opt_params(cfg)
+    theta = (bits.astype(np.uint32) << 16).view(np.float32)
+    tokens, labels = synth.opt_batch(cfg, batch, seq)
+    t0 = time.perf_counter()
+    mod.loss(theta, cfg, tokens, labels)
+    return batch * seq / (time.perf_counter() - t0)
+
+
+def _main(argv):
+    if argv[0] == "steps":
+        M, seed, n, eps, lr, lam, w, k = argv[1:9]
+        res = quad_steps(int(M), int(seed), int(n), float(eps), float(lr), float(lam), int(w), int(k))
+    elif argv[0] == "forward":
+        cfg = json.loads(argv[2])
+        if "class_ids" in cfg:
+            cfg["class_ids"] = tuple(cfg["class_ids"])
+        res = {"tokens_per_s": forward_tokens_per_s(argv[1], cfg, int(argv[3]))}
+    else:
+        raise SystemExit("usage: python -m oracle.timing steps|forward ...")
+    print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    _main(sys.argv[1:])
