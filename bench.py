@@ -4,7 +4,7 @@
 Workload (the default, one GPU): L = 1/2 sum_j D_j theta_j^2 with M = 2^24 fp32
 parameters, D_j log-uniform in [1e-3, 1e3], theta_0 ~ N(0, 1); n_pert = 64,
 eps = 1e-3, lr = 4e-7, damping = 1e-3, 1.5-SPSA.  One step = clean loss + 2*n_pert
-perturbed losses (the 64 losses of each four probe octets from one pass over theta and D) +
+perturbed losses (the 128 losses of each eight probe octets from one pass over theta and D) +
 preconditioner + update, all through the C ABI of libzo.so.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -44,13 +44,13 @@ FALLBACK_HBM_GBS = 6650.0
 # summarised in profiles/quad_octet_kernel.quadratic_M2p24.md, valid for the kernel sources
 # whose SHA-256 (of zo_loss.cu and zo_internal.cuh, concatenated) is recorded with it;
 # reported as null when a source has changed since the capture.
-LOSS_TRAFFIC = {"sources_sha256": "7bb7608b166db3be56fe2cf7593aff6d2a3b6efe28ae4edad4ee009c29282f7b",
-                "bytes": 140.3e6}
+LOSS_TRAFFIC = {"sources_sha256": "a42efd669357179163a5bb580b45090ffdc061d144209f6959c2a5195b3a96f3",
+                "bytes": 139.75e6}
 LOSS_SOURCES = ("zo_loss.cu", "zo_internal.cuh")
 # Warp instructions one launch of the loss kernel executes (ncu smsp__inst_executed.sum, same
 # capture and validity rule as LOSS_TRAFFIC): the pass is bound by instruction issue, so its
 # roofline is the issue limit, 148 SMs x 4 warp-instructions per clock at the sampled clock.
-LOSS_WARP_INSTRUCTIONS = 66.51e6
+LOSS_WARP_INSTRUCTIONS = 99.93e6
 SM_COUNT, ISSUE_PER_SM_CLOCK = 148, 4
 
 
@@ -289,8 +289,8 @@ def gpu_arm(args):
     def apply_step(Lp, Lm, L0):
         zo.zo_step(ctx, Lp, Lm, n, L0, LR, EPS, DAMPING)
 
-    # probes per rank and pass: up to four octets, fewer when the ranks would otherwise idle
-    block = min(32, max(8, -(-(n // world) // 8) * 8))
+    # probes per rank and pass: up to eight octets, fewer when the ranks would otherwise idle
+    block = min(64, max(8, -(-(n // world) // 8) * 8))
 
     def octet_at(first, count, out_plus, out_minus):
         zo.zo_quad_loss_octet(ctx, D, first, count, EPS, out_plus, out_minus)
@@ -338,17 +338,17 @@ def gpu_arm(args):
     value = args.steps / total_s  # steps of the one shared model
 
     # dominant kernel: the loss pass (perturbation on load).  At one GPU the probe phase
-    # holds n/32 launches of the octet kernel (the 64 losses L(theta +- eps z_i) of four probe
-    # octets from one pass over theta and D); with N ranks the phase is not bracketed
+    # holds n/64 launches of the octet kernel (the 128 losses L(theta +- eps z_i) of eight
+    # probe octets from one pass over theta and D); with N ranks the phase is not bracketed
     # separately: time the kernel alone.
-    n_oct = (n + 31) // 32
+    n_oct = (n + 63) // 64
     if world > 1:
         le = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         flush.zero_()
         le[0].record(stream)
         for o in range(n_oct):
-            zo.zo_quad_loss_octet(ctx, D, 32 * o, min(32, n - 32 * o), EPS, losses[1:33],
-                                  losses[33:65], losses[0:1] if o == 0 else None)
+            zo.zo_quad_loss_octet(ctx, D, 64 * o, min(64, n - 64 * o), EPS, losses[1:65],
+                                  losses[65:129], losses[0:1] if o == 0 else None)
         le[1].record(stream)
         torch.cuda.synchronize()
         probe_ms = [le[0].elapsed_time(le[1])]
@@ -483,8 +483,8 @@ def gpu_arm(args):
             "config": {"workload": WORKLOAD, "M": M_FULL, "n_pert": n, "eps": EPS, "lr": LR,
                        "damping": DAMPING, "parallelism": f"probe-parallel x{world}",
                        "l2": "flushed between steps (256 MiB write, untimed); theta+D = 128 MiB"},
-            "roofline": {"kernel": "quad_octet_kernel (the 64 losses L(theta +- eps z_i) of four "
-                                   "probe octets in one pass, perturbation on load, fp64 "
+            "roofline": {"kernel": "quad_octet_kernel (the 128 losses L(theta +- eps z_i) of "
+                                   "eight probe octets in one pass, perturbation on load, fp64 "
                                    "accumulation)",
                          "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "peak_kind": peak_kind,

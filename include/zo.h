@@ -202,7 +202,7 @@ zo_status zo_quad_loss_pair(zo_ctx *ctx, const float *D, int32_t probe, float ep
                             double *loss_plus, double *loss_minus);
 
 /* The 2*count losses of the probes first_probe .. first_probe+count-1 (first_probe a
- * multiple of 8, count 1..32: the probes of up to four octets; an octet's signs share one
+ * multiple of 8, count 1..64: the probes of up to eight octets; an octet's signs share one
  * generator block) from ONE pass over theta and D: L(theta + eps z_i) -> loss_plus[i - first_probe],
  * L(theta - eps z_i) -> loss_minus[i - first_probe] (device doubles).  Each element has
  * two perturbed values, rd(theta_j + eps) and rd(theta_j - eps), and each loss takes one of
@@ -291,7 +291,7 @@ zo_status zo_get_precond(zo_ctx *ctx, int32_t n, double *g, double *c, double *w
 
 /* ------------------------------------------------------------------ step driver */
 
-/* One full step on the diagonal quadratic [LOOP]: the losses at +eps and -eps of up to 32
+/* One full step on the diagonal quadratic [LOOP]: the losses at +eps and -eps of up to 64
  * probes per pass over theta and D (perturbation on load: zo_quad_loss_octet), the clean
  * loss (1.5-SPSA) fused into the first pass, then zo_step.
  *   D           device, M floats;  losses_out device, 2*n_pert+1 doubles receiving

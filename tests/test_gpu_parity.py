@@ -432,9 +432,9 @@ def test_quad_loss_pair_is_bit_identical_to_two_passes(zo, M):
 
 @pytest.mark.parametrize("M", [1, 7, 4096 * 3 + 5, 1 << 20, (1 << 22) + 17])
 @pytest.mark.parametrize("first,count", [(0, 8), (16, 8), (8, 3), (0, 16), (24, 11), (0, 32),
-                                         (8, 24), (16, 19)])
+                                         (8, 24), (16, 19), (0, 64), (8, 40), (0, 33)])
 def test_quad_loss_octet_matches_pairs_and_oracle(zo, M, first, count):
-    """zo_quad_loss_octet computes the 2*count losses of up to four probe octets in one pass
+    """zo_quad_loss_octet computes the 2*count losses of up to eight probe octets in one pass
     (each element's two perturbed values, each loss taking one per element; L- from the
     common sum of both terms): equal to the per-probe pair passes and to the oracle within
     fp64 rounding of sums of M terms (1e-12 relative), the clean loss from the same pass too.
@@ -443,8 +443,8 @@ def test_quad_loss_octet_matches_pairs_and_oracle(zo, M, first, count):
     th, D = dev(th_np), dev(D_np)
     ctx = zo.zo_create(th, seed=6)
     zo.zo_set_step(ctx, 2)
-    oct_p = torch.full((33,), -7.0, dtype=torch.float64, device="cuda")
-    oct_m = torch.full((33,), -7.0, dtype=torch.float64, device="cuda")
+    oct_p = torch.full((65,), -7.0, dtype=torch.float64, device="cuda")
+    oct_m = torch.full((65,), -7.0, dtype=torch.float64, device="cuda")
     clean = torch.zeros(2, dtype=torch.float64, device="cuda")
     zo.zo_quad_loss_octet(ctx, D, first, count, 1e-3, oct_p, oct_m, clean[0:1])
     zo.zo_quad_loss(ctx, D, clean[1:2])
@@ -466,7 +466,7 @@ def test_quad_loss_octet_matches_pairs_and_oracle(zo, M, first, count):
     with pytest.raises(zo.ZoError):
         zo.zo_quad_loss_octet(ctx, D, 3, 8, 1e-3, oct_p, oct_m)  # not an octet boundary
     with pytest.raises(zo.ZoError):
-        zo.zo_quad_loss_octet(ctx, D, 0, 33, 1e-3, oct_p, oct_m)  # more than four octets
+        zo.zo_quad_loss_octet(ctx, D, 0, 65, 1e-3, oct_p, oct_m)  # more than eight octets
     ctx.close()
 
 

@@ -456,8 +456,8 @@ zo_status zo_quad_loss_octet(zo_ctx *ctx, const float *D, int32_t first_probe, i
   if (ctx->dtype != ZO_F32) return fail(ctx, ZO_ERR_UNSUPPORTED, "quadratic loss needs an fp32 context");
   if (!D || !loss_plus || !loss_minus || !aligned16(D))
     return fail(ctx, ZO_ERR_INVALID, "D must be a 16-byte aligned device pointer; outputs non-null");
-  if (first_probe < 0 || first_probe % 8 || count < 1 || count > 32 || !(eps > 0.f) || !std::isfinite(eps))
-    return fail(ctx, ZO_ERR_INVALID, "first_probe must be a multiple of 8, count 1..32, eps > 0");
+  if (first_probe < 0 || first_probe % 8 || count < 1 || count > 64 || !(eps > 0.f) || !std::isfinite(eps))
+    return fail(ctx, ZO_ERR_INVALID, "first_probe must be a multiple of 8, count 1..64, eps > 0");
   if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "octet evaluation needs the clean state");
   ProbeKey pk = probe_key(ctx);
   pk.sign = +1;
@@ -477,9 +477,9 @@ zo_status zo_quad_step(zo_ctx *ctx, const float *D, int32_t n_pert, float eps, f
   if (!preconditioned)
     ZO_CUDA(ctx, cudaMemsetAsync(L0, 0, sizeof(double), ctx->stream), "clear L0");
   phase_mark(ctx, 1);
-  // the 64 losses of four probe octets from one pass; the first pass also adds the clean loss
-  for (int32_t i = 0; i < n_pert; i += 32)
-    ZO_CHECK(zo_quad_loss_octet(ctx, D, i, n_pert - i < 32 ? n_pert - i : 32, eps, Lp + i, Lm + i,
+  // the 128 losses of eight probe octets from one pass; the first pass also adds the clean loss
+  for (int32_t i = 0; i < n_pert; i += 64)
+    ZO_CHECK(zo_quad_loss_octet(ctx, D, i, n_pert - i < 64 ? n_pert - i : 64, eps, Lp + i, Lm + i,
                                 (preconditioned && i == 0) ? L0 : nullptr));
   phase_mark(ctx, 2);
   const zo_status st = zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);

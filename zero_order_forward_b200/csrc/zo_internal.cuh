@@ -143,7 +143,7 @@ struct zo_ctx {
 
 namespace zo {
 
-constexpr int kMaxPartials = 16384;
+constexpr int kMaxPartials = 32768;
 
 zo_status fail(zo_ctx *ctx, zo_status st, const char *fmt, ...);
 zo_status check_launch(zo_ctx *ctx, const char *what);

@@ -405,8 +405,8 @@ __device__ __forceinline__ uint32_t nibble_offset(uint32_t x, int t) {
   return (s >= 0 ? x >> s : x << -s) & 0x7800u;
 }
 
-// The losses L(theta +- eps z_i) of the 8 NOCT probes i = 8 octet + p, p < 8 NOCT (NOCT = 2
-// or 4 consecutive octets: 32 or 64 losses), from one pass over theta and D.
+// The losses L(theta +- eps z_i) of the 8 NOCT probes i = 8 octet + p, p < 8 NOCT (NOCT = 2,
+// 4 or 8 consecutive octets: 32, 64 or 128 losses), from one pass over theta and D.
 //
 // Each element has only two perturbed values, P_a = rd(theta + eps) and P_b = rd(theta - eps),
 // with terms t_a = (D/2) P_a^2 and t_b = (D/2) P_b^2 (fp64); the sign bit of probe i says
@@ -415,28 +415,32 @@ __device__ __forceinline__ uint32_t nibble_offset(uint32_t x, int t) {
 //
 // A consumer thread holds 4 consecutive elements per vector; the 4 sign bits of one probe
 // for them form a nibble, and the 16 possible sums (x_0 + x_1) + (x_2 + x_3), x_q in
-// {t_a, t_b}, go into the thread's table in shared memory once per vector.  Two neighbouring
-// lanes (a pair: adjacent vectors of one 16-element group) read each other's table: the even
-// lane accumulates the first NOCT/2 octets and the odd lane the others, for both vectors,
-// so a thread keeps 4 NOCT accumulators while each vector's terms and table serve all
-// 8 NOCT probes.  A probe then costs, per vector, a shift and a mask of the transposed
-// sign word, one table load and one fp64 add.  Summation order per loss: the vectors of a
-// thread in chunk order, each pair step adding the thread's own vector and then its
-// partner's; block and grid totals in a fixed order (8 lanes per value over a fixed
-// stride, then a butterfly).  Probes p >= count are computed and not stored.  CLEAN also
-// adds the clean loss L(theta) to the same pass (into *out_clean).
+// {t_a, t_b}, go into the thread's table in shared memory once per vector.  G neighbouring
+// lanes (a pair for NOCT 2 and 4, a quad for NOCT 8; a quad's vectors are one 16-element
+// group) read each other's tables, and each of them accumulates NOCT/G of the octets for
+// all G vectors, so a thread keeps at most 16 accumulators while each vector's terms and
+// table serve all 8 NOCT probes.  A pair gets its sign words from the quad's four Philox
+// blocks through shuffles; a quad lane generates the blocks of its own two octets, whose
+// four words are the quad's four vectors.  A probe then costs, per vector, a shift and a
+// mask of the transposed sign word, one table load and one fp64 add.  Summation order per
+// loss: the vector steps of a thread in chunk order, each adding the G vectors in a fixed
+// lane-dependent order; block and grid totals in a fixed order (LPV lanes per value over a
+// fixed stride, then a butterfly).  Probes p >= count are computed and not stored.  CLEAN
+// also adds the clean loss L(theta) to the same pass (into *out_clean).
 template <bool CLEAN, int NOCT>
 __global__ void __launch_bounds__(kQThreads, kOBlocksPerSm)
 quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, int64_t M,
                   ProbeKey pk, uint32_t octet, int count, int64_t n_chunks, double *partials,
                   unsigned int *counter, double *out_plus, double *out_minus, double *out_clean,
                   uint32_t *err) {
-  static_assert(NOCT == 2 || NOCT == 4, "two or four octets per pass");
-  constexpr int LO = NOCT / 2;       // octets per thread
-  constexpr int NL = 8 * LO;         // accumulators per thread
-  constexpr int NP = 8 * NOCT;       // probes per pass
-  constexpr int NV = NP + 2;         // block values: probes, T, clean loss
-  static_assert(8 * NV <= kQThreads, "eight lanes per value in the epilogue");
+  static_assert(NOCT == 2 || NOCT == 4 || NOCT == 8, "two, four or eight octets per pass");
+  constexpr int G = NOCT == 8 ? 4 : 2;     // lanes sharing their tables (a pair or a quad)
+  constexpr int LO = NOCT / G;             // octets per thread
+  constexpr int NL = 8 * LO;               // accumulators per thread
+  constexpr int NP = 8 * NOCT;             // probes per pass
+  constexpr int NV = NP + 2;               // block values: probes, T, clean loss
+  constexpr int LPV = NOCT == 8 ? 4 : 8;   // lanes per value in the epilogue
+  static_assert(LPV * NV <= kQThreads, "lanes per value in the epilogue");
   static_assert(kOStages * kOStageBytes == 16 * 2048 && kOTableBytes == 16 * 2048 && NL + 2 <= 32,
                 "epilogue rows: 16 in the stage buffers, the rest in the tables");
   extern __shared__ __align__(128) uint8_t qsm[];
@@ -457,6 +461,10 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
     const int cw = ct >> 5;
     const int q = lane & 3, quad = lane >> 2, h = lane & 1;
     const uint32_t own8 = (uint32_t)ct * 8u, par8 = (uint32_t)(ct ^ 1) * 8u;
+    // NOCT 8: round r reads the table of quad lane q ^ r (distinct per lane in every round)
+    uint32_t col8[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) col8[r] = (uint32_t)(ct ^ r) * 8u;
     uint8_t *const tab = qsm + kOTableOff;  // entry n of thread c at byte 2048 n + 8 c
     int it = 0;
     for (int64_t chunk = blockIdx.x; chunk < n_chunks; chunk += gridDim.x, ++it) {
@@ -497,9 +505,10 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
         const int e = 4 * (ct + k * 32 * kQConsumers);
         float tv[4], dv[4];
         quad_load4<kOChunk>(st, theta, D, base, e, cnt, tv, dv);
-        // wo / wp: the own / partner vector's word of each local octet j
+        // wo / wp: the own / partner vector's word of each local octet j (pairs)
         uint32_t wo[LO], wp[LO];
-        if constexpr (NOCT == 4) {
+        if constexpr (NOCT == 8) {
+        } else if constexpr (NOCT == 4) {
           // lane q generates octet q; lane l reads octet sw(l) in rounds 0, 1 and octet
           // sw(l) ^ 1 in rounds 2, 3 (sw swaps the two bits of q), even word then odd
           const int sw = ((q & 1) << 1) | (q >> 1);
@@ -541,15 +550,44 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
 #pragma unroll
         for (int n = 0; n < 16; ++n)
           *reinterpret_cast<double *>(tab + 2048 * n + own8) = __dadd_rn(lo[n & 3], hi[n >> 2]);
-        __syncwarp();  // both tables of the pair are written
+        __syncwarp();  // the tables of the pair (quad) are written
+        if constexpr (NOCT == 8) {
+          // the quad holds the whole 16-element group: lane q generates the blocks of its
+          // octets 2q, 2q + 1 itself; word m of a block is the vector of quad lane m
 #pragma unroll
-        for (int j = 0; j < LO; ++j) {
-          const uint32_t xo = probe_nibbles(wo[j]), xp = probe_nibbles(wp[j]);
+          for (int j = 0; j < LO; ++j) {
+            const uint4 blk = sign_block(g0 + 64 * k, octet + (uint32_t)(LO * q + j), step, pk.k0, pk.k1);
+            uint32_t w[4] = {blk.x, blk.y, blk.z, blk.w};
+            if (q & 1) {  // w[r] <- word q ^ r
+              const uint32_t a = w[0], b = w[2];
+              w[0] = w[1]; w[1] = a; w[2] = w[3]; w[3] = b;
+            }
+            if (q & 2) {
+              const uint32_t a = w[0], b = w[1];
+              w[0] = w[2]; w[1] = w[3]; w[2] = a; w[3] = b;
+            }
+            uint32_t x[4];
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const double vo = *reinterpret_cast<const double *>(tab + (nibble_offset(xo, t) | own8));
-            const double vq = *reinterpret_cast<const double *>(tab + (nibble_offset(xp, t) | par8));
-            lp[8 * j + t] = __dadd_rn(__dadd_rn(lp[8 * j + t], vo), vq);
+            for (int r = 0; r < 4; ++r) x[r] = probe_nibbles(w[r]);
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+              double acc = lp[8 * j + t];
+#pragma unroll
+              for (int r = 0; r < 4; ++r)
+                acc = __dadd_rn(acc, *reinterpret_cast<const double *>(tab + (nibble_offset(x[r], t) | col8[r])));
+              lp[8 * j + t] = acc;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < LO; ++j) {
+            const uint32_t xo = probe_nibbles(wo[j]), xp = probe_nibbles(wp[j]);
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+              const double vo = *reinterpret_cast<const double *>(tab + (nibble_offset(xo, t) | own8));
+              const double vq = *reinterpret_cast<const double *>(tab + (nibble_offset(xp, t) | par8));
+              lp[8 * j + t] = __dadd_rn(__dadd_rn(lp[8 * j + t], vo), vq);
+            }
           }
         }
       }
@@ -574,20 +612,19 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
     red_row(NL + 1)[ct] = l0;
   }
   __syncthreads();
-  // value v: probe v (accumulator v mod NL of the threads of parity v / NL), then T, then
-  // the clean loss; lane g of the value's 8 sums a fixed stride, then a butterfly
-  const int v = threadIdx.x >> 3, g = threadIdx.x & 7;
+  // value v: probe v (accumulator v mod NL of the threads ct with ct mod G = v / NL), then
+  // T, then the clean loss; lane g of the value's LPV sums a fixed stride, then a butterfly
+  const int v = threadIdx.x / LPV, g = threadIdx.x % LPV;
   double bv = 0.0;
   if (v < NP) {
     const double *row = red_row(v % NL) + v / NL;
-    for (int m = g; m < 128; m += 8) bv = __dadd_rn(bv, row[2 * m]);
+    for (int m = g; m < 256 / G; m += LPV) bv = __dadd_rn(bv, row[G * m]);
   } else if (v < NV) {
     const double *row = red_row(NL + v - NP);
-    for (int c = g; c < 256; c += 8) bv = __dadd_rn(bv, row[c]);
+    for (int c = g; c < 256; c += LPV) bv = __dadd_rn(bv, row[c]);
   }
-  bv = __dadd_rn(bv, __shfl_xor_sync(0xFFFFFFFFu, bv, 4));
-  bv = __dadd_rn(bv, __shfl_xor_sync(0xFFFFFFFFu, bv, 2));
-  bv = __dadd_rn(bv, __shfl_xor_sync(0xFFFFFFFFu, bv, 1));
+#pragma unroll
+  for (int o = LPV / 2; o > 0; o >>= 1) bv = __dadd_rn(bv, __shfl_xor_sync(0xFFFFFFFFu, bv, o));
 
   // The reduction scratch (partials, counter) is touched only after the previous kernel
   // in the stream has fully completed.
@@ -603,10 +640,9 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
   __threadfence();
   double tot = 0.0;
   if (v < NV)
-    for (unsigned int b = g; b < gridDim.x; b += 8) tot = __dadd_rn(tot, __ldcg(partials + v * gridDim.x + b));
-  tot = __dadd_rn(tot, __shfl_xor_sync(0xFFFFFFFFu, tot, 4));
-  tot = __dadd_rn(tot, __shfl_xor_sync(0xFFFFFFFFu, tot, 2));
-  tot = __dadd_rn(tot, __shfl_xor_sync(0xFFFFFFFFu, tot, 1));
+    for (unsigned int b = g; b < gridDim.x; b += LPV) tot = __dadd_rn(tot, __ldcg(partials + v * gridDim.x + b));
+#pragma unroll
+  for (int o = LPV / 2; o > 0; o >>= 1) tot = __dadd_rn(tot, __shfl_xor_sync(0xFFFFFFFFu, tot, o));
   if (g == 0 && v < NV) totals[v] = tot;
   __syncthreads();
   const int p = threadIdx.x;
@@ -752,6 +788,9 @@ zo_status launch_quad_octet_t(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, i
 
 zo_status launch_quad_octet(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, int count,
                             const float *D, double *out_plus, double *out_minus, double *out_clean) {
+  if (count > 32)
+    return out_clean ? launch_quad_octet_t<true, 8>(ctx, pk, octet, count, D, out_plus, out_minus, out_clean)
+                     : launch_quad_octet_t<false, 8>(ctx, pk, octet, count, D, out_plus, out_minus, nullptr);
   if (count > 16)
     return out_clean ? launch_quad_octet_t<true, 4>(ctx, pk, octet, count, D, out_plus, out_minus, out_clean)
                      : launch_quad_octet_t<false, 4>(ctx, pk, octet, count, D, out_plus, out_minus, nullptr);
