@@ -13,6 +13,7 @@
 // once per step.  Its fp32 summation order is fixed (octets of 8 probes through a
 // 256-entry table of signed partial sums per octet, octet sums added in order).
 #include "zo_internal.cuh"
+#include "zo_tc.cuh"
 
 namespace zo {
 namespace {
@@ -43,6 +44,11 @@ precond_kernel(const double *__restrict__ lp, const double *__restrict__ lm,
                double alpha, float *__restrict__ coef, double *__restrict__ diag,
                DevState *st) {
   __shared__ double red[6][kPrecondThreads / 32];
+  // Launched with programmatic dependent launch: the update may be scheduled now (it waits
+  // for this grid before it reads anything); the losses are read only once the loss passes
+  // before this kernel have completed.
+  tc::pdl_launch_dependents();
+  tc::pdl_wait();
   bool bad = false;
   for (int i = threadIdx.x; i < n; i += blockDim.x)
     bad |= !isfinite(lp[i]) || !isfinite(lm[i]);
@@ -155,6 +161,10 @@ update_kernel(T *__restrict__ theta, int64_t M, const float *__restrict__ coef, 
               const uint32_t *step_ptr, const uint32_t *ok_ptr, uint32_t k0, uint32_t k1) {
   constexpr int R = 1 << LOG_R;
   extern __shared__ float lut[];  // [octet][256 entries][R replicas]
+  // Launched with programmatic dependent launch: wait for the preconditioner (coefficients,
+  // step, ok flag).  This kernel never signals early, so the next kernel of the stream, which
+  // reads theta, starts only after it has completed.
+  tc::pdl_wait();
   if (ok_ptr != nullptr && *ok_ptr == 0u) return;
   const uint32_t step = *step_ptr;
   const int octets = (n + 7) >> 3;
@@ -236,8 +246,19 @@ zo_status launch_update_t(zo_ctx *ctx, const float *coef, int n, const uint32_t 
   int64_t blocks = (n_groups + kUpdThreads - 1) / kUpdThreads;
   const int64_t cap = (int64_t)kSmCount * (per_sm > 0 ? per_sm : 1);
   if (blocks > cap) blocks = cap;
-  kern<<<(unsigned)blocks, kUpdThreads, smem, ctx->stream>>>(static_cast<T *>(ctx->params), ctx->M,
-                                                             coef, n, step_ptr, ok_ptr, k0, k1);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(kUpdThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = ctx->stream;
+  cudaLaunchAttribute attr_pdl[1];
+  attr_pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr_pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr_pdl;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, static_cast<T *>(ctx->params), ctx->M, coef, n, step_ptr,
+                         ok_ptr, k0, k1);
+  if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "update_kernel: %s", cudaGetErrorString(e));
   return check_launch(ctx, "update_kernel");
 }
 
@@ -258,9 +279,19 @@ zo_status launch_update_r(zo_ctx *ctx, const float *coef, int n, const uint32_t 
 
 zo_status launch_precond(zo_ctx *ctx, const double *lp, const double *lm, const double *l0,
                          int n, float lr, float eps, float damping) {
-  precond_kernel<<<1, kPrecondThreads, 0, ctx->stream>>>(
-      lp, lm, l0, n, (double)lr, (double)eps, (double)damping, (double)ctx->alpha, ctx->coef,
-      ctx->diag, ctx->dstate);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(kPrecondThreads);
+  cfg.stream = ctx->stream;
+  cudaLaunchAttribute attr_pdl[1];
+  attr_pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr_pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr_pdl;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, precond_kernel, lp, lm, l0, n, (double)lr, (double)eps,
+                                           (double)damping, (double)ctx->alpha, ctx->coef, ctx->diag,
+                                           ctx->dstate);
+  if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "precond_kernel: %s", cudaGetErrorString(e));
   ctx->last_n = n;
   return check_launch(ctx, "precond_kernel");
 }
