@@ -422,7 +422,8 @@ __device__ __forceinline__ uint32_t nibble_offset(uint32_t x, int t) {
 // table serve all 8 NOCT probes.  A pair gets its sign words from the quad's four Philox
 // blocks through shuffles; a quad lane generates the blocks of its own two octets, whose
 // four words are the quad's four vectors.  A probe then costs, per vector, a shift and a
-// mask of the transposed sign word, one table load and one fp64 add.  Summation order per
+// mask of the transposed sign word (quads: half a multiply that gathers two probes' bits),
+// one table load and one fp64 add.  Summation order per
 // loss: the vector steps of a thread in chunk order, each adding the G vectors in a fixed
 // lane-dependent order; block and grid totals in a fixed order (LPV lanes per value over a
 // fixed stride, then a butterfly).  Probes p >= count are computed and not stored.  CLEAN
@@ -566,16 +567,20 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
               const uint32_t a = w[0], b = w[1];
               w[0] = w[2]; w[1] = w[3]; w[2] = a; w[3] = b;
             }
-            uint32_t x[4];
+            // probes t and t + 4 together: bits t and t + 4 of the word's 4 bytes, masked and
+            // multiplied by 0x01020408, gather at bits 24..27 and 28..31 (the other partial
+            // products fall at distinct positions below bit 24 or beyond bit 31)
 #pragma unroll
-            for (int r = 0; r < 4; ++r) x[r] = probe_nibbles(w[r]);
+            for (int t = 0; t < 4; ++t) {
+              double a0 = lp[8 * j + t], a1 = lp[8 * j + t + 4];
 #pragma unroll
-            for (int t = 0; t < 8; ++t) {
-              double acc = lp[8 * j + t];
-#pragma unroll
-              for (int r = 0; r < 4; ++r)
-                acc = __dadd_rn(acc, *reinterpret_cast<const double *>(tab + (nibble_offset(x[r], t) | col8[r])));
-              lp[8 * j + t] = acc;
+              for (int r = 0; r < 4; ++r) {
+                const uint32_t pr = ((w[r] >> t) & 0x11111111u) * 0x01020408u;
+                a0 = __dadd_rn(a0, *reinterpret_cast<const double *>(tab + (((pr >> 13) & 0x7800u) | col8[r])));
+                a1 = __dadd_rn(a1, *reinterpret_cast<const double *>(tab + (((pr >> 17) & 0x7800u) | col8[r])));
+              }
+              lp[8 * j + t] = a0;
+              lp[8 * j + t + 4] = a1;
             }
           }
         } else {
