@@ -385,26 +385,12 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
   }
 }
 
-// Sign word of 4 elements (byte q = element q, bit t = probe t of an octet) -> 8 nibbles:
-// nibble t (bits 4t..4t+3) holds bit t of bytes 0..3.  Bit 8q + t moves to 4t + q, a
-// rotation of the 5 bit-index bits, done as four swaps of index bits (4,2), (3,1), (2,0),
-// (1,0), each a masked exchange of the bit pairs that differ in them.
-__device__ __forceinline__ uint32_t delta_swap(uint32_t x, uint32_t m, int d) {
-  const uint32_t t = ((x >> d) ^ x) & m;
-  return x ^ t ^ (t << d);
-}
-__device__ __forceinline__ uint32_t probe_nibbles(uint32_t w) {
-  w = delta_swap(w, 0x0000F0F0u, 12);
-  w = delta_swap(w, 0x00CC00CCu, 6);
-  w = delta_swap(w, 0x0A0A0A0Au, 3);
-  return delta_swap(w, 0x22222222u, 1);
-}
-// 2048 * (nibble t of x): the byte offset of that table entry (t a compile-time constant).
-__device__ __forceinline__ uint32_t nibble_offset(uint32_t x, int t) {
-  const int s = 4 * t - 11;
-  return (s >= 0 ? x >> s : x << -s) & 0x7800u;
-}
-
+// Sign word of 4 elements: byte q holds element q's bits, bit t of a byte probe t of an
+// octet.  Masking bits t and t + 4 of every byte ((w >> t) & 0x11111111, t < 4) and
+// multiplying by 0x01020408 = 2^24 + 2^17 + 2^10 + 2^3 moves bit 8q + t to 24 + q and bit
+// 8q + t + 4 to 28 + q: the nibbles of probes t and t + 4, bit q = element q.  Every other
+// partial product lands at a distinct position below bit 24 or beyond bit 31, so nothing
+// carries into them.  The table offsets 2048 * nibble follow with one shift and mask each.
 // The losses L(theta +- eps z_i) of the 8 NOCT probes i = 8 octet + p, p < 8 NOCT (NOCT = 2,
 // 4 or 8 consecutive octets: 32, 64 or 128 losses), from one pass over theta and D.
 //
@@ -421,9 +407,9 @@ __device__ __forceinline__ uint32_t nibble_offset(uint32_t x, int t) {
 // all G vectors, so a thread keeps at most 16 accumulators while each vector's terms and
 // table serve all 8 NOCT probes.  A pair gets its sign words from the quad's four Philox
 // blocks through shuffles; a quad lane generates the blocks of its own two octets, whose
-// four words are the quad's four vectors.  A probe then costs, per vector, a shift and a
-// mask of the transposed sign word (quads: half a multiply that gathers two probes' bits),
-// one table load and one fp64 add.  Summation order per
+// four words are the quad's four vectors.  Per vector, two probes then cost one masked
+// multiply of the sign word (above), and each probe a shift and mask, one table load and
+// one fp64 add.  Summation order per
 // loss: the vector steps of a thread in chunk order, each adding the G vectors in a fixed
 // lane-dependent order; block and grid totals in a fixed order (LPV lanes per value over a
 // fixed stride, then a butterfly).  Probes p >= count are computed and not stored.  CLEAN
@@ -586,12 +572,16 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
         } else {
 #pragma unroll
           for (int j = 0; j < LO; ++j) {
-            const uint32_t xo = probe_nibbles(wo[j]), xp = probe_nibbles(wp[j]);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) {
-              const double vo = *reinterpret_cast<const double *>(tab + (nibble_offset(xo, t) | own8));
-              const double vq = *reinterpret_cast<const double *>(tab + (nibble_offset(xp, t) | par8));
-              lp[8 * j + t] = __dadd_rn(__dadd_rn(lp[8 * j + t], vo), vq);
+            for (int t = 0; t < 4; ++t) {  // probes t and t + 4 through one multiply per word
+              const uint32_t po = ((wo[j] >> t) & 0x11111111u) * 0x01020408u;
+              const uint32_t pp = ((wp[j] >> t) & 0x11111111u) * 0x01020408u;
+              const double vo0 = *reinterpret_cast<const double *>(tab + (((po >> 13) & 0x7800u) | own8));
+              const double vq0 = *reinterpret_cast<const double *>(tab + (((pp >> 13) & 0x7800u) | par8));
+              const double vo1 = *reinterpret_cast<const double *>(tab + (((po >> 17) & 0x7800u) | own8));
+              const double vq1 = *reinterpret_cast<const double *>(tab + (((pp >> 17) & 0x7800u) | par8));
+              lp[8 * j + t] = __dadd_rn(__dadd_rn(lp[8 * j + t], vo0), vq0);
+              lp[8 * j + t + 4] = __dadd_rn(__dadd_rn(lp[8 * j + t + 4], vo1), vq1);
             }
           }
         }
