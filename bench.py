@@ -889,7 +889,15 @@ def mlp_arm(args):
             "config": {"workload": "MLP 64-256-10 fp32 (M=19,210), batch 64, teacher labels, "
                                    "n_pert=16, eps=1e-3, lr=1e-2, damping=1e-3, 1.5-SPSA"},
             "final_loss": float(losses[0].item()),
-            "gpu_launches": (1 + 2 * n * 2 + 2) * args.steps}
+            # all 33 losses from one staged-parameter launch and its batch sums, then the
+            # preconditioner and the update
+            "gpu_launches": 4 * args.steps}
+    if not args.no_cpu_baseline:
+        ts = oracle_workers([("mlp", 4)])[0]["times"]
+        line["cpu_baseline"] = {"value": 1.0 / statistics.mean(ts), "unit": "steps/s", "cores": 1,
+                                "kind": "oracle",
+                                "sample": "4 full oracle steps of this workload after one untimed "
+                                          "step, one thread"}
     ctx.close()
     print(json.dumps(line), flush=True)
     return 0

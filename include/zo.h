@@ -318,8 +318,26 @@ zo_status zo_quad_step_host_async(zo_ctx *ctx, const float *D_host, int32_t n_pe
                                   float lr, float damping, int preconditioned,
                                   double *losses_host);
 
-/* One full MLP step [LOOP] (live buffer enabled by the call if needed): clean loss,
- * 2*n_pert perturbed losses through the live buffer, zo_step.  Arguments as
+/* Every loss of one MLP step from two launches: L(theta + eps z_i) -> loss_plus[i],
+ * L(theta - eps z_i) -> loss_minus[i] for i < n_pert, and the clean loss L(theta) ->
+ * *loss_clean unless it is NULL (device doubles; each = scale * sum of the batch's
+ * per-sample losses).  Each evaluation's block stages rd(theta + s eps z_i) in shared memory
+ * and runs zo_mlp_loss's per-sample arithmetic and batch sum in the same order, so every
+ * value equals the corresponding zo_perturb / zo_mlp_loss / zo_restore result bit for bit.
+ * Requires an fp32 context in the clean state with M = the MLP's parameter count and
+ * M + n_hidden <= 49152 (the staged parameters, W1's rows padded by one); uses the current step counter.  X, labels, batch,
+ * n_in, n_hidden, n_out as zo_mlp_loss; 1 <= n_pert <= ZO_MAX_PROBES, eps > 0.  Scratch of
+ * (2 n_pert + 1) * batch doubles is owned by the context.  Errors: ZO_ERR_INVALID,
+ * ZO_ERR_STATE, ZO_ERR_UNSUPPORTED (bf16 context or M above the limit), ZO_ERR_OOM,
+ * ZO_ERR_CUDA. */
+zo_status zo_mlp_losses(zo_ctx *ctx, const float *X, const int32_t *labels, int batch,
+                        int n_in, int n_hidden, int n_out, int32_t n_pert, float eps,
+                        double scale, double *loss_plus, double *loss_minus,
+                        double *loss_clean);
+
+/* One full MLP step [LOOP]: the clean loss (1.5-SPSA) and the 2*n_pert perturbed losses
+ * (zo_mlp_losses when M + n_hidden <= 49152; otherwise one perturb / loss / restore per evaluation
+ * through the live buffer, enabled by the call if needed), then zo_step.  Arguments as
  * zo_mlp_loss; losses_out as zo_quad_step. */
 zo_status zo_mlp_step(zo_ctx *ctx, const float *X, const int32_t *labels, int batch,
                       int n_in, int n_hidden, int n_out, int32_t n_pert, float eps,

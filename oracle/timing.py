@@ -8,6 +8,7 @@ processes on disjoint samples, each single-threaded).
 
   python -m oracle.timing steps M_SAMPLE SEED N_PERT EPS LR DAMPING WARMUP STEPS
   python -m oracle.timing forward FAMILY CFG_JSON SEQ
+  python -m oracle.timing mlp STEPS
 
 print one JSON object on stdout.
 """
@@ -39,6 +40,24 @@ def quad_steps(M_sample, seed, n_pert, eps, lr, damping, warmup, steps):
         if s >= warmup:
             times.append(time.perf_counter() - t0)
     return {"times": times, "t_start": t_start, "t_end": time.time()}
+
+
+def mlp_steps(steps, n_pert=16, eps=1e-3, lr=1e-2, damping=1e-3):
+    """Seconds of each of `steps` full oracle steps of the MLP workload (64-256-10, batch 64,
+    teacher labels), after one untimed step."""
+    import synth
+
+    from . import mlp, step
+    P = synth.mlp_params(0)
+    teacher = synth.mlp_params(0, tag="teacher")
+    times = []
+    for k in range(steps + 1):
+        X, y = synth.mlp_batch(0, k, teacher)
+        t0 = time.perf_counter()
+        P, _ = step.spsa_step(P, lambda Q: mlp.loss(Q, X, y), n_pert, eps, lr, damping, 0, k)
+        if k:
+            times.append(time.perf_counter() - t0)
+    return {"times": times}
 
 
 def element_rates(M_perturb, M_update, ns):
@@ -79,13 +98,15 @@ def _main(argv):
     if argv[0] == "steps":
         M, seed, n, eps, lr, lam, w, k = argv[1:9]
         res = quad_steps(int(M), int(seed), int(n), float(eps), float(lr), float(lam), int(w), int(k))
+    elif argv[0] == "mlp":
+        res = mlp_steps(int(argv[1]))
     elif argv[0] == "forward":
         cfg = json.loads(argv[2])
         if "class_ids" in cfg:
             cfg["class_ids"] = tuple(cfg["class_ids"])
         res = {"tokens_per_s": forward_tokens_per_s(argv[1], cfg, int(argv[3]))}
     else:
-        raise SystemExit("usage: python -m oracle.timing steps|forward ...")
+        raise SystemExit("usage: python -m oracle.timing steps|forward|mlp ...")
     print(json.dumps(res), flush=True)
 
 

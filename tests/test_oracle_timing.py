@@ -49,3 +49,8 @@ def test_forward_timing_runs_the_oracle_loss():
     theta = (bits.astype(np.uint32) << 16).view(np.float32)
     tok, lab = synth.opt_batch(cfg, 1, 8)
     assert np.isfinite(oracle.qwen.loss(theta, cfg, tok, lab))
+
+
+def test_mlp_step_timing():
+    r = oracle.timing.mlp_steps(1)
+    assert len(r["times"]) == 1 and r["times"][0] > 0

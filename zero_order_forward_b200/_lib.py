@@ -52,6 +52,7 @@ _SIGS = {
     "zo_quad_step_host": [_vp, _vp, _i32, _f32, _f32, _f32, _int, _vp],
     "zo_quad_step_host_async": [_vp, _vp, _i32, _f32, _f32, _f32, _int, _vp],
     "zo_mlp_step": [_vp, _vp, _vp, _int, _int, _int, _int, _i32, _f32, _f32, _f32, _int, _vp],
+    "zo_mlp_losses": [_vp, _vp, _vp, _int, _int, _int, _int, _i32, _f32, _f64, _vp, _vp, _vp],
     "zo_mlp_loss_noalloc": [_vp, _vp, _vp, _int, _int, _int, _int, _f64, _vp, _int, _vp],
     "zo_enable_phase_timing": [_vp, _i32],
     "zo_phase_times": [_vp, _i32, _vp],
@@ -263,6 +264,13 @@ def zo_mlp_step(ctx, X, labels, batch, n_in, n_hidden, n_out, n_pert, eps, lr, d
     return ctx.check(_L.zo_mlp_step(ctx.handle, _ptr(X), _ptr(labels), batch, n_in, n_hidden,
                                     n_out, n_pert, eps, lr, damping, int(preconditioned),
                                     _ptr(losses_out)))
+
+
+def zo_mlp_losses(ctx, X, labels, batch, n_in, n_hidden, n_out, n_pert, eps, scale, loss_plus,
+                  loss_minus, loss_clean=None):
+    return ctx.check(_L.zo_mlp_losses(ctx.handle, _ptr(X), _ptr(labels), batch, n_in, n_hidden,
+                                      n_out, n_pert, eps, scale, _ptr(loss_plus),
+                                      _ptr(loss_minus), _ptr(loss_clean)))
 
 
 def zo_mlp_loss_noalloc(P, X, labels, batch, n_in, n_hidden, n_out, scale, loss_out,

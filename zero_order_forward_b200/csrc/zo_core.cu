@@ -166,6 +166,7 @@ zo_status zo_destroy(zo_ctx *ctx) {
   cudaFree(ctx->live);
   cudaFree(ctx->staging);
   cudaFree(ctx->loss_scratch);
+  cudaFree(ctx->mlp_ce);
   if (ctx->copy_stream) cudaStreamSynchronize(ctx->copy_stream);
   for (int b = 0; b < 2; ++b) {
     cudaFree(ctx->pipe_d[b]);
@@ -534,6 +535,21 @@ zo_status zo_quad_step_host(zo_ctx *ctx, const float *D_host, int32_t n_pert, fl
   return ZO_OK;
 }
 
+zo_status zo_mlp_losses(zo_ctx *ctx, const float *X, const int32_t *labels, int batch, int n_in,
+                        int n_hidden, int n_out, int32_t n_pert, float eps, double scale,
+                        double *loss_plus, double *loss_minus, double *loss_clean) {
+  ZO_CHECK(check_ctx(ctx));
+  if (ctx->dtype != ZO_F32) return fail(ctx, ZO_ERR_UNSUPPORTED, "MLP losses need an fp32 context");
+  if (!X || !labels || !loss_plus || !loss_minus || batch < 1 || n_in < 1 || n_hidden < 1 ||
+      n_out < 1 || n_pert < 1 || n_pert > ZO_MAX_PROBES || !(eps > 0.f) || !std::isfinite(eps))
+    return fail(ctx, ZO_ERR_INVALID, "bad MLP loss arguments");
+  if ((int64_t)n_hidden * n_in + n_hidden + (int64_t)n_out * n_hidden + n_out != ctx->M)
+    return fail(ctx, ZO_ERR_INVALID, "MLP shape does not match M");
+  if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "MLP losses need the clean state");
+  return launch_mlp_probes(ctx, X, labels, batch, n_in, n_hidden, n_out, n_pert, eps, scale,
+                           loss_plus, loss_minus, loss_clean);
+}
+
 zo_status zo_mlp_step(zo_ctx *ctx, const float *X, const int32_t *labels, int batch, int n_in,
                       int n_hidden, int n_out, int32_t n_pert, float eps, float lr,
                       float damping, int preconditioned, double *losses_out) {
@@ -541,9 +557,22 @@ zo_status zo_mlp_step(zo_ctx *ctx, const float *X, const int32_t *labels, int ba
   ZO_CHECK(check_step_args(ctx, n_pert, lr, eps, damping));
   if (!losses_out) return fail(ctx, ZO_ERR_INVALID, "null losses_out");
   if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "step while perturbed");
-  if (!ctx->live_enabled) ZO_CHECK(zo_set_live_buffer(ctx, 1));
   const double scale = 1.0 / (double)batch;
   double *L0 = losses_out, *Lp = losses_out + 1, *Lm = losses_out + 1 + n_pert;
+  if (ctx->dtype == ZO_F32 && ctx->M + n_hidden <= kMlpStageMax) {
+    // every loss of the step from one launch (parameters staged per block), then zo_step
+    phase_mark(ctx, 0);
+    if (!preconditioned)
+      ZO_CUDA(ctx, cudaMemsetAsync(L0, 0, sizeof(double), ctx->stream), "clear L0");
+    phase_mark(ctx, 1);
+    ZO_CHECK(zo_mlp_losses(ctx, X, labels, batch, n_in, n_hidden, n_out, n_pert, eps, scale, Lp,
+                           Lm, preconditioned ? L0 : nullptr));
+    phase_mark(ctx, 2);
+    const zo_status st = zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
+    phase_mark(ctx, 3);
+    return st;
+  }
+  if (!ctx->live_enabled) ZO_CHECK(zo_set_live_buffer(ctx, 1));
   phase_mark(ctx, 0);
   if (preconditioned) {
     ZO_CHECK(zo_mlp_loss(ctx, X, labels, batch, n_in, n_hidden, n_out, scale, L0, 0));

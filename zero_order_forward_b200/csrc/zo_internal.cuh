@@ -134,6 +134,10 @@ struct zo_ctx {
   cudaEvent_t pipe_copied[2] = {nullptr, nullptr}, pipe_consumed[2] = {nullptr, nullptr};
   uint64_t pipe_k = 0;
 
+  // per-sample losses of the batched MLP evaluation ((2 n + 1) x batch doubles)
+  double *mlp_ce = nullptr;
+  size_t mlp_ce_cap = 0;
+
   // phase timing of the step drivers: 4 events per recorded step
   cudaEvent_t *phase_ev = nullptr;
   int32_t phase_cap = 0, phase_used = 0;
@@ -144,6 +148,8 @@ struct zo_ctx {
 namespace zo {
 
 constexpr int kMaxPartials = 32768;
+// Parameters an MLP evaluation block stages in shared memory (192 KB of fp32).
+constexpr int kMlpStageMax = 49152;
 
 zo_status fail(zo_ctx *ctx, zo_status st, const char *fmt, ...);
 zo_status check_launch(zo_ctx *ctx, const char *what);
@@ -172,6 +178,9 @@ zo_status launch_quad_octet(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, int
 // directions from vseed); out_minus != null evaluates both signs of pk's probe in one pass.
 zo_status launch_lowrank_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, const float lam[4],
                               uint64_t vseed, double *out, double *out_minus, int accumulate);
+zo_status launch_mlp_probes(zo_ctx *ctx, const float *X, const int32_t *y, int batch, int n_in,
+                            int n_hidden, int n_out, int n_pert, float eps, double scale,
+                            double *lp, double *lm, double *l0);
 zo_status launch_mlp_loss(zo_ctx *ctx, const float *P, const float *X, const int32_t *y,
                           int batch, int n_in, int n_hidden, int n_out, double scale,
                           double *out, int accumulate);

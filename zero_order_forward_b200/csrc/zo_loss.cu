@@ -653,23 +653,23 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
 
 constexpr int kMlpMax = 1024;
 
-// One block per sample: h = ReLU(W1 x + b1), logits = W2 h + b2, CE(logits, y).
-__global__ void __launch_bounds__(256)
-mlp_loss_kernel(const float *__restrict__ P, const float *__restrict__ X,
-                const int32_t *__restrict__ y, int n_in, int n_hidden, int n_out,
-                double *partials, unsigned int *counter, double *out, int accumulate,
-                double scale) {
-  __shared__ float xs[kMlpMax], hs[kMlpMax], ls[kMlpMax];
-  const float *W1 = P;
-  const float *b1 = W1 + (int64_t)n_hidden * n_in;
-  const float *W2 = b1 + n_hidden;
-  const float *b2 = W2 + (int64_t)n_out * n_hidden;
-  const int b = blockIdx.x;
+// One sample's cross-entropy computed by the whole block (blockDim a multiple of 32), valid
+// in thread 0: h = ReLU(W1 x + b1), logits = W2 h + b2, CE(logits, y).  The arithmetic of a
+// sample does not depend on the block size: each hidden unit is one thread's fmaf chain over
+// the inputs in order, each logit one warp's lane-strided fmaf chains combined by a fixed
+// shuffle-down tree, the cross-entropy one thread's.  The weights may sit in global or
+// shared memory; W1's rows are ld1 floats apart (ld1 >= n_in).  The caller may call it again
+// for another sample right away: the first barrier of the next call orders its writes of hs
+// and ls after this call's reads.
+__device__ double mlp_sample_ce(const float *W1, int ld1, const float *b1, const float *W2,
+                                const float *b2, const float *__restrict__ X,
+                                const int32_t *__restrict__ y, int b, int n_in, int n_hidden,
+                                int n_out, float *xs, float *hs, float *ls) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int k = threadIdx.x; k < n_in; k += blockDim.x) xs[k] = X[(int64_t)b * n_in + k];
   __syncthreads();
   for (int j = threadIdx.x; j < n_hidden; j += blockDim.x) {
-    const float *w = W1 + (int64_t)j * n_in;
+    const float *w = W1 + (int64_t)j * ld1;
     float a = 0.f;
     for (int k = 0; k < n_in; ++k) a = fmaf(w[k], xs[k], a);
     a = __fadd_rn(a, b1[j]);
@@ -695,7 +695,78 @@ mlp_loss_kernel(const float *__restrict__ P, const float *__restrict__ X,
     // an out-of-range label poisons the loss (the step is then skipped as non-finite)
     ce = (label >= 0 && label < n_out) ? (double)(m + logf(s)) - (double)ls[label] : (double)NAN;
   }
+  return ce;
+}
+
+// One block per sample; the per-sample losses are summed in sample order by the last block.
+__global__ void __launch_bounds__(256)
+mlp_loss_kernel(const float *__restrict__ P, const float *__restrict__ X,
+                const int32_t *__restrict__ y, int n_in, int n_hidden, int n_out,
+                double *partials, unsigned int *counter, double *out, int accumulate,
+                double scale) {
+  __shared__ float xs[kMlpMax], hs[kMlpMax], ls[kMlpMax];
+  const float *b1 = P + (int64_t)n_hidden * n_in;
+  const float *W2 = b1 + n_hidden;
+  const float *b2 = W2 + (int64_t)n_out * n_hidden;
+  const double ce = mlp_sample_ce(P, n_in, b1, W2, b2, X, y, blockIdx.x, n_in, n_hidden, n_out,
+                                  xs, hs, ls);
   finish_reduction(ce, partials, counter, out, accumulate, scale);
+}
+
+// All the losses of one MLP step in one launch: blockIdx.x = evaluation e (e < clean: the
+// clean loss; then probe (e - clean) / 2 at +eps for even e - clean and at -eps for odd),
+// blockIdx.y = a slice of per_cta samples.  The block stages its evaluation's parameters
+// rd(theta + s eps z) in shared memory (the sign masks of the 16-element groups first, then
+// one coalesced pass; W1's rows padded to n_in + 1 floats, so that the threads of the hidden
+// layer, one row each, read distinct banks) and writes each sample's cross-entropy to ce[e][b].
+__global__ void __launch_bounds__(256)
+mlp_probes_kernel(const float *__restrict__ theta, int M, const float *__restrict__ X,
+                  const int32_t *__restrict__ y, int batch, int n_in, int n_hidden, int n_out,
+                  ProbeKey pk, int clean, int per_cta, double *__restrict__ ce) {
+  extern __shared__ __align__(16) float Ps[];  // M + n_hidden parameters, then the masks
+  __shared__ float xs[kMlpMax], hs[kMlpMax], ls[kMlpMax];
+  const int n_w1 = n_hidden * n_in, ld1 = n_in + 1;
+  uint16_t *masks = reinterpret_cast<uint16_t *>(Ps + M + n_hidden);
+  const int e = blockIdx.x;
+  const bool perturbed = e >= clean;
+  const int k = e - clean;
+  const float delta = (k & 1) ? -pk.eps : pk.eps;
+  if (perturbed) {
+    const uint32_t step = *pk.step;
+    for (int g = threadIdx.x; g < (M + kGroup - 1) / kGroup; g += blockDim.x)
+      masks[g] = (uint16_t)probe_group_bits((uint64_t)g, (uint32_t)(k >> 1), step, pk.k0, pk.k1);
+    __syncthreads();
+  }
+  for (int j = threadIdx.x; j < M; j += blockDim.x) {
+    const float t = theta[j];
+    const float v = perturbed ? perturb_f32(t, delta, (masks[j >> 4] >> (j & 15)) & 1u) : t;
+    Ps[j < n_w1 ? (j / n_in) * ld1 + j % n_in : j + n_hidden] = v;
+  }
+  __syncthreads();
+  const float *b1s = Ps + n_hidden * ld1;
+  const float *W2s = b1s + n_hidden;
+  const float *b2s = W2s + n_out * n_hidden;
+  const int bend = min(batch, (blockIdx.y + 1) * per_cta);
+  for (int b = blockIdx.y * per_cta; b < bend; ++b) {
+    const double v = mlp_sample_ce(Ps, ld1, b1s, W2s, b2s, X, y, b, n_in, n_hidden, n_out, xs, hs, ls);
+    if (threadIdx.x == 0) ce[(int64_t)e * batch + b] = v;
+  }
+}
+
+// Block e sums evaluation e's per-sample losses in the order of mlp_loss_kernel's reduction
+// (same block size, strided sums, then the block tree) and stores scale * sum.
+__global__ void __launch_bounds__(256)
+mlp_probes_sum_kernel(const double *__restrict__ ce, int batch, double scale, int clean,
+                      double *l0, double *lp, double *lm) {
+  const int e = blockIdx.x;
+  double s = 0.0;
+  for (int i = threadIdx.x; i < batch; i += blockDim.x) s += ce[(int64_t)e * batch + i];
+  s = block_sum(s);
+  if (threadIdx.x == 0) {
+    const int k = e - clean;
+    double *o = e < clean ? l0 : ((k & 1) ? lm : lp) + (k >> 1);
+    *o = 0.0 + scale * s;
+  }
 }
 
 }  // namespace
@@ -802,6 +873,50 @@ zo_status launch_lowrank_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, c
   if (out_minus)
     return launch_quad<true, 4>(ctx, pk, D, out, out_minus, 0, ctx->partials, ctx->counter, lr);
   return launch_quad<false, 4>(ctx, pk, D, out, nullptr, accumulate, ctx->partials, ctx->counter, lr);
+}
+
+zo_status launch_mlp_probes(zo_ctx *ctx, const float *X, const int32_t *y, int batch, int n_in,
+                            int n_hidden, int n_out, int n_pert, float eps, double scale,
+                            double *lp, double *lm, double *l0) {
+  if (n_in > kMlpMax || n_hidden > kMlpMax || n_out > kMlpMax || batch < 1)
+    return fail(ctx, ZO_ERR_INVALID, "mlp shape beyond limits");
+  if (ctx->M + n_hidden > kMlpStageMax)
+    return fail(ctx, ZO_ERR_UNSUPPORTED, "batched MLP losses need M + n_hidden <= %d", kMlpStageMax);
+  const int clean = l0 ? 1 : 0;
+  const int E = 2 * n_pert + clean;
+  const size_t need = (size_t)E * (size_t)batch;
+  if (need > ctx->mlp_ce_cap) {
+    cudaFree(ctx->mlp_ce);
+    ctx->mlp_ce = nullptr;
+    ctx->mlp_ce_cap = 0;
+    const cudaError_t e = cudaMalloc(&ctx->mlp_ce, need * sizeof(double));
+    if (e != cudaSuccess) return fail(ctx, e == cudaErrorMemoryAllocation ? ZO_ERR_OOM : ZO_ERR_CUDA,
+                                      "mlp loss scratch: %s", cudaGetErrorString(e));
+    ctx->mlp_ce_cap = need;
+  }
+  const int M = (int)ctx->M;
+  const size_t smem = (size_t)(M + n_hidden) * sizeof(float) +
+                      (size_t)((M + kGroup - 1) / kGroup) * sizeof(uint16_t);
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e = cudaFuncSetAttribute(mlp_probes_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)(kMlpStageMax * sizeof(float) + kMlpStageMax / 8));
+    if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "mlp_probes_kernel attribute: %s", cudaGetErrorString(e));
+    attr = true;
+  }
+  ProbeKey pk = probe_key(ctx);
+  pk.sign = +1;
+  pk.eps = eps;
+  // about 8 samples per block: the blocks of a step fill the GPU once at the pages' sizes
+  const int per_cta = batch < 8 ? batch : 8;
+  const dim3 grid((unsigned)E, (unsigned)((batch + per_cta - 1) / per_cta));
+  mlp_probes_kernel<<<grid, 256, smem, ctx->stream>>>(static_cast<const float *>(ctx->params), M, X, y,
+                                                      batch, n_in, n_hidden, n_out, pk, clean,
+                                                      per_cta, ctx->mlp_ce);
+  const zo_status st = check_launch(ctx, "mlp_probes_kernel");
+  if (st != ZO_OK) return st;
+  mlp_probes_sum_kernel<<<E, 256, 0, ctx->stream>>>(ctx->mlp_ce, batch, scale, clean, l0, lp, lm);
+  return check_launch(ctx, "mlp_probes_sum_kernel");
 }
 
 zo_status launch_mlp_loss(zo_ctx *ctx, const float *P, const float *X, const int32_t *y,
