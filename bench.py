@@ -15,10 +15,12 @@ The decoder workloads (OPT- or Qwen3-shaped, bf16 weights N(0, 0.02), uniform to
 per-GEMM-shape breakdown of the tcgen05 projections against the measured bf16 peak.
 
 Prints ONE JSON line (rank 0).  With N > 1 (torchrun, one rank per GPU) the ranks share
-one model: every rank holds theta, evaluates its share of the probes (i = rank mod N), the
-2*n_pert fp64 losses are all-gathered over NCCL, and every rank applies the identical
-update ("scaling": "strong"); the step time is the max over ranks.  `--impl reference`
-times the CPU oracle on a bounded slice of the same workload.
+one model ("scaling": "strong"): every rank holds a contiguous slice of theta and D (its
+element offset keeps the global probe signs), evaluates all 2*n_pert + 1 losses over its
+slice's terms, the partial losses are all-gathered over NCCL and summed in rank order (the
+same bits everywhere), and every rank runs the preconditioner and updates its slice; the
+step time is the max over ranks.  `--impl reference` times the CPU oracle on bounded
+samples of the same workload.
 """
 import argparse
 import json
@@ -273,33 +275,36 @@ def gpu_arm(args):
     hbm_peak, peak_kind = peaks()
 
     th_np, D_np = synth.quad_problem(M_FULL, seed=0)  # one shared model across ranks
-    theta = torch.from_numpy(th_np).to(dev)
-    D = torch.from_numpy(D_np).to(dev)
+    # N > 1: every rank holds a contiguous slice of theta and D (its element offset keeps the
+    # global probe signs); the quadratic's loss is the sum of the slices' losses
+    first, count = 0, M_FULL
+    if world > 1:
+        from zero_order_forward_b200 import dist as zdist
+        first, count = zdist.shard_range(M_FULL, rank, world)
+    theta = torch.from_numpy(th_np[first:first + count]).to(dev)
+    D = torch.from_numpy(D_np[first:first + count]).to(dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     n = N_PERT
     losses = torch.zeros(2 * n + 1, dtype=torch.float64, device=dev)
     stream = torch.cuda.current_stream(dev)
     ctx = zo.zo_create(theta, seed=0, stream=stream.cuda_stream)
-
-    def loss_at(sign, probe, out):
-        zo.zo_perturb(ctx, sign, EPS, probe)
-        zo.zo_quad_loss(ctx, D, out)
-        zo.zo_restore(ctx)
+    if first:
+        zo.zo_set_element_offset(ctx, first)
+    n_oct = (n + 63) // 64  # loss passes per step (64 probes each)
 
     def apply_step(Lp, Lm, L0):
         zo.zo_step(ctx, Lp, Lm, n, L0, LR, EPS, DAMPING)
 
-    # probes per rank and pass: up to eight octets, fewer when the ranks would otherwise idle
-    block = min(64, max(8, -(-(n // world) // 8) * 8))
-
-    def octet_at(first, count, out_plus, out_minus):
-        zo.zo_quad_loss_octet(ctx, D, first, count, EPS, out_plus, out_minus)
+    def partial_losses(out):  # all 2n + 1 losses over this rank's slice, L0 in the first pass
+        for o in range(n_oct):
+            c = min(64, n - 64 * o)
+            zo.zo_quad_loss_octet(ctx, D, 64 * o, c, EPS, out[1 + 64 * o:1 + 64 * o + c],
+                                  out[1 + n + 64 * o:1 + n + 64 * o + c],
+                                  out[0:1] if o == 0 else None)
 
     def one_step():
-        if world > 1:  # probe-parallel: this rank's probe octets, loss all-gather, same update
-            from zero_order_forward_b200 import dist as zdist
-            zdist.probe_parallel_step(n, loss_at, lambda o: zo.zo_quad_loss(ctx, D, o),
-                                      apply_step, dev, block=block, block_at=octet_at)
+        if world > 1:  # element-parallel: partial losses, all-gather + rank-order sum, slice update
+            zdist.element_parallel_step(n, partial_losses, apply_step, dev)
         else:  # the native step driver: every launch of the step enqueued from C++
             zo.zo_quad_step(ctx, D, n, EPS, LR, DAMPING, True, losses)
 
@@ -350,7 +355,6 @@ def gpu_arm(args):
     # holds n/64 launches of the octet kernel (the 128 losses L(theta +- eps z_i) of eight
     # probe octets from one pass over theta and D); with N ranks the phase is not bracketed
     # separately: time the kernel alone.
-    n_oct = (n + 63) // 64
     if world > 1:
         le = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         flush.zero_()
@@ -362,9 +366,9 @@ def gpu_arm(args):
         torch.cuda.synchronize()
         probe_ms = [le[0].elapsed_time(le[1])]
     loss_us = 1e3 * statistics.mean(probe_ms) / n_oct
-    loss_bytes = 8 * M_FULL  # theta and D read once per pass, fp32
+    loss_bytes = 8 * count  # this rank's theta and D read once per pass, fp32
     achieved = loss_bytes / (loss_us * 1e-6) / 1e9
-    upd_bytes = 8 * M_FULL  # theta read + written, fp32
+    upd_bytes = 8 * count  # theta read + written, fp32
 
     # the one-probe form (both signs of one probe per pass), timed alone for comparison
     pe = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
@@ -429,7 +433,7 @@ def gpu_arm(args):
             del th_s, out_s
 
     # end to end through the public API with host buffers: D copied in, losses copied out
-    D_host = torch.from_numpy(D_np).pin_memory()
+    D_host = torch.from_numpy(D_np[first:first + count]).pin_memory()
     L_host = torch.zeros(2 * n + 1, dtype=torch.float64).pin_memory()
     e2e_steps = max(3, min(args.steps, 30))
 
@@ -437,11 +441,9 @@ def gpu_arm(args):
         if world == 1:  # pipelined: step k+1's copy of D overlaps step k's kernels
             zo.zo_quad_step_host_async(ctx, D_host, n, EPS, LR, DAMPING, True, L_host)
             return
-        D.copy_(D_host, non_blocking=True)
-        from zero_order_forward_b200 import dist as zdist
-        L0, Lp, Lm = zdist.probe_parallel_step(n, loss_at, lambda o: zo.zo_quad_loss(ctx, D, o),
-                                               apply_step, dev, block=16, block_at=octet_at)
-        L_host.copy_(torch.cat([L0, Lp, Lm]))  # synchronous device -> host read
+        D.copy_(D_host, non_blocking=True)  # this rank's slice of D
+        tot = zdist.element_parallel_step(n, partial_losses, apply_step, dev)
+        L_host.copy_(tot)  # synchronous device -> host read
     e2e_step()  # staging allocation
     if world > 1:
         dist.barrier()
@@ -479,18 +481,19 @@ def gpu_arm(args):
                 "update": rates["update"],
                 "sample": "oracle perturbation of 2^22 elements (one probe); oracle fp32-order "
                           "update of 2^20 elements with n probes regenerated"}
-        if world == 1:  # the loss passes (clean loss fused into the first), precond, update
-            launches_per_step = n_oct + 2
-        else:  # the clean loss, this rank's probe blocks, precond, update
-            from zero_order_forward_b200 import dist as zdist
-            launches_per_step = 1 + len(list(zdist.rank_units(n, rank, world, block))) + 2
+        # the loss passes (clean loss fused into the first), precond, update; with N ranks the
+        # same per rank on its slice (the loss exchange is NCCL's)
+        launches_per_step = n_oct + 2
         line = {
             "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
             "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "M": M_FULL, "n_pert": n, "eps": EPS, "lr": LR,
-                       "damping": DAMPING, "parallelism": f"probe-parallel x{world}",
+                       "damping": DAMPING,
+                       "parallelism": (f"element-parallel x{world}: theta and D sharded in "
+                                       f"contiguous slices, partial losses all-gathered"
+                                       if world > 1 else "1 GPU"),
                        "l2": "flushed between steps (256 MiB write, untimed); theta+D = 128 MiB"},
             "roofline": {"kernel": "quad_octet_kernel (the 128 losses L(theta +- eps z_i) of "
                                    "eight probe octets in one pass, perturbation on load, fp64 "
@@ -516,11 +519,11 @@ def gpu_arm(args):
                           "precond_update": statistics.mean(upd_ms)},
             "tokens_per_s": None,
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": 4 * M_FULL * world,
+            "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": 4 * M_FULL,
                     "d2h_bytes_per_step": 8 * (2 * n + 1) * world,
-                    "path": "D pinned host -> device every step on every rank, losses back "
-                            "(zo_quad_step_host_async at one GPU: copies on the context's copy "
-                            "stream overlap the previous step's kernels)"},
+                    "path": "D pinned host -> device every step (each rank its slice), losses "
+                            "back (zo_quad_step_host_async at one GPU: copies on the context's "
+                            "copy stream overlap the previous step's kernels)"},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
         }

@@ -136,6 +136,18 @@ zo_status zo_sync(zo_ctx *ctx, uint32_t *flags);
 zo_status zo_get_step(zo_ctx *ctx, uint32_t *step);
 zo_status zo_set_step(zo_ctx *ctx, uint32_t step);
 
+/* Element offset for a context that holds a slice of a larger parameter vector: params[j]
+ * is element first_element + j of that vector (first_element >= 0, a multiple of 16, so
+ * that slices keep whole 16-element sign groups).  Every sign the context generates
+ * (zo_perturb, zo_perturb_range, zo_pack_probe, the quadratic losses, zo_update, zo_step) is
+ * then the sign of the global element index, so contexts with the same seed and step on
+ * disjoint slices perturb and update exactly as one context on the whole vector would,
+ * element by element; a separable loss (the diagonal quadratic) is the sum of the slices'
+ * losses.  Default 0.  The MLP, low-rank and decoder entry points, whose losses are not sums
+ * over parameter slices, return ZO_ERR_UNSUPPORTED while the offset is not 0.  Errors:
+ * ZO_ERR_INVALID (negative or not a multiple of 16), ZO_ERR_STATE (perturbed). */
+zo_status zo_set_element_offset(zo_ctx *ctx, int64_t first_element);
+
 /* ------------------------------------------------------------------ tracing */
 
 /* Phase timing of the step drivers (zo_quad_step, zo_mlp_step, zo_model_step): the next

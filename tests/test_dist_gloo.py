@@ -1,5 +1,6 @@
-"""Host-side logic of the probe-parallel step on 2 and 3 CPU ranks (gloo): the probe
-partition, the loss exchange and bit-identical replicas.  The per-probe loss and the update
+"""Host-side logic of the probe-parallel and element-parallel steps on 2 and 3 CPU ranks
+(gloo): the probe partition, the element slices, the loss exchange and bit-identical
+replicas or slices.  The per-probe loss and the update
 are the oracle's here (CPU); on GPUs the same driver calls the CUDA library over NCCL."""
 import os
 import socket
@@ -93,3 +94,73 @@ def test_probe_parallel_step_matches_single_rank(tmp_path, world, block):
         assert np.array_equal(o["Lp"], rec["Lp"]) and np.array_equal(o["Lm"], rec["Lm"])
         assert o["L0"][0] == rec["L0"]
         assert o["theta"].tobytes() == nxt.tobytes()  # bit-identical replicas
+
+
+def test_shard_ranges_tile_the_vector():
+    for M in (16, 17, 3000, 1 << 20, (1 << 24) + 5):
+        for world in (1, 2, 3, 8):
+            ranges = [zdist.shard_range(M, r, world) for r in range(world)]
+            assert sum(c for _, c in ranges) == M
+            pos = 0
+            for first, count in ranges:
+                assert first == pos and count >= 0
+                assert count == 0 or first % 16 == 0  # empty slices only past the end
+                pos += count
+
+
+def _element_worker(rank, world, port, out_dir):
+    import torch.distributed as dist
+
+    import oracle
+    import synth
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        theta, D = synth.quad_problem(M, seed=1)
+        first, count = zdist.shard_range(M, rank, world)
+        th, Ds = theta[first:first + count].copy(), D[first:first + count]
+        e32 = float(np.float32(EPS))
+        state = {}
+
+        def partial_losses(out):  # this slice's terms, signs of the global element index
+            out[0] = oracle.core.quad_loss(th, Ds)
+            for i in range(N_PERT):
+                for s, off in ((+1, 1), (-1, 1 + N_PERT)):
+                    P = oracle.core.perturb(th, SEED, 0, i, s, e32, j0=first)
+                    out[off + i] = oracle.core.quad_loss(P, Ds)
+
+        def apply_step(Lp, Lm, L0):
+            pc = oracle.core.precond(Lp.numpy(), Lm.numpy(), float(L0[0]), e32,
+                                     float(np.float32(LR)), float(np.float32(LAM)),
+                                     float(np.float32(0.1)))
+            state["a"] = pc["a"].astype(np.float32)
+            state["theta"] = oracle.core.update_mirror(th, state["a"], SEED, 0, j0=first)
+
+        tot = zdist.element_parallel_step(N_PERT, partial_losses, apply_step, "cpu")
+        np.savez(os.path.join(out_dir, f"e{rank}.npz"), theta=state["theta"], a=state["a"],
+                 tot=tot.numpy(), first=first)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_element_parallel_step_matches_single_rank(tmp_path, world):
+    """Every rank sums the same totals (bit for bit); they equal the whole vector's losses to
+    fp64 rounding; each rank's updated slice equals the whole-vector update with the same
+    coefficients, element by element."""
+    import oracle
+    import synth
+    mp.start_processes(_element_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    theta, D = synth.quad_problem(M, seed=1)
+    _, rec = oracle.step.spsa_step(theta, lambda P: oracle.core.quad_loss(P, D), N_PERT, EPS,
+                                   LR, LAM, SEED, 0, update="mirror")
+    outs = [np.load(tmp_path / f"e{r}.npz") for r in range(world)]
+    ref = np.concatenate([[rec["L0"]], rec["Lp"], rec["Lm"]])
+    for o in outs:
+        assert np.array_equal(o["tot"], outs[0]["tot"]) and np.array_equal(o["a"], outs[0]["a"])
+        assert np.allclose(o["tot"], ref, rtol=1e-13, atol=0)
+    full = oracle.core.update_mirror(theta, outs[0]["a"], SEED, 0)
+    got = np.concatenate([o["theta"] for o in outs])
+    assert got.tobytes() == full.tobytes()

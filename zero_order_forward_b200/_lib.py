@@ -38,6 +38,7 @@ _SIGS = {
     "zo_sync": [_vp, ctypes.POINTER(_u32)],
     "zo_get_step": [_vp, ctypes.POINTER(_u32)],
     "zo_set_step": [_vp, _u32],
+    "zo_set_element_offset": [_vp, _i64],
     "zo_pack_probe": [_vp, _i32, _i64, _i64, _vp],
     "zo_perturb": [_vp, _int, _f32, _i32],
     "zo_restore": [_vp],
@@ -194,6 +195,10 @@ def zo_get_step(ctx):
 
 def zo_set_step(ctx, step):
     return ctx.check(_L.zo_set_step(ctx.handle, step))
+
+
+def zo_set_element_offset(ctx, first_element):
+    return ctx.check(_L.zo_set_element_offset(ctx.handle, int(first_element)))
 
 
 def zo_pack_probe(ctx, probe, first_byte, nbytes, out):

@@ -44,6 +44,7 @@ ProbeKey probe_key(const zo_ctx *ctx) {
   pk.probe = (uint32_t)ctx->probe;
   pk.sign = ctx->state == PState::Perturbed ? ctx->sign : 0;
   pk.eps = ctx->eps;
+  pk.g_off = (uint64_t)(ctx->first_element / kGroup);
   return pk;
 }
 
@@ -282,6 +283,15 @@ zo_status zo_set_step(zo_ctx *ctx, uint32_t step) {
   return ZO_OK;
 }
 
+zo_status zo_set_element_offset(zo_ctx *ctx, int64_t first_element) {
+  ZO_CHECK(check_ctx(ctx));
+  if (first_element < 0 || first_element % kGroup)
+    return fail(ctx, ZO_ERR_INVALID, "element offset must be a non-negative multiple of %d", kGroup);
+  if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "element offset set while perturbed");
+  ctx->first_element = first_element;
+  return ZO_OK;
+}
+
 zo_status zo_pack_probe(zo_ctx *ctx, int32_t probe, int64_t first_byte, int64_t nbytes,
                         uint8_t *dev_out) {
   ZO_CHECK(check_ctx(ctx));
@@ -351,6 +361,8 @@ zo_status zo_quad_loss_pair(zo_ctx *ctx, const float *D, int32_t probe, float ep
 zo_status zo_mlp_loss(zo_ctx *ctx, const float *X, const int32_t *labels, int batch, int n_in,
                       int n_hidden, int n_out, double scale, double *loss_out, int accumulate) {
   ZO_CHECK(check_ctx(ctx));
+  if (ctx->first_element != 0)
+    return fail(ctx, ZO_ERR_UNSUPPORTED, "MLP loss: not separable over parameter slices (element offset must be 0)");
   if (ctx->dtype != ZO_F32) return fail(ctx, ZO_ERR_UNSUPPORTED, "MLP loss needs an fp32 context");
   if (!X || !labels || !loss_out || batch < 1 || n_in < 1 || n_hidden < 1 || n_out < 1)
     return fail(ctx, ZO_ERR_INVALID, "bad MLP arguments");
@@ -407,6 +419,8 @@ zo_status check_lowrank(zo_ctx *ctx, const float *D, const zo_lowrank *q, float 
 zo_status zo_lowrank_loss(zo_ctx *ctx, const float *D, const zo_lowrank *q, double *loss_out,
                           int accumulate) {
   ZO_CHECK(check_ctx(ctx));
+  if (ctx->first_element != 0)
+    return fail(ctx, ZO_ERR_UNSUPPORTED, "low-rank loss: not separable over parameter slices (element offset must be 0)");
   float lam[4];
   ZO_CHECK(check_lowrank(ctx, D, q, lam));
   if (!loss_out) return fail(ctx, ZO_ERR_INVALID, "null loss_out");
@@ -416,6 +430,8 @@ zo_status zo_lowrank_loss(zo_ctx *ctx, const float *D, const zo_lowrank *q, doub
 zo_status zo_lowrank_loss_pair(zo_ctx *ctx, const float *D, const zo_lowrank *q, int32_t probe,
                                float eps, double *loss_plus, double *loss_minus) {
   ZO_CHECK(check_ctx(ctx));
+  if (ctx->first_element != 0)
+    return fail(ctx, ZO_ERR_UNSUPPORTED, "low-rank loss: not separable over parameter slices (element offset must be 0)");
   float lam[4];
   ZO_CHECK(check_lowrank(ctx, D, q, lam));
   if (!loss_plus || !loss_minus) return fail(ctx, ZO_ERR_INVALID, "null output");
@@ -432,6 +448,8 @@ zo_status zo_lowrank_step(zo_ctx *ctx, const float *D, const zo_lowrank *q, int3
                           float eps, float lr, float damping, int preconditioned,
                           double *losses_out) {
   ZO_CHECK(check_ctx(ctx));
+  if (ctx->first_element != 0)
+    return fail(ctx, ZO_ERR_UNSUPPORTED, "low-rank step: not separable over parameter slices (element offset must be 0)");
   ZO_CHECK(check_step_args(ctx, n_pert, lr, eps, damping));
   if (!losses_out) return fail(ctx, ZO_ERR_INVALID, "null losses_out");
   if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "step while perturbed");
@@ -539,6 +557,8 @@ zo_status zo_mlp_losses(zo_ctx *ctx, const float *X, const int32_t *labels, int 
                         int n_hidden, int n_out, int32_t n_pert, float eps, double scale,
                         double *loss_plus, double *loss_minus, double *loss_clean) {
   ZO_CHECK(check_ctx(ctx));
+  if (ctx->first_element != 0)
+    return fail(ctx, ZO_ERR_UNSUPPORTED, "MLP losses: not separable over parameter slices (element offset must be 0)");
   if (ctx->dtype != ZO_F32) return fail(ctx, ZO_ERR_UNSUPPORTED, "MLP losses need an fp32 context");
   if (!X || !labels || !loss_plus || !loss_minus || batch < 1 || n_in < 1 || n_hidden < 1 ||
       n_out < 1 || n_pert < 1 || n_pert > ZO_MAX_PROBES || !(eps > 0.f) || !std::isfinite(eps))
@@ -554,6 +574,8 @@ zo_status zo_mlp_step(zo_ctx *ctx, const float *X, const int32_t *labels, int ba
                       int n_hidden, int n_out, int32_t n_pert, float eps, float lr,
                       float damping, int preconditioned, double *losses_out) {
   ZO_CHECK(check_ctx(ctx));
+  if (ctx->first_element != 0)
+    return fail(ctx, ZO_ERR_UNSUPPORTED, "MLP step: not separable over parameter slices (element offset must be 0)");
   ZO_CHECK(check_step_args(ctx, n_pert, lr, eps, damping));
   if (!losses_out) return fail(ctx, ZO_ERR_INVALID, "null losses_out");
   if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "step while perturbed");

@@ -478,6 +478,8 @@ zo_status run_layers(zo_model *m, const int32_t *tokens, int B, int S, int n_run
 }
 
 zo_status check_batch(zo_model *m, const int32_t *tokens, int B, int S) {
+  if (m->ctx->first_element != 0)
+    return fail(m->ctx, ZO_ERR_UNSUPPORTED, "model: not separable over parameter slices (element offset must be 0)");
   if (!tokens || B < 1 || S < 1 || S > m->cfg.max_pos || (int64_t)B * S > m->max_tokens)
     return fail(m->ctx, ZO_ERR_INVALID, "batch %d x seq %d: need seq <= max_pos and B*S <= %lld",
                 B, S, (long long)m->max_tokens);
@@ -503,6 +505,8 @@ zo_status zo_model_create(zo_model **out, zo_ctx *ctx, const zo_model_cfg *cfg, 
   if (!make_layout(*cfg, &L)) return fail(ctx, ZO_ERR_INVALID, "invalid model configuration");
   if (ctx->dtype != ZO_BF16 || ctx->M != L.total)
     return fail(ctx, ZO_ERR_INVALID, "model needs a bf16 context with M = %lld", (long long)L.total);
+  if (ctx->first_element != 0)
+    return fail(ctx, ZO_ERR_UNSUPPORTED, "model: not separable over parameter slices (element offset must be 0)");
   if (max_tokens < 1) return fail(ctx, ZO_ERR_INVALID, "max_tokens must be >= 1");
   zo_model *m = new (std::nothrow) zo_model();
   if (!m) return ZO_ERR_OOM;
@@ -622,6 +626,8 @@ zo_status zo_model_step(zo_model *m, const int32_t *tokens, const int32_t *label
   if (!m) return ZO_ERR_INVALID;
   zo_ctx *ctx = m->ctx;
   if (n_micro < 1 || !losses_out) return fail(ctx, ZO_ERR_INVALID, "bad step arguments");
+  if (ctx->first_element != 0)
+    return fail(ctx, ZO_ERR_UNSUPPORTED, "model: not separable over parameter slices (element offset must be 0)");
   if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "step while perturbed");
   const double scale = 1.0 / ((double)n_micro * batch);
   const int64_t tok_stride = (int64_t)batch * seq;

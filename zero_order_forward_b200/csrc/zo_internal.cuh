@@ -34,6 +34,7 @@ struct ProbeKey {
   uint32_t probe;
   int sign;                 // +1 / -1 ; 0 = clean (no perturbation)
   float eps;
+  uint64_t g_off;           // global index of the context's first 16-element group
 };
 
 // ------------------------------------------------------------------ Philox4x32-10
@@ -114,6 +115,8 @@ struct zo_ctx {
   int sign = 0;
   float eps = 0.f;
   int32_t probe = 0;
+
+  int64_t first_element = 0;  // global index of params[0] (a multiple of 16)
 
   bool live_enabled = false;
   void *live = nullptr;        // M elements when enabled

@@ -296,7 +296,7 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
       // computes its 16 bits (groups past M are computed and never used).
       const uint64_t my_group = (uint64_t)(base / kGroup) + 8 * cw + 64 * (lane >> 3) + (lane & 7);
       uint32_t mine = 0u;
-      if (pk.sign) mine = probe_group_bits(my_group, pk.probe, step, pk.k0, pk.k1);
+      if (pk.sign) mine = probe_group_bits(my_group + pk.g_off, pk.probe, step, pk.k0, pk.k1);
       uint4 vmine = make_uint4(0u, 0u, 0u, 0u);
       if (R > 0) vmine = sign_block(my_group, 0u, 0u, lr.vk0, lr.vk1);
 #pragma unroll
@@ -464,7 +464,7 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
       // 4q..4q+3 (word q of each block of that group); the pair's vectors are words
       // 2 (q >> 1) and 2 (q >> 1) + 1.  The quad's lanes generate the blocks it needs and
       // four shuffles hand each lane the pair's two words of each of its octets.
-      const uint64_t g0 = (uint64_t)(base / kGroup) + 8 * cw + quad;
+      const uint64_t g0 = pk.g_off + (uint64_t)(base / kGroup) + 8 * cw + quad;
       // NOCT 2: once per chunk, lane q generates (vector q >> 1, octet q & 1); lane l reads
       // lane l in rounds 0, 1 and lane l ^ 2 (the other vector) in rounds 2, 3.
       uint32_t wo2[kOIters], wp2[kOIters];

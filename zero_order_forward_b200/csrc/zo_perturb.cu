@@ -78,7 +78,7 @@ perturb_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t first, 
       for (int i = 0; i < kTileGroups / 32; ++i) {
         const int64_t g = g0 + tile * kTileGroups + lane + 32 * i;
         masks[warp][lane + 32 * i] =
-            g * kGroup < end ? (uint16_t)probe_group_bits(g, pk.probe, step, pk.k0, pk.k1) : 0;
+            g * kGroup < end ? (uint16_t)probe_group_bits(g + pk.g_off, pk.probe, step, pk.k0, pk.k1) : 0;
       }
       __syncwarp();
     }
@@ -208,7 +208,7 @@ perturb_pipe_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t fi
       // The warp's 32 groups: slot q = 2N k + j is group 2N cw + 16N k + j of the chunk.
       uint32_t mine = 0u;
       if (pk.sign)
-        mine = probe_group_bits((uint64_t)(g0 + c * kTileGroups) + 2 * N * cw +
+        mine = probe_group_bits(pk.g_off + (uint64_t)(g0 + c * kTileGroups) + 2 * N * cw +
                                     16 * N * (lane / (2 * N)) + lane % (2 * N),
                                 pk.probe, step, pk.k0, pk.k1);
 #pragma unroll
@@ -246,12 +246,12 @@ perturb_pipe_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t fi
 // Bits of elements >= M are cleared.
 __global__ void pack_kernel(uint8_t *__restrict__ out, int64_t first_byte, int64_t nbytes,
                             int64_t M, uint32_t probe, const uint32_t *step_ptr, uint32_t k0,
-                            uint32_t k1) {
+                            uint32_t k1, uint64_t g_off) {
   const int64_t gfirst = first_byte / 2;
   const int64_t glast = (first_byte + nbytes - 1) / 2;
   const int64_t g = gfirst + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (g > glast) return;
-  const uint32_t m = probe_group_bits((uint64_t)g, probe, *step_ptr, k0, k1);
+  const uint32_t m = probe_group_bits((uint64_t)g + g_off, probe, *step_ptr, k0, k1);
   for (int q = 0; q < 2; ++q) {
     const int64_t byte = g * 2 + q;
     if (byte < first_byte || byte >= first_byte + nbytes) continue;
@@ -315,7 +315,7 @@ zo_status launch_pack(zo_ctx *ctx, uint32_t probe, int64_t first_byte, int64_t n
   const int64_t blocks = (groups + threads - 1) / threads;
   ProbeKey pk = probe_key(ctx);
   pack_kernel<<<(unsigned)blocks, threads, 0, ctx->stream>>>(
-      out, first_byte, nbytes, ctx->M, probe, &ctx->dstate->step, pk.k0, pk.k1);
+      out, first_byte, nbytes, ctx->M, probe, &ctx->dstate->step, pk.k0, pk.k1, pk.g_off);
   return check_launch(ctx, "pack_kernel");
 }
 

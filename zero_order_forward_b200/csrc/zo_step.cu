@@ -154,11 +154,14 @@ constexpr int kUpdThreads = 1024;
 // octet's table is the fp32 sum, left to right from its first signed term, of
 // (bit t of e ? -a : +a) over the octet's probes t; the octet sums are added in order and
 // subtracted once.  The tables are replicated R = 2^LOG_R times and lane l reads replica
-// l mod R, so the 32 lookups of a warp meet at most 32/R to a bank (none at R = 32).
+// l mod R, so the 32 lookups of a warp meet at most 32/R to a bank (none at R = 32).  g_off is
+// the global index of the context's first group: its elements take the signs of their
+// global indices.
 template <typename T, int LOG_R>
 __global__ void __launch_bounds__(kUpdThreads)
 update_kernel(T *__restrict__ theta, int64_t M, const float *__restrict__ coef, int n,
-              const uint32_t *step_ptr, const uint32_t *ok_ptr, uint32_t k0, uint32_t k1) {
+              const uint32_t *step_ptr, const uint32_t *ok_ptr, uint32_t k0, uint32_t k1,
+              uint64_t g_off) {
   constexpr int R = 1 << LOG_R;
   extern __shared__ float lut[];  // [octet][256 entries][R replicas]
   // Launched with programmatic dependent launch: wait for the preconditioner (coefficients,
@@ -206,7 +209,7 @@ update_kernel(T *__restrict__ theta, int64_t M, const float *__restrict__ coef, 
 #pragma unroll
     for (int e = 0; e < 16; ++e) acc[e] = 0.f;
     for (int o = 0; o < octets; ++o) {
-      const uint4 blk = sign_block((uint64_t)g, (uint32_t)o, step, k0, k1);
+      const uint4 blk = sign_block((uint64_t)g + g_off, (uint32_t)o, step, k0, k1);
       const uint32_t w[4] = {blk.x, blk.y, blk.z, blk.w};
       const float *tab = mine + ((o * 256) << LOG_R);
 #pragma unroll
@@ -257,7 +260,7 @@ zo_status launch_update_t(zo_ctx *ctx, const float *coef, int n, const uint32_t 
   cfg.attrs = attr_pdl;
   cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, kern, static_cast<T *>(ctx->params), ctx->M, coef, n, step_ptr,
-                         ok_ptr, k0, k1);
+                         ok_ptr, k0, k1, (uint64_t)(ctx->first_element / kGroup));
   if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "update_kernel: %s", cudaGetErrorString(e));
   return check_launch(ctx, "update_kernel");
 }

@@ -1,4 +1,4 @@
-"""Probe-parallel zero-order steps across ranks (one process per GPU).
+"""Probe-parallel and element-parallel zero-order steps across ranks (one process per GPU).
 
 Splitting probe evaluation across devices needs no gradient communication
 ("Stanford's 1.5-SPSA Trains OPT-30B Without Backpropagation", section "How 1.5-SPSA
@@ -8,6 +8,15 @@ probes i = r, r + N, r + 2N, ... (or, with block = B, the blocks of B consecutiv
 u = r, r + N, ...: the probe octets of the quadratic's one-pass evaluation).  The only exchange is an all-gather of the 2*n_pert fp64
 losses; afterwards every rank runs the same deterministic preconditioner and update, so the
 replicas of theta stay bit-identical with no parameter traffic.
+
+For a loss that is a sum of per-element terms (the diagonal quadratic), the parameters can
+instead be cut into contiguous slices, one per rank (element_parallel_step): every rank
+evaluates all 2 n + 1 losses over its own slice's terms (the context's element offset keeps
+each element's signs those of its global index), the partial losses are all-gathered and
+summed in rank order, so every rank holds the same totals bit for bit, and each rank runs the
+preconditioner and updates its own slice.  This is the batch-parallel split with the loss's
+terms as the batch; the parameters are sharded with them, so neither the evaluation nor the
+update is repeated on every rank, and only 2 n + 1 numbers per rank cross the network.
 
 The per-rank loss evaluation and the update are passed in as callables, so this module
 holds only the partition and the exchange (torch.distributed: NCCL on GPUs; gloo works for
@@ -105,3 +114,39 @@ def probe_parallel_step(n_pert, loss_at, clean_loss, apply_step, device, dtype=t
     Lp, Lm = gather_losses(local, n_pert, group, block)
     apply_step(Lp, Lm, L0)
     return L0, Lp, Lm
+
+
+def shard_range(M, rank, world, align=16):
+    """(first, count) of rank's contiguous slice of M elements: slices of ceil(M / world)
+    elements rounded up to a multiple of `align` (whole sign groups), the last one shorter."""
+    if not (0 <= rank < world) or M < 1 or align < 1:
+        raise ValueError("bad shard arguments")
+    per = -(-M // world)
+    per = -(-per // align) * align
+    first = min(M, rank * per)
+    return first, min(M, first + per) - first
+
+
+def sum_partials(local, group=None):
+    """All-gather every rank's partial sums (a 1-D tensor) and add them in rank order, so
+    that every rank obtains the same bits."""
+    world = dist.get_world_size(group)
+    parts = [torch.empty_like(local) for _ in range(world)]
+    dist.all_gather(parts, local.contiguous(), group=group)
+    total = parts[0].clone()
+    for p in parts[1:]:
+        total += p
+    return total
+
+
+def element_parallel_step(n_pert, partial_losses, apply_step, device, dtype=torch.float64,
+                          group=None):
+    """One step with the parameters sharded by elements, for a loss that is a sum over
+    elements.  partial_losses(out) writes this rank's [L0, L+_0..L+_{n-1}, L-_0..L-_{n-1}]
+    over its slice's terms (2 n + 1 values); apply_step(Lp, Lm, L0) runs the preconditioner and
+    the update of this rank's slice with the summed losses.  Returns the summed losses."""
+    local = torch.zeros(2 * n_pert + 1, dtype=dtype, device=device)
+    partial_losses(local)
+    total = sum_partials(local, group)
+    apply_step(total[1:1 + n_pert], total[1 + n_pert:], total[0:1])
+    return total
