@@ -46,13 +46,13 @@ FALLBACK_HBM_GBS = 6650.0
 # summarised in profiles/quad_octet_kernel.quadratic_M2p24.md, valid for the kernel sources
 # whose SHA-256 (of zo_loss.cu and zo_internal.cuh, concatenated) is recorded with it;
 # reported as null when a source has changed since the capture.
-LOSS_TRAFFIC = {"sources_sha256": "9b335eb404ea87eb12e71961072df3fb323ad181fc7a22ad54af96181b0493cb",
-                "bytes": 139.47e6}
+LOSS_TRAFFIC = {"sources_sha256": "37d27d15311f7dbb48056ece9469b07e3741a49c8658e8a77838f044d238ab3f",
+                "bytes": 140.4e6}
 LOSS_SOURCES = ("zo_loss.cu", "zo_internal.cuh")
 # Warp instructions one launch of the loss kernel executes (ncu smsp__inst_executed.sum, same
 # capture and validity rule as LOSS_TRAFFIC): the pass is bound by instruction issue, so its
 # roofline is the issue limit, 148 SMs x 4 warp-instructions per clock at the sampled clock.
-LOSS_WARP_INSTRUCTIONS = 90.54e6
+LOSS_WARP_INSTRUCTIONS = 90.23e6
 SM_COUNT, ISSUE_PER_SM_CLOCK = 148, 4
 
 
