@@ -46,13 +46,13 @@ FALLBACK_HBM_GBS = 6650.0
 # summarised in profiles/quad_octet_kernel.quadratic_M2p24.md, valid for the kernel sources
 # whose SHA-256 (of zo_loss.cu and zo_internal.cuh, concatenated) is recorded with it;
 # reported as null when a source has changed since the capture.
-LOSS_TRAFFIC = {"sources_sha256": "37d27d15311f7dbb48056ece9469b07e3741a49c8658e8a77838f044d238ab3f",
-                "bytes": 140.4e6}
+LOSS_TRAFFIC = {"sources_sha256": "40b6f128f7e71a7030ba65176bbfac529d5065dbd074e46c1b3d2b8ed8946608",
+                "bytes": 139.2e6}
 LOSS_SOURCES = ("zo_loss.cu", "zo_internal.cuh")
 # Warp instructions one launch of the loss kernel executes (ncu smsp__inst_executed.sum, same
 # capture and validity rule as LOSS_TRAFFIC): the pass is bound by instruction issue, so its
 # roofline is the issue limit, 148 SMs x 4 warp-instructions per clock at the sampled clock.
-LOSS_WARP_INSTRUCTIONS = 90.23e6
+LOSS_WARP_INSTRUCTIONS = 90.41e6
 SM_COUNT, ISSUE_PER_SM_CLOCK = 148, 4
 
 
@@ -791,8 +791,13 @@ def lowrank_arm(args):
     ph = zo.zo_phase_times(ctx, args.steps)
     zo.zo_enable_phase_timing(ctx, 0)
     total_s = sum(e[0].elapsed_time(e[1]) for e in evs) / 1e3
-    loss_us = 1e3 * float(ph[:, 1].mean()) / n
-    achieved = 8 * M_FULL / (loss_us * 1e-6) / 1e9
+    # the probe phase: per 64 probes one diagonal table pass (theta and D) and one pass per
+    # direction for the dot products (theta only), then the combination
+    rank = len(lam)
+    passes = ((n + 63) // 64) * (1 + rank)
+    loss_us = 1e3 * float(ph[:, 1].mean()) / passes
+    pass_bytes = (8 + 4 * rank) * M_FULL / (1 + rank)  # mean algorithmic bytes per pass
+    achieved = pass_bytes / (loss_us * 1e-6) / 1e9
     ctx.close()
 
     # the study: the same problem at M = 2^20, both methods, a learning-rate sweep
@@ -838,17 +843,18 @@ def lowrank_arm(args):
         "config": {"workload": "low-rank-plus-diagonal quadratic, M=2^24 fp32, rank 4, "
                                f"n_pert={n}, 1.5-SPSA", "M": M_FULL, "n_pert": n,
                    "l2": "flushed between steps (256 MiB write, untimed)"},
-        "roofline": {"kernel": "quad_loss_kernel<pair, rank 4>", "bound": "hbm",
-                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+        "roofline": {"kernel": "quad_octet_kernel (diagonal and dot-product table passes, 64 "
+                               "probes each; issue-bound like the diagonal quadratic's pass)",
+                     "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_kind": peak_kind,
-                     "bytes_per_launch": 8 * M_FULL, "avg_launch_us": loss_us, "traffic": None},
+                     "bytes_per_launch": pass_bytes, "avg_launch_us": loss_us, "traffic": None},
         "phases_ms": {"clean_loss": float(ph[:, 0].mean()), "probe_losses": float(ph[:, 1].mean()),
                       "precond_update": float(ph[:, 2].mean())},
         "study": {"M": STUDY_M, "n_pert": STUDY_N, "steps": STUDY_STEPS, "eps": EPS,
                   "lr_unit": unit, "trace_H": trH,
                   "damping": DAMPING, "alpha": 0.1, "eigenvalues_over_trD": list(synth.LOWRANK_SCALES),
                   "final_over_initial_loss": rows, "largest_stable_lr": stable},
-        "gpu_launches": (1 + n + 2) * args.steps,
+        "gpu_launches": (passes + 3) * args.steps,  # passes, combination, precond, update
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

@@ -84,3 +84,27 @@ def test_lowrank_rejects_bad_rank(zo):
     with pytest.raises(ValueError):
         zo.zo_lowrank_loss(ctx, D, [1.0] * 5, 1, out)
     ctx.close()
+
+
+@pytest.mark.parametrize("M,rank,n", [((1 << 20) + 17, 4, 64), (50001, 1, 20), (4096 * 3 + 77, 3, 5),
+                                      (1 << 16, 2, 70)])
+def test_lowrank_step_losses_equal_one_probe_passes(zo, M, rank, n):
+    """zo_lowrank_step's losses (one table pass for the diagonal part and one per direction for
+    the dot products, per 64 probes) equal the one-probe low-rank passes to fp64 rounding, with
+    the clean loss, for 1..4 directions and every pass size."""
+    th_np, D_np, lam, vseed = synth.lowrank_problem(M, seed=M + n, rank=rank)
+    th, D = dev(th_np), dev(D_np)
+    ctx = zo.zo_create(th, seed=12)
+    zo.zo_set_step(ctx, 3)
+    ref = torch.zeros(2 * n + 1, dtype=torch.float64, device="cuda")
+    zo.zo_lowrank_loss(ctx, D, lam, vseed, ref[0:1])
+    for i in range(n):
+        zo.zo_lowrank_loss_pair(ctx, D, lam, vseed, i, 1e-3, ref[1 + i:2 + i],
+                                ref[1 + n + i:2 + n + i])
+    losses = torch.zeros(2 * n + 1, dtype=torch.float64, device="cuda")
+    zo.zo_lowrank_step(ctx, D, lam, vseed, n, 1e-3, 0.0, 1e-3, True, losses)  # lr 0: theta kept
+    assert zo.zo_sync(ctx) == 0
+    got, want = losses.cpu().numpy(), ref.cpu().numpy()
+    assert np.allclose(got, want, rtol=1e-12, atol=0), np.abs(got / want - 1).max()
+    assert np.array_equal(th.cpu().numpy(), th_np)  # lr = 0 leaves theta unchanged
+    ctx.close()

@@ -168,6 +168,7 @@ zo_status zo_destroy(zo_ctx *ctx) {
   cudaFree(ctx->staging);
   cudaFree(ctx->loss_scratch);
   cudaFree(ctx->mlp_ce);
+  cudaFree(ctx->lowrank_scratch);
   if (ctx->copy_stream) cudaStreamSynchronize(ctx->copy_stream);
   for (int b = 0; b < 2; ++b) {
     cudaFree(ctx->pipe_d[b]);
@@ -453,16 +454,41 @@ zo_status zo_lowrank_step(zo_ctx *ctx, const float *D, const zo_lowrank *q, int3
   ZO_CHECK(check_step_args(ctx, n_pert, lr, eps, damping));
   if (!losses_out) return fail(ctx, ZO_ERR_INVALID, "null losses_out");
   if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "step while perturbed");
+  float lam[4];
+  ZO_CHECK(check_lowrank(ctx, D, q, lam));
   double *L0 = losses_out, *Lp = losses_out + 1, *Lm = losses_out + 1 + n_pert;
-  phase_mark(ctx, 0);
-  if (preconditioned) {
-    ZO_CHECK(zo_lowrank_loss(ctx, D, q, L0, 0));
-  } else {
-    ZO_CUDA(ctx, cudaMemsetAsync(L0, 0, sizeof(double), ctx->stream), "clear L0");
+  // The loss of probe i is its diagonal part plus sum_r (lam_r / 2M) (v_r . P_i)^2: one
+  // table pass per 64 probes for the diagonal part and one per direction for its dot
+  // products (the clean values in the first pass), then their combination.
+  const size_t per = (size_t)(2 * n_pert + 1), need = per * (size_t)(q->rank + 1);
+  if (need > ctx->lowrank_cap) {
+    cudaFree(ctx->lowrank_scratch);
+    ctx->lowrank_scratch = nullptr;
+    ctx->lowrank_cap = 0;
+    ZO_CUDA(ctx, cudaMalloc(&ctx->lowrank_scratch, need * sizeof(double)), "low-rank scratch");
+    ctx->lowrank_cap = need;
   }
+  double *base = ctx->lowrank_scratch, *dots = base + per;
+  phase_mark(ctx, 0);
+  if (!preconditioned)
+    ZO_CUDA(ctx, cudaMemsetAsync(L0, 0, sizeof(double), ctx->stream), "clear L0");
   phase_mark(ctx, 1);
-  for (int32_t i = 0; i < n_pert; ++i)
-    ZO_CHECK(zo_lowrank_loss_pair(ctx, D, q, i, eps, Lp + i, Lm + i));
+  ProbeKey pk = probe_key(ctx);
+  pk.sign = +1;
+  pk.eps = eps;
+  for (int32_t i = 0; i < n_pert; i += 64) {
+    const int c = n_pert - i < 64 ? n_pert - i : 64;
+    const bool clean = preconditioned && i == 0;
+    ZO_CHECK(launch_quad_octet(ctx, pk, (uint32_t)(i / 8), c, D, base + 1 + i, base + 1 + n_pert + i,
+                               clean ? base : nullptr));
+    for (int r = 0; r < q->rank; ++r) {
+      double *dr = dots + per * r;
+      ZO_CHECK(launch_lowrank_dot_octet(ctx, pk, (uint32_t)(i / 8), c, r, q->vseed, dr + 1 + i,
+                                        dr + 1 + n_pert + i, clean ? dr : nullptr));
+    }
+  }
+  ZO_CHECK(launch_lowrank_combine(ctx, base, dots, q->rank, n_pert, lam, preconditioned ? 1 : 0,
+                                  losses_out));
   phase_mark(ctx, 2);
   const zo_status st = zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
   phase_mark(ctx, 3);

@@ -137,6 +137,10 @@ struct zo_ctx {
   cudaEvent_t pipe_copied[2] = {nullptr, nullptr}, pipe_consumed[2] = {nullptr, nullptr};
   uint64_t pipe_k = 0;
 
+  // per-probe sums of the batched low-rank step ((rank + 1) x (2 n + 1) doubles)
+  double *lowrank_scratch = nullptr;
+  size_t lowrank_cap = 0;
+
   // per-sample losses of the batched MLP evaluation ((2 n + 1) x batch doubles)
   double *mlp_ce = nullptr;
   size_t mlp_ce_cap = 0;
@@ -181,6 +185,11 @@ zo_status launch_quad_octet(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, int
 // directions from vseed); out_minus != null evaluates both signs of pk's probe in one pass.
 zo_status launch_lowrank_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, const float lam[4],
                               uint64_t vseed, double *out, double *out_minus, int accumulate);
+zo_status launch_lowrank_dot_octet(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, int count,
+                                   int dir, uint64_t vseed, double *out_plus, double *out_minus,
+                                   double *out_clean);
+zo_status launch_lowrank_combine(zo_ctx *ctx, const double *base, const double *dots, int rank,
+                                 int n, const float lam[4], int clean, double *out);
 zo_status launch_mlp_probes(zo_ctx *ctx, const float *X, const int32_t *y, int batch, int n_in,
                             int n_hidden, int n_out, int n_pert, float eps, double scale,
                             double *lp, double *lm, double *l0);

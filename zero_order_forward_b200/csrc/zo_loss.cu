@@ -14,8 +14,6 @@
 namespace zo {
 namespace {
 
-constexpr int kWarps = 8;
-
 __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xFFFFFFFFu, v, o);
@@ -175,11 +173,11 @@ __device__ __forceinline__ void quad_produce(const QuadPipe &p, const float *the
     const int64_t base = chunk * p.chunk;
     const int cnt = (int)(M - base < (int64_t)p.chunk ? M - base : (int64_t)p.chunk);
     const int copy = cnt & ~3;
-    if (lane == 0) {
-      tc::mbar_arrive_expect_tx(&p.full[s], 2u * (uint32_t)copy * 4u);
+    if (lane == 0) {  // D may be null (passes that read theta only)
+      tc::mbar_arrive_expect_tx(&p.full[s], (D ? 2u : 1u) * (uint32_t)copy * 4u);
       if (copy) {
         tc::bulk_load(st, theta + base, (uint32_t)copy * 4u, &p.full[s]);
-        tc::bulk_load(st + p.chunk * 4, D + base, (uint32_t)copy * 4u, &p.full[s]);
+        if (D) tc::bulk_load(st + p.chunk * 4, D + base, (uint32_t)copy * 4u, &p.full[s]);
       }
     }
     __syncwarp();
@@ -209,20 +207,25 @@ __device__ __forceinline__ bool quad_acquire(const QuadPipe &p, int s, uint32_t 
 }
 
 // The 4 theta and D values of vector e (0 past the end of the chunk: their terms are 0).
-template <int CHUNK = kQChunk>
+// WITH_D false: theta only (dv left 0).
+template <int CHUNK = kQChunk, bool WITH_D = true>
 __device__ __forceinline__ void quad_load4(const uint8_t *st, const float *theta, const float *D,
                                            int64_t base, int e, int cnt, float tv[4], float dv[4]) {
   if (e + 4 <= (cnt & ~3)) {
     const float4 t = reinterpret_cast<const float4 *>(st)[e >> 2];
-    const float4 dd = reinterpret_cast<const float4 *>(st + CHUNK * 4)[e >> 2];
     tv[0] = t.x; tv[1] = t.y; tv[2] = t.z; tv[3] = t.w;
-    dv[0] = dd.x; dv[1] = dd.y; dv[2] = dd.z; dv[3] = dd.w;
+    if (WITH_D) {
+      const float4 dd = reinterpret_cast<const float4 *>(st + CHUNK * 4)[e >> 2];
+      dv[0] = dd.x; dv[1] = dd.y; dv[2] = dd.z; dv[3] = dd.w;
+    } else {
+      dv[0] = dv[1] = dv[2] = dv[3] = 0.f;
+    }
   } else {  // the last < 4 elements of theta (not covered by the 16-byte copies)
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const bool in = e + q < cnt;
       tv[q] = in ? theta[base + e + q] : 0.f;
-      dv[q] = in ? D[base + e + q] : 0.f;
+      dv[q] = (WITH_D && in) ? D[base + e + q] : 0.f;
     }
   }
 }
@@ -231,23 +234,6 @@ __device__ __forceinline__ void quad_load4(const uint8_t *st, const float *theta
 __device__ __forceinline__ double quad_term(float d, float p) {
   const double pd = (double)p;
   return __dmul_rn(__dmul_rn(0.5, (double)d), __dmul_rn(pd, pd));
-}
-
-// Quad exchange: lane q of a quad holds block r; afterwards W[k] is word q of the block held
-// by lane k of the quad.
-__device__ __forceinline__ void quad_exchange(const uint4 &r, int lane, uint32_t W[4]) {
-  const int q = lane & 3;
-  uint32_t R[4];
-#pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    const uint32_t send = word_of(r, (q - t) & 3);
-    R[t] = __shfl_sync(0xFFFFFFFFu, send, (lane & ~3) | ((q + t) & 3));
-  }
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int t = (k - q) & 3;  // W[k] = R[(k - q) & 3]
-    W[k] = t == 0 ? R[0] : t == 1 ? R[1] : t == 2 ? R[2] : R[3];
-  }
 }
 
 // PAIR: both losses of one probe, L(theta + eps z) into out and L(theta - eps z) into
@@ -414,12 +400,19 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
 // lane-dependent order; block and grid totals in a fixed order (LPV lanes per value over a
 // fixed stride, then a butterfly).  Probes p >= count are computed and not stored.  CLEAN
 // also adds the clean loss L(theta) to the same pass (into *out_clean).
-template <bool CLEAN, int NOCT>
+//
+// DOT: instead of the quadratic's terms, the terms of the dot product v . P with direction
+// `dir` of the low-rank quadratic (v_j = -1 where bit dir of element j's byte of the
+// directions' block, key (vk0, vk1), octet 0, step 0, is set; else +1): t_a = v_j P_a,
+// t_b = v_j P_b and the clean term v_j theta_j, exact in fp64.  The same tables then give
+// v . P(theta + eps z_i) and v . P(theta - eps z_i) = sum_j v_j (P_a + P_b)_j - v . P+; D is
+// not read.
+template <bool CLEAN, int NOCT, bool DOT>
 __global__ void __launch_bounds__(kQThreads, kOBlocksPerSm)
 quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, int64_t M,
                   ProbeKey pk, uint32_t octet, int count, int64_t n_chunks, double *partials,
                   unsigned int *counter, double *out_plus, double *out_minus, double *out_clean,
-                  uint32_t *err) {
+                  uint32_t *err, int dir, uint32_t vk0, uint32_t vk1) {
   static_assert(NOCT == 2 || NOCT == 4 || NOCT == 8, "two, four or eight octets per pass");
   constexpr int G = NOCT == 8 ? 4 : 2;     // lanes sharing their tables (a pair or a quad)
   constexpr int LO = NOCT / G;             // octets per thread
@@ -491,7 +484,9 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
         // build a table
         const int e = 4 * (ct + k * 32 * kQConsumers);
         float tv[4], dv[4];
-        quad_load4<kOChunk>(st, theta, D, base, e, cnt, tv, dv);
+        quad_load4<kOChunk, !DOT>(st, theta, D, base, e, cnt, tv, dv);
+        uint32_t vw = 0u;  // DOT: the directions' bits of this vector's 4 elements
+        if constexpr (DOT) vw = word_of(sign_block(g0 + 64 * k, 0u, 0u, vk0, vk1), q);
         // wo / wp: the own / partner vector's word of each local octet j (pairs)
         uint32_t wo[LO], wp[LO];
         if constexpr (NOCT == 8) {
@@ -521,10 +516,20 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
         double ta[4], tb[4];
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) {
-          ta[qq] = quad_term(dv[qq], __fadd_rn(tv[qq], pk.eps));
-          tb[qq] = quad_term(dv[qq], __fadd_rn(tv[qq], -pk.eps));
+          if constexpr (DOT) {
+            // elements past the chunk's end contribute nothing
+            const bool in = e + qq < cnt, neg = (vw >> (8 * qq + dir)) & 1u;
+            const double pa = in ? (double)__fadd_rn(tv[qq], pk.eps) : 0.0;
+            const double pb = in ? (double)__fadd_rn(tv[qq], -pk.eps) : 0.0;
+            ta[qq] = neg ? -pa : pa;
+            tb[qq] = neg ? -pb : pb;
+            if (CLEAN) l0 = __dadd_rn(l0, neg ? -(double)tv[qq] : (double)tv[qq]);
+          } else {
+            ta[qq] = quad_term(dv[qq], __fadd_rn(tv[qq], pk.eps));
+            tb[qq] = quad_term(dv[qq], __fadd_rn(tv[qq], -pk.eps));
+            if (CLEAN) l0 = __dadd_rn(l0, quad_term(dv[qq], tv[qq]));
+          }
           tsum = __dadd_rn(tsum, __dadd_rn(ta[qq], tb[qq]));
-          if (CLEAN) l0 = __dadd_rn(l0, quad_term(dv[qq], tv[qq]));
         }
         // table entry n: element q takes t_b if bit q of n is set
         double lo[4], hi[4];
@@ -819,9 +824,10 @@ zo_status launch_quad_loss_pair(zo_ctx *ctx, const ProbeKey &pk, const float *D,
   return launch_quad<true, 0>(ctx, pk, D, out_plus, out_minus, 0, ctx->partials, ctx->counter);
 }
 
-template <bool CLEAN, int NOCT>
+template <bool CLEAN, int NOCT, bool DOT>
 zo_status launch_quad_octet_t(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, int count,
-                              const float *D, double *out_plus, double *out_minus, double *out_clean) {
+                              const float *D, double *out_plus, double *out_minus, double *out_clean,
+                              int dir, uint32_t vk0, uint32_t vk1) {
   const int64_t n_chunks = (ctx->M + kOChunk - 1) / kOChunk;
   const int64_t cap = (int64_t)kSmCount * kOBlocksPerSm;
   const int64_t blocks = n_chunks < cap ? n_chunks : cap;
@@ -829,7 +835,7 @@ zo_status launch_quad_octet_t(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, i
                 "partials too small for the octet pass");
   static bool attr = false;
   if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(quad_octet_kernel<CLEAN, NOCT>,
+    const cudaError_t e = cudaFuncSetAttribute(quad_octet_kernel<CLEAN, NOCT, DOT>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, kOSmemBytes);
     if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "quad_octet_kernel attribute: %s", cudaGetErrorString(e));
     attr = true;
@@ -844,24 +850,68 @@ zo_status launch_quad_octet_t(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, i
   attr_pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr_pdl;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, quad_octet_kernel<CLEAN, NOCT>,
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, quad_octet_kernel<CLEAN, NOCT, DOT>,
                                            static_cast<const float *>(ctx->params), D, ctx->M, pk,
                                            octet, count, n_chunks, ctx->partials, ctx->counter,
-                                           out_plus, out_minus, out_clean, &ctx->dstate->flags);
+                                           out_plus, out_minus, out_clean, &ctx->dstate->flags, dir, vk0,
+                                           vk1);
   if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "quad_octet_kernel: %s", cudaGetErrorString(e));
   return check_launch(ctx, "quad_octet_kernel");
 }
 
+// NOCT by count: 8 octets above 32 probes, 4 above 16, else 2.
+template <bool DOT>
+zo_status launch_octet_any(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, int count,
+                           const float *D, double *out_plus, double *out_minus, double *out_clean,
+                           int dir, uint32_t vk0, uint32_t vk1) {
+#define ZO_OCTET(C, N) launch_quad_octet_t<C, N, DOT>(ctx, pk, octet, count, D, out_plus, out_minus, \
+                                                     C ? out_clean : nullptr, dir, vk0, vk1)
+  if (count > 32) return out_clean ? ZO_OCTET(true, 8) : ZO_OCTET(false, 8);
+  if (count > 16) return out_clean ? ZO_OCTET(true, 4) : ZO_OCTET(false, 4);
+  return out_clean ? ZO_OCTET(true, 2) : ZO_OCTET(false, 2);
+#undef ZO_OCTET
+}
+
 zo_status launch_quad_octet(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, int count,
                             const float *D, double *out_plus, double *out_minus, double *out_clean) {
-  if (count > 32)
-    return out_clean ? launch_quad_octet_t<true, 8>(ctx, pk, octet, count, D, out_plus, out_minus, out_clean)
-                     : launch_quad_octet_t<false, 8>(ctx, pk, octet, count, D, out_plus, out_minus, nullptr);
-  if (count > 16)
-    return out_clean ? launch_quad_octet_t<true, 4>(ctx, pk, octet, count, D, out_plus, out_minus, out_clean)
-                     : launch_quad_octet_t<false, 4>(ctx, pk, octet, count, D, out_plus, out_minus, nullptr);
-  return out_clean ? launch_quad_octet_t<true, 2>(ctx, pk, octet, count, D, out_plus, out_minus, out_clean)
-                   : launch_quad_octet_t<false, 2>(ctx, pk, octet, count, D, out_plus, out_minus, nullptr);
+  return launch_octet_any<false>(ctx, pk, octet, count, D, out_plus, out_minus, out_clean, 0, 0u, 0u);
+}
+
+zo_status launch_lowrank_dot_octet(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, int count,
+                                   int dir, uint64_t vseed, double *out_plus, double *out_minus,
+                                   double *out_clean) {
+  return launch_octet_any<true>(ctx, pk, octet, count, nullptr, out_plus, out_minus, out_clean, dir,
+                                (uint32_t)vseed, (uint32_t)(vseed >> 32));
+}
+
+namespace {
+// out[i] = base[i] + sum_r (lam_r / 2 / M) dots[r][i]^2 for the 2n + 1 values of a low-rank
+// step ([L0, L+..., L-...]; i = 0 only with the clean loss), with the combination of the
+// one-probe low-rank pass.
+__global__ void lowrank_combine_kernel(const double *__restrict__ base, const double *__restrict__ dots,
+                                       int rank, int n, LowRankArgs lr, int64_t M, int clean,
+                                       double *__restrict__ out) {
+  const double inv_m = 1.0 / (double)M;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x + (clean ? 0 : 1); i < 2 * n + 1;
+       i += gridDim.x * blockDim.x) {
+    double L = base[i];
+    for (int r = 0; r < rank; ++r) {
+      const double t = dots[(int64_t)r * (2 * n + 1) + i];
+      L = __dadd_rn(L, __dmul_rn(__dmul_rn(0.5 * (double)lr.lam[r], inv_m), __dmul_rn(t, t)));
+    }
+    out[i] = L;
+  }
+}
+}  // namespace
+
+zo_status launch_lowrank_combine(zo_ctx *ctx, const double *base, const double *dots, int rank,
+                                 int n, const float lam[4], int clean, double *out) {
+  LowRankArgs lr;
+  for (int k = 0; k < 4; ++k) lr.lam[k] = lam[k];
+  lr.vk0 = lr.vk1 = 0u;
+  const int blocks = (2 * n + 1 + 255) / 256;
+  lowrank_combine_kernel<<<blocks, 256, 0, ctx->stream>>>(base, dots, rank, n, lr, ctx->M, clean, out);
+  return check_launch(ctx, "lowrank_combine_kernel");
 }
 
 zo_status launch_lowrank_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, const float lam[4],
