@@ -13,7 +13,7 @@ LIB_PATH = os.path.join(_HERE, "libzo.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        "libzo.so is not built; run `python -m zero_order_forward_b200.build` "
+        "libzo.so is not built; run `python zero_order_forward_b200/build.py` "
         "(nvcc, sm_100a) before using zero_order_forward_b200")
 
 _L = ctypes.CDLL(LIB_PATH)
