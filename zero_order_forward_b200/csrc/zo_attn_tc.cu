@@ -340,12 +340,9 @@ template <int HD>
 zo_status launch_tc(zo_ctx *ctx, const CUtensorMap &tmq, const CUtensorMap &tmkv, const TcAttnArgs &a,
                     int B) {
   using SM = TcAttnSmem<HD>;
-  static bool attr = false;
-  if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)SM::kBytes);
+  {
+    const cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(attn_tc_kernel<HD>), (int)SM::kBytes);
     if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "attn_tc_kernel attribute: %s", cudaGetErrorString(e));
-    attr = true;
   }
   const dim3 grid((a.S + kTBM - 1) / kTBM, a.H, B);
   attn_tc_kernel<HD><<<grid, kTThreads, SM::kBytes, ctx->stream>>>(tmq, tmkv, a);

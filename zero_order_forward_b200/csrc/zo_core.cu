@@ -13,6 +13,10 @@
 #include <cstring>
 #include <new>
 
+#include <mutex>
+#include <utility>
+#include <vector>
+
 #include "zo_internal.cuh"
 
 namespace zo {
@@ -46,6 +50,20 @@ ProbeKey probe_key(const zo_ctx *ctx) {
   pk.eps = ctx->eps;
   pk.g_off = (uint64_t)(ctx->first_element / kGroup);
   return pk;
+}
+
+cudaError_t ensure_smem_limit(const void *kernel, int bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<const void *, int>> done;  // (kernel, device)
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto &d : done)
+    if (d.first == kernel && d.second == dev) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.emplace_back(kernel, dev);
+  return e;
 }
 
 void phase_mark(zo_ctx *ctx, int which) {

@@ -360,11 +360,9 @@ cudaError_t launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const CUten
                        const GemmArgs &g, cudaStream_t st) {
   using S = GemmSmem<BN, STAGES>;
   auto kern = gemm_bf16_kernel<BN, STAGES, EPI>;
-  static bool attr_set = false;  // per instantiation; benign race (idempotent call)
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::kBytes);
+  {
+    const cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), (int)S::kBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   constexpr int OUT_BN = EPI == ZO_EPI_SWIGLU_BF16 ? BN / 2 : BN;
   const int num_m = (g.M + kBM - 1) / kBM, num_n = (g.N + OUT_BN - 1) / OUT_BN;

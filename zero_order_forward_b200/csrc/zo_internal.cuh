@@ -190,6 +190,10 @@ zo_status launch_lowrank_dot_octet(zo_ctx *ctx, const ProbeKey &pk, uint32_t oct
                                    double *out_clean);
 zo_status launch_lowrank_combine(zo_ctx *ctx, const double *base, const double *dots, int rank,
                                  int n, const float lam[4], int clean, double *out);
+// Raise a kernel's dynamic shared-memory limit to `bytes` on the current device, once per
+// (kernel, device): the attribute belongs to a device's context, so a process with contexts
+// on several devices sets it on each.
+cudaError_t ensure_smem_limit(const void *kernel, int bytes);
 zo_status launch_mlp_probes(zo_ctx *ctx, const float *X, const int32_t *y, int batch, int n_in,
                             int n_hidden, int n_out, int n_pert, float eps, double scale,
                             double *lp, double *lm, double *l0);

@@ -784,12 +784,9 @@ zo_status launch_quad(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *o
                       const LowRankArgs &lr = LowRankArgs{}) {
   const int64_t n_chunks = (ctx->M + kQChunk - 1) / kQChunk;
   int64_t blocks = n_chunks < (int64_t)kSmCount * 2 ? n_chunks : (int64_t)kSmCount * 2;
-  static bool attr = false;
-  if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(quad_loss_kernel<PAIR, R>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmemBytes);
+  {
+    const cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(quad_loss_kernel<PAIR, R>), kQSmemBytes);
     if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "quad_loss_kernel attribute: %s", cudaGetErrorString(e));
-    attr = true;
   }
   // Programmatic dependent launch: this pass may begin while the previous loss pass of
   // the stream finishes its reduction (see pdl_wait in the kernel).  Kernels that write
@@ -833,12 +830,10 @@ zo_status launch_quad_octet_t(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, i
   const int64_t blocks = n_chunks < cap ? n_chunks : cap;
   static_assert((8 * NOCT + 2) * kSmCount * kOBlocksPerSm <= kMaxPartials,
                 "partials too small for the octet pass");
-  static bool attr = false;
-  if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(quad_octet_kernel<CLEAN, NOCT, DOT>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kOSmemBytes);
+  {
+    const cudaError_t e =
+        ensure_smem_limit(reinterpret_cast<const void *>(quad_octet_kernel<CLEAN, NOCT, DOT>), kOSmemBytes);
     if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "quad_octet_kernel attribute: %s", cudaGetErrorString(e));
-    attr = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)blocks);
@@ -947,12 +942,10 @@ zo_status launch_mlp_probes(zo_ctx *ctx, const float *X, const int32_t *y, int b
   const int M = (int)ctx->M;
   const size_t smem = (size_t)(M + n_hidden) * sizeof(float) +
                       (size_t)((M + kGroup - 1) / kGroup) * sizeof(uint16_t);
-  static bool attr = false;
-  if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(mlp_probes_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)(kMlpStageMax * sizeof(float) + kMlpStageMax / 8));
+  {
+    const cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(mlp_probes_kernel),
+                                            (int)(kMlpStageMax * sizeof(float) + kMlpStageMax / 8));
     if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "mlp_probes_kernel attribute: %s", cudaGetErrorString(e));
-    attr = true;
   }
   ProbeKey pk = probe_key(ctx);
   pk.sign = +1;

@@ -267,12 +267,9 @@ __global__ void pack_kernel(uint8_t *__restrict__ out, int64_t first_byte, int64
 template <typename T>
 zo_status launch_pipe(zo_ctx *ctx, const ProbeKey &pk, int64_t first, int64_t count, void *out) {
   using SM = PipeSmem<T>;
-  static bool attr = false;
-  if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(perturb_pipe_kernel<T>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kBytes);
+  {
+    const cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(perturb_pipe_kernel<T>), SM::kBytes);
     if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "perturb_pipe_kernel attribute: %s", cudaGetErrorString(e));
-    attr = true;
   }
   const int64_t g0 = first / kGroup;
   const int64_t g1 = (first + count + kGroup - 1) / kGroup;
