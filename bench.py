@@ -125,6 +125,20 @@ def time_oracle(M_sample, n_steps, seed=0):
     return times
 
 
+def host_cpu():
+    """The host's CPU model and logical core count (for the CPU baselines' context)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"model": model, "logical_cores": os.cpu_count()}
+
+
 def host_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -184,7 +198,7 @@ def reference_arm(args):
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "M": M_FULL, "n_pert": N_PERT},
             "cpu_baseline": {"value": value, "unit": "steps/s", "cores": P, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "host": host_cpu()},
             "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -468,7 +482,8 @@ def gpu_arm(args):
             per = sum(times) / len(times)
             cpu = {"value": (M_sample / M_FULL) / per, "unit": "steps/s", "cores": 1,
                    "kind": "oracle",
-                   "sample": "2 oracle steps on the first 2^20 of 2^24 parameters; steps/s scaled by 1/16"}
+                   "sample": "2 oracle steps on the first 2^20 of 2^24 parameters; steps/s scaled by 1/16",
+                   "host": host_cpu()}
             import oracle.timing
             ac, P = oracle_all_cores(M_sample, 0, 1)
             cpu["all_cores"] = {
