@@ -77,3 +77,35 @@ def test_model_param_count_matches_both_layouts(zo):
                 dict(d_ffn=6145), dict(class_ids=(0, q["vocab"]))):
         with pytest.raises(zo.ZoError):
             zo.zo_model_param_count({**q, **bad})
+
+
+def test_header_is_plain_c_and_links_from_c(zo, tmp_path):
+    """include/zo.h compiles as pedantic C99; a C program linked against libzo.so calls the
+    host-only entry points (no device needed)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include <string.h>
+#include "zo.h"
+int main(void) {
+  zo_model_cfg c;
+  int64_t M = 0;
+  memset(&c, 0, sizeof c);
+  c.n_layers = 12; c.d_model = 768; c.n_heads = 12; c.d_ffn = 3072; c.vocab = 50272;
+  c.max_pos = 2048; c.class_ids[0] = 1000; c.class_ids[1] = 2000; c.family = ZO_FAMILY_OPT;
+  if (zo_model_param_count(&c, &M) != ZO_OK) return 1;
+  printf("%lld %s %s\n", (long long)M, zo_status_name(ZO_OK), zo_status_name(ZO_ERR_TIMEOUT));
+  return 0;
+}
+""")
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(zo.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L", libdir, "-lzo", "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    assert out == ["125239296", "ZO_OK", "ZO_ERR_TIMEOUT"]
