@@ -921,7 +921,15 @@ def mlp_arm(args):
         line["cpu_baseline"] = {"value": 1.0 / statistics.mean(ts), "unit": "steps/s", "cores": 1,
                                 "kind": "oracle",
                                 "sample": "4 full oracle steps of this workload after one untimed "
-                                          "step, one thread"}
+                                          "step, one thread", "host": host_cpu()}
+        # every host core running the same steps in its own single-threaded process
+        P = max(1, min(host_cores(), 32))
+        res = oracle_workers([("mlp", 4)] * P)
+        wall = max(r["t_end"] for r in res) - min(r["t_start"] for r in res)
+        line["cpu_baseline"]["all_cores"] = {
+            "value": sum(len(r["times"]) for r in res) / wall, "unit": "steps/s", "cores": P,
+            "sample": f"{P} concurrent single-threaded oracle processes, 4 timed steps each; "
+                      "total steps / the union of their timed phases"}
     ctx.close()
     print(json.dumps(line), flush=True)
     return 0

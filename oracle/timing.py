@@ -50,14 +50,16 @@ def mlp_steps(steps, n_pert=16, eps=1e-3, lr=1e-2, damping=1e-3):
     from . import mlp, step
     P = synth.mlp_params(0)
     teacher = synth.mlp_params(0, tag="teacher")
-    times = []
+    times, t_start = [], None
     for k in range(steps + 1):
         X, y = synth.mlp_batch(0, k, teacher)
+        if k == 1:
+            t_start = time.time()
         t0 = time.perf_counter()
         P, _ = step.spsa_step(P, lambda Q: mlp.loss(Q, X, y), n_pert, eps, lr, damping, 0, k)
         if k:
             times.append(time.perf_counter() - t0)
-    return {"times": times}
+    return {"times": times, "t_start": t_start, "t_end": time.time()}
 
 
 def element_rates(M_perturb, M_update, ns):
