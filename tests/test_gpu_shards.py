@@ -3,7 +3,6 @@ as one context on the whole vector: perturbed windows, packed probe bytes and up
 element by element (bit for bit), and the quadratic's losses are the sums of the slices'
 losses (fp64 rounding).  One device holds all slices here; across devices the same contexts
 run one per rank (zero_order_forward_b200.dist.element_parallel_step)."""
-import numpy as np
 import pytest
 import torch
 
