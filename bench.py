@@ -1,28 +1,27 @@
 #!/usr/bin/env python
-"""Benchmark of one 1.5-SPSA step of the diagonal-quadratic workload on B200.
+"""Benchmark of one 1.5-SPSA step on B200: by default the OPT-30B-shaped decoder.
 
-Workload (the default, one GPU): L = 1/2 sum_j D_j theta_j^2 with M = 2^24 fp32
-parameters, D_j log-uniform in [1e-3, 1e3], theta_0 ~ N(0, 1); n_pert = 64,
-eps = 1e-3, lr = 4e-7, damping = 1e-3, 1.5-SPSA.  One step = clean loss + 2*n_pert
-perturbed losses (the 128 losses of each eight probe octets from one pass over theta and D) +
-preconditioner + update, all through the C ABI of libzo.so.
+Default workload (one GPU): OPT-30B-shaped decoder (48 layers, d 7168, 56 heads, FFN 28672,
+vocabulary 50272, learned positions, pre-LN; 29.97 B bf16 parameters N(0, 0.02), trained in
+place), batch 8 x 2048 uniform tokens, 2-class last-token cross-entropy with Bernoulli(0.5)
+labels; n_pert = 16, eps = 1e-3, lr = 1e-6, damping = 1e-3.  One step = the clean forward +
+2 n_pert perturbed forwards (each layer's perturbed weights materialised into one layer
+window) + the preconditioner + the update of all 29.97 B parameters, through zo_model_step of
+libzo.so.  The same run measures the diagonal-quadratic workload (M = 2^24 fp32, n_pert = 64)
+as a sub-record.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload quadratic|mlp|opt-125m|opt-1.3b|opt-30b|qwen3-1.7b|qwen3-8b]
+                  [--workload opt-30b|opt-1.3b|opt-125m|qwen3-1.7b|qwen3-8b|quadratic|mlp|lowrank]
 
-The decoder workloads (OPT- or Qwen3-shaped, bf16 weights N(0, 0.02), uniform tokens,
-2-class last-token loss) time whole 1.5-SPSA steps through zo_model_step and add a
-per-GEMM-shape breakdown of the tcgen05 projections against the measured bf16 peak.
-
-Prints ONE JSON line (rank 0).  With N > 1 (torchrun, one rank per GPU) the ranks share
-one model ("scaling": "strong"): every rank holds a contiguous slice of theta and D (its
-element offset keeps the global probe signs), evaluates all 2*n_pert + 1 losses over its
-slice's terms, the partial losses are all-gathered over NCCL and summed in rank order (the
-same bits everywhere), and every rank runs the preconditioner and updates its slice; the
-step time is the max over ranks.  `--impl reference` times the CPU oracle on bounded
-samples of the same workload.
+Prints ONE JSON line (rank 0).  With N > 1 (torchrun, one rank per GPU) the decoder runs
+probe-parallel: every rank holds a full replica of theta (same seed), evaluates its share of
+the probes and of the clean batch, the losses are all-gathered over NCCL, and every rank
+applies the same update, so the replicas stay bit-identical ("scaling": "strong"; the step
+time is the max over ranks).  `--impl reference` times the CPU oracle on bounded samples of
+the same workload.
 """
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -36,41 +35,41 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "1.5-SPSA steps/s & probe fwd tokens/s; perturb/update HBM GB/s as % of peak"
+DEFAULT_WORKLOAD = "opt-30b"
 M_FULL = 1 << 24
 N_PERT, EPS, LR, DAMPING = 64, 1e-3, 4e-7, 1e-3
 WORKLOAD = ("diagonal quadratic L=1/2*sum D_j theta_j^2, M=2^24 fp32, D log-uniform [1e-3,1e3], "
             "theta0~N(0,1); 1.5-SPSA n_pert=64 eps=1e-3 lr=4e-7 damping=1e-3")
 FALLBACK_HBM_GBS = 6650.0
-
-# DRAM bytes (read + write) per launch of the octet loss kernel from the ncu capture
-# summarised in profiles/quad_octet_kernel.quadratic_M2p24.md, valid for the kernel sources
-# whose SHA-256 (of zo_loss.cu and zo_internal.cuh, concatenated) is recorded with it;
-# reported as null when a source has changed since the capture.
-LOSS_TRAFFIC = {"sources_sha256": "d1b68b988680111f9d369faf40a77a5e8e770b8100af06f1e229ee733b2a03b3",
-                "bytes": 139.3e6}
-LOSS_SOURCES = ("zo_loss.cu", "zo_internal.cuh")
-# Warp instructions one launch of the loss kernel executes (ncu smsp__inst_executed.sum, same
-# capture and validity rule as LOSS_TRAFFIC): the pass is bound by instruction issue, so its
-# roofline is the issue limit, 148 SMs x 4 warp-instructions per clock at the sampled clock.
-LOSS_WARP_INSTRUCTIONS = 90.41e6
 SM_COUNT, ISSUE_PER_SM_CLOCK = 148, 4
 
+# Counters of single ncu captures, reported beside the live timings.  Each record holds the
+# SHA-256 of the kernel's sources at the time of the capture and is reported (as taken from
+# that capture, not from this run) only while the sources still hash to it; otherwise null.
+#   quad_octet_kernel, M = 2^24: DRAM bytes (read + write) and warp instructions per launch.
+LOSS_TRAFFIC = {"sources": ("zo_loss.cu", "zo_internal.cuh"),
+                "sources_sha256": "d1b68b988680111f9d369faf40a77a5e8e770b8100af06f1e229ee733b2a03b3",
+                "bytes": 139.3e6, "warp_instructions": 90.41e6}
+#   gemm_bf16_kernel at the OPT-30B layer shapes (T = 16384): DRAM bytes per launch averaged
+#   over the four projections of one layer (filled in from a capture; None until then).
+GEMM_TRAFFIC = {"sources": ("zo_gemm.cu", "zo_tc.cuh"), "sources_sha256": None, "bytes": None}
 
-def loss_sources_sha256():
-    import hashlib
+
+def sources_sha256(names):
     h = hashlib.sha256()
-    for name in LOSS_SOURCES:
+    for name in names:
         with open(os.path.join(ROOT, "zero_order_forward_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 
 
-def loss_traffic():
+def captured(record, key):
+    """record[key] if the kernel's sources are unchanged since the capture, else None."""
     try:
-        h = loss_sources_sha256()
+        ok = record["sources_sha256"] is not None and sources_sha256(record["sources"]) == record["sources_sha256"]
     except OSError:
-        return None
-    return LOSS_TRAFFIC["bytes"] if h == LOSS_TRAFFIC["sources_sha256"] else None
+        ok = False
+    return record[key] if ok else None
 
 
 FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS_SUSTAINED = 1590.0, 1400.0
@@ -171,10 +170,67 @@ def oracle_all_cores(M_sample, warmup, steps, max_procs=32):
     res = oracle_workers([("steps", M_sample, 100 + i, N_PERT, EPS, LR, DAMPING, warmup, steps)
                           for i in range(P)])
     wall = max(r["t_end"] for r in res) - min(r["t_start"] for r in res)
+    oracle_all_cores.last_wall_s = wall
     return P * steps * (M_sample / M_FULL) / wall, P
 
 
+def quad_config(world):
+    """The `config` object of the quadratic line (the same for the GPU and the reference arm)."""
+    return {"workload": WORKLOAD, "M": M_FULL, "n_pert": N_PERT, "eps": EPS, "lr": LR,
+            "damping": DAMPING,
+            "parallelism": (f"element-parallel x{world}: theta and D sharded in contiguous slices, "
+                            f"partial losses all-gathered" if world > 1 else "1 GPU"),
+            "l2": "flushed between steps (256 MiB write, untimed); theta+D = 128 MiB"}
+
+
+def decoder_reference_arm(args):
+    """The oracle as it stands on the machine's host cores (numpy's BLAS threads), on the decoder
+    workload's config: each of the W + K steps is a bounded sample, the oracle's fp64 forward of
+    one layer at the real width on one 64-token sequence (vocabulary cut to 4096, which only
+    feeds the embedding gather and the 2-row head); the full step's time is extrapolated
+    linearly in layers and tokens and labelled as such."""
+    import oracle
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    name = args.workload
+    cfg = decoder_cfg(name)
+    w = decoder_workload(name, args.n_pert)
+    B, S, k, n = w["batch"], w["seq"], w["n_micro"], w["n_pert"]
+    qwen = cfg.get("family") == "qwen3"
+    M = (oracle.qwen if qwen else oracle.opt).param_count(cfg)
+    red = dict(cfg, n_layers=1, vocab=4096)
+    seq = 64
+    P = host_cores()
+    res = oracle_workers([("forward_samples", "qwen3" if qwen else "opt", json.dumps(red), seq,
+                           args.warmup, args.steps)], threads=P)[0]
+    sample_s = statistics.mean(res["times"])
+    fwds = (2 * n + 1) * k
+    step_s = fwds * B * S * cfg["n_layers"] * sample_s / seq  # extrapolated full step
+    value = 1.0 / step_s
+    sample = (f"each step: the oracle's fp64 forward of 1 layer at the real width on 1 x {seq} "
+              f"tokens (vocabulary cut to 4096), {P} BLAS threads, {sample_s:.3f} s per sample; "
+              f"the full step ({fwds} forwards of {B * S} tokens x {cfg['n_layers']} layers) "
+              f"extrapolated linearly in layers and tokens (attention's quadratic term at the full "
+              f"length not included)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * step_s, "extrapolated": True,
+            "timed_region_s": sum(res["times"]), "sample_ms_per_step": 1e3 * sample_s,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": decoder_config(name, w, M, world),
+            "tokens_per_s": fwds * B * S / step_s,
+            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": P, "kind": "oracle",
+                             "extrapolated": True, "sample": sample, "host": host_cpu()},
+            "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def reference_arm(args):
+    if args.workload in DECODER_WORKLOADS:
+        return decoder_reference_arm(args)
     rank, _, world = dist_env()
     if rank != 0:
         return 0
@@ -194,9 +250,11 @@ def reference_arm(args):
               f"sample steps / wall time, scaled by 1/{M_FULL // M_sample}")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1e3 / value, "higher_is_better": True, "scaling": "strong",
+            "ms_per_step": 1e3 / value, "extrapolated": True,
+            "timed_region_s": oracle_all_cores.last_wall_s,
+            "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "M": M_FULL, "n_pert": N_PERT},
+            "config": quad_config(world),
             "cpu_baseline": {"value": value, "unit": "steps/s", "cores": P, "kind": "oracle",
                              "sample": sample, "host": host_cpu()},
             "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
@@ -272,7 +330,9 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ GPU arm
 
-def gpu_arm(args):
+def gpu_arm(args, sub=False):
+    """The diagonal-quadratic workload; returns rank 0's JSON line (None elsewhere).  sub=True
+    (the sub-record of the decoder line) leaves out the CPU baseline."""
     import torch
     import torch.distributed as dist
 
@@ -394,57 +454,55 @@ def gpu_arm(args):
     torch.cuda.synchronize()
     pair_us = 1e3 * pe[0].elapsed_time(pe[1]) / n
 
+    def timed_reps(fn, reps):
+        """Mean CUDA-event duration (us) of fn() over reps launches, L2 flushed before each
+        (the flush is outside the timed events)."""
+        tot = 0.0
+        for _ in range(reps):
+            flush.zero_()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            ev[0].record(stream)
+            fn()
+            ev[1].record(stream)
+            torch.cuda.synchronize()
+            tot += ev[0].elapsed_time(ev[1])
+        return 1e3 * tot / reps
+
     # single-kernel timing of the update (same stream), for its own roofline
     coef = torch.from_numpy(synth.coefficients(n, seed=1) * 0).to(dev)  # zero: theta unchanged
-    ue = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    flush.zero_()
-    ue[0].record(stream)
-    reps = 10
-    for _ in range(reps):
-        zo.zo_update(ctx, coef, n)
-    ue[1].record(stream)
-    torch.cuda.synchronize()
-    upd_us = 1e3 * ue[0].elapsed_time(ue[1]) / reps
+    upd_us = timed_reps(lambda: zo.zo_update(ctx, coef, n), 10)
 
-    # the streaming kernels across probe counts and dtypes (theta 128 MiB, larger than L2):
-    # the update's and the unpack/apply kernel's bandwidth against the measured HBM peak
+    # the streaming kernels across probe counts and dtypes (theta of 2^28 elements, 1 GiB fp32 /
+    # 512 MiB bf16, far larger than L2, and L2 flushed before every timed launch): the update's
+    # and the unpack/apply kernel's bandwidth against the measured HBM peak, and for the update
+    # the lane-instruction budget that bandwidth leaves per element
     streaming = {}
     if world == 1:
-        for dt, elems, esz in (("f32", 1 << 25, 4), ("bf16", 1 << 26, 2)):
+        elems = 1 << 28
+        for dt, esz in (("f32", 4), ("bf16", 2)):
             g = torch.Generator(device=dev)
             g.manual_seed(5)
-            th_s = (torch.randn(elems, device=dev, generator=g)
-                    .to(torch.float32 if dt == "f32" else torch.bfloat16))
+            th_s = torch.empty(elems, dtype=torch.float32 if dt == "f32" else torch.bfloat16, device=dev)
+            th_s.normal_(generator=g)
             out_s = torch.empty_like(th_s)
             cs = zo.zo_create(th_s, seed=7, stream=stream.cuda_stream)
-            ent = {"elements": elems, "update": {}}
+            ent = {"elements": elems, "l2": "flushed before every timed launch", "update": {}}
             for nn in (1, 2, 4, 8, 16, 32, 64, 160):
                 cz = torch.zeros(nn, dtype=torch.float32, device=dev)  # theta unchanged
                 zo.zo_update(cs, cz, nn)
-                ue2 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-                ue2[0].record(stream)
-                for _ in range(5):
-                    zo.zo_update(cs, cz, nn)
-                ue2[1].record(stream)
-                torch.cuda.synchronize()
-                us = 1e3 * ue2[0].elapsed_time(ue2[1]) / 5
+                us = timed_reps(lambda: zo.zo_update(cs, cz, nn), 5)
                 gbs = 2 * esz * elems / (us * 1e-6) / 1e9
                 ent["update"][str(nn)] = {"us": us, "GBps": gbs, "frac_hbm": gbs / hbm_peak}
             zo.zo_perturb(cs, +1, EPS, 3)
             zo.zo_perturb_range(cs, 0, elems, out_s)
-            pe2 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-            pe2[0].record(stream)
-            for _ in range(5):
-                zo.zo_perturb_range(cs, 0, elems, out_s)
-            pe2[1].record(stream)
-            torch.cuda.synchronize()
+            us = timed_reps(lambda: zo.zo_perturb_range(cs, 0, elems, out_s), 5)
             zo.zo_restore(cs)
-            us = 1e3 * pe2[0].elapsed_time(pe2[1]) / 5
             gbs = 2 * esz * elems / (us * 1e-6) / 1e9
             ent["perturb"] = {"us": us, "GBps": gbs, "frac_hbm": gbs / hbm_peak}
             cs.close()
             streaming[dt] = ent
             del th_s, out_s
+        torch.cuda.empty_cache()
 
     # end to end through the public API with host buffers: D copied in, losses copied out
     D_host = torch.from_numpy(D_np[first:first + count]).pin_memory()
@@ -476,7 +534,7 @@ def gpu_arm(args):
     line = None
     if rank == 0:
         cpu = None
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and not sub:
             M_sample = 1 << 20
             times = time_oracle(M_sample, 2)
             per = sum(times) / len(times)
@@ -504,12 +562,7 @@ def gpu_arm(args):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
             "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "M": M_FULL, "n_pert": n, "eps": EPS, "lr": LR,
-                       "damping": DAMPING,
-                       "parallelism": (f"element-parallel x{world}: theta and D sharded in "
-                                       f"contiguous slices, partial losses all-gathered"
-                                       if world > 1 else "1 GPU"),
-                       "l2": "flushed between steps (256 MiB write, untimed); theta+D = 128 MiB"},
+            "config": quad_config(world),
             "roofline": {"kernel": "quad_octet_kernel (the 128 losses L(theta +- eps z_i) of "
                                    "eight probe octets in one pass, perturbation on load, fp64 "
                                    "accumulation)",
@@ -542,32 +595,74 @@ def gpu_arm(args):
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
         }
-        line["roofline"]["traffic"] = args.traffic if args.traffic is not None else loss_traffic()
-        if loss_traffic() is not None:  # the recorded instruction count is valid: issue roofline
+        # The pass reads theta and D once (8 B per element): its roofline is HBM, against the
+        # algorithmic bytes.  It is bound by instruction issue in practice, so the issue-rate
+        # view is kept beside it, from the instruction count of the recorded capture.
+        line["roofline"]["traffic"] = (args.traffic if args.traffic is not None
+                                       else captured(LOSS_TRAFFIC, "bytes"))
+        line["roofline"]["traffic_from"] = ("--traffic" if args.traffic is not None else
+                                            "ncu capture of this kernel's current sources (not this run)"
+                                            if line["roofline"]["traffic"] is not None else None)
+        inst = captured(LOSS_TRAFFIC, "warp_instructions")
+        if inst is not None:
             mhz = (clocks or {}).get("sm_mhz") or 1965.0
             peak_inst = SM_COUNT * ISSUE_PER_SM_CLOCK * mhz * 1e6 / 1e9  # G warp-instr/s
-            ach_inst = LOSS_WARP_INSTRUCTIONS / (loss_us * 1e-6) / 1e9
-            hbm_view = {k: line["roofline"][k] for k in ("achieved", "peak", "unit", "frac")}
-            line["roofline"].update({
-                "bound": "alu", "achieved": ach_inst, "peak": peak_inst,
-                "unit": "G warp-instructions/s", "frac": ach_inst / peak_inst,
+            ach_inst = inst / (loss_us * 1e-6) / 1e9
+            line["roofline"]["issue_view"] = {
+                "achieved": ach_inst, "peak": peak_inst, "unit": "G warp-instructions/s",
+                "frac": ach_inst / peak_inst,
                 "peak_kind": f"issue limit: {SM_COUNT} SMs x {ISSUE_PER_SM_CLOCK} per clock at "
-                             f"{mhz:.0f} MHz",
-                "warp_instructions_per_launch": LOSS_WARP_INSTRUCTIONS, "hbm_view": hbm_view})
+                             f"{mhz:.0f} MHz (the sampled median)",
+                "warp_instructions_per_launch": inst,
+                "instructions_from": "ncu capture of this kernel's current sources (not this run)"}
     ctx.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
-    if line is not None:
-        print(json.dumps(line), flush=True)
-    return 0
+    del theta, D, flush
+    torch.cuda.empty_cache()
+    return line
 
 
 # ------------------------------------------------------------------ decoder workloads
 
+DEC_EPS, DEC_LR, DEC_DAMPING = 1e-3, 1e-6, 1e-3
+MEMORY_TARGET_GB = 80.0
+
+
 def decoder_cfg(name):
     import synth
     return synth.QWEN_CONFIGS[name] if name.startswith("qwen") else synth.OPT_CONFIGS[name]
+
+
+def decoder_workload(name, n_pert=None):
+    w = dict(DECODER_WORKLOADS[name])
+    if n_pert:
+        w["n_pert"] = n_pert
+    return w
+
+
+def decoder_config(name, w, M, world):
+    """The `config` object of a decoder line (the same for the GPU and the reference arm)."""
+    cfg = decoder_cfg(name)
+    B, S, k, n = w["batch"], w["seq"], w["n_micro"], w["n_pert"]
+    fam = "Qwen3" if cfg.get("family") == "qwen3" else "OPT"
+    heads = (f"{cfg['n_heads']} query / {cfg['n_kv_heads']} key-value heads of {cfg['head_dim']}"
+             if fam == "Qwen3" else f"{cfg['n_heads']} heads")
+    return {
+        "workload": (f"{name}-shaped {fam} decoder ({cfg['n_layers']} layers, d={cfg['d_model']}, "
+                     f"{heads}, FFN {cfg['d_ffn']}, vocab {cfg['vocab']}; {M} bf16 params "
+                     f"N(0,0.02)), micro-batch {B}x{S} uniform tokens x {k}, 2-class last-token "
+                     f"CE; 1.5-SPSA n_pert={n}, eps={DEC_EPS:g}, lr={DEC_LR:g}, "
+                     f"damping={DEC_DAMPING:g}, trained in place"),
+        "params": M, "batch": B, "seq": S, "n_micro": k, "n_pert": n, "eps": DEC_EPS,
+        "lr": DEC_LR, "damping": DEC_DAMPING,
+        "parallelism": (f"probe-parallel x{world}: full theta replica per GPU, probes and the clean "
+                        f"batch split across ranks, losses all-gathered (NCCL)" if world > 1
+                        else "1 GPU"),
+        "l2": "inputs larger than L2: every forward streams all the weights (and the perturbed "
+              "layer windows) from HBM",
+    }
 
 
 def init_decoder_params(theta, cfg, seed):
@@ -593,11 +688,47 @@ def init_decoder_params(theta, cfg, seed):
         o += n
 
 
-def decoder_arm(args):
-    import torch
+def add_kernel_times(tot, kt):
+    for c, v in kt.items():
+        for key in ("ms", "launches", "work"):
+            tot[c][key] += v[key]
 
-    import synth
+
+def kernel_summary(tot, hbm_peak, bf16_burst, bf16_sustained):
+    """Per kernel class of the timed region: launches, mean launch duration, achieved rate
+    from the algorithmic work, and its fraction of the measured peak."""
+    out = {}
+    for c, v in tot.items():
+        if not v["launches"]:
+            continue
+        sec = v["ms"] * 1e-3
+        e = {"launches": v["launches"], "total_ms": v["ms"], "avg_launch_us": 1e3 * v["ms"] / v["launches"],
+             "share_of_kernel_time": None}
+        if c in ("gemm", "attention"):
+            tf = v["work"] / sec / 1e12
+            e.update({"flops_per_launch": v["work"] / v["launches"], "tflops": tf,
+                      "frac_bf16_sustained": tf / bf16_sustained, "frac_bf16_burst": tf / bf16_burst})
+        else:
+            gb = v["work"] / sec / 1e9
+            e.update({"bytes_per_launch": v["work"] / v["launches"], "GBps": gb,
+                      "frac_hbm": gb / hbm_peak})
+        out[c] = e
+    total = sum(v["ms"] for v in tot.values())
+    for c in out:
+        out[c]["share_of_kernel_time"] = tot[c]["ms"] / total if total else None
+    return out
+
+
+def decoder_arm(args):
+    """Whole 1.5-SPSA steps of a decoder workload through zo_model_step (one GPU) or the
+    probe-parallel driver (N ranks); prints rank 0's JSON line."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
     import zero_order_forward_b200 as zo
+    from zero_order_forward_b200 import dist as zdist
 
     rank, local_rank, world = dist_env()
     torch.cuda.set_device(local_rank)
@@ -605,155 +736,288 @@ def decoder_arm(args):
     name = args.workload
     cfg = decoder_cfg(name)
     qwen = cfg.get("family") == "qwen3"
-    w = dict(DECODER_WORKLOADS[name])
-    if args.n_pert:
-        w["n_pert"] = args.n_pert
+    w = decoder_workload(name, args.n_pert)
     B, S, k, n = w["batch"], w["seq"], w["n_micro"], w["n_pert"]
+    hbm_peak, hbm_kind = peaks()
+    peak_b, peak_s, bf16_kind = bf16_peaks()
+
+    # the diagonal-quadratic workload, measured first in the same run (its memory is freed
+    # before the decoder's weights are allocated)
+    quad = None
+    if world == 1 and name == DEFAULT_WORKLOAD and not args.no_quadratic:
+        quad = gpu_arm(args, sub=True)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=900),
+                                device_id=dev)
+
     M = zo.zo_model_param_count(cfg)
     theta = torch.empty(M, dtype=torch.bfloat16, device=dev)
-    init_decoder_params(theta, cfg, seed=rank)
+    init_decoder_params(theta, cfg, seed=0)  # the same weights on every rank: replicas
     stream = torch.cuda.current_stream(dev)
-    ctx = zo.zo_create(theta, seed=rank, stream=stream.cuda_stream)
+    ctx = zo.zo_create(theta, seed=0, stream=stream.cuda_stream)
     model = zo.zo_model_create(ctx, cfg, B * S)
     gen = torch.Generator(device=dev)
-    gen.manual_seed(1000 + rank)
+    gen.manual_seed(1000)
     tokens = torch.randint(0, cfg["vocab"], (k, B, S), dtype=torch.int32, device=dev, generator=gen)
     labels = torch.randint(0, 2, (k, B), dtype=torch.int32, device=dev, generator=gen)
     losses = torch.zeros(2 * n + 1, dtype=torch.float64, device=dev)
-    eps, lr, lam = 1e-3, 1e-6, 1e-3
+    eps, lr, lam = DEC_EPS, DEC_LR, DEC_DAMPING
+    scale = 1.0 / (k * B)
 
-    def step():
-        zo.zo_model_step(model, tokens, labels, B, S, k, n, eps, lr, lam, True, losses)
+    if world == 1:
+        def step():
+            zo.zo_model_step(model, tokens, labels, B, S, k, n, eps, lr, lam, True, losses)
+    else:
+        b0, nb = zdist.batch_share(B, rank, world)
+
+        def loss_at(sign, probe, out):
+            zo.zo_perturb(ctx, sign, eps, probe)
+            for j in range(k):
+                zo.zo_model_loss(model, tokens[j], labels[j], B, S, scale, out, j > 0)
+            zo.zo_restore(ctx)
+
+        def clean(out):  # this rank's share of the clean batch
+            if nb == 0:
+                out.zero_()
+            for j in range(k if nb else 0):
+                zo.zo_model_loss(model, tokens[j, b0:b0 + nb], labels[j, b0:b0 + nb], nb, S,
+                                 scale, out, j > 0)
+
+        def apply_step(Lp, Lm, L0):
+            zo.zo_step(ctx, Lp, Lm, n, L0, lr, eps, lam)
+
+        def step():
+            L0, Lp, Lm = zdist.probe_parallel_step(n, loss_at, clean, apply_step, dev,
+                                                   clean_shared=True)
+            losses[0:1].copy_(L0)
+            losses[1:1 + n].copy_(Lp)
+            losses[1 + n:].copy_(Lm)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    zo.zo_sync(ctx)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    # timed region: K steps; every launch of the GEMM, attention, window-perturbation and
+    # update kernels is bracketed by CUDA events on the context's stream (drained after each
+    # step, which synchronises between steps)
+    tot = {c: {"ms": 0.0, "launches": 0, "work": 0.0} for c in zo.KERNEL_CLASSES}
+    dropped = 0
+    zo.zo_enable_kernel_timing(ctx, True)
+    zo.zo_kernel_times(ctx)
+    if world == 1:
+        zo.zo_enable_phase_timing(ctx, args.steps)
+    launches0 = zo.zo_launch_count(ctx)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    zo.zo_enable_phase_timing(ctx, args.steps)
     sampler = ClockSampler(local_rank) if rank == 0 else None
     ev[0].record(stream)
     for i in range(args.steps):
         step()
         ev[i + 1].record(stream)
+        kt, dr = zo.zo_kernel_times(ctx)
+        add_kernel_times(tot, kt)
+        dropped += dr
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
+    launches = zo.zo_launch_count(ctx) - launches0
+    zo.zo_enable_kernel_timing(ctx, False)
     zo.zo_sync(ctx)
-    phases = zo.zo_phase_times(ctx, args.steps)
-    zo.zo_enable_phase_timing(ctx, 0)
+    step_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
     total_s = ev[0].elapsed_time(ev[-1]) / 1e3
-    upd_ms = float(phases[:, 2].mean())  # preconditioner (one CTA, ~5 us) + update
-    upd_bytes = 2 * 2 * M  # bf16 theta read + written once
-    peak_mem = torch.cuda.max_memory_allocated(dev)
+    phases = None
+    if world == 1:
+        ph = zo.zo_phase_times(ctx, args.steps)
+        zo.zo_enable_phase_timing(ctx, 0)
+        phases = {"clean_loss": float(ph[:, 0].mean()), "probe_losses": float(ph[:, 1].mean()),
+                  "precond_update": float(ph[:, 2].mean())}
+    if world > 1:
+        t = torch.tensor([total_s, float(launches)], dtype=torch.float64, device=dev)
+        mx = t.clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        sm = t.clone()
+        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+        total_s, launches = float(mx[0].item()), int(sm[1].item())
     free_b, tot_b = torch.cuda.mem_get_info(dev)
-
-    # one clean forward, and each projection GEMM at this micro-batch's shape
-    T, d, f = B * S, cfg["d_model"], cfg["d_ffn"]
-    fe = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    fe[0].record(stream)
-    zo.zo_model_loss(model, tokens[0], labels[0], B, S, 1.0 / B, losses[0:1])
-    fe[1].record(stream)
-    torch.cuda.synchronize()
-    fwd_ms = fe[0].elapsed_time(fe[1])
-    peak_b, peak_s, peak_kind = bf16_peaks()
-    H = cfg["n_heads"]
-    Hk, e = (cfg["n_kv_heads"], cfg["head_dim"]) if qwen else (H, d // H)
-    nq, na = (H + 2 * Hk) * e, H * e
-    if qwen:  # no biases; SwiGLU's gate and up projections are one GEMM of width 2f
-        shapes = {"qkv": (T, nq, d, 0), "out": (T, d, na, 2), "gate_up": (T, 2 * f, d, 0),
-                  "down": (T, d, f, 2)}
-    else:
-        shapes = {"qkv": (T, nq, d, 0), "out": (T, d, na, 2), "fc1": (T, f, d, 1),
-                  "fc2": (T, d, f, 2)}
-    gemm = {}
-    A = torch.randn(T * max(K for _, _, K, _ in shapes.values()), dtype=torch.bfloat16, device=dev)
-    Wt = torch.randn(max(N * K for _, N, K, _ in shapes.values()), dtype=torch.bfloat16,
-                     device=dev) * 0.02
-    max_n = max(N for _, N, _, _ in shapes.values())
-    bias = None if qwen else torch.zeros(max_n, dtype=torch.bfloat16, device=dev)
-    out_b = torch.empty(T * max_n, dtype=torch.bfloat16, device=dev)
-    out_f = torch.zeros(T * d, dtype=torch.float32, device=dev)
-    flops_layer = 0
-    for key, (Mm, N, K, epi) in shapes.items():
-        out = out_f if epi == 2 else out_b
-        for _ in range(2):
-            zo.zo_gemm_bf16(ctx, A, Wt, bias, out, Mm, N, K, N, epi)
-        reps = 5
-        ge = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        ge[0].record(stream)
-        for _ in range(reps):
-            zo.zo_gemm_bf16(ctx, A, Wt, bias, out, Mm, N, K, N, epi)
-        ge[1].record(stream)
-        torch.cuda.synchronize()
-        us = 1e3 * ge[0].elapsed_time(ge[1]) / reps
-        fl = 2.0 * Mm * N * K
-        flops_layer += fl
-        gemm[key] = {"shape": [Mm, N, K], "avg_launch_us": us, "tflops": fl / us / 1e6,
-                     "frac_burst": fl / us / 1e6 / peak_b}
-    # causal attention at this micro-batch's shape (mma.sync path)
-    qkv = torch.randn(T * nq, dtype=torch.bfloat16, device=dev)
-    att = torch.empty(T * na, dtype=torch.bfloat16, device=dev)
-    for _ in range(2):
-        zo.zo_attention_gqa(ctx, qkv, att, B, S, H, Hk, e)
-    ae = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    ae[0].record(stream)
-    for _ in range(5):
-        zo.zo_attention_gqa(ctx, qkv, att, B, S, H, Hk, e)
-    ae[1].record(stream)
-    torch.cuda.synchronize()
-    attn_us = 1e3 * ae[0].elapsed_time(ae[1]) / 5
-    attn_flops = 2.0 * B * H * S * S * e  # causal half of 4 B H S^2 e
-    zo.zo_sync(ctx)
-    gemm_us = sum(g["avg_launch_us"] for g in gemm.values())
-    gemm_tflops = flops_layer / gemm_us / 1e6
-    fwds = (2 * n + 1) * k
-    tokens_per_step = fwds * T
+    used_gb = (tot_b - free_b) / 1e9
+    peak_alloc_gb = torch.cuda.max_memory_allocated(dev) / 1e9
     value = args.steps / total_s
+    fwds = (2 * n + 1) * k
+    T = B * S
+    kernels = kernel_summary(tot, hbm_peak, peak_b, peak_s)
+
+    # each projection GEMM and attention alone at this micro-batch's shape (one GPU)
+    gemm_shapes, attn_alone = {}, None
+    if world == 1:
+        d, f = cfg["d_model"], cfg["d_ffn"]
+        H = cfg["n_heads"]
+        Hk, e = (cfg["n_kv_heads"], cfg["head_dim"]) if qwen else (H, d // H)
+        nq, na = (H + 2 * Hk) * e, H * e
+        if qwen:  # no biases; SwiGLU's gate and up projections are one GEMM of width 2f
+            shapes = {"qkv": (T, nq, d, 0), "out": (T, d, na, 2), "gate_up": (T, f, d, 3),
+                      "down": (T, d, f, 2)}
+        else:
+            shapes = {"qkv": (T, nq, d, 0), "out": (T, d, na, 2), "fc1": (T, f, d, 1),
+                      "fc2": (T, d, f, 2)}
+        A = torch.randn(T * max(K for _, _, K, _ in shapes.values()), dtype=torch.bfloat16, device=dev)
+        Wt = torch.randn(max((2 if epi == 3 else 1) * N * K for _, N, K, epi in shapes.values()),
+                         dtype=torch.bfloat16, device=dev) * 0.02
+        max_n = max(N for _, N, _, _ in shapes.values())
+        bias = None if qwen else torch.zeros(max_n, dtype=torch.bfloat16, device=dev)
+        out_b = torch.empty(T * max_n, dtype=torch.bfloat16, device=dev)
+        out_f = torch.zeros(T * d, dtype=torch.float32, device=dev)
+        for key, (Mm, N, K, epi) in shapes.items():
+            out = out_f if epi == 2 else out_b
+            bb = None if epi == 3 else bias
+            for _ in range(2):
+                zo.zo_gemm_bf16(ctx, A, Wt, bb, out, Mm, N, K, N, epi)
+            ge = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            ge[0].record(stream)
+            for _ in range(5):
+                zo.zo_gemm_bf16(ctx, A, Wt, bb, out, Mm, N, K, N, epi)
+            ge[1].record(stream)
+            torch.cuda.synchronize()
+            us = 1e3 * ge[0].elapsed_time(ge[1]) / 5
+            fl = 2.0 * Mm * N * K * (2 if epi == 3 else 1)
+            gemm_shapes[key] = {"shape": [Mm, N, K], "avg_launch_us": us, "tflops": fl / us / 1e6,
+                                "frac_bf16_burst": fl / us / 1e6 / peak_b}
+        del A, Wt, out_b, out_f
+        qkv = torch.randn(T * nq, dtype=torch.bfloat16, device=dev)
+        att = torch.empty(T * na, dtype=torch.bfloat16, device=dev)
+        for _ in range(2):
+            zo.zo_attention_gqa(ctx, qkv, att, B, S, H, Hk, e)
+        ae = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ae[0].record(stream)
+        for _ in range(5):
+            zo.zo_attention_gqa(ctx, qkv, att, B, S, H, Hk, e)
+        ae[1].record(stream)
+        torch.cuda.synchronize()
+        attn_us = 1e3 * ae[0].elapsed_time(ae[1]) / 5
+        attn_flops = 4.0 * e * B * H * S * (S + 1) / 2
+        attn_alone = {"avg_launch_us": attn_us, "tflops": attn_flops / attn_us / 1e6,
+                      "frac_bf16_burst": attn_flops / attn_us / 1e6 / peak_b}
+        del qkv, att
+        zo.zo_sync(ctx)
+
+    # end to end through the C ABI with host buffers: every step copies its tokens and labels
+    # from pinned host memory to the device and reads the 2n + 1 losses back to the host
+    e2e_steps = max(1, min(args.steps, 2))
+    tok_host = tokens.cpu().pin_memory()
+    lab_host = labels.cpu().pin_memory()
+    L_host = torch.zeros(2 * n + 1, dtype=torch.float64).pin_memory()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        if world == 1:
+            zo.zo_model_step_host(model, tok_host, lab_host, B, S, k, n, eps, lr, lam, True, L_host)
+        else:
+            tokens.copy_(tok_host, non_blocking=True)
+            labels.copy_(lab_host, non_blocking=True)
+            step()
+            L_host.copy_(losses)  # synchronous device -> host read
+    torch.cuda.synchronize()
+    e2e_s = time.perf_counter() - t0
+    if world > 1:
+        t = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_s = float(t.item())
+    zo.zo_sync(ctx)
+    e2e = {"value": e2e_steps / e2e_s, "unit": "steps/s",
+           "h2d_bytes_per_step": 4 * (k * B * S + k * B) * world,
+           "d2h_bytes_per_step": 8 * (2 * n + 1) * world,
+           "steps": e2e_steps, "tokens_per_s": e2e_steps * fwds * T / e2e_s,
+           "path": ("zo_model_step_host: tokens and labels from pinned host memory, the 2n+1 "
+                    "losses copied back, synchronised every step" if world == 1 else
+                    "each rank copies the step's tokens and labels from pinned host memory, "
+                    "runs the probe-parallel step and reads the losses back")}
+
     cpu = None
-    if rank == 0 and not args.no_cpu_baseline:
-        # the oracle's forward of one layer at the real width (vocabulary cut to 4096: it only
-        # feeds the gather and the 2-row head), one thread; the step extrapolated from it
-        red = dict(cfg, n_layers=1, vocab=4096)
-        seq = 64
-        tps = oracle_workers([("forward", "qwen3" if qwen else "opt", json.dumps(red), seq)])[0][
-            "tokens_per_s"]
-        cpu_step_s = fwds * B * S * cfg["n_layers"] / tps
-        cpu = {"value": 1.0 / cpu_step_s, "unit": "steps/s", "cores": 1, "kind": "oracle",
-               "extrapolated": True,
-               "sample": f"oracle fp64 forward of 1 layer at the real width, 1 x {seq} tokens "
-                         f"(vocabulary cut to 4096): {tps:.1f} tokens/s; the step extrapolated "
-                         f"linearly in layers and tokens ({fwds} forwards of {B * S} tokens x "
-                         f"{cfg['n_layers']} layers), attention's quadratic term at the full "
-                         f"length not included"}
-    line = {
-        "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": 1, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
-        "config": {"workload": f"{name}-shaped decoder, micro-batch {B}x{S}, {k} micro-batches, "
-                               f"n_pert={n}, 1.5-SPSA", "layers": cfg["n_layers"], "d_model": d,
-                   "params": M},
-        "tokens_per_s": tokens_per_step * args.steps / total_s,
-        "forward_ms": fwd_ms,
-        "forwards_per_step": fwds,
-        "roofline": {"kernel": "gemm_bf16_kernel (tcgen05, 4 projections of one layer)",
-                     "bound": "tensor", "achieved": gemm_tflops, "peak": peak_b,
-                     "unit": "TFLOP/s", "frac": gemm_tflops / peak_b, "peak_kind": peak_kind,
-                     "flops_per_layer": flops_layer, "traffic": None},
-        "gemm": gemm,
-        "attention": {"avg_launch_us": attn_us, "tflops": attn_flops / attn_us / 1e6},
-        "phases_ms": {"clean_loss": float(phases[:, 0].mean()),
-                      "probe_losses": float(phases[:, 1].mean()), "precond_update": upd_ms},
-        "kernels": {"update_kernel": {"n_pert": n, "bytes": upd_bytes,
-                                      "achieved_GBps": upd_bytes / (upd_ms * 1e-3) / 1e9,
-                                      "frac_hbm": upd_bytes / (upd_ms * 1e-3) / 1e9 / peaks()[0]}},
-        "memory": {"peak_allocated_GB": peak_mem / 1e9, "device_used_GB": (tot_b - free_b) / 1e9},
-        "clocks": clocks,
-        "cpu_baseline": cpu,
-    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = decoder_cpu_baseline(name, cfg, w, fwds)
+
+    line = None
+    if rank == 0:
+        g = kernels.get("gemm", {})
+        line = {
+            "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "gpu_launches": launches,
+            "config": decoder_config(name, w, M, world),
+            "tokens_per_s": fwds * T * args.steps / total_s,
+            "tokens_per_step": fwds * T,
+            "forwards_per_step": fwds,
+            "step_ms": step_ms,
+            "roofline": {
+                "kernel": "gemm_bf16_kernel (tcgen05/TMEM, TMA-fed: the QKV, output and "
+                          "feed-forward projections of every forward)",
+                "bound": "tensor", "achieved": g.get("tflops"), "peak": peak_s,
+                "unit": "TFLOP/s", "frac": (g.get("tflops") or 0.0) / peak_s,
+                "peak_kind": f"{bf16_kind} sustained bf16 GEMM (the kernel runs inside a "
+                             f"seconds-long step under the power cap)",
+                "frac_of_burst": (g.get("tflops") or 0.0) / peak_b,
+                "flops_per_launch": g.get("flops_per_launch"),
+                "avg_launch_us": g.get("avg_launch_us"),
+                "timed": "CUDA events around every GEMM launch of the timed steps, on the "
+                         "context's stream",
+                "traffic": captured(GEMM_TRAFFIC, "bytes"),
+                "traffic_from": ("ncu capture of this kernel's current sources at the four "
+                                 "layer shapes (not this run)"
+                                 if captured(GEMM_TRAFFIC, "bytes") is not None else None)},
+            "kernels": kernels,
+            "kernel_timing_dropped": dropped,
+            "gemm_shapes_alone": gemm_shapes,
+            "attention_alone": attn_alone,
+            "phases_ms": phases,
+            "memory": {"device_used_GB": used_gb, "torch_peak_allocated_GB": peak_alloc_gb,
+                       "theta_GB": 2 * M / 1e9, "target_GB": MEMORY_TARGET_GB,
+                       "within_target": used_gb < MEMORY_TARGET_GB,
+                       "measured": "cudaMemGetInfo after the timed steps (every buffer of the "
+                                   "step is allocated once and kept; nothing grows per probe)"},
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "peaks": {"hbm_GBps": hbm_peak, "hbm_kind": hbm_kind, "bf16_burst_tflops": peak_b,
+                      "bf16_sustained_tflops": peak_s, "bf16_kind": bf16_kind},
+        }
+        if quad is not None:
+            line["quadratic"] = quad
+        if used_gb >= MEMORY_TARGET_GB:
+            print(f"warning: device memory {used_gb:.1f} GB is above the {MEMORY_TARGET_GB} GB "
+                  f"target", file=sys.stderr)
     model.close()
     ctx.close()
-    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
     return 0
+
+
+def decoder_cpu_baseline(name, cfg, w, fwds):
+    """The oracle's fp64 forward of one layer at the real width (1 x 64 tokens, vocabulary
+    cut to 4096: it only feeds the embedding gather and the 2-row head), one thread; the full
+    step extrapolated linearly in layers and tokens."""
+    B, S = w["batch"], w["seq"]
+    qwen = cfg.get("family") == "qwen3"
+    red = dict(cfg, n_layers=1, vocab=4096)
+    seq = 64
+    tps = oracle_workers([("forward", "qwen3" if qwen else "opt", json.dumps(red), seq)])[0]["tokens_per_s"]
+    cpu_step_s = fwds * B * S * cfg["n_layers"] / tps
+    return {"value": 1.0 / cpu_step_s, "unit": "steps/s", "cores": 1, "kind": "oracle",
+            "extrapolated": True,
+            "sample": f"oracle fp64 forward of 1 layer at the real width, 1 x {seq} tokens "
+                      f"(vocabulary cut to 4096): {tps:.2f} tokens/s on one thread; the step "
+                      f"extrapolated linearly in layers and tokens ({fwds} forwards of {B * S} "
+                      f"tokens x {cfg['n_layers']} layers); attention's quadratic term at the "
+                      f"full length not included",
+            "host": host_cpu()}
 
 
 # ------------------------------------------------------------------ conditioning study
@@ -939,20 +1203,22 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None,
-                    help="timed steps (default: 300 for the quadratic workloads and the MLP, 3 "
-                         "for the decoders)")
+                    help="timed steps (default: 3 for the decoders, 300 for the quadratic "
+                         "workloads and the MLP)")
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-quadratic", action="store_true",
+                    help="leave out the quadratic sub-record of the default workload's line")
     ap.add_argument("--traffic", type=float, default=None,
-                    help="ncu dram bytes per launch of the loss kernel, if measured")
-    ap.add_argument("--workload", default="quadratic",
+                    help="ncu dram bytes per launch of the quadratic's loss kernel, if measured")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=["quadratic", "mlp", "lowrank"] + sorted(DECODER_WORKLOADS))
     ap.add_argument("--n-pert", type=int, default=None, help="override n_pert (decoder workloads)")
     args = ap.parse_args()
     if args.steps is None:
         args.steps = 3 if args.workload in DECODER_WORKLOADS else 300
-    if args.warmup < 3 and args.workload == "quadratic":
+    if args.warmup < 3 and args.workload in ("quadratic",) + tuple(DECODER_WORKLOADS):
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return reference_arm(args)
@@ -962,7 +1228,10 @@ def main():
         return lowrank_arm(args)
     if args.workload != "quadratic":
         return decoder_arm(args)
-    return gpu_arm(args)
+    line = gpu_arm(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
 
 
 if __name__ == "__main__":

@@ -161,16 +161,50 @@ zo_status zo_enable_phase_timing(zo_ctx *ctx, int32_t n_steps);
  * milliseconds.  Errors: ZO_ERR_INVALID (n_steps outside what was recorded). */
 zo_status zo_phase_times(zo_ctx *ctx, int32_t n_steps, float *ms);
 
+/* Per-class kernel timing, for measuring kernels inside a running step.  While enabled,
+ * every launch of a timed class is bracketed by two CUDA events on the context's stream and
+ * recorded with its algorithmic work: ZO_KT_GEMM (the tcgen05 projections; work = 2 M N K
+ * flops, N counting both halves of a SwiGLU tile), ZO_KT_ATTENTION (causal attention; work =
+ * 4 hd B H S (S + 1) / 2 flops: Q K^T and P V over the causal pairs), ZO_KT_PERTURB (the
+ * unpack/apply kernel writing a perturbed window; work = 2 b count bytes: theta read, window
+ * written) and ZO_KT_UPDATE (work = 2 b M bytes: theta read and written once); b is the bytes
+ * per parameter.  The events cost a few microseconds per launch and break the programmatic
+ * launch overlap of the update.  At most 65,536 launches are recorded between two
+ * zo_kernel_times calls; later ones are counted as dropped.  Errors: ZO_ERR_INVALID. */
+#define ZO_KT_GEMM 0
+#define ZO_KT_ATTENTION 1
+#define ZO_KT_PERTURB 2
+#define ZO_KT_UPDATE 3
+#define ZO_KT_COUNT 4
+
+typedef struct {
+  double ms;         /* summed launch durations, milliseconds */
+  int64_t launches;  /* launches recorded */
+  double work;       /* summed algorithmic flops (GEMM, attention) or bytes (perturb, update) */
+} zo_kernel_time;
+
+zo_status zo_enable_kernel_timing(zo_ctx *ctx, int enable);
+
+/* Synchronise the context's stream, write the totals of the launches recorded since the
+ * last call into out[ZO_KT_COUNT] (host), the number of launches not recorded into *dropped
+ * (host, may be NULL), and start over.  Errors: ZO_ERR_INVALID (null out), ZO_ERR_CUDA. */
+zo_status zo_kernel_times(zo_ctx *ctx, zo_kernel_time *out, int64_t *dropped);
+
+/* Number of kernels this context has launched since it was created (every entry point that
+ * enqueues work counts its launches; memory copies are not counted).  Errors: ZO_ERR_INVALID. */
+zo_status zo_launch_count(zo_ctx *ctx, int64_t *count);
+
 /* ------------------------------------------------------------------ zo_rng */
 
-/* Write packed probe bytes [first_byte, first_byte + nbytes) of probe `probe` at the
- * current step into dev_out (device, nbytes bytes), 8 elements of the one probe per byte
+/* Write packed probe bytes [first_byte, first_byte + nbytes) of probe `probe` of step
+ * `step` (any step: the probes are a pure function of (seed, step, probe, element), so no
+ * state is read) into dev_out (device, nbytes bytes), 8 elements of the one probe per byte
  * (byte q: elements 8q..8q+7, bit t <-> element 8q+t).  Bits of
  * elements >= M are 0.  For tests and inspection: the training path regenerates probe
  * bits in registers and never stores them.
  * Errors: ZO_ERR_INVALID (probe < 0, range outside ceil(M/8) bytes, null dev_out). */
-zo_status zo_pack_probe(zo_ctx *ctx, int32_t probe, int64_t first_byte, int64_t nbytes,
-                        uint8_t *dev_out);
+zo_status zo_pack_probe(zo_ctx *ctx, uint32_t step, int32_t probe, int64_t first_byte,
+                        int64_t nbytes, uint8_t *dev_out);
 
 /* ------------------------------------------------------------------ zo_perturb */
 
@@ -289,6 +323,14 @@ zo_status zo_mlp_loss_noalloc(const float *P, const float *X, const int32_t *lab
  *         damping < 0), ZO_ERR_STATE (perturbed), ZO_ERR_CUDA. */
 zo_status zo_step(zo_ctx *ctx, const double *loss_plus, const double *loss_minus,
                   int32_t n_pert, const double *loss0, float lr, float eps, float damping);
+
+/* Where zo_step reads its losses [LOOP: the losses feed the estimate wherever they were
+ * produced]: on_device = 1 (the default) takes device pointers, which keeps a step free of
+ * host synchronisation; on_device = 0 takes host pointers: zo_step copies the 2 n_pert (+1)
+ * losses into the context's scratch on its stream and waits for the copies, so the host
+ * arrays may be reused when it returns.  The step drivers always pass device losses and are
+ * not affected.  Errors: ZO_ERR_INVALID (null context). */
+zo_status zo_set_loss_location(zo_ctx *ctx, int on_device);
 
 /* The update alone: theta <- rd(theta - sum_i coef_i z_i) with coef (device, n_pert
  * floats) at the current step, in the fixed fp32 order above.  Does not advance the
@@ -477,6 +519,17 @@ zo_status zo_model_step(zo_model *m, const int32_t *tokens, const int32_t *label
                         int32_t batch, int32_t seq, int32_t n_micro, int32_t n_pert,
                         float eps, float lr, float damping, int preconditioned,
                         double *losses_out);
+
+/* zo_model_step with host buffers: copies tokens_host [n_micro][batch][seq] and labels_host
+ * [n_micro][batch] (host int32; pinned memory makes the copies asynchronous DMA) to device
+ * staging owned by the model (allocated on first use, grown if a call needs more), runs
+ * zo_model_step on them, copies the 2*n_pert+1 losses [L0, L+..., L-...] back to losses_host
+ * (host doubles) and synchronises the context's stream.  Device flags (a skipped non-finite
+ * step) are reported by the next zo_sync.  Errors: as zo_model_step, ZO_ERR_OOM. */
+zo_status zo_model_step_host(zo_model *m, const int32_t *tokens_host, const int32_t *labels_host,
+                             int32_t batch, int32_t seq, int32_t n_micro, int32_t n_pert,
+                             float eps, float lr, float damping, int preconditioned,
+                             double *losses_host);
 
 /* ------------------------------------------------------------------ decoder components */
 

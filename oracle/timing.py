@@ -9,6 +9,7 @@ processes on disjoint samples, each single-threaded).
   python -m oracle.timing steps M_SAMPLE SEED N_PERT EPS LR DAMPING WARMUP STEPS
   python -m oracle.timing forward FAMILY CFG_JSON SEQ
   python -m oracle.timing mlp STEPS
+  python -m oracle.timing forward_samples FAMILY CFG_JSON SEQ WARMUP STEPS
 
 print one JSON object on stdout.
 """
@@ -96,6 +97,31 @@ def forward_tokens_per_s(family, cfg, seq, batch=1):
     return batch * seq / (time.perf_counter() - t0)
 
 
+def forward_samples(family, cfg, seq, warmup, steps):
+    """warmup + steps timed evaluations of the oracle's decoder loss (fp64) at the given
+    configuration on one sequence of `seq` tokens, the weights generated once beforehand;
+    returns the seconds of each timed evaluation and the wall-clock bounds of the timed phase."""
+    import synth
+
+    from . import opt, qwen
+    if family == "qwen3":
+        mod, bits = qwen, synth.qwen_params(cfg)
+    else:
+        mod, bits = opt, synth.opt_params(cfg)
+    theta = (bits.astype(np.uint32) << 16).view(np.float32)
+    del bits
+    tokens, labels = synth.opt_batch(cfg, 1, seq)
+    times, t_start = [], None
+    for s in range(warmup + steps):
+        if s == warmup:
+            t_start = time.time()
+        t0 = time.perf_counter()
+        mod.loss(theta, cfg, tokens, labels)
+        if s >= warmup:
+            times.append(time.perf_counter() - t0)
+    return {"times": times, "t_start": t_start, "t_end": time.time()}
+
+
 def _main(argv):
     if argv[0] == "steps":
         M, seed, n, eps, lr, lam, w, k = argv[1:9]
@@ -107,8 +133,13 @@ def _main(argv):
         if "class_ids" in cfg:
             cfg["class_ids"] = tuple(cfg["class_ids"])
         res = {"tokens_per_s": forward_tokens_per_s(argv[1], cfg, int(argv[3]))}
+    elif argv[0] == "forward_samples":
+        cfg = json.loads(argv[2])
+        if "class_ids" in cfg:
+            cfg["class_ids"] = tuple(cfg["class_ids"])
+        res = forward_samples(argv[1], cfg, int(argv[3]), int(argv[4]), int(argv[5]))
     else:
-        raise SystemExit("usage: python -m oracle.timing steps|forward|mlp ...")
+        raise SystemExit("usage: python -m oracle.timing steps|forward|forward_samples|mlp ...")
     print(json.dumps(res), flush=True)
 
 

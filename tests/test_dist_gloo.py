@@ -164,3 +164,59 @@ def test_element_parallel_step_matches_single_rank(tmp_path, world):
     full = oracle.core.update_mirror(theta, outs[0]["a"], SEED, 0)
     got = np.concatenate([o["theta"] for o in outs])
     assert got.tobytes() == full.tobytes()
+
+
+def test_batch_share_covers_every_sequence_once():
+    for batch in (0, 1, 2, 7, 8, 16):
+        for world in (1, 2, 3, 8):
+            got = []
+            for r in range(world):
+                first, count = zdist.batch_share(batch, r, world)
+                assert count >= 0
+                got += list(range(first, first + count))
+            assert got == list(range(batch))
+
+
+def _clean_shared_worker(rank, world, port, out_dir):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        per_seq = np.arange(1, 8, dtype=np.float64) * 0.1  # per-sequence clean losses
+        first, count = zdist.batch_share(per_seq.size, rank, world)
+
+        def clean(out):
+            out[0] = float(per_seq[first:first + count].sum())
+
+        def loss_at(sign, probe, out):
+            out[0] = 10.0 * probe + sign
+
+        seen = {}
+
+        def apply_step(Lp, Lm, L0):
+            seen["L0"] = float(L0[0])
+
+        L0, Lp, Lm = zdist.probe_parallel_step(5, loss_at, clean, apply_step, "cpu",
+                                               clean_shared=True)
+        np.savez(os.path.join(out_dir, f"c{rank}.npz"), L0=L0.numpy(), Lp=Lp.numpy(),
+                 Lm=Lm.numpy(), seen=seen["L0"])
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_clean_loss_shared_by_batch(tmp_path, world):
+    mp.start_processes(_clean_shared_worker, args=(world, _free_port(), str(tmp_path)),
+                       nprocs=world, start_method="spawn", join=True)
+    rs = [np.load(os.path.join(tmp_path, f"c{r}.npz")) for r in range(world)]
+    per_seq = np.arange(1, 8, dtype=np.float64) * 0.1
+    parts = [per_seq[slice(*(lambda f, c: (f, f + c))(*zdist.batch_share(7, r, world)))].sum()
+             for r in range(world)]
+    want = parts[0]
+    for p in parts[1:]:
+        want += p  # rank order
+    for r in rs:
+        assert r["L0"][0] == want and float(r["seen"]) == want
+        assert np.array_equal(r["Lp"], 10.0 * np.arange(5) + 1)
+        assert np.array_equal(r["Lm"], 10.0 * np.arange(5) - 1)

@@ -64,17 +64,17 @@ def test_pack_probe_bit_exact(zo, M):
     th = torch.zeros(max(M, 4), device="cuda")
     seed = 0x0123456789ABCDEF
     ctx = zo.zo_create(th, seed=seed, M=M)
-    for step in (0, 5):
-        zo.zo_set_step(ctx, step)
+    # the step is an argument: the context's own counter (0 here) is not read
+    for step in (0, 5, 0xFFFFFFFF):
         for probe in (0, 3, 1023):
             nbytes = (M + 7) // 8
             out = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
-            zo.zo_pack_probe(ctx, probe, 0, nbytes, out)
+            zo.zo_pack_probe(ctx, step, probe, 0, nbytes, out)
             torch.cuda.synchronize()
             assert (out.cpu().numpy() == core.pack_probe(seed, step, probe, M)).all()
             if nbytes > 20:  # a window starting mid-group
                 w = torch.zeros(nbytes - 19, dtype=torch.uint8, device="cuda")
-                zo.zo_pack_probe(ctx, probe, 19, nbytes - 19, w)
+                zo.zo_pack_probe(ctx, step, probe, 19, nbytes - 19, w)
                 torch.cuda.synchronize()
                 assert (w.cpu().numpy() == core.pack_probe(seed, step, probe, M)[19:]).all()
     ctx.close()

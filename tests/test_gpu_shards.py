@@ -39,7 +39,7 @@ def test_slices_perturb_and_pack_like_the_whole_vector(zo):
     zo.zo_perturb_range(full, 0, M, whole)
     zo.zo_restore(full)
     packed = torch.empty(M // 8 + 1, dtype=torch.uint8, device="cuda")
-    zo.zo_pack_probe(full, 13, 0, (M + 7) // 8, packed)
+    zo.zo_pack_probe(full, 0, 13, 0, (M + 7) // 8, packed)
     for first, count, c in parts:
         out = torch.empty(count, device="cuda")
         zo.zo_perturb(c, -1, 1e-3, 13)
@@ -47,7 +47,7 @@ def test_slices_perturb_and_pack_like_the_whole_vector(zo):
         zo.zo_restore(c)
         assert torch.equal(out, whole[first:first + count])
         pb = torch.empty((count + 7) // 8, dtype=torch.uint8, device="cuda")
-        zo.zo_pack_probe(c, 13, 0, (count + 7) // 8, pb)
+        zo.zo_pack_probe(c, 0, 13, 0, (count + 7) // 8, pb)
         assert torch.equal(pb, packed[first // 8:first // 8 + (count + 7) // 8])
         c.close()
     full.close()

@@ -51,6 +51,14 @@ def test_create_rejects_bad_arguments_before_touching_a_device(zo):
     assert L.zo_destroy(None) == zo.ZO_OK
     assert L.zo_perturb(None, 1, 1e-3, 0) == zo.ZO_ERR_INVALID
     assert L.zo_step(None, None, None, 1, None, 0.1, 1e-3, 0.0) == zo.ZO_ERR_INVALID
+    n = ctypes.c_int64(-1)
+    assert L.zo_launch_count(None, ctypes.byref(n)) == zo.ZO_ERR_INVALID
+    assert n.value == -1
+    assert L.zo_kernel_times(None, None, None) == zo.ZO_ERR_INVALID
+    assert L.zo_enable_kernel_timing(None, 1) == zo.ZO_ERR_INVALID
+    assert L.zo_set_loss_location(None, 0) == zo.ZO_ERR_INVALID
+    assert L.zo_pack_probe(None, 0, 0, 0, 1, None) == zo.ZO_ERR_INVALID
+    assert L.zo_model_step_host(None, None, None, 1, 1, 1, 1, 1e-3, 0.1, 0.0, 1, None) == zo.ZO_ERR_INVALID
 
 
 def test_product_path_has_no_oracle_dependency():

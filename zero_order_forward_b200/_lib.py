@@ -24,6 +24,8 @@ ZO_F32, ZO_BF16 = 0, 1
 ZO_FLAG_NONFINITE = 0x1
 ZO_FLAG_TIMEOUT = 0x2
 ZO_EPI_BIAS_BF16, ZO_EPI_RELU_BF16, ZO_EPI_RESID_F32 = 0, 1, 2
+ZO_KT_GEMM, ZO_KT_ATTENTION, ZO_KT_PERTURB, ZO_KT_UPDATE, ZO_KT_COUNT = 0, 1, 2, 3, 4
+KERNEL_CLASSES = ("gemm", "attention", "perturb", "update")
 ZO_MAX_PROBES = 1024
 ZO_NOALLOC_MAX_BATCH = 4096
 
@@ -39,7 +41,7 @@ _SIGS = {
     "zo_get_step": [_vp, ctypes.POINTER(_u32)],
     "zo_set_step": [_vp, _u32],
     "zo_set_element_offset": [_vp, _i64],
-    "zo_pack_probe": [_vp, _i32, _i64, _i64, _vp],
+    "zo_pack_probe": [_vp, _u32, _i32, _i64, _i64, _vp],
     "zo_perturb": [_vp, _int, _f32, _i32],
     "zo_restore": [_vp],
     "zo_perturb_range": [_vp, _i64, _i64, _vp],
@@ -74,6 +76,11 @@ _SIGS = {
     "zo_rmsnorm": [_vp, _vp, _vp, _vp, _i32, _i32, _f32],
     "zo_debug_gemm_timeout": [_vp, _vp, _vp, _vp, _i32, _i32, _i32],
     "zo_layernorm": [_vp, _vp, _vp, _vp, _vp, _i32, _i32],
+    "zo_enable_kernel_timing": [_vp, _int],
+    "zo_kernel_times": [_vp, _vp, ctypes.POINTER(_i64)],
+    "zo_launch_count": [_vp, ctypes.POINTER(_i64)],
+    "zo_set_loss_location": [_vp, _int],
+    "zo_model_step_host": [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _f32, _f32, _f32, _int, _vp],
 }
 for _name, _args in _SIGS.items():
     _fn = getattr(_L, _name)
@@ -201,8 +208,9 @@ def zo_set_element_offset(ctx, first_element):
     return ctx.check(_L.zo_set_element_offset(ctx.handle, int(first_element)))
 
 
-def zo_pack_probe(ctx, probe, first_byte, nbytes, out):
-    return ctx.check(_L.zo_pack_probe(ctx.handle, probe, first_byte, nbytes, _ptr(out)))
+def zo_pack_probe(ctx, step, probe, first_byte, nbytes, out):
+    return ctx.check(_L.zo_pack_probe(ctx.handle, int(step) & 0xFFFFFFFF, probe, first_byte, nbytes,
+                                      _ptr(out)))
 
 
 def zo_perturb(ctx, sign, eps, probe):
@@ -234,6 +242,11 @@ def zo_mlp_loss(ctx, X, labels, batch, n_in, n_hidden, n_out, scale, loss_out, a
 def zo_step(ctx, loss_plus, loss_minus, n_pert, loss0, lr, eps, damping):
     return ctx.check(_L.zo_step(ctx.handle, _ptr(loss_plus), _ptr(loss_minus), n_pert,
                                 _ptr(loss0), lr, eps, damping))
+
+
+def zo_set_loss_location(ctx, on_device):
+    """on_device False: zo_step takes host arrays (numpy) for its losses."""
+    return ctx.check(_L.zo_set_loss_location(ctx.handle, 1 if on_device else 0))
 
 
 def zo_update(ctx, coef, n_pert):
@@ -405,6 +418,15 @@ def zo_model_step(model, tokens, labels, batch, seq, n_micro, n_pert, eps, lr, d
                                             int(preconditioned), _ptr(losses_out)))
 
 
+def zo_model_step_host(model, tokens_host, labels_host, batch, seq, n_micro, n_pert, eps, lr,
+                       damping, preconditioned, losses_host):
+    """zo_model_step from host int32 tokens/labels (numpy or pinned CPU tensors) with the
+    2 n_pert + 1 losses copied back to losses_host (host float64); synchronises."""
+    return model.ctx.check(_L.zo_model_step_host(model.handle, _ptr(tokens_host), _ptr(labels_host),
+                                                 batch, seq, n_micro, n_pert, eps, lr, damping,
+                                                 int(preconditioned), _ptr(losses_host)))
+
+
 def zo_gemm_bf16(ctx, A, B, bias, out, M, N, K, ldo, epilogue):
     return ctx.check(_L.zo_gemm_bf16(ctx.handle, _ptr(A), _ptr(B), _ptr(bias), _ptr(out), M, N,
                                      K, ldo, epilogue))
@@ -439,6 +461,31 @@ def zo_phase_times(ctx, n_steps):
     ms = np.zeros((n_steps, 3), np.float32)
     ctx.check(_L.zo_phase_times(ctx.handle, n_steps, ms.ctypes.data))
     return ms
+
+
+class zo_kernel_time(ctypes.Structure):
+    _fields_ = [("ms", _f64), ("launches", _i64), ("work", _f64)]
+
+
+def zo_enable_kernel_timing(ctx, enable):
+    return ctx.check(_L.zo_enable_kernel_timing(ctx.handle, 1 if enable else 0))
+
+
+def zo_kernel_times(ctx):
+    """Per kernel class ({"gemm", "attention", "perturb", "update"}): summed ms, launches and
+    algorithmic work of the launches recorded since the last call (synchronises), and the
+    number of launches not recorded."""
+    out = (zo_kernel_time * ZO_KT_COUNT)()
+    dropped = _i64()
+    ctx.check(_L.zo_kernel_times(ctx.handle, out, ctypes.byref(dropped)))
+    return ({name: {"ms": out[i].ms, "launches": out[i].launches, "work": out[i].work}
+             for i, name in enumerate(KERNEL_CLASSES)}, dropped.value)
+
+
+def zo_launch_count(ctx):
+    n = _i64()
+    ctx.check(_L.zo_launch_count(ctx.handle, ctypes.byref(n)))
+    return n.value
 
 
 def zo_debug_gemm_timeout(ctx, A, B, out, M, N, K):

@@ -345,8 +345,13 @@ zo_status launch_tc(zo_ctx *ctx, const CUtensorMap &tmq, const CUtensorMap &tmkv
     if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "attn_tc_kernel attribute: %s", cudaGetErrorString(e));
   }
   const dim3 grid((a.S + kTBM - 1) / kTBM, a.H, B);
+  const int slot = ktime_begin(ctx);
   attn_tc_kernel<HD><<<grid, kTThreads, SM::kBytes, ctx->stream>>>(tmq, tmkv, a);
-  return check_launch(ctx, "attn_tc_kernel");
+  const zo_status st = check_launch(ctx, "attn_tc_kernel");
+  // algorithmic flops: Q K^T and P V over the causal pairs, 2 hd flops each per product
+  if (st == ZO_OK)
+    ktime_end(ctx, slot, ZO_KT_ATTENTION, 4.0 * HD * (double)B * a.H * ((double)a.S * (a.S + 1) / 2));
+  return st;
 }
 
 }  // namespace

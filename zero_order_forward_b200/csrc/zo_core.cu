@@ -37,6 +37,7 @@ zo_status check_launch(zo_ctx *ctx, const char *what) {
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
     return fail(ctx, ZO_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  ctx->launches += 1;
   return ZO_OK;
 }
 
@@ -72,9 +73,64 @@ void phase_mark(zo_ctx *ctx, int which) {
   if (which == 3) ctx->phase_used += 1;
 }
 
+// At most this many launches are recorded between two drains (zo_kernel_times); later ones
+// are counted as dropped.
+constexpr size_t kKtimeMaxRecords = 1u << 16;
+
+int ktime_begin(zo_ctx *ctx) {
+  if (!ctx->ktime_on) return -1;
+  const size_t k = ctx->ktime_recs.size();
+  if (k >= kKtimeMaxRecords) {
+    ctx->ktime_dropped += 1;
+    return -1;
+  }
+  while (ctx->ktime_ev.size() < 2 * (k + 1)) {
+    cudaEvent_t ev;
+    if (cudaEventCreate(&ev) != cudaSuccess) {
+      cudaGetLastError();
+      ctx->ktime_dropped += 1;
+      return -1;
+    }
+    ctx->ktime_ev.push_back(ev);
+  }
+  if (cudaEventRecord(ctx->ktime_ev[2 * k], ctx->stream) != cudaSuccess) {
+    cudaGetLastError();
+    ctx->ktime_dropped += 1;
+    return -1;
+  }
+  ctx->ktime_recs.push_back({-1, 0.0});
+  return (int)k;
+}
+
+void ktime_end(zo_ctx *ctx, int slot, int cls, double work) {
+  if (slot < 0) return;
+  if (cudaEventRecord(ctx->ktime_ev[2 * (size_t)slot + 1], ctx->stream) != cudaSuccess) {
+    cudaGetLastError();
+    return;  // the record keeps class -1 and is skipped by the drain
+  }
+  ctx->ktime_recs[(size_t)slot] = {cls, work};
+}
+
 }  // namespace zo
 
 using namespace zo;
+
+namespace {
+zo_status check_step_args(zo_ctx *ctx, int32_t n, float lr, float eps, float damping);
+}
+
+zo_status zo::step_device(zo_ctx *ctx, const double *loss_plus, const double *loss_minus,
+                          int32_t n_pert, const double *loss0, float lr, float eps, float damping) {
+  {
+    const zo_status s0 = check_step_args(ctx, n_pert, lr, eps, damping);
+    if (s0 != ZO_OK) return s0;
+  }
+  if (!loss_plus || !loss_minus) return fail(ctx, ZO_ERR_INVALID, "null loss arrays");
+  if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "zo_step while perturbed");
+  const zo_status st = launch_precond(ctx, loss_plus, loss_minus, loss0, n_pert, lr, eps, damping);
+  if (st != ZO_OK) return st;
+  return launch_update(ctx, ctx->coef, n_pert, &ctx->dstate->upd_step, &ctx->dstate->upd_ok);
+}
 
 namespace {
 
@@ -199,6 +255,7 @@ zo_status zo_destroy(zo_ctx *ctx) {
     for (int i = 0; i < 4 * ctx->phase_cap; ++i) cudaEventDestroy(ctx->phase_ev[i]);
     delete[] ctx->phase_ev;
   }
+  for (cudaEvent_t ev : ctx->ktime_ev) cudaEventDestroy(ev);
   delete ctx;
   return ZO_OK;
 }
@@ -238,6 +295,49 @@ zo_status zo_phase_times(zo_ctx *ctx, int32_t n_steps, float *ms) {
     for (int p = 0; p < 3; ++p)
       ZO_CUDA(ctx, cudaEventElapsedTime(&ms[3 * k + p], ctx->phase_ev[4 * k + p],
                                         ctx->phase_ev[4 * k + p + 1]), "cudaEventElapsedTime");
+  return ZO_OK;
+}
+
+zo_status zo_enable_kernel_timing(zo_ctx *ctx, int enable) {
+  ZO_CHECK(check_ctx(ctx));
+  ctx->ktime_on = enable != 0;
+  return ZO_OK;
+}
+
+zo_status zo_kernel_times(zo_ctx *ctx, zo_kernel_time *out, int64_t *dropped) {
+  ZO_CHECK(check_ctx(ctx));
+  if (!out) return fail(ctx, ZO_ERR_INVALID, "null output");
+  ZO_CUDA(ctx, cudaStreamSynchronize(ctx->stream), "sync");
+  for (int c = 0; c < ZO_KT_COUNT; ++c) out[c] = zo_kernel_time{0.0, 0, 0.0};
+  zo_status st = ZO_OK;
+  for (size_t k = 0; k < ctx->ktime_recs.size(); ++k) {
+    const auto &r = ctx->ktime_recs[k];
+    if (r.cls < 0 || r.cls >= ZO_KT_COUNT) continue;
+    float ms = 0.f;
+    const cudaError_t e = cudaEventElapsedTime(&ms, ctx->ktime_ev[2 * k], ctx->ktime_ev[2 * k + 1]);
+    if (e != cudaSuccess) {
+      st = cuda_fail(ctx, e, "cudaEventElapsedTime");
+      break;
+    }
+    out[r.cls].ms += ms;
+    out[r.cls].launches += 1;
+    out[r.cls].work += r.work;
+  }
+  if (dropped) *dropped = ctx->ktime_dropped;
+  ctx->ktime_recs.clear();
+  ctx->ktime_dropped = 0;
+  return st;
+}
+
+zo_status zo_launch_count(zo_ctx *ctx, int64_t *count) {
+  if (!ctx || !count) return ZO_ERR_INVALID;
+  *count = ctx->launches;
+  return ZO_OK;
+}
+
+zo_status zo_set_loss_location(zo_ctx *ctx, int on_device) {
+  ZO_CHECK(check_ctx(ctx));
+  ctx->host_losses = on_device == 0;
   return ZO_OK;
 }
 
@@ -311,13 +411,13 @@ zo_status zo_set_element_offset(zo_ctx *ctx, int64_t first_element) {
   return ZO_OK;
 }
 
-zo_status zo_pack_probe(zo_ctx *ctx, int32_t probe, int64_t first_byte, int64_t nbytes,
-                        uint8_t *dev_out) {
+zo_status zo_pack_probe(zo_ctx *ctx, uint32_t step, int32_t probe, int64_t first_byte,
+                        int64_t nbytes, uint8_t *dev_out) {
   ZO_CHECK(check_ctx(ctx));
   const int64_t total = (ctx->M + 7) / 8;
   if (probe < 0 || !dev_out || first_byte < 0 || nbytes < 0 || first_byte + nbytes > total)
     return fail(ctx, ZO_ERR_INVALID, "pack range outside [0, %lld) bytes", (long long)total);
-  return launch_pack(ctx, (uint32_t)probe, first_byte, nbytes, dev_out);
+  return launch_pack(ctx, step, (uint32_t)probe, first_byte, nbytes, dev_out);
 }
 
 zo_status zo_perturb(zo_ctx *ctx, int sign, float eps, int32_t probe) {
@@ -396,11 +496,22 @@ zo_status zo_mlp_loss(zo_ctx *ctx, const float *X, const int32_t *labels, int ba
 zo_status zo_step(zo_ctx *ctx, const double *loss_plus, const double *loss_minus, int32_t n_pert,
                   const double *loss0, float lr, float eps, float damping) {
   ZO_CHECK(check_ctx(ctx));
+  if (!ctx->host_losses) return step_device(ctx, loss_plus, loss_minus, n_pert, loss0, lr, eps, damping);
+  // host losses: staged into the context's loss scratch [L0, L+..., L-...] on its stream
   ZO_CHECK(check_step_args(ctx, n_pert, lr, eps, damping));
   if (!loss_plus || !loss_minus) return fail(ctx, ZO_ERR_INVALID, "null loss arrays");
   if (ctx->state != PState::Clean) return fail(ctx, ZO_ERR_STATE, "zo_step while perturbed");
-  ZO_CHECK(launch_precond(ctx, loss_plus, loss_minus, loss0, n_pert, lr, eps, damping));
-  return launch_update(ctx, ctx->coef, n_pert, &ctx->dstate->upd_step, &ctx->dstate->upd_ok);
+  if (!ctx->loss_scratch)
+    ZO_CUDA(ctx, cudaMalloc(&ctx->loss_scratch, (2 * ZO_MAX_PROBES + 1) * sizeof(double)), "loss scratch");
+  double *L0 = ctx->loss_scratch, *Lp = L0 + 1, *Lm = L0 + 1 + n_pert;
+  const size_t nb = (size_t)n_pert * sizeof(double);
+  ZO_CUDA(ctx, cudaMemcpyAsync(Lp, loss_plus, nb, cudaMemcpyHostToDevice, ctx->stream), "copy L+");
+  ZO_CUDA(ctx, cudaMemcpyAsync(Lm, loss_minus, nb, cudaMemcpyHostToDevice, ctx->stream), "copy L-");
+  if (loss0)
+    ZO_CUDA(ctx, cudaMemcpyAsync(L0, loss0, sizeof(double), cudaMemcpyHostToDevice, ctx->stream), "copy L0");
+  // the copies read host memory that the caller may reuse once zo_step returns
+  ZO_CUDA(ctx, cudaStreamSynchronize(ctx->stream), "sync");
+  return step_device(ctx, Lp, Lm, n_pert, loss0 ? L0 : nullptr, lr, eps, damping);
 }
 
 zo_status zo_update(zo_ctx *ctx, const float *coef, int32_t n_pert) {
@@ -508,7 +619,7 @@ zo_status zo_lowrank_step(zo_ctx *ctx, const float *D, const zo_lowrank *q, int3
   ZO_CHECK(launch_lowrank_combine(ctx, base, dots, q->rank, n_pert, lam, preconditioned ? 1 : 0,
                                   losses_out));
   phase_mark(ctx, 2);
-  const zo_status st = zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
+  const zo_status st = step_device(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
   phase_mark(ctx, 3);
   return st;
 }
@@ -545,7 +656,7 @@ zo_status zo_quad_step(zo_ctx *ctx, const float *D, int32_t n_pert, float eps, f
     ZO_CHECK(zo_quad_loss_octet(ctx, D, i, n_pert - i < 64 ? n_pert - i : 64, eps, Lp + i, Lm + i,
                                 (preconditioned && i == 0) ? L0 : nullptr));
   phase_mark(ctx, 2);
-  const zo_status st = zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
+  const zo_status st = step_device(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
   phase_mark(ctx, 3);
   return st;
 }
@@ -634,7 +745,7 @@ zo_status zo_mlp_step(zo_ctx *ctx, const float *X, const int32_t *labels, int ba
     ZO_CHECK(zo_mlp_losses(ctx, X, labels, batch, n_in, n_hidden, n_out, n_pert, eps, scale, Lp,
                            Lm, preconditioned ? L0 : nullptr));
     phase_mark(ctx, 2);
-    const zo_status st = zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
+    const zo_status st = step_device(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
     phase_mark(ctx, 3);
     return st;
   }
@@ -656,7 +767,7 @@ zo_status zo_mlp_step(zo_ctx *ctx, const float *X, const int32_t *labels, int ba
     }
   }
   phase_mark(ctx, 2);
-  const zo_status st = zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
+  const zo_status st = step_device(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
   phase_mark(ctx, 3);
   return st;
 }

@@ -334,6 +334,10 @@ struct zo_model {
   bool prune_enabled = true;
   float *hl = nullptr;      // residual rows [prune_rows][d]
   uint16_t *xl = nullptr, *ql = nullptr, *al = nullptr, *midl = nullptr;
+  // zo_model_step_host: device copies of one step's tokens and labels, and its losses
+  int32_t *stage = nullptr;
+  size_t stage_cap = 0;     // int32 words
+  double *stage_losses = nullptr;
 };
 
 namespace {
@@ -566,6 +570,8 @@ zo_status zo_model_destroy(zo_model *m) {
   cudaFree(m->ql);
   cudaFree(m->al);
   cudaFree(m->midl);
+  cudaFree(m->stage);
+  cudaFree(m->stage_losses);
   delete m;
   return ZO_OK;
 }
@@ -656,9 +662,48 @@ zo_status zo_model_step(zo_model *m, const int32_t *tokens, const int32_t *label
     }
   }
   phase_mark(ctx, 2);
-  st = zo_step(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
+  st = step_device(ctx, Lp, Lm, n_pert, preconditioned ? L0 : nullptr, lr, eps, damping);
   phase_mark(ctx, 3);
   return st;
+}
+
+zo_status zo_model_step_host(zo_model *m, const int32_t *tokens_host, const int32_t *labels_host,
+                             int32_t batch, int32_t seq, int32_t n_micro, int32_t n_pert, float eps,
+                             float lr, float damping, int preconditioned, double *losses_host) {
+  if (!m) return ZO_ERR_INVALID;
+  zo_ctx *ctx = m->ctx;
+  ctx->err.clear();
+  if (!tokens_host || !labels_host || !losses_host || batch < 1 || seq < 1 || n_micro < 1 ||
+      n_pert < 1 || n_pert > ZO_MAX_PROBES)
+    return fail(ctx, ZO_ERR_INVALID, "bad host step arguments");
+  const size_t n_tok = (size_t)n_micro * batch * seq, n_lab = (size_t)n_micro * batch;
+  zo_status st;
+  if (n_tok + n_lab > m->stage_cap) {
+    if ((st = model_cuda(ctx, cudaStreamSynchronize(ctx->stream), "sync")) != ZO_OK) return st;
+    cudaFree(m->stage);
+    m->stage = nullptr;
+    m->stage_cap = 0;
+    if ((st = model_cuda(ctx, cudaMalloc(&m->stage, (n_tok + n_lab) * sizeof(int32_t)), "token staging")) != ZO_OK)
+      return st;
+    m->stage_cap = n_tok + n_lab;
+  }
+  if (!m->stage_losses &&
+      (st = model_cuda(ctx, cudaMalloc(&m->stage_losses, (2 * ZO_MAX_PROBES + 1) * sizeof(double)),
+                       "loss staging")) != ZO_OK)
+    return st;
+  int32_t *dtok = m->stage, *dlab = m->stage + n_tok;
+  if ((st = model_cuda(ctx, cudaMemcpyAsync(dtok, tokens_host, n_tok * sizeof(int32_t), cudaMemcpyHostToDevice,
+                                            ctx->stream), "copy tokens")) != ZO_OK ||
+      (st = model_cuda(ctx, cudaMemcpyAsync(dlab, labels_host, n_lab * sizeof(int32_t), cudaMemcpyHostToDevice,
+                                            ctx->stream), "copy labels")) != ZO_OK)
+    return st;
+  if ((st = zo_model_step(m, dtok, dlab, batch, seq, n_micro, n_pert, eps, lr, damping, preconditioned,
+                          m->stage_losses)) != ZO_OK)
+    return st;
+  if ((st = model_cuda(ctx, cudaMemcpyAsync(losses_host, m->stage_losses, (2 * (size_t)n_pert + 1) * sizeof(double),
+                                            cudaMemcpyDeviceToHost, ctx->stream), "copy losses")) != ZO_OK)
+    return st;
+  return model_cuda(ctx, cudaStreamSynchronize(ctx->stream), "sync");
 }
 
 zo_status zo_gemm_bf16(zo_ctx *ctx, const void *A, const void *B, const void *bias, void *out,

@@ -392,6 +392,7 @@ zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bia
       !make_out_map(&tcm, out, M, N, ldo, epi == ZO_EPI_RESID_F32))
     return fail(ctx, ZO_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
   GemmArgs g{M, N, K, static_cast<const uint16_t *>(bias), out, ldo, &ctx->dstate->flags, extra_tx};
+  const int slot = ktime_begin(ctx);
   cudaError_t e;
   if (wide) {
     if (epi == ZO_EPI_BIAS_BF16) e = launch_one<256, 4, ZO_EPI_BIAS_BF16>(ta, tb, tcm, g, ctx->stream);
@@ -405,6 +406,8 @@ zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bia
     else e = launch_one<128, 6, ZO_EPI_SWIGLU_BF16>(ta, tb, tcm, g, ctx->stream);
   }
   if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "gemm launch: %s", cudaGetErrorString(e));
+  ctx->launches += 1;
+  ktime_end(ctx, slot, ZO_KT_GEMM, 2.0 * M * (double)NB * K);  // NB accumulator columns
   return ZO_OK;
 }
 

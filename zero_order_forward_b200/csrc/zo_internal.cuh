@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <string>
+#include <vector>
 
 #include "zo.h"
 
@@ -149,6 +150,23 @@ struct zo_ctx {
   cudaEvent_t *phase_ev = nullptr;
   int32_t phase_cap = 0, phase_used = 0;
 
+  // kernels this context has enqueued (every successful launch)
+  int64_t launches = 0;
+
+  // per-class kernel timing (zo_enable_kernel_timing): an event pair around every launch of
+  // the timed classes, with the launch's algorithmic work; drained by zo_kernel_times
+  struct KRec {
+    int cls;      // ZO_KT_* or -1 (launch failed after its start event)
+    double work;  // flops or bytes of this launch
+  };
+  bool ktime_on = false;
+  std::vector<KRec> ktime_recs;
+  std::vector<cudaEvent_t> ktime_ev;  // 2 per record, reused after each drain
+  int64_t ktime_dropped = 0;
+
+  // losses given to zo_step are host pointers (zo_set_loss_location(ctx, 0))
+  bool host_losses = false;
+
   std::string err;
 };
 
@@ -167,11 +185,21 @@ ProbeKey probe_key(const zo_ctx *ctx);  // current perturbation (sign 0 when cle
 // which == 3 closes the step.
 void phase_mark(zo_ctx *ctx, int which);
 
+// Kernel timing: ktime_begin records the start event of a launch of a timed class and
+// returns its slot (-1 when timing is off or the record cap is reached); ktime_end records
+// the end event after the launch, with the class and the launch's algorithmic work.
+int ktime_begin(zo_ctx *ctx);
+void ktime_end(zo_ctx *ctx, int slot, int cls, double work);
+
+// zo_step's body for device-resident losses (what the step drivers call).
+zo_status step_device(zo_ctx *ctx, const double *loss_plus, const double *loss_minus, int32_t n_pert,
+                      const double *loss0, float lr, float eps, float damping);
+
 // Launchers (each enqueues on ctx->stream and returns the launch status).
 zo_status launch_perturb(zo_ctx *ctx, const ProbeKey &pk, int64_t first, int64_t count,
                          void *out);
-zo_status launch_pack(zo_ctx *ctx, uint32_t probe, int64_t first_byte, int64_t nbytes,
-                      uint8_t *out);
+zo_status launch_pack(zo_ctx *ctx, uint32_t step, uint32_t probe, int64_t first_byte,
+                      int64_t nbytes, uint8_t *out);
 zo_status launch_quad_loss(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *out,
                            int accumulate, double *partials, unsigned int *counter);
 zo_status launch_quad_loss_pair(zo_ctx *ctx, const ProbeKey &pk, const float *D, double *out_plus,

@@ -245,13 +245,13 @@ perturb_pipe_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t fi
 // bit t <-> element 8q+t): one thread per 16-element group, i.e. per 2 output bytes.
 // Bits of elements >= M are cleared.
 __global__ void pack_kernel(uint8_t *__restrict__ out, int64_t first_byte, int64_t nbytes,
-                            int64_t M, uint32_t probe, const uint32_t *step_ptr, uint32_t k0,
-                            uint32_t k1, uint64_t g_off) {
+                            int64_t M, uint32_t probe, uint32_t step, uint32_t k0, uint32_t k1,
+                            uint64_t g_off) {
   const int64_t gfirst = first_byte / 2;
   const int64_t glast = (first_byte + nbytes - 1) / 2;
   const int64_t g = gfirst + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (g > glast) return;
-  const uint32_t m = probe_group_bits((uint64_t)g + g_off, probe, *step_ptr, k0, k1);
+  const uint32_t m = probe_group_bits((uint64_t)g + g_off, probe, step, k0, k1);
   for (int q = 0; q < 2; ++q) {
     const int64_t byte = g * 2 + q;
     if (byte < first_byte || byte >= first_byte + nbytes) continue;
@@ -281,9 +281,21 @@ zo_status launch_pipe(zo_ctx *ctx, const ProbeKey &pk, int64_t first, int64_t co
   return check_launch(ctx, "perturb_pipe_kernel");
 }
 
+zo_status launch_perturb_impl(zo_ctx *ctx, const ProbeKey &pk, int64_t first, int64_t count,
+                              void *out);
+
+// Timed as ZO_KT_PERTURB with its algorithmic bytes: theta read and the window written once.
 zo_status launch_perturb(zo_ctx *ctx, const ProbeKey &pk, int64_t first, int64_t count,
                          void *out) {
   if (count <= 0) return ZO_OK;
+  const int slot = ktime_begin(ctx);
+  const zo_status st = launch_perturb_impl(ctx, pk, first, count, out);
+  if (st == ZO_OK) ktime_end(ctx, slot, ZO_KT_PERTURB, 2.0 * (ctx->dtype == ZO_F32 ? 4 : 2) * (double)count);
+  return st;
+}
+
+zo_status launch_perturb_impl(zo_ctx *ctx, const ProbeKey &pk, int64_t first, int64_t count,
+                              void *out) {
   const int vec = ctx->dtype == ZO_F32 ? 4 : 8;
   if (count >= kPChunk && first % vec == 0 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0)
     return ctx->dtype == ZO_F32 ? launch_pipe<float>(ctx, pk, first, count, out)
@@ -304,15 +316,15 @@ zo_status launch_perturb(zo_ctx *ctx, const ProbeKey &pk, int64_t first, int64_t
   return check_launch(ctx, "perturb_kernel");
 }
 
-zo_status launch_pack(zo_ctx *ctx, uint32_t probe, int64_t first_byte, int64_t nbytes,
-                      uint8_t *out) {
+zo_status launch_pack(zo_ctx *ctx, uint32_t step, uint32_t probe, int64_t first_byte,
+                      int64_t nbytes, uint8_t *out) {
   if (nbytes <= 0) return ZO_OK;
   const int64_t groups = (first_byte + nbytes - 1) / 2 - first_byte / 2 + 1;
   const int threads = 256;
   const int64_t blocks = (groups + threads - 1) / threads;
   ProbeKey pk = probe_key(ctx);
   pack_kernel<<<(unsigned)blocks, threads, 0, ctx->stream>>>(
-      out, first_byte, nbytes, ctx->M, probe, &ctx->dstate->step, pk.k0, pk.k1, pk.g_off);
+      out, first_byte, nbytes, ctx->M, probe, step, pk.k0, pk.k1, pk.g_off);
   return check_launch(ctx, "pack_kernel");
 }
 

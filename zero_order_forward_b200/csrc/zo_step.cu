@@ -259,10 +259,13 @@ zo_status launch_update_t(zo_ctx *ctx, const float *coef, int n, const uint32_t 
   attr_pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr_pdl;
   cfg.numAttrs = 1;
+  const int slot = ktime_begin(ctx);
   e = cudaLaunchKernelEx(&cfg, kern, static_cast<T *>(ctx->params), ctx->M, coef, n, step_ptr,
                          ok_ptr, k0, k1, (uint64_t)(ctx->first_element / kGroup));
   if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "update_kernel: %s", cudaGetErrorString(e));
-  return check_launch(ctx, "update_kernel");
+  const zo_status st = check_launch(ctx, "update_kernel");
+  if (st == ZO_OK) ktime_end(ctx, slot, ZO_KT_UPDATE, 2.0 * sizeof(T) * (double)ctx->M);
+  return st;
 }
 
 template <typename T>

@@ -79,16 +79,28 @@ def gather_losses(local, n_pert, group=None, block=1):
     return Lp, Lm
 
 
+def batch_share(batch, rank, world):
+    """(first, count) of rank's contiguous share of `batch` sequences (count may be 0)."""
+    if not (0 <= rank < world) or batch < 0:
+        raise ValueError("bad batch partition arguments")
+    per = -(-batch // world) if batch else 0
+    first = min(batch, rank * per)
+    return first, min(batch, first + per) - first
+
+
 def probe_parallel_step(n_pert, loss_at, clean_loss, apply_step, device, dtype=torch.float64,
-                        group=None, pair_at=None, block=1, block_at=None):
+                        group=None, pair_at=None, block=1, block_at=None, clean_shared=False):
     """One step with this rank's share of the probes.
 
     loss_at(sign, probe, out) writes L(theta + sign*eps*z_probe) into the 1-element tensor
     `out`; pair_at(probe, out_plus, out_minus), if given, writes both signs at once instead;
     block_at(first, count, out_plus, out_minus), if given, writes both signs of the `count`
     probes from `first` (one block of the partition, `block` probes) at once;
-    clean_loss(out) writes L0 (every rank computes it: same theta, same data, same value, no
-    exchange); apply_step(Lp, Lm, L0) runs the preconditioner and the update.
+    clean_loss(out) writes L0: with clean_shared False every rank computes the whole clean
+    loss (same theta, same data, same value, no exchange); with clean_shared True it writes
+    this rank's partial sum over its share of the batch (batch_share), and the partials are
+    all-gathered and added in rank order, so every rank holds the same L0 bits;
+    apply_step(Lp, Lm, L0) runs the preconditioner and the update.
     Returns (L0, Lp, Lm)."""
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
@@ -98,6 +110,8 @@ def probe_parallel_step(n_pert, loss_at, clean_loss, apply_step, device, dtype=t
     local = torch.zeros((2, k), dtype=dtype, device=device)
     L0 = torch.zeros(1, dtype=dtype, device=device)
     clean_loss(L0)
+    if clean_shared:
+        L0 = sum_partials(L0, group)
     j = 0
     for first, count in rank_units(n_pert, rank, world, block):
         if block_at is not None:
