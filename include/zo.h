@@ -296,7 +296,10 @@ zo_status zo_mlp_loss(zo_ctx *ctx, const float *X, const int32_t *labels, int ba
  *   X, labels, batch, n_in, n_hidden, n_out, scale, loss_out, accumulate: as zo_mlp_loss.
  *   stream     cudaStream_t to enqueue on (NULL = legacy default stream).
  * The first call on a device looks up the scratch array's device address (once per
- * device, with that device current); make that first call before any stream capture.
+ * device and CUDA context, with that device current); make that first call before any stream
+ * capture.  The address is kept for the life of the process: after cudaDeviceReset of a
+ * device, whose context may come back with the same handle, the kept address is stale, so a
+ * process that resets a device must not call this entry point on it again.
  * Every call clears the scratch's counter before its kernel.  All calls in the process
  * share the one scratch array, which keeps the last call's contents: calls that overlap
  * on the GPU (other streams, other threads) race and must be serialised by the caller.

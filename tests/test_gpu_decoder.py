@@ -171,39 +171,77 @@ def test_decoder_rejects_bad_tokens_without_reading_out_of_range(zo):
     ctx.close()
 
 
+def _teacher_forced(bits, L, n, eps, lr, lam, seed, step=0):
+    """The oracle's preconditioner and fixed-order update fed with the given losses
+    [L0, L+..., L-...] (the GPU's): (theta', precond record)."""
+    e32 = float(np.float32(eps))
+    pc = core.precond(L[1:1 + n], L[1 + n:], L[0], e32, float(np.float32(lr)),
+                      float(np.float32(lam)), float(np.float32(0.1)))
+    return core.update_mirror(bits, pc["a"].astype(np.float32), seed, step), pc
+
+
+def _run_step(zo, cfg, bits, tokens, labels, B, S, k, n, eps, lr, lam, seed):
+    theta = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    ctx = zo.zo_create(theta, seed=seed)
+    model = zo.zo_model_create(ctx, cfg, B * S)
+    losses = torch.zeros(2 * n + 1, dtype=torch.float64, device="cuda")
+    zo.zo_model_step(model, torch.from_numpy(tokens).cuda(), torch.from_numpy(labels).cuda(),
+                     B, S, k, n, eps, lr, lam, True, losses)
+    assert zo.zo_sync(ctx) == 0
+    assert zo.zo_get_step(ctx) == 1
+    g, c, w, a = zo.zo_get_precond(ctx, n)
+    out = (theta.view(torch.int16).cpu().numpy().view(np.uint16), losses.cpu().numpy(), (g, c, w, a))
+    model.close()
+    ctx.close()
+    return out
+
+
 def test_decoder_step_matches_oracle(zo):
-    """One 1.5-SPSA step with 2 micro-batches: losses against the oracle's, and theta'
-    within the bound propagated from the measured loss discrepancy."""
+    """One 1.5-SPSA step with 2 micro-batches.  The losses match the oracle's within the bf16
+    forward's tolerance (2e-2), and, fed the GPU's own losses (teacher forcing), the oracle's
+    preconditioner gives the GPU's g, c, w, a and its fixed-order update gives the GPU's
+    theta' bit for bit: the step's arithmetic after the losses is exact, so any error in
+    the perturbation, the probe signs or the update shows up as a mismatch."""
     cfg = TINY[0]
     B, S, n_micro, n, eps, lr, lam = 2, 64, 2, 4, 1e-3, 2e-2, 1e-3
     bits = synth.opt_params(cfg, seed=1, varied=True)
-    theta = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
-    ctx = zo.zo_create(theta, seed=1)
-    model = zo.zo_model_create(ctx, cfg, B * S)
     toks, labs = zip(*(synth.opt_batch(cfg, B, S, seed=1, step=k) for k in range(n_micro)))
     tokens, labels = np.stack(toks), np.stack(labs)
-    losses = torch.zeros(2 * n + 1, dtype=torch.float64, device="cuda")
-    zo.zo_model_step(model, torch.from_numpy(tokens).cuda(), torch.from_numpy(labels).cuda(),
-                     B, S, n_micro, n, eps, lr, lam, True, losses)
-    assert zo.zo_sync(ctx) == 0
-    assert zo.zo_get_step(ctx) == 1
+    got, L, (g, c, w, a) = _run_step(zo, cfg, bits, tokens, labels, B, S, n_micro, n, eps, lr,
+                                     lam, 1)
     flat_t, flat_l = tokens.reshape(-1, S), labels.reshape(-1)
     loss = lambda Pb: oracle.opt.loss(core.bf16_to_f32(Pb), cfg, flat_t, flat_l)  # noqa: E731
-    nxt, rec = oracle.step.spsa_step(bits, loss, n, eps, lr, lam, 1, 0)
-    L = losses.cpu().numpy()
+    _, rec = oracle.step.spsa_step(bits, loss, n, eps, lr, lam, 1, 0)
     ref = np.concatenate([[rec["L0"]], rec["Lp"], rec["Lm"]])
     assert np.allclose(L, ref, rtol=2e-2, atol=0)
-    dL = np.abs(L - ref).max()
-    dg = dL / eps
-    dc = 4 * dL / eps ** 2
-    dw = 0.1 * rec["w"] * dc / (np.abs(rec["c"]) + lam)
-    da = float(np.float32(lr)) / n * (rec["w"] * dg + dw * np.abs(rec["g"]))
-    got = core.bf16_to_f32(theta.view(torch.int16).cpu().numpy().view(np.uint16)).astype(np.float64)
-    exp = core.bf16_to_f32(nxt).astype(np.float64)
-    ulp = np.spacing(np.abs(exp).astype(np.float32)).astype(np.float64) * 65536
-    assert np.all(np.abs(got - exp) <= da.sum() + 2 * ulp)
-    model.close()
-    ctx.close()
+    nxt, pc = _teacher_forced(bits, L, n, eps, lr, lam, 1)
+    assert np.array_equal(got, nxt)
+    assert np.allclose(g, pc["g"], rtol=1e-13, atol=0)
+    assert np.allclose(c, pc["c"], rtol=1e-12, atol=1e-6)
+    assert np.allclose(w, pc["w"], rtol=1e-13, atol=0)
+    assert np.array_equal(a, pc["a"].astype(np.float32))
+    assert not np.array_equal(got, bits)  # the step moved theta
+
+
+def test_c4_shaped_step_matches_oracle(zo):
+    """The OPT-1.3B workload's step structure at its real loop counts (8 micro-batches per
+    effective batch, n_pert = 160: 321 x 8 micro-forwards) on a narrow 2-layer model: every
+    loss against the oracle's (2e-2), and theta' bit for bit against the oracle's
+    preconditioner and fixed-order update fed with the GPU's losses."""
+    cfg = TINY[0]
+    B, S, k, n, eps, lr, lam = 2, 32, 8, 160, 1e-3, 1e-2, 1e-3
+    bits = synth.opt_params(cfg, seed=6, varied=True)
+    toks, labs = zip(*(synth.opt_batch(cfg, B, S, seed=6, step=j) for j in range(k)))
+    tokens, labels = np.stack(toks), np.stack(labs)
+    got, L, _ = _run_step(zo, cfg, bits, tokens, labels, B, S, k, n, eps, lr, lam, 6)
+    flat_t, flat_l = tokens.reshape(-1, S), labels.reshape(-1)
+    loss = lambda Pb: oracle.opt.loss(core.bf16_to_f32(Pb), cfg, flat_t, flat_l)  # noqa: E731
+    e32 = float(np.float32(eps))
+    ref = np.array([loss(bits)] + [loss(core.perturb(bits, 6, 0, i, s, e32))
+                                   for s in (+1, -1) for i in range(n)])
+    assert np.allclose(L, ref, rtol=2e-2, atol=0)
+    nxt, _ = _teacher_forced(bits, L, n, eps, lr, lam, 6)
+    assert np.array_equal(got, nxt)
 
 
 def test_opt125m_full_size_sampled(zo):

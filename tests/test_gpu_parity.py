@@ -128,6 +128,29 @@ def test_perturb_bit_exact_and_restore_exact(zo, M, dtype):
     ctx.close()
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("first,count", [(0, (1 << 23) + 40), (8, (1 << 23) + 5)])
+def test_perturb_window_many_chunks_per_cta(zo, dtype, first, count):
+    """A window far larger than one pass of the grid (each CTA streams several chunks through
+    its ring of stages): bit-exact against the oracle, clean and perturbed."""
+    M = first + count + 3
+    th_np = _theta(M, dtype, seed=5)
+    th = dev(th_np) if dtype == "f32" else bf16_dev(th_np)
+    ctx = zo.zo_create(th, seed=13)
+    zo.zo_set_step(ctx, 2)
+    out = torch.empty(count, dtype=th.dtype, device="cuda")
+    zo.zo_perturb_range(ctx, first, count, out)
+    torch.cuda.synchronize()
+    assert (host_bits(out) == host_bits(th)[first:first + count]).all()
+    zo.zo_perturb(ctx, -1, 1e-3, 21)
+    zo.zo_perturb_range(ctx, first, count, out)
+    torch.cuda.synchronize()
+    zo.zo_restore(ctx)
+    ref = core.perturb(th_np, 13, 2, 21, -1, 1e-3)
+    assert (host_bits(out) == ref[first:first + count]).all()
+    ctx.close()
+
+
 def test_live_buffer_switches_back_on_restore(zo):
     M = 19210
     th_np = _theta(M, "f32")
@@ -210,8 +233,10 @@ def test_mlp_loss_matches_oracle(zo):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("n", [1, 7, 8, 13, 64, 160])
-@pytest.mark.parametrize("M", [1, 127, 129, 19210, (1 << 20) + 77])
+@pytest.mark.parametrize("n,M", [(n, M) for n in (1, 7, 8, 13, 64, 160)
+                                  for M in (1, 127, 129, 19210, (1 << 20) + 77)] +
+                         # many chunks per CTA: the streaming ring wraps around several times
+                         [(16, (1 << 24) + 77), (17, (1 << 24) + 3)])
 def test_update_bit_exact_vs_mirror_order(zo, M, n, dtype):
     th_np = _theta(M, dtype, seed=M + n)
     th = dev(th_np) if dtype == "f32" else bf16_dev(th_np)

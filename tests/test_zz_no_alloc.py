@@ -30,13 +30,23 @@ def test_noalloc_matches_context_entry_point_on_two_calls(zo):
     ref = torch.zeros(1, dtype=torch.float64, device="cuda")
     zo.zo_mlp_loss(ctx, X, y, batch, 64, 256, 10, 1.0 / batch, ref)
     out = torch.full((2,), -1.0, dtype=torch.float64, device="cuda")
+    # a first call loads whatever the driver loads lazily for this code; the memory check
+    # covers the calls after it
+    zo.zo_mlp_loss_noalloc(P, X, y, batch, 64, 256, 10, 1.0 / batch, out[0:1])
+    torch.cuda.synchronize()
+    torch_before = torch.cuda.memory_allocated()
+    free_before, _ = torch.cuda.mem_get_info()
     # two calls in a row share the static scratch (the counter is re-armed each call)
     zo.zo_mlp_loss_noalloc(P, X, y, batch, 64, 256, 10, 1.0 / batch, out[0:1])
     zo.zo_mlp_loss_noalloc(P, X, y, batch, 64, 256, 10, 1.0 / batch, out[1:2])
     torch.cuda.synchronize()
+    # nothing was allocated, by torch or by the library
+    assert torch.cuda.memory_allocated() == torch_before
+    assert torch.cuda.mem_get_info()[0] == free_before
     r = ref.item()
     got = out.cpu().numpy()
-    assert np.all(np.abs(got - r) <= 1e-5 * abs(r)), (got, r)
+    # the same kernel in the same reduction order as the context's entry point: equal bits
+    assert np.all(got == r), (got, r)
     # accumulate mode on the second call of another pair
     acc = torch.zeros(1, dtype=torch.float64, device="cuda")
     zo.zo_mlp_loss_noalloc(P, X[:32], y[:32], 32, 64, 256, 10, 1.0 / batch, acc)

@@ -294,7 +294,9 @@ def zo_mlp_losses(ctx, X, labels, batch, n_in, n_hidden, n_out, n_pert, eps, sca
 def zo_mlp_loss_noalloc(P, X, labels, batch, n_in, n_hidden, n_out, scale, loss_out,
                         accumulate=False, stream=None):
     """MLP loss for callers that cannot allocate device memory (see include/zo.h): no
-    context, scratch in the library's static device memory.  Raises ZoError on failure."""
+    context, scratch in the library's static device memory.  stream=None enqueues on
+    torch.cuda.current_stream(); stream=0 passes NULL, the legacy default stream.  Raises
+    ZoError on failure."""
     st = _L.zo_mlp_loss_noalloc(_ptr(P), _ptr(X), _ptr(labels), batch, n_in, n_hidden, n_out,
                                 scale, _ptr(loss_out), int(accumulate), _stream(stream))
     if st != ZO_OK:

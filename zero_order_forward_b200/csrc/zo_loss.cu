@@ -983,29 +983,57 @@ namespace zo {
 namespace {
 
 constexpr size_t kNoallocPartialsBytes = (size_t)ZO_NOALLOC_MAX_BATCH * sizeof(double);
-constexpr int kNoallocMaxDevices = 64;
+constexpr int kNoallocMaxEntries = 64;
 
 // [0, kNoallocPartialsBytes): fp64 partials; then the unsigned ticket counter.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocPartialsBytes + 256];
 
+// The array's device address, looked up once per (device, CUDA context): a caller that makes
+// a context of its own current gets that context's copy of the array.
+struct NoallocEntry {
+  int device;
+  void *context;
+  void *addr;
+};
 std::mutex g_noalloc_mu;
-void *g_noalloc_addr[kNoallocMaxDevices] = {};
+NoallocEntry g_noalloc_cache[kNoallocMaxEntries];
+int g_noalloc_used = 0;
 
-// Device address of the scratch on the current device.  In host code the array's name is
-// only a host-side stand-in, so the address is looked up once per device.
+using CtxGetCurrentFn = int (*)(void **);  // cuCtxGetCurrent(CUcontext *)
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// Device address of the scratch in the current device's current context.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up (once per device
+// and context, with that device current) with cudaGetSymbolAddress.
 cudaError_t noalloc_scratch(void **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kNoallocMaxDevices) return cudaErrorInvalidDevice;
+  void *context = nullptr;
+  if (CtxGetCurrentFn fn = ctx_get_current()) fn(&context);
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
-    void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_noalloc_addr[dev] = p;
-  }
-  *out = g_noalloc_addr[dev];
+  for (int i = 0; i < g_noalloc_used; ++i)
+    if (g_noalloc_cache[i].device == dev && g_noalloc_cache[i].context == context) {
+      *out = g_noalloc_cache[i].addr;
+      return cudaSuccess;
+    }
+  void *p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess) return e;
+  if (g_noalloc_used < kNoallocMaxEntries) g_noalloc_cache[g_noalloc_used++] = {dev, context, p};
+  *out = p;
   return cudaSuccess;
 }
 

@@ -111,10 +111,11 @@ perturb_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t first, 
 
 // Pipelined form for 16-byte-aligned windows (first % (16 / sizeof(T)) == 0, out 16-byte
 // aligned): chunks of 256 groups (4096 elements, aligned to groups in the global index)
-// stream through a ring of shared-memory stages.  Warp 0 issues the bulk copy of a chunk;
-// 8 consumer warps each regenerate the bits of the 32 groups they write (one Philox block
-// per lane, shared by warp shuffles), apply the perturbation and write the window with
-// 16-byte stores.
+// stream through a ring of shared-memory stages.  Warp 0 issues the bulk copy of a chunk
+// into a stage; 8 consumer warps each regenerate the bits of the 32 groups of their slice
+// (one Philox block per lane, shared by warp shuffles), apply the perturbation in place in
+// the stage and write the slice back with one bulk copy, so that both directions move in
+// large asynchronous transfers.
 constexpr int kPChunk = kTileElems;  // 4096
 constexpr int kPStages = 6;
 constexpr int kPConsumers = 8;
@@ -186,9 +187,14 @@ perturb_pipe_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t fi
       }
     }
   } else {
-    const int ct = threadIdx.x - 32;
-    const int cw = ct >> 5;  // consumer warp: vectors (32 cw + lane + 256 k) N of the chunk
-    int it = 0;
+    // Consumer warp cw owns the contiguous slice [cw * kSlice, (cw + 1) * kSlice) of each
+    // chunk: its 32 sign groups (one Philox block per lane) are transformed in place in the
+    // stage, and one bulk store writes the slice's in-window part to the output.  The stage
+    // is released one iteration later, once that store has finished reading it.
+    constexpr int kSlice = kPChunk / kPConsumers;  // 512 elements = 32 groups
+    const int cw = warp - 1;
+    int it = 0, prev_s = -1;
+    bool ok_all = true;
     for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
       const int s = it % kPStages;
       const uint32_t ph = (uint32_t)(it / kPStages) & 1u;
@@ -198,45 +204,57 @@ perturb_pipe_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t fi
       if (ok && lane != 0) ok = tc::mbar_wait(&full[s], ph) ? 1 : 0;
       if (!__all_sync(0xFFFFFFFFu, ok)) {
         if (lane == 0) { atomicOr(err, ZO_FLAG_TIMEOUT); abort_flag = 1; }
+        ok_all = false;
         break;
       }
-      const uint8_t *st = psm + s * SM::kStage;
+      uint8_t *st = psm + s * SM::kStage;
       const int64_t cs = (g0 + c * kTileGroups) * kGroup;
       const int64_t vs = cs > first ? cs : first;
       const int64_t ve = cs + kPChunk < end ? cs + kPChunk : end;
       const int64_t copy_end = vs + ((ve - vs) & ~(int64_t)(N - 1));
-      // The warp's 32 groups: slot q = 2N k + j is group 2N cw + 16N k + j of the chunk.
+      const int64_t ws = cs + (int64_t)cw * kSlice;  // this warp's slice
       uint32_t mine = 0u;
       if (pk.sign)
-        mine = probe_group_bits(pk.g_off + (uint64_t)(g0 + c * kTileGroups) + 2 * N * cw +
-                                    16 * N * (lane / (2 * N)) + lane % (2 * N),
-                                pk.probe, step, pk.k0, pk.k1);
+        mine = probe_group_bits(pk.g_off + (uint64_t)(ws / kGroup) + lane, pk.probe, step, pk.k0, pk.k1);
 #pragma unroll
-      for (int k = 0; k < kPChunk / (N * 32 * kPConsumers); ++k) {
-        const int e_rel = (ct + k * 32 * kPConsumers) * N;
-        const int64_t e = cs + e_rel;
+      for (int k = 0; k < kSlice / (N * 32); ++k) {
+        const int v = lane + 32 * k;  // vector of the slice
+        const int64_t e = ws + (int64_t)v * N;
         const uint32_t bits =
-            pk.sign ? __shfl_sync(0xFFFFFFFFu, mine, 2 * N * k + lane * N / 16) >> ((lane * N) & 15)
-                    : 0u;
+            pk.sign ? __shfl_sync(0xFFFFFFFFu, mine, (v * N) >> 4) >> ((v * N) & 15) : 0u;
         if (e + N <= vs || e >= ve) continue;
         if (e >= vs && e + N <= copy_end) {
-          uint4 v = *reinterpret_cast<const uint4 *>(st + (int64_t)e_rel * (int64_t)sizeof(T));
-          if (pk.sign) v = apply_vec(v, bits, delta, (T *)nullptr);
-          *reinterpret_cast<uint4 *>(out + (e - first)) = v;
-        } else {
+          uint4 *p = reinterpret_cast<uint4 *>(st + (e - cs) * (int64_t)sizeof(T));
+          if (pk.sign) *p = apply_vec(*p, bits, delta, (T *)nullptr);
+        } else {  // the window's last < N elements: plain loads and stores
 #pragma unroll
           for (int t = 0; t < N; ++t) {
             const int64_t et = e + t;
             if (et >= first && et < end) {
-              T v = theta[et];
-              if (pk.sign) v = apply_one(v, (bits >> t) & 1u, delta);
-              out[et - first] = v;
+              T x = theta[et];
+              if (pk.sign) x = apply_one(x, (bits >> t) & 1u, delta);
+              out[et - first] = x;
             }
           }
         }
       }
+      tc::fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&empty[s]);
+      if (lane == 0) {
+        const int64_t b0 = ws > vs ? ws : vs;
+        const int64_t b1 = ws + kSlice < copy_end ? ws + kSlice : copy_end;
+        if (b1 > b0)
+          tc::bulk_store(out + (b0 - first), st + (b0 - cs) * (int64_t)sizeof(T),
+                         (uint32_t)((b1 - b0) * (int64_t)sizeof(T)));
+        tc::bulk_commit();      // one group per iteration (possibly empty)
+        tc::bulk_wait_read1();  // the previous iteration's store has read its stage
+        if (prev_s >= 0) tc::mbar_arrive(&empty[prev_s]);
+      }
+      prev_s = s;
+    }
+    if (lane == 0) {
+      tc::bulk_wait0();  // every store of this warp has landed
+      if (ok_all && prev_s >= 0) tc::mbar_arrive(&empty[prev_s]);
     }
   }
 }

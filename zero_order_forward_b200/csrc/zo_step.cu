@@ -115,6 +115,13 @@ template <> struct Elem<float> {
     for (int k = 0; k < 4; ++k)
       reinterpret_cast<float4 *>(p)[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
   }
+  __device__ static void load16s(const float *p, float v[16]) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 x = reinterpret_cast<const float4 *>(p)[k];
+      v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
+    }
+  }
   __device__ static float get(const float *p, int64_t i) { return p[i]; }
   __device__ static void put(float *p, int64_t i, float v) { p[i] = v; }
 };
@@ -142,14 +149,24 @@ template <> struct Elem<uint16_t> {
       reinterpret_cast<uint4 *>(p)[k] = make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
+  __device__ static void load16s(const uint16_t *p, float v[16]) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const uint4 x = reinterpret_cast<const uint4 *>(p)[k];
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        v[8 * k + 2 * t] = __uint_as_float(w[t] << 16);
+        v[8 * k + 2 * t + 1] = __uint_as_float(w[t] & 0xFFFF0000u);
+      }
+    }
+  }
   __device__ static float get(const uint16_t *p, int64_t i) { return bf16_bits_to_f32(p[i]); }
   __device__ static void put(uint16_t *p, int64_t i, float v) { p[i] = f32_to_bf16_bits(v); }
 };
 
-constexpr int kUpdThreads = 1024;
-
-// theta <- rd(theta - sum_i coef_i z_i).  One thread per 16-element group: for each probe
-// octet it computes the group's Philox block, whose byte b holds the octet's 8 signs of
+// theta <- rd(theta - sum_i coef_i z_i).  One consumer thread per 16-element group: for each
+// probe octet it computes the group's Philox block, whose byte b holds the octet's 8 signs of
 // element b, and adds to element b the octet's table entry for that byte.  Entry e of an
 // octet's table is the fp32 sum, left to right from its first signed term, of
 // (bit t of e ? -a : +a) over the octet's probes t; the octet sums are added in order and
@@ -157,19 +174,29 @@ constexpr int kUpdThreads = 1024;
 // l mod R, so the 32 lookups of a warp meet at most 32/R to a bank (none at R = 32).  g_off is
 // the global index of the context's first group: its elements take the signs of their
 // global indices.
-template <typename T, int LOG_R>
-__global__ void __launch_bounds__(kUpdThreads)
-update_kernel(T *__restrict__ theta, int64_t M, const float *__restrict__ coef, int n,
-              const uint32_t *step_ptr, const uint32_t *ok_ptr, uint32_t k0, uint32_t k1,
-              uint64_t g_off) {
-  constexpr int R = 1 << LOG_R;
-  extern __shared__ float lut[];  // [octet][256 entries][R replicas]
-  // Launched with programmatic dependent launch: wait for the preconditioner (coefficients,
-  // step, ok flag).  This kernel never signals early, so the next kernel of the stream, which
-  // reads theta, starts only after it has completed.
-  tc::pdl_wait();
-  if (ok_ptr != nullptr && *ok_ptr == 0u) return;
-  const uint32_t step = *step_ptr;
+//
+// theta streams through shared memory: one CTA per SM; warp 0 issues bulk copies of chunks
+// of 8192 elements into a ring of stages; 16 consumer warps update their groups in place in
+// the stage and each writes its contiguous 512-element slice back with one bulk copy, so that
+// both directions move in large asynchronous transfers while the consumers regenerate the
+// probes.  The last partial vector of theta (fewer than 16 bytes) is read and written
+// directly.
+constexpr int kUConsumers = 16;
+constexpr int kUThreads = 32 * (1 + kUConsumers);
+constexpr int kUChunk = kUConsumers * 32 * kGroup;  // 8192 elements
+constexpr int kUSlice = 32 * kGroup;                // 512 elements per consumer warp
+
+template <typename T> struct UpdPipe {
+  static constexpr int kStages = sizeof(T) == 2 ? 4 : 3;
+  static constexpr int kStage = kUChunk * (int)sizeof(T);
+  static constexpr int kRing = kStages * kStage;
+  static constexpr int kLut = kRing + 2 * kStages * 8;  // after the ring and its barriers
+  static constexpr int kFixed = kLut;
+};
+
+// The octets' tables, R replicas each (all threads of the CTA take part).
+template <int LOG_R>
+__device__ __forceinline__ void build_tables(float *lut, const float *__restrict__ coef, int n) {
   const int octets = (n + 7) >> 3;
   // A warp computes 32 consecutive entries (one per lane) and writes their R replicas as
   // 32 R consecutive words, 32 per store: no bank conflicts.
@@ -185,73 +212,180 @@ update_kernel(T *__restrict__ theta, int64_t M, const float *__restrict__ coef, 
       s = __fadd_rn(s, ((b >> t) & 1) ? -a : a);
     }
 #pragma unroll
-    for (int j = 0; j < R; ++j) {
+    for (int j = 0; j < (1 << LOG_R); ++j) {
       const int word = j * 32 + lane;  // replica (word & (R-1)) of entry base + (word >> LOG_R)
       lut[(base << LOG_R) + word] = __shfl_sync(0xFFFFFFFFu, s, word >> LOG_R);
     }
   }
+}
+
+// v[e] -= (sum over octets of the table entry of element e's sign byte), fixed order.
+template <int LOG_R>
+__device__ __forceinline__ void apply_probes(float v[16], const float *mine, uint64_t g, int octets,
+                                             uint32_t step, uint32_t k0, uint32_t k1) {
+  float acc[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+  for (int o = 0; o < octets; ++o) {
+    const uint4 blk = sign_block(g, (uint32_t)o, step, k0, k1);
+    const uint32_t w[4] = {blk.x, blk.y, blk.z, blk.w};
+    const float *tab = mine + ((o * 256) << LOG_R);
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      acc[e] = __fadd_rn(acc[e], tab[((w[e >> 2] >> (8 * (e & 3))) & 0xFFu) << LOG_R]);
+  }
+#pragma unroll
+  for (int e = 0; e < 16; ++e) v[e] = __fsub_rn(v[e], acc[e]);
+}
+
+template <typename T, int LOG_R>
+__global__ void __launch_bounds__(kUThreads, 1)
+update_kernel(T *__restrict__ theta, int64_t M, const float *__restrict__ coef, int n,
+              const uint32_t *step_ptr, const uint32_t *ok_ptr, uint32_t k0, uint32_t k1,
+              uint64_t g_off, uint32_t *err) {
+  using U = UpdPipe<T>;
+  constexpr int N = 16 / (int)sizeof(T);  // elements per 16-byte vector
+  extern __shared__ __align__(128) uint8_t usm[];
+  uint64_t *full = reinterpret_cast<uint64_t *>(usm + U::kRing);
+  uint64_t *empty = full + U::kStages;
+  float *lut = reinterpret_cast<float *>(usm + U::kLut);  // [octet][256 entries][R replicas]
+  __shared__ volatile int abort_flag;
+  // Launched with programmatic dependent launch: wait for the preconditioner (coefficients,
+  // step, ok flag).  This kernel never signals early, so the next kernel of the stream, which
+  // reads theta, starts only after it has completed.
+  tc::pdl_wait();
+  if (ok_ptr != nullptr && *ok_ptr == 0u) return;
+  const uint32_t step = *step_ptr;
+  const int octets = (n + 7) >> 3;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < U::kStages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], kUConsumers);
+    }
+    abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  build_tables<LOG_R>(lut, coef, n);
   __syncthreads();
 
-  const float *mine = lut + (threadIdx.x & (R - 1));
-  const int64_t n_groups = (M + kGroup - 1) / kGroup;
-  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n_groups;
-       g += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t e0 = g * kGroup;
-    const bool whole = e0 + kGroup <= M;
-    float v[16];
-    if (whole) {
-      Elem<T>::load16(theta + e0, v);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = e0 + e < M ? Elem<T>::get(theta, e0 + e) : 0.f;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t n_chunks = (M + kUChunk - 1) / kUChunk;
+  if (warp == 0) {  // producer
+    int it = 0, issued = 0;
+    for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
+      const int s = it % U::kStages;
+      const uint32_t ph = (uint32_t)(it / U::kStages) & 1u;
+      int ok = 1;
+      if (lane == 0) ok = tc::mbar_wait(&empty[s], ph ^ 1u) ? 1 : 0;
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok || abort_flag) {
+        if (lane == 0) { atomicOr(err, ZO_FLAG_TIMEOUT); abort_flag = 1; }
+        break;
+      }
+      const int64_t cs = c * kUChunk;
+      const int64_t copy = ((M - cs < kUChunk ? M - cs : kUChunk)) & ~(int64_t)(N - 1);
+      if (lane == 0) {
+        tc::mbar_arrive_expect_tx(&full[s], (uint32_t)(copy * (int64_t)sizeof(T)));
+        if (copy > 0)
+          tc::bulk_load(usm + s * U::kStage, theta + cs, (uint32_t)(copy * (int64_t)sizeof(T)), &full[s]);
+      }
+      __syncwarp();
+      issued = it + 1;
     }
-    float acc[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-    for (int o = 0; o < octets; ++o) {
-      const uint4 blk = sign_block((uint64_t)g + g_off, (uint32_t)o, step, k0, k1);
-      const uint32_t w[4] = {blk.x, blk.y, blk.z, blk.w};
-      const float *tab = mine + ((o * 256) << LOG_R);
-#pragma unroll
-      for (int e = 0; e < 16; ++e)
-        acc[e] = __fadd_rn(acc[e], tab[((w[e >> 2] >> (8 * (e & 3))) & 0xFFu) << LOG_R]);
+    if (abort_flag && lane == 0) {  // let this CTA's loads land before it exits (bounded)
+      for (int s = 0; s < U::kStages; ++s) {
+        int last = -1;
+        for (int i = s; i < issued; i += U::kStages) last = i;
+        if (last >= 0) tc::mbar_wait(&full[s], (uint32_t)(last / U::kStages) & 1u);
+      }
     }
-#pragma unroll
-    for (int e = 0; e < 16; ++e) v[e] = __fsub_rn(v[e], acc[e]);
-    if (whole) {
-      Elem<T>::store16(theta + e0, v);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 16; ++e)
-        if (e0 + e < M) Elem<T>::put(theta, e0 + e, v[e]);
+    return;
+  }
+  // consumers: thread ct updates group ct of each chunk; warp cw bulk-stores its slice
+  const int ct = threadIdx.x - 32, cw = warp - 1;
+  const float *mine = lut + (lane & ((1 << LOG_R) - 1));
+  int it = 0, prev_s = -1;
+  bool ok_all = true;
+  for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
+    const int s = it % U::kStages;
+    const uint32_t ph = (uint32_t)(it / U::kStages) & 1u;
+    int ok = 1;
+    if (lane == 0) ok = (!abort_flag && tc::mbar_wait(&full[s], ph)) ? 1 : 0;
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    if (ok && lane != 0) ok = tc::mbar_wait(&full[s], ph) ? 1 : 0;
+    if (!__all_sync(0xFFFFFFFFu, ok)) {
+      if (lane == 0) { atomicOr(err, ZO_FLAG_TIMEOUT); abort_flag = 1; }
+      ok_all = false;
+      break;
     }
+    T *st = reinterpret_cast<T *>(usm + s * U::kStage);
+    const int64_t cs = c * kUChunk;
+    const int64_t copy_end = cs + (((M - cs < kUChunk ? M - cs : kUChunk)) & ~(int64_t)(N - 1));
+    const int64_t e0 = cs + (int64_t)ct * kGroup;
+    if (e0 < M) {
+      float v[16];
+      const bool whole = e0 + kGroup <= copy_end;
+      if (whole) {
+        Elem<T>::load16s(st + ct * kGroup, v);
+      } else {  // the last group: elements below copy_end are staged, the rest are in theta
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          v[e] = e0 + e < copy_end ? Elem<T>::get(st, e0 + e - cs)
+                                   : (e0 + e < M ? Elem<T>::get(theta, e0 + e) : 0.f);
+      }
+      apply_probes<LOG_R>(v, mine, (uint64_t)(e0 / kGroup) + g_off, octets, step, k0, k1);
+      if (whole) {
+        Elem<T>::store16(st + ct * kGroup, v);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          if (e0 + e < copy_end) Elem<T>::put(st, e0 + e - cs, v[e]);
+          else if (e0 + e < M) Elem<T>::put(theta, e0 + e, v[e]);
+        }
+      }
+    }
+    tc::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      const int64_t b0 = cs + (int64_t)cw * kUSlice;
+      const int64_t b1 = b0 + kUSlice < copy_end ? b0 + kUSlice : copy_end;
+      if (b1 > b0)
+        tc::bulk_store(theta + b0, st + (b0 - cs), (uint32_t)((b1 - b0) * (int64_t)sizeof(T)));
+      tc::bulk_commit();      // one group per iteration (possibly empty)
+      tc::bulk_wait_read1();  // the previous iteration's store has read its stage
+      if (prev_s >= 0) tc::mbar_arrive(&empty[prev_s]);
+    }
+    prev_s = s;
+  }
+  if (lane == 0) {
+    tc::bulk_wait0();  // every store of this warp has landed
+    if (ok_all && prev_s >= 0) tc::mbar_arrive(&empty[prev_s]);
   }
 }
 
-// Replicas of the tables that fit in about 160 KB of shared memory for n probes.
+// Replicas of the tables that fit beside the ring in the CTA's shared memory.
+template <typename T>
 int update_log_replicas(int n) {
   const int64_t per_replica = (int64_t)((n + 7) / 8) * 256 * 4;
+  const int64_t budget = 227 * 1024 - UpdPipe<T>::kFixed - 1024;
   int lr = 5;
-  while (lr > 0 && (per_replica << lr) > 160 * 1024) --lr;
+  while (lr > 0 && (per_replica << lr) > budget) --lr;
   return lr;
 }
 
 template <typename T, int LOG_R>
 zo_status launch_update_t(zo_ctx *ctx, const float *coef, int n, const uint32_t *step_ptr,
                           const uint32_t *ok_ptr, uint32_t k0, uint32_t k1) {
-  const size_t smem = (size_t)((n + 7) / 8) * 256 * sizeof(float) << LOG_R;
+  const size_t smem = (size_t)UpdPipe<T>::kFixed + ((size_t)((n + 7) / 8) * 256 * sizeof(float) << LOG_R);
   auto kern = update_kernel<T, LOG_R>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  int per_sm = 1;
-  if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kUpdThreads, smem);
+  // the table size varies with n: raise the limit once to the largest a CTA may use
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), 227 * 1024);
   if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "update_kernel setup: %s", cudaGetErrorString(e));
-  const int64_t n_groups = (ctx->M + kGroup - 1) / kGroup;
-  int64_t blocks = (n_groups + kUpdThreads - 1) / kUpdThreads;
-  const int64_t cap = (int64_t)kSmCount * (per_sm > 0 ? per_sm : 1);
-  if (blocks > cap) blocks = cap;
+  const int64_t n_chunks = (ctx->M + kUChunk - 1) / kUChunk;
+  const int64_t blocks = n_chunks < kSmCount ? n_chunks : kSmCount;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)blocks);
-  cfg.blockDim = dim3(kUpdThreads);
+  cfg.blockDim = dim3(kUThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = ctx->stream;
   cudaLaunchAttribute attr_pdl[1];
@@ -261,7 +395,7 @@ zo_status launch_update_t(zo_ctx *ctx, const float *coef, int n, const uint32_t 
   cfg.numAttrs = 1;
   const int slot = ktime_begin(ctx);
   e = cudaLaunchKernelEx(&cfg, kern, static_cast<T *>(ctx->params), ctx->M, coef, n, step_ptr,
-                         ok_ptr, k0, k1, (uint64_t)(ctx->first_element / kGroup));
+                         ok_ptr, k0, k1, (uint64_t)(ctx->first_element / kGroup), &ctx->dstate->flags);
   if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "update_kernel: %s", cudaGetErrorString(e));
   const zo_status st = check_launch(ctx, "update_kernel");
   if (st == ZO_OK) ktime_end(ctx, slot, ZO_KT_UPDATE, 2.0 * sizeof(T) * (double)ctx->M);
@@ -271,7 +405,7 @@ zo_status launch_update_t(zo_ctx *ctx, const float *coef, int n, const uint32_t 
 template <typename T>
 zo_status launch_update_r(zo_ctx *ctx, const float *coef, int n, const uint32_t *step_ptr,
                           const uint32_t *ok_ptr, uint32_t k0, uint32_t k1) {
-  switch (update_log_replicas(n)) {
+  switch (update_log_replicas<T>(n)) {
     case 5: return launch_update_t<T, 5>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
     case 4: return launch_update_t<T, 4>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
     case 3: return launch_update_t<T, 3>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);

@@ -136,7 +136,19 @@ __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *map, const 
       "r"(smem_addr(smem_src)), "r"(x), "r"(y)
       : "memory");
 }
+// Untiled bulk copy shared -> global (bulk async group; both addresses 16-byte aligned,
+// bytes % 16 == 0).
+__device__ __forceinline__ void bulk_store(void *gdst, const void *smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+               "r"(smem_addr(smem_src)), "r"(bytes)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// All but the most recent committed bulk group of this thread have finished reading shared
+// memory.
+__device__ __forceinline__ void bulk_wait_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
 // All committed bulk stores of this thread have finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
