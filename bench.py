@@ -1000,6 +1000,103 @@ def decoder_arm(args):
     return 0
 
 
+def kernels_arm(args):
+    """Each hot kernel of a decoder workload alone, at the workload's shapes and without the
+    model's weights (for profiling and quick measurement): the four projection GEMMs and the
+    causal attention of one micro-batch, the perturbation of one layer window, and the update
+    of a 2^30-element bf16 slice at the workload's n_pert.  L2 is flushed before every timed
+    launch.  Prints one JSON line of per-kernel timings (not the benchmark's contract line)."""
+    import torch
+
+    import zero_order_forward_b200 as zo
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    name = args.workload
+    cfg = decoder_cfg(name)
+    qwen = cfg.get("family") == "qwen3"
+    w = decoder_workload(name, args.n_pert)
+    B, S, n = w["batch"], w["seq"], w["n_pert"]
+    T, d, f, H = B * S, cfg["d_model"], cfg["d_ffn"], cfg["n_heads"]
+    Hk, e = (cfg["n_kv_heads"], cfg["head_dim"]) if qwen else (H, d // H)
+    nq, na = (H + 2 * Hk) * e, H * e
+    hbm_peak, _ = peaks()
+    peak_b, peak_s, _ = bf16_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    reps = args.steps
+
+    def timed(fn):
+        tot = 0.0
+        fn()
+        for _ in range(reps):
+            flush.zero_()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            ev[0].record(stream)
+            fn()
+            ev[1].record(stream)
+            torch.cuda.synchronize()
+            tot += ev[0].elapsed_time(ev[1])
+        return 1e3 * tot / reps
+
+    small = torch.zeros(1024, dtype=torch.bfloat16, device=dev)
+    ctx = zo.zo_create(small, seed=0, stream=stream.cuda_stream)
+    out = {}
+    shapes = ({"qkv": (T, nq, d, 0), "out": (T, d, na, 2), "gate_up": (T, f, d, 3), "down": (T, d, f, 2)}
+              if qwen else
+              {"qkv": (T, nq, d, 0), "out": (T, d, na, 2), "fc1": (T, f, d, 1), "fc2": (T, d, f, 2)})
+    A = torch.randn(T * max(K for _, _, K, _ in shapes.values()), dtype=torch.bfloat16, device=dev)
+    Wt = torch.randn(max((2 if epi == 3 else 1) * N * K for _, N, K, epi in shapes.values()),
+                     dtype=torch.bfloat16, device=dev) * 0.02
+    max_n = max(N for _, N, _, _ in shapes.values())
+    bias = torch.zeros(max_n, dtype=torch.bfloat16, device=dev)
+    out_b = torch.empty(T * max_n, dtype=torch.bfloat16, device=dev)
+    out_f = torch.zeros(T * d, dtype=torch.float32, device=dev)
+    for key, (Mm, N, K, epi) in shapes.items():
+        o = out_f if epi == 2 else out_b
+        bb = None if (epi == 3 or qwen) else bias
+        us = timed(lambda: zo.zo_gemm_bf16(ctx, A, Wt, bb, o, Mm, N, K, N, epi))
+        fl = 2.0 * Mm * N * K * (2 if epi == 3 else 1)
+        out["gemm_" + key] = {"shape": [Mm, N, K], "us": us, "tflops": fl / us / 1e6,
+                              "frac_bf16_burst": fl / us / 1e6 / peak_b}
+    del A, Wt, out_b, out_f
+    qkv = torch.randn(T * nq, dtype=torch.bfloat16, device=dev)
+    att = torch.empty(T * na, dtype=torch.bfloat16, device=dev)
+    us = timed(lambda: zo.zo_attention_gqa(ctx, qkv, att, B, S, H, Hk, e))
+    fl = 4.0 * e * B * H * S * (S + 1) / 2
+    out["attention"] = {"us": us, "tflops": fl / us / 1e6, "frac_bf16_burst": fl / us / 1e6 / peak_b}
+    del qkv, att
+    ctx.close()
+    # one layer window, perturbed
+    import synth
+    segs = (synth.qwen_segments if qwen else synth.opt_segments)(dict(cfg, n_layers=1))
+    lead = 1 if qwen else 2
+    layer = sum(c for _, c in segs[lead:-(1 if qwen else 2)])
+    th = torch.empty(layer, dtype=torch.bfloat16, device=dev).normal_(0, 0.02)
+    win = torch.empty_like(th)
+    c2 = zo.zo_create(th, seed=0, stream=stream.cuda_stream)
+    zo.zo_perturb(c2, +1, 1e-3, 3)
+    us = timed(lambda: zo.zo_perturb_range(c2, 0, layer, win))
+    zo.zo_restore(c2)
+    gb = 4.0 * layer / (us * 1e-6) / 1e9
+    out["perturb_window"] = {"elements": layer, "us": us, "GBps": gb, "frac_hbm": gb / hbm_peak}
+    c2.close()
+    del th, win
+    # the update at this n_pert on a 2^30-element bf16 slice
+    Mu = 1 << 30
+    th = torch.empty(Mu, dtype=torch.bfloat16, device=dev).normal_(0, 0.02)
+    c3 = zo.zo_create(th, seed=0, stream=stream.cuda_stream)
+    coef = torch.zeros(n, dtype=torch.float32, device=dev)
+    us = timed(lambda: zo.zo_update(c3, coef, n))
+    gb = 4.0 * Mu / (us * 1e-6) / 1e9
+    out["update"] = {"elements": Mu, "n_pert": n, "us": us, "GBps": gb, "frac_hbm": gb / hbm_peak}
+    zo.zo_sync(c3)
+    c3.close()
+    print(json.dumps({"kernels_only": name, "batch": B, "seq": S, "reps": reps,
+                      "l2": "flushed before every timed launch", "kernels": out}), flush=True)
+    return 0
+
+
 def decoder_cpu_baseline(name, cfg, w, fwds):
     """The oracle's fp64 forward of one layer at the real width (1 x 64 tokens, vocabulary
     cut to 4096: it only feeds the embedding gather and the 2-row head), one thread; the full
@@ -1215,6 +1312,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=["quadratic", "mlp", "lowrank"] + sorted(DECODER_WORKLOADS))
     ap.add_argument("--n-pert", type=int, default=None, help="override n_pert (decoder workloads)")
+    ap.add_argument("--kernels-only", action="store_true",
+                    help="time each hot kernel of a decoder workload alone at its shapes "
+                         "(--steps = timed launches per kernel); prints a diagnostic line")
     args = ap.parse_args()
     if args.steps is None:
         args.steps = 3 if args.workload in DECODER_WORKLOADS else 300
@@ -1222,6 +1322,10 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return reference_arm(args)
+    if args.kernels_only:
+        if args.workload not in DECODER_WORKLOADS:
+            ap.error("--kernels-only needs a decoder workload")
+        return kernels_arm(args)
     if args.workload == "mlp":
         return mlp_arm(args)
     if args.workload == "lowrank":

@@ -37,7 +37,10 @@ def ctx(zo):
 
 
 GEMM_SHAPES = [(128, 128, 64), (256, 384, 256), (300, 200, 72), (129, 136, 8),
-               (2048, 2560, 512), (4096, 768, 768)]
+               (2048, 2560, 512), (4096, 768, 768),
+               # at least 148 tiles of 256 x 256: the CTA-pair kernel (cta_group::2), also
+               # with M, N and K off the tile grid
+               (4096, 2560, 512), (4000, 2600, 520), (2304, 4352, 1024)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)

@@ -307,6 +307,229 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   }
 }
 
+// ------------------------------------------------------------------ CTA-pair form (cta_group::2)
+// For the large projections: clusters of 2 CTAs on neighbouring SMs compute 256 x 256 tiles
+// (SwiGLU: 256 rows x 128 output columns).  Each CTA holds its 128 A rows and its 128 of the
+// 256 B rows per stage (32 KB instead of 48 KB per SM and stage), so the shared-memory traffic
+// per MMA is two thirds of the single-CTA form's.  Warp 0 of each CTA loads its halves into
+// its own stages, the bytes completing the leader's (CTA 0's) full barrier; one thread of the
+// leader issues tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16) and commits each stage and
+// each finished accumulator to the barriers of both CTAs; the 8 epilogue warps of each CTA
+// read their own tensor memory (their 128 rows) exactly as in the single-CTA form and release
+// the accumulator on the leader's barrier.
+constexpr int kPairBN = 256;  // accumulator columns of a pair tile (the MMA's N)
+
+template <int STAGES>
+struct PairSmem {
+  static constexpr uint32_t kABytes = kBM * kBK * 2;          // this CTA's 128 rows of A
+  static constexpr uint32_t kBBytes = (kPairBN / 2) * kBK * 2;  // this CTA's 128 rows of B
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  static constexpr uint32_t kOutOffset = STAGES * kStageBytes;  // 1024-aligned
+  static constexpr uint32_t kBarOffset = kOutOffset + kEpiWarps * kStageTile;
+  static constexpr uint32_t kBytes = kBarOffset + 256 + 1024;
+};
+
+__device__ __forceinline__ TileCoord pair_tile_coord(int t, int num_m, int num_n, int out_bn) {
+  const TileCoord c = tile_coord(t, num_m, num_n, out_bn);
+  return {c.m0 / kBM * (2 * kBM), c.n0};  // tile_coord's row tiles are pair tiles of 256 rows
+}
+
+template <int STAGES, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const __grid_constant__ CUtensorMap tmC, GemmArgs args) {
+  using S = PairSmem<STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + STAGES * S::kABytes;
+  uint8_t *sOut = smem + S::kOutOffset;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + S::kBarOffset);  // used in the leader
+  uint64_t *empty = full + STAGES;
+  uint64_t *acc_full = empty + STAGES;  // [2]
+  uint64_t *acc_empty = acc_full + 2;   // [2] used in the leader: both CTAs' epilogue warps
+  uint64_t *mma_done = acc_empty + 2;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+  constexpr bool kSwiGLU = EPI == ZO_EPI_SWIGLU_BF16;
+  constexpr int OUT_BN = kSwiGLU ? kPairBN / 2 : kPairBN;  // output columns per tile
+  const uint32_t rank = tc::cluster_ctarank();
+  const bool leader = rank == 0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int num_m = (args.M + 2 * kBM - 1) / (2 * kBM), num_n = (args.N + OUT_BN - 1) / OUT_BN;
+  const int num_tiles = num_m * num_n;
+  const int nk = (args.K + kBK - 1) / kBK;
+  const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&acc_full[b], 1);
+      tc::mbar_init(&acc_empty[b], 2 * kEpiWarps);  // the epilogue warps of both CTAs
+    }
+    tc::mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) tc::tmem_alloc_pair(tmem_holder, 2 * kPairBN);
+  tc::tc_fence_before();
+  tc::cluster_sync();  // both CTAs' barriers initialised and tensor memory allocated
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t full_leader = tc::map_to_rank(full, 0);
+  const uint32_t acc_empty_leader = tc::map_to_rank(acc_empty, 0);
+  const uint32_t abort_peer = tc::map_to_rank(const_cast<int *>(abort_flag), rank ^ 1u);
+  auto raise_abort = [&]() {
+    atomicOr(args.err, ZO_FLAG_TIMEOUT);
+    *abort_flag = 1;
+    tc::st_remote_u32(abort_peer, 1u);
+  };
+
+  uint32_t issued = 0;  // producer: k-blocks issued (global ring position)
+  if (warp == 0 && lane == 0) {
+    tc::tma_prefetch_desc(&tmA);
+    tc::tma_prefetch_desc(&tmB);
+    for (int t = cluster; t < num_tiles && !*abort_flag; t += n_clusters) {
+      const TileCoord tc0 = pair_tile_coord(t, num_m, num_n, OUT_BN);
+      // SwiGLU: CTA 0 loads the tile's gate rows, CTA 1 the matching up rows
+      const int b_row = kSwiGLU ? (int)(rank ? args.N + tc0.n0 : tc0.n0) : tc0.n0 + (int)rank * (kPairBN / 2);
+      for (int kb = 0; kb < nk; ++kb) {
+        const uint32_t s = issued % STAGES, ph = (issued / STAGES) & 1u;
+        if (*abort_flag || !tc::mbar_wait(&empty[s], ph ^ 1u)) {
+          raise_abort();
+          break;
+        }
+        if (leader) tc::mbar_arrive_expect_tx(&full[s], 2 * S::kStageBytes);  // both CTAs' halves
+        tc::tma_load_2d_pair(sA + s * S::kABytes, &tmA, full_leader + 8u * s, kb * kBK,
+                             tc0.m0 + (int)rank * kBM);
+        tc::tma_load_2d_pair(sB + s * S::kBBytes, &tmB, full_leader + 8u * s, kb * kBK, b_row);
+        ++issued;
+      }
+    }
+  } else if (warp == 1 && lane == 0 && leader) {
+    constexpr uint32_t idesc = tc::idesc_bf16_f32(2 * kBM, kPairBN);
+    uint32_t consumed = 0;
+    int i = 0;
+    for (int t = cluster; t < num_tiles && !*abort_flag; t += n_clusters, ++i) {
+      const int b = i & 1;
+      const uint32_t aph = (uint32_t)(i >> 1) & 1u;
+      if (!tc::mbar_wait(&acc_empty[b], aph ^ 1u)) {
+        raise_abort();
+        break;
+      }
+      tc::tc_fence_after();
+      const uint32_t d = tmem + (uint32_t)(b * kPairBN);
+      for (int kb = 0; kb < nk; ++kb) {
+        const uint32_t s = consumed % STAGES, ph = (consumed / STAGES) & 1u;
+        if (*abort_flag || !tc::mbar_wait(&full[s], ph)) {
+          raise_abort();
+          break;
+        }
+        tc::tc_fence_after();
+        const uint32_t a0 = tc::smem_addr(sA + s * S::kABytes);
+        const uint32_t b0 = tc::smem_addr(sB + s * S::kBBytes);
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k)
+          tc::mma_bf16_pair(d, tc::smem_desc_k128(a0 + 32 * k), tc::smem_desc_k128(b0 + 32 * k), idesc,
+                            (kb | k) != 0 ? 1u : 0u);
+        tc::mma_commit_pair(&empty[s]);
+        ++consumed;
+      }
+      if (*abort_flag) break;
+      tc::mma_commit_pair(&acc_full[b]);
+    }
+    tc::mma_commit_pair(mma_done);  // arrives (in both CTAs) once every MMA above has retired
+  } else if (warp >= 2) {
+    const int q = warp & 3;           // TMEM lanes 32q..32q+31 (this warp's rows)
+    const int half = (warp - 2) / 4;  // which half of the output columns
+    const int cbeg = half * (OUT_BN / 2), cend = cbeg + OUT_BN / 2;
+    uint8_t *stage = sOut + (warp - 2) * kStageTile;
+    if (lane == 0) tc::tma_prefetch_desc(&tmC);
+    int i = 0;
+    for (int t = cluster; t < num_tiles; t += n_clusters, ++i) {
+      const int b = i & 1;
+      const uint32_t aph = (uint32_t)(i >> 1) & 1u;
+      int ok = 1;
+      if (lane == 0) ok = (!*abort_flag && tc::mbar_wait(&acc_full[b], aph)) ? 1 : 0;
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (ok && lane != 0) ok = tc::mbar_wait(&acc_full[b], aph) ? 1 : 0;
+      if (!__all_sync(0xFFFFFFFFu, ok)) {
+        if (lane == 0) raise_abort();
+        break;
+      }
+      tc::tc_fence_after();
+      const TileCoord tc0 = pair_tile_coord(t, num_m, num_n, OUT_BN);
+      const int row0 = tc0.m0 + (int)rank * kBM + q * 32;
+      const uint32_t base = tmem + (uint32_t)(b * kPairBN) + ((uint32_t)(q * 32) << 16);
+#pragma unroll 1
+      for (int c0 = cbeg; c0 < cend; c0 += 32) {
+        if (tc0.n0 + c0 >= args.N) break;
+        float v[32];
+        tc::tmem_ld32(base + (uint32_t)c0, v);
+        if (kSwiGLU) {
+          float u[32];
+          tc::tmem_ld32(base + (uint32_t)(kPairBN / 2 + c0), u);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) v[k] = silu_mul(v[k], u[k]);
+        } else {
+          float bias[32];
+          load_bias32(args.bias, tc0.n0 + c0, args.N, bias);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            v[k] = __fadd_rn(v[k], bias[k]);
+            if (EPI == ZO_EPI_RELU_BF16) v[k] = fmaxf(v[k], 0.f);
+          }
+        }
+        // the previous chunk's bulk store must have finished reading the staging tile
+        if (lane == 0) tc::bulk_wait_read0();
+        __syncwarp();
+        stage_row<EPI>(stage, lane, v);
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < args.M) {
+          if (EPI == ZO_EPI_RESID_F32) tc::tma_reduce_add_2d(&tmC, stage, tc0.n0 + c0, row0);
+          else tc::tma_store_2d(&tmC, stage, tc0.n0 + c0, row0);
+          tc::bulk_commit();
+        }
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) tc::mbar_arrive(&acc_empty[b]);
+        else tc::mbar_arrive_remote(acc_empty_leader + 8u * (uint32_t)b);
+      }
+    }
+    if (lane == 0) tc::bulk_wait0();  // this warp's stores and reductions have landed
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 0 && lane == 0 && *abort_flag) {
+    if (leader) {
+      // let the pair's loads still in flight land before either CTA exits (bounded)
+      for (uint32_t s = 0; s < STAGES; ++s) {
+        if (issued <= s) continue;
+        const uint32_t last = s + ((issued - 1 - s) / STAGES) * STAGES;
+        if (!tc::mbar_wait(&full[s], (last / STAGES) & 1u)) atomicOr(args.err, ZO_FLAG_TIMEOUT);
+      }
+    } else {
+      __nanosleep(1000000);  // the peer cannot observe its loads' completion: give them time
+    }
+  }
+  __syncwarp();
+  if (warp == 1) {
+    if (lane == 0 && !tc::mbar_wait(mma_done, 0)) atomicOr(args.err, ZO_FLAG_TIMEOUT);
+    __syncwarp();
+    tc::tc_fence_after();
+  }
+  tc::cluster_sync();  // no remote arrival or MMA touches either CTA after this point
+  if (warp == 1) tc::tmem_dealloc_pair(tmem, 2 * kPairBN);
+}
+
 // ------------------------------------------------------------------ host side
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -371,7 +594,43 @@ cudaError_t launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const CUten
   return cudaGetLastError();
 }
 
+template <int STAGES, int EPI>
+cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tcm,
+                        const GemmArgs &g, cudaStream_t st) {
+  using S = PairSmem<STAGES>;
+  auto kern = gemm_pair_kernel<STAGES, EPI>;
+  {
+    const cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), (int)S::kBytes);
+    if (e != cudaSuccess) return e;
+  }
+  constexpr int OUT_BN = EPI == ZO_EPI_SWIGLU_BF16 ? kPairBN / 2 : kPairBN;
+  const int tiles = ((g.M + 2 * kBM - 1) / (2 * kBM)) * ((g.N + OUT_BN - 1) / OUT_BN);
+  const int clusters = tiles < kSmCount / 2 ? tiles : kSmCount / 2;
+  kern<<<2 * clusters, kGemmThreads, S::kBytes, st>>>(ta, tb, tcm, g);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+zo_status launch_gemm_pair(zo_ctx *ctx, const void *A, const void *B, const void *bias, void *out,
+                           int M, int N, int K, int ldo, int epi) {
+  const int NB = epi == ZO_EPI_SWIGLU_BF16 ? 2 * N : N;
+  CUtensorMap ta, tb, tcm;
+  if (!make_map(&ta, A, M, K, kBM) || !make_map(&tb, B, NB, K, kPairBN / 2) ||
+      !make_out_map(&tcm, out, M, N, ldo, epi == ZO_EPI_RESID_F32))
+    return fail(ctx, ZO_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
+  GemmArgs g{M, N, K, static_cast<const uint16_t *>(bias), out, ldo, &ctx->dstate->flags, 0u};
+  const int slot = ktime_begin(ctx);
+  cudaError_t e;
+  if (epi == ZO_EPI_BIAS_BF16) e = launch_pair<6, ZO_EPI_BIAS_BF16>(ta, tb, tcm, g, ctx->stream);
+  else if (epi == ZO_EPI_RELU_BF16) e = launch_pair<6, ZO_EPI_RELU_BF16>(ta, tb, tcm, g, ctx->stream);
+  else if (epi == ZO_EPI_RESID_F32) e = launch_pair<6, ZO_EPI_RESID_F32>(ta, tb, tcm, g, ctx->stream);
+  else e = launch_pair<6, ZO_EPI_SWIGLU_BF16>(ta, tb, tcm, g, ctx->stream);
+  if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "gemm (CTA pairs) launch: %s", cudaGetErrorString(e));
+  ctx->launches += 1;
+  ktime_end(ctx, slot, ZO_KT_GEMM, 2.0 * M * (double)NB * K);
+  return ZO_OK;
+}
 
 zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bias, void *out,
                       int M, int N, int K, int ldo, int epi, uint32_t extra_tx) {
@@ -384,6 +643,10 @@ zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bia
   const bool swiglu = epi == ZO_EPI_SWIGLU_BF16;
   if (swiglu && bias) return fail(ctx, ZO_ERR_INVALID, "gemm: the SwiGLU epilogue takes no bias");
   const int NB = swiglu ? 2 * N : N;  // rows of B, = accumulator columns over all tiles
+  // CTA pairs for shapes that give every cluster at least two 256 x 256 tiles
+  const int64_t pair_tiles = (int64_t)((M + 255) / 256) * ((NB + 255) / 256);
+  if (extra_tx == 0 && M >= 256 && NB >= 256 && pair_tiles >= (int64_t)kSmCount)
+    return launch_gemm_pair(ctx, A, B, bias, out, M, N, K, ldo, epi);
   // N <= 128 tiles use BN = 128 to fill the machine on narrow outputs.
   const bool wide = NB > 128 && ((int64_t)((M + 127) / 128) * ((NB + 255) / 256) >= kSmCount);
   const int box_b = (wide ? 256 : 128) / (swiglu ? 2 : 1);
