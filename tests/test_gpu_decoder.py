@@ -94,6 +94,27 @@ def test_attention_matches_numpy(zo, ctx, B, S, H, d):
     assert np.max(np.abs(f64(out) - ref)) <= 2e-2
 
 
+@pytest.mark.parametrize("B,S,H,d", [(2, 300, 2, 256), (1, 256, 2, 128)])
+def test_attention_rescaling_matches_numpy(zo, ctx, B, S, H, d):
+    """Scores that grow along the keys (k_j = mean(q) * j / 2 plus noise: about 2^16 from one
+    64-key tile to the next), so that the running maximum grows by more than 2^8 at every tile
+    and the softmax rescales O and the row sum each time (after waiting for the previous
+    tile's P V)."""
+    r = np.random.default_rng(S + d + 7)
+    hd = d // H
+    q = np.ones((B, S, H, hd)) * 2.0 / np.sqrt(hd) + 0.1 * r.standard_normal((B, S, H, hd))
+    k = q.mean(axis=1, keepdims=True) * (np.arange(S)[None, :, None, None] / 2.0) \
+        + 0.1 * r.standard_normal((B, S, H, hd))
+    v = r.standard_normal((B, S, H, hd))
+    qkv = bf16(np.stack([q, k, v], axis=2).reshape(B * S, 3 * d))
+    out = torch.zeros((B * S, d), dtype=torch.bfloat16, device="cuda")
+    zo.zo_attention(ctx, qkv, out, B, S, H, d)
+    torch.cuda.synchronize()
+    assert zo.zo_sync(ctx) == 0
+    ref = _np_attention(f64(qkv), B, S, H, d)
+    assert np.max(np.abs(f64(out) - ref)) <= 2e-2
+
+
 def test_layernorm_matches_numpy(zo, ctx):
     r = np.random.default_rng(0)
     rows, d = 37, 7168
@@ -224,6 +245,36 @@ def test_decoder_step_matches_oracle(zo):
     assert np.allclose(w, pc["w"], rtol=1e-13, atol=0)
     assert np.array_equal(a, pc["a"].astype(np.float32))
     assert not np.array_equal(got, bits)  # the step moved theta
+
+
+def test_probe_quantities_match_oracle(zo):
+    """The per-probe quantities the method consumes, as the library's preconditioner computes
+    them from its own losses (zo_get_precond), against the oracle's from its fp64 losses:
+    at the method's eps = 1e-3 every g_i = (L+ - L-)/(2 eps) with the oracle's sign and within
+    G_TOL; at eps = 1e-2, where the curvature is above the forward's rounding, every
+    c_i = (L+ + L- - 2 L0)/eps^2 within C_REL_TOL of the largest and every weight
+    w_i = (|c_i| + damping)^-0.1 within W_REL_TOL (tests/probe_tolerances.py)."""
+    from probe_tolerances import C_REL_TOL, G_TOL, W_REL_TOL
+    cfg = TINY[0]
+    B, S, n, lam = 4, 64, 8, 1e-3
+    bits = synth.opt_params(cfg, seed=1, varied=True)
+    tokens, labels = synth.opt_batch(cfg, B, S, seed=1)
+    lf = lambda Pb: oracle.opt.loss(core.bf16_to_f32(Pb).astype(np.float64), cfg, tokens, labels)  # noqa: E731
+    L0 = lf(bits)
+    for eps in (1e-3, 1e-2):
+        got, L, (g, c, w, a) = _run_step(zo, cfg, bits, tokens[None], labels[None], B, S, 1, n,
+                                         eps, 0.0, lam, 1)
+        assert np.array_equal(got, bits)  # lr = 0: theta unchanged
+        e32 = float(np.float32(eps))
+        Lp = np.array([lf(core.perturb(bits, 1, 0, i, +1, e32)) for i in range(n)])
+        Lm = np.array([lf(core.perturb(bits, 1, 0, i, -1, e32)) for i in range(n)])
+        pc = core.precond(Lp, Lm, L0, e32, 0.0, float(np.float32(lam)), float(np.float32(0.1)))
+        if eps == 1e-3:
+            assert np.all(np.sign(g) == np.sign(pc["g"])), (g, pc["g"])
+            assert np.max(np.abs(g - pc["g"])) <= G_TOL, (g, pc["g"])
+        else:
+            assert np.max(np.abs(c - pc["c"])) <= C_REL_TOL * np.max(np.abs(pc["c"])), (c, pc["c"])
+            assert np.max(np.abs(w / pc["w"] - 1)) <= W_REL_TOL, (w, pc["w"])
 
 
 def test_c4_shaped_step_matches_oracle(zo):

@@ -71,7 +71,7 @@ def test_gqa_attention_matches_numpy(zo, ctx, B, S, H, Hk, e):
 @pytest.mark.parametrize("M,N,K", [(128, 64, 64), (300, 320, 136), (1024, 1536, 512),
                                    (4096, 1024, 256),
                                    # CTA-pair tiles (>= 148 tiles of 256 x 256), ragged edges
-                                   (4096, 1280, 256), (4000, 1300, 136)])
+                                   (4096, 1280, 256), (4000, 1304, 136)])
 def test_swiglu_gemm_matches_numpy(zo, ctx, M, N, K):
     """Epilogue 3: out = silu(A Wg^T) * (A Wu^T) from one GEMM over [Wg; Wu], against fp64;
     one bf16 rounding of fp32-accumulated products (tolerance as the other bf16 outputs)."""

@@ -64,6 +64,7 @@ cudaError_t ensure_smem_limit(const void *kernel, int bytes) {
     if (d.first == kernel && d.second == dev) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e == cudaSuccess) done.emplace_back(kernel, dev);
+  else cudaGetLastError();  // reported by the caller; not left for a later launch check
   return e;
 }
 

@@ -367,7 +367,7 @@ update_kernel(T *__restrict__ theta, int64_t M, const float *__restrict__ coef, 
 template <typename T>
 int update_log_replicas(int n) {
   const int64_t per_replica = (int64_t)((n + 7) / 8) * 256 * 4;
-  const int64_t budget = 227 * 1024 - UpdPipe<T>::kFixed - 1024;
+  const int64_t budget = 226 * 1024 - UpdPipe<T>::kFixed;
   int lr = 5;
   while (lr > 0 && (per_replica << lr) > budget) --lr;
   return lr;
@@ -378,8 +378,10 @@ zo_status launch_update_t(zo_ctx *ctx, const float *coef, int n, const uint32_t 
                           const uint32_t *ok_ptr, uint32_t k0, uint32_t k1) {
   const size_t smem = (size_t)UpdPipe<T>::kFixed + ((size_t)((n + 7) / 8) * 256 * sizeof(float) << LOG_R);
   auto kern = update_kernel<T, LOG_R>;
-  // the table size varies with n: raise the limit once to the largest a CTA may use
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), 227 * 1024);
+  // the table size varies with n: raise the limit once to the largest a CTA may use (the
+  // replica budget keeps every launch within 226 KB; the kernel's static shared memory comes
+  // on top, within the 227 KB a CTA may have)
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), 226 * 1024);
   if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "update_kernel setup: %s", cudaGetErrorString(e));
   const int64_t n_chunks = (ctx->M + kUChunk - 1) / kUChunk;
   const int64_t blocks = n_chunks < kSmCount ? n_chunks : kSmCount;
