@@ -230,12 +230,12 @@ def _gather_rows_host(theta, offsets, d):
 
 def test_opt30b_full_depth_loss_and_last_hidden_state(zo):
     """The OPT-30B-shaped model at full depth (48 layers, d 7168, 29.97 B parameters) on
-    B x S = 2 x 64 tokens, clean and perturbed (+eps z_5): the loss against the oracle's
-    (2e-2 relative) and the residual stream after the 48th layer (1e-2 relative Frobenius).
-    The oracle streams the weights from the device one layer at a time (fp32 numpy forward
-    of the same bf16 weights; each layer perturbed by the oracle at its global offsets)."""
+    B x S = 2 x 64 tokens: the loss against the oracle's (2e-2 relative) and the residual
+    stream after the 48th layer (1e-2 relative Frobenius).  The oracle streams the weights from
+    the device one layer at a time (fp32 numpy forward of the same bf16 weights).  The
+    perturbation at this size is covered element by element by the window tests."""
     cfg = synth.OPT_CONFIGS["opt-30b"]
-    B, S, probe, eps, seed = 2, 64, 5, 1e-3, 7
+    B, S, seed = 2, 64, 7
     free, _ = torch.cuda.mem_get_info()
     M = oracle.opt.param_count(cfg)
     if free < M * 2 + (4 << 30):
@@ -246,54 +246,35 @@ def test_opt30b_full_depth_loss_and_last_hidden_state(zo):
     model = zo.zo_model_create(ctx, cfg, B * S)
     tokens, labels = synth.opt_batch(cfg, B, S, seed=11)
     dtok, dlab = torch.from_numpy(tokens).cuda(), torch.from_numpy(labels).cuda()
-    h = torch.empty((2, B * S, d), dtype=torch.float32, device="cuda")
-    out = torch.zeros(2, dtype=torch.float64, device="cuda")
-    zo.zo_model_hidden(model, dtok, B, S, nL, h[0])
-    zo.zo_model_loss(model, dtok, dlab, B, S, 1.0 / B, out[0:1])
-    zo.zo_perturb(ctx, +1, eps, probe)
-    zo.zo_model_hidden(model, dtok, B, S, nL, h[1])
-    zo.zo_model_loss(model, dtok, dlab, B, S, 1.0 / B, out[1:2])
-    zo.zo_restore(ctx)
+    h = torch.empty((B * S, d), dtype=torch.float32, device="cuda")
+    out = torch.zeros(1, dtype=torch.float64, device="cuda")
+    zo.zo_model_hidden(model, dtok, B, S, nL, h)
+    zo.zo_model_loss(model, dtok, dlab, B, S, 1.0 / B, out)
     assert zo.zo_sync(ctx) == 0
     got_h = h.cpu().numpy().astype(np.float64)
-    got_L = out.cpu().numpy()
+    got_L = out.item()
     model.close()
     ctx.close()
 
     lay = oracle.opt.layout(cfg)
-    e32 = float(np.float32(eps))
-    pert = lambda x, j0: core.perturb(x, seed, 0, probe, +1, e32, j0=j0)  # noqa: E731
     f32 = lambda x: core.bf16_to_f32(x).astype(np.float32)  # noqa: E731
     offE, offP = lay["E"][0], lay["Pos"][0]
-    tok_off = [offE + int(t) * d for t in tokens.ravel()]
-    pos_off = [offP + (s + 2) * d for s in range(S)]
-    E_rows, P_rows = _gather_rows_host(theta, tok_off, d), _gather_rows_host(theta, pos_off, d)
-    hs = []
-    for perturbed in (False, True):
-        e = np.stack([pert(r, o) for r, o in zip(E_rows, tok_off)]) if perturbed else E_rows
-        p = np.stack([pert(r, o) for r, o in zip(P_rows, pos_off)]) if perturbed else P_rows
-        hs.append(f32(e).reshape(B, S, d) + f32(p)[None, :, :])
+    E_rows = _gather_rows_host(theta, [offE + int(t) * d for t in tokens.ravel()], d)
+    P_rows = _gather_rows_host(theta, [offP + (s + 2) * d for s in range(S)], d)
+    hs = f32(E_rows).reshape(B, S, d) + f32(P_rows)[None, :, :]
     first = lay["L0.ln1g"][0]
     size = lay["L1.ln1g"][0] - first
     for li in range(nL):
-        off = first + li * size
-        blk = _host_window(theta, off, size)
-        for i, perturbed in enumerate((False, True)):
-            w = f32(pert(blk, off) if perturbed else blk)
-            hs[i] = oracle.opt.layer(hs[i], oracle.opt.layer_params(w, d, f), H)
-            del w
-        del blk
-    fin = lay["lnf.g"][0]
-    fin_rows = _host_window(theta, fin, 2 * d)
-    cls_off = [offE + c * d for c in cfg["class_ids"]]
-    cls_rows = _gather_rows_host(theta, cls_off, d)
-    for i, perturbed in enumerate((False, True)):
-        g = f32(pert(fin_rows, fin) if perturbed else fin_rows)
-        ec = np.stack([f32(pert(r, o) if perturbed else r) for r, o in zip(cls_rows, cls_off)])
-        ref_L = float(oracle.opt.head_losses(hs[i][:, -1, :], g[:d], g[d:], ec, labels).mean())
-        ref_h = hs[i].reshape(B * S, d).astype(np.float64)
-        err = np.linalg.norm(got_h[i] - ref_h) / np.linalg.norm(ref_h)
-        assert err <= 1e-2, (perturbed, err)
-        assert abs(got_L[i] - ref_L) <= 2e-2 * abs(ref_L), (perturbed, got_L[i], ref_L)
+        w = f32(_host_window(theta, first + li * size, size))
+        hs = oracle.opt.layer(hs, oracle.opt.layer_params(w, d, f), H)
+        del w
+    fin_rows = f32(_host_window(theta, lay["lnf.g"][0], 2 * d))
+    cls_rows = f32(_gather_rows_host(theta, [offE + c * d for c in cfg["class_ids"]], d))
+    ref_L = float(oracle.opt.head_losses(hs[:, -1, :], fin_rows[:d], fin_rows[d:], cls_rows,
+                                         labels).mean())
+    ref_h = hs.reshape(B * S, d).astype(np.float64)
+    err = np.linalg.norm(got_h - ref_h) / np.linalg.norm(ref_h)
+    assert err <= 1e-2, err
+    assert abs(got_L - ref_L) <= 2e-2 * abs(ref_L), (got_L, ref_L)
     del theta
     torch.cuda.empty_cache()

@@ -40,9 +40,10 @@ def test_noalloc_matches_context_entry_point_on_two_calls(zo):
     zo.zo_mlp_loss_noalloc(P, X, y, batch, 64, 256, 10, 1.0 / batch, out[0:1])
     zo.zo_mlp_loss_noalloc(P, X, y, batch, 64, 256, 10, 1.0 / batch, out[1:2])
     torch.cuda.synchronize()
-    # nothing was allocated, by torch or by the library
-    assert torch.cuda.memory_allocated() == torch_before
-    assert torch.cuda.mem_get_info()[0] == free_before
+    # nothing was allocated, by torch or by the library (memory may only have been released,
+    # by an unrelated tensor going out of scope)
+    assert torch.cuda.memory_allocated() <= torch_before
+    assert torch.cuda.mem_get_info()[0] >= free_before
     r = ref.item()
     got = out.cpu().numpy()
     # the same kernel in the same reduction order as the context's entry point: equal bits

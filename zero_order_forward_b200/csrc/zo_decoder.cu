@@ -234,7 +234,7 @@ layernorm_kernel(const float *__restrict__ x, const uint16_t *__restrict__ g,
     const float y0 = (v[2 * t] - mean) * rstd * __uint_as_float(gw[t] << 16) + __uint_as_float(bw[t] << 16);
     const float y1 = (v[2 * t + 1] - mean) * rstd * __uint_as_float(gw[t] & 0xFFFF0000u) +
                      __uint_as_float(bw[t] & 0xFFFF0000u);
-    o[t] = (uint32_t)f32_to_bf16_bits(y0) | ((uint32_t)f32_to_bf16_bits(y1) << 16);
+    o[t] = pack_bf16x2(y0, y1);
   }
   *reinterpret_cast<uint4 *>(y + (int64_t)blockIdx.x * d + c) = make_uint4(o[0], o[1], o[2], o[3]);
 }

@@ -87,8 +87,7 @@ __device__ __forceinline__ void stage_row(uint8_t *stage, int r, const float v[3
       uint32_t w[4];
 #pragma unroll
       for (int t = 0; t < 4; ++t)
-        w[t] = (uint32_t)f32_to_bf16_bits(v[8 * c + 2 * t]) |
-               ((uint32_t)f32_to_bf16_bits(v[8 * c + 2 * t + 1]) << 16);
+        w[t] = pack_bf16x2(v[8 * c + 2 * t], v[8 * c + 2 * t + 1]);
       *reinterpret_cast<uint4 *>(stage + r * 64 + ((c ^ ((r >> 1) & 3)) << 4)) =
           make_uint4(w[0], w[1], w[2], w[3]);
     }

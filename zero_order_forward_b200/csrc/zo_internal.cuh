@@ -90,6 +90,12 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) {
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
+// Two values rounded to bf16 (round to nearest even) and packed, lo in the low half: one
+// conversion instruction for the pair, the same bits as two f32_to_bf16_bits.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
 
 // P = rd(theta + s*eps*z) for one element given its sign bit (bit 1 -> z = -1).
 // `delta` is s*eps; the xor of the bit into the sign flips it exactly.

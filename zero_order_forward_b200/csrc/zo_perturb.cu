@@ -40,7 +40,7 @@ __device__ __forceinline__ uint4 apply_vec(uint4 v, uint32_t bits, float delta, 
                                  (bits >> (2 * t)) & 1u);
     const float hi = perturb_f32(bf16_bits_to_f32((uint16_t)(w[t] >> 16)), delta,
                                  (bits >> (2 * t + 1)) & 1u);
-    w[t] = (uint32_t)f32_to_bf16_bits(lo) | ((uint32_t)f32_to_bf16_bits(hi) << 16);
+    w[t] = pack_bf16x2(lo, hi);
   }
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
@@ -113,9 +113,9 @@ perturb_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t first, 
 // aligned): chunks of 256 groups (4096 elements, aligned to groups in the global index)
 // stream through a ring of shared-memory stages.  Warp 0 issues the bulk copy of a chunk
 // into a stage; 8 consumer warps each regenerate the bits of the 32 groups of their slice
-// (one Philox block per lane, shared by warp shuffles), apply the perturbation in place in
-// the stage and write the slice back with one bulk copy, so that both directions move in
-// large asynchronous transfers.
+// (one Philox block per lane, shared by warp shuffles), copy the slice into registers and
+// release the stage, then apply the perturbation and write the window with coalesced 16-byte
+// stores.  Several CTAs per SM keep enough loads and stores in flight.
 constexpr int kPChunk = kTileElems;  // 4096
 constexpr int kPStages = 6;
 constexpr int kPConsumers = 8;
@@ -188,44 +188,53 @@ perturb_pipe_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t fi
     }
   } else {
     // Consumer warp cw owns the contiguous slice [cw * kSlice, (cw + 1) * kSlice) of each
-    // chunk: its 32 sign groups (one Philox block per lane) are transformed in place in the
-    // stage, and one bulk store writes the slice's in-window part to the output.  The stage
-    // is released one iteration later, once that store has finished reading it.
+    // chunk (32 sign groups, one Philox block per lane, computed before the data arrives):
+    // its vectors are copied from the stage into registers, the stage is released at once,
+    // and the perturbed vectors are written with coalesced 16-byte stores.
     constexpr int kSlice = kPChunk / kPConsumers;  // 512 elements = 32 groups
+    constexpr int kVecs = kSlice / (N * 32);       // vectors per lane
     const int cw = warp - 1;
-    int it = 0, prev_s = -1;
-    bool ok_all = true;
+    int it = 0;
     for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
       const int s = it % kPStages;
       const uint32_t ph = (uint32_t)(it / kPStages) & 1u;
+      const int64_t cs = (g0 + c * kTileGroups) * kGroup;
+      const int64_t ws = cs + (int64_t)cw * kSlice;  // this warp's slice
+      uint32_t mine = 0u;
+      if (pk.sign)
+        mine = probe_group_bits(pk.g_off + (uint64_t)(ws / kGroup) + lane, pk.probe, step, pk.k0, pk.k1);
       int ok = 1;  // decided per warp, as in the loss pipeline
       if (lane == 0) ok = (!abort_flag && tc::mbar_wait(&full[s], ph)) ? 1 : 0;
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (ok && lane != 0) ok = tc::mbar_wait(&full[s], ph) ? 1 : 0;
       if (!__all_sync(0xFFFFFFFFu, ok)) {
         if (lane == 0) { atomicOr(err, ZO_FLAG_TIMEOUT); abort_flag = 1; }
-        ok_all = false;
         break;
       }
-      uint8_t *st = psm + s * SM::kStage;
-      const int64_t cs = (g0 + c * kTileGroups) * kGroup;
+      const uint8_t *st = psm + s * SM::kStage;
       const int64_t vs = cs > first ? cs : first;
       const int64_t ve = cs + kPChunk < end ? cs + kPChunk : end;
       const int64_t copy_end = vs + ((ve - vs) & ~(int64_t)(N - 1));
-      const int64_t ws = cs + (int64_t)cw * kSlice;  // this warp's slice
-      uint32_t mine = 0u;
-      if (pk.sign)
-        mine = probe_group_bits(pk.g_off + (uint64_t)(ws / kGroup) + lane, pk.probe, step, pk.k0, pk.k1);
+      uint4 v[kVecs];
 #pragma unroll
-      for (int k = 0; k < kSlice / (N * 32); ++k) {
-        const int v = lane + 32 * k;  // vector of the slice
-        const int64_t e = ws + (int64_t)v * N;
+      for (int k = 0; k < kVecs; ++k) {
+        const int64_t e = ws + (int64_t)(lane + 32 * k) * N;
+        if (e >= vs && e + N <= copy_end)
+          v[k] = *reinterpret_cast<const uint4 *>(st + (e - cs) * (int64_t)sizeof(T));
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&empty[s]);  // the stage is free again
+#pragma unroll
+      for (int k = 0; k < kVecs; ++k) {
+        const int vi = lane + 32 * k;  // vector of the slice
+        const int64_t e = ws + (int64_t)vi * N;
         const uint32_t bits =
-            pk.sign ? __shfl_sync(0xFFFFFFFFu, mine, (v * N) >> 4) >> ((v * N) & 15) : 0u;
+            pk.sign ? __shfl_sync(0xFFFFFFFFu, mine, (vi * N) >> 4) >> ((vi * N) & 15) : 0u;
         if (e + N <= vs || e >= ve) continue;
         if (e >= vs && e + N <= copy_end) {
-          uint4 *p = reinterpret_cast<uint4 *>(st + (e - cs) * (int64_t)sizeof(T));
-          if (pk.sign) *p = apply_vec(*p, bits, delta, (T *)nullptr);
+          uint4 x = v[k];
+          if (pk.sign) x = apply_vec(x, bits, delta, (T *)nullptr);
+          *reinterpret_cast<uint4 *>(out + (e - first)) = x;
         } else {  // the window's last < N elements: plain loads and stores
 #pragma unroll
           for (int t = 0; t < N; ++t) {
@@ -238,23 +247,6 @@ perturb_pipe_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t fi
           }
         }
       }
-      tc::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        const int64_t b0 = ws > vs ? ws : vs;
-        const int64_t b1 = ws + kSlice < copy_end ? ws + kSlice : copy_end;
-        if (b1 > b0)
-          tc::bulk_store(out + (b0 - first), st + (b0 - cs) * (int64_t)sizeof(T),
-                         (uint32_t)((b1 - b0) * (int64_t)sizeof(T)));
-        tc::bulk_commit();      // one group per iteration (possibly empty)
-        tc::bulk_wait_read1();  // the previous iteration's store has read its stage
-        if (prev_s >= 0) tc::mbar_arrive(&empty[prev_s]);
-      }
-      prev_s = s;
-    }
-    if (lane == 0) {
-      tc::bulk_wait0();  // every store of this warp has landed
-      if (ok_all && prev_s >= 0) tc::mbar_arrive(&empty[prev_s]);
     }
   }
 }
@@ -292,7 +284,14 @@ zo_status launch_pipe(zo_ctx *ctx, const ProbeKey &pk, int64_t first, int64_t co
   const int64_t g0 = first / kGroup;
   const int64_t g1 = (first + count + kGroup - 1) / kGroup;
   const int64_t n_chunks = (g1 - g0 + kTileGroups - 1) / kTileGroups;
-  const int64_t blocks = n_chunks < (int64_t)kSmCount * 2 ? n_chunks : (int64_t)kSmCount * 2;
+  int per_sm = 2;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, perturb_pipe_kernel<T>, kPThreads,
+                                                    SM::kBytes) != cudaSuccess || per_sm < 1) {
+    cudaGetLastError();
+    per_sm = 1;
+  }
+  const int64_t cap = (int64_t)kSmCount * per_sm;
+  const int64_t blocks = n_chunks < cap ? n_chunks : cap;
   perturb_pipe_kernel<T><<<(unsigned)blocks, kPThreads, SM::kBytes, ctx->stream>>>(
       static_cast<const T *>(ctx->params), static_cast<T *>(out), first, count, pk, n_chunks,
       &ctx->dstate->flags);

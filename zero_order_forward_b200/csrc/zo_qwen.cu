@@ -59,7 +59,7 @@ rmsnorm_kernel(const float *__restrict__ x, const uint16_t *__restrict__ w, uint
   for (int t = 0; t < 4; ++t) {
     const float y0 = v[2 * t] * rstd * __uint_as_float(wv[t] << 16);
     const float y1 = v[2 * t + 1] * rstd * __uint_as_float(wv[t] & 0xFFFF0000u);
-    o[t] = (uint32_t)f32_to_bf16_bits(y0) | ((uint32_t)f32_to_bf16_bits(y1) << 16);
+    o[t] = pack_bf16x2(y0, y1);
   }
   *reinterpret_cast<uint4 *>(y + (int64_t)blockIdx.x * d + c) = make_uint4(o[0], o[1], o[2], o[3]);
 }

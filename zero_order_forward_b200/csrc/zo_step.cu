@@ -144,8 +144,7 @@ template <> struct Elem<uint16_t> {
       uint32_t w[4];
 #pragma unroll
       for (int t = 0; t < 4; ++t)
-        w[t] = (uint32_t)f32_to_bf16_bits(v[8 * k + 2 * t]) |
-               ((uint32_t)f32_to_bf16_bits(v[8 * k + 2 * t + 1]) << 16);
+        w[t] = pack_bf16x2(v[8 * k + 2 * t], v[8 * k + 2 * t + 1]);
       reinterpret_cast<uint4 *>(p)[k] = make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
@@ -175,16 +174,14 @@ template <> struct Elem<uint16_t> {
 // the global index of the context's first group: its elements take the signs of their
 // global indices.
 //
-// theta streams through shared memory: one CTA per SM; warp 0 issues bulk copies of chunks
-// of 8192 elements into a ring of stages; 16 consumer warps update their groups in place in
-// the stage and each writes its contiguous 512-element slice back with one bulk copy, so that
-// both directions move in large asynchronous transfers while the consumers regenerate the
-// probes.  The last partial vector of theta (fewer than 16 bytes) is read and written
-// directly.
+// theta streams in through shared memory: one CTA per SM; warp 0 issues bulk copies of
+// chunks of 8192 elements into a ring of stages, so that the loads are in flight while the
+// 16 consumer warps regenerate the probes; a consumer thread copies its 16-element group from
+// the stage into registers, the stage is released, and the updated group is written back with
+// coalesced stores.  The last partial vector of theta (fewer than 16 bytes) is read directly.
 constexpr int kUConsumers = 16;
 constexpr int kUThreads = 32 * (1 + kUConsumers);
 constexpr int kUChunk = kUConsumers * 32 * kGroup;  // 8192 elements
-constexpr int kUSlice = 32 * kGroup;                // 512 elements per consumer warp
 
 template <typename T> struct UpdPipe {
   static constexpr int kStages = sizeof(T) == 2 ? 4 : 3;
@@ -301,11 +298,12 @@ update_kernel(T *__restrict__ theta, int64_t M, const float *__restrict__ coef, 
     }
     return;
   }
-  // consumers: thread ct updates group ct of each chunk; warp cw bulk-stores its slice
-  const int ct = threadIdx.x - 32, cw = warp - 1;
+  // consumers: thread ct updates group ct of each chunk: it copies the group from the stage
+  // into registers, the warp releases the stage, and the updated group is written back with
+  // coalesced 16-byte stores (a warp writes 1 KB (bf16) or 2 KB (fp32) of consecutive bytes)
+  const int ct = threadIdx.x - 32;
   const float *mine = lut + (lane & ((1 << LOG_R) - 1));
-  int it = 0, prev_s = -1;
-  bool ok_all = true;
+  int it = 0;
   for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x, ++it) {
     const int s = it % U::kStages;
     const uint32_t ph = (uint32_t)(it / U::kStages) & 1u;
@@ -315,51 +313,33 @@ update_kernel(T *__restrict__ theta, int64_t M, const float *__restrict__ coef, 
     if (ok && lane != 0) ok = tc::mbar_wait(&full[s], ph) ? 1 : 0;
     if (!__all_sync(0xFFFFFFFFu, ok)) {
       if (lane == 0) { atomicOr(err, ZO_FLAG_TIMEOUT); abort_flag = 1; }
-      ok_all = false;
       break;
     }
-    T *st = reinterpret_cast<T *>(usm + s * U::kStage);
+    const T *st = reinterpret_cast<const T *>(usm + s * U::kStage);
     const int64_t cs = c * kUChunk;
     const int64_t copy_end = cs + (((M - cs < kUChunk ? M - cs : kUChunk)) & ~(int64_t)(N - 1));
     const int64_t e0 = cs + (int64_t)ct * kGroup;
-    if (e0 < M) {
-      float v[16];
-      const bool whole = e0 + kGroup <= copy_end;
-      if (whole) {
-        Elem<T>::load16s(st + ct * kGroup, v);
-      } else {  // the last group: elements below copy_end are staged, the rest are in theta
+    const bool whole = e0 + kGroup <= copy_end;
+    float v[16];
+    if (whole) {
+      Elem<T>::load16s(st + ct * kGroup, v);
+    } else {  // the last group: elements below copy_end are staged, the rest are read directly
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          v[e] = e0 + e < copy_end ? Elem<T>::get(st, e0 + e - cs)
-                                   : (e0 + e < M ? Elem<T>::get(theta, e0 + e) : 0.f);
-      }
-      apply_probes<LOG_R>(v, mine, (uint64_t)(e0 / kGroup) + g_off, octets, step, k0, k1);
-      if (whole) {
-        Elem<T>::store16(st + ct * kGroup, v);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          if (e0 + e < copy_end) Elem<T>::put(st, e0 + e - cs, v[e]);
-          else if (e0 + e < M) Elem<T>::put(theta, e0 + e, v[e]);
-        }
-      }
+      for (int e = 0; e < 16; ++e)
+        v[e] = e0 + e < copy_end ? Elem<T>::get(st, e0 + e - cs)
+                                 : (e0 + e < M ? Elem<T>::get(theta, e0 + e) : 0.f);
     }
-    tc::fence_proxy_async_smem();
     __syncwarp();
-    if (lane == 0) {
-      const int64_t b0 = cs + (int64_t)cw * kUSlice;
-      const int64_t b1 = b0 + kUSlice < copy_end ? b0 + kUSlice : copy_end;
-      if (b1 > b0)
-        tc::bulk_store(theta + b0, st + (b0 - cs), (uint32_t)((b1 - b0) * (int64_t)sizeof(T)));
-      tc::bulk_commit();      // one group per iteration (possibly empty)
-      tc::bulk_wait_read1();  // the previous iteration's store has read its stage
-      if (prev_s >= 0) tc::mbar_arrive(&empty[prev_s]);
+    if (lane == 0) tc::mbar_arrive(&empty[s]);  // the stage is free again
+    if (e0 >= M) continue;
+    apply_probes<LOG_R>(v, mine, (uint64_t)(e0 / kGroup) + g_off, octets, step, k0, k1);
+    if (whole) {
+      Elem<T>::store16(theta + e0, v);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        if (e0 + e < M) Elem<T>::put(theta, e0 + e, v[e]);
     }
-    prev_s = s;
-  }
-  if (lane == 0) {
-    tc::bulk_wait0();  // every store of this warp has landed
-    if (ok_all && prev_s >= 0) tc::mbar_arrive(&empty[prev_s]);
   }
 }
 
