@@ -7,21 +7,23 @@
 // [B*S][(H + 2 Hk) hd] (query heads, key heads, value heads), out is [B*S][H hd].
 //
 // One CTA (6 warps) per (128-query tile, head, sequence), heavy (late) tiles first, two
-// CTAs per SM so that one CTA's softmax overlaps the other's MMAs and loads:
+// CTAs per SM.  Key tiles of 64 keys flow through a software pipeline in which the softmax
+// of tile j+1 overlaps the P V product of tile j:
 //   warp 0     one lane issues TMA loads: the Q tile once (boxes of 64 columns x 128 rows),
-//              then K and V tiles of 64 keys (boxes of 64 columns x 64 rows) into a 2-stage
-//              ring (two tensor maps over the qkv buffer, 128-byte swizzle);
-//   warp 1     allocates 256 TMEM columns (S: 64, P: 32, O: hd) and one lane issues
-//              S = Q K^T (tcgen05.mma M=128, N=64, both operands K-major from shared
-//              memory), the next tile's S as soon as the softmax has read this one, and,
-//              once the softmax has written P, O += P V (P from tensor memory, V MN-major
-//              from shared memory as loaded), committing to mbarriers;
+//              then K_j and V_{j-1} alternately into separate K and V rings (128-byte
+//              swizzle), each stage released by the MMA that reads it;
+//   warp 1     allocates 256 TMEM columns (two 64-column score buffers, O: hd) and one lane
+//              issues S_j = Q K_j^T into buffer j % 2 (tcgen05.mma M=128, N=64, both operands
+//              K-major in shared memory), O += P_j V_j once the softmax has written P_j (P read
+//              from TMEM as the A operand, V MN-major from shared memory as loaded), and
+//              S_{j+2} into the same buffer once that P V has completed;
 //   warps 2-5  the softmax, one query row per thread (TMEM lane quadrant = warp % 4): read the
-//              row of S from TMEM, scale, mask (diagonal and sequence-end tiles only), online
+//              row of S_j from TMEM, scale, mask (diagonal and sequence-end tiles only), online
 //              maximum with lazy rescaling (O and the row sum are rescaled only when the
-//              maximum grows by more than 2^8, so exponentials stay below 256), P = 2^(s - m)
-//              rounded to bf16 and stored to TMEM, row sum in fp32; at the end O / l is read
-//              from TMEM, rounded to bf16 and stored.
+//              maximum grows by more than 2^8, so exponentials stay below 256; only then does
+//              the softmax wait for the previous P V), P = 2^(s - m) rounded to bf16 and
+//              written over S_j in TMEM, row sum in fp32; at the end O / l is read from TMEM,
+//              rounded to bf16 and stored.
 // All waits are bounded (zo_tc.cuh); on expiry the kernel raises ZO_FLAG_TIMEOUT, lets its
 // loads and MMAs drain and frees TMEM.
 #include <cudaTypedefs.h>
@@ -34,28 +36,32 @@
 namespace zo {
 namespace {
 
-constexpr int kTBM = 128, kTThreads = 192;
+constexpr int kTBM = 128, kTThreads = 192, kTBN = 64;
 constexpr uint32_t kQBox = 128 * 128;  // bytes of one 128-row x 64-column bf16 box
+constexpr uint32_t kKBox = kTBN * 128; // bytes of one 64-row x 64-column bf16 box
 
-// Key tiles of BN keys (hd 128: 64; hd 64: 128, so that a tile's MMAs amortise the
-// softmax round trip), two K/V stages, 256 TMEM columns (S: BN, P: BN/2, O: hd) and 96 KB
-// (hd 128) or 80 KB (hd 64) of shared memory per CTA: two CTAs per SM.
+// Key tiles of 64 keys.  TMEM (256 columns per CTA, two CTAs per SM): two score buffers of
+// 64 columns, each later overwritten in place by its tile's bf16 probabilities (32 columns),
+// then O (hd columns).  Separate K and V rings in shared memory, so that a key tile is
+// released (and the next one loaded) as soon as its score MMA has completed.
 template <int HD> struct TcAttnCfg {
-  static constexpr int kBN = HD == 128 ? 64 : 128;
-  static constexpr int kStages = 2, kCtas = 2, kTmemCols = 256;
+  static constexpr int kKS = HD == 128 ? 2 : 4;  // K stages
+  static constexpr int kVS = HD == 128 ? 2 : 4;  // V stages
+  static constexpr int kCtas = 2, kTmemCols = 256;
 };
 
 template <int HD>
 struct TcAttnSmem {
-  static constexpr int kStages = TcAttnCfg<HD>::kStages;
-  static constexpr uint32_t kKBox = TcAttnCfg<HD>::kBN * 128;  // BN rows x 64 columns
+  static constexpr int kKS = TcAttnCfg<HD>::kKS, kVS = TcAttnCfg<HD>::kVS;
   static constexpr uint32_t kQTile = (HD / 64) * kQBox;   // 128 rows x HD columns
-  static constexpr uint32_t kKTile = (HD / 64) * kKBox;   // BN rows x HD columns
+  static constexpr uint32_t kKTile = (HD / 64) * kKBox;   // 64 rows x HD columns
   static constexpr uint32_t kQ = 0;
-  static constexpr uint32_t kK = kQ + kQTile;                // [kStages]
-  static constexpr uint32_t kV = kK + kStages * kKTile;      // [kStages]
-  static constexpr uint32_t kBar = kV + kStages * kKTile;
-  static constexpr uint32_t kBytes = kBar + 128 + 1024;      // barriers + alignment slack
+  static constexpr uint32_t kK = kQ + kQTile;              // [kKS]
+  static constexpr uint32_t kV = kK + kKS * kKTile;        // [kVS]
+  static constexpr uint32_t kBar = kV + kVS * kKTile;
+  static constexpr int kNumBars = 1 + 2 * kKS + 2 * kVS + 2 + 2 + 2 + 1;
+  static constexpr uint32_t kBytes = kBar + 256 + 1024;    // barriers + alignment slack
+  static_assert(kNumBars * 8 + 8 <= 256, "barrier area");
 };
 
 struct TcAttnArgs {
@@ -88,22 +94,29 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
   return __all_sync(0xFFFFFFFFu, ok) != 0;
 }
 
+// Phase bookkeeping of a ring of `n` barriers used once per item i: item i uses barrier
+// i % n, and its completion is phase i / n of that barrier.
+__device__ __forceinline__ uint32_t ring_parity(int i, int n) { return (uint32_t)(i / n) & 1u; }
+
 template <int HD>
 __global__ void __launch_bounds__(kTThreads, TcAttnCfg<HD>::kCtas)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmkv,
                TcAttnArgs a) {
   using SM = TcAttnSmem<HD>;
-  constexpr int kTStages = SM::kStages;
-  constexpr int kTBN = TcAttnCfg<HD>::kBN;
-  constexpr uint32_t kKBox = SM::kKBox;
+  constexpr int KS = SM::kKS, VS = SM::kVS;
   constexpr uint32_t kCols = TcAttnCfg<HD>::kTmemCols;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SM::kBar);
-  uint64_t *q_full = bars, *kv_full = bars + 1, *kv_empty = bars + 3, *s_full = bars + 5,
-           *s_free = bars + 6, *p_full = bars + 7, *pv_done = bars + 8, *mma_done = bars + 9;
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 10);  // 10 barriers + 2 words < 128 B
+  uint64_t *q_full = bars;
+  uint64_t *k_full = q_full + 1, *k_empty = k_full + KS;
+  uint64_t *v_full = k_empty + KS, *v_empty = v_full + VS;
+  uint64_t *s_full = v_empty + VS;  // [2] scores of tile j in buffer j % 2
+  uint64_t *p_full = s_full + 2;    // [2] probabilities of tile j written (4 softmax warps)
+  uint64_t *pv_done = p_full + 2;   // [2] O += P_j V_j completed
+  uint64_t *mma_done = pv_done + 2;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -116,16 +129,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
   const int n_kt = last_q / kTBN + 1;
 
   if (threadIdx.x == 0) {
-    tc::mbar_init(q_full, 1);
-    for (int s = 0; s < kTStages; ++s) {
-      tc::mbar_init(&kv_full[s], 1);
-      tc::mbar_init(&kv_empty[s], 1);
-    }
-    tc::mbar_init(s_full, 1);
-    tc::mbar_init(s_free, 4);  // one arrival per softmax warp
-    tc::mbar_init(p_full, 4);
-    tc::mbar_init(pv_done, 1);
-    tc::mbar_init(mma_done, 1);
+    for (int i = 0; i < SM::kNumBars; ++i) tc::mbar_init(&bars[i], 1);
+    tc::mbar_init(&p_full[0], 4);  // one arrival per softmax warp
+    tc::mbar_init(&p_full[1], 4);
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -134,43 +140,51 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  // S: BN columns, P: BN/2 (bf16 pairs), O: hd (hd 128: 0/64/128; hd 64: 0/128/192)
-  const uint32_t tS = tmem, tP = tmem + kTBN, tO = tmem + kTBN + kTBN / 2 + (HD == 128 ? 32 : 0);
+  const uint32_t tO = tmem + 2 * kTBN;  // S/P buffers at columns 0 and kTBN
 
   if (warp == 0) {
-    if (lane == 0) {  // TMA producer
+    if (lane == 0) {  // TMA producer: Q once, then K_j ahead of V_{j-1}
       tc::tma_prefetch_desc(&tmq);
       tc::tma_prefetch_desc(&tmkv);
       tc::mbar_arrive_expect_tx(q_full, SM::kQTile);
 #pragma unroll
       for (int c = 0; c < HD / 64; ++c)
         tc::tma_load_2d(sm + SM::kQ + c * kQBox, &tmq, q_full, a.q0 + h * HD + 64 * c, row0 + q_first);
-      int issued = 0;
-      for (int j = 0; j < n_kt; ++j) {
-        const int s = j % kTStages;
-        const uint32_t ph = (uint32_t)(j / kTStages) & 1u;
-        if (*abort_flag || !tc::mbar_wait(&kv_empty[s], ph ^ 1u)) {
-          atomicOr(a.err, ZO_FLAG_TIMEOUT);
-          *abort_flag = 1;
-          break;
-        }
-        tc::mbar_arrive_expect_tx(&kv_full[s], 2 * SM::kKTile);
+      int k_issued = 0, v_issued = 0;
+      auto load_k = [&](int j) -> bool {
+        if (*abort_flag || !tc::mbar_wait(&k_empty[j % KS], ring_parity(j, KS) ^ 1u)) return false;
+        tc::mbar_arrive_expect_tx(&k_full[j % KS], SM::kKTile);
 #pragma unroll
-        for (int c = 0; c < HD / 64; ++c) {
-          tc::tma_load_2d(sm + SM::kK + s * SM::kKTile + c * kKBox, &tmkv, &kv_full[s],
+        for (int c = 0; c < HD / 64; ++c)
+          tc::tma_load_2d(sm + SM::kK + (j % KS) * SM::kKTile + c * kKBox, &tmkv, &k_full[j % KS],
                           a.k0 + kvh * HD + 64 * c, row0 + j * kTBN);
-          tc::tma_load_2d(sm + SM::kV + s * SM::kKTile + c * kKBox, &tmkv, &kv_full[s],
+        k_issued = j + 1;
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
+        if (*abort_flag || !tc::mbar_wait(&v_empty[j % VS], ring_parity(j, VS) ^ 1u)) return false;
+        tc::mbar_arrive_expect_tx(&v_full[j % VS], SM::kKTile);
+#pragma unroll
+        for (int c = 0; c < HD / 64; ++c)
+          tc::tma_load_2d(sm + SM::kV + (j % VS) * SM::kKTile + c * kKBox, &tmkv, &v_full[j % VS],
                           a.v0 + kvh * HD + 64 * c, row0 + j * kTBN);
-        }
-        issued = j + 1;
+        v_issued = j + 1;
+        return true;
+      };
+      bool ok = true;
+      for (int j = 0; ok && j <= n_kt; ++j) {
+        if (j < n_kt) ok = load_k(j);
+        if (ok && j >= 1) ok = load_v(j - 1);
       }
-      if (*abort_flag) {  // let this CTA's loads land before it exits (bounded)
+      if (!ok) {
+        atomicOr(a.err, ZO_FLAG_TIMEOUT);
+        *abort_flag = 1;
+        // let this CTA's loads land before it exits (bounded)
         tc::mbar_wait(q_full, 0);
-        for (int s = 0; s < kTStages; ++s) {
-          int last = -1;
-          for (int i = s; i < issued; i += kTStages) last = i;
-          if (last >= 0) tc::mbar_wait(&kv_full[s], (uint32_t)(last / kTStages) & 1u);
-        }
+        for (int i = k_issued - KS > 0 ? k_issued - KS : 0; i < k_issued; ++i)
+          tc::mbar_wait(&k_full[i % KS], ring_parity(i, KS));
+        for (int i = v_issued - VS > 0 ? v_issued - VS : 0; i < v_issued; ++i)
+          tc::mbar_wait(&v_full[i % VS], ring_parity(i, VS));
       }
     }
   } else if (warp == 1) {
@@ -178,42 +192,43 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
       constexpr uint32_t idS = tc::idesc_bf16_f32(kTBM, kTBN);
       constexpr uint32_t idO = tc::idesc_bf16_f32(kTBM, HD) | (1u << 16);  // B (V) MN-major
       const uint32_t qa = tc::smem_addr(sm + SM::kQ);
-      // S_j = Q K_j^T into TMEM once K_j has landed and the softmax has read S_{j-1}
+      // S_j = Q K_j^T into score buffer j % 2
       auto issue_s = [&](int j) -> bool {
-        const int s = j % kTStages;
-        if (*abort_flag || !tc::mbar_wait(&kv_full[s], (uint32_t)(j / kTStages) & 1u) ||
-            (j > 0 && !tc::mbar_wait(s_free, (uint32_t)(j - 1) & 1u)))
-          return false;
+        if (*abort_flag || !tc::mbar_wait(&k_full[j % KS], ring_parity(j, KS))) return false;
         tc::tc_fence_after();
-        const uint32_t ka = tc::smem_addr(sm + SM::kK + s * SM::kKTile);
+        const uint32_t ka = tc::smem_addr(sm + SM::kK + (j % KS) * SM::kKTile);
+        const uint32_t tS = tmem + (uint32_t)((j & 1) * kTBN);
 #pragma unroll
         for (int k = 0; k < HD / 16; ++k) {
           const uint32_t kk = (uint32_t)(k & 3) * 32u;
           tc::mma_bf16(tS, tc::smem_desc_k128(qa + (uint32_t)(k >> 2) * kQBox + kk),
                        tc::smem_desc_k128(ka + (uint32_t)(k >> 2) * kKBox + kk), idS, k > 0 ? 1u : 0u);
         }
-        tc::mma_commit(s_full);
+        tc::mma_commit(&s_full[j & 1]);
+        tc::mma_commit(&k_empty[j % KS]);
         return true;
       };
-      bool ok = tc::mbar_wait(q_full, 0) && issue_s(0);
+      bool ok = tc::mbar_wait(q_full, 0) && issue_s(0) && (n_kt < 2 || issue_s(1));
       for (int j = 0; ok && j < n_kt; ++j) {
-        const int s = j % kTStages;
-        // with two stages the next tile's scores overlap this tile's softmax; with one, the
-        // next K arrives only after this tile's P V has released the stage
-        if (kTStages > 1 && j + 1 < n_kt && !(ok = issue_s(j + 1))) break;
-        ok = tc::mbar_wait(p_full, (uint32_t)j & 1u);
+        // O += P_j V_j once the softmax has written P_j (in place of S_j) and V_j has landed
+        ok = tc::mbar_wait(&p_full[j & 1], ring_parity(j, 2)) &&
+             tc::mbar_wait(&v_full[j % VS], ring_parity(j, VS));
         if (!ok) break;
         tc::tc_fence_after();
-        const uint32_t va = tc::smem_addr(sm + SM::kV + s * SM::kKTile);
+        const uint32_t va = tc::smem_addr(sm + SM::kV + (j % VS) * SM::kKTile);
+        const uint32_t tP = tmem + (uint32_t)((j & 1) * kTBN);
 #pragma unroll
         for (int k = 0; k < kTBN / 16; ++k) {
           const uint32_t boff = (uint32_t)k * 16u * 128u;  // 16 keys of 128-byte V rows
           tc::mma_bf16_tmem_a(tO, tP + 8u * k, tc::smem_desc_mn128(va + boff, kKBox), idO,
                               (j > 0 || k > 0) ? 1u : 0u);
         }
-        tc::mma_commit(pv_done);
-        tc::mma_commit(&kv_empty[s]);
-        if (kTStages == 1 && j + 1 < n_kt && !(ok = issue_s(j + 1))) break;
+        tc::mma_commit(&pv_done[j & 1]);
+        tc::mma_commit(&v_empty[j % VS]);
+        if (j + 2 < n_kt) {
+          // S_{j+2} reuses buffer j % 2: wait until P_j V_j has read it
+          ok = tc::mbar_wait(&pv_done[j & 1], ring_parity(j, 2)) && issue_s(j + 2);
+        }
       }
       if (!ok) {
         atomicOr(a.err, ZO_FLAG_TIMEOUT);
@@ -229,14 +244,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kt; ++j) {
-      if (!warp_wait(s_full, (uint32_t)j & 1u, abort_flag)) { ok = false; break; }
+      const uint32_t tS = tmem + (uint32_t)((j & 1) * kTBN) + lane_off;
+      if (!warp_wait(&s_full[j & 1], ring_parity(j, 2), abort_flag)) { ok = false; break; }
       tc::tc_fence_after();
       float s[kTBN];
 #pragma unroll
-      for (int c = 0; c < kTBN / 32; ++c) tc::tmem_ld32(tS + lane_off + 32u * c, s + 32 * c);
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(s_free);  // S may be overwritten by the next tile
+      for (int c = 0; c < kTBN / 32; ++c) tc::tmem_ld32(tS + 32u * c, s + 32 * c);
       const int key0 = j * kTBN;
       const bool edge = key0 + kTBN - 1 > q_first || key0 + kTBN > a.S;
       // the maximum of the raw scores (the scale is positive), then 2^(s * scale - m) with the
@@ -250,7 +263,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
       const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * a.scale_log2;
       const float m_new = fmaxf(m_used, mx);
       // Lazy rescaling: keep the running maximum unless it grows by more than 2^8 (then
-      // O and l are rescaled below, once the previous tile's P V has completed).
+      // O and l are rescaled, once the previous tile's P V has completed).
       const bool need = j > 0 && m_new > m_used + 8.f;
       const float m_old = m_used;
       if (j == 0 || need) m_used = m_new;
@@ -264,31 +277,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         pk[c / 2] = pack2_bf16(p0, p1);
       }
       const float lsum = (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
-      if (j > 0) {
-        // P and O are free once the previous tile's P V has completed
-        if (!warp_wait(pv_done, (uint32_t)(j - 1) & 1u, abort_flag)) { ok = false; break; }
+      if (__any_sync(0xFFFFFFFFu, need)) {
+        // O holds P_{j-1} V_{j-1} only once that MMA has completed
+        if (!warp_wait(&pv_done[(j - 1) & 1], ring_parity(j - 1, 2), abort_flag)) { ok = false; break; }
         tc::tc_fence_after();
-        if (__any_sync(0xFFFFFFFFu, need)) {
-          const float f = need ? ex2(m_old - m_new) : 1.f;
-          l *= f;
+        const float f = need ? ex2(m_old - m_new) : 1.f;
+        l *= f;
 #pragma unroll
-          for (int c = 0; c < HD / 32; ++c) {
-            float o[32];
-            tc::tmem_ld32(tO + lane_off + 32u * c, o);
+        for (int c = 0; c < HD / 32; ++c) {
+          float o[32];
+          tc::tmem_ld32(tO + lane_off + 32u * c, o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= f;
-            tc::tmem_st32(tO + lane_off + 32u * c, o);
-          }
+          for (int i = 0; i < 32; ++i) o[i] *= f;
+          tc::tmem_st32(tO + lane_off + 32u * c, o);
         }
       }
-#pragma unroll
-      for (int c = 0; c < kTBN / 64; ++c) tc::tmem_st32u(tP + lane_off + 32u * c, pk + 32 * c);
+      // P_j overwrites the first kTBN / 2 columns of S_j (already read into registers)
+      tc::tmem_st32u(tS, pk);
       l += lsum;
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(p_full);
+      if (lane == 0) tc::mbar_arrive(&p_full[j & 1]);
     }
-    if (ok && !warp_wait(pv_done, (uint32_t)(n_kt - 1) & 1u, abort_flag)) ok = false;
+    if (ok && !warp_wait(&pv_done[(n_kt - 1) & 1], ring_parity(n_kt - 1, 2), abort_flag)) ok = false;
     if (ok) {
       tc::tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -371,7 +382,7 @@ zo_status launch_attention_tc(zo_ctx *ctx, const uint16_t *qkv, uint16_t *out, i
   const cuuint64_t dims[2] = {(cuuint64_t)ld, (cuuint64_t)B * (cuuint64_t)S};
   const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
   const cuuint32_t boxq[2] = {64, (cuuint32_t)kTBM},
-                   boxkv[2] = {64, (cuuint32_t)(hd == 128 ? TcAttnCfg<128>::kBN : TcAttnCfg<64>::kBN)};
+                   boxkv[2] = {64, (cuuint32_t)kTBN};
   const cuuint32_t estr[2] = {1, 1};
   for (int m = 0; m < 2; ++m)
     if (fn(m ? &tmkv : &tmq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(qkv), dims,

@@ -20,8 +20,9 @@
 // output columns loads BN/2 gate rows and the matching BN/2 up rows into one BN-row
 // operand stage, so TMEM columns c and BN/2 + c of the accumulator hold the gate and up
 // products of output column c, combined as silu(g) * u in fp32 before one bf16 rounding.
-// Tiles are visited in groups of kGroupM row tiles so that the weight tiles of a group are
-// reused from L2.  All waits are bounded (see zo_tc.cuh); a timeout sets an error bit.
+// Tiles are visited in groups of row tiles (sized from K so that a group's rows of A, about
+// 64 MB, stay in the 126 MB L2) so that both the group's A rows and each weight tile are reused
+// from L2.  All waits are bounded (see zo_tc.cuh); a timeout sets an error bit.
 #include <cudaTypedefs.h>
 
 #include <cstdio>
@@ -34,10 +35,11 @@ namespace zo {
 
 namespace {
 
-constexpr int kBM = 128, kBK = 64, kGroupM = 8;
+constexpr int kBM = 128, kBK = 64;
 
 struct GemmArgs {
   int M, N, K;
+  int group_m;           // row tiles per group of the tile order
   const uint16_t *bias;  // [N] bf16 or null
   void *out;             // bf16 [M][ldo] or fp32 [M][ldo]
   int ldo;
@@ -112,15 +114,22 @@ struct TileCoord {
   int m0, n0;
 };
 
-// Grouped order: kGroupM row tiles share each sweep over the column tiles, so a group's
-// weight tiles are reused from L2.
-__device__ __forceinline__ TileCoord tile_coord(int t, int num_m, int num_n, int BN) {
-  const int group = t / (kGroupM * num_n);
-  const int first_m = group * kGroupM;
-  const int gsize = min(num_m - first_m, kGroupM);
+// Grouped order: group_m row tiles share each sweep over the column tiles, so a group's rows
+// of A and each weight tile are reused from L2.
+__device__ __forceinline__ TileCoord tile_coord(int t, int num_m, int num_n, int BN, int group_m) {
+  const int group = t / (group_m * num_n);
+  const int first_m = group * group_m;
+  const int gsize = min(num_m - first_m, group_m);
   const int m_tile = first_m + (t % gsize);
-  const int n_tile = (t % (kGroupM * num_n)) / gsize;
+  const int n_tile = (t % (group_m * num_n)) / gsize;
   return {m_tile * kBM, n_tile * BN};
+}
+
+// Row tiles per group: rows * K * 2 bytes of A near 64 MB, between 1 and 16 tiles.
+int group_rows_for(int K, int rows_per_tile) {
+  const int64_t per_tile = (int64_t)rows_per_tile * K * 2;
+  int64_t g = ((int64_t)64 << 20) / (per_tile > 0 ? per_tile : 1);
+  return (int)(g < 1 ? 1 : g > 16 ? 16 : g);
 }
 
 // Persistent: one CTA per SM walks tiles t = blockIdx.x, blockIdx.x + gridDim.x, ...
@@ -177,7 +186,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     tc::tma_prefetch_desc(&tmA);
     tc::tma_prefetch_desc(&tmB);
     for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
-      const TileCoord tc0 = tile_coord(t, num_m, num_n, OUT_BN);
+      const TileCoord tc0 = tile_coord(t, num_m, num_n, OUT_BN, args.group_m);
       for (int kb = 0; kb < nk; ++kb) {
         const uint32_t s = issued % STAGES, ph = (issued / STAGES) & 1u;
         if (*abort_flag || !tc::mbar_wait(&empty[s], ph ^ 1u)) {
@@ -248,7 +257,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         break;
       }
       tc::tc_fence_after();
-      const TileCoord tc0 = tile_coord(t, num_m, num_n, OUT_BN);
+      const TileCoord tc0 = tile_coord(t, num_m, num_n, OUT_BN, args.group_m);
       const int row0 = tc0.m0 + q * 32;
       const uint32_t base = tmem + (uint32_t)(b * BN) + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
@@ -328,8 +337,9 @@ struct PairSmem {
   static constexpr uint32_t kBytes = kBarOffset + 256 + 1024;
 };
 
-__device__ __forceinline__ TileCoord pair_tile_coord(int t, int num_m, int num_n, int out_bn) {
-  const TileCoord c = tile_coord(t, num_m, num_n, out_bn);
+__device__ __forceinline__ TileCoord pair_tile_coord(int t, int num_m, int num_n, int out_bn,
+                                                    int group_m) {
+  const TileCoord c = tile_coord(t, num_m, num_n, out_bn, group_m);
   return {c.m0 / kBM * (2 * kBM), c.n0};  // tile_coord's row tiles are pair tiles of 256 rows
 }
 
@@ -394,7 +404,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     tc::tma_prefetch_desc(&tmA);
     tc::tma_prefetch_desc(&tmB);
     for (int t = cluster; t < num_tiles && !*abort_flag; t += n_clusters) {
-      const TileCoord tc0 = pair_tile_coord(t, num_m, num_n, OUT_BN);
+      const TileCoord tc0 = pair_tile_coord(t, num_m, num_n, OUT_BN, args.group_m);
       // SwiGLU: CTA 0 loads the tile's gate rows, CTA 1 the matching up rows
       const int b_row = kSwiGLU ? (int)(rank ? args.N + tc0.n0 : tc0.n0) : tc0.n0 + (int)rank * (kPairBN / 2);
       for (int kb = 0; kb < nk; ++kb) {
@@ -462,7 +472,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         break;
       }
       tc::tc_fence_after();
-      const TileCoord tc0 = pair_tile_coord(t, num_m, num_n, OUT_BN);
+      const TileCoord tc0 = pair_tile_coord(t, num_m, num_n, OUT_BN, args.group_m);
       const int row0 = tc0.m0 + (int)rank * kBM + q * 32;
       const uint32_t base = tmem + (uint32_t)(b * kPairBN) + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
@@ -618,7 +628,8 @@ zo_status launch_gemm_pair(zo_ctx *ctx, const void *A, const void *B, const void
   if (!make_map(&ta, A, M, K, kBM) || !make_map(&tb, B, NB, K, kPairBN / 2) ||
       !make_out_map(&tcm, out, M, N, ldo, epi == ZO_EPI_RESID_F32))
     return fail(ctx, ZO_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
-  GemmArgs g{M, N, K, static_cast<const uint16_t *>(bias), out, ldo, &ctx->dstate->flags, 0u};
+  GemmArgs g{M, N, K, group_rows_for(K, 2 * kBM), static_cast<const uint16_t *>(bias), out, ldo,
+             &ctx->dstate->flags, 0u};
   const int slot = ktime_begin(ctx);
   cudaError_t e;
   if (epi == ZO_EPI_BIAS_BF16) e = launch_pair<6, ZO_EPI_BIAS_BF16>(ta, tb, tcm, g, ctx->stream);
@@ -653,7 +664,8 @@ zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bia
   if (!make_map(&ta, A, M, K, kBM) || !make_map(&tb, B, NB, K, box_b) ||
       !make_out_map(&tcm, out, M, N, ldo, epi == ZO_EPI_RESID_F32))
     return fail(ctx, ZO_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
-  GemmArgs g{M, N, K, static_cast<const uint16_t *>(bias), out, ldo, &ctx->dstate->flags, extra_tx};
+  GemmArgs g{M, N, K, group_rows_for(K, kBM), static_cast<const uint16_t *>(bias), out, ldo,
+             &ctx->dstate->flags, extra_tx};
   const int slot = ktime_begin(ctx);
   cudaError_t e;
   if (wide) {

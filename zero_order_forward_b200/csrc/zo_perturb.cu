@@ -25,21 +25,26 @@ template <> struct Vec<uint16_t> { static constexpr int N = 8; };
 // Apply the perturbation to one 16-byte vector of N elements whose sign bits are the
 // low N bits of `bits`.
 __device__ __forceinline__ uint4 apply_vec(uint4 v, uint32_t bits, float delta, float *) {
-  float f[4] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
-                __uint_as_float(v.w)};
+  const uint32_t db = __float_as_uint(delta);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float f[4];
 #pragma unroll
-  for (int t = 0; t < 4; ++t) f[t] = perturb_f32(f[t], delta, (bits >> t) & 1u);
+  for (int t = 0; t < 4; ++t)
+    f[t] = __fadd_rn(__uint_as_float(w[t]), __uint_as_float(db ^ ((bits << (31 - t)) & 0x80000000u)));
   return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
                     __float_as_uint(f[3]));
 }
 __device__ __forceinline__ uint4 apply_vec(uint4 v, uint32_t bits, float delta, uint16_t *) {
+  // element 2t takes sign bit 2t, element 2t+1 bit 2t+1: each shifted into bit 31 and xor-ed
+  // into eps (the same sum as perturb_f32)
+  const uint32_t db = __float_as_uint(delta);
   uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
-    const float lo = perturb_f32(bf16_bits_to_f32((uint16_t)(w[t] & 0xFFFFu)), delta,
-                                 (bits >> (2 * t)) & 1u);
-    const float hi = perturb_f32(bf16_bits_to_f32((uint16_t)(w[t] >> 16)), delta,
-                                 (bits >> (2 * t + 1)) & 1u);
+    const float lo = __fadd_rn(__uint_as_float(w[t] << 16),
+                               __uint_as_float(db ^ ((bits << (31 - 2 * t)) & 0x80000000u)));
+    const float hi = __fadd_rn(__uint_as_float(w[t] & 0xFFFF0000u),
+                               __uint_as_float(db ^ ((bits << (30 - 2 * t)) & 0x80000000u)));
     w[t] = pack_bf16x2(lo, hi);
   }
   return make_uint4(w[0], w[1], w[2], w[3]);
@@ -212,6 +217,28 @@ perturb_pipe_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t fi
         break;
       }
       const uint8_t *st = psm + s * SM::kStage;
+      if (cs >= first && cs + kPChunk <= end) {
+        // the whole chunk lies in the window (every chunk but the window's edges): 32-bit
+        // offsets, no per-vector bounds
+        const uint4 *src = reinterpret_cast<const uint4 *>(st + (int64_t)cw * kSlice * (int64_t)sizeof(T));
+        uint4 v[kVecs];
+#pragma unroll
+        for (int k = 0; k < kVecs; ++k) v[k] = src[lane + 32 * k];
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&empty[s]);  // the stage is free again
+        uint4 *dst = reinterpret_cast<uint4 *>(out + (ws - first));
+#pragma unroll
+        for (int k = 0; k < kVecs; ++k) {
+          const int vi = lane + 32 * k;
+          uint4 x = v[k];
+          if (pk.sign) {
+            const uint32_t bits = __shfl_sync(0xFFFFFFFFu, mine, (vi * N) >> 4) >> ((vi * N) & 15);
+            x = apply_vec(x, bits, delta, (T *)nullptr);
+          }
+          dst[vi] = x;
+        }
+        continue;
+      }
       const int64_t vs = cs > first ? cs : first;
       const int64_t ve = cs + kPChunk < end ? cs + kPChunk : end;
       const int64_t copy_end = vs + ((ve - vs) & ~(int64_t)(N - 1));

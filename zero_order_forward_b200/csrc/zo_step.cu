@@ -228,8 +228,8 @@ __device__ __forceinline__ void apply_probes(float v[16], const float *mine, uin
     const uint32_t w[4] = {blk.x, blk.y, blk.z, blk.w};
     const float *tab = mine + ((o * 256) << LOG_R);
 #pragma unroll
-    for (int e = 0; e < 16; ++e)
-      acc[e] = __fadd_rn(acc[e], tab[((w[e >> 2] >> (8 * (e & 3))) & 0xFFu) << LOG_R]);
+    for (int e = 0; e < 16; ++e)  // byte e & 3 of word e >> 2 selects the entry
+      acc[e] = __fadd_rn(acc[e], tab[__byte_perm(w[e >> 2], 0u, 0x4440u | (uint32_t)(e & 3)) << LOG_R]);
   }
 #pragma unroll
   for (int e = 0; e < 16; ++e) v[e] = __fsub_rn(v[e], acc[e]);
@@ -317,8 +317,17 @@ update_kernel(T *__restrict__ theta, int64_t M, const float *__restrict__ coef, 
     }
     const T *st = reinterpret_cast<const T *>(usm + s * U::kStage);
     const int64_t cs = c * kUChunk;
-    const int64_t copy_end = cs + (((M - cs < kUChunk ? M - cs : kUChunk)) & ~(int64_t)(N - 1));
     const int64_t e0 = cs + (int64_t)ct * kGroup;
+    if (cs + kUChunk <= M) {  // a full chunk: every group is whole and staged
+      float v[16];
+      Elem<T>::load16s(st + ct * kGroup, v);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&empty[s]);  // the stage is free again
+      apply_probes<LOG_R>(v, mine, (uint64_t)(e0 / kGroup) + g_off, octets, step, k0, k1);
+      Elem<T>::store16(theta + e0, v);
+      continue;
+    }
+    const int64_t copy_end = cs + ((M - cs) & ~(int64_t)(N - 1));
     const bool whole = e0 + kGroup <= copy_end;
     float v[16];
     if (whole) {
