@@ -48,8 +48,8 @@ SM_COUNT, ISSUE_PER_SM_CLOCK = 148, 4
 # that capture, not from this run) only while the sources still hash to it; otherwise null.
 #   quad_octet_kernel, M = 2^24: DRAM bytes (read + write) and warp instructions per launch.
 LOSS_TRAFFIC = {"sources": ("zo_loss.cu", "zo_internal.cuh"),
-                "sources_sha256": "d1b68b988680111f9d369faf40a77a5e8e770b8100af06f1e229ee733b2a03b3",
-                "bytes": 139.3e6, "warp_instructions": 90.41e6}
+                "sources_sha256": "725eacfcbeef93d6ed28cc732c5693f4d65e2341808033820719392cc2b40e5e",
+                "bytes": 138.57e6, "warp_instructions": 90.42e6}
 #   gemm_bf16_kernel at the OPT-30B layer shapes (T = 16384): DRAM bytes per launch averaged
 #   over the four projections of one layer (filled in from a capture; None until then).
 GEMM_TRAFFIC = {"sources": ("zo_gemm.cu", "zo_tc.cuh"), "sources_sha256": None, "bytes": None}

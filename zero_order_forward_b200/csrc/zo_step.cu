@@ -174,7 +174,8 @@ template <> struct Elem<uint16_t> {
 // the global index of the context's first group: its elements take the signs of their
 // global indices.
 //
-// theta streams in through shared memory: one CTA per SM; warp 0 issues bulk copies of
+// theta streams in through shared memory: one or two CTAs per SM (section on the table
+// budget below); warp 0 issues bulk copies of
 // chunks of 8192 elements into a ring of stages, so that the loads are in flight while the
 // 16 consumer warps regenerate the probes; a consumer thread copies its 16-element group from
 // the stage into registers, the stage is released, and the updated group is written back with
@@ -189,6 +190,8 @@ template <typename T> struct UpdPipe {
   static constexpr int kRing = kStages * kStage;
   static constexpr int kLut = kRing + 2 * kStages * 8;  // after the ring and its barriers
   static constexpr int kFixed = kLut;
+  // bf16 runs two CTAs per SM at small n (registers capped at 56 per thread), fp32 one
+  static constexpr int kMinBlocks = sizeof(T) == 2 ? 2 : 1;
 };
 
 // The octets' tables, R replicas each (all threads of the CTA take part).
@@ -236,7 +239,7 @@ __device__ __forceinline__ void apply_probes(float v[16], const float *mine, uin
 }
 
 template <typename T, int LOG_R>
-__global__ void __launch_bounds__(kUThreads, 1)
+__global__ void __launch_bounds__(kUThreads, UpdPipe<T>::kMinBlocks)
 update_kernel(T *__restrict__ theta, int64_t M, const float *__restrict__ coef, int n,
               const uint32_t *step_ptr, const uint32_t *ok_ptr, uint32_t k0, uint32_t k1,
               uint64_t g_off, uint32_t *err) {
@@ -352,13 +355,17 @@ update_kernel(T *__restrict__ theta, int64_t M, const float *__restrict__ coef, 
   }
 }
 
-// Replicas of the tables that fit beside the ring in the CTA's shared memory.
+// Replicas of the tables beside the ring: when 16 or more fit within half an SM's shared
+// memory (112 KB per CTA), two CTAs share an SM (34 warps: the kernel is bound by instruction
+// issue); otherwise one CTA takes up to 226 KB.
 template <typename T>
 int update_log_replicas(int n) {
   const int64_t per_replica = (int64_t)((n + 7) / 8) * 256 * 4;
-  const int64_t budget = 226 * 1024 - UpdPipe<T>::kFixed;
   int lr = 5;
-  while (lr > 0 && (per_replica << lr) > budget) --lr;
+  while (lr > 0 && (per_replica << lr) > 112 * 1024 - UpdPipe<T>::kFixed) --lr;
+  if ((per_replica << lr) <= 112 * 1024 - UpdPipe<T>::kFixed && lr >= 4) return lr;
+  lr = 5;
+  while (lr > 0 && (per_replica << lr) > 226 * 1024 - UpdPipe<T>::kFixed) --lr;
   return lr;
 }
 
@@ -372,8 +379,15 @@ zo_status launch_update_t(zo_ctx *ctx, const float *coef, int n, const uint32_t 
   // on top, within the 227 KB a CTA may have)
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), 226 * 1024);
   if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "update_kernel setup: %s", cudaGetErrorString(e));
+  int per_sm = 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kUThreads, smem) != cudaSuccess ||
+      per_sm < 1) {
+    cudaGetLastError();
+    per_sm = 1;
+  }
   const int64_t n_chunks = (ctx->M + kUChunk - 1) / kUChunk;
-  const int64_t blocks = n_chunks < kSmCount ? n_chunks : kSmCount;
+  const int64_t cap = (int64_t)kSmCount * per_sm;
+  const int64_t blocks = n_chunks < cap ? n_chunks : cap;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)blocks);
   cfg.blockDim = dim3(kUThreads);
