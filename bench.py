@@ -48,11 +48,18 @@ SM_COUNT, ISSUE_PER_SM_CLOCK = 148, 4
 # that capture, not from this run) only while the sources still hash to it; otherwise null.
 #   quad_octet_kernel, M = 2^24: DRAM bytes (read + write) and warp instructions per launch.
 LOSS_TRAFFIC = {"sources": ("zo_loss.cu", "zo_internal.cuh"),
-                "sources_sha256": "725eacfcbeef93d6ed28cc732c5693f4d65e2341808033820719392cc2b40e5e",
-                "bytes": 138.57e6, "warp_instructions": 90.42e6}
-#   gemm_bf16_kernel at the OPT-30B layer shapes (T = 16384): DRAM bytes per launch averaged
-#   over the four projections of one layer (filled in from a capture; None until then).
-GEMM_TRAFFIC = {"sources": ("zo_gemm.cu", "zo_tc.cuh"), "sources_sha256": None, "bytes": None}
+                "sources_sha256": "347def2504d19bf9fb19393e6166cf4226ca58880a5027e41e6f1770ef8b1a8b",
+                "bytes": 138.50e6, "warp_instructions": 89.22e6}
+#   update_kernel on 2^28 elements (the streaming sweep), per dtype and probe count: warp
+#   instructions per launch (`bench.py --streaming-only` under ncu).
+UPDATE_INSTR = {"sources": ("zo_step.cu", "zo_internal.cuh"), "sources_sha256": None,
+                "warp_instructions": None}
+#   gemm_pair_kernel at the OPT-30B layer shapes (T = 16384): DRAM bytes (read + write) per
+#   launch averaged over the four projections of one layer (the step's other GEMM launches,
+#   the pruned last layer's few rows, move a negligible share of its bytes).
+GEMM_TRAFFIC = {"sources": ("zo_gemm.cu", "zo_tc.cuh"),
+                "sources_sha256": "4fc2cd08f0f9c3ca4065b276d10f195ccbeff43a4bc77a4045f05cefb8c18796",
+                "bytes": 13.86e9}
 
 
 def sources_sha256(names):
@@ -328,6 +335,91 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ------------------------------------------------------------------ streaming kernels
+
+def streaming_sweep(zo, torch, dev, stream, flush, hbm_peak):
+    """The update (n = 1 .. 160) and the window perturbation on 2^28-element vectors (1 GiB
+    fp32, 512 MiB bf16: far larger than L2, and L2 flushed before every timed launch), fp32
+    then bf16; per launch class 1 untimed + 5 timed launches.  Each update entry carries two
+    rooflines: the HBM fraction of its algorithmic bytes, and its instruction-issue fraction,
+    the recorded ncu warp-instruction count of that (dtype, n) (UPDATE_INSTR, while the
+    sources are unchanged) per second against 148 SMs x 4 per clock at the median SM clock
+    sampled over the sweep; `bound` names the larger."""
+    elems = 1 << 28
+    reps = 5
+
+    def timed_reps(fn):
+        tot = 0.0
+        for _ in range(reps):
+            flush.zero_()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            ev[0].record(stream)
+            fn()
+            ev[1].record(stream)
+            torch.cuda.synchronize()
+            tot += ev[0].elapsed_time(ev[1])
+        return 1e3 * tot / reps
+
+    instr = captured(UPDATE_INSTR, "warp_instructions")
+    out = {}
+    cs_clock = ClockSampler(torch.cuda.current_device())
+    for dt, esz in (("f32", 4), ("bf16", 2)):
+        g = torch.Generator(device=dev)
+        g.manual_seed(5)
+        th_s = torch.empty(elems, dtype=torch.float32 if dt == "f32" else torch.bfloat16, device=dev)
+        th_s.normal_(generator=g)
+        out_s = torch.empty_like(th_s)
+        cs = zo.zo_create(th_s, seed=7, stream=stream.cuda_stream)
+        ent = {"elements": elems, "l2": "flushed before every timed launch", "update": {}}
+        for nn in (1, 2, 4, 8, 16, 32, 64, 160):
+            cz = torch.zeros(nn, dtype=torch.float32, device=dev)  # theta unchanged
+            zo.zo_update(cs, cz, nn)
+            us = timed_reps(lambda: zo.zo_update(cs, cz, nn))
+            gbs = 2 * esz * elems / (us * 1e-6) / 1e9
+            ent["update"][str(nn)] = {"us": us, "GBps": gbs, "frac_hbm": gbs / hbm_peak}
+        zo.zo_perturb(cs, +1, EPS, 3)
+        zo.zo_perturb_range(cs, 0, elems, out_s)
+        us = timed_reps(lambda: zo.zo_perturb_range(cs, 0, elems, out_s))
+        zo.zo_restore(cs)
+        gbs = 2 * esz * elems / (us * 1e-6) / 1e9
+        ent["perturb"] = {"us": us, "GBps": gbs, "frac_hbm": gbs / hbm_peak}
+        cs.close()
+        out[dt] = ent
+        del th_s, out_s
+    clk = cs_clock.stop()
+    mhz = clk["sm_mhz"] if clk else None
+    for dt, ent in out.items():
+        for nn, e in ent["update"].items():
+            wi = instr.get(dt, {}).get(nn) if instr else None
+            if wi is None or not mhz:
+                e["frac_issue"], e["bound"] = None, None
+                continue
+            e["warp_instructions"] = wi
+            e["frac_issue"] = wi / (e["us"] * 1e-6) / (SM_COUNT * ISSUE_PER_SM_CLOCK * mhz * 1e6)
+            e["bound"] = "issue" if e["frac_issue"] > e["frac_hbm"] else "hbm"
+    out["sm_mhz"] = mhz
+    out["instructions_from"] = ("ncu capture of these launches (smsp__inst_executed.sum), "
+                                "not this run" if instr else None)
+    torch.cuda.empty_cache()
+    return out
+
+
+def streaming_arm(args):
+    """Only the streaming sweep (the command its instruction-count capture profiles)."""
+    import torch
+
+    import zero_order_forward_b200 as zo
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    hbm_peak, kind = peaks()
+    print(json.dumps({"streaming_only": True, "peak_kind": kind,
+                      "streaming": streaming_sweep(zo, torch, dev, stream, flush, hbm_peak)}),
+          flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------ GPU arm
 
 def gpu_arm(args, sub=False):
@@ -472,37 +564,7 @@ def gpu_arm(args, sub=False):
     coef = torch.from_numpy(synth.coefficients(n, seed=1) * 0).to(dev)  # zero: theta unchanged
     upd_us = timed_reps(lambda: zo.zo_update(ctx, coef, n), 10)
 
-    # the streaming kernels across probe counts and dtypes (theta of 2^28 elements, 1 GiB fp32 /
-    # 512 MiB bf16, far larger than L2, and L2 flushed before every timed launch): the update's
-    # and the unpack/apply kernel's bandwidth against the measured HBM peak, and for the update
-    # the lane-instruction budget that bandwidth leaves per element
-    streaming = {}
-    if world == 1:
-        elems = 1 << 28
-        for dt, esz in (("f32", 4), ("bf16", 2)):
-            g = torch.Generator(device=dev)
-            g.manual_seed(5)
-            th_s = torch.empty(elems, dtype=torch.float32 if dt == "f32" else torch.bfloat16, device=dev)
-            th_s.normal_(generator=g)
-            out_s = torch.empty_like(th_s)
-            cs = zo.zo_create(th_s, seed=7, stream=stream.cuda_stream)
-            ent = {"elements": elems, "l2": "flushed before every timed launch", "update": {}}
-            for nn in (1, 2, 4, 8, 16, 32, 64, 160):
-                cz = torch.zeros(nn, dtype=torch.float32, device=dev)  # theta unchanged
-                zo.zo_update(cs, cz, nn)
-                us = timed_reps(lambda: zo.zo_update(cs, cz, nn), 5)
-                gbs = 2 * esz * elems / (us * 1e-6) / 1e9
-                ent["update"][str(nn)] = {"us": us, "GBps": gbs, "frac_hbm": gbs / hbm_peak}
-            zo.zo_perturb(cs, +1, EPS, 3)
-            zo.zo_perturb_range(cs, 0, elems, out_s)
-            us = timed_reps(lambda: zo.zo_perturb_range(cs, 0, elems, out_s), 5)
-            zo.zo_restore(cs)
-            gbs = 2 * esz * elems / (us * 1e-6) / 1e9
-            ent["perturb"] = {"us": us, "GBps": gbs, "frac_hbm": gbs / hbm_peak}
-            cs.close()
-            streaming[dt] = ent
-            del th_s, out_s
-        torch.cuda.empty_cache()
+    streaming = streaming_sweep(zo, torch, dev, stream, flush, hbm_peak) if world == 1 else {}
 
     # end to end through the public API with host buffers: D copied in, losses copied out
     D_host = torch.from_numpy(D_np[first:first + count]).pin_memory()
@@ -954,8 +1016,8 @@ def decoder_arm(args):
             "forwards_per_step": fwds,
             "step_ms": step_ms,
             "roofline": {
-                "kernel": "gemm_bf16_kernel (tcgen05/TMEM, TMA-fed: the QKV, output and "
-                          "feed-forward projections of every forward)",
+                "kernel": "gemm_pair_kernel (tcgen05 on CTA pairs, TMEM accumulators, TMA-fed: "
+                          "the QKV, output and feed-forward projections of every forward)",
                 "bound": "tensor", "achieved": g.get("tflops"), "peak": peak_s,
                 "unit": "TFLOP/s", "frac": (g.get("tflops") or 0.0) / peak_s,
                 "peak_kind": f"{bf16_kind} sustained bf16 GEMM (the kernel runs inside a "
@@ -1027,8 +1089,12 @@ def kernels_arm(args):
     reps = args.steps
 
     def timed(fn):
+        """Average launch time (us) with L2 flushed before each launch, and the median SM
+        clock sampled over the timed launches."""
         tot = 0.0
         fn()
+        torch.cuda.synchronize()
+        cs = ClockSampler(0)
         for _ in range(reps):
             flush.zero_()
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
@@ -1037,11 +1103,43 @@ def kernels_arm(args):
             ev[1].record(stream)
             torch.cuda.synchronize()
             tot += ev[0].elapsed_time(ev[1])
+        clk = cs.stop()
+        clocks[0] = clk["sm_mhz"] if clk else None
         return 1e3 * tot / reps
+
+    clocks = [None]
+    out = {}
+    # the streaming kernels first, before the GEMMs heat the GPU up to its power cap
+    import synth
+    segs = (synth.qwen_segments if qwen else synth.opt_segments)(dict(cfg, n_layers=1))
+    lead = 1 if qwen else 2
+    layer = sum(c for _, c in segs[lead:-(1 if qwen else 2)])
+    th = torch.empty(layer, dtype=torch.bfloat16, device=dev).normal_(0, 0.02)
+    win = torch.empty_like(th)
+    c2 = zo.zo_create(th, seed=0, stream=stream.cuda_stream)
+    zo.zo_perturb(c2, +1, 1e-3, 3)
+    us = timed(lambda: zo.zo_perturb_range(c2, 0, layer, win))
+    zo.zo_restore(c2)
+    gb = 4.0 * layer / (us * 1e-6) / 1e9
+    out["perturb_window"] = {"elements": layer, "us": us, "GBps": gb, "frac_hbm": gb / hbm_peak,
+                             "sm_mhz": clocks[0]}
+    c2.close()
+    del th, win
+    # the update at this n_pert on a 2^30-element bf16 slice
+    Mu = 1 << 30
+    th = torch.empty(Mu, dtype=torch.bfloat16, device=dev).normal_(0, 0.02)
+    c3 = zo.zo_create(th, seed=0, stream=stream.cuda_stream)
+    coef = torch.zeros(n, dtype=torch.float32, device=dev)
+    us = timed(lambda: zo.zo_update(c3, coef, n))
+    gb = 4.0 * Mu / (us * 1e-6) / 1e9
+    out["update"] = {"elements": Mu, "n_pert": n, "us": us, "GBps": gb, "frac_hbm": gb / hbm_peak,
+                     "sm_mhz": clocks[0]}
+    zo.zo_sync(c3)
+    c3.close()
+    del th, coef
 
     small = torch.zeros(1024, dtype=torch.bfloat16, device=dev)
     ctx = zo.zo_create(small, seed=0, stream=stream.cuda_stream)
-    out = {}
     shapes = ({"qkv": (T, nq, d, 0), "out": (T, d, na, 2), "gate_up": (T, f, d, 3), "down": (T, d, f, 2)}
               if qwen else
               {"qkv": (T, nq, d, 0), "out": (T, d, na, 2), "fc1": (T, f, d, 1), "fc2": (T, d, f, 2)})
@@ -1058,40 +1156,16 @@ def kernels_arm(args):
         us = timed(lambda: zo.zo_gemm_bf16(ctx, A, Wt, bb, o, Mm, N, K, N, epi))
         fl = 2.0 * Mm * N * K * (2 if epi == 3 else 1)
         out["gemm_" + key] = {"shape": [Mm, N, K], "us": us, "tflops": fl / us / 1e6,
-                              "frac_bf16_burst": fl / us / 1e6 / peak_b}
+                              "frac_bf16_burst": fl / us / 1e6 / peak_b, "sm_mhz": clocks[0]}
     del A, Wt, out_b, out_f
     qkv = torch.randn(T * nq, dtype=torch.bfloat16, device=dev)
     att = torch.empty(T * na, dtype=torch.bfloat16, device=dev)
     us = timed(lambda: zo.zo_attention_gqa(ctx, qkv, att, B, S, H, Hk, e))
     fl = 4.0 * e * B * H * S * (S + 1) / 2
-    out["attention"] = {"us": us, "tflops": fl / us / 1e6, "frac_bf16_burst": fl / us / 1e6 / peak_b}
+    out["attention"] = {"us": us, "tflops": fl / us / 1e6, "frac_bf16_burst": fl / us / 1e6 / peak_b,
+                        "sm_mhz": clocks[0]}
     del qkv, att
     ctx.close()
-    # one layer window, perturbed
-    import synth
-    segs = (synth.qwen_segments if qwen else synth.opt_segments)(dict(cfg, n_layers=1))
-    lead = 1 if qwen else 2
-    layer = sum(c for _, c in segs[lead:-(1 if qwen else 2)])
-    th = torch.empty(layer, dtype=torch.bfloat16, device=dev).normal_(0, 0.02)
-    win = torch.empty_like(th)
-    c2 = zo.zo_create(th, seed=0, stream=stream.cuda_stream)
-    zo.zo_perturb(c2, +1, 1e-3, 3)
-    us = timed(lambda: zo.zo_perturb_range(c2, 0, layer, win))
-    zo.zo_restore(c2)
-    gb = 4.0 * layer / (us * 1e-6) / 1e9
-    out["perturb_window"] = {"elements": layer, "us": us, "GBps": gb, "frac_hbm": gb / hbm_peak}
-    c2.close()
-    del th, win
-    # the update at this n_pert on a 2^30-element bf16 slice
-    Mu = 1 << 30
-    th = torch.empty(Mu, dtype=torch.bfloat16, device=dev).normal_(0, 0.02)
-    c3 = zo.zo_create(th, seed=0, stream=stream.cuda_stream)
-    coef = torch.zeros(n, dtype=torch.float32, device=dev)
-    us = timed(lambda: zo.zo_update(c3, coef, n))
-    gb = 4.0 * Mu / (us * 1e-6) / 1e9
-    out["update"] = {"elements": Mu, "n_pert": n, "us": us, "GBps": gb, "frac_hbm": gb / hbm_peak}
-    zo.zo_sync(c3)
-    c3.close()
     print(json.dumps({"kernels_only": name, "batch": B, "seq": S, "reps": reps,
                       "l2": "flushed before every timed launch", "kernels": out}), flush=True)
     return 0
@@ -1312,6 +1386,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=["quadratic", "mlp", "lowrank"] + sorted(DECODER_WORKLOADS))
     ap.add_argument("--n-pert", type=int, default=None, help="override n_pert (decoder workloads)")
+    ap.add_argument("--streaming-only", action="store_true",
+                    help="only the streaming sweep (update over n_pert, window perturbation); "
+                         "prints a diagnostic line")
     ap.add_argument("--kernels-only", action="store_true",
                     help="time each hot kernel of a decoder workload alone at its shapes "
                          "(--steps = timed launches per kernel); prints a diagnostic line")
@@ -1322,6 +1399,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return reference_arm(args)
+    if args.streaming_only:
+        return streaming_arm(args)
     if args.kernels_only:
         if args.workload not in DECODER_WORKLOADS:
             ap.error("--kernels-only needs a decoder workload")

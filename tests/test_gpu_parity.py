@@ -236,7 +236,10 @@ def test_mlp_loss_matches_oracle(zo):
 @pytest.mark.parametrize("n,M", [(n, M) for n in (1, 7, 8, 13, 64, 160)
                                   for M in (1, 127, 129, 19210, (1 << 20) + 77)] +
                          # many chunks per CTA: the streaming ring wraps around several times
-                         [(16, (1 << 24) + 77), (17, (1 << 24) + 3)])
+                         [(16, (1 << 24) + 77), (17, (1 << 24) + 3)] +
+                         # every shared-memory plan: 32 or 16 table replicas beside a 4- or
+                         # 3-stage ring, two CTAs per SM or one
+                         [(32, (1 << 22) + 5), (40, (1 << 20) + 77)])
 def test_update_bit_exact_vs_mirror_order(zo, M, n, dtype):
     th_np = _theta(M, dtype, seed=M + n)
     th = dev(th_np) if dtype == "f32" else bf16_dev(th_np)

@@ -36,25 +36,30 @@
 namespace zo {
 namespace {
 
-constexpr int kTBM = 128, kTThreads = 192, kTBN = 64;
+constexpr int kTBM = 128, kTThreads = 192;
 constexpr uint32_t kQBox = 128 * 128;  // bytes of one 128-row x 64-column bf16 box
-constexpr uint32_t kKBox = kTBN * 128; // bytes of one 64-row x 64-column bf16 box
 
 // Key tiles of 64 keys.  TMEM (256 columns per CTA, two CTAs per SM): two score buffers of
 // 64 columns, each later overwritten in place by its tile's bf16 probabilities (32 columns),
 // then O (hd columns).  Separate K and V rings in shared memory, so that a key tile is
 // released (and the next one loaded) as soon as its score MMA has completed.
 template <int HD> struct TcAttnCfg {
+  // head dim 128: key tiles of 64, two CTAs per SM (256 TMEM columns each); head dim 64: key
+  // tiles of 32, three CTAs per SM (128 TMEM columns: two 32-column score buffers and O), so
+  // that more query tiles are in flight where a tile's MMAs are short
+  static constexpr int kBN = HD == 128 ? 64 : 32;
   static constexpr int kKS = HD == 128 ? 2 : 4;  // K stages
   static constexpr int kVS = HD == 128 ? 2 : 4;  // V stages
-  static constexpr int kCtas = 2, kTmemCols = 256;
+  static constexpr int kCtas = HD == 128 ? 2 : 3;
+  static constexpr int kTmemCols = HD == 128 ? 256 : 128;
+  static constexpr uint32_t kKBox = kBN * 128;  // bytes of one kBN-row x 64-column bf16 box
 };
 
 template <int HD>
 struct TcAttnSmem {
   static constexpr int kKS = TcAttnCfg<HD>::kKS, kVS = TcAttnCfg<HD>::kVS;
   static constexpr uint32_t kQTile = (HD / 64) * kQBox;   // 128 rows x HD columns
-  static constexpr uint32_t kKTile = (HD / 64) * kKBox;   // 64 rows x HD columns
+  static constexpr uint32_t kKTile = (HD / 64) * TcAttnCfg<HD>::kKBox;  // kBN rows x HD columns
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kK = kQ + kQTile;              // [kKS]
   static constexpr uint32_t kV = kK + kKS * kKTile;        // [kVS]
@@ -83,6 +88,29 @@ __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
   return pack_bf16x2(lo, hi);
 }
 
+// max(a, b, c): one three-input instruction instead of two.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Two lanes of fp32 arithmetic per instruction (sm_100's packed f32x2 forms), each lane
+// rounded exactly as the scalar instruction: (d0, d1) = (a0 * b + c, a1 * b + c).
+__device__ __forceinline__ void fma2_bc(float a0, float a1, float b, float c, float &d0, float &d1) {
+  asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %4};\n\tmov.b64 c, {%5, %5};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+// (s0, s1) += (a0, a1)
+__device__ __forceinline__ void add2(float &s0, float &s1, float a0, float a1) {
+  asm("{\n\t.reg .b64 s, a;\n\t"
+      "mov.b64 s, {%0, %1};\n\tmov.b64 a, {%2, %3};\n\t"
+      "add.rn.f32x2 s, s, a;\n\tmov.b64 {%0, %1}, s;\n\t}"
+      : "+f"(s0), "+f"(s1) : "f"(a0), "f"(a1));
+}
+
 // All lanes of the warp wait for `parity` on `bar`: lane 0 decides (bounded), then every lane
 // observes the completed phase.  Returns false (on every lane) on expiry or abort.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
@@ -105,6 +133,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
   using SM = TcAttnSmem<HD>;
   constexpr int KS = SM::kKS, VS = SM::kVS;
   constexpr uint32_t kCols = TcAttnCfg<HD>::kTmemCols;
+  constexpr int kTBN = TcAttnCfg<HD>::kBN;
+  constexpr uint32_t kKBox = TcAttnCfg<HD>::kKBox;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -251,16 +281,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
 #pragma unroll
       for (int c = 0; c < kTBN / 32; ++c) tc::tmem_ld32(tS + 32u * c, s + 32 * c);
       const int key0 = j * kTBN;
-      const bool edge = key0 + kTBN - 1 > q_first || key0 + kTBN > a.S;
+      // the causal / sequence-end mask touches only the tiles that reach the diagonal or the
+      // end (uniform across the CTA: a real branch, not per-element selects)
+      if (key0 + kTBN - 1 > q_first || key0 + kTBN > a.S) {
+#pragma unroll
+        for (int c = 0; c < kTBN; ++c)
+          if (key0 + c > r || key0 + c >= a.S) s[c] = -INFINITY;
+      }
       // the maximum of the raw scores (the scale is positive), then 2^(s * scale - m) with the
       // scaling folded into the exponent's fused multiply-add
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // 4 independent chains
 #pragma unroll
-      for (int c = 0; c < kTBN; ++c) {
-        if (edge && (key0 + c > r || key0 + c >= a.S)) s[c] = -INFINITY;
-        mx4[c & 3] = fmaxf(mx4[c & 3], s[c]);
-      }
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * a.scale_log2;
+      for (int c = 0; c < kTBN; c += 2) mx4[(c >> 1) & 3] = max3f(mx4[(c >> 1) & 3], s[c], s[c + 1]);
+      const float mx = max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * a.scale_log2;
       const float m_new = fmaxf(m_used, mx);
       // Lazy rescaling: keep the running maximum unless it grows by more than 2^8 (then
       // O and l are rescaled, once the previous tile's P V has completed).
@@ -269,11 +302,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
       if (j == 0 || need) m_used = m_new;
       const float msc = m_used == -INFINITY ? 0.f : m_used;
       uint32_t pk[kTBN / 2];
-      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+      float ls4[4] = {0.f, 0.f, 0.f, 0.f};  // two packed pairs of partial sums
 #pragma unroll
       for (int c = 0; c < kTBN; c += 2) {
-        const float p0 = ex2(fmaf(s[c], a.scale_log2, -msc)), p1 = ex2(fmaf(s[c + 1], a.scale_log2, -msc));
-        ls4[(c >> 1) & 3] += p0 + p1;
+        float x0, x1;
+        fma2_bc(s[c], s[c + 1], a.scale_log2, -msc, x0, x1);
+        const float p0 = ex2(x0), p1 = ex2(x1);
+        if ((c >> 1) & 1) add2(ls4[2], ls4[3], p0, p1);
+        else add2(ls4[0], ls4[1], p0, p1);
         pk[c / 2] = pack2_bf16(p0, p1);
       }
       const float lsum = (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
@@ -293,7 +329,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         }
       }
       // P_j overwrites the first kTBN / 2 columns of S_j (already read into registers)
-      tc::tmem_st32u(tS, pk);
+      if (kTBN == 64) tc::tmem_st32u(tS, pk);
+      else tc::tmem_st16u(tS, pk);
       l += lsum;
       tc::tc_fence_before();
       __syncwarp();
@@ -382,7 +419,7 @@ zo_status launch_attention_tc(zo_ctx *ctx, const uint16_t *qkv, uint16_t *out, i
   const cuuint64_t dims[2] = {(cuuint64_t)ld, (cuuint64_t)B * (cuuint64_t)S};
   const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
   const cuuint32_t boxq[2] = {64, (cuuint32_t)kTBM},
-                   boxkv[2] = {64, (cuuint32_t)kTBN};
+                   boxkv[2] = {64, (cuuint32_t)(hd == 128 ? TcAttnCfg<128>::kBN : TcAttnCfg<64>::kBN)};
   const cuuint32_t estr[2] = {1, 1};
   for (int m = 0; m < 2; ++m)
     if (fn(m ? &tmkv : &tmq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(qkv), dims,

@@ -55,6 +55,34 @@ __device__ __forceinline__ uint4 philox10(uint4 c, uint32_t k0, uint32_t k1) {
   return c;
 }
 
+// The ten rounds' keys (k0 + r W0, k1 + r W1), computed once on the host.  A kernel that takes
+// them as a __grid_constant__ parameter reads each key from the constant bank inside the
+// round's three-input xor, instead of advancing two key registers every round.
+struct RoundKeys {
+  uint32_t k[20];  // round r: k[2r] (xor-ed into word 0), k[2r + 1] (into word 2)
+};
+
+inline RoundKeys round_keys(uint32_t k0, uint32_t k1) {
+  RoundKeys rk;
+  for (int r = 0; r < 10; ++r) {
+    rk.k[2 * r] = k0 + (uint32_t)r * 0x9E3779B9u;
+    rk.k[2 * r + 1] = k1 + (uint32_t)r * 0xBB67AE85u;
+  }
+  return rk;
+}
+
+// The same ten rounds with the key schedule read from rk.
+__device__ __forceinline__ uint4 philox10(uint4 c, const RoundKeys &rk) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t a = c.x, b = c.z;
+    const uint32_t hi_a = __umulhi(0xD2511F53u, a), lo_a = 0xD2511F53u * a;
+    const uint32_t hi_b = __umulhi(0xCD9E8D57u, b), lo_b = 0xCD9E8D57u * b;
+    c = make_uint4(hi_b ^ c.y ^ rk.k[2 * r], lo_b, hi_a ^ c.w ^ rk.k[2 * r + 1], lo_a);
+  }
+  return c;
+}
+
 // Sign layout ("8 signs per byte"): one Philox block holds the signs of the 16 elements of
 // group g (elements 16g .. 16g+15) under the 8 probes of one octet (probes 8p .. 8p+7).
 // Byte b of the little-endian block (bits 8(b&3).. of word b>>2) belongs to element 16g+b,
@@ -63,6 +91,11 @@ __device__ __forceinline__ uint4 philox10(uint4 c, uint32_t k0, uint32_t k1) {
 __device__ __forceinline__ uint4 sign_block(uint64_t g, uint32_t octet, uint32_t step,
                                             uint32_t k0, uint32_t k1) {
   return philox10(make_uint4((uint32_t)g, (uint32_t)(g >> 32), octet, step), k0, k1);
+}
+
+__device__ __forceinline__ uint4 sign_block(uint64_t g, uint32_t octet, uint32_t step,
+                                            const RoundKeys &rk) {
+  return philox10(make_uint4((uint32_t)g, (uint32_t)(g >> 32), octet, step), rk);
 }
 
 // The 16 sign bits of probe `probe` in the block of its octet: element 16g+b at bit b.
@@ -77,6 +110,11 @@ __device__ __forceinline__ uint32_t probe_bits16(const uint4 &v, uint32_t probe)
 __device__ __forceinline__ uint32_t probe_group_bits(uint64_t g, uint32_t probe, uint32_t step,
                                                      uint32_t k0, uint32_t k1) {
   return probe_bits16(sign_block(g, probe >> 3, step, k0, k1), probe);
+}
+
+__device__ __forceinline__ uint32_t probe_group_bits(uint64_t g, uint32_t probe, uint32_t step,
+                                                     const RoundKeys &rk) {
+  return probe_bits16(sign_block(g, probe >> 3, step, rk), probe);
 }
 
 __device__ __forceinline__ uint32_t word_of(const uint4 &v, int w) {

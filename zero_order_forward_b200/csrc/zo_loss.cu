@@ -410,9 +410,10 @@ quad_loss_kernel(const float *__restrict__ theta, const float *__restrict__ D, i
 template <bool CLEAN, int NOCT, bool DOT>
 __global__ void __launch_bounds__(kQThreads, kOBlocksPerSm)
 quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, int64_t M,
-                  ProbeKey pk, uint32_t octet, int count, int64_t n_chunks, double *partials,
-                  unsigned int *counter, double *out_plus, double *out_minus, double *out_clean,
-                  uint32_t *err, int dir, uint32_t vk0, uint32_t vk1) {
+                  ProbeKey pk, const __grid_constant__ RoundKeys rk, uint32_t octet, int count,
+                  int64_t n_chunks, double *partials, unsigned int *counter, double *out_plus,
+                  double *out_minus, double *out_clean, uint32_t *err, int dir, uint32_t vk0,
+                  uint32_t vk1) {
   static_assert(NOCT == 2 || NOCT == 4 || NOCT == 8, "two, four or eight octets per pass");
   constexpr int G = NOCT == 8 ? 4 : 2;     // lanes sharing their tables (a pair or a quad)
   constexpr int LO = NOCT / G;             // octets per thread
@@ -462,7 +463,7 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
       // lane l in rounds 0, 1 and lane l ^ 2 (the other vector) in rounds 2, 3.
       uint32_t wo2[kOIters], wp2[kOIters];
       if constexpr (NOCT == 2) {
-        const uint4 blk = sign_block(g0 + 64 * (q >> 1), octet + (uint32_t)(q & 1), step, pk.k0, pk.k1);
+        const uint4 blk = sign_block(g0 + 64 * (q >> 1), octet + (uint32_t)(q & 1), step, rk);
         uint32_t R[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
@@ -494,7 +495,7 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
           // lane q generates octet q; lane l reads octet sw(l) in rounds 0, 1 and octet
           // sw(l) ^ 1 in rounds 2, 3 (sw swaps the two bits of q), even word then odd
           const int sw = ((q & 1) << 1) | (q >> 1);
-          const uint4 blk = sign_block(g0 + 64 * k, octet + (uint32_t)q, step, pk.k0, pk.k1);
+          const uint4 blk = sign_block(g0 + 64 * k, octet + (uint32_t)q, step, rk);
           uint32_t R[4];
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
@@ -548,7 +549,7 @@ quad_octet_kernel(const float *__restrict__ theta, const float *__restrict__ D, 
           // octets 2q, 2q + 1 itself; word m of a block is the vector of quad lane m
 #pragma unroll
           for (int j = 0; j < LO; ++j) {
-            const uint4 blk = sign_block(g0 + 64 * k, octet + (uint32_t)(LO * q + j), step, pk.k0, pk.k1);
+            const uint4 blk = sign_block(g0 + 64 * k, octet + (uint32_t)(LO * q + j), step, rk);
             uint32_t w[4] = {blk.x, blk.y, blk.z, blk.w};
             if (q & 1) {  // w[r] <- word q ^ r
               const uint32_t a = w[0], b = w[2];
@@ -847,7 +848,7 @@ zo_status launch_quad_octet_t(zo_ctx *ctx, const ProbeKey &pk, uint32_t octet, i
   cfg.numAttrs = 1;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, quad_octet_kernel<CLEAN, NOCT, DOT>,
                                            static_cast<const float *>(ctx->params), D, ctx->M, pk,
-                                           octet, count, n_chunks, ctx->partials, ctx->counter,
+                                           round_keys(pk.k0, pk.k1), octet, count, n_chunks, ctx->partials, ctx->counter,
                                            out_plus, out_minus, out_clean, &ctx->dstate->flags, dir, vk0,
                                            vk1);
   if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "quad_octet_kernel: %s", cudaGetErrorString(e));

@@ -136,7 +136,8 @@ struct PipeSmem {
 template <typename T>
 __global__ void __launch_bounds__(kPThreads)
 perturb_pipe_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t first,
-                    int64_t count, ProbeKey pk, int64_t n_chunks, uint32_t *err) {
+                    int64_t count, ProbeKey pk, const __grid_constant__ RoundKeys rk,
+                    int64_t n_chunks, uint32_t *err) {
   using SM = PipeSmem<T>;
   constexpr int N = Vec<T>::N;
   extern __shared__ __align__(128) uint8_t psm[];
@@ -207,7 +208,7 @@ perturb_pipe_kernel(const T *__restrict__ theta, T *__restrict__ out, int64_t fi
       const int64_t ws = cs + (int64_t)cw * kSlice;  // this warp's slice
       uint32_t mine = 0u;
       if (pk.sign)
-        mine = probe_group_bits(pk.g_off + (uint64_t)(ws / kGroup) + lane, pk.probe, step, pk.k0, pk.k1);
+        mine = probe_group_bits(pk.g_off + (uint64_t)(ws / kGroup) + lane, pk.probe, step, rk);
       int ok = 1;  // decided per warp, as in the loss pipeline
       if (lane == 0) ok = (!abort_flag && tc::mbar_wait(&full[s], ph)) ? 1 : 0;
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -320,8 +321,8 @@ zo_status launch_pipe(zo_ctx *ctx, const ProbeKey &pk, int64_t first, int64_t co
   const int64_t cap = (int64_t)kSmCount * per_sm;
   const int64_t blocks = n_chunks < cap ? n_chunks : cap;
   perturb_pipe_kernel<T><<<(unsigned)blocks, kPThreads, SM::kBytes, ctx->stream>>>(
-      static_cast<const T *>(ctx->params), static_cast<T *>(out), first, count, pk, n_chunks,
-      &ctx->dstate->flags);
+      static_cast<const T *>(ctx->params), static_cast<T *>(out), first, count, pk,
+      round_keys(pk.k0, pk.k1), n_chunks, &ctx->dstate->flags);
   return check_launch(ctx, "perturb_pipe_kernel");
 }
 

@@ -184,13 +184,13 @@ constexpr int kUConsumers = 16;
 constexpr int kUThreads = 32 * (1 + kUConsumers);
 constexpr int kUChunk = kUConsumers * 32 * kGroup;  // 8192 elements
 
-template <typename T> struct UpdPipe {
-  static constexpr int kStages = sizeof(T) == 2 ? 4 : 3;
+template <typename T, int STAGES> struct UpdPipe {
+  static constexpr int kStages = STAGES;
   static constexpr int kStage = kUChunk * (int)sizeof(T);
   static constexpr int kRing = kStages * kStage;
   static constexpr int kLut = kRing + 2 * kStages * 8;  // after the ring and its barriers
   static constexpr int kFixed = kLut;
-  // bf16 runs two CTAs per SM at small n (registers capped at 56 per thread), fp32 one
+  // bf16 runs two CTAs per SM (registers capped at 56 per thread), fp32 one
   static constexpr int kMinBlocks = sizeof(T) == 2 ? 2 : 1;
 };
 
@@ -222,12 +222,12 @@ __device__ __forceinline__ void build_tables(float *lut, const float *__restrict
 // v[e] -= (sum over octets of the table entry of element e's sign byte), fixed order.
 template <int LOG_R>
 __device__ __forceinline__ void apply_probes(float v[16], const float *mine, uint64_t g, int octets,
-                                             uint32_t step, uint32_t k0, uint32_t k1) {
+                                             uint32_t step, const RoundKeys &rk) {
   float acc[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) acc[e] = 0.f;
   for (int o = 0; o < octets; ++o) {
-    const uint4 blk = sign_block(g, (uint32_t)o, step, k0, k1);
+    const uint4 blk = sign_block(g, (uint32_t)o, step, rk);
     const uint32_t w[4] = {blk.x, blk.y, blk.z, blk.w};
     const float *tab = mine + ((o * 256) << LOG_R);
 #pragma unroll
@@ -238,12 +238,12 @@ __device__ __forceinline__ void apply_probes(float v[16], const float *mine, uin
   for (int e = 0; e < 16; ++e) v[e] = __fsub_rn(v[e], acc[e]);
 }
 
-template <typename T, int LOG_R>
-__global__ void __launch_bounds__(kUThreads, UpdPipe<T>::kMinBlocks)
+template <typename T, int LOG_R, int STAGES>
+__global__ void __launch_bounds__(kUThreads, UpdPipe<T, STAGES>::kMinBlocks)
 update_kernel(T *__restrict__ theta, int64_t M, const float *__restrict__ coef, int n,
-              const uint32_t *step_ptr, const uint32_t *ok_ptr, uint32_t k0, uint32_t k1,
+              const uint32_t *step_ptr, const uint32_t *ok_ptr, const __grid_constant__ RoundKeys rk,
               uint64_t g_off, uint32_t *err) {
-  using U = UpdPipe<T>;
+  using U = UpdPipe<T, STAGES>;
   constexpr int N = 16 / (int)sizeof(T);  // elements per 16-byte vector
   extern __shared__ __align__(128) uint8_t usm[];
   uint64_t *full = reinterpret_cast<uint64_t *>(usm + U::kRing);
@@ -326,7 +326,7 @@ update_kernel(T *__restrict__ theta, int64_t M, const float *__restrict__ coef, 
       Elem<T>::load16s(st + ct * kGroup, v);
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&empty[s]);  // the stage is free again
-      apply_probes<LOG_R>(v, mine, (uint64_t)(e0 / kGroup) + g_off, octets, step, k0, k1);
+      apply_probes<LOG_R>(v, mine, (uint64_t)(e0 / kGroup) + g_off, octets, step, rk);
       Elem<T>::store16(theta + e0, v);
       continue;
     }
@@ -344,7 +344,7 @@ update_kernel(T *__restrict__ theta, int64_t M, const float *__restrict__ coef, 
     __syncwarp();
     if (lane == 0) tc::mbar_arrive(&empty[s]);  // the stage is free again
     if (e0 >= M) continue;
-    apply_probes<LOG_R>(v, mine, (uint64_t)(e0 / kGroup) + g_off, octets, step, k0, k1);
+    apply_probes<LOG_R>(v, mine, (uint64_t)(e0 / kGroup) + g_off, octets, step, rk);
     if (whole) {
       Elem<T>::store16(theta + e0, v);
     } else {
@@ -355,29 +355,49 @@ update_kernel(T *__restrict__ theta, int64_t M, const float *__restrict__ coef, 
   }
 }
 
-// Replicas of the tables beside the ring: when 16 or more fit within half an SM's shared
-// memory (112 KB per CTA), two CTAs share an SM (34 warps: the kernel is bound by instruction
-// issue); otherwise one CTA takes up to 226 KB.
+// Shared-memory plan: table replicas R = 2^log_r and ring stages.  A lookup is conflict-free
+// at R = 32 (lane l reads replica l); at R = 16 lanes l and l + 16 share a replica and split
+// into two wavefronts whenever their entries differ in bank.  bf16 prefers two CTAs per SM
+// (34 warps; the kernel is bound by instruction issue and shared-memory wavefronts): R = 32
+// with the deepest ring (4 or 3 stages) that fits, else R = 16.  Otherwise (fp32, or large
+// n) one CTA takes up to 226 KB with the largest R that fits beside its ring.
+struct UpdPlan {
+  int log_r, stages;
+};
+
+// Two CTAs per SM: 228 KB per SM, less 1 KB reserved per CTA and the kernel's static words.
+constexpr int64_t kTwoCtaBudget = 113 * 1024 - 64;
+constexpr int64_t kOneCtaBudget = 226 * 1024;
+
 template <typename T>
-int update_log_replicas(int n) {
+UpdPlan update_plan(int n) {
   const int64_t per_replica = (int64_t)((n + 7) / 8) * 256 * 4;
+  if constexpr (sizeof(T) == 2) {
+    const int64_t ring4 = UpdPipe<T, 4>::kFixed, ring3 = UpdPipe<T, 3>::kFixed;
+    for (int lr = 5; lr >= 4; --lr) {
+      if (ring4 + (per_replica << lr) <= kTwoCtaBudget) return {lr, 4};
+      if (ring3 + (per_replica << lr) <= kTwoCtaBudget) return {lr, 3};
+    }
+    int lr = 5;
+    while (lr > 0 && ring4 + (per_replica << lr) > kOneCtaBudget) --lr;
+    return {lr, 4};
+  }
+  const int64_t ring = UpdPipe<T, 3>::kFixed;
   int lr = 5;
-  while (lr > 0 && (per_replica << lr) > 112 * 1024 - UpdPipe<T>::kFixed) --lr;
-  if ((per_replica << lr) <= 112 * 1024 - UpdPipe<T>::kFixed && lr >= 4) return lr;
-  lr = 5;
-  while (lr > 0 && (per_replica << lr) > 226 * 1024 - UpdPipe<T>::kFixed) --lr;
-  return lr;
+  while (lr > 0 && ring + (per_replica << lr) > kOneCtaBudget) --lr;
+  return {lr, 3};
 }
 
-template <typename T, int LOG_R>
+template <typename T, int LOG_R, int STAGES>
 zo_status launch_update_t(zo_ctx *ctx, const float *coef, int n, const uint32_t *step_ptr,
                           const uint32_t *ok_ptr, uint32_t k0, uint32_t k1) {
-  const size_t smem = (size_t)UpdPipe<T>::kFixed + ((size_t)((n + 7) / 8) * 256 * sizeof(float) << LOG_R);
-  auto kern = update_kernel<T, LOG_R>;
+  const size_t smem = (size_t)UpdPipe<T, STAGES>::kFixed +
+                      ((size_t)((n + 7) / 8) * 256 * sizeof(float) << LOG_R);
+  auto kern = update_kernel<T, LOG_R, STAGES>;
   // the table size varies with n: raise the limit once to the largest a CTA may use (the
-  // replica budget keeps every launch within 226 KB; the kernel's static shared memory comes
-  // on top, within the 227 KB a CTA may have)
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), 226 * 1024);
+  // plan keeps every launch within 226 KB; the kernel's static shared memory comes on top,
+  // within the 227 KB a CTA may have)
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), (int)kOneCtaBudget);
   if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "update_kernel setup: %s", cudaGetErrorString(e));
   int per_sm = 1;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kUThreads, smem) != cudaSuccess ||
@@ -400,24 +420,36 @@ zo_status launch_update_t(zo_ctx *ctx, const float *coef, int n, const uint32_t 
   cfg.numAttrs = 1;
   const int slot = ktime_begin(ctx);
   e = cudaLaunchKernelEx(&cfg, kern, static_cast<T *>(ctx->params), ctx->M, coef, n, step_ptr,
-                         ok_ptr, k0, k1, (uint64_t)(ctx->first_element / kGroup), &ctx->dstate->flags);
+                         ok_ptr, round_keys(k0, k1), (uint64_t)(ctx->first_element / kGroup),
+                         &ctx->dstate->flags);
   if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "update_kernel: %s", cudaGetErrorString(e));
   const zo_status st = check_launch(ctx, "update_kernel");
   if (st == ZO_OK) ktime_end(ctx, slot, ZO_KT_UPDATE, 2.0 * sizeof(T) * (double)ctx->M);
   return st;
 }
 
+template <typename T, int STAGES>
+zo_status launch_update_s(zo_ctx *ctx, int log_r, const float *coef, int n,
+                          const uint32_t *step_ptr, const uint32_t *ok_ptr, uint32_t k0,
+                          uint32_t k1) {
+  switch (log_r) {
+    case 5: return launch_update_t<T, 5, STAGES>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
+    case 4: return launch_update_t<T, 4, STAGES>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
+    case 3: return launch_update_t<T, 3, STAGES>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
+    case 2: return launch_update_t<T, 2, STAGES>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
+    case 1: return launch_update_t<T, 1, STAGES>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
+    default: return launch_update_t<T, 0, STAGES>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
+  }
+}
+
 template <typename T>
 zo_status launch_update_r(zo_ctx *ctx, const float *coef, int n, const uint32_t *step_ptr,
                           const uint32_t *ok_ptr, uint32_t k0, uint32_t k1) {
-  switch (update_log_replicas<T>(n)) {
-    case 5: return launch_update_t<T, 5>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
-    case 4: return launch_update_t<T, 4>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
-    case 3: return launch_update_t<T, 3>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
-    case 2: return launch_update_t<T, 2>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
-    case 1: return launch_update_t<T, 1>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
-    default: return launch_update_t<T, 0>(ctx, coef, n, step_ptr, ok_ptr, k0, k1);
+  const UpdPlan p = update_plan<T>(n);
+  if constexpr (sizeof(T) == 2) {
+    if (p.stages == 4) return launch_update_s<T, 4>(ctx, p.log_r, coef, n, step_ptr, ok_ptr, k0, k1);
   }
+  return launch_update_s<T, 3>(ctx, p.log_r, coef, n, step_ptr, ok_ptr, k0, k1);
 }
 
 }  // namespace
