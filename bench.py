@@ -52,8 +52,13 @@ LOSS_TRAFFIC = {"sources": ("zo_loss.cu", "zo_internal.cuh"),
                 "bytes": 138.50e6, "warp_instructions": 89.22e6}
 #   update_kernel on 2^28 elements (the streaming sweep), per dtype and probe count: warp
 #   instructions per launch (`bench.py --streaming-only` under ncu).
-UPDATE_INSTR = {"sources": ("zo_step.cu", "zo_internal.cuh"), "sources_sha256": None,
-                "warp_instructions": None}
+UPDATE_INSTR = {"sources": ("zo_step.cu", "zo_internal.cuh"),
+                "sources_sha256": "e9bb413b69819c1a09adbe59f72eca7616d2ec92b53c210f213d25589e5224b2",
+                "warp_instructions": {
+                    "f32": {"1": 127.80e6, "2": 127.87e6, "4": 127.87e6, "8": 127.91e6,
+                            "16": 184.14e6, "32": 297.79e6, "64": 523.93e6, "160": 1196.59e6},
+                    "bf16": {"1": 150.25e6, "2": 150.34e6, "4": 150.40e6, "8": 150.48e6,
+                             "16": 207.25e6, "32": 323.66e6, "64": 551.14e6, "160": 1238.20e6}}}
 #   gemm_pair_kernel at the OPT-30B layer shapes (T = 16384): DRAM bytes (read + write) per
 #   launch averaged over the four projections of one layer (the step's other GEMM launches,
 #   the pruned last layer's few rows, move a negligible share of its bytes).
@@ -936,30 +941,38 @@ def decoder_arm(args):
             for _ in range(2):
                 zo.zo_gemm_bf16(ctx, A, Wt, bb, out, Mm, N, K, N, epi)
             ge = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            clk = ClockSampler(local_rank)
             ge[0].record(stream)
             for _ in range(5):
                 zo.zo_gemm_bf16(ctx, A, Wt, bb, out, Mm, N, K, N, epi)
             ge[1].record(stream)
             torch.cuda.synchronize()
+            clk = clk.stop()
             us = 1e3 * ge[0].elapsed_time(ge[1]) / 5
             fl = 2.0 * Mm * N * K * (2 if epi == 3 else 1)
             gemm_shapes[key] = {"shape": [Mm, N, K], "avg_launch_us": us, "tflops": fl / us / 1e6,
-                                "frac_bf16_burst": fl / us / 1e6 / peak_b}
+                                "frac_bf16_burst": fl / us / 1e6 / peak_b,
+                                "sm_mhz": clk["sm_mhz"] if clk else None}
         del A, Wt, out_b, out_f
         qkv = torch.randn(T * nq, dtype=torch.bfloat16, device=dev)
         att = torch.empty(T * na, dtype=torch.bfloat16, device=dev)
         for _ in range(2):
             zo.zo_attention_gqa(ctx, qkv, att, B, S, H, Hk, e)
         ae = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        clk = ClockSampler(local_rank)
         ae[0].record(stream)
         for _ in range(5):
             zo.zo_attention_gqa(ctx, qkv, att, B, S, H, Hk, e)
         ae[1].record(stream)
         torch.cuda.synchronize()
+        clk = clk.stop()
         attn_us = 1e3 * ae[0].elapsed_time(ae[1]) / 5
         attn_flops = 4.0 * e * B * H * S * (S + 1) / 2
         attn_alone = {"avg_launch_us": attn_us, "tflops": attn_flops / attn_us / 1e6,
-                      "frac_bf16_burst": attn_flops / attn_us / 1e6 / peak_b}
+                      "frac_bf16_burst": attn_flops / attn_us / 1e6 / peak_b,
+                      "sm_mhz": clk["sm_mhz"] if clk else None,
+                      "note": "timed after the steps, at the clock the power cap leaves; "
+                              "`bench.py --kernels-only` times it on a cool GPU"}
         del qkv, att
         zo.zo_sync(ctx)
 
