@@ -90,6 +90,7 @@ def test_attention_matches_numpy(zo, ctx, B, S, H, d):
     out = torch.zeros((B * S, d), dtype=torch.bfloat16, device="cuda")
     zo.zo_attention(ctx, qkv, out, B, S, H, d)
     torch.cuda.synchronize()
+    assert zo.zo_sync(ctx) == 0  # no bounded wait expired
     ref = _np_attention(f64(qkv), B, S, H, d)
     assert np.max(np.abs(f64(out) - ref)) <= 2e-2
 

@@ -62,6 +62,7 @@ def test_gqa_attention_matches_numpy(zo, ctx, B, S, H, Hk, e):
     out = torch.zeros((B * S, H * e), dtype=torch.bfloat16, device="cuda")
     zo.zo_attention_gqa(ctx, qkv, out, B, S, H, Hk, e)
     torch.cuda.synchronize()
+    assert zo.zo_sync(ctx) == 0  # no bounded wait expired
     assert np.max(np.abs(f64(out) - _np_gqa(f64(qkv), B, S, H, Hk, e))) <= 2e-2
     bad = next(k for k in range(2, H + 1) if H % k)  # H not a multiple of Hk: rejected
     with pytest.raises(zo.ZoError):

@@ -44,14 +44,13 @@ constexpr uint32_t kQBox = 128 * 128;  // bytes of one 128-row x 64-column bf16 
 // then O (hd columns).  Separate K and V rings in shared memory, so that a key tile is
 // released (and the next one loaded) as soon as its score MMA has completed.
 template <int HD> struct TcAttnCfg {
-  // head dim 128: key tiles of 64, two CTAs per SM (256 TMEM columns each); head dim 64: key
-  // tiles of 32, three CTAs per SM (128 TMEM columns: two 32-column score buffers and O), so
-  // that more query tiles are in flight where a tile's MMAs are short
-  static constexpr int kBN = HD == 128 ? 64 : 32;
+  // (Measured at head dim 64: key tiles of 32 with three CTAs per SM, or four, were slower
+  // than this: a tile's softmax then carries its fixed costs over half as many scores.)
+  static constexpr int kBN = 64;
   static constexpr int kKS = HD == 128 ? 2 : 4;  // K stages
   static constexpr int kVS = HD == 128 ? 2 : 4;  // V stages
-  static constexpr int kCtas = HD == 128 ? 2 : 3;
-  static constexpr int kTmemCols = HD == 128 ? 256 : 128;
+  static constexpr int kCtas = 2;
+  static constexpr int kTmemCols = 256;
   static constexpr uint32_t kKBox = kBN * 128;  // bytes of one kBN-row x 64-column bf16 box
 };
 
@@ -329,8 +328,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         }
       }
       // P_j overwrites the first kTBN / 2 columns of S_j (already read into registers)
-      if (kTBN == 64) tc::tmem_st32u(tS, pk);
-      else tc::tmem_st16u(tS, pk);
+      tc::tmem_st32u(tS, pk);
       l += lsum;
       tc::tc_fence_before();
       __syncwarp();
@@ -419,7 +417,7 @@ zo_status launch_attention_tc(zo_ctx *ctx, const uint16_t *qkv, uint16_t *out, i
   const cuuint64_t dims[2] = {(cuuint64_t)ld, (cuuint64_t)B * (cuuint64_t)S};
   const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
   const cuuint32_t boxq[2] = {64, (cuuint32_t)kTBM},
-                   boxkv[2] = {64, (cuuint32_t)(hd == 128 ? TcAttnCfg<128>::kBN : TcAttnCfg<64>::kBN)};
+                   boxkv[2] = {64, (cuuint32_t)TcAttnCfg<128>::kBN};  // the same for both head dims
   const cuuint32_t estr[2] = {1, 1};
   for (int m = 0; m < 2; ++m)
     if (fn(m ? &tmkv : &tmq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(qkv), dims,
