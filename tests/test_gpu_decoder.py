@@ -116,9 +116,11 @@ def test_attention_rescaling_matches_numpy(zo, ctx, B, S, H, d):
     assert np.max(np.abs(f64(out) - ref)) <= 2e-2
 
 
-def test_layernorm_matches_numpy(zo, ctx):
-    r = np.random.default_rng(0)
-    rows, d = 37, 7168
+# rows of whole and ragged last warps (8 columns per thread), up to the 8192-column limit
+@pytest.mark.parametrize("d", [7168, 8192, 2064, 2056, 768])
+def test_layernorm_matches_numpy(zo, ctx, d):
+    r = np.random.default_rng(d)
+    rows = 37
     x = torch.from_numpy((r.standard_normal((rows, d)) * 3 + 1).astype(np.float32)).cuda()
     g = bf16(1 + 0.1 * r.standard_normal(d))
     b = bf16(0.1 * r.standard_normal(d))
