@@ -63,8 +63,8 @@ UPDATE_INSTR = {"sources": ("zo_step.cu", "zo_internal.cuh"),
 #   launch averaged over the four projections of one layer (the step's other GEMM launches,
 #   the pruned last layer's few rows, move a negligible share of its bytes).
 GEMM_TRAFFIC = {"sources": ("zo_gemm.cu", "zo_tc.cuh"),
-                "sources_sha256": "4fc2cd08f0f9c3ca4065b276d10f195ccbeff43a4bc77a4045f05cefb8c18796",
-                "bytes": 13.86e9}
+                "sources_sha256": "b99c0b1fb5febbbb22e40ea6f99828b41d44285422fa60716c9395469a7edb85",
+                "bytes": 15.71e9}
 
 
 def sources_sha256(names):
@@ -1079,7 +1079,8 @@ def kernels_arm(args):
     """Each hot kernel of a decoder workload alone, at the workload's shapes and without the
     model's weights (for profiling and quick measurement): the four projection GEMMs and the
     causal attention of one micro-batch, the perturbation of one layer window, and the update
-    of a 2^30-element bf16 slice at the workload's n_pert.  L2 is flushed before every timed
+    of a 2^30-element bf16 slice at the workload's n_pert; for the OPT shapes also each
+    projection with the perturbation fused into its operand path against the window path.  L2 is flushed before every timed
     launch.  Prints one JSON line of per-kernel timings (not the benchmark's contract line)."""
     import torch
 
@@ -1170,6 +1171,27 @@ def kernels_arm(args):
         fl = 2.0 * Mm * N * K * (2 if epi == 3 else 1)
         out["gemm_" + key] = {"shape": [Mm, N, K], "us": us, "tflops": fl / us / 1e6,
                               "frac_bf16_burst": fl / us / 1e6 / peak_b, "sm_mhz": clocks[0]}
+    if not qwen:
+        # the perturbation fused into the GEMM's operand path (single-CTA form: every row tile
+        # regenerates the signs of the weight tiles it reads) against the window path (the
+        # layer's weights perturbed into a window once, then the GEMM on the window)
+        cw = zo.zo_create(Wt, seed=0, stream=stream.cuda_stream)
+        zo.zo_perturb(cw, +1, 1e-3, 3)
+        win = torch.empty(max(N * K for _, N, K, _ in shapes.values()), dtype=torch.bfloat16, device=dev)
+        fused = {}
+        for key, (Mm, N, K, epi) in shapes.items():
+            o = out_f if epi == 2 else out_b
+            us_f = timed(lambda: zo.zo_gemm_bf16_perturbed(cw, A, 0, bias, o, Mm, N, K, N, epi))
+            mhz_f = clocks[0]
+            us_w = timed(lambda: (zo.zo_perturb_range(cw, 0, N * K, win),
+                                  zo.zo_gemm_bf16(ctx, A, win, bias, o, Mm, N, K, N, epi)))
+            fused[key] = {"shape": [Mm, N, K], "fused_us": us_f, "window_then_gemm_us": us_w,
+                          "fused_over_window": us_f / us_w, "sm_mhz": [mhz_f, clocks[0]]}
+        zo.zo_restore(cw)
+        zo.zo_sync(cw)
+        cw.close()
+        del win
+        out["fused_perturbation"] = fused
     del A, Wt, out_b, out_f
     qkv = torch.randn(T * nq, dtype=torch.bfloat16, device=dev)
     att = torch.empty(T * na, dtype=torch.bfloat16, device=dev)

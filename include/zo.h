@@ -554,6 +554,23 @@ zo_status zo_model_step_host(zo_model *m, const int32_t *tokens_host, const int3
 zo_status zo_gemm_bf16(zo_ctx *ctx, const void *A, const void *B, const void *bias, void *out,
                        int32_t M, int32_t N, int32_t K, int32_t ldo, int32_t epilogue);
 
+/* zo_gemm_bf16 with B = the context's own bf16 parameters, read under its current
+ * perturbation with the perturbation fused into the GEMM's operand path ("Probe-Space
+ * Preconditioning for Fast and Stable Zero-Order Training", abstract: the probes are applied
+ * by fused unpack/apply kernels; here the apply runs inside the GEMM instead of into a
+ * window): B[n][k] = P at flat index w_offset + n K + k of the context, P = rd(theta + s eps
+ * z_i) as zo_perturb set it (theta itself when the context is clean), computed per weight
+ * tile in shared memory with no copy in HBM.  The product equals zo_gemm_bf16 on the
+ * zo_perturb_range window of the same weights, element for element, when both use the same
+ * single-CTA kernel form.  Every row tile of A regenerates the signs of the weight tiles it
+ * reads (M / 128 times per weight).  ctx must be bf16 with first_element % 16 == 0;
+ * w_offset % 16 == 0, K % 16 == 0, [w_offset, w_offset + N K) inside the context; epilogue
+ * ZO_EPI_BIAS_BF16, ZO_EPI_RELU_BF16 or ZO_EPI_RESID_F32 (else ZO_ERR_UNSUPPORTED); A, bias,
+ * out as zo_gemm_bf16.  Enqueued on ctx's stream; bounded waits as zo_gemm_bf16. */
+zo_status zo_gemm_bf16_perturbed(zo_ctx *ctx, const void *A, int64_t w_offset, const void *bias,
+                                 void *out, int32_t M, int32_t N, int32_t K, int32_t ldo,
+                                 int32_t epilogue);
+
 /* Test hook for the bounded waits of the tensor-core pipeline: runs zo_gemm_bf16 (no
  * bias, bf16 output) with the first stage's expected transaction count 16 bytes larger than
  * what its loads deliver, so that stage's barrier is never satisfied.  Every waiter gives

@@ -132,6 +132,78 @@ def test_layernorm_matches_numpy(zo, ctx, d):
     assert np.all(np.abs(f64(out) - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-3)
 
 
+# the perturbation fused into the GEMM's operand path: narrow (128-column) and wide
+# (256-column) tiles, ragged M and N, K off the 64-column stage grid, all three epilogues
+@pytest.mark.parametrize("M,N,K,epi", [(300, 320, 144, 0), (1024, 1536, 512, 1),
+                                       (4096, 1024, 272, 2), (4100, 2048, 2048, 0)])
+@pytest.mark.parametrize("sign", [+1, -1])
+def test_fused_perturbation_gemm_equals_the_window_product(zo, M, N, K, epi, sign):
+    """zo_gemm_bf16_perturbed (signs regenerated per weight tile in shared memory) against the
+    same single-CTA kernel run clean on the zo_perturb_range window: bit for bit; the window
+    itself against the oracle's perturbation, bit for bit."""
+    r = np.random.default_rng(M + N + K + epi)
+    w_off, eps, probe, seed, step = 48, 1e-3, 13, 21, 5
+    total = w_off + N * K + 40
+    theta = bf16(r.standard_normal(total) * 0.02)
+    A = bf16(r.standard_normal((M, K)))
+    bias = bf16(r.standard_normal(N) * 0.1)
+    if epi == 2:
+        h0 = torch.from_numpy(r.standard_normal((M, N)).astype(np.float32)).cuda()
+        out1, out2 = h0.clone(), h0.clone()
+    else:
+        out1 = torch.zeros((M, N), dtype=torch.bfloat16, device="cuda")
+        out2 = torch.zeros_like(out1)
+    c = zo.zo_create(theta, seed=seed)
+    zo.zo_set_step(c, step)
+    zo.zo_perturb(c, sign, eps, probe)
+    zo.zo_gemm_bf16_perturbed(c, A, w_off, bias, out1, M, N, K, N, epi)
+    win = torch.empty(N * K, dtype=torch.bfloat16, device="cuda")
+    zo.zo_perturb_range(c, w_off, N * K, win)
+    zo.zo_restore(c)
+    cw = zo.zo_create(win, seed=seed)  # clean: the same kernel form on the window
+    zo.zo_gemm_bf16_perturbed(cw, A, 0, bias, out2, M, N, K, N, epi)
+    torch.cuda.synchronize()
+    assert zo.zo_sync(c) == 0 and zo.zo_sync(cw) == 0
+    bits = theta.view(torch.int16).cpu().numpy().view(np.uint16)
+    ref_win = core.perturb(bits, seed, step, probe, sign, float(np.float32(eps)))[w_off:w_off + N * K]
+    assert np.array_equal(win.view(torch.int16).cpu().numpy().view(np.uint16), ref_win)
+    if epi == 2:
+        assert torch.equal(out1, out2)
+    else:
+        assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    # and the product itself, against fp64 on the window
+    ref = f64(A) @ f64(win.reshape(N, K)).T + f64(bias)
+    if epi == 2:
+        scale = np.abs(f64(A)) @ np.abs(f64(win.reshape(N, K))).T + np.abs(f64(bias))
+        got = out1.cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(got - (h0.cpu().numpy() + ref)) <= 1e-5 * (scale + 1) + 1e-6)
+    else:
+        if epi == 1:
+            ref = np.maximum(ref, 0.0)
+        rms = np.sqrt(np.mean(ref ** 2)) + 1e-30  # one bf16 rounding of the output
+        assert np.all(np.abs(f64(out1) - ref) <= 2.0 ** -8 * (np.abs(ref) + rms))
+    cw.close()
+    c.close()
+
+
+def test_fused_perturbation_gemm_rejects_bad_arguments(zo):
+    theta = torch.zeros(4096, dtype=torch.bfloat16, device="cuda")
+    A = torch.zeros((64, 32), dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros((64, 64), dtype=torch.bfloat16, device="cuda")
+    c = zo.zo_create(theta, seed=1)
+    for w_off, N, K, epi in [(8, 64, 32, 0),      # offset not 16-element aligned
+                             (0, 64, 24, 0),      # K % 16 != 0
+                             (2048, 64, 64, 0),   # past the end of the context
+                             (0, 32, 32, 3)]:     # SwiGLU
+        with pytest.raises(zo.ZoError):
+            zo.zo_gemm_bf16_perturbed(c, A, w_off, None, out, 64, N, K, 64, epi)
+    c.close()
+    f = zo.zo_create(torch.zeros(4096, dtype=torch.float32, device="cuda"), seed=1)
+    with pytest.raises(zo.ZoError):  # fp32 context
+        zo.zo_gemm_bf16_perturbed(f, A, 0, None, out, 64, 64, 32, 64, 0)
+    f.close()
+
+
 TINY = [
     dict(n_layers=2, d_model=128, n_heads=2, d_ffn=512, vocab=1000, max_pos=128, class_ids=(3, 7)),
     dict(n_layers=2, d_model=256, n_heads=2, d_ffn=320, vocab=777, max_pos=160, class_ids=(0, 776)),

@@ -66,6 +66,7 @@ _SIGS = {
     "zo_model_hidden": [_vp, _vp, _i32, _i32, _i32, _vp],
     "zo_model_step": [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _f32, _f32, _f32, _int, _vp],
     "zo_gemm_bf16": [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32],
+    "zo_gemm_bf16_perturbed": [_vp, _vp, _i64, _vp, _vp, _i32, _i32, _i32, _i32, _i32],
     "zo_attention": [_vp, _vp, _vp, _i32, _i32, _i32, _i32],
     "zo_attention_gqa": [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32],
     "zo_model_set_pruning": [_vp, _int],
@@ -432,6 +433,13 @@ def zo_model_step_host(model, tokens_host, labels_host, batch, seq, n_micro, n_p
 def zo_gemm_bf16(ctx, A, B, bias, out, M, N, K, ldo, epilogue):
     return ctx.check(_L.zo_gemm_bf16(ctx.handle, _ptr(A), _ptr(B), _ptr(bias), _ptr(out), M, N,
                                      K, ldo, epilogue))
+
+
+def zo_gemm_bf16_perturbed(ctx, A, w_offset, bias, out, M, N, K, ldo, epilogue):
+    """The GEMM with B = ctx's parameters [w_offset, w_offset + N K) under ctx's current
+    perturbation, fused into the operand path (zo.h)."""
+    return ctx.check(_L.zo_gemm_bf16_perturbed(ctx.handle, _ptr(A), w_offset, _ptr(bias), _ptr(out),
+                                               M, N, K, ldo, epilogue))
 
 
 def zo_attention(ctx, qkv, out, batch, seq, n_heads, d_model):

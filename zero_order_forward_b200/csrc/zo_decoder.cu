@@ -34,6 +34,8 @@ namespace zo {
 
 zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bias, void *out,
                       int M, int N, int K, int ldo, int epi, uint32_t extra_tx = 0);
+zo_status launch_gemm_perturbed(zo_ctx *ctx, const void *A, int64_t w_off, const void *bias,
+                                void *out, int M, int N, int K, int ldo, int epi);
 zo_status launch_attention(zo_ctx *ctx, const uint16_t *qkv, uint16_t *out, int B, int S, int H,
                            int d);
 zo_status launch_attention_gqa(zo_ctx *ctx, const uint16_t *qkv, uint16_t *out, int B, int S,
@@ -712,6 +714,15 @@ zo_status zo_gemm_bf16(zo_ctx *ctx, const void *A, const void *B, const void *bi
   ctx->err.clear();
   if (!A || !B || !out) return fail(ctx, ZO_ERR_INVALID, "null gemm operand");
   return launch_gemm(ctx, A, B, bias, out, M, N, K, ldo, epilogue);
+}
+
+zo_status zo_gemm_bf16_perturbed(zo_ctx *ctx, const void *A, int64_t w_offset, const void *bias,
+                                 void *out, int32_t M, int32_t N, int32_t K, int32_t ldo,
+                                 int32_t epilogue) {
+  if (!ctx) return ZO_ERR_INVALID;
+  ctx->err.clear();
+  if (!A || !out) return fail(ctx, ZO_ERR_INVALID, "null gemm operand");
+  return launch_gemm_perturbed(ctx, A, w_offset, bias, out, M, N, K, ldo, epilogue);
 }
 
 zo_status zo_debug_gemm_timeout(zo_ctx *ctx, const void *A, const void *B, void *out, int32_t M,

@@ -45,6 +45,7 @@ struct GemmArgs {
   int ldo;
   uint32_t *err;         // device error word (ZO_FLAG_TIMEOUT raised on a bounded-wait expiry)
   uint32_t extra_tx;     // 0; a test hook sets it so that the first stage never completes
+  int64_t w_off;         // fused perturbation: flat index of B's element (0, 0) in the context
 };
 
 __device__ __forceinline__ void load_bias32(const uint16_t *bias, int col0, int N, float b[32]) {
@@ -98,6 +99,8 @@ __device__ __forceinline__ void stage_row(uint8_t *stage, int r, const float v[3
 
 constexpr int kEpiWarps = 8;                      // two warps per TMEM lane quadrant
 constexpr int kGemmThreads = 32 * (2 + kEpiWarps);  // producer, MMA, epilogue
+constexpr int kXWarps = 4;                          // fused perturbation: transform warps
+constexpr int kGemmThreadsX = kGemmThreads + 32 * kXWarps;
 constexpr uint32_t kStageTile = 32 * 128;           // one 32 x 32 fp32 (or bf16) output tile
 
 template <int BN, int STAGES>
@@ -108,6 +111,8 @@ struct GemmSmem {
   static constexpr uint32_t kOutOffset = STAGES * kStageBytes;         // 1024-aligned
   static constexpr uint32_t kBarOffset = kOutOffset + kEpiWarps * kStageTile;
   static constexpr uint32_t kBytes = kBarOffset + 256 + 1024;  // + barriers + alignment slack
+  // full, empty, ready [STAGES]; acc_full, acc_empty [2]; mma_done; TMEM address; abort flag
+  static_assert((3 * STAGES + 5) * 8 + 8 <= 256, "barrier area");
 };
 
 struct TileCoord {
@@ -134,14 +139,51 @@ int group_rows_for(int K, int rows_per_tile) {
   return (int)(g < 1 ? 1 : g > 16 ? 16 : g);
 }
 
+// Eight bf16 weights of one 16-byte chunk perturbed as the window kernel does it: element t
+// takes sign bit t of `bits` (1: z = -1), P = rd_bf16(theta + (s eps) z) with the sign xor-ed
+// into s eps (db: the bits of s eps).
+__device__ __forceinline__ uint4 perturb8_bf16(uint4 v, uint32_t bits, uint32_t db) {
+  uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const float lo = __fadd_rn(__uint_as_float(w[t] << 16),
+                               __uint_as_float(db ^ ((bits << (31 - 2 * t)) & 0x80000000u)));
+    const float hi = __fadd_rn(__uint_as_float(w[t] & 0xFFFF0000u),
+                               __uint_as_float(db ^ ((bits << (30 - 2 * t)) & 0x80000000u)));
+    w[t] = pack_bf16x2(lo, hi);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// All lanes of the warp wait for `parity` on `bar` (lane 0 decides, bounded; then every lane
+// observes the completed phase).  False on every lane on expiry or abort.
+__device__ __forceinline__ bool gemm_warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+  const int lane = threadIdx.x & 31;
+  int ok = 1;
+  if (lane == 0) ok = (!*abort_flag && tc::mbar_wait(bar, parity)) ? 1 : 0;
+  ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+  if (ok && lane != 0) ok = tc::mbar_wait(bar, parity) ? 1 : 0;
+  return __all_sync(0xFFFFFFFFu, ok) != 0;
+}
+
 // Persistent: one CTA per SM walks tiles t = blockIdx.x, blockIdx.x + gridDim.x, ...
 // The shared-memory ring runs across tile boundaries, and the accumulator is
 // double-buffered in TMEM (2 x BN columns) so the epilogue of tile i overlaps the
 // main loop of tile i+1.
-template <int BN, int STAGES, int EPI>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+//
+// PERT (the perturbation fused into the operand path): B is a bf16 weight matrix inside the
+// context's parameters (row n, column k at flat index args.w_off + n K + k), and the MMA
+// multiplies by its perturbed copy P = rd(theta + s eps z_i) under `pk` without a window in
+// HBM.  Four more warps wait for each stage, regenerate the probe's signs for its B tile
+// (one Philox block per 16-column group of a row) and perturb the tile in shared memory in
+// place (the 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r & 7)), then
+// release the stage to the MMA through ready[s].  Every row tile re-does this for the weight
+// tiles it reads.
+template <int BN, int STAGES, int EPI, bool PERT>
+__global__ void __launch_bounds__(PERT ? kGemmThreadsX : kGemmThreads, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const __grid_constant__ CUtensorMap tmC, GemmArgs args) {
+                 const __grid_constant__ CUtensorMap tmC, GemmArgs args, ProbeKey pk,
+                 const __grid_constant__ RoundKeys rk) {
   using S = GemmSmem<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -154,10 +196,12 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   uint64_t *acc_full = empty + STAGES;   // [2] MMA -> epilogue
   uint64_t *acc_empty = acc_full + 2;    // [2] epilogue -> MMA
   uint64_t *mma_done = acc_empty + 2;    // all MMAs of this CTA retired
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(mma_done + 1);
+  uint64_t *ready = mma_done + 1;        // [STAGES] PERT: B tile of the stage perturbed
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(ready + STAGES);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
   constexpr bool kSwiGLU = EPI == ZO_EPI_SWIGLU_BF16;
+  static_assert(!(PERT && kSwiGLU), "the fused perturbation takes one weight matrix");
   constexpr int OUT_BN = kSwiGLU ? BN / 2 : BN;  // output columns per tile
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int num_m = (args.M + kBM - 1) / kBM, num_n = (args.N + OUT_BN - 1) / OUT_BN;
@@ -174,6 +218,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       tc::mbar_init(&acc_empty[b], kEpiWarps);  // one arrival per epilogue warp
     }
     tc::mbar_init(mma_done, 1);
+    if (PERT)
+      for (int s = 0; s < STAGES; ++s) tc::mbar_init(&ready[s], kXWarps);
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -224,7 +270,9 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const uint32_t d = tmem + (uint32_t)(b * BN);
       for (int kb = 0; kb < nk; ++kb) {
         const uint32_t s = consumed % STAGES, ph = (consumed / STAGES) & 1u;
-        if (*abort_flag || !tc::mbar_wait(&full[s], ph)) {
+        // PERT: the stage is complete once its B tile has been perturbed (which follows the
+        // transform warps' wait on full[s])
+        if (*abort_flag || !tc::mbar_wait(PERT ? &ready[s] : &full[s], ph)) {
           atomicOr(args.err, ZO_FLAG_TIMEOUT);
           *abort_flag = 1;
           break;
@@ -243,6 +291,50 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       tc::mma_commit(&acc_full[b]);
     }
     tc::mma_commit(mma_done);  // arrives once every MMA issued above has retired
+  } else if (PERT && warp >= 2 + kEpiWarps) {
+    // transform warps: thread xt perturbs rows xt, xt + 128, ... of each stage's B tile
+    const int xt = threadIdx.x - 32 * (2 + kEpiWarps);
+    const uint32_t step = pk.sign ? *pk.step : 0u;
+    const uint32_t db = __float_as_uint(pk.sign > 0 ? pk.eps : -pk.eps);
+    uint32_t consumed = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+      const TileCoord tc0 = tile_coord(t, num_m, num_n, OUT_BN, args.group_m);
+      for (int kb = 0; kb < nk; ++kb) {
+        const uint32_t s = consumed % STAGES, ph = (consumed / STAGES) & 1u;
+        if (!gemm_warp_wait(&full[s], ph, abort_flag)) {
+          if (lane == 0) atomicOr(args.err, ZO_FLAG_TIMEOUT);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        if (pk.sign) {
+          uint8_t *st = sB + s * S::kBBytes;
+#pragma unroll 1
+          for (int r = xt; r < BN; r += 32 * kXWarps) {
+            const int n = tc0.n0 + r;
+            if (n >= args.N) break;  // rows past N stay as loaded (zero)
+            const int64_t e0 = args.w_off + (int64_t)n * args.K + (int64_t)kb * kBK;
+#pragma unroll
+            for (int q = 0; q < kBK / 16; ++q) {
+              if (kb * kBK + 16 * q >= args.K) break;  // K % 16 == 0: a group is whole or absent
+              const uint32_t bits =
+                  probe_group_bits(pk.g_off + (uint64_t)((e0 + 16 * q) >> 4), pk.probe, step, rk);
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int c = 2 * q + h;  // 16-byte chunk of the 128-byte row
+                uint4 *p = reinterpret_cast<uint4 *>(st + r * 128 + ((c ^ (r & 7)) << 4));
+                *p = perturb8_bf16(*p, bits >> (8 * h), db);
+              }
+            }
+          }
+          tc::fence_proxy_async_smem();  // these writes precede the tensor core's reads
+        }
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&ready[s]);
+        ++consumed;
+      }
+    }
   } else if (warp >= 2) {
     const int q = warp & 3;                    // TMEM lanes 32q..32q+31 (this warp's rows)
     const int half = (warp - 2) / 4;           // which half of the output columns
@@ -589,11 +681,12 @@ bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int 
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, int EPI>
+template <int BN, int STAGES, int EPI, bool PERT = false>
 cudaError_t launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tcm,
-                       const GemmArgs &g, cudaStream_t st) {
+                       const GemmArgs &g, cudaStream_t st, const ProbeKey &pk = ProbeKey{},
+                       const RoundKeys &rk = RoundKeys{}) {
   using S = GemmSmem<BN, STAGES>;
-  auto kern = gemm_bf16_kernel<BN, STAGES, EPI>;
+  auto kern = gemm_bf16_kernel<BN, STAGES, EPI, PERT>;
   {
     const cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kern), (int)S::kBytes);
     if (e != cudaSuccess) return e;
@@ -601,7 +694,8 @@ cudaError_t launch_one(const CUtensorMap &ta, const CUtensorMap &tb, const CUten
   constexpr int OUT_BN = EPI == ZO_EPI_SWIGLU_BF16 ? BN / 2 : BN;
   const int num_m = (g.M + kBM - 1) / kBM, num_n = (g.N + OUT_BN - 1) / OUT_BN;
   const int tiles = num_m * num_n;
-  kern<<<tiles < kSmCount ? tiles : kSmCount, kGemmThreads, S::kBytes, st>>>(ta, tb, tcm, g);
+  kern<<<tiles < kSmCount ? tiles : kSmCount, PERT ? kGemmThreadsX : kGemmThreads, S::kBytes, st>>>(
+      ta, tb, tcm, g, pk, rk);
   return cudaGetLastError();
 }
 
@@ -684,6 +778,47 @@ zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bia
   if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "gemm launch: %s", cudaGetErrorString(e));
   ctx->launches += 1;
   ktime_end(ctx, slot, ZO_KT_GEMM, 2.0 * M * (double)NB * K);  // NB accumulator columns
+  return ZO_OK;
+}
+
+// The GEMM with B = the context's bf16 parameters [w_off, w_off + N K) read under the
+// context's current perturbation (fused into the operand path, single-CTA form).
+zo_status launch_gemm_perturbed(zo_ctx *ctx, const void *A, int64_t w_off, const void *bias,
+                                void *out, int M, int N, int K, int ldo, int epi) {
+  if (ctx->dtype != ZO_BF16) return fail(ctx, ZO_ERR_INVALID, "perturbed gemm: needs a bf16 context");
+  if (M < 1 || N < 1 || K < 16 || (K % 16) != 0 || (ldo % 8) != 0 || ldo < N)
+    return fail(ctx, ZO_ERR_INVALID, "perturbed gemm: need M,N >= 1, K %% 16 == 0, ldo %% 8 == 0, ldo >= N");
+  if (w_off < 0 || w_off % 16 != 0 || ctx->first_element % 16 != 0 || w_off + (int64_t)N * K > ctx->M)
+    return fail(ctx, ZO_ERR_INVALID, "perturbed gemm: weights must lie in the context, 16-element aligned");
+  if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(out) |
+       reinterpret_cast<uintptr_t>(bias)) & 15u)
+    return fail(ctx, ZO_ERR_INVALID, "perturbed gemm: operands must be 16-byte aligned");
+  if (epi != ZO_EPI_BIAS_BF16 && epi != ZO_EPI_RELU_BF16 && epi != ZO_EPI_RESID_F32)
+    return fail(ctx, ZO_ERR_UNSUPPORTED, "perturbed gemm: bias, ReLU or residual epilogue only");
+  const uint16_t *B = static_cast<const uint16_t *>(ctx->params) + w_off;
+  const bool wide = N > 128 && ((int64_t)((M + 127) / 128) * ((N + 255) / 256) >= kSmCount);
+  CUtensorMap ta, tb, tcm;
+  if (!make_map(&ta, A, M, K, kBM) || !make_map(&tb, B, N, K, wide ? 256 : 128) ||
+      !make_out_map(&tcm, out, M, N, ldo, epi == ZO_EPI_RESID_F32))
+    return fail(ctx, ZO_ERR_CUDA, "perturbed gemm: cuTensorMapEncodeTiled failed");
+  GemmArgs g{M, N, K, group_rows_for(K, kBM), static_cast<const uint16_t *>(bias), out, ldo,
+             &ctx->dstate->flags, 0u, w_off};
+  const ProbeKey pk = probe_key(ctx);
+  const RoundKeys rk = round_keys(pk.k0, pk.k1);
+  const int slot = ktime_begin(ctx);
+  cudaError_t e;
+  if (wide) {
+    if (epi == ZO_EPI_BIAS_BF16) e = launch_one<256, 4, ZO_EPI_BIAS_BF16, true>(ta, tb, tcm, g, ctx->stream, pk, rk);
+    else if (epi == ZO_EPI_RELU_BF16) e = launch_one<256, 4, ZO_EPI_RELU_BF16, true>(ta, tb, tcm, g, ctx->stream, pk, rk);
+    else e = launch_one<256, 4, ZO_EPI_RESID_F32, true>(ta, tb, tcm, g, ctx->stream, pk, rk);
+  } else {
+    if (epi == ZO_EPI_BIAS_BF16) e = launch_one<128, 6, ZO_EPI_BIAS_BF16, true>(ta, tb, tcm, g, ctx->stream, pk, rk);
+    else if (epi == ZO_EPI_RELU_BF16) e = launch_one<128, 6, ZO_EPI_RELU_BF16, true>(ta, tb, tcm, g, ctx->stream, pk, rk);
+    else e = launch_one<128, 6, ZO_EPI_RESID_F32, true>(ta, tb, tcm, g, ctx->stream, pk, rk);
+  }
+  if (e != cudaSuccess) return fail(ctx, ZO_ERR_CUDA, "perturbed gemm launch: %s", cudaGetErrorString(e));
+  ctx->launches += 1;
+  ktime_end(ctx, slot, ZO_KT_GEMM, 2.0 * M * (double)N * K);
   return ZO_OK;
 }
 
