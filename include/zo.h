@@ -72,7 +72,7 @@ typedef enum {
   ZO_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
   ZO_ERR_OOM = 4,         /* device allocation failed */
   ZO_ERR_NONFINITE = 5,   /* a loss was NaN/Inf: the step was skipped (theta unchanged) */
-  ZO_ERR_UNSUPPORTED = 6, /* valid request this build does not support */
+  ZO_ERR_UNSUPPORTED = 6, /* valid request this library does not support */
   ZO_ERR_TIMEOUT = 7      /* a kernel gave up a bounded wait (see ZO_FLAG_TIMEOUT) */
 } zo_status;
 
