@@ -47,7 +47,7 @@
  *     (e.g. torch CUDA tensors); "host" pointers are ordinary host memory.
  *   - Calls enqueue work on the context's stream and return without synchronising,
  *     unless documented otherwise.  The step counter lives in device memory, so a
- *     sequence of calls can be captured into a CUDA graph and replayed.
+ *     whole step is enqueued without a host synchronisation.
  *   - Every call returns a zo_status; on failure zo_last_error(ctx) describes it.
  *     No call throws, aborts or prints.  A context is not thread-safe.
  */
@@ -286,8 +286,7 @@ zo_status zo_mlp_loss(zo_ctx *ctx, const float *X, const int32_t *labels, int ba
 /* zo_mlp_loss without a context and without any device allocation.  The pages have no
  * counterpart: this entry point exists for callers that must not call cudaMalloc, e.g.
  * code running inside a host framework that owns every device allocation through its own
- * pool, or code that enqueues work while a stream is being captured, where a new
- * allocation would break the capture or its memory budget.  Such callers pass inputs and
+ * pool and memory budget.  Such callers pass inputs and
  * outputs only; the reduction scratch is a static device array of libzo.so, which every GPU
  * that loads the library holds (about 32 KB) until the process exits.
  *   P          device, M = n_hidden*n_in + n_hidden + n_out*n_hidden + n_out floats,
@@ -296,8 +295,8 @@ zo_status zo_mlp_loss(zo_ctx *ctx, const float *X, const int32_t *labels, int ba
  *   X, labels, batch, n_in, n_hidden, n_out, scale, loss_out, accumulate: as zo_mlp_loss.
  *   stream     cudaStream_t to enqueue on (NULL = legacy default stream).
  * The first call on a device looks up the scratch array's device address (once per
- * device and CUDA context, with that device current); make that first call before any stream
- * capture.  The address is kept for the life of the process: after cudaDeviceReset of a
+ * device and CUDA context, with that device current).  The address is kept for the life of
+ * the process: after cudaDeviceReset of a
  * device, whose context may come back with the same handle, the kept address is stale, so a
  * process that resets a device must not call this entry point on it again.
  * Every call clears the scratch's counter before its kernel.  All calls in the process

@@ -1,8 +1,8 @@
 """The allocation-free MLP loss (zo_mlp_loss_noalloc) against the context-based one.
 
 zo_mlp_loss_noalloc serves callers that must not call cudaMalloc (a host framework that
-owns every device allocation, or work enqueued during a stream capture): it takes inputs
-and outputs only and keeps its reduction scratch in the library's static device memory.
+owns every device allocation): it takes inputs and outputs only and keeps its reduction
+scratch in the library's static device memory.
 This file is collected last so that a run stopping at the first failure has already run
 every other test; it also passes when run alone in a fresh process.
 """
