@@ -139,7 +139,8 @@ zo_status zo_set_step(zo_ctx *ctx, uint32_t step);
 /* Element offset for a context that holds a slice of a larger parameter vector: params[j]
  * is element first_element + j of that vector (first_element >= 0, a multiple of 16, so
  * that slices keep whole 16-element sign groups).  Every sign the context generates
- * (zo_perturb, zo_perturb_range, zo_pack_probe, the quadratic losses, zo_update, zo_step) is
+ * (zo_perturb, zo_perturb_range, zo_gemm_bf16_perturbed, zo_pack_probe, the quadratic
+ * losses, zo_update, zo_step) is
  * then the sign of the global element index, so contexts with the same seed and step on
  * disjoint slices perturb and update exactly as one context on the whole vector would,
  * element by element; a separable loss (the diagonal quadratic) is the sum of the slices'

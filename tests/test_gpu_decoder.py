@@ -134,10 +134,12 @@ def test_layernorm_matches_numpy(zo, ctx, d):
 
 # the perturbation fused into the GEMM's operand path: narrow (128-column) and wide
 # (256-column) tiles, ragged M and N, K off the 64-column stage grid, all three epilogues
-@pytest.mark.parametrize("M,N,K,epi", [(300, 320, 144, 0), (1024, 1536, 512, 1),
-                                       (4096, 1024, 272, 2), (4100, 2048, 2048, 0)])
+@pytest.mark.parametrize("M,N,K,epi,j0", [(300, 320, 144, 0, 0), (1024, 1536, 512, 1, 0),
+                                          (4096, 1024, 272, 2, 0), (4100, 2048, 2048, 0, 0),
+                                          # a context over a slice: signs of global indices
+                                          (512, 384, 320, 1, (1 << 20) + 48)])
 @pytest.mark.parametrize("sign", [+1, -1])
-def test_fused_perturbation_gemm_equals_the_window_product(zo, M, N, K, epi, sign):
+def test_fused_perturbation_gemm_equals_the_window_product(zo, M, N, K, epi, j0, sign):
     """zo_gemm_bf16_perturbed (signs regenerated per weight tile in shared memory) against the
     same single-CTA kernel run clean on the zo_perturb_range window: bit for bit; the window
     itself against the oracle's perturbation, bit for bit."""
@@ -154,6 +156,8 @@ def test_fused_perturbation_gemm_equals_the_window_product(zo, M, N, K, epi, sig
         out1 = torch.zeros((M, N), dtype=torch.bfloat16, device="cuda")
         out2 = torch.zeros_like(out1)
     c = zo.zo_create(theta, seed=seed)
+    if j0:
+        zo.zo_set_element_offset(c, j0)
     zo.zo_set_step(c, step)
     zo.zo_perturb(c, sign, eps, probe)
     zo.zo_gemm_bf16_perturbed(c, A, w_off, bias, out1, M, N, K, N, epi)
@@ -165,7 +169,7 @@ def test_fused_perturbation_gemm_equals_the_window_product(zo, M, N, K, epi, sig
     torch.cuda.synchronize()
     assert zo.zo_sync(c) == 0 and zo.zo_sync(cw) == 0
     bits = theta.view(torch.int16).cpu().numpy().view(np.uint16)
-    ref_win = core.perturb(bits, seed, step, probe, sign, float(np.float32(eps)))[w_off:w_off + N * K]
+    ref_win = core.perturb(bits, seed, step, probe, sign, float(np.float32(eps)), j0)[w_off:w_off + N * K]
     assert np.array_equal(win.view(torch.int16).cpu().numpy().view(np.uint16), ref_win)
     if epi == 2:
         assert torch.equal(out1, out2)
