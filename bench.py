@@ -61,10 +61,12 @@ UPDATE_INSTR = {"sources": ("zo_step.cu", "zo_internal.cuh"),
                              "16": 207.25e6, "32": 323.66e6, "64": 551.14e6, "160": 1238.20e6}}}
 #   gemm_pair_kernel at the OPT-30B layer shapes (T = 16384): DRAM bytes (read + write) per
 #   launch averaged over the four projections of one layer (the step's other GEMM launches,
-#   the pruned last layer's few rows, move a negligible share of its bytes).
+#   the pruned last layer's few rows, move a negligible share of its bytes).  Captured with
+#   contiguous A operands; inside the step the FC2 GEMM reads its A (the FFN intermediate)
+#   with a padded row stride, which measured about 8 GB less per FC2 launch at this shape.
 GEMM_TRAFFIC = {"sources": ("zo_gemm.cu", "zo_tc.cuh"),
-                "sources_sha256": "b99c0b1fb5febbbb22e40ea6f99828b41d44285422fa60716c9395469a7edb85",
-                "bytes": 15.71e9}
+                "sources_sha256": "39166dc3dd0be582ecf2af1142e38a68cc4c27363793ed105cafc578f837207f",
+                "bytes": 11.69e9}
 
 
 def sources_sha256(names):

@@ -33,7 +33,8 @@
 namespace zo {
 
 zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bias, void *out,
-                      int M, int N, int K, int ldo, int epi, uint32_t extra_tx = 0);
+                      int M, int N, int K, int ldo, int epi, uint32_t extra_tx = 0,
+                      int64_t lda = 0);
 zo_status launch_gemm_perturbed(zo_ctx *ctx, const void *A, int64_t w_off, const void *bias,
                                 void *out, int M, int N, int K, int ldo, int epi);
 zo_status launch_attention(zo_ctx *ctx, const uint16_t *qkv, uint16_t *out, int B, int S, int H,
@@ -329,6 +330,7 @@ struct zo_model {
   uint16_t *window = nullptr;
   float *h = nullptr;
   uint16_t *xn = nullptr, *qkv = nullptr, *attn = nullptr, *mid = nullptr;
+  int64_t ld_mid = 0;       // row stride of mid: d_ffn + 64 (see launch_gemm's lda)
   float2 *rope = nullptr;   // Qwen3: (cos, sin) of position s and pair i at [s][e/2]
   bool qwen = false;
   // pruned last layer of the loss forward: the last position of each sequence only
@@ -371,9 +373,10 @@ zo_status run_qwen_layer(zo_model *m, const uint16_t *lp, int B, int S) {
   if ((st = launch_gemm(ctx, m->attn, lp + L.wo, nullptr, m->h, T, d, na, d,
                         ZO_EPI_RESID_F32)) != ZO_OK) return st;
   if ((st = launch_rmsnorm(ctx, m->h, lp + L.post_norm, m->xn, T, d, eps)) != ZO_OK) return st;
-  if ((st = launch_gemm(ctx, m->xn, lp + L.wgu, nullptr, m->mid, T, f, d, f,
+  if ((st = launch_gemm(ctx, m->xn, lp + L.wgu, nullptr, m->mid, T, f, d, (int)m->ld_mid,
                         ZO_EPI_SWIGLU_BF16)) != ZO_OK) return st;
-  return launch_gemm(ctx, m->mid, lp + L.wd, nullptr, m->h, T, d, f, d, ZO_EPI_RESID_F32);
+  return launch_gemm(ctx, m->mid, lp + L.wd, nullptr, m->h, T, d, f, d, ZO_EPI_RESID_F32, 0,
+                     m->ld_mid);
 }
 
 zo_status gather_last(zo_model *m, const void *src, void *dst, int64_t row_bytes, int B, int S) {
@@ -475,10 +478,10 @@ zo_status run_layers(zo_model *m, const int32_t *tokens, int B, int S, int n_run
                           ZO_EPI_RESID_F32)) != ZO_OK) return st;
     layernorm_kernel<<<T, ln_threads(d), 0, ctx->stream>>>(m->h, lp + L.ln2g, lp + L.ln2b, m->xn, d);
     if ((st = check_launch(ctx, "layernorm_kernel")) != ZO_OK) return st;
-    if ((st = launch_gemm(ctx, m->xn, lp + L.w1, lp + L.b1, m->mid, T, f, d, f,
+    if ((st = launch_gemm(ctx, m->xn, lp + L.w1, lp + L.b1, m->mid, T, f, d, (int)m->ld_mid,
                           ZO_EPI_RELU_BF16)) != ZO_OK) return st;
     if ((st = launch_gemm(ctx, m->mid, lp + L.w2, lp + L.b2, m->h, T, d, f, d,
-                          ZO_EPI_RESID_F32)) != ZO_OK) return st;
+                          ZO_EPI_RESID_F32, 0, m->ld_mid)) != ZO_OK) return st;
   }
   return ZO_OK;
 }
@@ -527,7 +530,8 @@ zo_status zo_model_create(zo_model **out, zo_ctx *ctx, const zo_model_cfg *cfg, 
   if (e == cudaSuccess) e = cudaMalloc(&m->xn, (size_t)T * d * 2);
   if (e == cudaSuccess) e = cudaMalloc(&m->qkv, (size_t)T * L.qkv_cols * 2);
   if (e == cudaSuccess) e = cudaMalloc(&m->attn, (size_t)T * L.attn_cols * 2);
-  if (e == cudaSuccess) e = cudaMalloc(&m->mid, (size_t)T * f * 2);  // FC1 / SwiGLU output
+  m->ld_mid = f + 64;  // FC1 / SwiGLU output rows, padded (the FC2 / down GEMM's A)
+  if (e == cudaSuccess) e = cudaMalloc(&m->mid, (size_t)T * m->ld_mid * 2);
   m->prune_rows = (int)(max_tokens < 512 ? max_tokens : 512);
   const int64_t R = m->prune_rows;
   if (e == cudaSuccess) e = cudaMalloc(&m->hl, (size_t)R * d * 4);

@@ -668,11 +668,12 @@ bool make_out_map(CUtensorMap *m, void *base, int64_t rows, int64_t cols, int64_
 
 // 2-D bf16 tensor [rows][cols] (row-major, cols contiguous), box = box_rows x 64 columns,
 // 128-byte swizzle, zero fill outside the tensor.
-bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int box_rows) {
+bool make_map(CUtensorMap *m, const void *base, int64_t rows, int64_t cols, int box_rows,
+              int64_t ld = 0) {  // ld: elements between row starts (0: cols)
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint64_t strides[1] = {(cuuint64_t)(ld ? ld : cols) * 2};
   const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
@@ -718,10 +719,10 @@ cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUte
 }  // namespace
 
 zo_status launch_gemm_pair(zo_ctx *ctx, const void *A, const void *B, const void *bias, void *out,
-                           int M, int N, int K, int ldo, int epi) {
+                           int M, int N, int K, int ldo, int epi, int64_t lda) {
   const int NB = epi == ZO_EPI_SWIGLU_BF16 ? 2 * N : N;
   CUtensorMap ta, tb, tcm;
-  if (!make_map(&ta, A, M, K, kBM) || !make_map(&tb, B, NB, K, kPairBN / 2) ||
+  if (!make_map(&ta, A, M, K, kBM, lda) || !make_map(&tb, B, NB, K, kPairBN / 2) ||
       !make_out_map(&tcm, out, M, N, ldo, epi == ZO_EPI_RESID_F32))
     return fail(ctx, ZO_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
   GemmArgs g{M, N, K, group_rows_for(K, 2 * kBM), static_cast<const uint16_t *>(bias), out, ldo,
@@ -738,10 +739,16 @@ zo_status launch_gemm_pair(zo_ctx *ctx, const void *A, const void *B, const void
   return ZO_OK;
 }
 
+// lda: elements between the starts of A's rows (0: K; a multiple of 8, at least K).  A padded
+// row stride keeps the 128-byte pieces of A that a stage reads from colliding in L2 sets: at
+// the OPT-30B FC2 shape (K = 28672) a stride of K + 64 measured 16 GB of DRAM reads per launch
+// instead of 24 GB.
 zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bias, void *out,
-                      int M, int N, int K, int ldo, int epi, uint32_t extra_tx) {
+                      int M, int N, int K, int ldo, int epi, uint32_t extra_tx, int64_t lda) {
   if (M < 1 || N < 1 || K < 1 || (K % 8) != 0 || (ldo % 8) != 0 || ldo < N)
     return fail(ctx, ZO_ERR_INVALID, "gemm: need M,N,K >= 1, K %% 8 == 0, ldo %% 8 == 0, ldo >= N");
+  if (lda != 0 && (lda < K || lda % 8 != 0))
+    return fail(ctx, ZO_ERR_INVALID, "gemm: lda must be a multiple of 8, at least K");
   if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B) |
        reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(bias)) & 15u)
     return fail(ctx, ZO_ERR_INVALID, "gemm: operands must be 16-byte aligned");
@@ -752,12 +759,12 @@ zo_status launch_gemm(zo_ctx *ctx, const void *A, const void *B, const void *bia
   // CTA pairs for shapes that give every cluster at least two 256 x 256 tiles
   const int64_t pair_tiles = (int64_t)((M + 255) / 256) * ((NB + 255) / 256);
   if (extra_tx == 0 && M >= 256 && NB >= 256 && pair_tiles >= (int64_t)kSmCount)
-    return launch_gemm_pair(ctx, A, B, bias, out, M, N, K, ldo, epi);
+    return launch_gemm_pair(ctx, A, B, bias, out, M, N, K, ldo, epi, lda);
   // N <= 128 tiles use BN = 128 to fill the machine on narrow outputs.
   const bool wide = NB > 128 && ((int64_t)((M + 127) / 128) * ((NB + 255) / 256) >= kSmCount);
   const int box_b = (wide ? 256 : 128) / (swiglu ? 2 : 1);
   CUtensorMap ta, tb, tcm;
-  if (!make_map(&ta, A, M, K, kBM) || !make_map(&tb, B, NB, K, box_b) ||
+  if (!make_map(&ta, A, M, K, kBM, lda) || !make_map(&tb, B, NB, K, box_b) ||
       !make_out_map(&tcm, out, M, N, ldo, epi == ZO_EPI_RESID_F32))
     return fail(ctx, ZO_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
   GemmArgs g{M, N, K, group_rows_for(K, kBM), static_cast<const uint16_t *>(bias), out, ldo,
